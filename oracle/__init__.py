@@ -1,0 +1,10 @@
+"""fp64 CPU oracle of the DeepSeekMoE layer forward (test infrastructure only).
+
+Only the tests, the package's smoke check and the benchmark's CPU-baseline / reference leg
+import this package.  It never imports the CUDA library or its binding.
+"""
+from .moe_oracle import (  # noqa: F401
+    silu, linear, expert_ffn, swiglu_hidden, route, gates_from_indices, permute, layer,
+    linear_macs, linear_params, expert_macs, expert_params, hit_entropy, n_routings,
+    split_expert,
+)

@@ -1,0 +1,266 @@
+"""fp64 CPU oracle of the DeepSeekMoE layer forward.
+
+TEST INFRASTRUCTURE.  Only the tests, the package's smoke check and the CPU-baseline /
+reference leg of the benchmark may import this module.  It shares no code with the CUDA
+library and imports nothing from it; it is plain NumPy in float64, written to be read
+against the pages, not to be fast.
+
+What it computes, and where it comes from:
+
+* Router ("《DeepSeekMoE》深度解读报告", §3.1, Eq. 3-5 in prose): the affinity of token t
+  with routed expert i is the inner product of the token's hidden state with the expert's
+  centroid; s_{i,t} is the softmax of these over all N_m experts; the gate g_{i,t} keeps
+  s_{i,t} for the N_r largest and is zero for the rest.  No renormalisation, no scale, no
+  router bias.  Ties go to the lower expert index; the picks of a token are ordered by
+  descending score, then ascending index.
+* Expert FFN (the `Expert` module of "DeepSeek MoE模型优化与未来演进及字节超稀疏内存技术"):
+  w2(silu(w1 x) * w3 x) with nn.Linear layout ([out, in]) and a bias on every Linear.
+* Layer output (DeepSeekMoE report §2.3 and §3.1, Eq. 9-11 in prose): the K_s shared experts
+  are applied to every token with weight 1 and bypass the router; the routed experts are
+  added with their gates, each gate multiplying the whole expert output (bias included).
+  The residual term of the original paper is not part of this layer (the pages do not
+  give it); a caller adds it.
+* Per-expert token lists (DeepSeek-V2 explainer, eliteato.com/news/32734, §3.1 and §3.3:
+  top-k indices first, then a gather of tokens per expert): a stable grouping of the T*N_r
+  (token, pick) slots by expert, ascending token order inside an expert.
+* Accounting helpers: ptflops-style MAC and parameter counts of one Expert (the ptflops
+  printout on the first page), the expert-hit entropy diagnostic (DeepSeek-V2 explainer
+  §6), and the combination count of fine-grained routing (DeepSeekMoE report §2.2).
+"""
+from __future__ import annotations
+
+import math
+from typing import Callable, Dict, Optional, Sequence, Union
+
+import numpy as np
+
+Weights = Dict[str, Optional[np.ndarray]]
+
+
+# --------------------------------------------------------------------------------------
+# the expert FFN
+# --------------------------------------------------------------------------------------
+def silu(a: np.ndarray) -> np.ndarray:
+    """SiLU(a) = a * sigmoid(a) = a / (1 + e^-a)."""
+    return a / (1.0 + np.exp(-a))
+
+
+def linear(x: np.ndarray, w: np.ndarray, b: Optional[np.ndarray]) -> np.ndarray:
+    """nn.Linear: y = x W^T + b with W stored [out_features, in_features]."""
+    y = x @ w.T
+    if b is not None:
+        y = y + b
+    return y
+
+
+def expert_ffn(x: np.ndarray, w1, b1, w3, b3, w2, b2) -> np.ndarray:
+    """One Expert: w2(silu(w1 x) * w3 x), each Linear with its (optional) bias."""
+    return linear(silu(linear(x, w1, b1)) * linear(x, w3, b3), w2, b2)
+
+
+def swiglu_hidden(x: np.ndarray, w1, b1, w3, b3) -> np.ndarray:
+    """The Expert's hidden activation silu(w1 x + b1) * (w3 x + b3), before w2."""
+    return silu(linear(x, w1, b1)) * linear(x, w3, b3)
+
+
+# --------------------------------------------------------------------------------------
+# the router
+# --------------------------------------------------------------------------------------
+def route(x: np.ndarray, centroids: np.ndarray, top_k: int) -> Dict[str, np.ndarray]:
+    """Scores, softmax and top-N_r gates of every token.
+
+    Returns z [T,N] logits, s [T,N] softmax, idx [T,k] picks (descending score, ties to the
+    lower index), gate [T,k] = s at the picks, and two near-tie gaps in logit units:
+    `gap` = z_(k) - z_(k+1) (the boundary of the picked set; +inf when k == N) and
+    `gap_order` = the smallest gap between consecutive picks or across the boundary.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    c = np.asarray(centroids, dtype=np.float64)
+    T, N = x.shape[0], c.shape[0]
+    if not (1 <= top_k <= N):
+        raise ValueError("top_k must be in [1, N_m]")
+    z = x @ c.T
+    zmax = z.max(axis=1, keepdims=True)
+    e = np.exp(z - zmax)
+    s = e / e.sum(axis=1, keepdims=True)
+    # stable sort of -z: descending logit, equal logits keep ascending expert index.
+    # softmax is strictly increasing in z, so this is also the order of s.
+    order = np.argsort(-z, axis=1, kind="stable")
+    idx = order[:, :top_k]
+    gate = np.take_along_axis(s, idx, axis=1)
+    zs = np.take_along_axis(z, order, axis=1)
+    if top_k < N:
+        gap = zs[:, top_k - 1] - zs[:, top_k]
+        diffs = zs[:, :top_k] - zs[:, 1:top_k + 1]
+    else:
+        gap = np.full(T, np.inf)
+        diffs = zs[:, :top_k - 1] - zs[:, 1:top_k]
+    gap_order = diffs.min(axis=1) if diffs.shape[1] > 0 else np.full(T, np.inf)
+    return {"z": z, "s": s, "idx": idx.astype(np.int64), "gate": gate,
+            "gap": gap, "gap_order": gap_order}
+
+
+def gates_from_indices(x: np.ndarray, centroids: np.ndarray, idx: np.ndarray) -> np.ndarray:
+    """s_{i,t} of the softmax over all experts, read at given picks (used when a near-tie
+    lets another valid pick set stand in for the oracle's own)."""
+    z = np.asarray(x, np.float64) @ np.asarray(centroids, np.float64).T
+    zmax = z.max(axis=1, keepdims=True)
+    e = np.exp(z - zmax)
+    s = e / e.sum(axis=1, keepdims=True)
+    return np.take_along_axis(s, np.asarray(idx, np.int64), axis=1)
+
+
+# --------------------------------------------------------------------------------------
+# per-expert token lists
+# --------------------------------------------------------------------------------------
+def permute(idx: np.ndarray, gate: np.ndarray, n_experts: int) -> Dict[str, np.ndarray]:
+    """Group the T*k slots (slot = t*k + j) by expert, ascending slot order within an expert.
+
+    counts[e], offsets[e] (exclusive prefix sum, N+1 entries), sorted_token[p] (token of the
+    p-th grouped slot), sorted_gate[p], sorted_slot[p], and slot_of[slot] = p.
+    """
+    idx = np.asarray(idx, np.int64)
+    T, k = idx.shape
+    flat = idx.reshape(-1)
+    counts = np.bincount(flat, minlength=n_experts)
+    offsets = np.zeros(n_experts + 1, np.int64)
+    offsets[1:] = np.cumsum(counts)
+    sorted_slot = np.argsort(flat, kind="stable")
+    slot_of = np.empty(T * k, np.int64)
+    slot_of[sorted_slot] = np.arange(T * k)
+    return {"counts": counts, "offsets": offsets, "sorted_slot": sorted_slot,
+            "sorted_token": sorted_slot // k,
+            "sorted_gate": np.asarray(gate, np.float64).reshape(-1)[sorted_slot],
+            "slot_of": slot_of}
+
+
+# --------------------------------------------------------------------------------------
+# the layer
+# --------------------------------------------------------------------------------------
+ExpertSource = Union[Weights, Callable[[int], Weights]]
+
+
+def _expert(src: ExpertSource, e: int) -> Weights:
+    if callable(src):
+        return src(e)
+    return {k: (None if v is None else np.asarray(v[e], np.float64)) for k, v in src.items()}
+
+
+def layer(x: np.ndarray, centroids: np.ndarray, routed: ExpertSource, n_experts: int, top_k: int,
+          shared: Optional[ExpertSource] = None, n_shared: int = 0,
+          idx_override: Optional[np.ndarray] = None, keep_hidden: bool = False) -> Dict[str, np.ndarray]:
+    """The DeepSeekMoE layer forward in fp64.
+
+    routed / shared: either dicts of stacked arrays (w1,b1,w3,b3,w2,b2 indexed by expert) or
+    a callable e -> dict of one expert's arrays (used to stream large weight sets).
+    idx_override: route with these picks instead of the oracle's own (gates are then the
+    softmax read at those picks); used where a near-tie makes another pick set valid.
+
+    Returns out [T,d], routed_sum, shared_sum, idx, gate, gap, gap_order, counts, and
+    Y [T*k, d] = gate * Expert_e(x_t) per slot (slot = t*k + j); with keep_hidden also
+    H [T*k, inter] (routed hidden activations per slot) and Hs [K_s, T, inter_s].
+    """
+    x = np.asarray(x, np.float64)
+    T, d = x.shape
+    r = route(x, centroids, top_k)
+    if idx_override is not None:
+        idx = np.asarray(idx_override, np.int64)
+        gate = gates_from_indices(x, centroids, idx)
+    else:
+        idx, gate = r["idx"], r["gate"]
+    k = top_k
+    Y = np.zeros((T * k, d))
+    H = None
+    for e in np.unique(idx):
+        w = _expert(routed, int(e))
+        tt, jj = np.nonzero(idx == e)
+        xe = x[tt]
+        he = swiglu_hidden(xe, w["w1"], w["b1"], w["w3"], w["b3"])
+        ye = linear(he, w["w2"], w["b2"])
+        if keep_hidden:
+            if H is None:
+                H = np.zeros((T * k, he.shape[1]))
+            H[tt * k + jj] = he
+        Y[tt * k + jj] = gate[tt, jj][:, None] * ye
+    routed_sum = Y.reshape(T, k, d).sum(axis=1)
+    shared_sum = np.zeros((T, d))
+    Hs = []
+    for j in range(n_shared):
+        w = _expert(shared, j)
+        hs = swiglu_hidden(x, w["w1"], w["b1"], w["w3"], w["b3"])
+        if keep_hidden:
+            Hs.append(hs)
+        shared_sum = shared_sum + linear(hs, w["w2"], w["b2"])
+    out = shared_sum + routed_sum
+    res = {"out": out, "routed_sum": routed_sum, "shared_sum": shared_sum, "idx": idx, "gate": gate,
+           "gap": r["gap"], "gap_order": r["gap_order"], "z": r["z"],
+           "counts": np.bincount(idx.reshape(-1), minlength=n_experts), "Y": Y}
+    if keep_hidden:
+        res["H"] = H if H is not None else np.zeros((T * k, 0))
+        res["Hs"] = np.stack(Hs) if Hs else None
+    return res
+
+
+# --------------------------------------------------------------------------------------
+# accounting and diagnostics
+# --------------------------------------------------------------------------------------
+def linear_macs(tokens: int, in_f: int, out_f: int, bias: bool = True) -> int:
+    """ptflops' count for nn.Linear: one MAC per weight per token plus one per output
+    element for the bias."""
+    return tokens * (in_f * out_f + (out_f if bias else 0))
+
+
+def linear_params(in_f: int, out_f: int, bias: bool = True) -> int:
+    return in_f * out_f + (out_f if bias else 0)
+
+
+def expert_macs(tokens: int, dim: int, inter: int, bias: bool = True) -> Dict[str, int]:
+    """MACs of one Expert the way ptflops reports them: the three Linears, plus one MAC per
+    element for the functional SiLU (ptflops hooks torch.nn.functional; the elementwise
+    product is a tensor method it does not count)."""
+    w1 = linear_macs(tokens, dim, inter, bias)
+    w3 = linear_macs(tokens, dim, inter, bias)
+    w2 = linear_macs(tokens, inter, dim, bias)
+    act = tokens * inter
+    return {"w1": w1, "w2": w2, "w3": w3, "silu": act, "modules": w1 + w2 + w3, "total": w1 + w2 + w3 + act}
+
+
+def expert_params(dim: int, inter: int, bias: bool = True) -> Dict[str, int]:
+    w1 = linear_params(dim, inter, bias)
+    w2 = linear_params(inter, dim, bias)
+    return {"w1": w1, "w2": w2, "w3": w1, "total": 2 * w1 + w2}
+
+
+def hit_entropy(idx: np.ndarray, n_experts: int):
+    """Expert-hit counts over all picks, their entropy (natural log) and the active ratio."""
+    counts = np.bincount(np.asarray(idx).reshape(-1), minlength=n_experts).astype(np.float64)
+    p = counts / counts.sum()
+    nz = p[p > 0]
+    ent = float(-(nz * np.log(nz)).sum())
+    return ent, float((counts > 0).mean()), counts
+
+
+def n_routings(n_experts: int, top_k: int) -> int:
+    """How many distinct expert sets a token can be routed to: C(N_m, N_r)."""
+    return math.comb(n_experts, top_k)
+
+
+def split_expert(w: Weights, m: int) -> Sequence[Weights]:
+    """Fine-grained segmentation of one Expert into m smaller ones along the intermediate
+    dimension (DeepSeekMoE report §2.2): piece p keeps rows [p*I/m, (p+1)*I/m) of w1/w3 and
+    b1/b3 and the same columns of w2; each piece carries b2/m so that the pieces summed
+    give back the unsplit Expert."""
+    I = w["w1"].shape[0]
+    if I % m:
+        raise ValueError("inter must be divisible by m")
+    q = I // m
+    pieces = []
+    for p in range(m):
+        sl = slice(p * q, (p + 1) * q)
+        pieces.append({
+            "w1": w["w1"][sl], "w3": w["w3"][sl], "w2": w["w2"][:, sl],
+            "b1": None if w["b1"] is None else w["b1"][sl],
+            "b3": None if w["b3"] is None else w["b3"][sl],
+            "b2": None if w["b2"] is None else w["b2"] / m,
+        })
+    return pieces

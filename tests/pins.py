@@ -1,0 +1,290 @@
+"""Checks that pin the fp64 oracle to facts fixed outside of it.
+
+Each check takes the oracle module and raises AssertionError when the oracle disagrees with
+a printed value, a closed form, an invariant, a brute-force enumeration or an independent
+library implementation (torch.nn / torch.nn.functional in float64, scipy.special).  The
+same checks run against deliberately broken copies of the oracle in test_oracle_mutants.py,
+which shows that each plausible mistake is caught by at least one of them.
+"""
+from __future__ import annotations
+
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import scipy.special
+import scipy.stats
+import torch
+import torch.nn.functional as F
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _rng(seed):
+    return np.random.default_rng(seed)
+
+
+def _rand_expert(rng, d, I, bias=True, std=0.3):
+    w = {"w1": rng.normal(0, std, (I, d)), "w3": rng.normal(0, std, (I, d)), "w2": rng.normal(0, std, (d, I))}
+    for b, n in (("b1", I), ("b3", I), ("b2", d)):
+        w[b] = rng.normal(0, std, n) if bias else None
+    return w
+
+
+def _stack(experts):
+    keys = experts[0].keys()
+    return {k: (None if experts[0][k] is None else np.stack([e[k] for e in experts])) for k in keys}
+
+
+class TorchExpert(torch.nn.Module):
+    """The page's Expert module rebuilt from torch.nn parts (float64): an independent
+    implementation of the per-expert function."""
+
+    def __init__(self, w):
+        super().__init__()
+        I, d = w["w1"].shape
+        bias = w["b1"] is not None
+        self.w1 = torch.nn.Linear(d, I, bias=bias, dtype=torch.float64)
+        self.w2 = torch.nn.Linear(I, d, bias=bias, dtype=torch.float64)
+        self.w3 = torch.nn.Linear(d, I, bias=bias, dtype=torch.float64)
+        with torch.no_grad():
+            for name in ("w1", "w2", "w3"):
+                getattr(self, name).weight.copy_(torch.from_numpy(w[name]))
+                if bias:
+                    getattr(self, name).bias.copy_(torch.from_numpy(w["b" + name[1]]))
+
+    def forward(self, x):
+        return self.w2(F.silu(self.w1(x)) * self.w3(x))
+
+
+def torch_expert(w, x):
+    with torch.no_grad():
+        return TorchExpert(w)(torch.from_numpy(np.asarray(x, np.float64))).numpy()
+
+
+# ----------------------------------------------------------------------------- P1
+def check_ptflops_printout(O):
+    """P1: the ptflops printout of one Expert at dim=7168, inter=2048, 256 tokens."""
+    g = json.load(open(os.path.join(GOLDEN, "expert_ptflops.json")))
+    T, d, I = g["tokens"], g["dim"], g["inter_dim"]
+    macs = O.expert_macs(T, d, I, bias=True)
+    params = O.expert_params(d, I, bias=True)
+    pr = g["printed"]
+    assert f"{params['total'] / 1e6:.2f} M" == pr["expert"]["params"]
+    assert f"{macs['modules'] / 1e9:.2f} GMac" == pr["expert"]["macs"]
+    assert f"{100.0 * macs['modules'] / macs['total']:.3f}%" == pr["expert"]["macs_pct"]
+    for name in ("w1", "w2", "w3"):
+        assert f"{params[name] / 1e6:.2f} M" == pr[name]["params"], name
+        assert f"{100.0 * params[name] / params['total']:.3f}%" == pr[name]["params_pct"], name
+        assert f"{macs[name] / 1e9:.2f} GMac" == pr[name]["macs"], name
+        assert f"{100.0 * macs[name] / macs['total']:.3f}%" == pr[name]["macs_pct"], name
+        assert O.linear_params(pr[name]["in_features"], pr[name]["out_features"], True) == params[name]
+
+
+# ----------------------------------------------------------------------------- P5 helper
+def check_combinations(O):
+    g = json.load(open(os.path.join(GOLDEN, "routing_counts.json")))
+    for c in g["cases"]:
+        assert O.n_routings(c["n_experts"], c["top_k"]) == c["combinations"]
+    for n, k in ((6, 2), (8, 3), (10, 4)):
+        assert O.n_routings(n, k) == sum(1 for _ in itertools.combinations(range(n), k))
+
+
+# ----------------------------------------------------------------------------- P6
+def check_textbook_single_expert(O):
+    """P6: N_m = N_r = 1, K_s = 0 makes the gate 1 and the layer one Expert module."""
+    rng = _rng(6)
+    for bias in (True, False):
+        T, d, I = 9, 12, 10
+        x = rng.normal(0, 1, (T, d))
+        w = _rand_expert(rng, d, I, bias)
+        c = rng.normal(0, 1, (1, d))
+        res = O.layer(x, c, _stack([w]), n_experts=1, top_k=1)
+        ref = torch_expert(w, x)
+        assert np.allclose(res["gate"], 1.0, rtol=0, atol=1e-15)
+        assert np.allclose(res["out"], ref, rtol=1e-12, atol=1e-12)
+        assert np.allclose(O.expert_ffn(x, w["w1"], w["b1"], w["w3"], w["b3"], w["w2"], w["b2"]), ref,
+                           rtol=1e-12, atol=1e-12)
+
+
+# ----------------------------------------------------------------------------- P4
+def check_gate_invariants(O):
+    """P4: gates are the softmax over all experts read at the top-N_r picks."""
+    rng = _rng(4)
+    T, d, N, k = 40, 16, 12, 4
+    x = rng.normal(0, 1, (T, d))
+    c = rng.normal(0, 0.5, (N, d))
+    r = O.route(x, c, k)
+    s_ref = scipy.special.softmax(x @ c.T, axis=1)          # library softmax
+    assert np.allclose(r["s"], s_ref, rtol=1e-12, atol=0)
+    g = r["gate"]
+    assert np.array_equal(g, np.take_along_axis(s_ref, r["idx"], 1)) or \
+        np.allclose(g, np.take_along_axis(s_ref, r["idx"], 1), rtol=1e-13, atol=0)
+    assert (g > 0).all() and (g <= 1).all()
+    assert (g.sum(1) <= 1 + 1e-12).all()
+    assert (np.diff(g, axis=1) <= 0).all(), "picks ordered by descending score"
+    for t in range(T):
+        sel = set(r["idx"][t].tolist())
+        assert len(sel) == k
+        rest = [s_ref[t, i] for i in range(N) if i not in sel]
+        assert max(rest) <= g[t].min()
+    # closed form: two experts, top-1 -> gate = sigmoid(|z1 - z2|)
+    x2 = rng.normal(0, 1, (20, d))
+    c2 = rng.normal(0, 0.7, (2, d))
+    r2 = O.route(x2, c2, 1)
+    dz = np.abs(x2 @ c2[0] - x2 @ c2[1])
+    assert np.allclose(r2["gate"][:, 0], 1.0 / (1.0 + np.exp(-dz)), rtol=1e-13, atol=0)
+    # all-equal scores: every gate is 1/N and ties go to the lowest indices
+    ce = np.tile(rng.normal(0, 1, (1, d)), (N, 1))
+    r3 = O.route(x, ce, k)
+    assert np.array_equal(r3["idx"], np.tile(np.arange(k), (T, 1)))
+    assert np.allclose(r3["gate"], 1.0 / N, rtol=1e-14, atol=0)
+    # known logits: x = unit vector, centroid column 0 holds the logits
+    logits = np.array([0.3, -1.0, 2.0, 2.0, 0.1, 5.0])
+    cx = np.zeros((6, 3)); cx[:, 0] = logits
+    xu = np.array([[1.0, 0.0, 0.0]])
+    r4 = O.route(xu, cx, 3)
+    assert r4["idx"][0].tolist() == [5, 2, 3]
+    ex = [math.exp(v) for v in logits]
+    assert np.allclose(r4["gate"][0], [ex[5] / sum(ex), ex[2] / sum(ex), ex[3] / sum(ex)], rtol=1e-14, atol=0)
+    assert r4["gap"][0] == 2.0 - 0.3
+
+
+# ----------------------------------------------------------------------------- P5
+def check_bruteforce_routing(O):
+    """P5: on tiny inputs the picked set is the unique subset of size N_r with the largest
+    total score, and the layer equals the explicit sum over that subset (torch float64)."""
+    rng = _rng(5)
+    for (T, d, N, k, Ks) in ((7, 6, 5, 2, 0), (6, 8, 7, 3, 1), (5, 4, 8, 4, 2)):
+        x = rng.normal(0, 1, (T, d))
+        c = rng.normal(0, 0.8, (N, d))
+        experts = [_rand_expert(rng, d, 6) for _ in range(N)]
+        shared = [_rand_expert(rng, d, 5) for _ in range(Ks)]
+        res = O.layer(x, c, _stack(experts), N, k, _stack(shared) if Ks else None, Ks)
+        z = x @ c.T
+        s = scipy.special.softmax(z, axis=1)
+        subsets = list(itertools.combinations(range(N), k))
+        assert len(subsets) == O.n_routings(N, k)
+        for t in range(T):
+            scores = [sum(s[t, i] for i in sub) for sub in subsets]
+            best = subsets[int(np.argmax(scores))]
+            assert sorted(scores)[-1] - sorted(scores)[-2] > 1e-9
+            assert set(res["idx"][t].tolist()) == set(best)
+            want = np.zeros(d)
+            for i in best:
+                want += s[t, i] * torch_expert(experts[i], x[t:t + 1])[0]
+            for w in shared:
+                want += torch_expert(w, x[t:t + 1])[0]
+            assert np.allclose(res["out"][t], want, rtol=1e-11, atol=1e-11)
+
+
+# ----------------------------------------------------------------------------- P2
+def check_split_identity(O):
+    """P2: an Expert split along its intermediate dimension into m pieces, all active with
+    equal gate, gives back the unsplit Expert (params and FLOPs unchanged)."""
+    rng = _rng(2)
+    T, d, I = 11, 10, 12
+    x = rng.normal(0, 1, (T, d))
+    for bias in (True, False):
+        w = _rand_expert(rng, d, I, bias)
+        full = torch_expert(w, x)
+        for m in (2, 3, 4):
+            pieces = O.split_expert(w, m)
+            tot = sum(torch_expert(p, x) for p in pieces)
+            assert np.allclose(tot, full, rtol=1e-12, atol=1e-12)
+            p_full = O.expert_params(d, I, bias)["total"]
+            p_split = sum(O.linear_params(d, I // m, bias) * 2 + O.linear_params(I // m, d, bias) for _ in range(m))
+            # weights unchanged; the split adds (m-1) copies of the b2 vector
+            assert p_split - p_full == (m - 1) * d * (1 if bias else 0)
+            # through the layer: m identical centroids, N_r = N_m = m -> gates 1/m
+            c = np.tile(rng.normal(0, 1, (1, d)), (m, 1))
+            res = O.layer(x, c, _stack(list(pieces)), m, m)
+            assert np.allclose(res["gate"], 1.0 / m, rtol=1e-14, atol=0)
+            assert np.allclose(m * res["routed_sum"], full, rtol=1e-11, atol=1e-11)
+            # plus one shared expert: out - shared is still the routed part
+            sh = _rand_expert(rng, d, 7, bias)
+            res2 = O.layer(x, c, _stack(list(pieces)), m, m, _stack([sh]), 1)
+            assert np.allclose(res2["out"], full / m + torch_expert(sh, x), rtol=1e-11, atol=1e-11)
+
+
+# ----------------------------------------------------------------------------- P3
+def check_shared_bypasses_router(O):
+    """P3: the shared experts see every token with weight 1 whatever the router does."""
+    rng = _rng(3)
+    T, d, N, k = 13, 8, 6, 2
+    x = rng.normal(0, 1, (T, d))
+    experts = _stack([_rand_expert(rng, d, 5) for _ in range(N)])
+    shared = [_rand_expert(rng, d, 4) for _ in range(2)]
+    outs = []
+    for seed in range(3):
+        c = np.random.default_rng(100 + seed).normal(0, 1, (N, d))
+        res = O.layer(x, c, experts, N, k, _stack(shared), 2)
+        outs.append(res)
+        assert np.allclose(res["out"] - res["routed_sum"], res["shared_sum"], rtol=1e-13, atol=1e-13)
+    for r in outs[1:]:
+        assert np.array_equal(r["shared_sum"], outs[0]["shared_sum"])
+    want = torch_expert(shared[0], x) + torch_expert(shared[1], x)
+    assert np.allclose(outs[0]["shared_sum"], want, rtol=1e-12, atol=1e-12)
+    # routed experts that output zero leave exactly the shared part
+    zero = {kk: (None if v is None else np.zeros_like(v)) for kk, v in experts.items()}
+    res = O.layer(x, np.random.default_rng(9).normal(0, 1, (N, d)), zero, N, k, _stack(shared), 2)
+    assert np.allclose(res["out"], want, rtol=1e-12, atol=1e-12)
+
+
+# ----------------------------------------------------------------------------- P7
+def check_hit_entropy(O):
+    """P7: entropy of the expert-hit distribution is at most ln N, with equality exactly
+    when every expert is hit equally often."""
+    g = json.load(open(os.path.join(GOLDEN, "hit_entropy.json")))
+    for c in g["cases"]:
+        N = c["n_experts"]
+        idx = np.arange(N * 5).reshape(-1, 1) % N
+        ent, act, counts = O.hit_entropy(idx, N)
+        assert f"{ent:.{c['decimals']}f}" == c["max_entropy_printed"]
+        assert abs(ent - math.log(N)) < 1e-12 and act == 1.0
+    rng = _rng(7)
+    for _ in range(20):
+        N = int(rng.integers(2, 12))
+        idx = rng.integers(0, N, (30, 2))
+        ent, act, counts = O.hit_entropy(idx, N)
+        assert np.array_equal(counts, np.bincount(idx.reshape(-1), minlength=N))
+        assert ent <= math.log(N) + 1e-12
+        uniform = (counts == counts[0]).all()
+        assert (abs(ent - math.log(N)) < 1e-12) == bool(uniform)
+        p = counts / counts.sum()
+        assert abs(ent - scipy.stats.entropy(p)) < 1e-12          # library entropy
+    ent, act, _ = O.hit_entropy(np.zeros((10, 1), np.int64), 4)
+    assert ent == 0.0 and act == 0.25
+
+
+# ----------------------------------------------------------------------------- grouping
+def check_permute(O):
+    """The per-expert token lists against a plain loop: for each expert in order, every slot
+    (token t, pick j) that chose it, in ascending slot order."""
+    rng = _rng(8)
+    for (T, N, k) in ((1, 3, 1), (17, 6, 3), (40, 16, 4), (9, 4, 4)):
+        idx = np.stack([rng.permutation(N)[:k] for _ in range(T)])
+        gate = rng.random((T, k))
+        p = O.permute(idx, gate, N)
+        order = []
+        for e in range(N):
+            for t in range(T):
+                for j in range(k):
+                    if idx[t, j] == e:
+                        order.append(t * k + j)
+        order = np.array(order)
+        assert np.array_equal(p["sorted_slot"], order)
+        assert np.array_equal(p["sorted_token"], order // k)
+        assert np.array_equal(p["sorted_gate"], gate.reshape(-1)[order])
+        cnt = [int((idx == e).sum()) for e in range(N)]
+        assert p["counts"].tolist() == cnt
+        assert p["offsets"].tolist() == [sum(cnt[:e]) for e in range(N + 1)]
+        for pos, slot in enumerate(order):
+            assert p["slot_of"][slot] == pos
+
+
+ALL_CHECKS = [check_ptflops_printout, check_combinations, check_textbook_single_expert,
+              check_gate_invariants, check_bruteforce_routing, check_split_identity,
+              check_shared_bypasses_router, check_hit_entropy, check_permute]

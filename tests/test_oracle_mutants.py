@@ -1,0 +1,117 @@
+"""Plant plausible mistakes in the oracle (on the CPU) and check that the pins catch each one.
+
+A pin set that a wrong oracle also passes proves nothing; every mutant below must make at
+least one check of tests/pins.py fail.
+"""
+import numpy as np
+import pytest
+
+import oracle.moe_oracle as O
+from tests import pins
+
+_orig = {name: getattr(O, name) for name in ("silu", "linear", "route", "swiglu_hidden", "permute",
+                                             "expert_macs", "split_expert", "hit_entropy")}
+
+
+def _sigmoid_for_silu(a):                      # silu without the factor a
+    return 1.0 / (1.0 + np.exp(-a))
+
+
+def _linear_no_bias(x, w, b):                  # dropped bias term
+    return x @ w.T
+
+
+def _linear_bias_sign(x, w, b):                # wrong sign on the bias
+    y = x @ w.T
+    if b is not None:
+        y = y - b
+    return y
+
+
+def _route_renormalised(x, c, k):              # softmax over the picks only
+    r = _orig["route"](x, c, k)
+    r = dict(r)
+    r["gate"] = r["gate"] / r["gate"].sum(axis=1, keepdims=True)
+    return r
+
+
+def _route_lowest(x, c, k):                    # picks the smallest scores
+    r = _orig["route"](-np.asarray(x), c, k)
+    r = dict(r)
+    z = np.asarray(x, np.float64) @ np.asarray(c, np.float64).T
+    s = np.exp(z - z.max(1, keepdims=True)); s /= s.sum(1, keepdims=True)
+    r["gate"] = np.take_along_axis(s, r["idx"], 1)
+    return r
+
+
+def _route_ties_high(x, c, k):                 # ties resolved toward the higher index
+    z = np.asarray(x, np.float64) @ np.asarray(c, np.float64).T
+    N = z.shape[1]
+    r = _orig["route"](x, np.asarray(c)[::-1], k)
+    r = dict(r)
+    r["idx"] = (N - 1) - r["idx"]
+    s = np.exp(z - z.max(1, keepdims=True)); s /= s.sum(1, keepdims=True)
+    r["gate"] = np.take_along_axis(s, r["idx"], 1)
+    return r
+
+
+def _swiglu_swapped(x, w1, b1, w3, b3):         # gate on w3 instead of w1
+    return O.silu(O.linear(x, w3, b3)) * O.linear(x, w1, b1)
+
+
+def _permute_unstable(idx, gate, n):           # descending slot order inside an expert
+    p = dict(_orig["permute"](idx, gate, n))
+    idx = np.asarray(idx)
+    k = idx.shape[1]
+    flat = idx.reshape(-1)
+    order = np.concatenate([np.nonzero(flat == e)[0][::-1] for e in range(n)]).astype(np.int64)
+    p["sorted_slot"] = order
+    p["sorted_token"] = order // k
+    p["sorted_gate"] = np.asarray(gate).reshape(-1)[order]
+    so = np.empty_like(order); so[order] = np.arange(order.size); p["slot_of"] = so
+    return p
+
+
+def _macs_no_bias(tokens, dim, inter, bias=True):
+    return _orig["expert_macs"](tokens, dim, inter, False)
+
+
+def _split_no_b2_scale(w, m):                  # every piece keeps the whole b2
+    pieces = _orig["split_expert"](w, m)
+    for p in pieces:
+        if p["b2"] is not None:
+            p["b2"] = p["b2"] * m
+    return pieces
+
+
+def _entropy_log2(idx, n):
+    e, a, c = _orig["hit_entropy"](idx, n)
+    return e / np.log(2.0), a, c
+
+
+MUTANTS = {
+    "silu_is_sigmoid": ("silu", _sigmoid_for_silu),
+    "linear_drops_bias": ("linear", _linear_no_bias),
+    "linear_bias_sign": ("linear", _linear_bias_sign),
+    "gates_renormalised": ("route", _route_renormalised),
+    "picks_lowest_scores": ("route", _route_lowest),
+    "ties_to_higher_index": ("route", _route_ties_high),
+    "swiglu_roles_swapped": ("swiglu_hidden", _swiglu_swapped),
+    "permute_unstable": ("permute", _permute_unstable),
+    "macs_without_bias": ("expert_macs", _macs_no_bias),
+    "split_keeps_full_b2": ("split_expert", _split_no_b2_scale),
+    "entropy_in_bits": ("hit_entropy", _entropy_log2),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_mutant_is_caught(name, monkeypatch):
+    attr, fn = MUTANTS[name]
+    monkeypatch.setattr(O, attr, fn)
+    failed = []
+    for check in pins.ALL_CHECKS:
+        try:
+            check(O)
+        except AssertionError:
+            failed.append(check.__name__)
+    assert failed, f"mutant {name} passed every pin"
