@@ -1,0 +1,726 @@
+// Tensor-core kernels of the bf16 DeepSeekMoE layer: one persistent, warp-specialised
+// tcgen05 pipeline with four epilogues.
+//
+//   ROUTER  scores z = x C^T of 128 tokens x N_m experts; the epilogue thread that owns a
+//           token row does the softmax over all N_m experts and the top-N_r selection
+//           ("《DeepSeekMoE》深度解读报告" §3.1, Eq. 3-5 in prose).
+//   GEMM1   [x_e] [w1_e | w3_e]^T for 128 rows x (128 + 128) columns with bias and SwiGLU in
+//           the epilogue: h = silu(x w1^T + b1) * (x w3^T + b3) (the `Expert` module of
+//           "DeepSeek MoE模型优化与未来演进及字节超稀疏内存技术").  Routed groups read the
+//           expert's gathered rows, shared groups read x itself.
+//   GEMM2R  routed w2 contraction; the epilogue adds b2 and scales by the gate: the gate
+//           multiplies the whole expert output.
+//   GEMM2S  the K_s shared experts' w2 contractions accumulated along K in one accumulator;
+//           the epilogue adds the shared biases and then the token's N_r gated routed rows in
+//           pick order (§2.3 and §3.1 of the DeepSeekMoE report: shared experts first, then
+//           the gated routed sum), and rounds once.
+//
+// Pipeline (192 threads, one CTA per SM, persistent over a static round-robin tile order):
+//   warp 0      TMA producer: 128B-swizzled K-major tiles of A (16 KB) and B (up to 32 KB)
+//               into a 4-stage shared-memory ring, completion counted on mbarriers;
+//   warp 1      allocates 512 TMEM columns; one thread issues tcgen05.mma (M=128, N<=256,
+//               K=16, bf16 x bf16 -> fp32) and commits each stage back to the producer and
+//               each finished accumulator to the epilogue;
+//   warps 2-5   epilogue: tcgen05.ld of their 32 TMEM lanes (one accumulator row each),
+//               fp32 math, bf16 stores.  Two accumulators (2 x 256 columns) let the
+//               epilogue of one tile overlap the main loop of the next.
+// Every mbarrier wait is bounded (a few seconds of %globaltimer); on expiry the kernel sets
+// an error bit, stops issuing, waits (bounded) for its own copies and MMAs in flight, frees
+// TMEM and returns.  No cluster launch and no multicast anywhere.
+#include <cuda.h>
+
+#include "common.cuh"
+#include "launch.h"
+
+namespace moe {
+namespace tc {
+
+constexpr int BM = 128;                  // rows per tile (TMEM lanes)
+constexpr int BK = 64;                   // K per stage: 64 bf16 = one 128-byte swizzle row
+constexpr int STAGES = 4;
+constexpr int A_BYTES = BM * BK * 2;     // 16 KB
+constexpr int B_BYTES = 256 * BK * 2;    // 32 KB (N <= 256)
+constexpr int THREADS = 192;
+constexpr int TMEM_COLS = 512;
+constexpr int ACC_COLS = 256;
+constexpr int SMEM_BYTES = 1024 /*align slack*/ + STAGES * (A_BYTES + B_BYTES) + 256 /*barriers*/;
+constexpr unsigned long long WAIT_NS = 4000000000ull;
+
+enum Mode : int { ROUTER = 0, GEMM1 = 1, GEMM2R = 2, GEMM2S = 3 };
+
+struct Params {
+    CUtensorMap tmA[2];
+    CUtensorMap tmB[4];
+    const int32_t* tile_start;
+    const int32_t* offsets;
+    int g_begin, g_end;
+    int T, d, E, I, Is, k, Ks;
+    int n_mma;                 // MMA N (256, or N_m for the router)
+    long long S;
+    const __nv_bfloat16 *b1, *b3, *b2, *sb1, *sb3, *sb2;
+    __nv_bfloat16* h_r;
+    __nv_bfloat16* h_s;
+    const float* sorted_gate;
+    __nv_bfloat16* y;
+    const __nv_bfloat16* y_in;
+    const int32_t* slot_of;
+    __nv_bfloat16* out;
+    int32_t* idx_out;
+    float* gate_out;
+    uint32_t* err;
+};
+
+// ------------------------------------------------------------------------------ PTX helpers
+__device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ unsigned long long globaltimer() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+// Bounded wait; false when the pipeline was aborted or the wait ran out of time.
+__device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag, uint32_t* err,
+                                       bool honour_abort = true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const unsigned long long t0 = globaltimer();
+    for (uint32_t i = 1;; ++i) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((i & 63u) == 0u) {
+            if (honour_abort && *abort_flag) return false;
+            if (globaltimer() - t0 > WAIT_NS) {
+                *abort_flag = 1;
+                flag_error(err, ERR_PIPE_TIMEOUT);
+                return false;
+            }
+        }
+    }
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar, int c0, int c1) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+        "l"((unsigned long long)map), "r"(bar), "r"(c0), "r"(c1)
+        : "memory");
+}
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, uint32_t bar, int c0, int c1, int c2) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(
+            dst),
+        "l"((unsigned long long)map), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
+        : "memory");
+}
+__device__ __forceinline__ void prefetch_map(const CUtensorMap* map) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"((unsigned long long)map) : "memory");
+}
+
+// Shared-memory matrix descriptor: K-major operand, 128-byte swizzle, 8-row core-matrix
+// groups 1024 bytes apart (stride byte offset); leading byte offset unused for this layout;
+// descriptor version 1 (bits 46-47); layout type 2 = SWIZZLE_128B (bits 61-63).
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t addr) {
+    uint64_t d = 0;
+    d |= (uint64_t)((addr & 0x3FFFFu) >> 4);
+    d |= (uint64_t)1 << 16;
+    d |= (uint64_t)(1024 >> 4) << 32;
+    d |= (uint64_t)1 << 46;
+    d |= (uint64_t)2 << 61;
+    return d;
+}
+// Instruction descriptor, kind::f16: fp32 accumulator, bf16 A and B, both K-major, M=128.
+__host__ __device__ constexpr uint32_t idesc_bf16(int n) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a), "l"(b), "r"(idesc), "r"(acc)
+        : "memory");
+}
+__device__ __forceinline__ void mma_commit(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+          "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]),
+          "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+          "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+          "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// ------------------------------------------------------------------------------ tile order
+struct Tile {
+    int g;       // group: expert (routed), E + s (shared GEMM1), 0 otherwise
+    int m0;      // first row of the tile inside its group
+    int n0;      // first output column
+    int rows;    // rows of the group
+    int row0;    // first row of the group in A and in the output
+    int num_kb;  // K blocks of 64
+};
+
+template <int MODE>
+__device__ __forceinline__ int total_tiles(const Params& p) {
+    if (MODE == ROUTER) return ceil_div(p.T, BM);
+    if (MODE == GEMM1) return p.tile_start[p.g_end] - p.tile_start[p.g_begin];
+    if (MODE == GEMM2R) return p.tile_start[p.E];
+    return ceil_div(p.T, BM) * ceil_div(p.d, 256);
+}
+
+// largest g in [lo, hi) with ts[g] <= t   (ts non-decreasing, ts[hi] > t)
+__device__ __forceinline__ int find_group(const int32_t* ts, int lo, int hi, int t) {
+    while (hi - lo > 1) {
+        int mid = (lo + hi) >> 1;
+        if (ts[mid] <= t) lo = mid;
+        else hi = mid;
+    }
+    return lo;
+}
+
+template <int MODE>
+__device__ __forceinline__ Tile decode(const Params& p, int t) {
+    Tile x;
+    if (MODE == ROUTER) {
+        x.g = 0; x.m0 = t * BM; x.n0 = 0; x.rows = p.T; x.row0 = 0; x.num_kb = ceil_div(p.d, BK);
+    } else if (MODE == GEMM1) {
+        const int tt = t + p.tile_start[p.g_begin];
+        const int g = find_group(p.tile_start, p.g_begin, p.g_end, tt);
+        const int local = tt - p.tile_start[g];
+        const bool shared = g >= p.E;
+        x.g = g;
+        x.rows = shared ? p.T : p.offsets[g + 1] - p.offsets[g];
+        x.row0 = shared ? 0 : p.offsets[g];
+        const int mt = ceil_div(x.rows, BM);
+        x.m0 = (local % mt) * BM;
+        x.n0 = (local / mt) * 128;
+        x.num_kb = ceil_div(p.d, BK);
+    } else if (MODE == GEMM2R) {
+        const int e = find_group(p.tile_start, 0, p.E, t);
+        const int local = t - p.tile_start[e];
+        x.g = e;
+        x.rows = p.offsets[e + 1] - p.offsets[e];
+        x.row0 = p.offsets[e];
+        const int mt = ceil_div(x.rows, BM);
+        x.m0 = (local % mt) * BM;
+        x.n0 = (local / mt) * 256;
+        x.num_kb = ceil_div(p.I, BK);
+    } else {
+        const int mt = ceil_div(p.T, BM);
+        x.g = 0; x.rows = p.T; x.row0 = 0;
+        x.m0 = (t % mt) * BM;
+        x.n0 = (t / mt) * 256;
+        x.num_kb = p.Ks * ceil_div(p.Is, BK);
+    }
+    return x;
+}
+
+// ------------------------------------------------------------------------------ epilogues
+// Top-k insertion keeping (value desc, index asc); candidates arrive in ascending index.
+template <int KMAX>
+__device__ __forceinline__ void topk_insert(float (&tv)[KMAX], int (&ti)[KMAX], float v, int e) {
+    if (v > tv[KMAX - 1]) {
+        tv[KMAX - 1] = v;
+        ti[KMAX - 1] = e;
+#pragma unroll
+        for (int j = KMAX - 1; j > 0; --j) {
+            if (tv[j] > tv[j - 1]) {
+                float a = tv[j]; tv[j] = tv[j - 1]; tv[j - 1] = a;
+                int b = ti[j]; ti[j] = ti[j - 1]; ti[j - 1] = b;
+            }
+        }
+    }
+}
+
+template <int KMAX>
+__device__ __forceinline__ void epilogue_router(const Params& p, const Tile& x, uint32_t tacc, int row) {
+    float tv[KMAX];
+    int ti[KMAX];
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j) { tv[j] = -INFINITY; ti[j] = 0; }
+    for (int c0 = 0; c0 < p.n_mma; c0 += 16) {
+        uint32_t r[16];
+        tmem_ld16(tacc + c0, r);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+            if (c0 + j < p.E) topk_insert<KMAX>(tv, ti, __uint_as_float(r[j]), c0 + j);
+    }
+    const float zmax = tv[0];
+    float s = 0.f;
+    for (int c0 = 0; c0 < p.n_mma; c0 += 16) {
+        uint32_t r[16];
+        tmem_ld16(tacc + c0, r);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+            if (c0 + j < p.E) s += expf(__uint_as_float(r[j]) - zmax);
+    }
+    const int t = x.m0 + row;
+    if (t < p.T) {
+        const float inv = 1.0f / s;
+#pragma unroll
+        for (int j = 0; j < KMAX; ++j) {
+            if (j < p.k) {
+                p.idx_out[(size_t)t * p.k + j] = ti[j];
+                p.gate_out[(size_t)t * p.k + j] = expf(tv[j] - zmax) * inv;
+            }
+        }
+    }
+}
+
+__device__ __forceinline__ void epilogue_gemm1(const Params& p, const Tile& x, uint32_t tacc, int row) {
+    const bool shared = x.g >= p.E;
+    const int e = shared ? x.g - p.E : x.g;
+    const int I = shared ? p.Is : p.I;
+    const __nv_bfloat16* b1 = shared ? p.sb1 : p.b1;
+    const __nv_bfloat16* b3 = shared ? p.sb3 : p.b3;
+    if (b1) b1 += (size_t)e * I;
+    if (b3) b3 += (size_t)e * I;
+    const int r = x.m0 + row;
+    const bool live = r < x.rows;
+    __nv_bfloat16* hrow = shared ? p.h_s + ((size_t)e * p.T + r) * I : p.h_r + (size_t)(x.row0 + r) * I;
+#pragma unroll 1
+    for (int c = 0; c < 4; ++c) {
+        uint32_t u[32], v[32];
+        tmem_ld32(tacc + c * 32, u);
+        tmem_ld32(tacc + 128 + c * 32, v);
+        tmem_wait_ld();
+        const int col0 = x.n0 + c * 32;
+        if (!live || col0 >= I) continue;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int col = col0 + q * 8;
+            if (col >= I) break;
+            uint32_t pk[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                float hv[2];
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int j = q * 8 + i * 2 + h;
+                    float a = __uint_as_float(u[j]) + (b1 ? __bfloat162float(b1[col + i * 2 + h]) : 0.f);
+                    float g = __uint_as_float(v[j]) + (b3 ? __bfloat162float(b3[col + i * 2 + h]) : 0.f);
+                    hv[h] = silu_f32(a) * g;
+                }
+                pk[i] = pack_bf16(hv[0], hv[1]);
+            }
+            *reinterpret_cast<uint4*>(hrow + col) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        }
+    }
+}
+
+__device__ __forceinline__ void epilogue_gemm2r(const Params& p, const Tile& x, uint32_t tacc, int row) {
+    const int r = x.m0 + row;
+    const bool live = r < x.rows;
+    const long long pos = x.row0 + r;
+    const float gate = live ? (p.sorted_gate ? p.sorted_gate[pos] : 1.f) : 0.f;
+    const __nv_bfloat16* b2 = p.b2 ? p.b2 + (size_t)x.g * p.d : nullptr;
+    __nv_bfloat16* yrow = p.y + (size_t)pos * p.d;
+#pragma unroll 1
+    for (int c = 0; c < 8; ++c) {
+        uint32_t u[32];
+        tmem_ld32(tacc + c * 32, u);
+        tmem_wait_ld();
+        const int col0 = x.n0 + c * 32;
+        if (!live || col0 >= p.d) continue;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int col = col0 + q * 8;
+            if (col >= p.d) break;
+            uint32_t pk[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int j = q * 8 + i * 2;
+                float a = __uint_as_float(u[j]) + (b2 ? __bfloat162float(b2[col + i * 2]) : 0.f);
+                float b = __uint_as_float(u[j + 1]) + (b2 ? __bfloat162float(b2[col + i * 2 + 1]) : 0.f);
+                pk[i] = pack_bf16(gate * a, gate * b);
+            }
+            *reinterpret_cast<uint4*>(yrow + col) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        }
+    }
+}
+
+__device__ __forceinline__ void epilogue_gemm2s(const Params& p, const Tile& x, uint32_t tacc, int row) {
+    const int t = x.m0 + row;
+    const bool live = t < p.T;
+#pragma unroll 1
+    for (int c = 0; c < 8; ++c) {
+        uint32_t u[32];
+        tmem_ld32(tacc + c * 32, u);
+        tmem_wait_ld();
+        const int col0 = x.n0 + c * 32;
+        if (!live || col0 >= p.d) continue;
+        float acc[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) acc[j] = __uint_as_float(u[j]);
+        if (p.sb2) {
+            for (int s = 0; s < p.Ks; ++s) {
+                const __nv_bfloat16* b = p.sb2 + (size_t)s * p.d + col0;
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                    if (col0 + j < p.d) acc[j] += __bfloat162float(b[j]);
+            }
+        }
+        for (int jj = 0; jj < p.k; ++jj) {
+            const int pos = p.slot_of[(size_t)t * p.k + jj];
+            if (pos < 0 || pos >= p.S) { flag_error(p.err, ERR_INDEX_RANGE); continue; }
+            const uint4* src = reinterpret_cast<const uint4*>(p.y_in + (size_t)pos * p.d + col0);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                if (col0 + q * 8 >= p.d) break;
+                uint4 w = __ldg(src + q);
+                const __nv_bfloat16* e = reinterpret_cast<const __nv_bfloat16*>(&w);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) acc[q * 8 + i] += __bfloat162float(e[i]);
+            }
+        }
+        __nv_bfloat16* orow = p.out + (size_t)t * p.d;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int col = col0 + q * 8;
+            if (col >= p.d) break;
+            uint32_t pk[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) pk[i] = pack_bf16(acc[q * 8 + i * 2], acc[q * 8 + i * 2 + 1]);
+            *reinterpret_cast<uint4*>(orow + col) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        }
+    }
+}
+
+// ------------------------------------------------------------------------------ the kernel
+template <int MODE, int KMAX>
+__global__ void __launch_bounds__(THREADS, 1) moe_tc_kernel(const __grid_constant__ Params p) {
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    uint8_t* gbase = smem_raw + (base - raw);
+    const uint32_t sA = base;
+    const uint32_t sB = base + STAGES * A_BYTES;
+    const uint32_t bar0 = sB + STAGES * B_BYTES;
+    // barrier addresses (8 bytes each)
+    auto full_bar = [&](int s) { return bar0 + 8u * s; };
+    auto empty_bar = [&](int s) { return bar0 + 8u * (STAGES + s); };
+    auto tfull_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + a); };
+    auto tempty_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + 2 + a); };
+    const uint32_t drain_bar = bar0 + 8u * (2 * STAGES + 4);
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(gbase + (bar0 - base) + 8 * (2 * STAGES + 5));
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) { mbar_init(full_bar(s), 1); mbar_init(empty_bar(s), 1); }
+        for (int a = 0; a < 2; ++a) { mbar_init(tfull_bar(a), 1); mbar_init(tempty_bar(a), 4); }
+        mbar_init(drain_bar, 1);
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_holder)),
+                     "r"(TMEM_COLS)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_holder;
+    const int ntiles = total_tiles<MODE>(p);
+
+    if (warp == 0) {
+        // ------------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            prefetch_map(&p.tmA[0]);
+            prefetch_map(&p.tmB[0]);
+            int stage = 0;
+            uint32_t phase = 0;
+            int last_parity[STAGES];
+#pragma unroll
+            for (int s = 0; s < STAGES; ++s) last_parity[s] = -1;
+            bool ok = true;
+            for (int t = blockIdx.x; ok && t < ntiles; t += gridDim.x) {
+                const Tile x = decode<MODE>(p, t);
+                for (int kb = 0; kb < x.num_kb; ++kb) {
+                    if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, p.err)) { ok = false; break; }
+                    const uint32_t fb = full_bar(stage);
+                    const uint32_t a_dst = sA + stage * A_BYTES, b_dst = sB + stage * B_BYTES;
+                    if (MODE == ROUTER) {
+                        mbar_expect_tx(fb, A_BYTES + p.n_mma * BK * 2);
+                        tma_load_2d(a_dst, &p.tmA[0], fb, kb * BK, x.m0);
+                        tma_load_2d(b_dst, &p.tmB[0], fb, kb * BK, 0);
+                    } else if (MODE == GEMM1) {
+                        mbar_expect_tx(fb, A_BYTES + B_BYTES);
+                        const bool shared = x.g >= p.E;
+                        const int e = shared ? x.g - p.E : x.g;
+                        tma_load_2d(a_dst, &p.tmA[shared ? 1 : 0], fb, kb * BK, x.row0 + x.m0);
+                        tma_load_3d(b_dst, &p.tmB[shared ? 2 : 0], fb, kb * BK, x.n0, e);
+                        tma_load_3d(b_dst + B_BYTES / 2, &p.tmB[shared ? 3 : 1], fb, kb * BK, x.n0, e);
+                    } else if (MODE == GEMM2R) {
+                        mbar_expect_tx(fb, A_BYTES + B_BYTES);
+                        tma_load_2d(a_dst, &p.tmA[0], fb, kb * BK, x.row0 + x.m0);
+                        tma_load_3d(b_dst, &p.tmB[0], fb, kb * BK, x.n0, x.g);
+                    } else {
+                        const int kbs = ceil_div(p.Is, BK);
+                        const int s = kb / kbs, kk = kb % kbs;
+                        mbar_expect_tx(fb, A_BYTES + B_BYTES);
+                        tma_load_3d(a_dst, &p.tmA[0], fb, kk * BK, x.m0, s);
+                        tma_load_3d(b_dst, &p.tmB[0], fb, kk * BK, x.n0, s);
+                    }
+                    last_parity[stage] = (int)phase;
+                    if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+                }
+            }
+            // drain: every copy this thread issued has landed before the CTA may exit
+#pragma unroll
+            for (int s = 0; s < STAGES; ++s)
+                if (last_parity[s] >= 0) mbar_wait(full_bar(s), (uint32_t)last_parity[s], abort_flag, p.err, false);
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            const uint32_t idesc = idesc_bf16(p.n_mma);
+            int stage = 0;
+            uint32_t phase = 0;
+            int acc = 0;
+            uint32_t acc_phase = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; ok && t < ntiles; t += gridDim.x) {
+                const Tile x = decode<MODE>(p, t);
+                if (!mbar_wait(tempty_bar(acc), acc_phase ^ 1u, abort_flag, p.err)) break;
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + (uint32_t)(acc * ACC_COLS);
+                for (int kb = 0; kb < x.num_kb; ++kb) {
+                    if (!mbar_wait(full_bar(stage), phase, abort_flag, p.err)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t a_addr = sA + stage * A_BYTES, b_addr = sB + stage * B_BYTES;
+#pragma unroll
+                    for (int k = 0; k < BK / 16; ++k) {
+                        mma_bf16(d_tmem, sw128_desc(a_addr + k * 32), sw128_desc(b_addr + k * 32), idesc,
+                                 (kb > 0 || k > 0) ? 1u : 0u);
+                    }
+                    mma_commit(empty_bar(stage));
+                    if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+                }
+                if (!ok) break;
+                mma_commit(tfull_bar(acc));
+                if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+            }
+            // drain: all MMAs issued by this thread have completed before TMEM is freed
+            mma_commit(drain_bar);
+            mbar_wait(drain_bar, 0, abort_flag, p.err, false);
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------------ epilogue
+        const int quad = warp & 3;                  // TMEM lanes 32*quad .. 32*quad+31
+        const int row = quad * 32 + lane;
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
+            const Tile x = decode<MODE>(p, t);
+            if (!mbar_wait(tfull_bar(acc), acc_phase, abort_flag, p.err)) break;
+            tc_fence_after();
+            const uint32_t tacc = tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(acc * ACC_COLS);
+            if (MODE == ROUTER) epilogue_router<KMAX>(p, x, tacc, row);
+            else if (MODE == GEMM1) epilogue_gemm1(p, x, tacc, row);
+            else if (MODE == GEMM2R) epilogue_gemm2r(p, x, tacc, row);
+            else epilogue_gemm2s(p, x, tacc, row);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(tempty_bar(acc));
+            if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(TMEM_COLS) : "memory");
+    }
+}
+
+// ------------------------------------------------------------------------------ host side
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = (EncodeTiledFn)ptr;
+    }
+    return fn;
+}
+
+// bf16 tensor [outer][mid][inner] (mid = 1 for 2-D) with a box of box_inner x box_mid (x 1)
+bool make_map(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t mid, uint64_t outer, uint32_t box_inner,
+              uint32_t box_mid, bool three_d) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {inner, mid, outer};
+    cuuint64_t strides[2] = {inner * 2, inner * mid * 2};
+    cuuint32_t box[3] = {box_inner, box_mid, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, three_d ? 3 : 2, const_cast<void*>(ptr), dims, strides, box,
+                    estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+template <int MODE, int KMAX>
+cudaError_t launch(const Params& p, int grid, cudaStream_t stream) {
+    auto kern = moe_tc_kernel<MODE, KMAX>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    kern<<<grid, THREADS, SMEM_BYTES, stream>>>(p);
+    return cudaGetLastError();
+}
+
+Params base_params(const Dims& D, uint32_t* err) {
+    Params p;
+    memset(&p, 0, sizeof(p));
+    p.T = D.T; p.d = D.d; p.E = D.E; p.I = D.I; p.Is = D.Ks > 0 ? D.Is : 8; p.k = D.k; p.Ks = D.Ks;
+    p.S = D.slots();
+    p.n_mma = 256;
+    p.err = err;
+    return p;
+}
+
+}  // namespace tc
+
+int num_sms() {
+    static int n = 0;
+    if (!n) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        if (n <= 0) n = 148;
+    }
+    return n;
+}
+
+bool tc_router_supported(const Dims& D) { return D.bf16 && D.E % 16 == 0 && D.E >= 16 && D.E <= 256; }
+
+cudaError_t launch_tc_router(const Dims& D, const void* x, const void* centroids, int32_t* idx, float* gate,
+                             uint32_t* err, cudaStream_t stream) {
+    using namespace tc;
+    if (D.T == 0) return cudaSuccess;
+    Params p = base_params(D, err);
+    p.n_mma = D.E;
+    p.idx_out = idx;
+    p.gate_out = gate;
+    if (!make_map(&p.tmA[0], x, D.d, D.T, 1, BK, BM, false)) return cudaErrorInvalidValue;
+    if (!make_map(&p.tmB[0], centroids, D.d, D.E, 1, BK, D.E, false)) return cudaErrorInvalidValue;
+    const int tiles = ceil_div(D.T, BM);
+    const int grid = tiles < num_sms() ? tiles : num_sms();
+    return D.k <= 8 ? launch<ROUTER, 8>(p, grid, stream) : launch<ROUTER, 32>(p, grid, stream);
+}
+
+cudaError_t launch_tc_gemm1(const Dims& D, const void* x, const void* x_perm, const int32_t* offsets,
+                            const int32_t* tile_start1, const FfnWeights& R, const FfnWeights& Sh, void* h_r, void* h_s,
+                            int g_begin, int g_end, uint32_t* err, cudaStream_t stream) {
+    using namespace tc;
+    if (D.T == 0 || g_end <= g_begin) return cudaSuccess;
+    Params p = base_params(D, err);
+    p.tile_start = tile_start1;
+    p.offsets = offsets;
+    p.g_begin = g_begin;
+    p.g_end = g_end;
+    p.b1 = (const __nv_bfloat16*)R.b1; p.b3 = (const __nv_bfloat16*)R.b3;
+    p.sb1 = (const __nv_bfloat16*)Sh.b1; p.sb3 = (const __nv_bfloat16*)Sh.b3;
+    p.h_r = (__nv_bfloat16*)h_r; p.h_s = (__nv_bfloat16*)h_s;
+    bool ok = true;
+    if (g_begin < D.E) {
+        ok &= make_map(&p.tmA[0], x_perm, D.d, (uint64_t)D.slots(), 1, BK, BM, false);
+        ok &= make_map(&p.tmB[0], R.w1, D.d, D.I, D.E, BK, 128, true);
+        ok &= make_map(&p.tmB[1], R.w3, D.d, D.I, D.E, BK, 128, true);
+    }
+    if (g_end > D.E) {
+        ok &= make_map(&p.tmA[1], x, D.d, D.T, 1, BK, BM, false);
+        ok &= make_map(&p.tmB[2], Sh.w1, D.d, D.Is, D.Ks, BK, 128, true);
+        ok &= make_map(&p.tmB[3], Sh.w3, D.d, D.Is, D.Ks, BK, 128, true);
+    }
+    if (!ok) return cudaErrorInvalidValue;
+    return launch<GEMM1, 8>(p, num_sms(), stream);
+}
+
+cudaError_t launch_tc_gemm2_routed(const Dims& D, const int32_t* offsets, const int32_t* tile_start2,
+                                   const float* sorted_gate, const FfnWeights& R, const void* h_r, void* y_sorted,
+                                   uint32_t* err, cudaStream_t stream) {
+    using namespace tc;
+    if (D.T == 0) return cudaSuccess;
+    Params p = base_params(D, err);
+    p.tile_start = tile_start2;
+    p.offsets = offsets;
+    p.sorted_gate = sorted_gate;
+    p.b2 = (const __nv_bfloat16*)R.b2;
+    p.y = (__nv_bfloat16*)y_sorted;
+    bool ok = make_map(&p.tmA[0], h_r, D.I, (uint64_t)D.slots(), 1, BK, BM, false);
+    ok &= make_map(&p.tmB[0], R.w2, D.I, D.d, D.E, BK, 256, true);
+    if (!ok) return cudaErrorInvalidValue;
+    return launch<GEMM2R, 8>(p, num_sms(), stream);
+}
+
+cudaError_t launch_tc_gemm2_shared(const Dims& D, const FfnWeights& Sh, const void* h_s, const void* y_sorted,
+                                   const int32_t* slot_of, void* out, uint32_t* err, cudaStream_t stream) {
+    using namespace tc;
+    if (D.T == 0 || D.Ks == 0) return cudaSuccess;
+    Params p = base_params(D, err);
+    p.sb2 = (const __nv_bfloat16*)Sh.b2;
+    p.y_in = (const __nv_bfloat16*)y_sorted;
+    p.slot_of = slot_of;
+    p.out = (__nv_bfloat16*)out;
+    bool ok = make_map(&p.tmA[0], h_s, D.Is, D.T, D.Ks, BK, BM, true);
+    ok &= make_map(&p.tmB[0], Sh.w2, D.Is, D.d, D.Ks, BK, 256, true);
+    if (!ok) return cudaErrorInvalidValue;
+    const int tiles = ceil_div(D.T, BM) * ceil_div(D.d, 256);
+    const int grid = tiles < num_sms() ? tiles : num_sms();
+    return launch<GEMM2S, 8>(p, grid, stream);
+}
+
+}  // namespace moe

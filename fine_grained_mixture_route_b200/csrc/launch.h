@@ -1,0 +1,90 @@
+// Host-side launchers of the sm_100a MoE kernels (internal to the library; the public
+// interface is include/moe.h).  Every launcher enqueues on `stream` and returns the
+// launch status; none of them synchronises.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace moe {
+
+// Layer sizes in the notation of the DeepSeekMoE report: T tokens, hidden d, E = N_m routed
+// experts of intermediate I, k = N_r picks per token, Ks = K_s shared experts of intermediate Is.
+struct Dims {
+    int T, d, E, I, k, Ks, Is;
+    bool bias;
+    bool bf16;
+    long long slots() const { return (long long)T * k; }
+};
+
+// ---- router ---------------------------------------------------------------------------
+// CUDA-core router for any dtype and N_m <= 1024: block-tiled scores, then one warp per
+// token for softmax and top-k.
+cudaError_t launch_router_simt(const Dims& D, const void* x, const void* centroids, int32_t* idx,
+                               float* gate, cudaStream_t stream);
+
+// ---- per-expert token lists -----------------------------------------------------------
+constexpr int PERMUTE_CHUNK = 1024;  // slots per histogram / scatter block
+inline int permute_blocks(const Dims& D) { return (int)((D.slots() + PERMUTE_CHUNK - 1) / PERMUTE_CHUNK); }
+
+cudaError_t launch_permute(const Dims& D, const int32_t* idx, const float* gate, int32_t* counts,
+                           int32_t* offsets, int32_t* sorted_token, float* sorted_gate, int32_t* slot_of,
+                           int32_t* block_hist, uint32_t* err, cudaStream_t stream);
+
+// Tile tables of the grouped GEMMs.  Groups 0..E-1 are the routed experts (rows from
+// offsets, or 0 when offsets is NULL), groups E..E+Ks-1 the shared experts (T rows each).
+// tile_start1[G+1]: GEMM1 tiles of 128 rows x 128 hidden columns; tile_start2[E+1]: routed
+// GEMM2 tiles of 128 rows x 256 output columns.
+cudaError_t launch_plan(const Dims& D, const int32_t* offsets, int32_t* tile_start1, int32_t* tile_start2,
+                        uint32_t* err, cudaStream_t stream);
+
+// x_perm[p, :] = x[sorted_token[p], :] (bf16 rows, 16-byte vectors).
+cudaError_t launch_gather(const Dims& D, const void* x, const int32_t* sorted_token, void* x_perm,
+                          uint32_t* err, cudaStream_t stream);
+
+// out[t, :] = sum_j y_sorted[slot_of[t*k + j], :] in fp32, rounded once (no shared experts).
+cudaError_t launch_combine(const Dims& D, const void* y_sorted, const int32_t* slot_of, void* out,
+                           uint32_t* err, cudaStream_t stream);
+
+// ---- CUDA-core grouped FFN (fp32 layers) ----------------------------------------------
+struct FfnWeights {
+    const void *w1, *b1, *w3, *b3, *w2, *b2;
+};
+
+// h rows of groups [g_begin, g_end): routed group e -> h_r[offsets[e] + r], shared group
+// E + s -> h_s[s*T + r].
+cudaError_t launch_simt_gemm1(const Dims& D, const void* x, const int32_t* offsets, const int32_t* sorted_token,
+                              const FfnWeights& routed, const FfnWeights& shared, void* h_r, void* h_s,
+                              int g_begin, int g_end, uint32_t* err, cudaStream_t stream);
+// y_sorted[p] = gate_p * (h_r[p] w2_e^T + b2_e)
+cudaError_t launch_simt_gemm2_routed(const Dims& D, const int32_t* offsets, const float* sorted_gate,
+                                     const FfnWeights& routed, const void* h_r, void* y_sorted,
+                                     uint32_t* err, cudaStream_t stream);
+// out[t] = sum_s (h_s[s, t] w2s_s^T + b2s_s) + sum_j y_sorted[slot_of[t*k+j]]   (Ks >= 1)
+cudaError_t launch_simt_gemm2_shared(const Dims& D, const FfnWeights& shared, const void* h_s,
+                                     const void* y_sorted, const int32_t* slot_of, void* out,
+                                     uint32_t* err, cudaStream_t stream);
+
+// ---- tensor-core (tcgen05 / TMEM / TMA) kernels for bf16 layers -------------------------
+// All four run the same persistent warp-specialised pipeline: a TMA producer warp, one MMA
+// issuing thread, four epilogue warps reading the fp32 accumulators out of tensor memory.
+bool tc_router_supported(const Dims& D);
+cudaError_t launch_tc_router(const Dims& D, const void* x, const void* centroids, int32_t* idx, float* gate,
+                             uint32_t* err, cudaStream_t stream);
+// GEMM1 + SwiGLU over groups [g_begin, g_end): A rows from x_perm (routed) or x (shared).
+cudaError_t launch_tc_gemm1(const Dims& D, const void* x, const void* x_perm, const int32_t* offsets,
+                            const int32_t* tile_start1, const FfnWeights& routed, const FfnWeights& shared,
+                            void* h_r, void* h_s, int g_begin, int g_end, uint32_t* err, cudaStream_t stream);
+// routed GEMM2 with the gate (and b2) applied in the epilogue -> y_sorted
+cudaError_t launch_tc_gemm2_routed(const Dims& D, const int32_t* offsets, const int32_t* tile_start2,
+                                   const float* sorted_gate, const FfnWeights& routed, const void* h_r,
+                                   void* y_sorted, uint32_t* err, cudaStream_t stream);
+// shared GEMM2 (all K_s experts accumulated along K) whose epilogue adds the routed rows
+// of every token in pick order -> out
+cudaError_t launch_tc_gemm2_shared(const Dims& D, const FfnWeights& shared, const void* h_s,
+                                   const void* y_sorted, const int32_t* slot_of, void* out, uint32_t* err,
+                                   cudaStream_t stream);
+
+int num_sms();
+
+}  // namespace moe

@@ -1,0 +1,316 @@
+// The C ABI of include/moe.h: argument validation, workspace layout, and the launch
+// sequence of each entry point on the caller's stream.  No allocation, no host sync (except
+// in moe_check_device_error), no exceptions.
+#include <cstring>
+
+#include "common.cuh"
+#include "launch.h"
+
+#define MOE_EXPORT __attribute__((visibility("default")))
+
+namespace moe {
+namespace {
+
+size_t al(size_t x) { return (x + 255) & ~(size_t)255; }
+
+struct Layout {
+    size_t err, hist, ts1, ts2, idx, gate, counts, offsets, stok, sgate, slot_of, xperm, hr, hs, y, total;
+};
+
+Layout layout(const Dims& D) {
+    Layout L;
+    const size_t S = (size_t)D.slots();
+    const size_t esz = D.bf16 ? 2 : 4;
+    const size_t nblk = (size_t)permute_blocks(D);
+    size_t o = 0;
+    L.err = o; o += 256;
+    L.hist = o; o += al((nblk ? nblk : 1) * D.E * 4);
+    L.ts1 = o; o += al((size_t)(D.E + D.Ks + 1) * 4);
+    L.ts2 = o; o += al((size_t)(D.E + 1) * 4);
+    L.idx = o; o += al(S * 4);
+    L.gate = o; o += al(S * 4);
+    L.counts = o; o += al((size_t)D.E * 4);
+    L.offsets = o; o += al((size_t)(D.E + 1) * 4);
+    L.stok = o; o += al(S * 4);
+    L.sgate = o; o += al(S * 4);
+    L.slot_of = o; o += al(S * 4);
+    L.xperm = o; o += D.bf16 ? al(S * D.d * esz) : 0;
+    L.hr = o; o += al(S * D.I * esz);
+    L.hs = o; o += al((size_t)D.Ks * D.T * (D.Ks ? D.Is : 0) * esz);
+    L.y = o; o += al(S * D.d * esz);
+    L.total = o;
+    return L;
+}
+
+moe_status_t to_dims(const moe_shape_t* s, Dims* D) {
+    if (!s) return MOE_ERR_INVALID_ARG;
+    if (s->dtype != MOE_F32 && s->dtype != MOE_BF16) return MOE_ERR_INVALID_ARG;
+    if (s->T < 0 || s->d < 1 || s->n_experts < 1 || s->inter < 1 || s->top_k < 1 || s->n_shared < 0)
+        return MOE_ERR_INVALID_ARG;
+    if (s->top_k > s->n_experts) return MOE_ERR_INVALID_ARG;
+    if (s->n_shared > 0 && s->inter_shared < 1) return MOE_ERR_INVALID_ARG;
+    if (s->has_bias != 0 && s->has_bias != 1) return MOE_ERR_INVALID_ARG;
+    if ((long long)s->T * s->top_k >= (1LL << 31)) return MOE_ERR_UNSUPPORTED;
+    if (s->n_experts > 1024 || s->top_k > 32 || s->n_shared > 16) return MOE_ERR_UNSUPPORTED;
+    if (s->dtype == MOE_BF16) {
+        if (s->d % 8 || s->inter % 8 || (s->n_shared > 0 && s->inter_shared % 8)) return MOE_ERR_UNSUPPORTED;
+    }
+    D->T = s->T; D->d = s->d; D->E = s->n_experts; D->I = s->inter; D->k = s->top_k;
+    D->Ks = s->n_shared; D->Is = s->n_shared > 0 ? s->inter_shared : 0;
+    D->bias = s->has_bias != 0; D->bf16 = s->dtype == MOE_BF16;
+    return MOE_OK;
+}
+
+moe_status_t check_ws(const Dims& D, void* ws, size_t ws_bytes) {
+    if (!ws || ws_bytes < layout(D).total || ((uintptr_t)ws & 15u)) return MOE_ERR_WORKSPACE;
+    return MOE_OK;
+}
+
+moe_status_t check_weights(const Dims& D, const moe_ffn_weights_t* w) {
+    if (!w || !w->w1 || !w->w3 || !w->w2) return MOE_ERR_INVALID_ARG;
+    const bool b = w->b1 && w->b3 && w->b2;
+    const bool none = !w->b1 && !w->b3 && !w->b2;
+    if (D.bias ? !b : !none) return MOE_ERR_INVALID_ARG;
+    return MOE_OK;
+}
+
+moe_status_t check_device() {
+    int dev = 0, major = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return MOE_ERR_CUDA;
+    if (major != 10) return MOE_ERR_UNSUPPORTED;   // built for sm_100a only
+    return MOE_OK;
+}
+
+#define MOE_TRY(expr)                              \
+    do {                                           \
+        moe_status_t _s = (expr);                  \
+        if (_s != MOE_OK) return _s;               \
+    } while (0)
+#define MOE_CUDA(expr)                             \
+    do {                                           \
+        if ((expr) != cudaSuccess) return MOE_ERR_CUDA; \
+    } while (0)
+
+template <typename T>
+T* at(void* ws, size_t off) { return reinterpret_cast<T*>(static_cast<char*>(ws) + off); }
+
+FfnWeights to_ffn(const moe_ffn_weights_t* w) {
+    FfnWeights f = {nullptr, nullptr, nullptr, nullptr, nullptr, nullptr};
+    if (w) { f.w1 = w->w1; f.b1 = w->b1; f.w3 = w->w3; f.b3 = w->b3; f.w2 = w->w2; f.b2 = w->b2; }
+    return f;
+}
+
+moe_status_t do_route(const Dims& D, const void* x, const void* c, int32_t* idx, float* gate, uint32_t* err,
+                      cudaStream_t st) {
+    if (D.T == 0) return MOE_OK;
+    if (tc_router_supported(D)) MOE_CUDA(launch_tc_router(D, x, c, idx, gate, err, st));
+    else MOE_CUDA(launch_router_simt(D, x, c, idx, gate, st));
+    return MOE_OK;
+}
+
+// routed experts: y_sorted = gate * FFN_e(x[sorted_token])
+moe_status_t do_expert_ffn(const Dims& D, const Layout& L, void* ws, const void* x, const int32_t* offsets,
+                           const int32_t* stok, const float* sgate, const FfnWeights& R, void* y, bool plan_done,
+                           cudaStream_t st) {
+    uint32_t* err = at<uint32_t>(ws, L.err);
+    int32_t* ts1 = at<int32_t>(ws, L.ts1);
+    int32_t* ts2 = at<int32_t>(ws, L.ts2);
+    if (!plan_done) MOE_CUDA(launch_plan(D, offsets, ts1, ts2, err, st));
+    if (D.bf16) {
+        void* xp = at<void>(ws, L.xperm);
+        MOE_CUDA(launch_gather(D, x, stok, xp, err, st));
+        FfnWeights none = {nullptr, nullptr, nullptr, nullptr, nullptr, nullptr};
+        MOE_CUDA(launch_tc_gemm1(D, x, xp, offsets, ts1, R, none, at<void>(ws, L.hr), nullptr, 0, D.E, err, st));
+        MOE_CUDA(launch_tc_gemm2_routed(D, offsets, ts2, sgate, R, at<void>(ws, L.hr), y, err, st));
+    } else {
+        FfnWeights none = {nullptr, nullptr, nullptr, nullptr, nullptr, nullptr};
+        MOE_CUDA(launch_simt_gemm1(D, x, offsets, stok, R, none, at<void>(ws, L.hr), nullptr, 0, D.E, err, st));
+        MOE_CUDA(launch_simt_gemm2_routed(D, offsets, sgate, R, at<void>(ws, L.hr), y, err, st));
+    }
+    return MOE_OK;
+}
+
+}  // namespace
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+MOE_EXPORT size_t moe_workspace_bytes(const moe_shape_t* shape) {
+    Dims D;
+    if (to_dims(shape, &D) != MOE_OK) return 0;
+    return layout(D).total;
+}
+
+MOE_EXPORT const char* moe_status_string(moe_status_t s) {
+    switch (s) {
+        case MOE_OK: return "MOE_OK";
+        case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG: null pointer, size out of range or bias mismatch";
+        case MOE_ERR_UNSUPPORTED: return "MOE_ERR_UNSUPPORTED: valid layer outside what these kernels handle";
+        case MOE_ERR_WORKSPACE: return "MOE_ERR_WORKSPACE: workspace missing, misaligned or too small";
+        case MOE_ERR_CUDA: return "MOE_ERR_CUDA: a CUDA call or kernel launch failed";
+        case MOE_ERR_INTERNAL: return "MOE_ERR_INTERNAL: a kernel flagged an error";
+    }
+    return "MOE_ERR_UNKNOWN";
+}
+
+MOE_EXPORT const char* moe_version(void) { return "moe_b200 0.1 sm_100a"; }
+
+MOE_EXPORT moe_status_t moe_ws_init(void* ws, size_t ws_bytes, moe_stream_t stream) {
+    if (!ws || ws_bytes < 256) return MOE_ERR_WORKSPACE;
+    if (cudaMemsetAsync(ws, 0, 256, (cudaStream_t)stream) != cudaSuccess) return MOE_ERR_CUDA;
+    return MOE_OK;
+}
+
+MOE_EXPORT moe_status_t moe_check_device_error(void* ws, size_t ws_bytes, moe_stream_t stream, uint32_t* detail) {
+    if (!ws || ws_bytes < 256) return MOE_ERR_WORKSPACE;
+    cudaStream_t st = (cudaStream_t)stream;
+    uint32_t h = 0;
+    if (cudaMemcpyAsync(&h, ws, sizeof(h), cudaMemcpyDeviceToHost, st) != cudaSuccess) return MOE_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return MOE_ERR_CUDA;
+    if (detail) *detail = h;
+    if (h) {
+        if (cudaMemsetAsync(ws, 0, sizeof(h), st) != cudaSuccess) return MOE_ERR_CUDA;
+        if (cudaStreamSynchronize(st) != cudaSuccess) return MOE_ERR_CUDA;
+        return MOE_ERR_INTERNAL;
+    }
+    return MOE_OK;
+}
+
+MOE_EXPORT moe_status_t moe_route(const moe_shape_t* shape, const void* x, const void* centroids, int32_t* topk_idx,
+                                  float* topk_gate, void* ws, size_t ws_bytes, moe_stream_t stream) {
+    Dims D;
+    MOE_TRY(to_dims(shape, &D));
+    if (!x || !centroids || !topk_idx || !topk_gate) return MOE_ERR_INVALID_ARG;
+    MOE_TRY(check_ws(D, ws, ws_bytes));
+    if (D.T == 0) return MOE_OK;
+    MOE_TRY(check_device());
+    cudaGetLastError();
+    const Layout L = layout(D);
+    return do_route(D, x, centroids, topk_idx, topk_gate, at<uint32_t>(ws, L.err), (cudaStream_t)stream);
+}
+
+MOE_EXPORT moe_status_t moe_permute(const moe_shape_t* shape, const int32_t* topk_idx, const float* topk_gate,
+                                    int32_t* counts, int32_t* offsets, int32_t* sorted_token, float* sorted_gate,
+                                    int32_t* slot_of, void* ws, size_t ws_bytes, moe_stream_t stream) {
+    Dims D;
+    MOE_TRY(to_dims(shape, &D));
+    if (!counts || !offsets || (D.T > 0 && (!topk_idx || !topk_gate || !sorted_token || !sorted_gate || !slot_of)))
+        return MOE_ERR_INVALID_ARG;
+    MOE_TRY(check_ws(D, ws, ws_bytes));
+    MOE_TRY(check_device());
+    cudaGetLastError();
+    const Layout L = layout(D);
+    MOE_CUDA(launch_permute(D, topk_idx, topk_gate, counts, offsets, sorted_token, sorted_gate, slot_of,
+                            at<int32_t>(ws, L.hist), at<uint32_t>(ws, L.err), (cudaStream_t)stream));
+    return MOE_OK;
+}
+
+MOE_EXPORT moe_status_t moe_expert_ffn(const moe_shape_t* shape, const void* x, const int32_t* offsets,
+                                       const int32_t* sorted_token, const float* sorted_gate,
+                                       const moe_ffn_weights_t* routed, void* y_sorted, void* ws, size_t ws_bytes,
+                                       moe_stream_t stream) {
+    Dims D;
+    MOE_TRY(to_dims(shape, &D));
+    if (!x || !offsets || !sorted_token || !y_sorted) return MOE_ERR_INVALID_ARG;
+    MOE_TRY(check_weights(D, routed));
+    MOE_TRY(check_ws(D, ws, ws_bytes));
+    if (D.T == 0) return MOE_OK;
+    MOE_TRY(check_device());
+    cudaGetLastError();
+    const Layout L = layout(D);
+    return do_expert_ffn(D, L, ws, x, offsets, sorted_token, sorted_gate, to_ffn(routed), y_sorted, false,
+                         (cudaStream_t)stream);
+}
+
+MOE_EXPORT moe_status_t moe_combine(const moe_shape_t* shape, const void* x, const moe_ffn_weights_t* shared,
+                                    const void* y_sorted, const int32_t* slot_of, void* out, void* ws,
+                                    size_t ws_bytes, moe_stream_t stream) {
+    Dims D;
+    MOE_TRY(to_dims(shape, &D));
+    if (!y_sorted || !slot_of || !out) return MOE_ERR_INVALID_ARG;
+    if (D.Ks > 0) {
+        if (!x) return MOE_ERR_INVALID_ARG;
+        MOE_TRY(check_weights(D, shared));
+    } else if (shared) {
+        return MOE_ERR_INVALID_ARG;
+    }
+    MOE_TRY(check_ws(D, ws, ws_bytes));
+    if (D.T == 0) return MOE_OK;
+    MOE_TRY(check_device());
+    cudaGetLastError();
+    const Layout L = layout(D);
+    cudaStream_t st = (cudaStream_t)stream;
+    uint32_t* err = at<uint32_t>(ws, L.err);
+    if (D.Ks == 0) {
+        MOE_CUDA(launch_combine(D, y_sorted, slot_of, out, err, st));
+        return MOE_OK;
+    }
+    const FfnWeights Sh = to_ffn(shared);
+    const FfnWeights none = {nullptr, nullptr, nullptr, nullptr, nullptr, nullptr};
+    void* hs = at<void>(ws, L.hs);
+    if (D.bf16) {
+        int32_t* ts1 = at<int32_t>(ws, L.ts1);
+        MOE_CUDA(launch_plan(D, nullptr, ts1, at<int32_t>(ws, L.ts2), err, st));
+        MOE_CUDA(launch_tc_gemm1(D, x, nullptr, nullptr, ts1, none, Sh, nullptr, hs, D.E, D.E + D.Ks, err, st));
+        MOE_CUDA(launch_tc_gemm2_shared(D, Sh, hs, y_sorted, slot_of, out, err, st));
+    } else {
+        MOE_CUDA(launch_simt_gemm1(D, x, nullptr, nullptr, none, Sh, nullptr, hs, D.E, D.E + D.Ks, err, st));
+        MOE_CUDA(launch_simt_gemm2_shared(D, Sh, hs, y_sorted, slot_of, out, err, st));
+    }
+    return MOE_OK;
+}
+
+MOE_EXPORT moe_status_t moe_layer_forward(const moe_shape_t* shape, const void* x, const void* centroids,
+                                          const moe_ffn_weights_t* routed, const moe_ffn_weights_t* shared, void* out,
+                                          int32_t* topk_idx_out, float* topk_gate_out, int32_t* counts_out, void* ws,
+                                          size_t ws_bytes, moe_stream_t stream) {
+    Dims D;
+    MOE_TRY(to_dims(shape, &D));
+    if (!x || !centroids || !out) return MOE_ERR_INVALID_ARG;
+    MOE_TRY(check_weights(D, routed));
+    if (D.Ks > 0) MOE_TRY(check_weights(D, shared));
+    else if (shared) return MOE_ERR_INVALID_ARG;
+    MOE_TRY(check_ws(D, ws, ws_bytes));
+    if (D.T == 0) return MOE_OK;
+    MOE_TRY(check_device());
+    cudaGetLastError();
+    const Layout L = layout(D);
+    cudaStream_t st = (cudaStream_t)stream;
+    uint32_t* err = at<uint32_t>(ws, L.err);
+    int32_t* idx = topk_idx_out ? topk_idx_out : at<int32_t>(ws, L.idx);
+    float* gate = topk_gate_out ? topk_gate_out : at<float>(ws, L.gate);
+    int32_t* counts = counts_out ? counts_out : at<int32_t>(ws, L.counts);
+    int32_t* offsets = at<int32_t>(ws, L.offsets);
+    int32_t* stok = at<int32_t>(ws, L.stok);
+    float* sgate = at<float>(ws, L.sgate);
+    int32_t* slot_of = at<int32_t>(ws, L.slot_of);
+    void* y = at<void>(ws, L.y);
+    void* hr = at<void>(ws, L.hr);
+    void* hs = at<void>(ws, L.hs);
+    int32_t* ts1 = at<int32_t>(ws, L.ts1);
+    int32_t* ts2 = at<int32_t>(ws, L.ts2);
+    const FfnWeights R = to_ffn(routed), Sh = to_ffn(shared);
+
+    MOE_TRY(do_route(D, x, centroids, idx, gate, err, st));
+    MOE_CUDA(launch_permute(D, idx, gate, counts, offsets, stok, sgate, slot_of, at<int32_t>(ws, L.hist), err, st));
+    MOE_CUDA(launch_plan(D, offsets, ts1, ts2, err, st));
+    if (D.bf16) {
+        void* xp = at<void>(ws, L.xperm);
+        MOE_CUDA(launch_gather(D, x, stok, xp, err, st));
+        MOE_CUDA(launch_tc_gemm1(D, x, xp, offsets, ts1, R, Sh, hr, hs, 0, D.E + D.Ks, err, st));
+        MOE_CUDA(launch_tc_gemm2_routed(D, offsets, ts2, sgate, R, hr, y, err, st));
+        if (D.Ks > 0) MOE_CUDA(launch_tc_gemm2_shared(D, Sh, hs, y, slot_of, out, err, st));
+        else MOE_CUDA(launch_combine(D, y, slot_of, out, err, st));
+    } else {
+        MOE_CUDA(launch_simt_gemm1(D, x, offsets, stok, R, Sh, hr, hs, 0, D.E + D.Ks, err, st));
+        MOE_CUDA(launch_simt_gemm2_routed(D, offsets, sgate, R, hr, y, err, st));
+        if (D.Ks > 0) MOE_CUDA(launch_simt_gemm2_shared(D, Sh, hs, y, slot_of, out, err, st));
+        else MOE_CUDA(launch_combine(D, y, slot_of, out, err, st));
+    }
+    return MOE_OK;
+}
+
+}  // extern "C"

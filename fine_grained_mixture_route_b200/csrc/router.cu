@@ -1,0 +1,124 @@
+// CUDA-core router of the DeepSeekMoE layer ("《DeepSeekMoE》深度解读报告" §3.1, Eq. 3-5 in
+// prose): z = x . e_i for every expert centroid, softmax over all N_m experts, keep the
+// N_r largest probabilities as gates (no renormalisation; ties to the lower index).
+//
+// Used for fp32 layers and for expert counts the tensor-core router does not take.  Phase
+// 1 computes a [32 tokens x N_m] block of fp32 logits from shared-memory tiles of x and the
+// centroids; phase 2 gives each token to one warp, which keeps the token's logits in shared
+// memory, reduces max and sum-of-exponentials with shuffles and takes N_r rounds of warp
+// argmax on the key (logit, -index).
+#include "common.cuh"
+#include "launch.h"
+
+namespace moe {
+namespace {
+
+constexpr int RT_TOK = 32;      // tokens per block
+constexpr int RT_EXP = 64;      // experts per score tile
+constexpr int RT_K = 64;        // hidden elements per score tile
+constexpr int RT_THREADS = 256;
+
+template <typename T>
+__global__ void __launch_bounds__(RT_THREADS)
+router_simt_kernel(const T* __restrict__ x, const T* __restrict__ cen, int32_t* __restrict__ idx_out,
+                   float* __restrict__ gate_out, int Tn, int d, int E, int k) {
+    extern __shared__ float sm[];
+    float* xs = sm;                                  // [RT_TOK][RT_K + 1]
+    float* cs = xs + RT_TOK * (RT_K + 1);            // [RT_EXP][RT_K + 1]
+    float* z = cs + RT_EXP * (RT_K + 1);             // [RT_TOK][E]
+    const int t0 = blockIdx.x * RT_TOK;
+    const int tid = threadIdx.x;
+    const int tt = tid / 8;                          // token of this thread in phase 1
+    const int eo = tid % 8;                          // expert lane: experts eo + 8q
+
+    for (int e0 = 0; e0 < E; e0 += RT_EXP) {
+        float acc[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) acc[q] = 0.f;
+        for (int k0 = 0; k0 < d; k0 += RT_K) {
+            __syncthreads();
+            for (int i = tid; i < RT_TOK * RT_K; i += RT_THREADS) {
+                int r = i / RT_K, c = i % RT_K;
+                int t = t0 + r, kk = k0 + c;
+                xs[r * (RT_K + 1) + c] = (t < Tn && kk < d) ? to_f32(x[(size_t)t * d + kk]) : 0.f;
+            }
+            for (int i = tid; i < RT_EXP * RT_K; i += RT_THREADS) {
+                int r = i / RT_K, c = i % RT_K;
+                int e = e0 + r, kk = k0 + c;
+                cs[r * (RT_K + 1) + c] = (e < E && kk < d) ? to_f32(cen[(size_t)e * d + kk]) : 0.f;
+            }
+            __syncthreads();
+#pragma unroll 4
+            for (int c = 0; c < RT_K; ++c) {
+                float xv = xs[tt * (RT_K + 1) + c];
+#pragma unroll
+                for (int q = 0; q < 8; ++q) acc[q] = fmaf(xv, cs[(eo + 8 * q) * (RT_K + 1) + c], acc[q]);
+            }
+        }
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            int e = e0 + eo + 8 * q;
+            if (e < E) z[tt * E + e] = acc[q];
+        }
+    }
+    __syncthreads();
+
+    // phase 2: one warp per token
+    const int warp = tid / 32, lane = tid % 32;
+    for (int r = warp; r < RT_TOK; r += RT_THREADS / 32) {
+        const int t = t0 + r;
+        if (t >= Tn) break;
+        float* zr = z + r * E;
+        float m = -INFINITY;
+        for (int e = lane; e < E; e += 32) m = fmaxf(m, zr[e]);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        float s = 0.f;
+        for (int e = lane; e < E; e += 32) s += expf(zr[e] - m);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+        const float inv = 1.0f / s;
+        for (int j = 0; j < k; ++j) {
+            float bv = -INFINITY;
+            int bi = 0x7fffffff;
+            for (int e = lane; e < E; e += 32) {
+                float v = zr[e];
+                if (v > bv) { bv = v; bi = e; }     // ascending e: equal values keep the lower index
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+                int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+                if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
+            }
+            if (lane == 0) {
+                idx_out[(size_t)t * k + j] = bi;
+                gate_out[(size_t)t * k + j] = expf(bv - m) * inv;
+            }
+            if (bi < E && (bi % 32) == lane) zr[bi] = -INFINITY;   // owner lane removes the pick
+            __syncwarp();
+        }
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_router_simt(const Dims& D, const void* x, const void* centroids, int32_t* idx, float* gate,
+                               cudaStream_t stream) {
+    const int blocks = ceil_div(D.T, RT_TOK);
+    const size_t smem = sizeof(float) * ((size_t)RT_TOK * (RT_K + 1) + (size_t)RT_EXP * (RT_K + 1) + (size_t)RT_TOK * D.E);
+    if (D.bf16) {
+        auto kern = router_simt_kernel<__nv_bfloat16>;
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        kern<<<blocks, RT_THREADS, smem, stream>>>((const __nv_bfloat16*)x, (const __nv_bfloat16*)centroids, idx, gate,
+                                                   D.T, D.d, D.E, D.k);
+    } else {
+        auto kern = router_simt_kernel<float>;
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        kern<<<blocks, RT_THREADS, smem, stream>>>((const float*)x, (const float*)centroids, idx, gate, D.T, D.d, D.E,
+                                                   D.k);
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,206 @@
+"""Thin ctypes binding of the C ABI in include/moe.h, taking torch tensors.
+
+Argument marshalling only: every step of the layer runs in the library's sm_100a kernels.
+torch supplies device memory and the current CUDA stream.  There is no fallback: if the
+shared library is missing or the device is not a B200, calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Dict, Optional
+
+import torch
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe_b200.so")
+
+MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_CUDA, MOE_ERR_INTERNAL = range(6)
+MOE_F32, MOE_BF16 = 0, 1
+
+EXPORTED = ("moe_workspace_bytes", "moe_status_string", "moe_version", "moe_check_device_error", "moe_ws_init",
+            "moe_route", "moe_permute", "moe_expert_ffn", "moe_combine", "moe_layer_forward")
+
+
+class MoeShape(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in
+                ("T", "d", "n_experts", "inter", "top_k", "n_shared", "inter_shared", "has_bias", "dtype")]
+
+
+class MoeWeights(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in ("w1", "b1", "w3", "b3", "w2", "b2")]
+
+
+class MoeError(RuntimeError):
+    def __init__(self, status: int, where: str, detail: int = 0):
+        self.status = status
+        self.detail = detail
+        msg = _lib().moe_status_string(status).decode()
+        super().__init__(f"{where}: {msg}" + (f" (device error bits {detail:#x})" if detail else ""))
+
+
+_LIB = None
+
+
+def _lib():
+    global _LIB
+    if _LIB is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with `python -m fine_grained_mixture_route_b200.build`")
+        lib = ctypes.CDLL(LIB_PATH)
+        vp, sz, i32p, f32p = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p, ctypes.c_void_p
+        sh = ctypes.POINTER(MoeShape)
+        wp = ctypes.POINTER(MoeWeights)
+        lib.moe_workspace_bytes.argtypes = [sh]
+        lib.moe_workspace_bytes.restype = sz
+        lib.moe_status_string.argtypes = [ctypes.c_int]
+        lib.moe_status_string.restype = ctypes.c_char_p
+        lib.moe_version.argtypes = []
+        lib.moe_version.restype = ctypes.c_char_p
+        lib.moe_check_device_error.argtypes = [vp, sz, vp, ctypes.POINTER(ctypes.c_uint32)]
+        lib.moe_ws_init.argtypes = [vp, sz, vp]
+        lib.moe_route.argtypes = [sh, vp, vp, i32p, f32p, vp, sz, vp]
+        lib.moe_permute.argtypes = [sh, i32p, f32p, i32p, i32p, i32p, f32p, i32p, vp, sz, vp]
+        lib.moe_expert_ffn.argtypes = [sh, vp, i32p, i32p, f32p, wp, vp, vp, sz, vp]
+        lib.moe_combine.argtypes = [sh, vp, wp, vp, i32p, vp, vp, sz, vp]
+        lib.moe_layer_forward.argtypes = [sh, vp, vp, wp, wp, vp, i32p, f32p, i32p, vp, sz, vp]
+        for n in ("moe_check_device_error", "moe_ws_init", "moe_route", "moe_permute", "moe_expert_ffn",
+                  "moe_combine", "moe_layer_forward"):
+            getattr(lib, n).restype = ctypes.c_int
+        _LIB = lib
+    return _LIB
+
+
+def lib_handle():
+    """The loaded ctypes library (for tests that check the exported symbols)."""
+    return _lib()
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(status: int, where: str):
+    if status != MOE_OK:
+        raise MoeError(status, where)
+
+
+def make_shape(T: int, d: int, n_experts: int, inter: int, top_k: int, n_shared: int = 0, inter_shared: int = 0,
+               has_bias: bool = True, dtype: torch.dtype = torch.bfloat16) -> MoeShape:
+    return MoeShape(T, d, n_experts, inter, top_k, n_shared, inter_shared if n_shared else 0, int(bool(has_bias)),
+                    MOE_BF16 if dtype == torch.bfloat16 else MOE_F32)
+
+
+def shape_of(x: torch.Tensor, centroids_or_E, routed: Dict, top_k: int, shared: Optional[Dict] = None) -> MoeShape:
+    E = centroids_or_E if isinstance(centroids_or_E, int) else centroids_or_E.shape[0]
+    I = routed["w1"].shape[1]
+    Ks = 0 if shared is None else shared["w1"].shape[0]
+    Is = 0 if shared is None else shared["w1"].shape[1]
+    return make_shape(x.shape[0], x.shape[1], E, I, top_k, Ks, Is, routed.get("b1") is not None, x.dtype)
+
+
+def _weights(w: Optional[Dict]):
+    if w is None:
+        return None
+    for k in ("w1", "w3", "w2", "b1", "b3", "b2"):
+        t = w.get(k)
+        if t is not None and not t.is_contiguous():
+            raise ValueError(f"weight {k} must be contiguous")
+    return MoeWeights(*(None if w.get(k) is None else w[k].data_ptr() for k in ("w1", "b1", "w3", "b3", "w2", "b2")))
+
+
+def workspace_bytes(shape: MoeShape) -> int:
+    return int(_lib().moe_workspace_bytes(ctypes.byref(shape)))
+
+
+def new_workspace(shape: MoeShape, device="cuda") -> torch.Tensor:
+    n = workspace_bytes(shape)
+    if n == 0:
+        raise ValueError("invalid layer shape")
+    ws = torch.empty(n, dtype=torch.uint8, device=device)
+    _check(_lib().moe_ws_init(_ptr(ws), n, _stream()), "moe_ws_init")
+    return ws
+
+
+def check_device_error(ws: torch.Tensor, stream=None) -> int:
+    """Synchronises the stream and raises MoeError if a kernel flagged an error."""
+    detail = ctypes.c_uint32(0)
+    st = _lib().moe_check_device_error(_ptr(ws), ws.numel(), _stream(stream), ctypes.byref(detail))
+    if st != MOE_OK:
+        raise MoeError(st, "moe_check_device_error", detail.value)
+    return 0
+
+
+def route(shape: MoeShape, x, centroids, ws, idx=None, gate=None, stream=None):
+    T, k = shape.T, shape.top_k
+    idx = torch.empty((T, k), dtype=torch.int32, device=x.device) if idx is None else idx
+    gate = torch.empty((T, k), dtype=torch.float32, device=x.device) if gate is None else gate
+    _check(_lib().moe_route(ctypes.byref(shape), _ptr(x), _ptr(centroids), _ptr(idx), _ptr(gate), _ptr(ws),
+                            ws.numel(), _stream(stream)), "moe_route")
+    return idx, gate
+
+
+def permute(shape: MoeShape, idx, gate, ws, stream=None):
+    S, E = shape.T * shape.top_k, shape.n_experts
+    dev = idx.device
+    counts = torch.empty(E, dtype=torch.int32, device=dev)
+    offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    sorted_token = torch.empty(S, dtype=torch.int32, device=dev)
+    sorted_gate = torch.empty(S, dtype=torch.float32, device=dev)
+    slot_of = torch.empty(S, dtype=torch.int32, device=dev)
+    _check(_lib().moe_permute(ctypes.byref(shape), _ptr(idx), _ptr(gate), _ptr(counts), _ptr(offsets),
+                              _ptr(sorted_token), _ptr(sorted_gate), _ptr(slot_of), _ptr(ws), ws.numel(),
+                              _stream(stream)), "moe_permute")
+    return {"counts": counts, "offsets": offsets, "sorted_token": sorted_token, "sorted_gate": sorted_gate,
+            "slot_of": slot_of}
+
+
+def expert_ffn(shape: MoeShape, x, offsets, sorted_token, sorted_gate, routed: Dict, ws, y=None, stream=None):
+    S = shape.T * shape.top_k
+    y = torch.empty((S, shape.d), dtype=x.dtype, device=x.device) if y is None else y
+    w = _weights(routed)
+    _check(_lib().moe_expert_ffn(ctypes.byref(shape), _ptr(x), _ptr(offsets), _ptr(sorted_token), _ptr(sorted_gate),
+                                 ctypes.byref(w), _ptr(y), _ptr(ws), ws.numel(), _stream(stream)), "moe_expert_ffn")
+    return y
+
+
+def combine(shape: MoeShape, x, shared: Optional[Dict], y_sorted, slot_of, ws, out=None, stream=None):
+    out = torch.empty((shape.T, shape.d), dtype=y_sorted.dtype, device=y_sorted.device) if out is None else out
+    w = _weights(shared)
+    _check(_lib().moe_combine(ctypes.byref(shape), _ptr(x), None if w is None else ctypes.byref(w), _ptr(y_sorted),
+                              _ptr(slot_of), _ptr(out), _ptr(ws), ws.numel(), _stream(stream)), "moe_combine")
+    return out
+
+
+def layer_forward(shape: MoeShape, x, centroids, routed: Dict, shared: Optional[Dict], ws, out=None,
+                  idx=None, gate=None, counts=None, stream=None):
+    """One call of the whole layer; idx / gate / counts are optional output tensors."""
+    out = torch.empty((shape.T, shape.d), dtype=x.dtype, device=x.device) if out is None else out
+    rw = _weights(routed)
+    sw = _weights(shared)
+    _check(_lib().moe_layer_forward(ctypes.byref(shape), _ptr(x), _ptr(centroids), ctypes.byref(rw),
+                                    None if sw is None else ctypes.byref(sw), _ptr(out), _ptr(idx), _ptr(gate),
+                                    _ptr(counts), _ptr(ws), ws.numel(), _stream(stream)), "moe_layer_forward")
+    return out
+
+
+class MoELayer:
+    """Convenience holder: the layer's device tensors, its shape and one workspace."""
+
+    def __init__(self, centroids: torch.Tensor, routed: Dict, shared: Optional[Dict], top_k: int, max_tokens: int):
+        self.centroids, self.routed, self.shared, self.top_k = centroids, routed, shared, top_k
+        self.max_tokens = max_tokens
+        dummy = torch.empty((max_tokens, centroids.shape[1]), dtype=centroids.dtype, device="meta")
+        self.shape_max = shape_of(dummy, centroids, routed, top_k, shared)
+        self.ws = new_workspace(self.shape_max, centroids.device)
+
+    def __call__(self, x: torch.Tensor, out=None, idx=None, gate=None, counts=None, stream=None):
+        if x.shape[0] > self.max_tokens:
+            raise ValueError("more tokens than the workspace was sized for")
+        shape = shape_of(x, self.centroids, self.routed, self.top_k, self.shared)
+        return layer_forward(shape, x, self.centroids, self.routed, self.shared, self.ws, out, idx, gate, counts,
+                             stream)

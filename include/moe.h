@@ -1,0 +1,182 @@
+/*
+ * moe.h — C ABI of the B200 (sm_100a) DeepSeekMoE layer forward.
+ *
+ * The layer (as defined in "《DeepSeekMoE》深度解读报告", §2.2-§2.3 and §3.1, Eq. 3-5 and
+ * Eq. 9-11 in prose, with the per-expert FFN of the `Expert` module in "DeepSeek MoE模型
+ * 优化与未来演进及字节超稀疏内存技术"):
+ *
+ *   z[t,i]   = x[t,:] . centroids[i,:]                      (no scale, no router bias)
+ *   s[t,:]   = softmax_i z[t,:]                             (over all N_m routed experts)
+ *   picks    = the top_k largest s[t,i]; gate = s at the picks, NOT renormalised
+ *   FFN_e(u) = w2_e( silu(w1_e u + b1_e) * (w3_e u + b3_e) ) + b2_e
+ *   out[t,:] = sum_{k<K_s} FFN^shared_k(x[t]) + sum_{j<top_k} gate[t,j] * FFN_{idx[t,j]}(x[t])
+ *
+ * The gate multiplies the whole expert output, bias included.  The residual connection of
+ * the original paper is not part of this layer; callers add it.  Ties between equal scores
+ * go to the lower expert index; the picks of a token are stored by descending score.
+ *
+ * Conventions shared by every entry point:
+ *  - Every pointer argument is DEVICE memory owned by the caller.  The library allocates
+ *    nothing and keeps no state between calls: every intermediate lives in the caller's
+ *    workspace `ws` of at least moe_workspace_bytes(shape) bytes (16-byte aligned or better;
+ *    256-byte alignment recommended).  One workspace serves every entry point of one shape.
+ *  - Every compute call is asynchronous on `stream` (NULL = the legacy default stream) and
+ *    does no host synchronisation.  Calls that share a workspace must be ordered on one
+ *    stream; calls with distinct workspaces may run concurrently.
+ *  - Argument errors are returned synchronously before any launch (MOE_ERR_INVALID_ARG,
+ *    MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE).  A failed launch returns MOE_ERR_CUDA.
+ *    Errors the kernels detect (an expert index out of range, a bounded wait that ran out)
+ *    are recorded in an error word inside the workspace and reported by
+ *    moe_check_device_error().  No C++ exception crosses this interface.
+ *  - Data types are uniform per call: x, centroids, all weights and biases, hidden states,
+ *    routed outputs and `out` share shape->dtype (MOE_F32 or MOE_BF16).  Gates are always
+ *    fp32; indices and counts are int32.  Accumulation is fp32 for both data types.
+ *  - Layouts are row-major.  Stacked expert weights use the nn.Linear [out, in] layout:
+ *    w1, w3: [E, inter, d]; w2: [E, d, inter]; b1, b3: [E, inter]; b2: [E, d].  Bias
+ *    pointers must be NULL when has_bias == 0 and non-NULL otherwise.
+ *  - Sizes: 0 <= T, T * top_k < 2^31; 1 <= n_experts <= 1024; 1 <= top_k <= min(32,
+ *    n_experts); 0 <= n_shared <= 16; d, inter, inter_shared >= 1.  For MOE_BF16, d, inter
+ *    and inter_shared must be multiples of 8 (16-byte rows for the tensor-memory-access
+ *    unit).  T == 0 is a valid no-op.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t / CUstream. */
+typedef struct CUstream_st* moe_stream_t;
+
+typedef enum {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = 1, /* null pointer, size out of range, bias pointer mismatch */
+    MOE_ERR_UNSUPPORTED = 2, /* valid layer, but outside what these kernels handle */
+    MOE_ERR_WORKSPACE = 3,   /* ws NULL or ws_bytes < moe_workspace_bytes(shape) */
+    MOE_ERR_CUDA = 4,        /* a CUDA runtime call or a kernel launch failed */
+    MOE_ERR_INTERNAL = 5     /* a kernel flagged an error (see moe_check_device_error) */
+} moe_status_t;
+
+typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype_t;
+
+typedef struct {
+    int32_t T;            /* tokens */
+    int32_t d;            /* hidden size */
+    int32_t n_experts;    /* N_m, routed experts */
+    int32_t inter;        /* intermediate size of a routed expert */
+    int32_t top_k;        /* N_r, routed experts per token */
+    int32_t n_shared;     /* K_s, shared experts (0 allowed) */
+    int32_t inter_shared; /* intermediate size of a shared expert (ignored when n_shared == 0) */
+    int32_t has_bias;     /* 1: every Linear has a bias (the page's Expert); 0: no biases */
+    int32_t dtype;        /* moe_dtype_t */
+} moe_shape_t;
+
+/* One stack of experts (routed: E = n_experts; shared: E = n_shared), nn.Linear layout. */
+typedef struct {
+    const void* w1; /* [E, I, d] */
+    const void* b1; /* [E, I] or NULL */
+    const void* w3; /* [E, I, d] */
+    const void* b3; /* [E, I] or NULL */
+    const void* w2; /* [E, d, I] */
+    const void* b2; /* [E, d] or NULL */
+} moe_ffn_weights_t;
+
+/* Bytes of workspace every entry point needs for this shape (0 if the shape is invalid). */
+size_t moe_workspace_bytes(const moe_shape_t* shape);
+
+/* Static description of a status code; never NULL. */
+const char* moe_status_string(moe_status_t status);
+
+/* Library version string, e.g. "moe_b200 0.1 sm_100a". */
+const char* moe_version(void);
+
+/* Synchronises `stream`, then reads and clears the error word the kernels keep in `ws`.
+ * Returns MOE_OK if no kernel flagged an error since the last check or moe_ws_init(),
+ * MOE_ERR_INTERNAL otherwise (*detail, when non-NULL, receives the raw error bits:
+ * 1 = expert index out of range, 2 = bounded wait timed out in a GEMM pipeline,
+ * 4 = token or slot index out of range).  The only call that synchronises. */
+moe_status_t moe_check_device_error(void* ws, size_t ws_bytes, moe_stream_t stream, uint32_t* detail);
+
+/* Clears the workspace's error word (asynchronously on `stream`).  Call once after
+ * allocating a workspace; moe_check_device_error() also clears it. */
+moe_status_t moe_ws_init(void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * Router: scores, softmax over all experts, top_k picks and gates ("《DeepSeekMoE》深度解读报告"
+ * §3.1, Eq. 3-5 in prose).
+ *   x:          [T, d]           dtype
+ *   centroids:  [n_experts, d]   dtype (the expert centroids e_i)
+ *   topk_idx:   [T, top_k] int32 out: expert indices, descending score, ties to lower index
+ *   topk_gate:  [T, top_k] fp32  out: softmax probability of each pick (not renormalised)
+ */
+moe_status_t moe_route(const moe_shape_t* shape, const void* x, const void* centroids,
+                       int32_t* topk_idx, float* topk_gate,
+                       void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * Per-expert token lists (the "top-k indices, then gather tokens per expert" step of the
+ * DeepSeek-V2 explainer, eliteato.com/news/32734, §3.1 and §3.3).  Slot s = t*top_k + j.
+ * Slots are grouped by expert; inside an expert they keep ascending slot order, so the
+ * result is deterministic.
+ *   topk_idx, topk_gate: [T, top_k] as produced by moe_route (any values in [0, n_experts))
+ *   counts:       [n_experts]     out: slots per expert
+ *   offsets:      [n_experts + 1] out: exclusive prefix sum of counts (offsets[E] = T*top_k)
+ *   sorted_token: [T*top_k]       out: token of the p-th grouped slot
+ *   sorted_gate:  [T*top_k] fp32  out: gate of the p-th grouped slot
+ *   slot_of:      [T*top_k]       out: slot_of[s] = grouped position p of slot s
+ * An index outside [0, n_experts) sets error bit 1 and the slot is dropped.
+ */
+moe_status_t moe_permute(const moe_shape_t* shape, const int32_t* topk_idx, const float* topk_gate,
+                         int32_t* counts, int32_t* offsets, int32_t* sorted_token,
+                         float* sorted_gate, int32_t* slot_of,
+                         void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * Routed experts on their token lists (the `Expert` module applied per expert):
+ *   y_sorted[p, :] = gate_p * FFN_e(x[sorted_token[p], :]) for every grouped position p of
+ *   expert e, i.e. offsets[e] <= p < offsets[e+1].  sorted_gate == NULL means gate 1.
+ *   x: [T, d]; offsets: [n_experts+1]; sorted_token, sorted_gate: [T*top_k];
+ *   routed: stacked weights of the n_experts routed experts; y_sorted: [T*top_k, d] out.
+ * offsets must be non-decreasing with offsets[0] = 0 and offsets[E] = T*top_k (as written by
+ * moe_permute); sorted_token entries must lie in [0, T) (bit 4 otherwise).
+ */
+moe_status_t moe_expert_ffn(const moe_shape_t* shape, const void* x, const int32_t* offsets,
+                            const int32_t* sorted_token, const float* sorted_gate,
+                            const moe_ffn_weights_t* routed, void* y_sorted,
+                            void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * Shared experts and the combine ("《DeepSeekMoE》深度解读报告" §2.3 and §3.1: the shared
+ * experts are summed first, for every token and without the router, then the gated routed
+ * outputs are added):
+ *   out[t, :] = sum_{k<K_s} FFN^shared_k(x[t]) + sum_{j<top_k} y_sorted[slot_of[t*top_k + j], :]
+ * The routed terms are added in ascending j, in fp32, and the sum is rounded once.
+ *   x: [T, d]; shared: stacked weights of the K_s shared experts (NULL iff n_shared == 0);
+ *   y_sorted: [T*top_k, d]; slot_of: [T*top_k]; out: [T, d] out.
+ */
+moe_status_t moe_combine(const moe_shape_t* shape, const void* x, const moe_ffn_weights_t* shared,
+                         const void* y_sorted, const int32_t* slot_of, void* out,
+                         void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * The whole layer: moe_route -> moe_permute -> moe_expert_ffn -> moe_combine, all on
+ * `stream`, every intermediate in `ws`.
+ *   x: [T, d]; centroids: [n_experts, d]; routed / shared weights as above (shared NULL iff
+ *   n_shared == 0); out: [T, d].
+ *   topk_idx_out [T, top_k], topk_gate_out [T, top_k] and counts_out [n_experts] are
+ *   optional (NULL = not returned).
+ */
+moe_status_t moe_layer_forward(const moe_shape_t* shape, const void* x, const void* centroids,
+                               const moe_ffn_weights_t* routed, const moe_ffn_weights_t* shared,
+                               void* out, int32_t* topk_idx_out, float* topk_gate_out,
+                               int32_t* counts_out, void* ws, size_t ws_bytes, moe_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

@@ -1,0 +1,107 @@
+"""The C-ABI library loads, exports every entry point include/moe.h declares, and rejects bad
+arguments synchronously, before touching the GPU (CPU only: no compute call runs here)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from fine_grained_mixture_route_b200 import moe
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    names = set()
+    for f in os.listdir(os.path.join(ROOT, "include")):
+        if f.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", f)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names |= set(re.findall(r"\b(moe_[a-z_0-9]+)\s*\(", src))
+    return names
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(moe.LIB_PATH):
+        from fine_grained_mixture_route_b200 import build
+        build.build()
+    return moe.lib_handle()
+
+
+def test_exports_every_declared_symbol(lib):
+    declared = _declared()
+    assert {"moe_route", "moe_permute", "moe_expert_ffn", "moe_combine", "moe_layer_forward",
+            "moe_workspace_bytes"} <= declared
+    for name in declared:
+        assert hasattr(lib, name), name
+    assert set(moe.EXPORTED) == declared
+
+
+def test_version_and_status_strings(lib):
+    assert b"sm_100a" in lib.moe_version()
+    for s in range(6):
+        assert lib.moe_status_string(s)
+    assert lib.moe_status_string(99) == b"MOE_ERR_UNKNOWN"
+
+
+def _shape(**kw):
+    base = dict(T=256, d=7168, n_experts=256, inter=2048, top_k=8, n_shared=1, inter_shared=2048, has_bias=1,
+                dtype=moe.MOE_BF16)
+    base.update(kw)
+    return moe.MoeShape(*[base[f] for f, _ in moe.MoeShape._fields_])
+
+
+def test_workspace_bytes(lib):
+    n = moe.workspace_bytes(_shape())
+    S, d, I = 256 * 8, 7168, 2048
+    # x_perm, h_r, Y (bf16) and the shared hidden states at least
+    assert n >= 2 * (S * d + S * I + S * d + 256 * 2048)
+    assert n < 2 * (S * d + S * I + S * d + 256 * 2048) + 4 * 1024 * 1024
+    assert moe.workspace_bytes(_shape(T=512)) > n
+    assert moe.workspace_bytes(_shape(T=0)) > 0
+    # fp32 layers keep no gathered copy of x
+    assert moe.workspace_bytes(_shape(dtype=moe.MOE_F32)) < 2 * n
+    for bad in (dict(top_k=0), dict(top_k=300), dict(n_experts=0), dict(d=0), dict(T=-1), dict(dtype=7),
+                dict(n_experts=2048, top_k=8), dict(d=7170), dict(inter=2047), dict(top_k=33, n_experts=64),
+                dict(has_bias=2), dict(n_shared=1, inter_shared=0)):
+        assert moe.workspace_bytes(_shape(**bad)) == 0, bad
+    assert moe.workspace_bytes(_shape(d=7170, dtype=moe.MOE_F32)) > 0
+
+
+def test_argument_errors_return_before_any_launch(lib):
+    sh = _shape()
+    fake = ctypes.c_void_p(1 << 40)            # never dereferenced: validation fails first
+    n = moe.workspace_bytes(sh)
+    w = moe.MoeWeights(fake.value, fake.value, fake.value, fake.value, fake.value, fake.value)
+    S = ctypes.byref
+    # null pointers
+    assert lib.moe_route(S(sh), None, fake, fake, fake, fake, n, None) == moe.MOE_ERR_INVALID_ARG
+    assert lib.moe_layer_forward(S(sh), fake, fake, None, S(w), fake, None, None, None, fake, n, None) == \
+        moe.MOE_ERR_INVALID_ARG
+    # bias pointers must match has_bias
+    wnb = moe.MoeWeights(fake.value, None, fake.value, None, fake.value, None)
+    assert lib.moe_expert_ffn(S(sh), fake, fake, fake, fake, S(wnb), fake, fake, n, None) == moe.MOE_ERR_INVALID_ARG
+    sh_nb = _shape(has_bias=0)
+    assert lib.moe_expert_ffn(S(sh_nb), fake, fake, fake, fake, S(w), fake, fake, n, None) == moe.MOE_ERR_INVALID_ARG
+    # shared weights given for a layer without shared experts, and missing when needed
+    sh0 = _shape(n_shared=0)
+    assert lib.moe_combine(S(sh0), fake, S(w), fake, fake, fake, fake, n, None) == moe.MOE_ERR_INVALID_ARG
+    assert lib.moe_combine(S(sh), fake, None, fake, fake, fake, fake, n, None) == moe.MOE_ERR_INVALID_ARG
+    # workspace too small, missing or misaligned
+    assert lib.moe_route(S(sh), fake, fake, fake, fake, fake, n - 1, None) == moe.MOE_ERR_WORKSPACE
+    assert lib.moe_route(S(sh), fake, fake, fake, fake, None, n, None) == moe.MOE_ERR_WORKSPACE
+    assert lib.moe_route(S(sh), fake, fake, fake, fake, ctypes.c_void_p((1 << 40) + 8), n, None) == \
+        moe.MOE_ERR_WORKSPACE
+    # unsupported sizes
+    assert lib.moe_route(S(_shape(d=7172)), fake, fake, fake, fake, fake, n, None) == moe.MOE_ERR_UNSUPPORTED
+    assert lib.moe_route(S(_shape(top_k=40, n_experts=64)), fake, fake, fake, fake, fake, n, None) == \
+        moe.MOE_ERR_UNSUPPORTED
+    assert lib.moe_route(None, fake, fake, fake, fake, fake, n, None) == moe.MOE_ERR_INVALID_ARG
+    # T == 0 is a valid no-op (returns before any CUDA call)
+    sh_e = _shape(T=0)
+    ne = moe.workspace_bytes(sh_e)
+    assert lib.moe_route(S(sh_e), fake, fake, fake, fake, fake, ne, None) == moe.MOE_OK
+    assert lib.moe_layer_forward(S(sh_e), fake, fake, S(w), S(w), fake, None, None, None, fake, ne, None) == moe.MOE_OK
+    assert lib.moe_ws_init(None, 0, None) == moe.MOE_ERR_WORKSPACE
+    assert lib.moe_check_device_error(None, 0, None, None) == moe.MOE_ERR_WORKSPACE

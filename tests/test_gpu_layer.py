@@ -1,0 +1,166 @@
+"""Parity of the sm_100a layer with the fp64 oracle, through the C ABI (needs a B200).
+
+Every configuration runs the fused moe_layer_forward and the four step entry points
+(moe_route -> moe_permute -> moe_expert_ffn -> moe_combine) and checks:
+  * expert picks: exact except at counted near-ties (fp64 logit gap < 1e-5);
+  * gates: fp32, 1e-4 relative to the softmax read at the picks;
+  * grouping: bit-exact with the oracle's stable grouping of the same picks;
+  * routed outputs Y (gate * expert output per slot) and the layer output: normwise relative
+    error within 2e-2 (bf16) / 1e-4 (fp32);
+  * the step chain reproduces the fused call bit for bit, and two calls agree bit for bit.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle.moe_oracle as O
+from fine_grained_mixture_route_b200 import moe
+from fine_grained_mixture_route_b200 import workloads as W
+from tests.parity import (TOL, check_permute, check_routing, expert_source, f64, normwise)
+
+pytestmark = pytest.mark.gpu
+
+_CACHE = {}
+
+
+def _layer(cfg, seed=0):
+    key = (cfg, seed)
+    if key not in _CACHE:
+        _CACHE.clear()
+        torch.cuda.empty_cache()
+        _CACHE[key] = W.make_layer(cfg, "cuda", seed)
+    return _CACHE[key]
+
+
+def _run(cfg, L, ws=None):
+    x, C, R, Sh = L["x"], L["centroids"], L["routed"], L["shared"]
+    shape = moe.shape_of(x, C, R, cfg.top_k, Sh)
+    ws = moe.new_workspace(shape) if ws is None else ws
+    T, k = x.shape[0], cfg.top_k
+    idx = torch.empty((T, k), dtype=torch.int32, device="cuda")
+    gate = torch.empty((T, k), dtype=torch.float32, device="cuda")
+    counts = torch.empty(cfg.n_experts, dtype=torch.int32, device="cuda")
+    out = moe.layer_forward(shape, x, C, R, Sh, ws, idx=idx, gate=gate, counts=counts)
+    moe.check_device_error(ws)
+    return shape, ws, out, idx, gate, counts
+
+
+def _steps(shape, L, ws, idx_ref=None):
+    x, C, R, Sh = L["x"], L["centroids"], L["routed"], L["shared"]
+    idx, gate = moe.route(shape, x, C, ws)
+    perm = moe.permute(shape, idx, gate, ws)
+    y = moe.expert_ffn(shape, x, perm["offsets"], perm["sorted_token"], perm["sorted_gate"], R, ws)
+    out = moe.combine(shape, x, Sh, y, perm["slot_of"], ws)
+    moe.check_device_error(ws)
+    return idx, gate, perm, y, out
+
+
+def _full_check(cfg, L, tokens=None):
+    shape, ws, out, idx, gate, counts = _run(cfg, L)
+    x64, c64 = f64(L["x"]), f64(L["centroids"])
+    idx_np, gate_np = idx.cpu().numpy().astype(np.int64), gate.cpu().numpy()
+    near, n_set, n_ord = check_routing(idx_np, gate_np, x64, c64, cfg.top_k)
+    assert np.array_equal(counts.cpu().numpy(), np.bincount(idx_np.reshape(-1), minlength=cfg.n_experts))
+
+    # step entry points: same picks, bit-exact grouping, bit-identical output
+    idx2, gate2, perm, y, out2 = _steps(shape, L, ws)
+    assert torch.equal(idx2, idx) and torch.equal(gate2, gate)
+    assert torch.equal(out2, out), "step chain differs from the fused call"
+    perm_np = {k: v.cpu().numpy() for k, v in perm.items()}
+    p = check_permute(idx_np, gate_np, perm_np, cfg.n_experts)
+
+    # oracle on all tokens, or on a sample (per-token independence of the layer)
+    sel = np.arange(cfg.T) if tokens is None else np.asarray(tokens)
+    Sh = L["shared"]
+    ref = O.layer(x64[sel], c64, expert_source(L["routed"]), cfg.n_experts, cfg.top_k,
+                  expert_source(Sh) if Sh is not None else None, cfg.n_shared, idx_override=idx_np[sel])
+    tol = TOL[cfg.dtype]
+    e_out = normwise(f64(out)[sel], ref["out"])
+    assert e_out <= tol, f"out error {e_out:.3e} > {tol}"
+    # routed rows (gate * expert output) on their own: the shared term cannot hide them
+    k = cfg.top_k
+    slots = (sel[:, None] * k + np.arange(k)[None, :]).reshape(-1)
+    y_np = f64(y)[p["slot_of"][slots]]
+    e_y = normwise(y_np, ref["Y"])
+    assert e_y <= tol, f"routed Y error {e_y:.3e} > {tol}"
+    e_routed = normwise(y_np.reshape(len(sel), k, -1).sum(1), ref["routed_sum"])
+    assert e_routed <= tol, f"routed sum error {e_routed:.3e}"
+
+    # determinism
+    out3 = moe.layer_forward(shape, L["x"], L["centroids"], L["routed"], Sh, ws)
+    assert torch.equal(out3, out)
+    return {"near_tie_tokens": int(near.sum()), "set_ties": n_set, "order_ties": n_ord, "err_out": e_out, "err_y": e_y}
+
+
+@pytest.mark.parametrize("name", ["tiny", "small", "mid", "decode"])
+def test_config_full(name):
+    cfg = W.CONFIGS[name]
+    stats = _full_check(cfg, _layer(cfg))
+    print(name, stats)
+
+
+def test_prefill_sampled():
+    cfg = W.CONFIGS["prefill"]
+    L = _layer(cfg)
+    rng = np.random.default_rng(0)
+    tokens = np.unique(np.concatenate([[0, 1, 127, 128, cfg.T - 1], rng.choice(cfg.T, 91, replace=False)]))
+    stats = _full_check(cfg, L, tokens)
+    print("prefill", stats)
+
+
+EDGE = [
+    # (name, overrides of a base config)
+    ("bf16_T1", "small", dict(T=1)),
+    ("bf16_ragged_T", "small", dict(T=77)),
+    ("bf16_all_experts", "small", dict(T=200, n_experts=16, top_k=16, inter=64, inter_shared=64)),
+    ("bf16_no_shared", "small", dict(T=300, n_shared=0)),
+    ("bf16_two_shared_uneven", "mid", dict(T=260, d=512, inter=200, n_shared=2, inter_shared=136)),
+    ("bf16_odd_dims", "small", dict(T=131, d=136, inter=40, inter_shared=24, n_experts=48, top_k=5)),
+    ("bf16_simt_router_E20", "small", dict(T=150, n_experts=20, top_k=3, d=256, inter=64, inter_shared=64)),
+    ("bf16_simt_router_E512", "decode", dict(T=64, n_experts=512, top_k=12, d=512, inter=128, inter_shared=128)),
+    ("bf16_zipf_empty_experts", "prefill", dict(T=1000, d=512, inter=128, inter_shared=128, n_experts=64)),
+    ("bf16_topk32", "small", dict(T=96, n_experts=64, top_k=32, d=256, inter=64, inter_shared=64)),
+    ("f32_ragged", "tiny", dict(T=77, d=200, inter=40, inter_shared=24)),
+    ("f32_no_shared_no_bias", "tiny", dict(T=65, n_shared=0, has_bias=False)),
+    ("f32_T1", "tiny", dict(T=1)),
+]
+
+
+@pytest.mark.parametrize("case", EDGE, ids=[c[0] for c in EDGE])
+def test_edge_cases(case):
+    _, base, kw = case
+    cfg = W.scaled(W.CONFIGS[base], **kw)
+    stats = _full_check(cfg, W.make_layer(cfg, "cuda", seed=3))
+    print(case[0], stats)
+
+
+def test_all_tokens_one_expert_set():
+    """Equal centroids: every score ties, every token picks experts 0..k-1 (lowest indices),
+    so the first k experts get all T tokens and the rest none."""
+    cfg = W.scaled(W.CONFIGS["small"], T=300, d=256, n_experts=32, top_k=4, inter=64, inter_shared=64)
+    L = W.make_layer(cfg, "cuda", seed=5)
+    L["centroids"] = L["centroids"][:1].repeat(cfg.n_experts, 1).contiguous()
+    shape, ws, out, idx, gate, counts = _run(cfg, L)
+    assert torch.equal(idx.cpu(), torch.arange(4, dtype=torch.int32).repeat(300, 1))
+    c = counts.cpu().numpy()
+    assert (c[:4] == 300).all() and (c[4:] == 0).all()
+    assert torch.allclose(gate, torch.full_like(gate, 1.0 / 32), rtol=1e-6, atol=0)
+    ref = O.layer(f64(L["x"]), f64(L["centroids"]), expert_source(L["routed"]), 32, 4,
+                  expert_source(L["shared"]), 1)
+    assert normwise(f64(out), ref["out"]) <= TOL[cfg.dtype]
+
+
+def test_bad_expert_index_is_flagged():
+    """An out-of-range expert index handed to moe_permute is dropped by the kernel's own
+    range check and reported through the workspace error word."""
+    cfg = W.scaled(W.CONFIGS["small"], T=64, d=256, n_experts=16, top_k=2, inter=64, inter_shared=64)
+    shape = moe.make_shape(64, 256, 16, 64, 2, 1, 64, True, torch.bfloat16)
+    ws = moe.new_workspace(shape)
+    idx = torch.randint(0, 16, (64, 2), dtype=torch.int32, device="cuda")
+    idx[5, 1] = 16
+    gate = torch.rand((64, 2), device="cuda")
+    moe.permute(shape, idx, gate, ws)
+    with pytest.raises(moe.MoeError) as ei:
+        moe.check_device_error(ws)
+    assert ei.value.status == moe.MOE_ERR_INTERNAL and ei.value.detail & 1
+    moe.check_device_error(ws)          # cleared by the previous check
