@@ -1,0 +1,446 @@
+#!/usr/bin/env python
+"""Benchmark of the B200 DeepSeekMoE layer forward.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload prefill|decode|mid|small|tiny]
+                    [--impl ours|reference]
+
+One step = one moe_layer_forward over one batch of synthetic tokens (router, grouping, row
+gather, GEMM1+SwiGLU, GEMM2+gate, shared GEMM2+combine), inputs resident in HBM.  The
+default workload is the prefill-shaped layer: T=16384 tokens, d=7168, 256 routed experts of
+inter 2048, top-8, one shared expert, biases on, Zipf(1.1)-skewed routing.  The weights
+(22.6 GB) and the activations are far larger than the 126 MB L2, so no flush is needed
+between steps.
+
+Multi-GPU runs are replicas: every rank holds the same weights and processes its own batch
+(the layer is independent per token; there is no exchange), so the per-GPU work is fixed
+(weak scaling) and value = tokens of all ranks / the slowest rank's time.
+
+--impl reference times the fp64 CPU oracle (the only reference that exists for this layer)
+on bounded samples of the same workload, on rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from fine_grained_mixture_route_b200 import workloads as W  # noqa: E402
+
+METRIC = "MoE-layer tokens/s, TFLOP/s (prefill) and HBM GB/s (decode) on 1 B200"
+UNIT = "tokens/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ----------------------------------------------------------------------------- helpers
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def dist_env():
+    return int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("LOCAL_RANK", "0"))
+
+
+def init_dist(world: int, backend: str):
+    if world > 1 and not torch.distributed.is_initialized():
+        torch.distributed.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
+
+
+def reduce_max(v: float, device) -> float:
+    """Max of a scalar over all ranks (identity when not distributed)."""
+    if not (torch.distributed.is_available() and torch.distributed.is_initialized()):
+        return v
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier():
+    if torch.distributed.is_available() and torch.distributed.is_initialized():
+        torch.distributed.barrier()
+
+
+def aggregate_throughput(tokens_per_rank: int, n_ranks: int, max_ms_per_step: float) -> float:
+    """Whole-job tokens/s: every rank's tokens over the slowest rank's step time."""
+    return tokens_per_rank * n_ranks / (max_ms_per_step / 1e3)
+
+
+def stage_work(cfg: W.LayerConfig, touched: int):
+    """Algorithmic FLOPs and HBM bytes of each stage of one layer call.
+
+    Bytes count each operand once at its storage size: weights of the experts that received
+    at least one token (`touched`), activations read and written by the stage, routing
+    metadata.  FLOPs count 2 per multiply-add of the contractions only.
+    """
+    T, d, E, I, k, Ks, Is = cfg.T, cfg.d, cfg.n_experts, cfg.inter, cfg.top_k, cfg.n_shared, cfg.inter_shared
+    b = cfg.elem_bytes()
+    S = T * k
+    bias = 1 if cfg.has_bias else 0
+    w = {
+        "router": (2.0 * T * d * E, (T * d + E * d) * b + S * 8),
+        "permute": (0.0, S * 8 + S * 16),
+        "plan": (0.0, (E + 1) * 4),
+        "gather": (0.0, 2 * S * d * b + S * 4),
+        "gemm1_swiglu": (2.0 * S * d * 2 * I + 2.0 * Ks * T * d * 2 * Is,
+                         touched * (2 * I * d + 2 * I * bias) * b + Ks * (2 * Is * d + 2 * Is * bias) * b
+                         + S * d * b + (T * d * b if Ks else 0) + (S * I + Ks * T * Is) * b),
+        "gemm2_gate": (2.0 * S * I * d, touched * (d * I + d * bias) * b + S * I * b + S * d * b + S * 8),
+        "combine": (2.0 * Ks * T * Is * d, Ks * (d * Is + d * bias) * b + Ks * T * Is * b + S * d * b + T * d * b
+                    + S * 4),
+    }
+    return w
+
+
+def layer_bytes(cfg: W.LayerConfig, touched: int) -> float:
+    """Algorithmic bytes of the whole layer: weights of touched experts, shared experts,
+    centroids, x in and out once (intermediates excluded: the method need not keep them)."""
+    b = cfg.elem_bytes()
+    bias = 1 if cfg.has_bias else 0
+    return (touched * (3 * cfg.d * cfg.inter + (2 * cfg.inter + cfg.d) * bias) * b
+            + cfg.n_shared * (3 * cfg.d * cfg.inter_shared + (2 * cfg.inter_shared + cfg.d) * bias) * b
+            + cfg.n_experts * cfg.d * b + 2 * cfg.T * cfg.d * b)
+
+
+def src_hash(path: str) -> str:
+    return hashlib.sha256(open(path, "rb").read()).hexdigest()[:16]
+
+
+def ncu_traffic(workload: str, stage: str):
+    """Per-launch DRAM bytes of a kernel from the committed ncu summary, if the kernel's
+    source has not changed since the counters were taken; else None."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p))
+    ent = d.get(workload, {}).get(stage)
+    if not ent:
+        return None
+    src = os.path.join(ROOT, "fine_grained_mixture_route_b200", "csrc", ent["source"])
+    if not os.path.exists(src) or src_hash(src) != ent["source_sha256_16"]:
+        return None
+    return float(ent["dram_bytes_per_launch"])
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling in the background during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu: str):
+        self.proc = None
+        self.gpu = gpu
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", gpu, f"--query-gpu={self.Q}", "--format=csv,noheader",
+                                          "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1].split()[0]))
+                mx.append(float(f[2].split()[0]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return None
+        smax = max(mx)
+        loaded = [s for s in sm if s >= 0.5 * smax] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def visible_gpu_id(local_rank: int) -> str:
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        ids = [v.strip() for v in vis.split(",") if v.strip()]
+        if local_rank < len(ids):
+            return ids[local_rank]
+    return str(local_rank)
+
+
+# ----------------------------------------------------------------------------- oracle legs
+class HostExperts:
+    """Expert weights copied to host memory on first use; the oracle converts each expert to
+    float64 itself (its own input handling, inside its timing)."""
+
+    def __init__(self, stack):
+        self.stack = stack
+        self.cache = {}
+
+    def prefetch(self, experts):
+        for e in experts:
+            self._host(int(e))
+
+    def _host(self, e):
+        if e not in self.cache:
+            self.cache[e] = {k: (None if v is None else v[e].detach().to("cpu")) for k, v in self.stack.items()}
+        return self.cache[e]
+
+    def __call__(self, e):
+        h = self._host(int(e))
+        return {k: (None if v is None else v.float().numpy().astype(np.float64)) for k, v in h.items()}
+
+
+def oracle_sample(O, L, cfg, host_routed, host_shared, tokens):
+    x = L["x"][tokens].float().cpu().numpy().astype(np.float64)
+    c = L["centroids"].float().cpu().numpy().astype(np.float64)
+    t0 = time.perf_counter()
+    O.layer(x, c, host_routed, cfg.n_experts, cfg.top_k, host_shared, cfg.n_shared)
+    return time.perf_counter() - t0
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        info = [i for i in threadpool_info() if i.get("user_api") == "blas"]
+        if info:
+            return int(info[0]["num_threads"])
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def cpu_baseline(cfg, L, idx_gpu, n_tokens=16):
+    """The oracle, as it stands, on the first n_tokens tokens of this step's batch."""
+    import oracle.moe_oracle as O
+    tokens = np.arange(min(n_tokens, cfg.T))
+    hr = HostExperts(L["routed"])
+    hs = HostExperts(L["shared"]) if L["shared"] is not None else None
+    hr.prefetch(np.unique(idx_gpu[tokens]))
+    if hs is not None:
+        hs.prefetch(range(cfg.n_shared))
+    dt = oracle_sample(O, L, cfg, hr, hs, tokens)
+    return {"value": len(tokens) / dt, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+            "sample": f"fp64 NumPy oracle on the first {len(tokens)} tokens of the {cfg.name} batch "
+                      f"(all experts they route to; weights staged in host memory as bf16, converted by the oracle)",
+            "seconds": dt}
+
+
+def run_reference(args, cfg, rank, world):
+    """--impl reference: the fp64 oracle on bounded samples of the same workload."""
+    if rank != 0:
+        return
+    import oracle.moe_oracle as O
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    L = W.make_layer(cfg, dev, seed=0)
+    hr = HostExperts(L["routed"])
+    hs = HostExperts(L["shared"]) if L["shared"] is not None else None
+    budget_s = 150.0
+    n = min(8, cfg.T)
+    t_first = oracle_sample(O, L, cfg, hr, hs, np.arange(n))           # sizing run (also warms the cache)
+    per_tok = t_first / n
+    n = int(max(1, min(64, cfg.T, budget_s / max(1, args.steps + args.warmup) / max(per_tok, 1e-6))))
+    pos = 0
+    times = []
+    for i in range(args.warmup + args.steps):
+        toks = (np.arange(n) + pos) % cfg.T
+        pos += n
+        dt = oracle_sample(O, L, cfg, hr, hs, toks)
+        if i >= args.warmup:
+            times.append(dt)
+    total = sum(times)
+    value = n * len(times) / total
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "impl": "reference", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / len(times),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": cfg.name, "tokens_per_step": n, "T": cfg.T, "d": cfg.d,
+                       "n_experts": cfg.n_experts, "inter": cfg.inter, "top_k": cfg.top_k,
+                       "n_shared": cfg.n_shared, "parallelism": "replicas" if world > 1 else "single"},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                             "sample": f"{n} consecutive tokens of the {cfg.name} batch per step"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------- our arm
+def run_ours(args, cfg, rank, world, local_rank):
+    from fine_grained_mixture_route_b200 import moe
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+    # same weights on every replica, a different token batch per rank
+    L = W.make_layer(cfg, dev, seed=0)
+    if rank > 0:
+        L["x"] = W.make_x(cfg, dev, seed=1000 + rank)
+    x, C, R, Sh = L["x"], L["centroids"], L["routed"], L["shared"]
+    shape = moe.shape_of(x, C, R, cfg.top_k, Sh)
+    ws = moe.new_workspace(shape, dev)
+    out = torch.empty_like(x)
+    idx = torch.empty((cfg.T, cfg.top_k), dtype=torch.int32, device=dev)
+    gate = torch.empty((cfg.T, cfg.top_k), dtype=torch.float32, device=dev)
+    counts = torch.empty(cfg.n_experts, dtype=torch.int32, device=dev)
+
+    for _ in range(args.warmup):
+        moe.layer_forward(shape, x, C, R, Sh, ws, out=out, idx=idx, gate=gate, counts=counts)
+    moe.check_device_error(ws)
+    touched = int((counts > 0).sum().item())
+    work = stage_work(cfg, touched)
+
+    # ---- device-timed region: K steps, per-stage events on the launching stream
+    evs = [moe.stage_events(stream) for _ in range(args.steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(visible_gpu_id(local_rank))
+    start.record(stream)
+    for i in range(args.steps):
+        moe.layer_forward_timed(shape, x, C, R, Sh, ws, evs[i], out=out, idx=idx, gate=gate, counts=counts)
+    stop.record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    barrier()
+    moe.check_device_error(ws)
+    ms_local = start.elapsed_time(stop) / args.steps
+    ms = reduce_max(ms_local, dev)
+    stage_ms = {}
+    for j, name in enumerate(moe.STAGE_NAMES):
+        stage_ms[name] = statistics.mean(e[j].elapsed_time(e[j + 1]) for e in evs)
+    launches_per_step = 9 if cfg.dtype == torch.bfloat16 else 8
+
+    # ---- end to end through the public API: pinned host input, H2D, layer, D2H
+    e2e = None
+    if not args.no_e2e:
+        xh = x.detach().to("cpu").pin_memory()
+        oh = torch.empty(x.shape, dtype=x.dtype).pin_memory()
+        xd = torch.empty_like(x)
+        for _ in range(2):
+            xd.copy_(xh, non_blocking=True)
+            moe.layer_forward(shape, xd, C, R, Sh, ws, out=out)
+            oh.copy_(out, non_blocking=True)
+        torch.cuda.synchronize()
+        barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.steps):
+            xd.copy_(xh, non_blocking=True)
+            moe.layer_forward(shape, xd, C, R, Sh, ws, out=out)
+            oh.copy_(out, non_blocking=True)
+        b.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        e2e_ms = reduce_max(a.elapsed_time(b) / args.steps, dev)
+        e2e = {"value": aggregate_throughput(cfg.T, world, e2e_ms), "unit": UNIT,
+               "h2d_bytes_per_step": x.numel() * x.element_size(),
+               "d2h_bytes_per_step": out.numel() * out.element_size(), "ms_per_step": e2e_ms}
+        moe.check_device_error(ws)
+
+    peaks, peak_src = load_peaks()
+    # dominant stage and its roofline
+    dom = max(stage_ms, key=stage_ms.get)
+    flops, nbytes = work[dom]
+    ridge = peaks["bf16_tflops_sustained"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    if cfg.dtype == torch.float32:
+        bound = "hbm" if nbytes > 0 and flops / nbytes < 10 else "alu"
+    else:
+        bound = "tensor" if nbytes == 0 or flops / nbytes > ridge else "hbm"
+    t = stage_ms[dom] / 1e3
+    if bound == "tensor":
+        achieved, peak, unit = flops / t / 1e12, peaks["bf16_tflops_sustained"], "TFLOP/s"
+    elif bound == "hbm":
+        achieved, peak, unit = nbytes / t / 1e9, peaks["hbm_gbs"], "GB/s"
+    else:
+        # fp32 CUDA-core FMA peak: 148 SMs x 128 lanes x 2 FLOP x max SM clock
+        achieved, peak, unit = flops / t / 1e12, 148 * 128 * 2 * 1.965e9 / 1e12, "TFLOP/s"
+    roofline = {"bound": bound, "kernel": dom, "achieved": achieved, "peak": peak, "unit": unit,
+                "frac": achieved / peak, "peak_source": f"{peak_src} ({'bf16 sustained' if bound == 'tensor' else 'HBM copy' if bound == 'hbm' else 'fp32 FMA nominal'})",
+                "traffic": ncu_traffic(cfg.name, dom),
+                "algorithmic_per_launch": flops if bound != "hbm" else nbytes}
+    if bound == "tensor":
+        roofline["frac_of_burst"] = achieved / peaks["bf16_tflops"]
+
+    step_s = ms / 1e3
+    total_flops = cfg.flops()
+    lbytes = layer_bytes(cfg, touched)
+    value = aggregate_throughput(cfg.T, world, ms)
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16" if cfg.dtype == torch.bfloat16 else "f32", "data": "synthetic",
+        "config": {"workload": cfg.name, "T": cfg.T, "d": cfg.d, "n_experts": cfg.n_experts, "inter": cfg.inter,
+                   "top_k": cfg.top_k, "n_shared": cfg.n_shared, "inter_shared": cfg.inter_shared,
+                   "bias": cfg.has_bias, "routing": cfg.centroid_init,
+                   "parallelism": f"replicas{world}" if world > 1 else "single",
+                   "l2": "inputs larger than L2 (weights and activations), no flush",
+                   "tokens_per_gpu": cfg.T},
+        "tflops": total_flops / step_s / 1e12 * world,
+        "hbm_gbs_algorithmic": lbytes / step_s / 1e9,
+        "experts_touched": touched,
+        "stage_ms": stage_ms,
+        "roofline": roofline,
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks,
+        "e2e": e2e,
+    }
+    del evs
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(cfg, L, idx.cpu().numpy())
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="prefill", choices=sorted(W.CONFIGS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    rank, world, local_rank = dist_env()
+    if world != args.gpus and world > 1:
+        ap.error(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    cfg = W.CONFIGS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, cfg, rank, world)
+        return
+    init_dist(world, "nccl")
+    try:
+        run_ours(args, cfg, rank, world, local_rank)
+    finally:
+        if torch.distributed.is_available() and torch.distributed.is_initialized():
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

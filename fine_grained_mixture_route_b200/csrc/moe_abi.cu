@@ -263,10 +263,17 @@ MOE_EXPORT moe_status_t moe_combine(const moe_shape_t* shape, const void* x, con
     return MOE_OK;
 }
 
-MOE_EXPORT moe_status_t moe_layer_forward(const moe_shape_t* shape, const void* x, const void* centroids,
-                                          const moe_ffn_weights_t* routed, const moe_ffn_weights_t* shared, void* out,
-                                          int32_t* topk_idx_out, float* topk_gate_out, int32_t* counts_out, void* ws,
-                                          size_t ws_bytes, moe_stream_t stream) {
+}  // extern "C"
+
+namespace moe {
+namespace {
+
+// The whole layer; when `ev` is non-NULL, ev[i] is recorded on the stream before stage i
+// and ev[MOE_NUM_STAGES] after the last one.
+moe_status_t layer_forward_impl(const moe_shape_t* shape, const void* x, const void* centroids,
+                                const moe_ffn_weights_t* routed, const moe_ffn_weights_t* shared, void* out,
+                                int32_t* topk_idx_out, float* topk_gate_out, int32_t* counts_out, void* ws,
+                                size_t ws_bytes, cudaStream_t st, cudaEvent_t const* ev) {
     Dims D;
     MOE_TRY(to_dims(shape, &D));
     if (!x || !centroids || !out) return MOE_ERR_INVALID_ARG;
@@ -278,7 +285,6 @@ MOE_EXPORT moe_status_t moe_layer_forward(const moe_shape_t* shape, const void* 
     MOE_TRY(check_device());
     cudaGetLastError();
     const Layout L = layout(D);
-    cudaStream_t st = (cudaStream_t)stream;
     uint32_t* err = at<uint32_t>(ws, L.err);
     int32_t* idx = topk_idx_out ? topk_idx_out : at<int32_t>(ws, L.idx);
     float* gate = topk_gate_out ? topk_gate_out : at<float>(ws, L.gate);
@@ -293,24 +299,61 @@ MOE_EXPORT moe_status_t moe_layer_forward(const moe_shape_t* shape, const void* 
     int32_t* ts1 = at<int32_t>(ws, L.ts1);
     int32_t* ts2 = at<int32_t>(ws, L.ts2);
     const FfnWeights R = to_ffn(routed), Sh = to_ffn(shared);
+    auto mark = [&](int i) -> bool { return !ev || cudaEventRecord(ev[i], st) == cudaSuccess; };
 
+    if (!mark(0)) return MOE_ERR_CUDA;
     MOE_TRY(do_route(D, x, centroids, idx, gate, err, st));
+    if (!mark(1)) return MOE_ERR_CUDA;
     MOE_CUDA(launch_permute(D, idx, gate, counts, offsets, stok, sgate, slot_of, at<int32_t>(ws, L.hist), err, st));
+    if (!mark(2)) return MOE_ERR_CUDA;
     MOE_CUDA(launch_plan(D, offsets, ts1, ts2, err, st));
+    if (!mark(3)) return MOE_ERR_CUDA;
     if (D.bf16) {
         void* xp = at<void>(ws, L.xperm);
         MOE_CUDA(launch_gather(D, x, stok, xp, err, st));
+        if (!mark(4)) return MOE_ERR_CUDA;
         MOE_CUDA(launch_tc_gemm1(D, x, xp, offsets, ts1, R, Sh, hr, hs, 0, D.E + D.Ks, err, st));
+        if (!mark(5)) return MOE_ERR_CUDA;
         MOE_CUDA(launch_tc_gemm2_routed(D, offsets, ts2, sgate, R, hr, y, err, st));
+        if (!mark(6)) return MOE_ERR_CUDA;
         if (D.Ks > 0) MOE_CUDA(launch_tc_gemm2_shared(D, Sh, hs, y, slot_of, out, err, st));
         else MOE_CUDA(launch_combine(D, y, slot_of, out, err, st));
     } else {
+        if (!mark(4)) return MOE_ERR_CUDA;
         MOE_CUDA(launch_simt_gemm1(D, x, offsets, stok, R, Sh, hr, hs, 0, D.E + D.Ks, err, st));
+        if (!mark(5)) return MOE_ERR_CUDA;
         MOE_CUDA(launch_simt_gemm2_routed(D, offsets, sgate, R, hr, y, err, st));
+        if (!mark(6)) return MOE_ERR_CUDA;
         if (D.Ks > 0) MOE_CUDA(launch_simt_gemm2_shared(D, Sh, hs, y, slot_of, out, err, st));
         else MOE_CUDA(launch_combine(D, y, slot_of, out, err, st));
     }
+    if (!mark(7)) return MOE_ERR_CUDA;
     return MOE_OK;
+}
+
+}  // namespace
+}  // namespace moe
+
+extern "C" {
+
+MOE_EXPORT moe_status_t moe_layer_forward(const moe_shape_t* shape, const void* x, const void* centroids,
+                                          const moe_ffn_weights_t* routed, const moe_ffn_weights_t* shared, void* out,
+                                          int32_t* topk_idx_out, float* topk_gate_out, int32_t* counts_out, void* ws,
+                                          size_t ws_bytes, moe_stream_t stream) {
+    return layer_forward_impl(shape, x, centroids, routed, shared, out, topk_idx_out, topk_gate_out, counts_out, ws,
+                              ws_bytes, (cudaStream_t)stream, nullptr);
+}
+
+MOE_EXPORT moe_status_t moe_layer_forward_timed(const moe_shape_t* shape, const void* x, const void* centroids,
+                                                const moe_ffn_weights_t* routed, const moe_ffn_weights_t* shared,
+                                                void* out, int32_t* topk_idx_out, float* topk_gate_out,
+                                                int32_t* counts_out, void* ws, size_t ws_bytes, moe_stream_t stream,
+                                                void* const* stage_events, int32_t n_events) {
+    if (!stage_events || n_events != MOE_NUM_STAGES + 1) return MOE_ERR_INVALID_ARG;
+    for (int i = 0; i < n_events; ++i)
+        if (!stage_events[i]) return MOE_ERR_INVALID_ARG;
+    return layer_forward_impl(shape, x, centroids, routed, shared, out, topk_idx_out, topk_gate_out, counts_out, ws,
+                              ws_bytes, (cudaStream_t)stream, reinterpret_cast<cudaEvent_t const*>(stage_events));
 }
 
 }  // extern "C"

@@ -18,7 +18,10 @@ MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_CUD
 MOE_F32, MOE_BF16 = 0, 1
 
 EXPORTED = ("moe_workspace_bytes", "moe_status_string", "moe_version", "moe_check_device_error", "moe_ws_init",
-            "moe_route", "moe_permute", "moe_expert_ffn", "moe_combine", "moe_layer_forward")
+            "moe_route", "moe_permute", "moe_expert_ffn", "moe_combine", "moe_layer_forward",
+            "moe_layer_forward_timed")
+NUM_STAGES = 7
+STAGE_NAMES = ("router", "permute", "plan", "gather", "gemm1_swiglu", "gemm2_gate", "combine")
 
 
 class MoeShape(ctypes.Structure):
@@ -63,8 +66,10 @@ def _lib():
         lib.moe_expert_ffn.argtypes = [sh, vp, i32p, i32p, f32p, wp, vp, vp, sz, vp]
         lib.moe_combine.argtypes = [sh, vp, wp, vp, i32p, vp, vp, sz, vp]
         lib.moe_layer_forward.argtypes = [sh, vp, vp, wp, wp, vp, i32p, f32p, i32p, vp, sz, vp]
+        lib.moe_layer_forward_timed.argtypes = [sh, vp, vp, wp, wp, vp, i32p, f32p, i32p, vp, sz, vp,
+                                                ctypes.POINTER(ctypes.c_void_p), ctypes.c_int32]
         for n in ("moe_check_device_error", "moe_ws_init", "moe_route", "moe_permute", "moe_expert_ffn",
-                  "moe_combine", "moe_layer_forward"):
+                  "moe_combine", "moe_layer_forward", "moe_layer_forward_timed"):
             getattr(lib, n).restype = ctypes.c_int
         _LIB = lib
     return _LIB
@@ -185,6 +190,29 @@ def layer_forward(shape: MoeShape, x, centroids, routed: Dict, shared: Optional[
     _check(_lib().moe_layer_forward(ctypes.byref(shape), _ptr(x), _ptr(centroids), ctypes.byref(rw),
                                     None if sw is None else ctypes.byref(sw), _ptr(out), _ptr(idx), _ptr(gate),
                                     _ptr(counts), _ptr(ws), ws.numel(), _stream(stream)), "moe_layer_forward")
+    return out
+
+
+def stage_events(stream=None):
+    """NUM_STAGES + 1 recorded torch CUDA events whose handles the timed entry point reuses."""
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(NUM_STAGES + 1)]
+    s = torch.cuda.current_stream() if stream is None else stream
+    for e in evs:
+        e.record(s)            # creates the underlying CUDA event
+    return evs
+
+
+def layer_forward_timed(shape: MoeShape, x, centroids, routed: Dict, shared: Optional[Dict], ws, events,
+                        out=None, idx=None, gate=None, counts=None, stream=None):
+    """layer_forward that also records `events` (from stage_events) at the stage boundaries."""
+    out = torch.empty((shape.T, shape.d), dtype=x.dtype, device=x.device) if out is None else out
+    rw = _weights(routed)
+    sw = _weights(shared)
+    arr = (ctypes.c_void_p * len(events))(*[e.cuda_event for e in events])
+    _check(_lib().moe_layer_forward_timed(ctypes.byref(shape), _ptr(x), _ptr(centroids), ctypes.byref(rw),
+                                          None if sw is None else ctypes.byref(sw), _ptr(out), _ptr(idx), _ptr(gate),
+                                          _ptr(counts), _ptr(ws), ws.numel(), _stream(stream), arr, len(events)),
+           "moe_layer_forward_timed")
     return out
 
 

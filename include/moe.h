@@ -175,6 +175,24 @@ moe_status_t moe_layer_forward(const moe_shape_t* shape, const void* x, const vo
                                void* out, int32_t* topk_idx_out, float* topk_gate_out,
                                int32_t* counts_out, void* ws, size_t ws_bytes, moe_stream_t stream);
 
+/*
+ * moe_layer_forward with stage timing: identical work and results, and in addition
+ * stage_events[i] (each a cudaEvent_t / CUevent created by the caller) is recorded on
+ * `stream` before stage i and stage_events[MOE_NUM_STAGES] after the last stage, so that
+ * cudaEventElapsedTime between neighbours gives each stage's device time.  Stages, in order:
+ *   0 router (scores, softmax, top-k)      1 grouping (histogram, scan, scatter)
+ *   2 tile tables of the grouped GEMMs     3 row gather of the routed tokens (bf16 only)
+ *   4 GEMM1 + SwiGLU (routed and shared)   5 routed GEMM2 with gates
+ *   6 shared GEMM2 + combine (or the combine alone when n_shared == 0)
+ * n_events must be MOE_NUM_STAGES + 1; MOE_ERR_INVALID_ARG otherwise.
+ */
+#define MOE_NUM_STAGES 7
+moe_status_t moe_layer_forward_timed(const moe_shape_t* shape, const void* x, const void* centroids,
+                                     const moe_ffn_weights_t* routed, const moe_ffn_weights_t* shared,
+                                     void* out, int32_t* topk_idx_out, float* topk_gate_out,
+                                     int32_t* counts_out, void* ws, size_t ws_bytes, moe_stream_t stream,
+                                     void* const* stage_events, int32_t n_events);
+
 #ifdef __cplusplus
 }
 #endif

@@ -1,0 +1,72 @@
+"""Host-side logic of bench.py on the CPU: the max-over-ranks reduction and whole-job
+throughput with two gloo ranks (the replica layout of multi-GPU runs), the per-stage
+algorithmic work, and the reference arm's JSON line on the tiny fp32 workload."""
+import json
+import os
+import subprocess
+import sys
+
+import pytest
+import torch
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+import bench  # noqa: E402
+from fine_grained_mixture_route_b200 import workloads as W  # noqa: E402
+
+
+def _rank(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world),
+                      LOCAL_RANK=str(rank))
+    bench.init_dist(world, "gloo")
+    try:
+        step_ms = 10.0 + 5.0 * rank                 # rank 1 is the slow one
+        ms = bench.reduce_max(step_ms, "cpu")
+        bench.barrier()
+        q.put((rank, ms, bench.aggregate_throughput(1000, world, ms)))
+    finally:
+        torch.distributed.destroy_process_group()
+
+
+def test_max_over_ranks_gloo():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = 29500 + os.getpid() % 1000
+    procs = [ctx.Process(target=_rank, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for rank, ms, tput in res:
+        assert ms == 15.0
+        assert abs(tput - 2 * 1000 / 0.015) < 1e-6
+
+
+def test_stage_work_sums_to_layer_flops():
+    for name, cfg in W.CONFIGS.items():
+        w = bench.stage_work(cfg, cfg.n_experts)
+        assert abs(sum(f for f, _ in w.values()) - cfg.flops()) < 1e-6 * cfg.flops(), name
+        assert all(b > 0 for _, b in w.values())
+    dec = W.CONFIGS["decode"]
+    # weight bytes of the whole layer when every expert is touched: 256 routed + 1 shared
+    per_expert = (3 * 7168 * 2048 + 2 * 2048 + 7168) * 2
+    assert abs(bench.layer_bytes(dec, 256) - (257 * per_expert + 256 * 7168 * 2 + 2 * 256 * 7168 * 2)) < 1
+
+
+def test_reference_arm_line():
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--workload", "tiny",
+                        "--steps", "3", "--warmup", "3"], capture_output=True, text=True, timeout=600,
+                       env={**os.environ, "CUDA_VISIBLE_DEVICES": ""})
+    assert r.returncode == 0, r.stderr
+    line = json.loads(r.stdout.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["unit"] == "tokens/s" and line["value"] > 0
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["kind"] == "oracle"
+    assert line["metric"] == bench.METRIC
+
+
+def test_warmup_must_be_three():
+    with pytest.raises(SystemExit):
+        bench.main(["--warmup", "2"])
