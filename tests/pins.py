@@ -122,6 +122,11 @@ def check_gate_invariants(O):
     g = r["gate"]
     assert np.array_equal(g, np.take_along_axis(s_ref, r["idx"], 1)) or \
         np.allclose(g, np.take_along_axis(s_ref, r["idx"], 1), rtol=1e-13, atol=0)
+    # softmax read at given picks: equals the routed gates at the oracle's own picks, and at
+    # arbitrary picks equals the library softmax read there
+    assert np.allclose(O.gates_from_indices(x, c, r["idx"]), g, rtol=1e-14, atol=0)
+    other = np.stack([np.random.default_rng(t).permutation(N)[:k] for t in range(T)])
+    assert np.allclose(O.gates_from_indices(x, c, other), np.take_along_axis(s_ref, other, 1), rtol=1e-12, atol=0)
     assert (g > 0).all() and (g <= 1).all()
     assert (g.sum(1) <= 1 + 1e-12).all()
     assert (np.diff(g, axis=1) <= 0).all(), "picks ordered by descending score"
