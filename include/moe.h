@@ -193,6 +193,37 @@ moe_status_t moe_layer_forward_timed(const moe_shape_t* shape, const void* x, co
                                      int32_t* counts_out, void* ws, size_t ws_bytes, moe_stream_t stream,
                                      void* const* stage_events, int32_t n_events);
 
+/*
+ * moe_permute_no_alloc — the paper has no counterpart to this entry point; it exists for
+ * callers of this library that cannot allocate device memory.  moe_permute needs scratch
+ * space, which it takes from the caller's workspace.  A caller that cannot call cudaMalloc
+ * (its framework already gave all device memory to its own caching allocator, it is a
+ * plug-in handed only input and output pointers, or it runs on a latency-critical path
+ * where an allocation, which may synchronise the device, is not allowed) has no workspace
+ * to give.  This variant computes exactly what moe_permute computes (same outputs, bit for
+ * bit) but keeps its scratch in a fixed array inside the library, and allocates nothing.
+ *
+ *   Arguments: as moe_permute, without ws / ws_bytes.  Inputs and outputs are still the
+ *   caller's device buffers.
+ *   Limit: the scratch is MOE_PERMUTE_NO_ALLOC_SCRATCH_BYTES (1 MiB) per GPU, held by every
+ *   GPU that loads the library until the process exits.  A call needs
+ *   ceil(T*top_k / 1024) * n_experts * 4 bytes of it (e.g. up to 1,048,576 slots with 256
+ *   experts); larger shapes are rejected with MOE_ERR_UNSUPPORTED before any launch.
+ *   Set-up: the first call on each device looks up the scratch's device address
+ *   (cudaGetSymbolAddress, with that device current); make that first call before any
+ *   stream capture.
+ *   Sharing: every call on a device uses the same scratch, which keeps the last call's
+ *   contents (nothing in it needs to start at zero).  Calls that overlap on the GPU race:
+ *   order them on one stream.
+ *   Errors: argument errors as moe_permute.  This variant has no error word: an expert
+ *   index outside [0, n_experts) drops that slot, its slot_of entry is -1 and
+ *   offsets[n_experts] comes out smaller than T*top_k.
+ */
+#define MOE_PERMUTE_NO_ALLOC_SCRATCH_BYTES (1u << 20)
+moe_status_t moe_permute_no_alloc(const moe_shape_t* shape, const int32_t* topk_idx, const float* topk_gate,
+                                  int32_t* counts, int32_t* offsets, int32_t* sorted_token,
+                                  float* sorted_gate, int32_t* slot_of, moe_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif
