@@ -332,7 +332,7 @@ def run_ours(args, cfg, rank, world, local_rank):
     stage_ms = {}
     for j, name in enumerate(moe.STAGE_NAMES):
         stage_ms[name] = statistics.mean(e[j].elapsed_time(e[j + 1]) for e in evs)
-    launches_per_step = 9 if cfg.dtype == torch.bfloat16 else 8
+    launches_per_step = moe.layer_launches(shape)
 
     # ---- end to end through the public API: pinned host input, H2D, layer, D2H
     e2e = None

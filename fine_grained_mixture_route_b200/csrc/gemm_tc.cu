@@ -15,15 +15,18 @@
 //           pick order (§2.3 and §3.1 of the DeepSeekMoE report: shared experts first, then
 //           the gated routed sum), and rounds once.
 //
-// Pipeline (192 threads, one CTA per SM, persistent over a static round-robin tile order):
+// Pipeline (320 threads, one CTA per SM, persistent over a static round-robin tile order):
 //   warp 0      TMA producer: 128B-swizzled K-major tiles of A (16 KB) and B (up to 32 KB)
 //               into a 4-stage shared-memory ring, completion counted on mbarriers;
 //   warp 1      allocates 512 TMEM columns; one thread issues tcgen05.mma (M=128, N<=256,
 //               K=16, bf16 x bf16 -> fp32) and commits each stage back to the producer and
 //               each finished accumulator to the epilogue;
-//   warps 2-5   epilogue: tcgen05.ld of their 32 TMEM lanes (one accumulator row each),
-//               fp32 math, bf16 stores.  Two accumulators (2 x 256 columns) let the
-//               epilogue of one tile overlap the main loop of the next.
+//   warps 2-9   epilogue: tcgen05.ld of their 32 TMEM lanes (one accumulator row per
+//               thread; the two warps of a lane quadrant split the columns), fp32 math,
+//               bf16 stores.  Two accumulators (2 x 256 columns) let the epilogue of one
+//               tile overlap the main loop of the next.
+//   ROUTERP     split-K variant of ROUTER for few token tiles: fp32 partial logits per
+//               K range, summed and ranked by a small CUDA-core kernel afterwards.
 // Every mbarrier wait is bounded (a few seconds of %globaltimer); on expiry the kernel sets
 // an error bit, stops issuing, waits (bounded) for its own copies and MMAs in flight, frees
 // TMEM and returns.  No cluster launch and no multicast anywhere.
@@ -40,13 +43,14 @@ constexpr int BK = 64;                   // K per stage: 64 bf16 = one 128-byte 
 constexpr int STAGES = 4;
 constexpr int A_BYTES = BM * BK * 2;     // 16 KB
 constexpr int B_BYTES = 256 * BK * 2;    // 32 KB (N <= 256)
-constexpr int THREADS = 192;
+constexpr int THREADS = 320;              // warp 0 TMA, warp 1 MMA, warps 2-9 epilogue
+constexpr int EPI_WARPS = 8;
 constexpr int TMEM_COLS = 512;
 constexpr int ACC_COLS = 256;
 constexpr int SMEM_BYTES = 1024 /*align slack*/ + STAGES * (A_BYTES + B_BYTES) + 256 /*barriers*/;
 constexpr unsigned long long WAIT_NS = 4000000000ull;
 
-enum Mode : int { ROUTER = 0, GEMM1 = 1, GEMM2R = 2, GEMM2S = 3 };
+enum Mode : int { ROUTER = 0, GEMM1 = 1, GEMM2R = 2, GEMM2S = 3, ROUTERP = 4 };
 
 struct Params {
     CUtensorMap tmA[2];
@@ -67,6 +71,8 @@ struct Params {
     __nv_bfloat16* out;
     int32_t* idx_out;
     float* gate_out;
+    float* partial;            // ROUTERP: [nsplit][T][E] fp32 partial logits
+    int kb_per_split;          // ROUTERP: K blocks per split
     uint32_t* err;
 };
 
@@ -197,11 +203,13 @@ struct Tile {
     int rows;    // rows of the group
     int row0;    // first row of the group in A and in the output
     int num_kb;  // K blocks of 64
+    int kb0;     // first K block (split-K router)
 };
 
 template <int MODE>
 __device__ __forceinline__ int total_tiles(const Params& p) {
     if (MODE == ROUTER) return ceil_div(p.T, BM);
+    if (MODE == ROUTERP) return ceil_div(p.T, BM) * ceil_div(ceil_div(p.d, BK), p.kb_per_split);
     if (MODE == GEMM1) return p.tile_start[p.g_end] - p.tile_start[p.g_begin];
     if (MODE == GEMM2R) return p.tile_start[p.E];
     return ceil_div(p.T, BM) * ceil_div(p.d, 256);
@@ -220,8 +228,16 @@ __device__ __forceinline__ int find_group(const int32_t* ts, int lo, int hi, int
 template <int MODE>
 __device__ __forceinline__ Tile decode(const Params& p, int t) {
     Tile x;
+    x.kb0 = 0;
     if (MODE == ROUTER) {
         x.g = 0; x.m0 = t * BM; x.n0 = 0; x.rows = p.T; x.row0 = 0; x.num_kb = ceil_div(p.d, BK);
+    } else if (MODE == ROUTERP) {
+        const int mt = ceil_div(p.T, BM);
+        const int split = t / mt;
+        const int kbt = ceil_div(p.d, BK);
+        x.g = split; x.m0 = (t % mt) * BM; x.n0 = 0; x.rows = p.T; x.row0 = 0;
+        x.kb0 = split * p.kb_per_split;
+        x.num_kb = min(p.kb_per_split, kbt - x.kb0);
     } else if (MODE == GEMM1) {
         const int tt = t + p.tile_start[p.g_begin];
         const int g = find_group(p.tile_start, p.g_begin, p.g_end, tt);
@@ -308,7 +324,8 @@ __device__ __forceinline__ void epilogue_router(const Params& p, const Tile& x, 
     }
 }
 
-__device__ __forceinline__ void epilogue_gemm1(const Params& p, const Tile& x, uint32_t tacc, int row) {
+// GEMM1: the two epilogue warps of a TMEM lane quadrant split the 128 hidden columns.
+__device__ __forceinline__ void epilogue_gemm1(const Params& p, const Tile& x, uint32_t tacc, int row, int half) {
     const bool shared = x.g >= p.E;
     const int e = shared ? x.g - p.E : x.g;
     const int I = shared ? p.Is : p.I;
@@ -320,7 +337,7 @@ __device__ __forceinline__ void epilogue_gemm1(const Params& p, const Tile& x, u
     const bool live = r < x.rows;
     __nv_bfloat16* hrow = shared ? p.h_s + ((size_t)e * p.T + r) * I : p.h_r + (size_t)(x.row0 + r) * I;
 #pragma unroll 1
-    for (int c = 0; c < 4; ++c) {
+    for (int c = half * 2; c < half * 2 + 2; ++c) {
         uint32_t u[32], v[32];
         tmem_ld32(tacc + c * 32, u);
         tmem_ld32(tacc + 128 + c * 32, v);
@@ -349,7 +366,8 @@ __device__ __forceinline__ void epilogue_gemm1(const Params& p, const Tile& x, u
     }
 }
 
-__device__ __forceinline__ void epilogue_gemm2r(const Params& p, const Tile& x, uint32_t tacc, int row) {
+// GEMM2R: each epilogue warp of a quadrant takes 128 of the 256 output columns.
+__device__ __forceinline__ void epilogue_gemm2r(const Params& p, const Tile& x, uint32_t tacc, int row, int half) {
     const int r = x.m0 + row;
     const bool live = r < x.rows;
     const long long pos = x.row0 + r;
@@ -357,7 +375,7 @@ __device__ __forceinline__ void epilogue_gemm2r(const Params& p, const Tile& x, 
     const __nv_bfloat16* b2 = p.b2 ? p.b2 + (size_t)x.g * p.d : nullptr;
     __nv_bfloat16* yrow = p.y + (size_t)pos * p.d;
 #pragma unroll 1
-    for (int c = 0; c < 8; ++c) {
+    for (int c = half * 4; c < half * 4 + 4; ++c) {
         uint32_t u[32];
         tmem_ld32(tacc + c * 32, u);
         tmem_wait_ld();
@@ -380,49 +398,112 @@ __device__ __forceinline__ void epilogue_gemm2r(const Params& p, const Tile& x, 
     }
 }
 
-__device__ __forceinline__ void epilogue_gemm2s(const Params& p, const Tile& x, uint32_t tacc, int row) {
+__device__ __forceinline__ void add_bf16x8(float (&acc)[8], const uint4& w) {
+    const __nv_bfloat16* e = reinterpret_cast<const __nv_bfloat16*>(&w);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] += __bfloat162float(e[i]);
+}
+
+// GEMM2S: out[t] = shared accumulator + shared biases + the token's routed rows, j ascending.
+// Each thread owns one token row and 128 columns, walked in 16 steps of 8 columns; the
+// routed-row loads of step i+1 are in flight while step i is summed.
+constexpr int COMBINE_FAST_K = 8;
+__device__ __forceinline__ void epilogue_gemm2s(const Params& p, const Tile& x, uint32_t tacc, int row, int half) {
     const int t = x.m0 + row;
     const bool live = t < p.T;
+    const int cbase = half * 128;                    // first accumulator column of this thread
+    __nv_bfloat16* orow = p.out + (size_t)t * p.d;
+    if (p.k <= COMBINE_FAST_K) {
+        int sl[COMBINE_FAST_K];
+#pragma unroll
+        for (int j = 0; j < COMBINE_FAST_K; ++j) {
+            int pos = -1;
+            if (live && j < p.k) {
+                pos = p.slot_of[(size_t)t * p.k + j];
+                if (pos < 0 || pos >= p.S) { flag_error(p.err, ERR_INDEX_RANGE); pos = -1; }
+            }
+            sl[j] = pos;
+        }
+        uint4 buf[2][COMBINE_FAST_K];
+        auto issue = [&](uint4 (&b)[COMBINE_FAST_K], int step) {
+            const int col = x.n0 + cbase + step * 8;
+#pragma unroll
+            for (int j = 0; j < COMBINE_FAST_K; ++j)
+                b[j] = (sl[j] >= 0 && col < p.d)
+                           ? __ldg(reinterpret_cast<const uint4*>(p.y_in + (size_t)sl[j] * p.d + col))
+                           : make_uint4(0, 0, 0, 0);
+        };
+        issue(buf[0], 0);
+#pragma unroll
+        for (int step = 0; step < 16; ++step) {
+            if (step + 1 < 16) issue(buf[(step + 1) & 1], step + 1);
+            uint32_t u[8];
+            asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                         : "=r"(u[0]), "=r"(u[1]), "=r"(u[2]), "=r"(u[3]), "=r"(u[4]), "=r"(u[5]), "=r"(u[6]),
+                           "=r"(u[7])
+                         : "r"(tacc + cbase + step * 8));
+            tmem_wait_ld();
+            const int col = x.n0 + cbase + step * 8;
+            if (!live || col >= p.d) continue;
+            float acc[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) acc[i] = __uint_as_float(u[i]);
+            if (p.sb2)
+                for (int s = 0; s < p.Ks; ++s)
+                    add_bf16x8(acc, __ldg(reinterpret_cast<const uint4*>(p.sb2 + (size_t)s * p.d + col)));
+#pragma unroll
+            for (int j = 0; j < COMBINE_FAST_K; ++j) add_bf16x8(acc, buf[step & 1][j]);
+            uint4 o;
+            o.x = pack_bf16(acc[0], acc[1]); o.y = pack_bf16(acc[2], acc[3]);
+            o.z = pack_bf16(acc[4], acc[5]); o.w = pack_bf16(acc[6], acc[7]);
+            *reinterpret_cast<uint4*>(orow + col) = o;
+        }
+    } else {
 #pragma unroll 1
-    for (int c = 0; c < 8; ++c) {
-        uint32_t u[32];
-        tmem_ld32(tacc + c * 32, u);
+        for (int step = 0; step < 16; ++step) {
+            uint32_t u[8];
+            asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                         : "=r"(u[0]), "=r"(u[1]), "=r"(u[2]), "=r"(u[3]), "=r"(u[4]), "=r"(u[5]), "=r"(u[6]),
+                           "=r"(u[7])
+                         : "r"(tacc + cbase + step * 8));
+            tmem_wait_ld();
+            const int col = x.n0 + cbase + step * 8;
+            if (!live || col >= p.d) continue;
+            float acc[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) acc[i] = __uint_as_float(u[i]);
+            if (p.sb2)
+                for (int s = 0; s < p.Ks; ++s)
+                    add_bf16x8(acc, __ldg(reinterpret_cast<const uint4*>(p.sb2 + (size_t)s * p.d + col)));
+            for (int j = 0; j < p.k; ++j) {
+                const int pos = p.slot_of[(size_t)t * p.k + j];
+                if (pos < 0 || pos >= p.S) { flag_error(p.err, ERR_INDEX_RANGE); continue; }
+                add_bf16x8(acc, __ldg(reinterpret_cast<const uint4*>(p.y_in + (size_t)pos * p.d + col)));
+            }
+            uint4 o;
+            o.x = pack_bf16(acc[0], acc[1]); o.y = pack_bf16(acc[2], acc[3]);
+            o.z = pack_bf16(acc[4], acc[5]); o.w = pack_bf16(acc[6], acc[7]);
+            *reinterpret_cast<uint4*>(orow + col) = o;
+        }
+    }
+}
+
+// ROUTERP (split-K router): each thread writes its token row's partial logits over this
+// tile's K range; the two warps of a quadrant alternate 16-column groups.
+__device__ __forceinline__ void epilogue_router_partial(const Params& p, const Tile& x, uint32_t tacc, int row,
+                                                        int half) {
+    const int t = x.m0 + row;
+    float* dst = p.partial + ((size_t)x.g * p.T + t) * p.E;
+    for (int c0 = half * 16; c0 < p.n_mma; c0 += 32) {
+        uint32_t r[16];
+        tmem_ld16(tacc + c0, r);
         tmem_wait_ld();
-        const int col0 = x.n0 + c * 32;
-        if (!live || col0 >= p.d) continue;
-        float acc[32];
+        if (t < p.T) {
 #pragma unroll
-        for (int j = 0; j < 32; ++j) acc[j] = __uint_as_float(u[j]);
-        if (p.sb2) {
-            for (int s = 0; s < p.Ks; ++s) {
-                const __nv_bfloat16* b = p.sb2 + (size_t)s * p.d + col0;
-#pragma unroll
-                for (int j = 0; j < 32; ++j)
-                    if (col0 + j < p.d) acc[j] += __bfloat162float(b[j]);
-            }
-        }
-        for (int jj = 0; jj < p.k; ++jj) {
-            const int pos = p.slot_of[(size_t)t * p.k + jj];
-            if (pos < 0 || pos >= p.S) { flag_error(p.err, ERR_INDEX_RANGE); continue; }
-            const uint4* src = reinterpret_cast<const uint4*>(p.y_in + (size_t)pos * p.d + col0);
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                if (col0 + q * 8 >= p.d) break;
-                uint4 w = __ldg(src + q);
-                const __nv_bfloat16* e = reinterpret_cast<const __nv_bfloat16*>(&w);
-#pragma unroll
-                for (int i = 0; i < 8; ++i) acc[q * 8 + i] += __bfloat162float(e[i]);
-            }
-        }
-        __nv_bfloat16* orow = p.out + (size_t)t * p.d;
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const int col = col0 + q * 8;
-            if (col >= p.d) break;
-            uint32_t pk[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) pk[i] = pack_bf16(acc[q * 8 + i * 2], acc[q * 8 + i * 2 + 1]);
-            *reinterpret_cast<uint4*>(orow + col) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            for (int q = 0; q < 4; ++q)
+                *reinterpret_cast<float4*>(dst + c0 + q * 4) =
+                    make_float4(__uint_as_float(r[q * 4]), __uint_as_float(r[q * 4 + 1]), __uint_as_float(r[q * 4 + 2]),
+                                __uint_as_float(r[q * 4 + 3]));
         }
     }
 }
@@ -449,7 +530,7 @@ __global__ void __launch_bounds__(THREADS, 1) moe_tc_kernel(const __grid_constan
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) { mbar_init(full_bar(s), 1); mbar_init(empty_bar(s), 1); }
-        for (int a = 0; a < 2; ++a) { mbar_init(tfull_bar(a), 1); mbar_init(tempty_bar(a), 4); }
+        for (int a = 0; a < 2; ++a) { mbar_init(tfull_bar(a), 1); mbar_init(tempty_bar(a), EPI_WARPS); }
         mbar_init(drain_bar, 1);
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -480,11 +561,12 @@ __global__ void __launch_bounds__(THREADS, 1) moe_tc_kernel(const __grid_constan
             bool ok = true;
             for (int t = blockIdx.x; ok && t < ntiles; t += gridDim.x) {
                 const Tile x = decode<MODE>(p, t);
-                for (int kb = 0; kb < x.num_kb; ++kb) {
+                for (int kk_ = 0; kk_ < x.num_kb; ++kk_) {
+                    const int kb = x.kb0 + kk_;
                     if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, p.err)) { ok = false; break; }
                     const uint32_t fb = full_bar(stage);
                     const uint32_t a_dst = sA + stage * A_BYTES, b_dst = sB + stage * B_BYTES;
-                    if (MODE == ROUTER) {
+                    if (MODE == ROUTER || MODE == ROUTERP) {
                         mbar_expect_tx(fb, A_BYTES + p.n_mma * BK * 2);
                         tma_load_2d(a_dst, &p.tmA[0], fb, kb * BK, x.m0);
                         tma_load_2d(b_dst, &p.tmB[0], fb, kb * BK, 0);
@@ -553,6 +635,7 @@ __global__ void __launch_bounds__(THREADS, 1) moe_tc_kernel(const __grid_constan
     } else {
         // ------------------------------------------------------------------ epilogue
         const int quad = warp & 3;                  // TMEM lanes 32*quad .. 32*quad+31
+        const int half = (warp - 2) / 4;            // which half of the columns (0 or 1)
         const int row = quad * 32 + lane;
         int acc = 0;
         uint32_t acc_phase = 0;
@@ -561,10 +644,17 @@ __global__ void __launch_bounds__(THREADS, 1) moe_tc_kernel(const __grid_constan
             if (!mbar_wait(tfull_bar(acc), acc_phase, abort_flag, p.err)) break;
             tc_fence_after();
             const uint32_t tacc = tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(acc * ACC_COLS);
-            if (MODE == ROUTER) epilogue_router<KMAX>(p, x, tacc, row);
-            else if (MODE == GEMM1) epilogue_gemm1(p, x, tacc, row);
-            else if (MODE == GEMM2R) epilogue_gemm2r(p, x, tacc, row);
-            else epilogue_gemm2s(p, x, tacc, row);
+            if (MODE == ROUTER) {
+                if (half == 0) epilogue_router<KMAX>(p, x, tacc, row);
+            } else if (MODE == ROUTERP) {
+                epilogue_router_partial(p, x, tacc, row, half);
+            } else if (MODE == GEMM1) {
+                epilogue_gemm1(p, x, tacc, row, half);
+            } else if (MODE == GEMM2R) {
+                epilogue_gemm2r(p, x, tacc, row, half);
+            } else {
+                epilogue_gemm2s(p, x, tacc, row, half);
+            }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(tempty_bar(acc));
@@ -646,8 +736,19 @@ int num_sms() {
 
 bool tc_router_supported(const Dims& D) { return D.bf16 && D.E % 16 == 0 && D.E >= 16 && D.E <= 256; }
 
+int router_splits(const Dims& D) {
+    if (!tc_router_supported(D) || D.T == 0) return 1;
+    const int mt = ceil_div(D.T, tc::BM);
+    const int kbt = ceil_div(D.d, tc::BK);
+    if (mt > 32 || kbt < 8) return 1;
+    constexpr int kCtas = 148;                       // fixed so the workspace size never depends on the GPU
+    const int want = ceil_div(kCtas, mt);
+    const int per = ceil_div(kbt, want < kbt ? want : kbt);
+    return ceil_div(kbt, per < 2 ? 2 : per);
+}
+
 cudaError_t launch_tc_router(const Dims& D, const void* x, const void* centroids, int32_t* idx, float* gate,
-                             uint32_t* err, cudaStream_t stream) {
+                             float* partial, uint32_t* err, cudaStream_t stream) {
     using namespace tc;
     if (D.T == 0) return cudaSuccess;
     Params p = base_params(D, err);
@@ -656,8 +757,19 @@ cudaError_t launch_tc_router(const Dims& D, const void* x, const void* centroids
     p.gate_out = gate;
     if (!make_map(&p.tmA[0], x, D.d, D.T, 1, BK, BM, false)) return cudaErrorInvalidValue;
     if (!make_map(&p.tmB[0], centroids, D.d, D.E, 1, BK, D.E, false)) return cudaErrorInvalidValue;
-    const int tiles = ceil_div(D.T, BM);
-    const int grid = tiles < num_sms() ? tiles : num_sms();
+    const int mt = ceil_div(D.T, BM);
+    const int nsplit = router_splits(D);
+    if (nsplit > 1 && partial) {
+        const int kbt = ceil_div(D.d, BK);
+        p.kb_per_split = ceil_div(kbt, nsplit);
+        p.partial = partial;
+        const int tiles = mt * ceil_div(kbt, p.kb_per_split);
+        const int grid = tiles < num_sms() ? tiles : num_sms();
+        cudaError_t e = launch<ROUTERP, 8>(p, grid, stream);
+        if (e != cudaSuccess) return e;
+        return launch_router_finish(D, partial, ceil_div(kbt, p.kb_per_split), idx, gate, stream);
+    }
+    const int grid = mt < num_sms() ? mt : num_sms();
     return D.k <= 8 ? launch<ROUTER, 8>(p, grid, stream) : launch<ROUTER, 32>(p, grid, stream);
 }
 

@@ -69,8 +69,18 @@ cudaError_t launch_simt_gemm2_shared(const Dims& D, const FfnWeights& shared, co
 // All four run the same persistent warp-specialised pipeline: a TMA producer warp, one MMA
 // issuing thread, four epilogue warps reading the fp32 accumulators out of tensor memory.
 bool tc_router_supported(const Dims& D);
+// Split-K policy of the tensor-core router: with few 128-token tiles (decode-sized T) the K
+// range is split over CTAs and each writes fp32 partial logits [nsplit][T][N_m]; a CUDA-core
+// kernel sums them in split order and does the softmax / top-k.  Returns 1 for no split.
+int router_splits(const Dims& D);
+inline size_t router_partial_bytes(const Dims& D) {
+    const int n = router_splits(D);
+    return n > 1 ? (size_t)n * D.T * D.E * sizeof(float) : 0;
+}
 cudaError_t launch_tc_router(const Dims& D, const void* x, const void* centroids, int32_t* idx, float* gate,
-                             uint32_t* err, cudaStream_t stream);
+                             float* partial, uint32_t* err, cudaStream_t stream);
+cudaError_t launch_router_finish(const Dims& D, const float* partial, int nsplit, int32_t* idx, float* gate,
+                                 cudaStream_t stream);
 // GEMM1 + SwiGLU over groups [g_begin, g_end): A rows from x_perm (routed) or x (shared).
 cudaError_t launch_tc_gemm1(const Dims& D, const void* x, const void* x_perm, const int32_t* offsets,
                             const int32_t* tile_start1, const FfnWeights& routed, const FfnWeights& shared,

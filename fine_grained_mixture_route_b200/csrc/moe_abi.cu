@@ -14,7 +14,7 @@ namespace {
 size_t al(size_t x) { return (x + 255) & ~(size_t)255; }
 
 struct Layout {
-    size_t err, hist, ts1, ts2, idx, gate, counts, offsets, stok, sgate, slot_of, xperm, hr, hs, y, total;
+    size_t err, hist, rpart, ts1, ts2, idx, gate, counts, offsets, stok, sgate, slot_of, xperm, hr, hs, y, total;
 };
 
 Layout layout(const Dims& D) {
@@ -25,6 +25,7 @@ Layout layout(const Dims& D) {
     size_t o = 0;
     L.err = o; o += 256;
     L.hist = o; o += al((nblk ? nblk : 1) * D.E * 4);
+    L.rpart = o; o += al(router_partial_bytes(D));
     L.ts1 = o; o += al((size_t)(D.E + D.Ks + 1) * 4);
     L.ts2 = o; o += al((size_t)(D.E + 1) * 4);
     L.idx = o; o += al(S * 4);
@@ -101,10 +102,10 @@ FfnWeights to_ffn(const moe_ffn_weights_t* w) {
     return f;
 }
 
-moe_status_t do_route(const Dims& D, const void* x, const void* c, int32_t* idx, float* gate, uint32_t* err,
-                      cudaStream_t st) {
+moe_status_t do_route(const Dims& D, const void* x, const void* c, int32_t* idx, float* gate, float* partial,
+                      uint32_t* err, cudaStream_t st) {
     if (D.T == 0) return MOE_OK;
-    if (tc_router_supported(D)) MOE_CUDA(launch_tc_router(D, x, c, idx, gate, err, st));
+    if (tc_router_supported(D)) MOE_CUDA(launch_tc_router(D, x, c, idx, gate, partial, err, st));
     else MOE_CUDA(launch_router_simt(D, x, c, idx, gate, st));
     return MOE_OK;
 }
@@ -156,6 +157,20 @@ MOE_EXPORT const char* moe_status_string(moe_status_t s) {
     return "MOE_ERR_UNKNOWN";
 }
 
+MOE_EXPORT int32_t moe_layer_launches(const moe_shape_t* shape) {
+    Dims D;
+    if (to_dims(shape, &D) != MOE_OK) return -1;
+    if (D.T == 0) return 0;
+    int n = 0;
+    if (tc_router_supported(D)) n += router_splits(D) > 1 ? 2 : 1;   // scores (+ split-K finish)
+    else n += 1;
+    n += 3;                                                         // histogram, scan, scatter
+    n += 1;                                                         // tile tables
+    if (D.bf16) n += 1;                                             // row gather
+    n += 3;                                                         // GEMM1, GEMM2, shared GEMM2 / combine
+    return n;
+}
+
 MOE_EXPORT const char* moe_version(void) { return "moe_b200 0.1 sm_100a"; }
 
 MOE_EXPORT moe_status_t moe_ws_init(void* ws, size_t ws_bytes, moe_stream_t stream) {
@@ -189,7 +204,8 @@ MOE_EXPORT moe_status_t moe_route(const moe_shape_t* shape, const void* x, const
     MOE_TRY(check_device());
     cudaGetLastError();
     const Layout L = layout(D);
-    return do_route(D, x, centroids, topk_idx, topk_gate, at<uint32_t>(ws, L.err), (cudaStream_t)stream);
+    return do_route(D, x, centroids, topk_idx, topk_gate, at<float>(ws, L.rpart), at<uint32_t>(ws, L.err),
+                    (cudaStream_t)stream);
 }
 
 MOE_EXPORT moe_status_t moe_permute(const moe_shape_t* shape, const int32_t* topk_idx, const float* topk_gate,
@@ -302,7 +318,7 @@ moe_status_t layer_forward_impl(const moe_shape_t* shape, const void* x, const v
     auto mark = [&](int i) -> bool { return !ev || cudaEventRecord(ev[i], st) == cudaSuccess; };
 
     if (!mark(0)) return MOE_ERR_CUDA;
-    MOE_TRY(do_route(D, x, centroids, idx, gate, err, st));
+    MOE_TRY(do_route(D, x, centroids, idx, gate, at<float>(ws, L.rpart), err, st));
     if (!mark(1)) return MOE_ERR_CUDA;
     MOE_CUDA(launch_permute(D, idx, gate, counts, offsets, stok, sgate, slot_of, at<int32_t>(ws, L.hist), err, st));
     if (!mark(2)) return MOE_ERR_CUDA;

@@ -18,6 +18,41 @@ constexpr int RT_EXP = 64;      // experts per score tile
 constexpr int RT_K = 64;        // hidden elements per score tile
 constexpr int RT_THREADS = 256;
 
+// Softmax over the E logits in zr (shared memory, clobbered) and the top-k picks by one warp:
+// max and sum of exponentials by shuffles, then k rounds of warp argmax on (logit, -index),
+// so equal logits go to the lower index and picks come out by descending score.
+__device__ void warp_softmax_topk(float* zr, int E, int k, int lane, int32_t* idx_row, float* gate_row) {
+    float m = -INFINITY;
+    for (int e = lane; e < E; e += 32) m = fmaxf(m, zr[e]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    float s = 0.f;
+    for (int e = lane; e < E; e += 32) s += expf(zr[e] - m);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    const float inv = 1.0f / s;
+    for (int j = 0; j < k; ++j) {
+        float bv = -INFINITY;
+        int bi = 0x7fffffff;
+        for (int e = lane; e < E; e += 32) {
+            float v = zr[e];
+            if (v > bv) { bv = v; bi = e; }     // ascending e: equal values keep the lower index
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+            int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+            if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
+        }
+        if (lane == 0) {
+            idx_row[j] = bi;
+            gate_row[j] = expf(bv - m) * inv;
+        }
+        if (bi < E && (bi % 32) == lane) zr[bi] = -INFINITY;   // owner lane removes the pick
+        __syncwarp();
+    }
+}
+
 template <typename T>
 __global__ void __launch_bounds__(RT_THREADS)
 router_simt_kernel(const T* __restrict__ x, const T* __restrict__ cen, int32_t* __restrict__ idx_out,
@@ -68,37 +103,29 @@ router_simt_kernel(const T* __restrict__ x, const T* __restrict__ cen, int32_t* 
     for (int r = warp; r < RT_TOK; r += RT_THREADS / 32) {
         const int t = t0 + r;
         if (t >= Tn) break;
-        float* zr = z + r * E;
-        float m = -INFINITY;
-        for (int e = lane; e < E; e += 32) m = fmaxf(m, zr[e]);
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-        float s = 0.f;
-        for (int e = lane; e < E; e += 32) s += expf(zr[e] - m);
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-        const float inv = 1.0f / s;
-        for (int j = 0; j < k; ++j) {
-            float bv = -INFINITY;
-            int bi = 0x7fffffff;
-            for (int e = lane; e < E; e += 32) {
-                float v = zr[e];
-                if (v > bv) { bv = v; bi = e; }     // ascending e: equal values keep the lower index
-            }
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-                float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-                int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-                if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
-            }
-            if (lane == 0) {
-                idx_out[(size_t)t * k + j] = bi;
-                gate_out[(size_t)t * k + j] = expf(bv - m) * inv;
-            }
-            if (bi < E && (bi % 32) == lane) zr[bi] = -INFINITY;   // owner lane removes the pick
-            __syncwarp();
-        }
+        warp_softmax_topk(z + r * E, E, k, lane, idx_out + (size_t)t * k, gate_out + (size_t)t * k);
     }
+}
+
+
+// Split-K router, last step: z = sum of the per-split partial logits in ascending split order
+// (deterministic), then the same softmax / top-k as above.  One warp per token.
+constexpr int FIN_WARPS = 8;
+__global__ void __launch_bounds__(FIN_WARPS * 32)
+router_finish_kernel(const float* __restrict__ partial, int nsplit, int Tn, int E, int k, int32_t* __restrict__ idx_out,
+                     float* __restrict__ gate_out) {
+    extern __shared__ float zs[];
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const int t = blockIdx.x * FIN_WARPS + warp;
+    if (t >= Tn) return;
+    float* zr = zs + warp * E;
+    for (int e = lane; e < E; e += 32) {
+        float v = 0.f;
+        for (int s = 0; s < nsplit; ++s) v += partial[((size_t)s * Tn + t) * E + e];
+        zr[e] = v;
+    }
+    __syncwarp();
+    warp_softmax_topk(zr, E, k, lane, idx_out + (size_t)t * k, gate_out + (size_t)t * k);
 }
 
 }  // namespace
@@ -118,6 +145,14 @@ cudaError_t launch_router_simt(const Dims& D, const void* x, const void* centroi
         kern<<<blocks, RT_THREADS, smem, stream>>>((const float*)x, (const float*)centroids, idx, gate, D.T, D.d, D.E,
                                                    D.k);
     }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_router_finish(const Dims& D, const float* partial, int nsplit, int32_t* idx, float* gate,
+                                 cudaStream_t stream) {
+    const int blocks = ceil_div(D.T, FIN_WARPS);
+    const size_t smem = sizeof(float) * FIN_WARPS * D.E;
+    router_finish_kernel<<<blocks, FIN_WARPS * 32, smem, stream>>>(partial, nsplit, D.T, D.E, D.k, idx, gate);
     return cudaGetLastError();
 }
 

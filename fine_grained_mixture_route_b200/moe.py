@@ -17,7 +17,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe_b200
 MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_CUDA, MOE_ERR_INTERNAL = range(6)
 MOE_F32, MOE_BF16 = 0, 1
 
-EXPORTED = ("moe_workspace_bytes", "moe_status_string", "moe_version", "moe_check_device_error", "moe_ws_init",
+EXPORTED = ("moe_workspace_bytes", "moe_layer_launches", "moe_status_string", "moe_version", "moe_check_device_error", "moe_ws_init",
             "moe_route", "moe_permute", "moe_expert_ffn", "moe_combine", "moe_layer_forward",
             "moe_layer_forward_timed", "moe_permute_no_alloc")
 NUM_STAGES = 7
@@ -55,6 +55,8 @@ def _lib():
         wp = ctypes.POINTER(MoeWeights)
         lib.moe_workspace_bytes.argtypes = [sh]
         lib.moe_workspace_bytes.restype = sz
+        lib.moe_layer_launches.argtypes = [sh]
+        lib.moe_layer_launches.restype = ctypes.c_int32
         lib.moe_status_string.argtypes = [ctypes.c_int]
         lib.moe_status_string.restype = ctypes.c_char_p
         lib.moe_version.argtypes = []
@@ -120,6 +122,11 @@ def _weights(w: Optional[Dict]):
 
 def workspace_bytes(shape: MoeShape) -> int:
     return int(_lib().moe_workspace_bytes(ctypes.byref(shape)))
+
+
+def layer_launches(shape: MoeShape) -> int:
+    """Kernel launches one layer_forward call makes for this shape."""
+    return int(_lib().moe_layer_launches(ctypes.byref(shape)))
 
 
 def new_workspace(shape: MoeShape, device="cuda") -> torch.Tensor:

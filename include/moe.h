@@ -91,6 +91,10 @@ size_t moe_workspace_bytes(const moe_shape_t* shape);
 /* Static description of a status code; never NULL. */
 const char* moe_status_string(moe_status_t status);
 
+/* Number of kernel launches one moe_layer_forward call makes for this shape (-1 if the
+ * shape is invalid, 0 when T == 0). */
+int32_t moe_layer_launches(const moe_shape_t* shape);
+
 /* Library version string, e.g. "moe_b200 0.1 sm_100a". */
 const char* moe_version(void);
 

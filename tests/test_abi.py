@@ -57,7 +57,8 @@ def test_workspace_bytes(lib):
     S, d, I = 256 * 8, 7168, 2048
     # x_perm, h_r, Y (bf16) and the shared hidden states at least
     assert n >= 2 * (S * d + S * I + S * d + 256 * 2048)
-    assert n < 2 * (S * d + S * I + S * d + 256 * 2048) + 4 * 1024 * 1024
+    # ... plus the split-K router's fp32 partial logits (at most 148 CTAs x 128 tokens x N_m)
+    assert n < 2 * (S * d + S * I + S * d + 256 * 2048) + 4 * 1024 * 1024 + 148 * 128 * 256 * 4
     assert moe.workspace_bytes(_shape(T=512)) > n
     assert moe.workspace_bytes(_shape(T=0)) > 0
     # fp32 layers keep no gathered copy of x
@@ -67,6 +68,15 @@ def test_workspace_bytes(lib):
                 dict(has_bias=2), dict(n_shared=1, inter_shared=0)):
         assert moe.workspace_bytes(_shape(**bad)) == 0, bad
     assert moe.workspace_bytes(_shape(d=7170, dtype=moe.MOE_F32)) > 0
+
+
+def test_launch_count(lib):
+    assert moe.layer_launches(_shape()) == 10          # split-K router at T=256: scores + finish
+    assert moe.layer_launches(_shape(T=16384)) == 9
+    assert moe.layer_launches(_shape(T=128, d=256, n_experts=16, inter=64, inter_shared=64, top_k=4,
+                                     dtype=moe.MOE_F32)) == 8
+    assert moe.layer_launches(_shape(T=0)) == 0
+    assert moe.layer_launches(_shape(top_k=0)) == -1
 
 
 def test_argument_errors_return_before_any_launch(lib):
