@@ -102,8 +102,9 @@ def stage_work(cfg: W.LayerConfig, touched: int):
                          touched * (2 * I * d + 2 * I * bias) * b + Ks * (2 * Is * d + 2 * Is * bias) * b
                          + S * d * b + (T * d * b if Ks else 0) + (S * I + Ks * T * Is) * b),
         "gemm2_gate": (2.0 * S * I * d, touched * (d * I + d * bias) * b + S * I * b + S * d * b + S * 8),
-        "combine": (2.0 * Ks * T * Is * d, Ks * (d * Is + d * bias) * b + Ks * T * Is * b + S * d * b + T * d * b
-                    + S * 4),
+        "gemm2_shared": (2.0 * Ks * T * Is * d, Ks * (d * Is + d * bias) * b + Ks * T * Is * b
+                         + (T * d * 4 if Ks else 0)),
+        "combine": (0.0, S * d * b + (T * d * 4 if Ks else 0) + T * d * b + S * 4),
     }
     return w
 

@@ -11,9 +11,9 @@
 //   GEMM2R  routed w2 contraction; the epilogue adds b2 and scales by the gate: the gate
 //           multiplies the whole expert output.
 //   GEMM2S  the K_s shared experts' w2 contractions accumulated along K in one accumulator;
-//           the epilogue adds the shared biases and then the token's N_r gated routed rows in
-//           pick order (§2.3 and §3.1 of the DeepSeekMoE report: shared experts first, then
-//           the gated routed sum), and rounds once.
+//           the epilogue adds the shared biases and writes the fp32 shared output, to which
+//           the combine kernel adds each token's gated routed rows in pick order (§2.3 and
+//           §3.1 of the DeepSeekMoE report: shared experts first, then the gated routed sum).
 //
 // Pipeline (320 threads, one CTA per SM, persistent over a static round-robin tile order):
 //   warp 0      TMA producer: 128B-swizzled K-major tiles of A (16 KB) and B (up to 32 KB)
@@ -66,9 +66,7 @@ struct Params {
     __nv_bfloat16* h_s;
     const float* sorted_gate;
     __nv_bfloat16* y;
-    const __nv_bfloat16* y_in;
-    const int32_t* slot_of;
-    __nv_bfloat16* out;
+    float* sout;               // GEMM2S: fp32 shared-expert output [T][d]
     int32_t* idx_out;
     float* gate_out;
     float* partial;            // ROUTERP: [nsplit][T][E] fp32 partial logits
@@ -398,92 +396,31 @@ __device__ __forceinline__ void epilogue_gemm2r(const Params& p, const Tile& x, 
     }
 }
 
-__device__ __forceinline__ void add_bf16x8(float (&acc)[8], const uint4& w) {
-    const __nv_bfloat16* e = reinterpret_cast<const __nv_bfloat16*>(&w);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) acc[i] += __bfloat162float(e[i]);
-}
-
-// GEMM2S: out[t] = shared accumulator + shared biases + the token's routed rows, j ascending.
-// Each thread owns one token row and 128 columns, walked in 16 steps of 8 columns; the
-// routed-row loads of step i+1 are in flight while step i is summed.
-constexpr int COMBINE_FAST_K = 8;
+// GEMM2S: the shared experts' output (accumulator + their b2 summed), fp32, for the combine.
 __device__ __forceinline__ void epilogue_gemm2s(const Params& p, const Tile& x, uint32_t tacc, int row, int half) {
     const int t = x.m0 + row;
     const bool live = t < p.T;
-    const int cbase = half * 128;                    // first accumulator column of this thread
-    __nv_bfloat16* orow = p.out + (size_t)t * p.d;
-    if (p.k <= COMBINE_FAST_K) {
-        int sl[COMBINE_FAST_K];
-#pragma unroll
-        for (int j = 0; j < COMBINE_FAST_K; ++j) {
-            int pos = -1;
-            if (live && j < p.k) {
-                pos = p.slot_of[(size_t)t * p.k + j];
-                if (pos < 0 || pos >= p.S) { flag_error(p.err, ERR_INDEX_RANGE); pos = -1; }
-            }
-            sl[j] = pos;
-        }
-        uint4 buf[2][COMBINE_FAST_K];
-        auto issue = [&](uint4 (&b)[COMBINE_FAST_K], int step) {
-            const int col = x.n0 + cbase + step * 8;
-#pragma unroll
-            for (int j = 0; j < COMBINE_FAST_K; ++j)
-                b[j] = (sl[j] >= 0 && col < p.d)
-                           ? __ldg(reinterpret_cast<const uint4*>(p.y_in + (size_t)sl[j] * p.d + col))
-                           : make_uint4(0, 0, 0, 0);
-        };
-        issue(buf[0], 0);
-#pragma unroll
-        for (int step = 0; step < 16; ++step) {
-            if (step + 1 < 16) issue(buf[(step + 1) & 1], step + 1);
-            uint32_t u[8];
-            asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
-                         : "=r"(u[0]), "=r"(u[1]), "=r"(u[2]), "=r"(u[3]), "=r"(u[4]), "=r"(u[5]), "=r"(u[6]),
-                           "=r"(u[7])
-                         : "r"(tacc + cbase + step * 8));
-            tmem_wait_ld();
-            const int col = x.n0 + cbase + step * 8;
-            if (!live || col >= p.d) continue;
-            float acc[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) acc[i] = __uint_as_float(u[i]);
-            if (p.sb2)
-                for (int s = 0; s < p.Ks; ++s)
-                    add_bf16x8(acc, __ldg(reinterpret_cast<const uint4*>(p.sb2 + (size_t)s * p.d + col)));
-#pragma unroll
-            for (int j = 0; j < COMBINE_FAST_K; ++j) add_bf16x8(acc, buf[step & 1][j]);
-            uint4 o;
-            o.x = pack_bf16(acc[0], acc[1]); o.y = pack_bf16(acc[2], acc[3]);
-            o.z = pack_bf16(acc[4], acc[5]); o.w = pack_bf16(acc[6], acc[7]);
-            *reinterpret_cast<uint4*>(orow + col) = o;
-        }
-    } else {
+    float* srow = p.sout + (size_t)t * p.d;
 #pragma unroll 1
-        for (int step = 0; step < 16; ++step) {
-            uint32_t u[8];
-            asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
-                         : "=r"(u[0]), "=r"(u[1]), "=r"(u[2]), "=r"(u[3]), "=r"(u[4]), "=r"(u[5]), "=r"(u[6]),
-                           "=r"(u[7])
-                         : "r"(tacc + cbase + step * 8));
-            tmem_wait_ld();
-            const int col = x.n0 + cbase + step * 8;
-            if (!live || col >= p.d) continue;
-            float acc[8];
+    for (int c = half * 4; c < half * 4 + 4; ++c) {
+        uint32_t u[32];
+        tmem_ld32(tacc + c * 32, u);
+        tmem_wait_ld();
+        const int col0 = x.n0 + c * 32;
+        if (!live || col0 >= p.d) continue;
 #pragma unroll
-            for (int i = 0; i < 8; ++i) acc[i] = __uint_as_float(u[i]);
+        for (int q = 0; q < 8; ++q) {
+            const int col = col0 + q * 4;
+            if (col >= p.d) break;
+            float4 v = make_float4(__uint_as_float(u[q * 4]), __uint_as_float(u[q * 4 + 1]),
+                                   __uint_as_float(u[q * 4 + 2]), __uint_as_float(u[q * 4 + 3]));
             if (p.sb2)
-                for (int s = 0; s < p.Ks; ++s)
-                    add_bf16x8(acc, __ldg(reinterpret_cast<const uint4*>(p.sb2 + (size_t)s * p.d + col)));
-            for (int j = 0; j < p.k; ++j) {
-                const int pos = p.slot_of[(size_t)t * p.k + j];
-                if (pos < 0 || pos >= p.S) { flag_error(p.err, ERR_INDEX_RANGE); continue; }
-                add_bf16x8(acc, __ldg(reinterpret_cast<const uint4*>(p.y_in + (size_t)pos * p.d + col)));
-            }
-            uint4 o;
-            o.x = pack_bf16(acc[0], acc[1]); o.y = pack_bf16(acc[2], acc[3]);
-            o.z = pack_bf16(acc[4], acc[5]); o.w = pack_bf16(acc[6], acc[7]);
-            *reinterpret_cast<uint4*>(orow + col) = o;
+                for (int s = 0; s < p.Ks; ++s) {
+                    const __nv_bfloat16* b = p.sb2 + (size_t)s * p.d + col;
+                    v.x += __bfloat162float(b[0]); v.y += __bfloat162float(b[1]);
+                    v.z += __bfloat162float(b[2]); v.w += __bfloat162float(b[3]);
+                }
+            *reinterpret_cast<float4*>(srow + col) = v;
         }
     }
 }
@@ -740,11 +677,11 @@ int router_splits(const Dims& D) {
     if (!tc_router_supported(D) || D.T == 0) return 1;
     const int mt = ceil_div(D.T, tc::BM);
     const int kbt = ceil_div(D.d, tc::BK);
-    if (mt > 32 || kbt < 8) return 1;
+    if (mt > 32 || kbt < 16) return 1;
     constexpr int kCtas = 148;                       // fixed so the workspace size never depends on the GPU
     const int want = ceil_div(kCtas, mt);
     const int per = ceil_div(kbt, want < kbt ? want : kbt);
-    return ceil_div(kbt, per < 2 ? 2 : per);
+    return ceil_div(kbt, per < 4 ? 4 : per);
 }
 
 cudaError_t launch_tc_router(const Dims& D, const void* x, const void* centroids, int32_t* idx, float* gate,
@@ -818,15 +755,13 @@ cudaError_t launch_tc_gemm2_routed(const Dims& D, const int32_t* offsets, const 
     return launch<GEMM2R, 8>(p, num_sms(), stream);
 }
 
-cudaError_t launch_tc_gemm2_shared(const Dims& D, const FfnWeights& Sh, const void* h_s, const void* y_sorted,
-                                   const int32_t* slot_of, void* out, uint32_t* err, cudaStream_t stream) {
+cudaError_t launch_tc_gemm2_shared(const Dims& D, const FfnWeights& Sh, const void* h_s, float* sout, uint32_t* err,
+                                   cudaStream_t stream) {
     using namespace tc;
     if (D.T == 0 || D.Ks == 0) return cudaSuccess;
     Params p = base_params(D, err);
     p.sb2 = (const __nv_bfloat16*)Sh.b2;
-    p.y_in = (const __nv_bfloat16*)y_sorted;
-    p.slot_of = slot_of;
-    p.out = (__nv_bfloat16*)out;
+    p.sout = sout;
     bool ok = make_map(&p.tmA[0], h_s, D.Is, D.T, D.Ks, BK, BM, true);
     ok &= make_map(&p.tmB[0], Sh.w2, D.Is, D.d, D.Ks, BK, 256, true);
     if (!ok) return cudaErrorInvalidValue;

@@ -42,9 +42,10 @@ cudaError_t launch_plan(const Dims& D, const int32_t* offsets, int32_t* tile_sta
 cudaError_t launch_gather(const Dims& D, const void* x, const int32_t* sorted_token, void* x_perm,
                           uint32_t* err, cudaStream_t stream);
 
-// out[t, :] = sum_j y_sorted[slot_of[t*k + j], :] in fp32, rounded once (no shared experts).
-cudaError_t launch_combine(const Dims& D, const void* y_sorted, const int32_t* slot_of, void* out,
-                           uint32_t* err, cudaStream_t stream);
+// out[t, :] = base[t, :] + sum_j y_sorted[slot_of[t*k + j], :] in fp32, rounded once; base is
+// the shared experts' fp32 output [T, d], or NULL when there are none.
+cudaError_t launch_combine(const Dims& D, const void* y_sorted, const int32_t* slot_of, const float* base,
+                           void* out, uint32_t* err, cudaStream_t stream);
 
 // ---- CUDA-core grouped FFN (fp32 layers) ----------------------------------------------
 struct FfnWeights {
@@ -89,11 +90,9 @@ cudaError_t launch_tc_gemm1(const Dims& D, const void* x, const void* x_perm, co
 cudaError_t launch_tc_gemm2_routed(const Dims& D, const int32_t* offsets, const int32_t* tile_start2,
                                    const float* sorted_gate, const FfnWeights& routed, const void* h_r,
                                    void* y_sorted, uint32_t* err, cudaStream_t stream);
-// shared GEMM2 (all K_s experts accumulated along K) whose epilogue adds the routed rows
-// of every token in pick order -> out
-cudaError_t launch_tc_gemm2_shared(const Dims& D, const FfnWeights& shared, const void* h_s,
-                                   const void* y_sorted, const int32_t* slot_of, void* out, uint32_t* err,
-                                   cudaStream_t stream);
+// shared GEMM2: all K_s experts accumulated along K, plus their b2 -> fp32 sout [T, d]
+cudaError_t launch_tc_gemm2_shared(const Dims& D, const FfnWeights& shared, const void* h_s, float* sout,
+                                   uint32_t* err, cudaStream_t stream);
 
 int num_sms();
 

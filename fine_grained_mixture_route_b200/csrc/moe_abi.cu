@@ -14,7 +14,7 @@ namespace {
 size_t al(size_t x) { return (x + 255) & ~(size_t)255; }
 
 struct Layout {
-    size_t err, hist, rpart, ts1, ts2, idx, gate, counts, offsets, stok, sgate, slot_of, xperm, hr, hs, y, total;
+    size_t err, hist, rpart, sout, ts1, ts2, idx, gate, counts, offsets, stok, sgate, slot_of, xperm, hr, hs, y, total;
 };
 
 Layout layout(const Dims& D) {
@@ -26,6 +26,7 @@ Layout layout(const Dims& D) {
     L.err = o; o += 256;
     L.hist = o; o += al((nblk ? nblk : 1) * D.E * 4);
     L.rpart = o; o += al(router_partial_bytes(D));
+    L.sout = o; o += (D.bf16 && D.Ks > 0) ? al((size_t)D.T * D.d * 4) : 0;
     L.ts1 = o; o += al((size_t)(D.E + D.Ks + 1) * 4);
     L.ts2 = o; o += al((size_t)(D.E + 1) * 4);
     L.idx = o; o += al(S * 4);
@@ -167,7 +168,9 @@ MOE_EXPORT int32_t moe_layer_launches(const moe_shape_t* shape) {
     n += 3;                                                         // histogram, scan, scatter
     n += 1;                                                         // tile tables
     if (D.bf16) n += 1;                                             // row gather
-    n += 3;                                                         // GEMM1, GEMM2, shared GEMM2 / combine
+    n += 2;                                                         // GEMM1, GEMM2
+    if (D.bf16 && D.Ks > 0) n += 2;                                 // shared GEMM2, combine
+    else n += 1;                                                    // combine (fused for fp32)
     return n;
 }
 
@@ -261,7 +264,7 @@ MOE_EXPORT moe_status_t moe_combine(const moe_shape_t* shape, const void* x, con
     cudaStream_t st = (cudaStream_t)stream;
     uint32_t* err = at<uint32_t>(ws, L.err);
     if (D.Ks == 0) {
-        MOE_CUDA(launch_combine(D, y_sorted, slot_of, out, err, st));
+        MOE_CUDA(launch_combine(D, y_sorted, slot_of, nullptr, out, err, st));
         return MOE_OK;
     }
     const FfnWeights Sh = to_ffn(shared);
@@ -271,7 +274,9 @@ MOE_EXPORT moe_status_t moe_combine(const moe_shape_t* shape, const void* x, con
         int32_t* ts1 = at<int32_t>(ws, L.ts1);
         MOE_CUDA(launch_plan(D, nullptr, ts1, at<int32_t>(ws, L.ts2), err, st));
         MOE_CUDA(launch_tc_gemm1(D, x, nullptr, nullptr, ts1, none, Sh, nullptr, hs, D.E, D.E + D.Ks, err, st));
-        MOE_CUDA(launch_tc_gemm2_shared(D, Sh, hs, y_sorted, slot_of, out, err, st));
+        float* sout = at<float>(ws, L.sout);
+        MOE_CUDA(launch_tc_gemm2_shared(D, Sh, hs, sout, err, st));
+        MOE_CUDA(launch_combine(D, y_sorted, slot_of, sout, out, err, st));
     } else {
         MOE_CUDA(launch_simt_gemm1(D, x, nullptr, nullptr, none, Sh, nullptr, hs, D.E, D.E + D.Ks, err, st));
         MOE_CUDA(launch_simt_gemm2_shared(D, Sh, hs, y_sorted, slot_of, out, err, st));
@@ -332,8 +337,10 @@ moe_status_t layer_forward_impl(const moe_shape_t* shape, const void* x, const v
         if (!mark(5)) return MOE_ERR_CUDA;
         MOE_CUDA(launch_tc_gemm2_routed(D, offsets, ts2, sgate, R, hr, y, err, st));
         if (!mark(6)) return MOE_ERR_CUDA;
-        if (D.Ks > 0) MOE_CUDA(launch_tc_gemm2_shared(D, Sh, hs, y, slot_of, out, err, st));
-        else MOE_CUDA(launch_combine(D, y, slot_of, out, err, st));
+        float* sout = D.Ks > 0 ? at<float>(ws, L.sout) : nullptr;
+        if (D.Ks > 0) MOE_CUDA(launch_tc_gemm2_shared(D, Sh, hs, sout, err, st));
+        if (!mark(7)) return MOE_ERR_CUDA;
+        MOE_CUDA(launch_combine(D, y, slot_of, sout, out, err, st));
     } else {
         if (!mark(4)) return MOE_ERR_CUDA;
         MOE_CUDA(launch_simt_gemm1(D, x, offsets, stok, R, Sh, hr, hs, 0, D.E + D.Ks, err, st));
@@ -341,9 +348,10 @@ moe_status_t layer_forward_impl(const moe_shape_t* shape, const void* x, const v
         MOE_CUDA(launch_simt_gemm2_routed(D, offsets, sgate, R, hr, y, err, st));
         if (!mark(6)) return MOE_ERR_CUDA;
         if (D.Ks > 0) MOE_CUDA(launch_simt_gemm2_shared(D, Sh, hs, y, slot_of, out, err, st));
-        else MOE_CUDA(launch_combine(D, y, slot_of, out, err, st));
+        else MOE_CUDA(launch_combine(D, y, slot_of, nullptr, out, err, st));
+        if (!mark(7)) return MOE_ERR_CUDA;
     }
-    if (!mark(7)) return MOE_ERR_CUDA;
+    if (!mark(8)) return MOE_ERR_CUDA;
     return MOE_OK;
 }
 

@@ -184,24 +184,54 @@ __global__ void gather_rows_kernel(const uint4* __restrict__ x, const int32_t* _
     }
 }
 
-// out[t] = sum_j y[slot_of[t*k + j]] (fp32 sum in ascending j, one rounding).  V elements
-// per thread step: 16-byte vectors when the row length allows, else single elements.
-template <typename T, int V>
-__global__ void combine_kernel(const T* __restrict__ y, const int32_t* __restrict__ slot_of, T* __restrict__ out,
-                               int Tn, int d, int k, long long S, uint32_t* err) {
+// out[t] = base[t] + sum_j y[slot_of[t*k + j]]: the shared experts' fp32 output (optional)
+// first, then the routed rows in ascending pick order, summed in fp32 and rounded once.  One
+// block per token: its slot rows are read as whole contiguous rows, V elements (16 bytes)
+// per thread step; with k <= KF all k row loads of a step are issued before they are summed.
+template <typename T, int V, int KF>
+__global__ void __launch_bounds__(128) combine_kernel(const T* __restrict__ y, const int32_t* __restrict__ slot_of,
+                                                      const float* __restrict__ base, T* __restrict__ out, int Tn,
+                                                      int d, int k, long long S, uint32_t* err) {
     struct alignas(sizeof(T) * V) Vec { T e[V]; };
+    __shared__ int sl[32];
     const int nv = d / V;
     for (int t = blockIdx.x; t < Tn; t += gridDim.x) {
+        __syncthreads();
+        if ((int)threadIdx.x < k) {
+            int p = slot_of[(size_t)t * k + threadIdx.x];
+            if (p < 0 || p >= S) { flag_error(err, ERR_INDEX_RANGE); p = -1; }
+            sl[threadIdx.x] = p;
+        }
+        __syncthreads();
         for (int v = threadIdx.x; v < nv; v += blockDim.x) {
             float acc[V];
+            if (base) {
 #pragma unroll
-            for (int i = 0; i < V; ++i) acc[i] = 0.f;
-            for (int j = 0; j < k; ++j) {
-                const int p = slot_of[(size_t)t * k + j];
-                if (p < 0 || p >= S) { flag_error(err, ERR_INDEX_RANGE); continue; }
-                const Vec raw = reinterpret_cast<const Vec*>(y + (size_t)p * d)[v];
+                for (int i = 0; i < V; ++i) acc[i] = base[(size_t)t * d + (size_t)v * V + i];
+            } else {
 #pragma unroll
-                for (int i = 0; i < V; ++i) acc[i] += to_f32(raw.e[i]);
+                for (int i = 0; i < V; ++i) acc[i] = 0.f;
+            }
+            if (KF > 0) {
+                Vec raw[KF > 0 ? KF : 1];
+#pragma unroll
+                for (int j = 0; j < KF; ++j) {
+                    if (j < k && sl[j] >= 0) raw[j] = reinterpret_cast<const Vec*>(y + (size_t)sl[j] * d)[v];
+                    else
+#pragma unroll
+                        for (int i = 0; i < V; ++i) raw[j].e[i] = from_f32<T>(0.f);
+                }
+#pragma unroll
+                for (int j = 0; j < KF; ++j)
+#pragma unroll
+                    for (int i = 0; i < V; ++i) acc[i] += to_f32(raw[j].e[i]);
+            } else {
+                for (int j = 0; j < k; ++j) {
+                    if (sl[j] < 0) continue;
+                    const Vec raw = reinterpret_cast<const Vec*>(y + (size_t)sl[j] * d)[v];
+#pragma unroll
+                    for (int i = 0; i < V; ++i) acc[i] += to_f32(raw.e[i]);
+                }
             }
             Vec o;
 #pragma unroll
@@ -250,22 +280,25 @@ cudaError_t launch_gather(const Dims& D, const void* x, const int32_t* sorted_to
     return cudaGetLastError();
 }
 
-cudaError_t launch_combine(const Dims& D, const void* y_sorted, const int32_t* slot_of, void* out, uint32_t* err,
-                           cudaStream_t stream) {
-    if (D.T == 0) return cudaSuccess;
-    const int blocks = D.T < 148 * 8 ? D.T : 148 * 8;
-    if (D.bf16 && D.d % 8 == 0)
-        combine_kernel<__nv_bfloat16, 8><<<blocks, 128, 0, stream>>>((const __nv_bfloat16*)y_sorted, slot_of,
-                                                                     (__nv_bfloat16*)out, D.T, D.d, D.k, D.slots(), err);
-    else if (D.bf16)
-        combine_kernel<__nv_bfloat16, 1><<<blocks, 128, 0, stream>>>((const __nv_bfloat16*)y_sorted, slot_of,
-                                                                     (__nv_bfloat16*)out, D.T, D.d, D.k, D.slots(), err);
-    else if (D.d % 4 == 0)
-        combine_kernel<float, 4><<<blocks, 128, 0, stream>>>((const float*)y_sorted, slot_of, (float*)out, D.T, D.d,
-                                                             D.k, D.slots(), err);
+template <typename T, int V>
+void combine_dispatch(const Dims& D, const void* y, const int32_t* slot_of, const float* base, void* out, uint32_t* err,
+                      int blocks, cudaStream_t stream) {
+    if (D.k <= 8)
+        combine_kernel<T, V, 8><<<blocks, 128, 0, stream>>>((const T*)y, slot_of, base, (T*)out, D.T, D.d, D.k,
+                                                            D.slots(), err);
     else
-        combine_kernel<float, 1><<<blocks, 128, 0, stream>>>((const float*)y_sorted, slot_of, (float*)out, D.T, D.d,
-                                                             D.k, D.slots(), err);
+        combine_kernel<T, V, 0><<<blocks, 128, 0, stream>>>((const T*)y, slot_of, base, (T*)out, D.T, D.d, D.k,
+                                                            D.slots(), err);
+}
+
+cudaError_t launch_combine(const Dims& D, const void* y_sorted, const int32_t* slot_of, const float* base, void* out,
+                           uint32_t* err, cudaStream_t stream) {
+    if (D.T == 0) return cudaSuccess;
+    const int blocks = D.T < 148 * 16 ? D.T : 148 * 16;
+    if (D.bf16 && D.d % 8 == 0) combine_dispatch<__nv_bfloat16, 8>(D, y_sorted, slot_of, base, out, err, blocks, stream);
+    else if (D.bf16) combine_dispatch<__nv_bfloat16, 1>(D, y_sorted, slot_of, base, out, err, blocks, stream);
+    else if (D.d % 4 == 0) combine_dispatch<float, 4>(D, y_sorted, slot_of, base, out, err, blocks, stream);
+    else combine_dispatch<float, 1>(D, y_sorted, slot_of, base, out, err, blocks, stream);
     return cudaGetLastError();
 }
 

@@ -109,23 +109,35 @@ router_simt_kernel(const T* __restrict__ x, const T* __restrict__ cen, int32_t* 
 
 
 // Split-K router, last step: z = sum of the per-split partial logits in ascending split order
-// (deterministic), then the same softmax / top-k as above.  One warp per token.
-constexpr int FIN_WARPS = 8;
-__global__ void __launch_bounds__(FIN_WARPS * 32)
+// (deterministic), then the same softmax / top-k as above.  A block sums FIN_TOK tokens with
+// coalesced float4 loads (consecutive threads read consecutive experts of one split row),
+// then one warp per token ranks them.
+constexpr int FIN_TOK = 8;
+__global__ void __launch_bounds__(FIN_TOK * 32)
 router_finish_kernel(const float* __restrict__ partial, int nsplit, int Tn, int E, int k, int32_t* __restrict__ idx_out,
                      float* __restrict__ gate_out) {
     extern __shared__ float zs[];
-    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    const int t = blockIdx.x * FIN_WARPS + warp;
-    if (t >= Tn) return;
-    float* zr = zs + warp * E;
-    for (int e = lane; e < E; e += 32) {
-        float v = 0.f;
-        for (int s = 0; s < nsplit; ++s) v += partial[((size_t)s * Tn + t) * E + e];
-        zr[e] = v;
+    const int t0 = blockIdx.x * FIN_TOK;
+    const int E4 = E / 4;
+    const size_t stride4 = (size_t)Tn * E4;                 // float4s between consecutive splits
+    for (int c = threadIdx.x; c < FIN_TOK * E4; c += blockDim.x) {
+        const int tt = c / E4, e4 = c % E4;
+        const int t = t0 + tt;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (t < Tn) {
+            const float4* src = reinterpret_cast<const float4*>(partial) + (size_t)t * E4 + e4;
+#pragma unroll 4
+            for (int s = 0; s < nsplit; ++s) {
+                const float4 v = src[(size_t)s * stride4];
+                acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+            }
+        }
+        reinterpret_cast<float4*>(zs + tt * E)[e4] = acc;
     }
-    __syncwarp();
-    warp_softmax_topk(zr, E, k, lane, idx_out + (size_t)t * k, gate_out + (size_t)t * k);
+    __syncthreads();
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const int t = t0 + warp;
+    if (t < Tn) warp_softmax_topk(zs + warp * E, E, k, lane, idx_out + (size_t)t * k, gate_out + (size_t)t * k);
 }
 
 }  // namespace
@@ -150,9 +162,9 @@ cudaError_t launch_router_simt(const Dims& D, const void* x, const void* centroi
 
 cudaError_t launch_router_finish(const Dims& D, const float* partial, int nsplit, int32_t* idx, float* gate,
                                  cudaStream_t stream) {
-    const int blocks = ceil_div(D.T, FIN_WARPS);
-    const size_t smem = sizeof(float) * FIN_WARPS * D.E;
-    router_finish_kernel<<<blocks, FIN_WARPS * 32, smem, stream>>>(partial, nsplit, D.T, D.E, D.k, idx, gate);
+    const int blocks = ceil_div(D.T, FIN_TOK);
+    const size_t smem = sizeof(float) * FIN_TOK * D.E;
+    router_finish_kernel<<<blocks, FIN_TOK * 32, smem, stream>>>(partial, nsplit, D.T, D.E, D.k, idx, gate);
     return cudaGetLastError();
 }
 
