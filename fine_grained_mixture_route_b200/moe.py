@@ -239,3 +239,55 @@ class MoELayer:
         shape = shape_of(x, self.centroids, self.routed, self.top_k, self.shared)
         return layer_forward(shape, x, self.centroids, self.routed, self.shared, self.ws, out, idx, gate, counts,
                              stream)
+
+
+class HostPipeline:
+    """The layer over batches that live in pinned host memory, with the copies overlapped.
+
+    Batch i is copied host-to-device on one stream, the layer runs on a second, and the result
+    is copied device-to-host on a third; the copy-in of batch i+1 and the copy-out of batch
+    i-1 run while batch i is computed.  Two device buffers for input and output alternate, so
+    memory use is fixed.  Every batch still crosses PCIe both ways.
+    """
+
+    def __init__(self, shape: MoeShape, centroids, routed: Dict, shared: Optional[Dict], ws, device=None):
+        self.shape, self.centroids, self.routed, self.shared, self.ws = shape, centroids, routed, shared, ws
+        dev = centroids.device if device is None else device
+        T, d = shape.T, shape.d
+        self.xd = [torch.empty((T, d), dtype=centroids.dtype, device=dev) for _ in range(2)]
+        self.od = [torch.empty((T, d), dtype=centroids.dtype, device=dev) for _ in range(2)]
+        self.s_in, self.s_comp, self.s_out = (torch.cuda.Stream(dev) for _ in range(3))
+        self.in_done = [torch.cuda.Event() for _ in range(2)]
+        self.comp_done = [torch.cuda.Event() for _ in range(2)]
+        self.out_done = [torch.cuda.Event() for _ in range(2)]
+        for e in self.comp_done + self.out_done:
+            e.record(torch.cuda.current_stream(dev))
+
+    def run(self, x_host, out_host, start_event=None, stop_event=None):
+        """x_host / out_host: equal-length lists of pinned CPU tensors [T, d].  Optional
+        timing events are recorded before the first copy-in and after the last copy-out."""
+        if start_event is not None:
+            start_event.record(self.s_in)
+            self.s_comp.wait_event(start_event)
+            self.s_out.wait_event(start_event)
+        for i, (xh, oh) in enumerate(zip(x_host, out_host)):
+            b = i & 1
+            with torch.cuda.stream(self.s_in):
+                self.s_in.wait_event(self.comp_done[b])          # layer of batch i-2 has read xd[b]
+                self.xd[b].copy_(xh, non_blocking=True)
+                self.in_done[b].record(self.s_in)
+            with torch.cuda.stream(self.s_comp):
+                self.s_comp.wait_event(self.in_done[b])
+                self.s_comp.wait_event(self.out_done[b])         # copy-out of batch i-2 has read od[b]
+                layer_forward(self.shape, self.xd[b], self.centroids, self.routed, self.shared, self.ws,
+                              out=self.od[b], stream=self.s_comp)
+                self.comp_done[b].record(self.s_comp)
+            with torch.cuda.stream(self.s_out):
+                self.s_out.wait_event(self.comp_done[b])
+                oh.copy_(self.od[b], non_blocking=True)
+                self.out_done[b].record(self.s_out)
+        if stop_event is not None:
+            self.s_in.wait_event(self.out_done[(len(x_host) - 1) & 1])
+            self.s_out.wait_event(self.in_done[(len(x_host) - 1) & 1])
+            stop_event.record(self.s_out)
+        return out_host

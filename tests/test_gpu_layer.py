@@ -164,3 +164,22 @@ def test_bad_expert_index_is_flagged():
         moe.check_device_error(ws)
     assert ei.value.status == moe.MOE_ERR_INTERNAL and ei.value.detail & 1
     moe.check_device_error(ws)          # cleared by the previous check
+
+
+def test_host_pipeline_matches_device_calls():
+    """moe.HostPipeline (pinned host batches, copies overlapped with the layer) returns, for
+    every batch, exactly what a plain layer_forward on the device returns."""
+    cfg = W.scaled(W.CONFIGS["small"], T=500, d=256, n_experts=32, top_k=4, inter=128, inter_shared=128)
+    L = W.make_layer(cfg, "cuda", seed=11)
+    shape = moe.shape_of(L["x"], L["centroids"], L["routed"], cfg.top_k, L["shared"])
+    ws = moe.new_workspace(shape)
+    xs = [W.make_x(cfg, "cuda", seed=20 + i) for i in range(5)]
+    want = [moe.layer_forward(shape, x, L["centroids"], L["routed"], L["shared"], ws).cpu() for x in xs]
+    xh = [x.cpu().pin_memory() for x in xs]
+    oh = [torch.empty_like(h).pin_memory() for h in xh]
+    pipe = moe.HostPipeline(shape, L["centroids"], L["routed"], L["shared"], ws)
+    pipe.run(xh, oh)
+    torch.cuda.synchronize()
+    moe.check_device_error(ws)
+    for w, o in zip(want, oh):
+        assert torch.equal(w, o)
