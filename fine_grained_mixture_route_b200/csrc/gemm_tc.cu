@@ -6,8 +6,8 @@
 //           ("《DeepSeekMoE》深度解读报告" §3.1, Eq. 3-5 in prose).
 //   GEMM1   [x_e] [w1_e | w3_e]^T for 128 rows x (128 + 128) columns with bias and SwiGLU in
 //           the epilogue: h = silu(x w1^T + b1) * (x w3^T + b3) (the `Expert` module of
-//           "DeepSeek MoE模型优化与未来演进及字节超稀疏内存技术").  Routed groups gather
-//           their token rows straight from x with tile::gather4; shared groups read x tiles.
+//           "DeepSeek MoE模型优化与未来演进及字节超稀疏内存技术").  Routed groups read the
+//           expert's gathered rows, shared groups read x itself.
 //   GEMM2R  routed w2 contraction; the epilogue adds b2 and scales by the gate: the gate
 //           multiplies the whole expert output.
 //   GEMM2S  the K_s shared experts' w2 contractions accumulated along K in one accumulator;
@@ -57,7 +57,6 @@ struct Params {
     CUtensorMap tmB[4];
     const int32_t* tile_start;
     const int32_t* offsets;
-    const int32_t* sorted_token;   // GEMM1: token of each grouped row (gathered from x)
     int g_begin, g_end;
     int T, d, E, I, Is, k, Ks;
     int n_mma;                 // MMA N (256, or N_m for the router)
@@ -133,16 +132,6 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
         "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(
             dst),
         "l"((unsigned long long)map), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
-        : "memory");
-}
-// Four rows (y0..y3) of `box_inner` elements starting at column c0 of a 2-D map whose box is
-// one row high; the rows land back to back at dst (4 x 128 bytes for a 64-element bf16 box).
-__device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap* map, uint32_t bar, int c0, int y0, int y1,
-                                            int y2, int y3) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(dst),
-        "l"((unsigned long long)map), "r"(bar), "r"(c0), "r"(y0), "r"(y1), "r"(y2), "r"(y3)
         : "memory");
 }
 __device__ __forceinline__ void prefetch_map(const CUtensorMap* map) {
@@ -498,44 +487,22 @@ __global__ void __launch_bounds__(THREADS, 1) moe_tc_kernel(const __grid_constan
 
     if (warp == 0) {
         // ------------------------------------------------------------------ TMA producer
-        // Lane 0 waits for free stages and loads the weight tiles; for routed GEMM1 tiles every
-        // lane then gathers 4 of the 128 token rows straight from x (tile::gather4, 4 rows of
-        // 128 bytes per instruction), so no permuted copy of x is ever written.
-        if (lane == 0 && (MODE != GEMM1 || p.g_begin < p.E)) {   // maps that exist in this launch
+        if (lane == 0) {
             prefetch_map(&p.tmA[0]);
             prefetch_map(&p.tmB[0]);
-        }
-        int stage = 0;
-        uint32_t phase = 0;
-        int last_parity[STAGES];
+            int stage = 0;
+            uint32_t phase = 0;
+            int last_parity[STAGES];
 #pragma unroll
-        for (int s = 0; s < STAGES; ++s) last_parity[s] = -1;
-        bool ok = true;
-        for (int t = blockIdx.x; ok && t < ntiles; t += gridDim.x) {
-            const Tile x = decode<MODE>(p, t);
-            const bool gather = MODE == GEMM1 && x.g < p.E;
-            int grow[4] = {0, 0, 0, 0};
-            if (gather) {
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const int r = x.m0 + lane * 4 + q;       // row of the group; past its end: any row
-                    int tok = 0;
-                    if (r < x.rows) {
-                        tok = p.sorted_token[x.row0 + r];
-                        if (tok < 0 || tok >= p.T) { flag_error(p.err, ERR_INDEX_RANGE); tok = 0; }
-                    }
-                    grow[q] = tok;
-                }
-            }
-            for (int kk_ = 0; kk_ < x.num_kb; ++kk_) {
-                const int kb = x.kb0 + kk_;
-                int w = 1;
-                if (lane == 0) w = mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, p.err) ? 1 : 0;
-                w = __shfl_sync(0xffffffffu, w, 0);
-                if (!w) { ok = false; break; }
-                const uint32_t fb = full_bar(stage);
-                const uint32_t a_dst = sA + stage * A_BYTES, b_dst = sB + stage * B_BYTES;
-                if (lane == 0) {
+            for (int s = 0; s < STAGES; ++s) last_parity[s] = -1;
+            bool ok = true;
+            for (int t = blockIdx.x; ok && t < ntiles; t += gridDim.x) {
+                const Tile x = decode<MODE>(p, t);
+                for (int kk_ = 0; kk_ < x.num_kb; ++kk_) {
+                    const int kb = x.kb0 + kk_;
+                    if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, p.err)) { ok = false; break; }
+                    const uint32_t fb = full_bar(stage);
+                    const uint32_t a_dst = sA + stage * A_BYTES, b_dst = sB + stage * B_BYTES;
                     if (MODE == ROUTER || MODE == ROUTERP) {
                         mbar_expect_tx(fb, A_BYTES + p.n_mma * BK * 2);
                         tma_load_2d(a_dst, &p.tmA[0], fb, kb * BK, x.m0);
@@ -544,7 +511,7 @@ __global__ void __launch_bounds__(THREADS, 1) moe_tc_kernel(const __grid_constan
                         mbar_expect_tx(fb, A_BYTES + B_BYTES);
                         const bool shared = x.g >= p.E;
                         const int e = shared ? x.g - p.E : x.g;
-                        if (shared) tma_load_2d(a_dst, &p.tmA[1], fb, kb * BK, x.m0);
+                        tma_load_2d(a_dst, &p.tmA[shared ? 1 : 0], fb, kb * BK, x.row0 + x.m0);
                         tma_load_3d(b_dst, &p.tmB[shared ? 2 : 0], fb, kb * BK, x.n0, e);
                         tma_load_3d(b_dst + B_BYTES / 2, &p.tmB[shared ? 3 : 1], fb, kb * BK, x.n0, e);
                     } else if (MODE == GEMM2R) {
@@ -558,22 +525,15 @@ __global__ void __launch_bounds__(THREADS, 1) moe_tc_kernel(const __grid_constan
                         tma_load_3d(a_dst, &p.tmA[0], fb, kk * BK, x.m0, s);
                         tma_load_3d(b_dst, &p.tmB[0], fb, kk * BK, x.n0, s);
                     }
+                    last_parity[stage] = (int)phase;
+                    if (++stage == STAGES) { stage = 0; phase ^= 1u; }
                 }
-                if (gather) {
-                    __syncwarp();                                   // expect_tx before the row copies
-                    tma_gather4(a_dst + lane * 512, &p.tmA[0], fb, kb * BK, grow[0], grow[1], grow[2], grow[3]);
-                }
-                last_parity[stage] = (int)phase;
-                if (++stage == STAGES) { stage = 0; phase ^= 1u; }
             }
-        }
-        // drain: every copy this warp issued has landed before the CTA may exit
-        if (lane == 0) {
+            // drain: every copy this thread issued has landed before the CTA may exit
 #pragma unroll
             for (int s = 0; s < STAGES; ++s)
                 if (last_parity[s] >= 0) mbar_wait(full_bar(s), (uint32_t)last_parity[s], abort_flag, p.err, false);
         }
-        __syncwarp();
     } else if (warp == 1) {
         // ------------------------------------------------------------------ MMA issuer
         if (lane == 0) {
@@ -750,7 +710,7 @@ cudaError_t launch_tc_router(const Dims& D, const void* x, const void* centroids
     return D.k <= 8 ? launch<ROUTER, 8>(p, grid, stream) : launch<ROUTER, 32>(p, grid, stream);
 }
 
-cudaError_t launch_tc_gemm1(const Dims& D, const void* x, const int32_t* sorted_token, const int32_t* offsets,
+cudaError_t launch_tc_gemm1(const Dims& D, const void* x, const void* x_perm, const int32_t* offsets,
                             const int32_t* tile_start1, const FfnWeights& R, const FfnWeights& Sh, void* h_r, void* h_s,
                             int g_begin, int g_end, uint32_t* err, cudaStream_t stream) {
     using namespace tc;
@@ -758,7 +718,6 @@ cudaError_t launch_tc_gemm1(const Dims& D, const void* x, const int32_t* sorted_
     Params p = base_params(D, err);
     p.tile_start = tile_start1;
     p.offsets = offsets;
-    p.sorted_token = sorted_token;
     p.g_begin = g_begin;
     p.g_end = g_end;
     p.b1 = (const __nv_bfloat16*)R.b1; p.b3 = (const __nv_bfloat16*)R.b3;
@@ -766,7 +725,7 @@ cudaError_t launch_tc_gemm1(const Dims& D, const void* x, const int32_t* sorted_
     p.h_r = (__nv_bfloat16*)h_r; p.h_s = (__nv_bfloat16*)h_s;
     bool ok = true;
     if (g_begin < D.E) {
-        ok &= make_map(&p.tmA[0], x, D.d, D.T, 1, BK, 1, false);        // one-row box for tile::gather4
+        ok &= make_map(&p.tmA[0], x_perm, D.d, (uint64_t)D.slots(), 1, BK, BM, false);
         ok &= make_map(&p.tmB[0], R.w1, D.d, D.I, D.E, BK, 128, true);
         ok &= make_map(&p.tmB[1], R.w3, D.d, D.I, D.E, BK, 128, true);
     }

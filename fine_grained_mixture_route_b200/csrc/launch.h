@@ -38,6 +38,10 @@ cudaError_t launch_permute(const Dims& D, const int32_t* idx, const float* gate,
 cudaError_t launch_plan(const Dims& D, const int32_t* offsets, int32_t* tile_start1, int32_t* tile_start2,
                         uint32_t* err, cudaStream_t stream);
 
+// x_perm[p, :] = x[sorted_token[p], :] (bf16 rows, 16-byte vectors).
+cudaError_t launch_gather(const Dims& D, const void* x, const int32_t* sorted_token, void* x_perm,
+                          uint32_t* err, cudaStream_t stream);
+
 // out[t, :] = base[t, :] + sum_j y_sorted[slot_of[t*k + j], :] in fp32, rounded once; base is
 // the shared experts' fp32 output [T, d], or NULL when there are none.
 cudaError_t launch_combine(const Dims& D, const void* y_sorted, const int32_t* slot_of, const float* base,
@@ -78,9 +82,8 @@ cudaError_t launch_tc_router(const Dims& D, const void* x, const void* centroids
                              float* partial, uint32_t* err, cudaStream_t stream);
 cudaError_t launch_router_finish(const Dims& D, const float* partial, int nsplit, int32_t* idx, float* gate,
                                  cudaStream_t stream);
-// GEMM1 + SwiGLU over groups [g_begin, g_end): routed A rows gathered from x by sorted_token
-// inside the kernel; shared groups read x directly.
-cudaError_t launch_tc_gemm1(const Dims& D, const void* x, const int32_t* sorted_token, const int32_t* offsets,
+// GEMM1 + SwiGLU over groups [g_begin, g_end): A rows from x_perm (routed) or x (shared).
+cudaError_t launch_tc_gemm1(const Dims& D, const void* x, const void* x_perm, const int32_t* offsets,
                             const int32_t* tile_start1, const FfnWeights& routed, const FfnWeights& shared,
                             void* h_r, void* h_s, int g_begin, int g_end, uint32_t* err, cudaStream_t stream);
 // routed GEMM2 with the gate (and b2) applied in the epilogue -> y_sorted

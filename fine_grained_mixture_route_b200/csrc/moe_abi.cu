@@ -14,7 +14,7 @@ namespace {
 size_t al(size_t x) { return (x + 255) & ~(size_t)255; }
 
 struct Layout {
-    size_t err, hist, rpart, sout, ts1, ts2, idx, gate, counts, offsets, stok, sgate, slot_of, hr, hs, y, total;
+    size_t err, hist, rpart, sout, ts1, ts2, idx, gate, counts, offsets, stok, sgate, slot_of, xperm, hr, hs, y, total;
 };
 
 Layout layout(const Dims& D) {
@@ -36,6 +36,7 @@ Layout layout(const Dims& D) {
     L.stok = o; o += al(S * 4);
     L.sgate = o; o += al(S * 4);
     L.slot_of = o; o += al(S * 4);
+    L.xperm = o; o += D.bf16 ? al(S * D.d * esz) : 0;
     L.hr = o; o += al(S * D.I * esz);
     L.hs = o; o += al((size_t)D.Ks * D.T * (D.Ks ? D.Is : 0) * esz);
     L.y = o; o += al(S * D.d * esz);
@@ -119,8 +120,10 @@ moe_status_t do_expert_ffn(const Dims& D, const Layout& L, void* ws, const void*
     int32_t* ts2 = at<int32_t>(ws, L.ts2);
     if (!plan_done) MOE_CUDA(launch_plan(D, offsets, ts1, ts2, err, st));
     if (D.bf16) {
+        void* xp = at<void>(ws, L.xperm);
+        MOE_CUDA(launch_gather(D, x, stok, xp, err, st));
         FfnWeights none = {nullptr, nullptr, nullptr, nullptr, nullptr, nullptr};
-        MOE_CUDA(launch_tc_gemm1(D, x, stok, offsets, ts1, R, none, at<void>(ws, L.hr), nullptr, 0, D.E, err, st));
+        MOE_CUDA(launch_tc_gemm1(D, x, xp, offsets, ts1, R, none, at<void>(ws, L.hr), nullptr, 0, D.E, err, st));
         MOE_CUDA(launch_tc_gemm2_routed(D, offsets, ts2, sgate, R, at<void>(ws, L.hr), y, err, st));
     } else {
         FfnWeights none = {nullptr, nullptr, nullptr, nullptr, nullptr, nullptr};
@@ -164,6 +167,7 @@ MOE_EXPORT int32_t moe_layer_launches(const moe_shape_t* shape) {
     else n += 1;
     n += 3;                                                         // histogram, scan, scatter
     n += 1;                                                         // tile tables
+    if (D.bf16) n += 1;                                             // row gather
     n += 2;                                                         // GEMM1, GEMM2
     if (D.bf16 && D.Ks > 0) n += 2;                                 // shared GEMM2, combine
     else n += 1;                                                    // combine (fused for fp32)
@@ -326,24 +330,28 @@ moe_status_t layer_forward_impl(const moe_shape_t* shape, const void* x, const v
     MOE_CUDA(launch_plan(D, offsets, ts1, ts2, err, st));
     if (!mark(3)) return MOE_ERR_CUDA;
     if (D.bf16) {
-        MOE_CUDA(launch_tc_gemm1(D, x, stok, offsets, ts1, R, Sh, hr, hs, 0, D.E + D.Ks, err, st));
+        void* xp = at<void>(ws, L.xperm);
+        MOE_CUDA(launch_gather(D, x, stok, xp, err, st));
         if (!mark(4)) return MOE_ERR_CUDA;
-        MOE_CUDA(launch_tc_gemm2_routed(D, offsets, ts2, sgate, R, hr, y, err, st));
+        MOE_CUDA(launch_tc_gemm1(D, x, xp, offsets, ts1, R, Sh, hr, hs, 0, D.E + D.Ks, err, st));
         if (!mark(5)) return MOE_ERR_CUDA;
+        MOE_CUDA(launch_tc_gemm2_routed(D, offsets, ts2, sgate, R, hr, y, err, st));
+        if (!mark(6)) return MOE_ERR_CUDA;
         float* sout = D.Ks > 0 ? at<float>(ws, L.sout) : nullptr;
         if (D.Ks > 0) MOE_CUDA(launch_tc_gemm2_shared(D, Sh, hs, sout, err, st));
-        if (!mark(6)) return MOE_ERR_CUDA;
+        if (!mark(7)) return MOE_ERR_CUDA;
         MOE_CUDA(launch_combine(D, y, slot_of, sout, out, err, st));
     } else {
-        MOE_CUDA(launch_simt_gemm1(D, x, offsets, stok, R, Sh, hr, hs, 0, D.E + D.Ks, err, st));
         if (!mark(4)) return MOE_ERR_CUDA;
-        MOE_CUDA(launch_simt_gemm2_routed(D, offsets, sgate, R, hr, y, err, st));
+        MOE_CUDA(launch_simt_gemm1(D, x, offsets, stok, R, Sh, hr, hs, 0, D.E + D.Ks, err, st));
         if (!mark(5)) return MOE_ERR_CUDA;
+        MOE_CUDA(launch_simt_gemm2_routed(D, offsets, sgate, R, hr, y, err, st));
+        if (!mark(6)) return MOE_ERR_CUDA;
         if (D.Ks > 0) MOE_CUDA(launch_simt_gemm2_shared(D, Sh, hs, y, slot_of, out, err, st));
         else MOE_CUDA(launch_combine(D, y, slot_of, nullptr, out, err, st));
-        if (!mark(6)) return MOE_ERR_CUDA;
+        if (!mark(7)) return MOE_ERR_CUDA;
     }
-    if (!mark(7)) return MOE_ERR_CUDA;
+    if (!mark(8)) return MOE_ERR_CUDA;
     return MOE_OK;
 }
 

@@ -1,4 +1,4 @@
-// Per-expert token lists, the grouped GEMMs' tile tables and the combine.
+// Per-expert token lists, the grouped GEMMs' tile tables, the row gather and the combine.
 //
 // The grouping follows the "top-k indices first, then gather the tokens of each expert"
 // step of the DeepSeek-V2 explainer (eliteato.com/news/32734, §3.1 and §3.3): the T*N_r
@@ -171,6 +171,19 @@ __global__ void plan_kernel(const int32_t* __restrict__ offsets, long long S, in
     }
 }
 
+// x_perm[p] = x[sorted_token[p]]: one row per block-iteration, 16-byte vectors
+__global__ void gather_rows_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ sorted_token,
+                                   uint4* __restrict__ xp, long long S, int T, int vec_per_row, uint32_t* err) {
+    for (long long p = blockIdx.x; p < S; p += gridDim.x) {
+        const int t = sorted_token[p];
+        const bool ok = t >= 0 && t < T;
+        if (!ok && threadIdx.x == 0) flag_error(err, ERR_INDEX_RANGE);
+        const uint4* src = x + (size_t)(ok ? t : 0) * vec_per_row;
+        uint4* dst = xp + (size_t)p * vec_per_row;
+        for (int v = threadIdx.x; v < vec_per_row; v += blockDim.x) dst[v] = ok ? __ldg(src + v) : make_uint4(0, 0, 0, 0);
+    }
+}
+
 // out[t] = base[t] + sum_j y[slot_of[t*k + j]]: the shared experts' fp32 output (optional)
 // first, then the routed rows in ascending pick order, summed in fp32 and rounded once.  One
 // block per token: its slot rows are read as whole contiguous rows, V elements (16 bytes)
@@ -253,6 +266,17 @@ cudaError_t launch_plan(const Dims& D, const int32_t* offsets, int32_t* tile_sta
     const size_t smem = sizeof(int) * ((size_t)G + 1 + D.E + 1 + 32);
     plan_kernel<<<1, SCAN_THREADS, smem, stream>>>(offsets, D.slots(), D.T, D.d, D.E, D.I, D.Ks, D.Ks > 0 ? D.Is : 1,
                                                    tile_start1, tile_start2, err);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_gather(const Dims& D, const void* x, const int32_t* sorted_token, void* x_perm, uint32_t* err,
+                          cudaStream_t stream) {
+    const long long S = D.slots();
+    if (S == 0) return cudaSuccess;
+    const int esz = D.bf16 ? 2 : 4;
+    const int vec = D.d * esz / 16;
+    const long long blocks = S < 148LL * 32 ? S : 148LL * 32;
+    gather_rows_kernel<<<(int)blocks, 128, 0, stream>>>((const uint4*)x, sorted_token, (uint4*)x_perm, S, D.T, vec, err);
     return cudaGetLastError();
 }
 

@@ -185,13 +185,13 @@ moe_status_t moe_layer_forward(const moe_shape_t* shape, const void* x, const vo
  * `stream` before stage i and stage_events[MOE_NUM_STAGES] after the last stage, so that
  * cudaEventElapsedTime between neighbours gives each stage's device time.  Stages, in order:
  *   0 router (scores, softmax, top-k)      1 grouping (histogram, scan, scatter)
- *   2 tile tables of the grouped GEMMs     3 GEMM1 + SwiGLU (routed rows gathered in-kernel)
- *   4 routed GEMM2 with gates              5 shared GEMM2 (bf16; fp32 layers fuse it with
- *                                            the combine here)
- *   6 combine (bf16; empty for fp32 layers)
+ *   2 tile tables of the grouped GEMMs     3 row gather of the routed tokens (bf16 only)
+ *   4 GEMM1 + SwiGLU (routed and shared)   5 routed GEMM2 with gates
+ *   6 shared GEMM2 (bf16; fp32 layers fuse it with the combine here)
+ *   7 combine (bf16; empty for fp32 layers)
  * n_events must be MOE_NUM_STAGES + 1; MOE_ERR_INVALID_ARG otherwise.
  */
-#define MOE_NUM_STAGES 7
+#define MOE_NUM_STAGES 8
 moe_status_t moe_layer_forward_timed(const moe_shape_t* shape, const void* x, const void* centroids,
                                      const moe_ffn_weights_t* routed, const moe_ffn_weights_t* shared,
                                      void* out, int32_t* topk_idx_out, float* topk_gate_out,

@@ -55,10 +55,10 @@ def _shape(**kw):
 def test_workspace_bytes(lib):
     n = moe.workspace_bytes(_shape())
     S, d, I = 256 * 8, 7168, 2048
-    # h_r, Y (bf16), the shared hidden states and the fp32 shared output at least
-    assert n >= 2 * (S * I + S * d + 256 * 2048) + 4 * 256 * d
+    # x_perm, h_r, Y (bf16) and the shared hidden states at least
+    assert n >= 2 * (S * d + S * I + S * d + 256 * 2048)
     # ... plus the split-K router's fp32 partial logits (at most 148 CTAs x 128 tokens x N_m)
-    assert n < 2 * (S * I + S * d + 256 * 2048) + 4 * 256 * d + 4 * 1024 * 1024 + 148 * 128 * 256 * 4
+    assert n < 2 * (S * d + S * I + S * d + 256 * 2048) + 4 * 1024 * 1024 + 148 * 128 * 256 * 4
     assert moe.workspace_bytes(_shape(T=512)) > n
     assert moe.workspace_bytes(_shape(T=0)) > 0
     # fp32 layers keep no gathered copy of x
@@ -71,9 +71,9 @@ def test_workspace_bytes(lib):
 
 
 def test_launch_count(lib):
-    assert moe.layer_launches(_shape()) == 10          # split-K router at T=256: scores + finish
-    assert moe.layer_launches(_shape(T=16384)) == 9
-    assert moe.layer_launches(_shape(T=16384, n_shared=0)) == 8
+    assert moe.layer_launches(_shape()) == 11          # split-K router at T=256: scores + finish
+    assert moe.layer_launches(_shape(T=16384)) == 10
+    assert moe.layer_launches(_shape(T=16384, n_shared=0)) == 9
     assert moe.layer_launches(_shape(T=128, d=256, n_experts=16, inter=64, inter_shared=64, top_k=4,
                                      dtype=moe.MOE_F32)) == 8
     assert moe.layer_launches(_shape(T=0)) == 0
