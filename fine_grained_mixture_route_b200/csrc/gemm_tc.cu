@@ -38,19 +38,30 @@
 namespace moe {
 namespace tc {
 
-constexpr int BM = 128;                  // rows per tile (TMEM lanes)
+constexpr int BM = 128;                  // rows per CTA (TMEM lanes)
 constexpr int BK = 64;                   // K per stage: 64 bf16 = one 128-byte swizzle row
-constexpr int STAGES = 4;
 constexpr int A_BYTES = BM * BK * 2;     // 16 KB
-constexpr int B_BYTES = 256 * BK * 2;    // 32 KB (N <= 256)
 constexpr int THREADS = 320;              // warp 0 TMA, warp 1 MMA, warps 2-9 epilogue
 constexpr int EPI_WARPS = 8;
 constexpr int TMEM_COLS = 512;
 constexpr int ACC_COLS = 256;
-constexpr int SMEM_BYTES = 1024 /*align slack*/ + STAGES * (A_BYTES + B_BYTES) + 256 /*barriers*/;
+constexpr int RING_BYTES = 192 * 1024;   // shared-memory ring (stages x (A + B))
+constexpr int SMEM_BYTES = 1024 /*align slack*/ + RING_BYTES + 256 /*barriers*/;
 constexpr unsigned long long WAIT_NS = 4000000000ull;
+constexpr uint32_t PEER_BIT_MASK = 0xFEFFFFFFu;   // shared::cluster address of CTA rank 0 of a pair
 
 enum Mode : int { ROUTER = 0, GEMM1 = 1, GEMM2R = 2, GEMM2S = 3, ROUTERP = 4 };
+
+// The expert GEMMs run on CTA pairs (cta_group::2): a 256-row tile, each CTA holding 128 rows
+// of A, half of the 256 B rows and its 128 x 256 slice of the accumulator, so each SM loads
+// 32 KB per K stage instead of 48 KB.  The router modes run on single CTAs.
+template <int MODE>
+struct Cfg {
+    static constexpr bool PAIR = MODE == GEMM1 || MODE == GEMM2R || MODE == GEMM2S;
+    static constexpr int TM = PAIR ? 2 * BM : BM;                 // rows per tile
+    static constexpr int B_BYTES = (PAIR ? 128 : 256) * BK * 2;   // B rows held by one CTA
+    static constexpr int STAGES = RING_BYTES / (A_BYTES + B_BYTES);
+};
 
 struct Params {
     CUtensorMap tmA[2];
@@ -193,6 +204,62 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
     return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// ---- CTA-pair (cta_group::2) forms
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// TMA load into this CTA's shared memory whose completion is counted on the pair leader's
+// barrier (the peer bit of the barrier address cleared).
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map, uint32_t bar, int c0, int c1) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::"r"(
+            dst),
+        "l"((unsigned long long)map), "r"(bar & PEER_BIT_MASK), "r"(c0), "r"(c1)
+        : "memory");
+}
+__device__ __forceinline__ void tma_load_3d_pair(uint32_t dst, const CUtensorMap* map, uint32_t bar, int c0, int c1,
+                                                 int c2) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(
+            dst),
+        "l"((unsigned long long)map), "r"(bar & PEER_BIT_MASK), "r"(c0), "r"(c1), "r"(c2)
+        : "memory");
+}
+__device__ __forceinline__ void mma_bf16_pair(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a), "l"(b), "r"(idesc), "r"(acc)
+        : "memory");
+}
+// arrive (when this thread's MMAs finish) on the barrier at the same offset in both CTAs
+__device__ __forceinline__ void mma_commit_pair_both(uint32_t bar) {
+    const uint16_t mask = 0x3;
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(bar),
+        "h"(mask)
+        : "memory");
+}
+__device__ __forceinline__ void mma_commit_pair_local(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+}
+// plain arrive on the barrier at the same offset in CTA rank 0 of the cluster
+__device__ __forceinline__ void mbar_arrive_rank0(uint32_t bar) {
+    uint32_t remote;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, 0;" : "=r"(remote) : "r"(bar));
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(remote) : "memory");
+}
+// Instruction descriptor for the pair MMA: M = 256 (128 rows per CTA).
+__host__ __device__ constexpr uint32_t idesc_bf16_pair(int n) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(256 >> 4) << 24);
+}
+
 // ------------------------------------------------------------------------------ tile order
 struct Tile {
     int g;       // group: expert (routed), E + s (shared GEMM1), 0 otherwise
@@ -206,11 +273,12 @@ struct Tile {
 
 template <int MODE>
 __device__ __forceinline__ int total_tiles(const Params& p) {
-    if (MODE == ROUTER) return ceil_div(p.T, BM);
-    if (MODE == ROUTERP) return ceil_div(p.T, BM) * ceil_div(ceil_div(p.d, BK), p.kb_per_split);
+    constexpr int TM = Cfg<MODE>::TM;
+    if (MODE == ROUTER) return ceil_div(p.T, TM);
+    if (MODE == ROUTERP) return ceil_div(p.T, TM) * ceil_div(ceil_div(p.d, BK), p.kb_per_split);
     if (MODE == GEMM1) return p.tile_start[p.g_end] - p.tile_start[p.g_begin];
     if (MODE == GEMM2R) return p.tile_start[p.E];
-    return ceil_div(p.T, BM) * ceil_div(p.d, 256);
+    return ceil_div(p.T, TM) * ceil_div(p.d, 256);
 }
 
 // largest g in [lo, hi) with ts[g] <= t   (ts non-decreasing, ts[hi] > t)
@@ -225,15 +293,16 @@ __device__ __forceinline__ int find_group(const int32_t* ts, int lo, int hi, int
 
 template <int MODE>
 __device__ __forceinline__ Tile decode(const Params& p, int t) {
+    constexpr int TM = Cfg<MODE>::TM;
     Tile x;
     x.kb0 = 0;
     if (MODE == ROUTER) {
-        x.g = 0; x.m0 = t * BM; x.n0 = 0; x.rows = p.T; x.row0 = 0; x.num_kb = ceil_div(p.d, BK);
+        x.g = 0; x.m0 = t * TM; x.n0 = 0; x.rows = p.T; x.row0 = 0; x.num_kb = ceil_div(p.d, BK);
     } else if (MODE == ROUTERP) {
-        const int mt = ceil_div(p.T, BM);
+        const int mt = ceil_div(p.T, TM);
         const int split = t / mt;
         const int kbt = ceil_div(p.d, BK);
-        x.g = split; x.m0 = (t % mt) * BM; x.n0 = 0; x.rows = p.T; x.row0 = 0;
+        x.g = split; x.m0 = (t % mt) * TM; x.n0 = 0; x.rows = p.T; x.row0 = 0;
         x.kb0 = split * p.kb_per_split;
         x.num_kb = min(p.kb_per_split, kbt - x.kb0);
     } else if (MODE == GEMM1) {
@@ -244,8 +313,8 @@ __device__ __forceinline__ Tile decode(const Params& p, int t) {
         x.g = g;
         x.rows = shared ? p.T : p.offsets[g + 1] - p.offsets[g];
         x.row0 = shared ? 0 : p.offsets[g];
-        const int mt = ceil_div(x.rows, BM);
-        x.m0 = (local % mt) * BM;
+        const int mt = ceil_div(x.rows, TM);
+        x.m0 = (local % mt) * TM;
         x.n0 = (local / mt) * 128;
         x.num_kb = ceil_div(p.d, BK);
     } else if (MODE == GEMM2R) {
@@ -254,14 +323,14 @@ __device__ __forceinline__ Tile decode(const Params& p, int t) {
         x.g = e;
         x.rows = p.offsets[e + 1] - p.offsets[e];
         x.row0 = p.offsets[e];
-        const int mt = ceil_div(x.rows, BM);
-        x.m0 = (local % mt) * BM;
+        const int mt = ceil_div(x.rows, TM);
+        x.m0 = (local % mt) * TM;
         x.n0 = (local / mt) * 256;
         x.num_kb = ceil_div(p.I, BK);
     } else {
-        const int mt = ceil_div(p.T, BM);
+        const int mt = ceil_div(p.T, TM);
         x.g = 0; x.rows = p.T; x.row0 = 0;
-        x.m0 = (t % mt) * BM;
+        x.m0 = (t % mt) * TM;
         x.n0 = (t / mt) * 256;
         x.num_kb = p.Ks * ceil_div(p.Is, BK);
     }
@@ -446,41 +515,68 @@ __device__ __forceinline__ void epilogue_router_partial(const Params& p, const T
 }
 
 // ------------------------------------------------------------------------------ the kernel
+// Pair protocol (expert GEMMs): both CTAs of a cluster pair run the same roles.  Each CTA's
+// producer waits on its own "empty" barriers and loads its halves of A and B into its own
+// ring, completing on the leader's "full" barrier; only the leader expects the pair's bytes,
+// issues the MMAs (reading both CTAs' rings) and commits stages and accumulators to the
+// barriers of both CTAs.  Each CTA's epilogue reads its own TMEM rows and arrives on the
+// leader's "accumulator empty" barrier.  A cluster barrier after set-up makes the leader's
+// barriers valid before any peer copy lands, and one before teardown keeps every shared
+// memory and TMEM range alive until the leader's last MMA has finished.
 template <int MODE, int KMAX>
 __global__ void __launch_bounds__(THREADS, 1) moe_tc_kernel(const __grid_constant__ Params p) {
+    using C = Cfg<MODE>;
+    constexpr bool PAIR = C::PAIR;
+    constexpr int STAGES = C::STAGES;
+    constexpr int B_BYTES = C::B_BYTES;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
     uint8_t* gbase = smem_raw + (base - raw);
     const uint32_t sA = base;
     const uint32_t sB = base + STAGES * A_BYTES;
-    const uint32_t bar0 = sB + STAGES * B_BYTES;
+    const uint32_t bar0 = base + RING_BYTES;
     // barrier addresses (8 bytes each)
     auto full_bar = [&](int s) { return bar0 + 8u * s; };
     auto empty_bar = [&](int s) { return bar0 + 8u * (STAGES + s); };
     auto tfull_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + a); };
     auto tempty_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + 2 + a); };
     const uint32_t drain_bar = bar0 + 8u * (2 * STAGES + 4);
-    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(gbase + (bar0 - base) + 8 * (2 * STAGES + 5));
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(gbase + RING_BYTES + 8 * (2 * STAGES + 5));
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const uint32_t rank = PAIR ? cluster_rank() : 0u;        // 0 = leader of the pair
+    const bool leader = rank == 0;
+    const int cta_slot = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;   // pair index
+    const int cta_slots = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) { mbar_init(full_bar(s), 1); mbar_init(empty_bar(s), 1); }
-        for (int a = 0; a < 2; ++a) { mbar_init(tfull_bar(a), 1); mbar_init(tempty_bar(a), EPI_WARPS); }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(tfull_bar(a), 1);
+            mbar_init(tempty_bar(a), PAIR ? 2 * EPI_WARPS : EPI_WARPS);
+        }
         mbar_init(drain_bar, 1);
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     }
     if (warp == 1) {
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_holder)),
-                     "r"(TMEM_COLS)
-                     : "memory");
-        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+        if (PAIR) {
+            asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_holder)),
+                         "r"(TMEM_COLS)
+                         : "memory");
+            asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+        } else {
+            asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_holder)),
+                         "r"(TMEM_COLS)
+                         : "memory");
+            asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+        }
     }
     tc_fence_before();
     __syncthreads();
+    if (PAIR) cluster_sync();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_holder;
     const int ntiles = total_tiles<MODE>(p);
@@ -488,7 +584,7 @@ __global__ void __launch_bounds__(THREADS, 1) moe_tc_kernel(const __grid_constan
     if (warp == 0) {
         // ------------------------------------------------------------------ TMA producer
         if (lane == 0) {
-            prefetch_map(&p.tmA[0]);
+            if (MODE != GEMM1 || p.g_begin < p.E) prefetch_map(&p.tmA[0]);
             prefetch_map(&p.tmB[0]);
             int stage = 0;
             uint32_t phase = 0;
@@ -496,7 +592,8 @@ __global__ void __launch_bounds__(THREADS, 1) moe_tc_kernel(const __grid_constan
 #pragma unroll
             for (int s = 0; s < STAGES; ++s) last_parity[s] = -1;
             bool ok = true;
-            for (int t = blockIdx.x; ok && t < ntiles; t += gridDim.x) {
+            const int arow = (int)rank * BM;                 // this CTA's rows inside a pair tile
+            for (int t = cta_slot; ok && t < ntiles; t += cta_slots) {
                 const Tile x = decode<MODE>(p, t);
                 for (int kk_ = 0; kk_ < x.num_kb; ++kk_) {
                     const int kb = x.kb0 + kk_;
@@ -507,43 +604,49 @@ __global__ void __launch_bounds__(THREADS, 1) moe_tc_kernel(const __grid_constan
                         mbar_expect_tx(fb, A_BYTES + p.n_mma * BK * 2);
                         tma_load_2d(a_dst, &p.tmA[0], fb, kb * BK, x.m0);
                         tma_load_2d(b_dst, &p.tmB[0], fb, kb * BK, 0);
-                    } else if (MODE == GEMM1) {
-                        mbar_expect_tx(fb, A_BYTES + B_BYTES);
-                        const bool shared = x.g >= p.E;
-                        const int e = shared ? x.g - p.E : x.g;
-                        tma_load_2d(a_dst, &p.tmA[shared ? 1 : 0], fb, kb * BK, x.row0 + x.m0);
-                        tma_load_3d(b_dst, &p.tmB[shared ? 2 : 0], fb, kb * BK, x.n0, e);
-                        tma_load_3d(b_dst + B_BYTES / 2, &p.tmB[shared ? 3 : 1], fb, kb * BK, x.n0, e);
-                    } else if (MODE == GEMM2R) {
-                        mbar_expect_tx(fb, A_BYTES + B_BYTES);
-                        tma_load_2d(a_dst, &p.tmA[0], fb, kb * BK, x.row0 + x.m0);
-                        tma_load_3d(b_dst, &p.tmB[0], fb, kb * BK, x.n0, x.g);
                     } else {
-                        const int kbs = ceil_div(p.Is, BK);
-                        const int s = kb / kbs, kk = kb % kbs;
-                        mbar_expect_tx(fb, A_BYTES + B_BYTES);
-                        tma_load_3d(a_dst, &p.tmA[0], fb, kk * BK, x.m0, s);
-                        tma_load_3d(b_dst, &p.tmB[0], fb, kk * BK, x.n0, s);
+                        if (leader) mbar_expect_tx(fb, 2 * (A_BYTES + B_BYTES));
+                        if (MODE == GEMM1) {
+                            // leader: W1 rows n0..n0+127 (accumulator columns 0-127);
+                            // follower: the same rows of W3 (columns 128-255)
+                            const bool shared = x.g >= p.E;
+                            const int e = shared ? x.g - p.E : x.g;
+                            tma_load_2d_pair(a_dst, &p.tmA[shared ? 1 : 0], fb, kb * BK, x.row0 + x.m0 + arow);
+                            tma_load_3d_pair(b_dst, &p.tmB[(shared ? 2 : 0) + (int)rank], fb, kb * BK, x.n0, e);
+                        } else if (MODE == GEMM2R) {
+                            tma_load_2d_pair(a_dst, &p.tmA[0], fb, kb * BK, x.row0 + x.m0 + arow);
+                            tma_load_3d_pair(b_dst, &p.tmB[0], fb, kb * BK, x.n0 + arow, x.g);
+                        } else {
+                            const int kbs = ceil_div(p.Is, BK);
+                            const int s = kb / kbs, kk = kb % kbs;
+                            tma_load_3d_pair(a_dst, &p.tmA[0], fb, kk * BK, x.m0 + arow, s);
+                            tma_load_3d_pair(b_dst, &p.tmB[0], fb, kk * BK, x.n0 + arow, s);
+                        }
                     }
                     last_parity[stage] = (int)phase;
                     if (++stage == STAGES) { stage = 0; phase ^= 1u; }
                 }
             }
-            // drain: every copy this thread issued has landed before the CTA may exit
+            // drain: every copy this thread issued has landed before the CTA may exit.  The
+            // leader sees the pair's bytes on its own full barriers; a follower knows its copies
+            // landed once the leader's MMA has released the stage they filled.
 #pragma unroll
-            for (int s = 0; s < STAGES; ++s)
-                if (last_parity[s] >= 0) mbar_wait(full_bar(s), (uint32_t)last_parity[s], abort_flag, p.err, false);
+            for (int s = 0; s < STAGES; ++s) {
+                if (last_parity[s] < 0) continue;
+                if (leader) mbar_wait(full_bar(s), (uint32_t)last_parity[s], abort_flag, p.err, false);
+                else mbar_wait(empty_bar(s), (uint32_t)last_parity[s], abort_flag, p.err, false);
+            }
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            const uint32_t idesc = idesc_bf16(p.n_mma);
+        if (lane == 0 && leader) {
+            const uint32_t idesc = PAIR ? idesc_bf16_pair(p.n_mma) : idesc_bf16(p.n_mma);
             int stage = 0;
             uint32_t phase = 0;
             int acc = 0;
             uint32_t acc_phase = 0;
             bool ok = true;
-            for (int t = blockIdx.x; ok && t < ntiles; t += gridDim.x) {
+            for (int t = cta_slot; ok && t < ntiles; t += cta_slots) {
                 const Tile x = decode<MODE>(p, t);
                 if (!mbar_wait(tempty_bar(acc), acc_phase ^ 1u, abort_flag, p.err)) break;
                 tc_fence_after();
@@ -554,18 +657,23 @@ __global__ void __launch_bounds__(THREADS, 1) moe_tc_kernel(const __grid_constan
                     const uint32_t a_addr = sA + stage * A_BYTES, b_addr = sB + stage * B_BYTES;
 #pragma unroll
                     for (int k = 0; k < BK / 16; ++k) {
-                        mma_bf16(d_tmem, sw128_desc(a_addr + k * 32), sw128_desc(b_addr + k * 32), idesc,
-                                 (kb > 0 || k > 0) ? 1u : 0u);
+                        const uint64_t ad = sw128_desc(a_addr + k * 32), bd = sw128_desc(b_addr + k * 32);
+                        const uint32_t accum = (kb > 0 || k > 0) ? 1u : 0u;
+                        if (PAIR) mma_bf16_pair(d_tmem, ad, bd, idesc, accum);
+                        else mma_bf16(d_tmem, ad, bd, idesc, accum);
                     }
-                    mma_commit(empty_bar(stage));
+                    if (PAIR) mma_commit_pair_both(empty_bar(stage));
+                    else mma_commit(empty_bar(stage));
                     if (++stage == STAGES) { stage = 0; phase ^= 1u; }
                 }
                 if (!ok) break;
-                mma_commit(tfull_bar(acc));
+                if (PAIR) mma_commit_pair_both(tfull_bar(acc));
+                else mma_commit(tfull_bar(acc));
                 if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
             }
             // drain: all MMAs issued by this thread have completed before TMEM is freed
-            mma_commit(drain_bar);
+            if (PAIR) mma_commit_pair_local(drain_bar);
+            else mma_commit(drain_bar);
             mbar_wait(drain_bar, 0, abort_flag, p.err, false);
         }
         __syncwarp();
@@ -573,10 +681,10 @@ __global__ void __launch_bounds__(THREADS, 1) moe_tc_kernel(const __grid_constan
         // ------------------------------------------------------------------ epilogue
         const int quad = warp & 3;                  // TMEM lanes 32*quad .. 32*quad+31
         const int half = (warp - 2) / 4;            // which half of the columns (0 or 1)
-        const int row = quad * 32 + lane;
+        const int row = (int)rank * BM + quad * 32 + lane;   // row inside the (pair) tile
         int acc = 0;
         uint32_t acc_phase = 0;
-        for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
+        for (int t = cta_slot; t < ntiles; t += cta_slots) {
             const Tile x = decode<MODE>(p, t);
             if (!mbar_wait(tfull_bar(acc), acc_phase, abort_flag, p.err)) break;
             tc_fence_after();
@@ -594,16 +702,25 @@ __global__ void __launch_bounds__(THREADS, 1) moe_tc_kernel(const __grid_constan
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(tempty_bar(acc));
+            if (lane == 0) {
+                if (PAIR) mbar_arrive_rank0(tempty_bar(acc));
+                else mbar_arrive(tempty_bar(acc));
+            }
             if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
         }
     }
 
     tc_fence_before();
     __syncthreads();
+    if (PAIR) cluster_sync();
     if (warp == 1) {
         tc_fence_after();
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(TMEM_COLS) : "memory");
+        if (PAIR)
+            asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(TMEM_COLS)
+                         : "memory");
+        else
+            asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(TMEM_COLS)
+                         : "memory");
     }
 }
 
@@ -639,12 +756,40 @@ bool make_map(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t mid, uin
     return r == CUDA_SUCCESS;
 }
 
+// Launches MODE.  Pair modes run as clusters of 2 CTAs; `tiles` bounds the useful CTAs (pairs
+// for pair modes), and the grid never exceeds what can be resident at once (persistent loop).
 template <int MODE, int KMAX>
-cudaError_t launch(const Params& p, int grid, cudaStream_t stream) {
+cudaError_t launch(const Params& p, int tiles, cudaStream_t stream) {
     auto kern = moe_tc_kernel<MODE, KMAX>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    kern<<<grid, THREADS, SMEM_BYTES, stream>>>(p);
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    cfg.blockDim = dim3(THREADS);
+    cfg.dynamicSmemBytes = SMEM_BYTES;
+    cfg.stream = stream;
+    if (Cfg<MODE>::PAIR) {
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        static int max_pairs = 0;
+        if (!max_pairs) {
+            cfg.gridDim = dim3(2 * (num_sms() / 2));
+            int n = 0;
+            if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n <= 0) n = num_sms() / 2;
+            max_pairs = n;
+        }
+        const int pairs = tiles < max_pairs ? (tiles > 0 ? tiles : 1) : max_pairs;
+        cfg.gridDim = dim3(2 * pairs);
+    } else {
+        const int grid = tiles < num_sms() ? (tiles > 0 ? tiles : 1) : num_sms();
+        cfg.gridDim = dim3(grid);
+    }
+    e = cudaLaunchKernelEx(&cfg, kern, p);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 
@@ -701,13 +846,11 @@ cudaError_t launch_tc_router(const Dims& D, const void* x, const void* centroids
         p.kb_per_split = ceil_div(kbt, nsplit);
         p.partial = partial;
         const int tiles = mt * ceil_div(kbt, p.kb_per_split);
-        const int grid = tiles < num_sms() ? tiles : num_sms();
-        cudaError_t e = launch<ROUTERP, 8>(p, grid, stream);
+        cudaError_t e = launch<ROUTERP, 8>(p, tiles, stream);
         if (e != cudaSuccess) return e;
         return launch_router_finish(D, partial, ceil_div(kbt, p.kb_per_split), idx, gate, stream);
     }
-    const int grid = mt < num_sms() ? mt : num_sms();
-    return D.k <= 8 ? launch<ROUTER, 8>(p, grid, stream) : launch<ROUTER, 32>(p, grid, stream);
+    return D.k <= 8 ? launch<ROUTER, 8>(p, mt, stream) : launch<ROUTER, 32>(p, mt, stream);
 }
 
 cudaError_t launch_tc_gemm1(const Dims& D, const void* x, const void* x_perm, const int32_t* offsets,
@@ -735,7 +878,7 @@ cudaError_t launch_tc_gemm1(const Dims& D, const void* x, const void* x_perm, co
         ok &= make_map(&p.tmB[3], Sh.w3, D.d, D.Is, D.Ks, BK, 128, true);
     }
     if (!ok) return cudaErrorInvalidValue;
-    return launch<GEMM1, 8>(p, num_sms(), stream);
+    return launch<GEMM1, 8>(p, num_sms(), stream);          // tile count lives on the device
 }
 
 cudaError_t launch_tc_gemm2_routed(const Dims& D, const int32_t* offsets, const int32_t* tile_start2,
@@ -750,9 +893,9 @@ cudaError_t launch_tc_gemm2_routed(const Dims& D, const int32_t* offsets, const 
     p.b2 = (const __nv_bfloat16*)R.b2;
     p.y = (__nv_bfloat16*)y_sorted;
     bool ok = make_map(&p.tmA[0], h_r, D.I, (uint64_t)D.slots(), 1, BK, BM, false);
-    ok &= make_map(&p.tmB[0], R.w2, D.I, D.d, D.E, BK, 256, true);
+    ok &= make_map(&p.tmB[0], R.w2, D.I, D.d, D.E, BK, 128, true);      // each CTA of a pair: 128 rows
     if (!ok) return cudaErrorInvalidValue;
-    return launch<GEMM2R, 8>(p, num_sms(), stream);
+    return launch<GEMM2R, 8>(p, num_sms(), stream);         // tile count lives on the device
 }
 
 cudaError_t launch_tc_gemm2_shared(const Dims& D, const FfnWeights& Sh, const void* h_s, float* sout, uint32_t* err,
@@ -763,11 +906,9 @@ cudaError_t launch_tc_gemm2_shared(const Dims& D, const FfnWeights& Sh, const vo
     p.sb2 = (const __nv_bfloat16*)Sh.b2;
     p.sout = sout;
     bool ok = make_map(&p.tmA[0], h_s, D.Is, D.T, D.Ks, BK, BM, true);
-    ok &= make_map(&p.tmB[0], Sh.w2, D.Is, D.d, D.Ks, BK, 256, true);
+    ok &= make_map(&p.tmB[0], Sh.w2, D.Is, D.d, D.Ks, BK, 128, true);
     if (!ok) return cudaErrorInvalidValue;
-    const int tiles = ceil_div(D.T, BM) * ceil_div(D.d, 256);
-    const int grid = tiles < num_sms() ? tiles : num_sms();
-    return launch<GEMM2S, 8>(p, grid, stream);
+    return launch<GEMM2S, 8>(p, ceil_div(D.T, Cfg<GEMM2S>::TM) * ceil_div(D.d, 256), stream);
 }
 
 }  // namespace moe

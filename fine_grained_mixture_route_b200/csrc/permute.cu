@@ -156,7 +156,7 @@ __global__ void plan_kernel(const int32_t* __restrict__ offsets, long long S, in
         } else {
             rows = T;
         }
-        const int m = ceil_div(rows, 128);
+        const int m = ceil_div(rows, GEMM_TILE_ROWS);
         t1[g] = m * (g < E ? n1r : n1s);
         if (g < E) t2[g] = m * n2;
     }
