@@ -37,6 +37,7 @@
 
 namespace moe {
 namespace tc {
+bool pairs_for(const Dims& D);
 
 constexpr int BM = 128;                  // rows per CTA (TMEM lanes)
 constexpr int BK = 64;                   // K per stage: 64 bf16 = one 128-byte swizzle row
@@ -52,12 +53,14 @@ constexpr uint32_t PEER_BIT_MASK = 0xFEFFFFFFu;   // shared::cluster address of 
 
 enum Mode : int { ROUTER = 0, GEMM1 = 1, GEMM2R = 2, GEMM2S = 3, ROUTERP = 4 };
 
-// The expert GEMMs run on CTA pairs (cta_group::2): a 256-row tile, each CTA holding 128 rows
-// of A, half of the 256 B rows and its 128 x 256 slice of the accumulator, so each SM loads
-// 32 KB per K stage instead of 48 KB.  The router modes run on single CTAs.
-template <int MODE>
+// The expert GEMMs can run on CTA pairs (cta_group::2): a 256-row tile, each CTA holding 128
+// rows of A, half of the 256 B rows and its 128 x 256 slice of the accumulator, so each SM
+// loads 32 KB per K stage instead of 48 KB.  Pairs pay off when experts hold many rows; with a
+// few rows per expert (decode) single CTAs keep twice as many weight tiles in flight.  The
+// router modes always run on single CTAs.
+template <int MODE, bool PAIR_ = false>
 struct Cfg {
-    static constexpr bool PAIR = MODE == GEMM1 || MODE == GEMM2R || MODE == GEMM2S;
+    static constexpr bool PAIR = PAIR_ && (MODE == GEMM1 || MODE == GEMM2R || MODE == GEMM2S);
     static constexpr int TM = PAIR ? 2 * BM : BM;                 // rows per tile
     static constexpr int B_BYTES = (PAIR ? 128 : 256) * BK * 2;   // B rows held by one CTA
     static constexpr int STAGES = RING_BYTES / (A_BYTES + B_BYTES);
@@ -271,9 +274,9 @@ struct Tile {
     int kb0;     // first K block (split-K router)
 };
 
-template <int MODE>
+template <int MODE, bool PAIR>
 __device__ __forceinline__ int total_tiles(const Params& p) {
-    constexpr int TM = Cfg<MODE>::TM;
+    constexpr int TM = Cfg<MODE, PAIR>::TM;
     if (MODE == ROUTER) return ceil_div(p.T, TM);
     if (MODE == ROUTERP) return ceil_div(p.T, TM) * ceil_div(ceil_div(p.d, BK), p.kb_per_split);
     if (MODE == GEMM1) return p.tile_start[p.g_end] - p.tile_start[p.g_begin];
@@ -291,9 +294,9 @@ __device__ __forceinline__ int find_group(const int32_t* ts, int lo, int hi, int
     return lo;
 }
 
-template <int MODE>
+template <int MODE, bool PAIR>
 __device__ __forceinline__ Tile decode(const Params& p, int t) {
-    constexpr int TM = Cfg<MODE>::TM;
+    constexpr int TM = Cfg<MODE, PAIR>::TM;
     Tile x;
     x.kb0 = 0;
     if (MODE == ROUTER) {
@@ -523,9 +526,9 @@ __device__ __forceinline__ void epilogue_router_partial(const Params& p, const T
 // leader's "accumulator empty" barrier.  A cluster barrier after set-up makes the leader's
 // barriers valid before any peer copy lands, and one before teardown keeps every shared
 // memory and TMEM range alive until the leader's last MMA has finished.
-template <int MODE, int KMAX>
+template <int MODE, int KMAX, bool PAIR_>
 __global__ void __launch_bounds__(THREADS, 1) moe_tc_kernel(const __grid_constant__ Params p) {
-    using C = Cfg<MODE>;
+    using C = Cfg<MODE, PAIR_>;
     constexpr bool PAIR = C::PAIR;
     constexpr int STAGES = C::STAGES;
     constexpr int B_BYTES = C::B_BYTES;
@@ -579,7 +582,7 @@ __global__ void __launch_bounds__(THREADS, 1) moe_tc_kernel(const __grid_constan
     if (PAIR) cluster_sync();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_holder;
-    const int ntiles = total_tiles<MODE>(p);
+    const int ntiles = total_tiles<MODE, PAIR>(p);
 
     if (warp == 0) {
         // ------------------------------------------------------------------ TMA producer
@@ -594,7 +597,7 @@ __global__ void __launch_bounds__(THREADS, 1) moe_tc_kernel(const __grid_constan
             bool ok = true;
             const int arow = (int)rank * BM;                 // this CTA's rows inside a pair tile
             for (int t = cta_slot; ok && t < ntiles; t += cta_slots) {
-                const Tile x = decode<MODE>(p, t);
+                const Tile x = decode<MODE, PAIR>(p, t);
                 for (int kk_ = 0; kk_ < x.num_kb; ++kk_) {
                     const int kb = x.kb0 + kk_;
                     if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, p.err)) { ok = false; break; }
@@ -604,7 +607,7 @@ __global__ void __launch_bounds__(THREADS, 1) moe_tc_kernel(const __grid_constan
                         mbar_expect_tx(fb, A_BYTES + p.n_mma * BK * 2);
                         tma_load_2d(a_dst, &p.tmA[0], fb, kb * BK, x.m0);
                         tma_load_2d(b_dst, &p.tmB[0], fb, kb * BK, 0);
-                    } else {
+                    } else if (PAIR) {
                         if (leader) mbar_expect_tx(fb, 2 * (A_BYTES + B_BYTES));
                         if (MODE == GEMM1) {
                             // leader: W1 rows n0..n0+127 (accumulator columns 0-127);
@@ -621,6 +624,23 @@ __global__ void __launch_bounds__(THREADS, 1) moe_tc_kernel(const __grid_constan
                             const int s = kb / kbs, kk = kb % kbs;
                             tma_load_3d_pair(a_dst, &p.tmA[0], fb, kk * BK, x.m0 + arow, s);
                             tma_load_3d_pair(b_dst, &p.tmB[0], fb, kk * BK, x.n0 + arow, s);
+                        }
+                    } else {
+                        mbar_expect_tx(fb, A_BYTES + B_BYTES);
+                        if (MODE == GEMM1) {
+                            const bool shared = x.g >= p.E;
+                            const int e = shared ? x.g - p.E : x.g;
+                            tma_load_2d(a_dst, &p.tmA[shared ? 1 : 0], fb, kb * BK, x.row0 + x.m0);
+                            tma_load_3d(b_dst, &p.tmB[shared ? 2 : 0], fb, kb * BK, x.n0, e);
+                            tma_load_3d(b_dst + B_BYTES / 2, &p.tmB[shared ? 3 : 1], fb, kb * BK, x.n0, e);
+                        } else if (MODE == GEMM2R) {
+                            tma_load_2d(a_dst, &p.tmA[0], fb, kb * BK, x.row0 + x.m0);
+                            tma_load_3d(b_dst, &p.tmB[0], fb, kb * BK, x.n0, x.g);
+                        } else {
+                            const int kbs = ceil_div(p.Is, BK);
+                            const int s = kb / kbs, kk = kb % kbs;
+                            tma_load_3d(a_dst, &p.tmA[0], fb, kk * BK, x.m0, s);
+                            tma_load_3d(b_dst, &p.tmB[0], fb, kk * BK, x.n0, s);
                         }
                     }
                     last_parity[stage] = (int)phase;
@@ -647,7 +667,7 @@ __global__ void __launch_bounds__(THREADS, 1) moe_tc_kernel(const __grid_constan
             uint32_t acc_phase = 0;
             bool ok = true;
             for (int t = cta_slot; ok && t < ntiles; t += cta_slots) {
-                const Tile x = decode<MODE>(p, t);
+                const Tile x = decode<MODE, PAIR>(p, t);
                 if (!mbar_wait(tempty_bar(acc), acc_phase ^ 1u, abort_flag, p.err)) break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + (uint32_t)(acc * ACC_COLS);
@@ -685,7 +705,7 @@ __global__ void __launch_bounds__(THREADS, 1) moe_tc_kernel(const __grid_constan
         int acc = 0;
         uint32_t acc_phase = 0;
         for (int t = cta_slot; t < ntiles; t += cta_slots) {
-            const Tile x = decode<MODE>(p, t);
+            const Tile x = decode<MODE, PAIR>(p, t);
             if (!mbar_wait(tfull_bar(acc), acc_phase, abort_flag, p.err)) break;
             tc_fence_after();
             const uint32_t tacc = tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(acc * ACC_COLS);
@@ -758,9 +778,9 @@ bool make_map(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t mid, uin
 
 // Launches MODE.  Pair modes run as clusters of 2 CTAs; `tiles` bounds the useful CTAs (pairs
 // for pair modes), and the grid never exceeds what can be resident at once (persistent loop).
-template <int MODE, int KMAX>
+template <int MODE, int KMAX, bool PAIR = false>
 cudaError_t launch(const Params& p, int tiles, cudaStream_t stream) {
-    auto kern = moe_tc_kernel<MODE, KMAX>;
+    auto kern = moe_tc_kernel<MODE, KMAX, PAIR>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
@@ -768,7 +788,7 @@ cudaError_t launch(const Params& p, int tiles, cudaStream_t stream) {
     cfg.blockDim = dim3(THREADS);
     cfg.dynamicSmemBytes = SMEM_BYTES;
     cfg.stream = stream;
-    if (Cfg<MODE>::PAIR) {
+    if (Cfg<MODE, PAIR>::PAIR) {
         attr[0].id = cudaLaunchAttributeClusterDimension;
         attr[0].val.clusterDim.x = 2;
         attr[0].val.clusterDim.y = 1;
@@ -814,6 +834,22 @@ int num_sms() {
         if (n <= 0) n = 148;
     }
     return n;
+}
+
+// Whether the expert GEMMs run on CTA pairs.  Measured on one B200 with both variants
+// interleaved (prefill 14.3 vs 15.0 ms per layer, decode 3.9 vs 5.8 ms, mid 0.73 vs 0.77 ms),
+// single CTAs are faster for every layer shape here, so pairs are off unless a build sets
+// MOE_PAIR_POLICY=1.
+bool gemm_pairs(const Dims& D) {
+    (void)D;
+#if defined(MOE_PAIR_POLICY) && MOE_PAIR_POLICY > 0
+    return true;
+#else
+    return false;
+#endif
+}
+namespace tc {
+bool pairs_for(const Dims& D) { return gemm_pairs(D); }
 }
 
 bool tc_router_supported(const Dims& D) { return D.bf16 && D.E % 16 == 0 && D.E >= 16 && D.E <= 256; }
@@ -878,7 +914,8 @@ cudaError_t launch_tc_gemm1(const Dims& D, const void* x, const void* x_perm, co
         ok &= make_map(&p.tmB[3], Sh.w3, D.d, D.Is, D.Ks, BK, 128, true);
     }
     if (!ok) return cudaErrorInvalidValue;
-    return launch<GEMM1, 8>(p, num_sms(), stream);          // tile count lives on the device
+    // tile count lives on the device
+    return tc::pairs_for(D) ? launch<GEMM1, 8, true>(p, num_sms(), stream) : launch<GEMM1, 8, false>(p, num_sms(), stream);
 }
 
 cudaError_t launch_tc_gemm2_routed(const Dims& D, const int32_t* offsets, const int32_t* tile_start2,
@@ -893,9 +930,10 @@ cudaError_t launch_tc_gemm2_routed(const Dims& D, const int32_t* offsets, const 
     p.b2 = (const __nv_bfloat16*)R.b2;
     p.y = (__nv_bfloat16*)y_sorted;
     bool ok = make_map(&p.tmA[0], h_r, D.I, (uint64_t)D.slots(), 1, BK, BM, false);
-    ok &= make_map(&p.tmB[0], R.w2, D.I, D.d, D.E, BK, 128, true);      // each CTA of a pair: 128 rows
+    ok &= make_map(&p.tmB[0], R.w2, D.I, D.d, D.E, BK, tc::pairs_for(D) ? 128 : 256, true);
     if (!ok) return cudaErrorInvalidValue;
-    return launch<GEMM2R, 8>(p, num_sms(), stream);         // tile count lives on the device
+    return tc::pairs_for(D) ? launch<GEMM2R, 8, true>(p, num_sms(), stream)
+                         : launch<GEMM2R, 8, false>(p, num_sms(), stream);
 }
 
 cudaError_t launch_tc_gemm2_shared(const Dims& D, const FfnWeights& Sh, const void* h_s, float* sout, uint32_t* err,
@@ -906,9 +944,11 @@ cudaError_t launch_tc_gemm2_shared(const Dims& D, const FfnWeights& Sh, const vo
     p.sb2 = (const __nv_bfloat16*)Sh.b2;
     p.sout = sout;
     bool ok = make_map(&p.tmA[0], h_s, D.Is, D.T, D.Ks, BK, BM, true);
-    ok &= make_map(&p.tmB[0], Sh.w2, D.Is, D.d, D.Ks, BK, 128, true);
+    ok &= make_map(&p.tmB[0], Sh.w2, D.Is, D.d, D.Ks, BK, tc::pairs_for(D) ? 128 : 256, true);
     if (!ok) return cudaErrorInvalidValue;
-    return launch<GEMM2S, 8>(p, ceil_div(D.T, Cfg<GEMM2S>::TM) * ceil_div(D.d, 256), stream);
+    const int n = ceil_div(D.d, 256);
+    return tc::pairs_for(D) ? launch<GEMM2S, 8, true>(p, ceil_div(D.T, 256) * n, stream)
+                         : launch<GEMM2S, 8, false>(p, ceil_div(D.T, 128) * n, stream);
 }
 
 }  // namespace moe

@@ -34,9 +34,11 @@ cudaError_t launch_permute(const Dims& D, const int32_t* idx, const float* gate,
 // Tile tables of the grouped GEMMs.  Groups 0..E-1 are the routed experts (rows from
 // offsets, or 0 when offsets is NULL), groups E..E+Ks-1 the shared experts (T rows each).
 // tile_start1[G+1]: GEMM1 tiles of GEMM_TILE_ROWS rows x 128 hidden columns; tile_start2[E+1]:
-// routed GEMM2 tiles of GEMM_TILE_ROWS rows x 256 output columns.  A tile is computed by a
-// pair of CTAs, 128 rows each.
-constexpr int GEMM_TILE_ROWS = 256;
+// routed GEMM2 tiles of gemm_tile_rows(D) rows x 256 output columns.
+// The expert GEMMs run on CTA pairs (256-row tiles, 128 rows per CTA) when gemm_pairs(D), else
+// on single CTAs (128-row tiles).
+bool gemm_pairs(const Dims& D);
+inline int gemm_tile_rows(const Dims& D) { return gemm_pairs(D) ? 256 : 128; }
 cudaError_t launch_plan(const Dims& D, const int32_t* offsets, int32_t* tile_start1, int32_t* tile_start2,
                         uint32_t* err, cudaStream_t stream);
 

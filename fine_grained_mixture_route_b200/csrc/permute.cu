@@ -132,7 +132,7 @@ __global__ void permute_scatter_kernel(const int32_t* __restrict__ idx, const fl
 
 // tile tables of the grouped GEMMs (see launch.h)
 __global__ void plan_kernel(const int32_t* __restrict__ offsets, long long S, int T, int d, int E, int I, int Ks,
-                            int Is, int32_t* __restrict__ tile_start1, int32_t* __restrict__ tile_start2, uint32_t* err) {
+                            int Is, int tile_rows, int32_t* __restrict__ tile_start1, int32_t* __restrict__ tile_start2, uint32_t* err) {
     extern __shared__ int sh[];
     const int G = E + Ks;
     int* t1 = sh;                // [G + 1]
@@ -156,7 +156,7 @@ __global__ void plan_kernel(const int32_t* __restrict__ offsets, long long S, in
         } else {
             rows = T;
         }
-        const int m = ceil_div(rows, GEMM_TILE_ROWS);
+        const int m = ceil_div(rows, tile_rows);
         t1[g] = m * (g < E ? n1r : n1s);
         if (g < E) t2[g] = m * n2;
     }
@@ -265,6 +265,7 @@ cudaError_t launch_plan(const Dims& D, const int32_t* offsets, int32_t* tile_sta
     const int G = D.E + D.Ks;
     const size_t smem = sizeof(int) * ((size_t)G + 1 + D.E + 1 + 32);
     plan_kernel<<<1, SCAN_THREADS, smem, stream>>>(offsets, D.slots(), D.T, D.d, D.E, D.I, D.Ks, D.Ks > 0 ? D.Is : 1,
+                                                   gemm_tile_rows(D),
                                                    tile_start1, tile_start2, err);
     return cudaGetLastError();
 }
