@@ -71,47 +71,71 @@ __global__ void permute_hist_kernel(const int32_t* __restrict__ idx, long long S
     for (int e = threadIdx.x; e < E; e += blockDim.x) block_hist[(size_t)blockIdx.x * E + e] = hist[e];
 }
 
-// pass 2: counts, offsets, and each block's starting position per expert (in place)
+// pass 2: counts, offsets, and each block's starting position per expert (in place).  One
+// warp per expert scans that expert's column of block counts 32 blocks at a time.
 __global__ void permute_scan_kernel(int32_t* __restrict__ block_hist, int nblk, int E,
                                     int32_t* __restrict__ counts, int32_t* __restrict__ offsets) {
     extern __shared__ int sh[];
     int* cnt = sh;               // [E]
     int* warp_sums = sh + E;     // [32]
-    for (int e = threadIdx.x; e < E; e += blockDim.x) {
-        int run = 0;
-        for (int b = 0; b < nblk; ++b) {
-            int c = block_hist[(size_t)b * E + e];
-            block_hist[(size_t)b * E + e] = run;
-            run += c;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+    for (int e = warp; e < E; e += nwarps) {
+        int carry = 0;
+        for (int b0 = 0; b0 < nblk; b0 += 32) {
+            const int b = b0 + lane;
+            const int c = b < nblk ? block_hist[(size_t)b * E + e] : 0;
+            int incl = c;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += y;
+            }
+            if (b < nblk) block_hist[(size_t)b * E + e] = carry + incl - c;
+            carry += __shfl_sync(0xffffffffu, incl, 31);
         }
-        cnt[e] = run;
-        counts[e] = run;
+        if (lane == 0) { cnt[e] = carry; counts[e] = carry; }
     }
     __syncthreads();
     const int total = block_exclusive_scan(cnt, E, warp_sums);
-    for (int e = threadIdx.x; e < E; e += blockDim.x) {
-        offsets[e] = cnt[e];
-        for (int b = 0; b < nblk; ++b) block_hist[(size_t)b * E + e] += cnt[e];
+    for (int e = warp; e < E; e += nwarps) {
+        const int base = cnt[e];
+        for (int b = lane; b < nblk; b += 32) block_hist[(size_t)b * E + e] += base;
     }
+    for (int e = threadIdx.x; e < E; e += blockDim.x) offsets[e] = cnt[e];
     if (threadIdx.x == 0) offsets[E] = total;
 }
 
-// pass 3: one warp per block walks its chunk of slots in order, 32 at a time
-__global__ void permute_scatter_kernel(const int32_t* __restrict__ idx, const float* __restrict__ gate, long long S,
-                                       int k, int E, const int32_t* __restrict__ block_base,
-                                       int32_t* __restrict__ sorted_token, float* __restrict__ sorted_gate,
-                                       int32_t* __restrict__ slot_of) {
+// pass 3: one warp per block walks its chunk of slots in order, 32 at a time.  The chunk's
+// picks and gates are loaded up front (32 per lane), so the ordered walk itself only touches
+// shared memory and issues independent stores.
+__global__ void __launch_bounds__(32) permute_scatter_kernel(const int32_t* __restrict__ idx,
+                                                             const float* __restrict__ gate, long long S, int k,
+                                                             int E, const int32_t* __restrict__ block_base,
+                                                             int32_t* __restrict__ sorted_token,
+                                                             float* __restrict__ sorted_gate,
+                                                             int32_t* __restrict__ slot_of) {
+    constexpr int STEPS = PERMUTE_CHUNK / 32;
     extern __shared__ int running[];
     const int lane = threadIdx.x;
     for (int e = lane; e < E; e += 32) running[e] = block_base[(size_t)blockIdx.x * E + e];
-    __syncwarp();
     const long long s0 = (long long)blockIdx.x * PERMUTE_CHUNK;
     const long long s1 = min(S, s0 + PERMUTE_CHUNK);
+    int ev[STEPS];
+    float gv[STEPS];
+#pragma unroll
+    for (int i = 0; i < STEPS; ++i) {
+        const long long s = s0 + 32 * i + lane;
+        ev[i] = s < s1 ? idx[s] : -1;
+        gv[i] = s < s1 ? gate[s] : 0.f;
+    }
+    __syncwarp();
     const unsigned lt = (1u << lane) - 1u;
-    for (long long sb = s0; sb < s1; sb += 32) {
-        const long long s = sb + lane;
+#pragma unroll
+    for (int i = 0; i < STEPS; ++i) {
+        const long long s = s0 + 32 * i + lane;
+        if (s0 + 32 * i >= s1) break;
         const bool live = s < s1;
-        int e = live ? idx[s] : -1;
+        int e = ev[i];
         const bool ok = live && e >= 0 && e < E;
         if (!ok) e = -1 - lane;                       // unique key: never matches a real expert
         const unsigned peers = __match_any_sync(0xffffffffu, e);
@@ -122,7 +146,7 @@ __global__ void permute_scatter_kernel(const int32_t* __restrict__ idx, const fl
         __syncwarp();
         if (ok) {
             sorted_token[pos] = (int32_t)(s / k);
-            sorted_gate[pos] = gate[s];
+            sorted_gate[pos] = gv[i];
             slot_of[s] = pos;
         } else if (live) {
             slot_of[s] = -1;

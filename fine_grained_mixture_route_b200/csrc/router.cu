@@ -109,35 +109,36 @@ router_simt_kernel(const T* __restrict__ x, const T* __restrict__ cen, int32_t* 
 
 
 // Split-K router, last step: z = sum of the per-split partial logits in ascending split order
-// (deterministic), then the same softmax / top-k as above.  A block sums FIN_TOK tokens with
-// coalesced float4 loads (consecutive threads read consecutive experts of one split row),
-// then one warp per token ranks them.
-constexpr int FIN_TOK = 8;
-__global__ void __launch_bounds__(FIN_TOK * 32)
+// (deterministic), then the same softmax / top-k as above.  One block per token: E/4 threads
+// each sum a float4 of consecutive experts over the splits (coalesced across the block), then
+// warp 0 ranks the token.
+__global__ void __launch_bounds__(256)
 router_finish_kernel(const float* __restrict__ partial, int nsplit, int Tn, int E, int k, int32_t* __restrict__ idx_out,
                      float* __restrict__ gate_out) {
     extern __shared__ float zs[];
-    const int t0 = blockIdx.x * FIN_TOK;
+    const int t = blockIdx.x;
     const int E4 = E / 4;
     const size_t stride4 = (size_t)Tn * E4;                 // float4s between consecutive splits
-    for (int c = threadIdx.x; c < FIN_TOK * E4; c += blockDim.x) {
-        const int tt = c / E4, e4 = c % E4;
-        const int t = t0 + tt;
+    for (int e4 = threadIdx.x; e4 < E4; e4 += blockDim.x) {
+        const float4* src = reinterpret_cast<const float4*>(partial) + (size_t)t * E4 + e4;
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (t < Tn) {
-            const float4* src = reinterpret_cast<const float4*>(partial) + (size_t)t * E4 + e4;
-#pragma unroll 4
-            for (int s = 0; s < nsplit; ++s) {
-                const float4 v = src[(size_t)s * stride4];
-                acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
-            }
+        int s = 0;
+        for (; s + 4 <= nsplit; s += 4) {
+            const float4 v0 = src[(size_t)s * stride4], v1 = src[(size_t)(s + 1) * stride4];
+            const float4 v2 = src[(size_t)(s + 2) * stride4], v3 = src[(size_t)(s + 3) * stride4];
+            acc.x += v0.x; acc.y += v0.y; acc.z += v0.z; acc.w += v0.w;
+            acc.x += v1.x; acc.y += v1.y; acc.z += v1.z; acc.w += v1.w;
+            acc.x += v2.x; acc.y += v2.y; acc.z += v2.z; acc.w += v2.w;
+            acc.x += v3.x; acc.y += v3.y; acc.z += v3.z; acc.w += v3.w;
         }
-        reinterpret_cast<float4*>(zs + tt * E)[e4] = acc;
+        for (; s < nsplit; ++s) {
+            const float4 v = src[(size_t)s * stride4];
+            acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+        }
+        reinterpret_cast<float4*>(zs)[e4] = acc;
     }
     __syncthreads();
-    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    const int t = t0 + warp;
-    if (t < Tn) warp_softmax_topk(zs + warp * E, E, k, lane, idx_out + (size_t)t * k, gate_out + (size_t)t * k);
+    if (threadIdx.x < 32) warp_softmax_topk(zs, E, k, threadIdx.x, idx_out + (size_t)t * k, gate_out + (size_t)t * k);
 }
 
 }  // namespace
@@ -162,9 +163,9 @@ cudaError_t launch_router_simt(const Dims& D, const void* x, const void* centroi
 
 cudaError_t launch_router_finish(const Dims& D, const float* partial, int nsplit, int32_t* idx, float* gate,
                                  cudaStream_t stream) {
-    const int blocks = ceil_div(D.T, FIN_TOK);
-    const size_t smem = sizeof(float) * FIN_TOK * D.E;
-    router_finish_kernel<<<blocks, FIN_TOK * 32, smem, stream>>>(partial, nsplit, D.T, D.E, D.k, idx, gate);
+    const int E4 = D.E / 4;
+    const int threads = E4 < 32 ? 32 : (E4 > 256 ? 256 : (E4 + 31) / 32 * 32);
+    router_finish_kernel<<<D.T, threads, sizeof(float) * D.E, stream>>>(partial, nsplit, D.T, D.E, D.k, idx, gate);
     return cudaGetLastError();
 }
 
