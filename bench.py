@@ -101,11 +101,15 @@ def stage_work(cfg: W.LayerConfig, touched: int):
         "gemm1_swiglu": (2.0 * S * d * 2 * I + 2.0 * Ks * T * d * 2 * Is,
                          touched * (2 * I * d + 2 * I * bias) * b + Ks * (2 * Is * d + 2 * Is * bias) * b
                          + S * d * b + (T * d * b if Ks else 0) + (S * I + Ks * T * Is) * b),
-        "gemm2_gate": (2.0 * S * I * d, touched * (d * I + d * bias) * b + S * I * b + S * d * b + S * 8),
-        "gemm2_shared": (2.0 * Ks * T * Is * d, Ks * (d * Is + d * bias) * b + Ks * T * Is * b
-                         + (T * d * 4 if Ks else 0)),
+        "gemm2": (2.0 * S * I * d + 2.0 * Ks * T * Is * d,
+                  touched * (d * I + d * bias) * b + S * I * b + S * d * b + S * 8
+                  + Ks * (d * Is + d * bias) * b + Ks * T * Is * b + (T * d * 4 if Ks else 0)),
         "combine": (0.0, S * d * b + (T * d * 4 if Ks else 0) + T * d * b + S * 4),
     }
+    if cfg.dtype == torch.float32:   # fp32 layers: the shared GEMM2 runs inside the combine stage
+        f2, b2_ = w["gemm2"]
+        w["gemm2"] = (2.0 * S * I * d, touched * (d * I + d * bias) * b + S * I * b + S * d * b + S * 8)
+        w["combine"] = (f2 - w["gemm2"][0], w["combine"][1] + b2_ - w["gemm2"][1])
     return w
 
 

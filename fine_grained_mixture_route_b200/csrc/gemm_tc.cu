@@ -49,6 +49,9 @@ constexpr int ACC_COLS = 256;
 constexpr int RING_BYTES = 192 * 1024;   // shared-memory ring (stages x (A + B))
 constexpr int SMEM_BYTES = 1024 /*align slack*/ + RING_BYTES + 256 /*barriers*/;
 constexpr unsigned long long WAIT_NS = 4000000000ull;
+#ifndef MOE_GROUP_M
+#define MOE_GROUP_M 8                    // M-tiles per raster band of the expert GEMMs
+#endif
 constexpr uint32_t PEER_BIT_MASK = 0xFEFFFFFFu;   // shared::cluster address of CTA rank 0 of a pair
 
 enum Mode : int { ROUTER = 0, GEMM1 = 1, GEMM2R = 2, GEMM2S = 3, ROUTERP = 4 };
@@ -85,6 +88,8 @@ struct Params {
     float* gate_out;
     float* partial;            // ROUTERP: [nsplit][T][E] fp32 partial logits
     int kb_per_split;          // ROUTERP: K blocks per split
+    int group_m;               // tile raster: bands of group_m M-tiles swept across all N-tiles
+    int fold_shared;           // GEMM2R: shared-expert GEMM2 tiles follow the routed ones (-> sout)
     uint32_t* err;
 };
 
@@ -280,7 +285,8 @@ __device__ __forceinline__ int total_tiles(const Params& p) {
     if (MODE == ROUTER) return ceil_div(p.T, TM);
     if (MODE == ROUTERP) return ceil_div(p.T, TM) * ceil_div(ceil_div(p.d, BK), p.kb_per_split);
     if (MODE == GEMM1) return p.tile_start[p.g_end] - p.tile_start[p.g_begin];
-    if (MODE == GEMM2R) return p.tile_start[p.E];
+    if (MODE == GEMM2R)
+        return p.tile_start[p.E] + (p.fold_shared ? ceil_div(p.T, TM) * ceil_div(p.d, 256) : 0);
     return ceil_div(p.T, TM) * ceil_div(p.d, 256);
 }
 
@@ -292,6 +298,17 @@ __device__ __forceinline__ int find_group(const int32_t* ts, int lo, int hi, int
         else hi = mid;
     }
     return lo;
+}
+
+// Banded raster inside a group of mt x nt tiles: bands of up to gm M-tiles; inside a band the
+// M-tile index runs fastest, then N.  CTAs working at the same time then share a few A row
+// blocks and sweep the B tiles of one band, which keeps both in L2.
+__device__ __forceinline__ void band_mn(int local, int mt, int nt, int gm, int& m, int& n) {
+    const int band = local / (gm * nt);
+    const int rem = local - band * gm * nt;
+    const int rows = min(gm, mt - band * gm);
+    n = rem / rows;
+    m = band * gm + rem % rows;
 }
 
 template <int MODE, bool PAIR>
@@ -317,9 +334,20 @@ __device__ __forceinline__ Tile decode(const Params& p, int t) {
         x.rows = shared ? p.T : p.offsets[g + 1] - p.offsets[g];
         x.row0 = shared ? 0 : p.offsets[g];
         const int mt = ceil_div(x.rows, TM);
-        x.m0 = (local % mt) * TM;
-        x.n0 = (local / mt) * 128;
+        int m, n;
+        band_mn(local, mt, ceil_div(shared ? p.Is : p.I, 128), p.group_m, m, n);
+        x.m0 = m * TM;
+        x.n0 = n * 128;
         x.num_kb = ceil_div(p.d, BK);
+    } else if (MODE == GEMM2R && t >= p.tile_start[p.E]) {
+        // shared-expert tile (fold_shared): all K_s experts accumulated along K
+        const int mt = ceil_div(p.T, TM);
+        x.g = -1; x.rows = p.T; x.row0 = 0;
+        int m, n;
+        band_mn(t - p.tile_start[p.E], mt, ceil_div(p.d, 256), p.group_m, m, n);
+        x.m0 = m * TM;
+        x.n0 = n * 256;
+        x.num_kb = p.Ks * ceil_div(p.Is, BK);
     } else if (MODE == GEMM2R) {
         const int e = find_group(p.tile_start, 0, p.E, t);
         const int local = t - p.tile_start[e];
@@ -327,14 +355,18 @@ __device__ __forceinline__ Tile decode(const Params& p, int t) {
         x.rows = p.offsets[e + 1] - p.offsets[e];
         x.row0 = p.offsets[e];
         const int mt = ceil_div(x.rows, TM);
-        x.m0 = (local % mt) * TM;
-        x.n0 = (local / mt) * 256;
+        int m, n;
+        band_mn(local, mt, ceil_div(p.d, 256), p.group_m, m, n);
+        x.m0 = m * TM;
+        x.n0 = n * 256;
         x.num_kb = ceil_div(p.I, BK);
     } else {
         const int mt = ceil_div(p.T, TM);
         x.g = 0; x.rows = p.T; x.row0 = 0;
-        x.m0 = (t % mt) * TM;
-        x.n0 = (t / mt) * 256;
+        int m, n;
+        band_mn(t, mt, ceil_div(p.d, 256), p.group_m, m, n);
+        x.m0 = m * TM;
+        x.n0 = n * 256;
         x.num_kb = p.Ks * ceil_div(p.Is, BK);
     }
     return x;
@@ -616,9 +648,14 @@ __global__ void __launch_bounds__(THREADS, 1) moe_tc_kernel(const __grid_constan
                             const int e = shared ? x.g - p.E : x.g;
                             tma_load_2d_pair(a_dst, &p.tmA[shared ? 1 : 0], fb, kb * BK, x.row0 + x.m0 + arow);
                             tma_load_3d_pair(b_dst, &p.tmB[(shared ? 2 : 0) + (int)rank], fb, kb * BK, x.n0, e);
-                        } else if (MODE == GEMM2R) {
+                        } else if (MODE == GEMM2R && x.g >= 0) {
                             tma_load_2d_pair(a_dst, &p.tmA[0], fb, kb * BK, x.row0 + x.m0 + arow);
                             tma_load_3d_pair(b_dst, &p.tmB[0], fb, kb * BK, x.n0 + arow, x.g);
+                        } else if (MODE == GEMM2R) {
+                            const int kbs = ceil_div(p.Is, BK);
+                            const int s = kb / kbs, kk = kb % kbs;
+                            tma_load_3d_pair(a_dst, &p.tmA[1], fb, kk * BK, x.m0 + arow, s);
+                            tma_load_3d_pair(b_dst, &p.tmB[1], fb, kk * BK, x.n0 + arow, s);
                         } else {
                             const int kbs = ceil_div(p.Is, BK);
                             const int s = kb / kbs, kk = kb % kbs;
@@ -633,9 +670,14 @@ __global__ void __launch_bounds__(THREADS, 1) moe_tc_kernel(const __grid_constan
                             tma_load_2d(a_dst, &p.tmA[shared ? 1 : 0], fb, kb * BK, x.row0 + x.m0);
                             tma_load_3d(b_dst, &p.tmB[shared ? 2 : 0], fb, kb * BK, x.n0, e);
                             tma_load_3d(b_dst + B_BYTES / 2, &p.tmB[shared ? 3 : 1], fb, kb * BK, x.n0, e);
-                        } else if (MODE == GEMM2R) {
+                        } else if (MODE == GEMM2R && x.g >= 0) {
                             tma_load_2d(a_dst, &p.tmA[0], fb, kb * BK, x.row0 + x.m0);
                             tma_load_3d(b_dst, &p.tmB[0], fb, kb * BK, x.n0, x.g);
+                        } else if (MODE == GEMM2R) {
+                            const int kbs = ceil_div(p.Is, BK);
+                            const int s = kb / kbs, kk = kb % kbs;
+                            tma_load_3d(a_dst, &p.tmA[1], fb, kk * BK, x.m0, s);
+                            tma_load_3d(b_dst, &p.tmB[1], fb, kk * BK, x.n0, s);
                         } else {
                             const int kbs = ceil_div(p.Is, BK);
                             const int s = kb / kbs, kk = kb % kbs;
@@ -716,7 +758,8 @@ __global__ void __launch_bounds__(THREADS, 1) moe_tc_kernel(const __grid_constan
             } else if (MODE == GEMM1) {
                 epilogue_gemm1(p, x, tacc, row, half);
             } else if (MODE == GEMM2R) {
-                epilogue_gemm2r(p, x, tacc, row, half);
+                if (x.g >= 0) epilogue_gemm2r(p, x, tacc, row, half);
+                else epilogue_gemm2s(p, x, tacc, row, half);
             } else {
                 epilogue_gemm2s(p, x, tacc, row, half);
             }
@@ -819,6 +862,7 @@ Params base_params(const Dims& D, uint32_t* err) {
     p.T = D.T; p.d = D.d; p.E = D.E; p.I = D.I; p.Is = D.Ks > 0 ? D.Is : 8; p.k = D.k; p.Ks = D.Ks;
     p.S = D.slots();
     p.n_mma = 256;
+    p.group_m = MOE_GROUP_M;
     p.err = err;
     return p;
 }
@@ -920,7 +964,8 @@ cudaError_t launch_tc_gemm1(const Dims& D, const void* x, const void* x_perm, co
 
 cudaError_t launch_tc_gemm2_routed(const Dims& D, const int32_t* offsets, const int32_t* tile_start2,
                                    const float* sorted_gate, const FfnWeights& R, const void* h_r, void* y_sorted,
-                                   uint32_t* err, cudaStream_t stream) {
+                                   const FfnWeights* Sh, const void* h_s, float* sout, uint32_t* err,
+                                   cudaStream_t stream) {
     using namespace tc;
     if (D.T == 0) return cudaSuccess;
     Params p = base_params(D, err);
@@ -929,11 +974,19 @@ cudaError_t launch_tc_gemm2_routed(const Dims& D, const int32_t* offsets, const 
     p.sorted_gate = sorted_gate;
     p.b2 = (const __nv_bfloat16*)R.b2;
     p.y = (__nv_bfloat16*)y_sorted;
+    const bool pairs = tc::pairs_for(D);
     bool ok = make_map(&p.tmA[0], h_r, D.I, (uint64_t)D.slots(), 1, BK, BM, false);
-    ok &= make_map(&p.tmB[0], R.w2, D.I, D.d, D.E, BK, tc::pairs_for(D) ? 128 : 256, true);
+    ok &= make_map(&p.tmB[0], R.w2, D.I, D.d, D.E, BK, pairs ? 128 : 256, true);
+    if (Sh && D.Ks > 0 && sout) {
+        p.fold_shared = 1;
+        p.sb2 = (const __nv_bfloat16*)Sh->b2;
+        p.sout = sout;
+        ok &= make_map(&p.tmA[1], h_s, D.Is, D.T, D.Ks, BK, BM, true);
+        ok &= make_map(&p.tmB[1], Sh->w2, D.Is, D.d, D.Ks, BK, pairs ? 128 : 256, true);
+    }
     if (!ok) return cudaErrorInvalidValue;
-    return tc::pairs_for(D) ? launch<GEMM2R, 8, true>(p, num_sms(), stream)
-                         : launch<GEMM2R, 8, false>(p, num_sms(), stream);
+    return pairs ? launch<GEMM2R, 8, true>(p, num_sms(), stream)
+                 : launch<GEMM2R, 8, false>(p, num_sms(), stream);
 }
 
 cudaError_t launch_tc_gemm2_shared(const Dims& D, const FfnWeights& Sh, const void* h_s, float* sout, uint32_t* err,

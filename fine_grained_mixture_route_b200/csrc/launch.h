@@ -90,10 +90,13 @@ cudaError_t launch_router_finish(const Dims& D, const float* partial, int nsplit
 cudaError_t launch_tc_gemm1(const Dims& D, const void* x, const void* x_perm, const int32_t* offsets,
                             const int32_t* tile_start1, const FfnWeights& routed, const FfnWeights& shared,
                             void* h_r, void* h_s, int g_begin, int g_end, uint32_t* err, cudaStream_t stream);
-// routed GEMM2 with the gate (and b2) applied in the epilogue -> y_sorted
+// routed GEMM2 with the gate (and b2) applied in the epilogue -> y_sorted; when shared and
+// sout are given, the shared experts' GEMM2 tiles (-> fp32 sout, their b2 added) follow the
+// routed tiles in the same launch.
 cudaError_t launch_tc_gemm2_routed(const Dims& D, const int32_t* offsets, const int32_t* tile_start2,
                                    const float* sorted_gate, const FfnWeights& routed, const void* h_r,
-                                   void* y_sorted, uint32_t* err, cudaStream_t stream);
+                                   void* y_sorted, const FfnWeights* shared, const void* h_s, float* sout,
+                                   uint32_t* err, cudaStream_t stream);
 // shared GEMM2: all K_s experts accumulated along K, plus their b2 -> fp32 sout [T, d]
 cudaError_t launch_tc_gemm2_shared(const Dims& D, const FfnWeights& shared, const void* h_s, float* sout,
                                    uint32_t* err, cudaStream_t stream);

@@ -124,7 +124,8 @@ moe_status_t do_expert_ffn(const Dims& D, const Layout& L, void* ws, const void*
         MOE_CUDA(launch_gather(D, x, stok, xp, err, st));
         FfnWeights none = {nullptr, nullptr, nullptr, nullptr, nullptr, nullptr};
         MOE_CUDA(launch_tc_gemm1(D, x, xp, offsets, ts1, R, none, at<void>(ws, L.hr), nullptr, 0, D.E, err, st));
-        MOE_CUDA(launch_tc_gemm2_routed(D, offsets, ts2, sgate, R, at<void>(ws, L.hr), y, err, st));
+        MOE_CUDA(launch_tc_gemm2_routed(D, offsets, ts2, sgate, R, at<void>(ws, L.hr), y, nullptr, nullptr, nullptr,
+                                        err, st));
     } else {
         FfnWeights none = {nullptr, nullptr, nullptr, nullptr, nullptr, nullptr};
         MOE_CUDA(launch_simt_gemm1(D, x, offsets, stok, R, none, at<void>(ws, L.hr), nullptr, 0, D.E, err, st));
@@ -168,9 +169,7 @@ MOE_EXPORT int32_t moe_layer_launches(const moe_shape_t* shape) {
     n += 3;                                                         // histogram, scan, scatter
     n += 1;                                                         // tile tables
     if (D.bf16) n += 1;                                             // row gather
-    n += 2;                                                         // GEMM1, GEMM2
-    if (D.bf16 && D.Ks > 0) n += 2;                                 // shared GEMM2, combine
-    else n += 1;                                                    // combine (fused for fp32)
+    n += 3;                                   // GEMM1, GEMM2 (routed + shared tiles), combine
     return n;
 }
 
@@ -335,11 +334,9 @@ moe_status_t layer_forward_impl(const moe_shape_t* shape, const void* x, const v
         if (!mark(4)) return MOE_ERR_CUDA;
         MOE_CUDA(launch_tc_gemm1(D, x, xp, offsets, ts1, R, Sh, hr, hs, 0, D.E + D.Ks, err, st));
         if (!mark(5)) return MOE_ERR_CUDA;
-        MOE_CUDA(launch_tc_gemm2_routed(D, offsets, ts2, sgate, R, hr, y, err, st));
-        if (!mark(6)) return MOE_ERR_CUDA;
         float* sout = D.Ks > 0 ? at<float>(ws, L.sout) : nullptr;
-        if (D.Ks > 0) MOE_CUDA(launch_tc_gemm2_shared(D, Sh, hs, sout, err, st));
-        if (!mark(7)) return MOE_ERR_CUDA;
+        MOE_CUDA(launch_tc_gemm2_routed(D, offsets, ts2, sgate, R, hr, y, D.Ks > 0 ? &Sh : nullptr, hs, sout, err, st));
+        if (!mark(6)) return MOE_ERR_CUDA;
         MOE_CUDA(launch_combine(D, y, slot_of, sout, out, err, st));
     } else {
         if (!mark(4)) return MOE_ERR_CUDA;
@@ -349,9 +346,8 @@ moe_status_t layer_forward_impl(const moe_shape_t* shape, const void* x, const v
         if (!mark(6)) return MOE_ERR_CUDA;
         if (D.Ks > 0) MOE_CUDA(launch_simt_gemm2_shared(D, Sh, hs, y, slot_of, out, err, st));
         else MOE_CUDA(launch_combine(D, y, slot_of, nullptr, out, err, st));
-        if (!mark(7)) return MOE_ERR_CUDA;
     }
-    if (!mark(8)) return MOE_ERR_CUDA;
+    if (!mark(7)) return MOE_ERR_CUDA;
     return MOE_OK;
 }
 

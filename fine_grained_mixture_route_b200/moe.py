@@ -20,8 +20,8 @@ MOE_F32, MOE_BF16 = 0, 1
 EXPORTED = ("moe_workspace_bytes", "moe_layer_launches", "moe_status_string", "moe_version", "moe_check_device_error", "moe_ws_init",
             "moe_route", "moe_permute", "moe_expert_ffn", "moe_combine", "moe_layer_forward",
             "moe_layer_forward_timed", "moe_permute_no_alloc")
-NUM_STAGES = 8
-STAGE_NAMES = ("router", "permute", "plan", "gather", "gemm1_swiglu", "gemm2_gate", "gemm2_shared", "combine")
+NUM_STAGES = 7
+STAGE_NAMES = ("router", "permute", "plan", "gather", "gemm1_swiglu", "gemm2", "combine")
 
 
 class MoeShape(ctypes.Structure):

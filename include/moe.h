@@ -186,12 +186,12 @@ moe_status_t moe_layer_forward(const moe_shape_t* shape, const void* x, const vo
  * cudaEventElapsedTime between neighbours gives each stage's device time.  Stages, in order:
  *   0 router (scores, softmax, top-k)      1 grouping (histogram, scan, scatter)
  *   2 tile tables of the grouped GEMMs     3 row gather of the routed tokens (bf16 only)
- *   4 GEMM1 + SwiGLU (routed and shared)   5 routed GEMM2 with gates
- *   6 shared GEMM2 (bf16; fp32 layers fuse it with the combine here)
- *   7 combine (bf16; empty for fp32 layers)
+ *   4 GEMM1 + SwiGLU (routed and shared)   5 GEMM2: routed with gates, then (bf16) the
+ *                                            shared experts' tiles in the same launch
+ *   6 combine (fp32 layers: shared GEMM2 and combine in one kernel)
  * n_events must be MOE_NUM_STAGES + 1; MOE_ERR_INVALID_ARG otherwise.
  */
-#define MOE_NUM_STAGES 8
+#define MOE_NUM_STAGES 7
 moe_status_t moe_layer_forward_timed(const moe_shape_t* shape, const void* x, const void* centroids,
                                      const moe_ffn_weights_t* routed, const moe_ffn_weights_t* shared,
                                      void* out, int32_t* topk_idx_out, float* topk_gate_out,

@@ -71,8 +71,8 @@ def test_workspace_bytes(lib):
 
 
 def test_launch_count(lib):
-    assert moe.layer_launches(_shape()) == 11          # split-K router at T=256: scores + finish
-    assert moe.layer_launches(_shape(T=16384)) == 10
+    assert moe.layer_launches(_shape()) == 10          # split-K router at T=256: scores + finish
+    assert moe.layer_launches(_shape(T=16384)) == 9
     assert moe.layer_launches(_shape(T=16384, n_shared=0)) == 9
     assert moe.layer_launches(_shape(T=128, d=256, n_experts=16, inter=64, inter_shared=64, top_k=4,
                                      dtype=moe.MOE_F32)) == 8
