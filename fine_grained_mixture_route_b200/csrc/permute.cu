@@ -72,36 +72,41 @@ __global__ void permute_hist_kernel(const int32_t* __restrict__ idx, long long S
 }
 
 // pass 2: counts, offsets, and each block's starting position per expert (in place).  One
-// warp per expert scans that expert's column of block counts 32 blocks at a time.
+// thread per expert walks that expert's column of block counts (consecutive threads read
+// consecutive experts of a block row, so every load is coalesced; loads are unrolled).
 __global__ void permute_scan_kernel(int32_t* __restrict__ block_hist, int nblk, int E,
                                     int32_t* __restrict__ counts, int32_t* __restrict__ offsets) {
     extern __shared__ int sh[];
     int* cnt = sh;               // [E]
     int* warp_sums = sh + E;     // [32]
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
-    for (int e = warp; e < E; e += nwarps) {
-        int carry = 0;
-        for (int b0 = 0; b0 < nblk; b0 += 32) {
-            const int b = b0 + lane;
-            const int c = b < nblk ? block_hist[(size_t)b * E + e] : 0;
-            int incl = c;
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        int run = 0;
+        int b = 0;
+        for (; b + 8 <= nblk; b += 8) {
+            int c[8];
 #pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const int y = __shfl_up_sync(0xffffffffu, incl, o);
-                if (lane >= o) incl += y;
+            for (int i = 0; i < 8; ++i) c[i] = block_hist[(size_t)(b + i) * E + e];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                block_hist[(size_t)(b + i) * E + e] = run;
+                run += c[i];
             }
-            if (b < nblk) block_hist[(size_t)b * E + e] = carry + incl - c;
-            carry += __shfl_sync(0xffffffffu, incl, 31);
         }
-        if (lane == 0) { cnt[e] = carry; counts[e] = carry; }
+        for (; b < nblk; ++b) {
+            const int c = block_hist[(size_t)b * E + e];
+            block_hist[(size_t)b * E + e] = run;
+            run += c;
+        }
+        cnt[e] = run;
+        counts[e] = run;
     }
     __syncthreads();
     const int total = block_exclusive_scan(cnt, E, warp_sums);
-    for (int e = warp; e < E; e += nwarps) {
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        offsets[e] = cnt[e];
         const int base = cnt[e];
-        for (int b = lane; b < nblk; b += 32) block_hist[(size_t)b * E + e] += base;
+        for (int b = 0; b < nblk; ++b) block_hist[(size_t)b * E + e] += base;
     }
-    for (int e = threadIdx.x; e < E; e += blockDim.x) offsets[e] = cnt[e];
     if (threadIdx.x == 0) offsets[E] = total;
 }
 
