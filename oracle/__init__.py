@@ -6,5 +6,5 @@ import this package.  It never imports the CUDA library or its binding.
 from .moe_oracle import (  # noqa: F401
     silu, linear, expert_ffn, swiglu_hidden, route, gates_from_indices, permute, layer,
     linear_macs, linear_params, expert_macs, expert_params, hit_entropy, n_routings,
-    split_expert,
+    split_expert, GATE_SOFTMAX_TOPK, GATE_TOPK_SOFTMAX, GATE_SIGMOID_BIAS,
 )

@@ -12,7 +12,10 @@ What it computes, and where it comes from:
   centroid; s_{i,t} is the softmax of these over all N_m experts; the gate g_{i,t} keeps
   s_{i,t} for the N_r largest and is zero for the rest.  No renormalisation, no scale, no
   router bias.  Ties go to the lower expert index; the picks of a token are ordered by
-  descending score, then ascending index.
+  descending score, then ascending index.  Two variants are selectable (route(), gate_mode):
+  softmax over the top-k logits of a biased router (DeepSeek-V2 explainer §3.1), and a sigmoid
+  gate with a selection-only routing bias (mentioned for DeepSeek-V3 in the report's §6.2; no
+  formula on the pages: PARITY UNPINNED for that variant).
 * Expert FFN (the `Expert` module of "DeepSeek MoE模型优化与未来演进及字节超稀疏内存技术"):
   w2(silu(w1 x) * w3 x) with nn.Linear layout ([out, in]) and a bias on every Linear.
 * Layer output (DeepSeekMoE report §2.3 and §3.1, Eq. 9-11 in prose): the K_s shared experts
@@ -66,48 +69,98 @@ def swiglu_hidden(x: np.ndarray, w1, b1, w3, b3) -> np.ndarray:
 # --------------------------------------------------------------------------------------
 # the router
 # --------------------------------------------------------------------------------------
-def route(x: np.ndarray, centroids: np.ndarray, top_k: int) -> Dict[str, np.ndarray]:
-    """Scores, softmax and top-N_r gates of every token.
+GATE_SOFTMAX_TOPK = 0      # softmax over all experts, keep the top-k probabilities (DeepSeekMoE report §3.1)
+GATE_TOPK_SOFTMAX = 1      # top-k of the (biased) logits, softmax over the k picks (DeepSeek-V2 explainer §3.1)
+GATE_SIGMOID_BIAS = 2      # sigmoid scores, picks by score + routing bias, gates renormalised (parity unpinned)
 
-    Returns z [T,N] logits, s [T,N] softmax, idx [T,k] picks (descending score, ties to the
-    lower index), gate [T,k] = s at the picks, and two near-tie gaps in logit units:
-    `gap` = z_(k) - z_(k+1) (the boundary of the picked set; +inf when k == N) and
-    `gap_order` = the smallest gap between consecutive picks or across the boundary.
+
+def _sigmoid(z):
+    return 1.0 / (1.0 + np.exp(-z))
+
+
+def route(x: np.ndarray, centroids: np.ndarray, top_k: int, gate_mode: int = GATE_SOFTMAX_TOPK,
+          bias: Optional[np.ndarray] = None) -> Dict[str, np.ndarray]:
+    """Scores, picks and gates of every token.
+
+    gate_mode 0 (the DeepSeekMoE report, §3.1): z = x . e_i (+ bias_i when a router bias is given),
+      s = softmax of z over all N_m experts, picks = the N_r largest z (softmax is increasing, so
+      these are the N_r largest s), gate = s at the picks, not renormalised.
+    gate_mode 1 (the `FineGrainedMoE` listing of the DeepSeek-V2 explainer, §3.1, whose router is a
+      Linear layer with a bias): picks = the N_r largest z = x . e_i + bias_i, gate = softmax over
+      the N_r picked logits (the gates of a token sum to 1).
+    gate_mode 2 (the sigmoid gate with aux-loss-free routing bias mentioned for DeepSeek-V3 in the
+      DeepSeekMoE report §6.2; the pages give no formula, so this reading is PARITY UNPINNED):
+      s = sigmoid(x . e_i), picks = the N_r largest s_i + bias_i (the bias steers only the choice),
+      gate = s at the picks divided by their sum.
+
+    Ties go to the lower expert index; picks are ordered by descending selection key.  Returns z,
+    s (softmax, softmax or sigmoid), key (the selection key), idx, gate, and two near-tie gaps of
+    the key: `gap` (k-th vs (k+1)-th; +inf when k == N) and `gap_order` (smallest gap between
+    consecutive picks or across the boundary).
     """
     x = np.asarray(x, dtype=np.float64)
     c = np.asarray(centroids, dtype=np.float64)
     T, N = x.shape[0], c.shape[0]
     if not (1 <= top_k <= N):
         raise ValueError("top_k must be in [1, N_m]")
+    b = np.zeros(N) if bias is None else np.asarray(bias, np.float64)
     z = x @ c.T
-    zmax = z.max(axis=1, keepdims=True)
-    e = np.exp(z - zmax)
-    s = e / e.sum(axis=1, keepdims=True)
-    # stable sort of -z: descending logit, equal logits keep ascending expert index.
-    # softmax is strictly increasing in z, so this is also the order of s.
-    order = np.argsort(-z, axis=1, kind="stable")
+    if gate_mode == GATE_SIGMOID_BIAS:
+        s = _sigmoid(z)
+        key = s + b
+    else:
+        z = z + b
+        zmax = z.max(axis=1, keepdims=True)
+        e = np.exp(z - zmax)
+        s = e / e.sum(axis=1, keepdims=True)
+        key = z
+    # stable sort of -key: descending key, equal keys keep ascending expert index
+    order = np.argsort(-key, axis=1, kind="stable")
     idx = order[:, :top_k]
-    gate = np.take_along_axis(s, idx, axis=1)
-    zs = np.take_along_axis(z, order, axis=1)
+    if gate_mode == GATE_SOFTMAX_TOPK:
+        gate = np.take_along_axis(s, idx, axis=1)
+    elif gate_mode == GATE_TOPK_SOFTMAX:
+        zp = np.take_along_axis(z, idx, axis=1)
+        ep = np.exp(zp - zp.max(axis=1, keepdims=True))
+        gate = ep / ep.sum(axis=1, keepdims=True)
+    elif gate_mode == GATE_SIGMOID_BIAS:
+        sp = np.take_along_axis(s, idx, axis=1)
+        gate = sp / sp.sum(axis=1, keepdims=True)
+    else:
+        raise ValueError("unknown gate_mode")
+    ks = np.take_along_axis(key, order, axis=1)
     if top_k < N:
-        gap = zs[:, top_k - 1] - zs[:, top_k]
-        diffs = zs[:, :top_k] - zs[:, 1:top_k + 1]
+        gap = ks[:, top_k - 1] - ks[:, top_k]
+        diffs = ks[:, :top_k] - ks[:, 1:top_k + 1]
     else:
         gap = np.full(T, np.inf)
-        diffs = zs[:, :top_k - 1] - zs[:, 1:top_k]
+        diffs = ks[:, :top_k - 1] - ks[:, 1:top_k]
     gap_order = diffs.min(axis=1) if diffs.shape[1] > 0 else np.full(T, np.inf)
-    return {"z": z, "s": s, "idx": idx.astype(np.int64), "gate": gate,
+    return {"z": z, "s": s, "key": key, "idx": idx.astype(np.int64), "gate": gate,
             "gap": gap, "gap_order": gap_order}
 
 
-def gates_from_indices(x: np.ndarray, centroids: np.ndarray, idx: np.ndarray) -> np.ndarray:
-    """s_{i,t} of the softmax over all experts, read at given picks (used when a near-tie
-    lets another valid pick set stand in for the oracle's own)."""
-    z = np.asarray(x, np.float64) @ np.asarray(centroids, np.float64).T
+def gates_from_indices(x: np.ndarray, centroids: np.ndarray, idx: np.ndarray, gate_mode: int = GATE_SOFTMAX_TOPK,
+                       bias: Optional[np.ndarray] = None) -> np.ndarray:
+    """The gates the given picks receive under gate_mode (used where a near-tie lets another
+    valid pick set stand in for the oracle's own)."""
+    x = np.asarray(x, np.float64)
+    c = np.asarray(centroids, np.float64)
+    idx = np.asarray(idx, np.int64)
+    b = np.zeros(c.shape[0]) if bias is None else np.asarray(bias, np.float64)
+    z = x @ c.T
+    if gate_mode == GATE_SIGMOID_BIAS:
+        sp = np.take_along_axis(_sigmoid(z), idx, axis=1)
+        return sp / sp.sum(axis=1, keepdims=True)
+    z = z + b
+    if gate_mode == GATE_TOPK_SOFTMAX:
+        zp = np.take_along_axis(z, idx, axis=1)
+        ep = np.exp(zp - zp.max(axis=1, keepdims=True))
+        return ep / ep.sum(axis=1, keepdims=True)
     zmax = z.max(axis=1, keepdims=True)
     e = np.exp(z - zmax)
     s = e / e.sum(axis=1, keepdims=True)
-    return np.take_along_axis(s, np.asarray(idx, np.int64), axis=1)
+    return np.take_along_axis(s, idx, axis=1)
 
 
 # --------------------------------------------------------------------------------------
@@ -148,13 +201,15 @@ def _expert(src: ExpertSource, e: int) -> Weights:
 
 def layer(x: np.ndarray, centroids: np.ndarray, routed: ExpertSource, n_experts: int, top_k: int,
           shared: Optional[ExpertSource] = None, n_shared: int = 0,
-          idx_override: Optional[np.ndarray] = None, keep_hidden: bool = False) -> Dict[str, np.ndarray]:
+          idx_override: Optional[np.ndarray] = None, keep_hidden: bool = False,
+          gate_mode: int = GATE_SOFTMAX_TOPK, router_bias: Optional[np.ndarray] = None) -> Dict[str, np.ndarray]:
     """The DeepSeekMoE layer forward in fp64.
 
     routed / shared: either dicts of stacked arrays (w1,b1,w3,b3,w2,b2 indexed by expert) or
     a callable e -> dict of one expert's arrays (used to stream large weight sets).
     idx_override: route with these picks instead of the oracle's own (gates are then the
-    softmax read at those picks); used where a near-tie makes another pick set valid.
+    gates those picks receive); used where a near-tie makes another pick set valid.
+    gate_mode / router_bias: see route().
 
     Returns out [T,d], routed_sum, shared_sum, idx, gate, gap, gap_order, counts, and
     Y [T*k, d] = gate * Expert_e(x_t) per slot (slot = t*k + j); with keep_hidden also
@@ -162,10 +217,10 @@ def layer(x: np.ndarray, centroids: np.ndarray, routed: ExpertSource, n_experts:
     """
     x = np.asarray(x, np.float64)
     T, d = x.shape
-    r = route(x, centroids, top_k)
+    r = route(x, centroids, top_k, gate_mode, router_bias)
     if idx_override is not None:
         idx = np.asarray(idx_override, np.int64)
-        gate = gates_from_indices(x, centroids, idx)
+        gate = gates_from_indices(x, centroids, idx, gate_mode, router_bias)
     else:
         idx, gate = r["idx"], r["gate"]
     k = top_k

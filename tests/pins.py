@@ -290,6 +290,68 @@ def check_permute(O):
             assert p["slot_of"][slot] == pos
 
 
+# ----------------------------------------------------------------------------- router variants
+def check_gate_modes(O):
+    """Router variants.  Mode 1 (top-k of a biased router's logits, softmax over the picks)
+    against torch.topk + F.softmax in float64, closed forms and hand-set logits; mode 2 (sigmoid
+    gate with a selection-only bias; the formula is a reading, not on the pages) against
+    scipy.special.expit and brute-force selection."""
+    rng = _rng(11)
+    T, d, N, k = 30, 12, 9, 3
+    x = rng.normal(0, 1, (T, d))
+    c = rng.normal(0, 0.6, (N, d))
+    b = rng.normal(0, 0.5, N)
+    # mode 1 against the listing's torch ops
+    r1 = O.route(x, c, k, O.GATE_TOPK_SOFTMAX, b)
+    with torch.no_grad():
+        scores = torch.from_numpy(x) @ torch.from_numpy(c).T + torch.from_numpy(b)
+        logits, idx = torch.topk(scores, k, dim=-1)
+        w = F.softmax(logits, dim=-1)
+    assert np.array_equal(r1["idx"], idx.numpy())
+    assert np.allclose(r1["gate"], w.numpy(), rtol=1e-13, atol=0)
+    assert np.allclose(r1["gate"].sum(1), 1.0, rtol=1e-14, atol=0)
+    assert np.allclose(O.gates_from_indices(x, c, r1["idx"], O.GATE_TOPK_SOFTMAX, b), r1["gate"], rtol=1e-14, atol=0)
+    # k = N: the plain softmax of the biased logits, in descending order; k = 1: gate 1
+    rN = O.route(x, c, N, O.GATE_TOPK_SOFTMAX, b)
+    sN = scipy.special.softmax(x @ c.T + b, axis=1)
+    assert np.allclose(rN["gate"], np.take_along_axis(sN, rN["idx"], 1), rtol=1e-12, atol=0)
+    assert np.allclose(O.route(x, c, 1, O.GATE_TOPK_SOFTMAX, b)["gate"], 1.0, rtol=0, atol=1e-15)
+    # hand-set logits with a bias that reorders them
+    logits_ = np.array([0.3, -1.0, 2.0, 2.0, 0.1, 5.0])
+    cx = np.zeros((6, 3)); cx[:, 0] = logits_
+    bias_ = np.array([0.0, 0.0, 0.0, 0.5, 0.0, -10.0])
+    r4 = O.route(np.array([[1.0, 0.0, 0.0]]), cx, 3, O.GATE_TOPK_SOFTMAX, bias_)
+    assert r4["idx"][0].tolist() == [3, 2, 0]
+    ex = [math.exp(v) for v in (2.5, 2.0, 0.3)]
+    assert np.allclose(r4["gate"][0], [e / sum(ex) for e in ex], rtol=1e-14, atol=0)
+    # mode 0 with a bias is the report's gate on the biased logits
+    r0 = O.route(x, c, k, O.GATE_SOFTMAX_TOPK, b)
+    s0 = scipy.special.softmax(x @ c.T + b, axis=1)
+    assert np.allclose(r0["gate"], np.take_along_axis(s0, r0["idx"], 1), rtol=1e-12, atol=0)
+    # mode 2: picks maximise sum of (sigmoid + bias) over subsets; gates = sigmoid at picks / sum
+    r2 = O.route(x, c, k, O.GATE_SIGMOID_BIAS, b)
+    sg = scipy.special.expit(x @ c.T)
+    key = sg + b
+    for t in range(T):
+        subs = list(itertools.combinations(range(N), k))
+        best = subs[int(np.argmax([key[t, list(sb)].sum() for sb in subs]))]
+        assert set(r2["idx"][t].tolist()) == set(best)
+        sp = sg[t, r2["idx"][t]]
+        assert np.allclose(r2["gate"][t], sp / sp.sum(), rtol=1e-13, atol=0)
+    assert (np.diff(key[np.arange(T)[:, None], r2["idx"]], axis=1) <= 0).all()
+    assert np.allclose(O.gates_from_indices(x, c, r2["idx"], O.GATE_SIGMOID_BIAS, b), r2["gate"], rtol=1e-14, atol=0)
+    # the bias steers only the choice: with zero bias mode 2 picks the same experts as mode 0
+    assert np.array_equal(O.route(x, c, k, O.GATE_SIGMOID_BIAS)["idx"], O.route(x, c, k)["idx"])
+    # layer-level: gates summing to 1 make the routed part a convex mix of the picked experts
+    experts = [_rand_expert(rng, d, 5) for _ in range(N)]
+    res = O.layer(x, c, _stack(experts), N, k, gate_mode=O.GATE_TOPK_SOFTMAX, router_bias=b)
+    want = np.zeros_like(res["out"])
+    for t in range(T):
+        for j, e in enumerate(r1["idx"][t]):
+            want[t] += r1["gate"][t, j] * torch_expert(experts[e], x[t:t + 1])[0]
+    assert np.allclose(res["out"], want, rtol=1e-11, atol=1e-11)
+
+
 ALL_CHECKS = [check_ptflops_printout, check_combinations, check_textbook_single_expert,
               check_gate_invariants, check_bruteforce_routing, check_split_identity,
-              check_shared_bypasses_router, check_hit_entropy, check_permute]
+              check_shared_bypasses_router, check_hit_entropy, check_permute, check_gate_modes]

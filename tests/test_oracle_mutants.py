@@ -28,15 +28,15 @@ def _linear_bias_sign(x, w, b):                # wrong sign on the bias
     return y
 
 
-def _route_renormalised(x, c, k):              # softmax over the picks only
-    r = _orig["route"](x, c, k)
+def _route_renormalised(x, c, k, gate_mode=0, bias=None):   # softmax over the picks only
+    r = _orig["route"](x, c, k, gate_mode, bias)
     r = dict(r)
     r["gate"] = r["gate"] / r["gate"].sum(axis=1, keepdims=True)
     return r
 
 
-def _route_lowest(x, c, k):                    # picks the smallest scores
-    r = _orig["route"](-np.asarray(x), c, k)
+def _route_lowest(x, c, k, gate_mode=0, bias=None):         # picks the smallest scores
+    r = _orig["route"](-np.asarray(x), c, k, gate_mode, bias)
     r = dict(r)
     z = np.asarray(x, np.float64) @ np.asarray(c, np.float64).T
     s = np.exp(z - z.max(1, keepdims=True)); s /= s.sum(1, keepdims=True)
@@ -44,10 +44,10 @@ def _route_lowest(x, c, k):                    # picks the smallest scores
     return r
 
 
-def _route_ties_high(x, c, k):                 # ties resolved toward the higher index
+def _route_ties_high(x, c, k, gate_mode=0, bias=None):      # ties resolved toward the higher index
     z = np.asarray(x, np.float64) @ np.asarray(c, np.float64).T
     N = z.shape[1]
-    r = _orig["route"](x, np.asarray(c)[::-1], k)
+    r = _orig["route"](x, np.asarray(c)[::-1], k, gate_mode, None if bias is None else np.asarray(bias)[::-1])
     r = dict(r)
     r["idx"] = (N - 1) - r["idx"]
     s = np.exp(z - z.max(1, keepdims=True)); s /= s.sum(1, keepdims=True)
