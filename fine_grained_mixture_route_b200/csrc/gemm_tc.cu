@@ -86,6 +86,8 @@ struct Params {
     float* sout;               // GEMM2S: fp32 shared-expert output [T][d]
     int32_t* idx_out;
     float* gate_out;
+    const float* router_bias;  // ROUTER / ROUTERP: optional per-expert bias [E]
+    int gate_mode;             // ROUTER: moe_gate_mode_t
     float* partial;            // ROUTERP: [nsplit][T][E] fp32 partial logits
     int kb_per_split;          // ROUTERP: K blocks per split
     int group_m;               // tile raster: bands of group_m M-tiles swept across all N-tiles
@@ -374,53 +376,86 @@ __device__ __forceinline__ Tile decode(const Params& p, int t) {
 
 // ------------------------------------------------------------------------------ epilogues
 // Top-k insertion keeping (value desc, index asc); candidates arrive in ascending index.
+// Top-k insertion keeping (key desc, index asc) with a payload; candidates arrive in ascending
+// index, so an equal key never displaces an earlier (lower-index) entry.
 template <int KMAX>
-__device__ __forceinline__ void topk_insert(float (&tv)[KMAX], int (&ti)[KMAX], float v, int e) {
+__device__ __forceinline__ void topk_insert(float (&tv)[KMAX], int (&ti)[KMAX], float (&tp)[KMAX], float v, int e,
+                                            float payload) {
     if (v > tv[KMAX - 1]) {
         tv[KMAX - 1] = v;
         ti[KMAX - 1] = e;
+        tp[KMAX - 1] = payload;
 #pragma unroll
         for (int j = KMAX - 1; j > 0; --j) {
             if (tv[j] > tv[j - 1]) {
                 float a = tv[j]; tv[j] = tv[j - 1]; tv[j - 1] = a;
                 int b = ti[j]; ti[j] = ti[j - 1]; ti[j - 1] = b;
+                float c = tp[j]; tp[j] = tp[j - 1]; tp[j - 1] = c;
             }
         }
     }
 }
 
+// Router epilogue: the thread owning a token row reads its N_m logits from TMEM.  Selection key
+// z + bias (gate modes 0, 1) or sigmoid(z) + bias (mode 2); gates: mode 0 the softmax of z + bias
+// over all experts at the picks (a second pass sums the exponentials), mode 1 the softmax over
+// the k picked keys, mode 2 the picks' sigmoids divided by their sum.
 template <int KMAX>
 __device__ __forceinline__ void epilogue_router(const Params& p, const Tile& x, uint32_t tacc, int row) {
-    float tv[KMAX];
+    float tv[KMAX], tp[KMAX];
     int ti[KMAX];
 #pragma unroll
-    for (int j = 0; j < KMAX; ++j) { tv[j] = -INFINITY; ti[j] = 0; }
+    for (int j = 0; j < KMAX; ++j) { tv[j] = -INFINITY; ti[j] = 0; tp[j] = 0.f; }
+    const int mode = p.gate_mode;
     for (int c0 = 0; c0 < p.n_mma; c0 += 16) {
         uint32_t r[16];
         tmem_ld16(tacc + c0, r);
         tmem_wait_ld();
 #pragma unroll
-        for (int j = 0; j < 16; ++j)
-            if (c0 + j < p.E) topk_insert<KMAX>(tv, ti, __uint_as_float(r[j]), c0 + j);
+        for (int j = 0; j < 16; ++j) {
+            const int e = c0 + j;
+            if (e < p.E) {
+                const float z = __uint_as_float(r[j]);
+                const float bb = p.router_bias ? p.router_bias[e] : 0.f;
+                if (mode == 2) {
+                    const float sg = 1.0f / (1.0f + expf(-z));
+                    topk_insert<KMAX>(tv, ti, tp, sg + bb, e, sg);
+                } else {
+                    topk_insert<KMAX>(tv, ti, tp, z + bb, e, z + bb);
+                }
+            }
+        }
     }
-    const float zmax = tv[0];
-    float s = 0.f;
-    for (int c0 = 0; c0 < p.n_mma; c0 += 16) {
-        uint32_t r[16];
-        tmem_ld16(tacc + c0, r);
-        tmem_wait_ld();
+    float gsum = 0.f;
+    if (mode == 0) {
+        const float zmax = tv[0];
+        for (int c0 = 0; c0 < p.n_mma; c0 += 16) {
+            uint32_t r[16];
+            tmem_ld16(tacc + c0, r);
+            tmem_wait_ld();
 #pragma unroll
-        for (int j = 0; j < 16; ++j)
-            if (c0 + j < p.E) s += expf(__uint_as_float(r[j]) - zmax);
+            for (int j = 0; j < 16; ++j)
+                if (c0 + j < p.E)
+                    gsum += expf(__uint_as_float(r[j]) + (p.router_bias ? p.router_bias[c0 + j] : 0.f) - zmax);
+        }
     }
     const int t = x.m0 + row;
     if (t < p.T) {
-        const float inv = 1.0f / s;
+        float g[KMAX];
+        float norm = 0.f;
+#pragma unroll
+        for (int j = 0; j < KMAX; ++j) {
+            if (mode == 0) g[j] = expf(tp[j] - tv[0]) / gsum;
+            else if (mode == 1) g[j] = expf(tp[j] - tp[0]);
+            else g[j] = tp[j];
+            if (j < p.k) norm += g[j];
+        }
+        const float rn = mode == 0 ? 1.f : 1.0f / norm;
 #pragma unroll
         for (int j = 0; j < KMAX; ++j) {
             if (j < p.k) {
                 p.idx_out[(size_t)t * p.k + j] = ti[j];
-                p.gate_out[(size_t)t * p.k + j] = expf(tv[j] - zmax) * inv;
+                p.gate_out[(size_t)t * p.k + j] = g[j] * rn;
             }
         }
     }
@@ -909,14 +944,16 @@ int router_splits(const Dims& D) {
     return ceil_div(kbt, per < 4 ? 4 : per);
 }
 
-cudaError_t launch_tc_router(const Dims& D, const void* x, const void* centroids, int32_t* idx, float* gate,
-                             float* partial, uint32_t* err, cudaStream_t stream) {
+cudaError_t launch_tc_router(const Dims& D, const void* x, const void* centroids, const float* bias, int32_t* idx,
+                             float* gate, float* partial, uint32_t* err, cudaStream_t stream) {
     using namespace tc;
     if (D.T == 0) return cudaSuccess;
     Params p = base_params(D, err);
     p.n_mma = D.E;
     p.idx_out = idx;
     p.gate_out = gate;
+    p.router_bias = bias;
+    p.gate_mode = D.gate_mode;
     if (!make_map(&p.tmA[0], x, D.d, D.T, 1, BK, BM, false)) return cudaErrorInvalidValue;
     if (!make_map(&p.tmB[0], centroids, D.d, D.E, 1, BK, D.E, false)) return cudaErrorInvalidValue;
     const int mt = ceil_div(D.T, BM);
@@ -928,7 +965,7 @@ cudaError_t launch_tc_router(const Dims& D, const void* x, const void* centroids
         const int tiles = mt * ceil_div(kbt, p.kb_per_split);
         cudaError_t e = launch<ROUTERP, 8>(p, tiles, stream);
         if (e != cudaSuccess) return e;
-        return launch_router_finish(D, partial, ceil_div(kbt, p.kb_per_split), idx, gate, stream);
+        return launch_router_finish(D, partial, ceil_div(kbt, p.kb_per_split), bias, idx, gate, stream);
     }
     return D.k <= 8 ? launch<ROUTER, 8>(p, mt, stream) : launch<ROUTER, 32>(p, mt, stream);
 }

@@ -14,14 +14,15 @@ struct Dims {
     int T, d, E, I, k, Ks, Is;
     bool bias;
     bool bf16;
+    int gate_mode = 0;     // moe_gate_mode_t
     long long slots() const { return (long long)T * k; }
 };
 
 // ---- router ---------------------------------------------------------------------------
 // CUDA-core router for any dtype and N_m <= 1024: block-tiled scores, then one warp per
 // token for softmax and top-k.
-cudaError_t launch_router_simt(const Dims& D, const void* x, const void* centroids, int32_t* idx,
-                               float* gate, cudaStream_t stream);
+cudaError_t launch_router_simt(const Dims& D, const void* x, const void* centroids, const float* bias,
+                               int32_t* idx, float* gate, cudaStream_t stream);
 
 // ---- per-expert token lists -----------------------------------------------------------
 constexpr int PERMUTE_CHUNK = 1024;  // slots per histogram / scatter block
@@ -82,10 +83,10 @@ inline size_t router_partial_bytes(const Dims& D) {
     const int n = router_splits(D);
     return n > 1 ? (size_t)n * D.T * D.E * sizeof(float) : 0;
 }
-cudaError_t launch_tc_router(const Dims& D, const void* x, const void* centroids, int32_t* idx, float* gate,
-                             float* partial, uint32_t* err, cudaStream_t stream);
-cudaError_t launch_router_finish(const Dims& D, const float* partial, int nsplit, int32_t* idx, float* gate,
-                                 cudaStream_t stream);
+cudaError_t launch_tc_router(const Dims& D, const void* x, const void* centroids, const float* bias, int32_t* idx,
+                             float* gate, float* partial, uint32_t* err, cudaStream_t stream);
+cudaError_t launch_router_finish(const Dims& D, const float* partial, int nsplit, const float* bias, int32_t* idx,
+                                 float* gate, cudaStream_t stream);
 // GEMM1 + SwiGLU over groups [g_begin, g_end): A rows from x_perm (routed) or x (shared).
 cudaError_t launch_tc_gemm1(const Dims& D, const void* x, const void* x_perm, const int32_t* offsets,
                             const int32_t* tile_start1, const FfnWeights& routed, const FfnWeights& shared,

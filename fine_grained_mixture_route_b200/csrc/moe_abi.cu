@@ -52,6 +52,7 @@ moe_status_t to_dims(const moe_shape_t* s, Dims* D) {
     if (s->top_k > s->n_experts) return MOE_ERR_INVALID_ARG;
     if (s->n_shared > 0 && s->inter_shared < 1) return MOE_ERR_INVALID_ARG;
     if (s->has_bias != 0 && s->has_bias != 1) return MOE_ERR_INVALID_ARG;
+    if (s->gate_mode < MOE_GATE_SOFTMAX_TOPK || s->gate_mode > MOE_GATE_SIGMOID_BIAS) return MOE_ERR_INVALID_ARG;
     if ((long long)s->T * s->top_k >= (1LL << 31)) return MOE_ERR_UNSUPPORTED;
     if (s->n_experts > 1024 || s->top_k > 32 || s->n_shared > 16) return MOE_ERR_UNSUPPORTED;
     if (s->dtype == MOE_BF16) {
@@ -60,6 +61,7 @@ moe_status_t to_dims(const moe_shape_t* s, Dims* D) {
     D->T = s->T; D->d = s->d; D->E = s->n_experts; D->I = s->inter; D->k = s->top_k;
     D->Ks = s->n_shared; D->Is = s->n_shared > 0 ? s->inter_shared : 0;
     D->bias = s->has_bias != 0; D->bf16 = s->dtype == MOE_BF16;
+    D->gate_mode = s->gate_mode;
     return MOE_OK;
 }
 
@@ -103,11 +105,11 @@ FfnWeights to_ffn(const moe_ffn_weights_t* w) {
     return f;
 }
 
-moe_status_t do_route(const Dims& D, const void* x, const void* c, int32_t* idx, float* gate, float* partial,
-                      uint32_t* err, cudaStream_t st) {
+moe_status_t do_route(const Dims& D, const void* x, const void* c, const float* bias, int32_t* idx, float* gate,
+                      float* partial, uint32_t* err, cudaStream_t st) {
     if (D.T == 0) return MOE_OK;
-    if (tc_router_supported(D)) MOE_CUDA(launch_tc_router(D, x, c, idx, gate, partial, err, st));
-    else MOE_CUDA(launch_router_simt(D, x, c, idx, gate, st));
+    if (tc_router_supported(D)) MOE_CUDA(launch_tc_router(D, x, c, bias, idx, gate, partial, err, st));
+    else MOE_CUDA(launch_router_simt(D, x, c, bias, idx, gate, st));
     return MOE_OK;
 }
 
@@ -196,8 +198,9 @@ MOE_EXPORT moe_status_t moe_check_device_error(void* ws, size_t ws_bytes, moe_st
     return MOE_OK;
 }
 
-MOE_EXPORT moe_status_t moe_route(const moe_shape_t* shape, const void* x, const void* centroids, int32_t* topk_idx,
-                                  float* topk_gate, void* ws, size_t ws_bytes, moe_stream_t stream) {
+MOE_EXPORT moe_status_t moe_route(const moe_shape_t* shape, const void* x, const void* centroids,
+                                  const float* router_bias, int32_t* topk_idx, float* topk_gate, void* ws,
+                                  size_t ws_bytes, moe_stream_t stream) {
     Dims D;
     MOE_TRY(to_dims(shape, &D));
     if (!x || !centroids || !topk_idx || !topk_gate) return MOE_ERR_INVALID_ARG;
@@ -206,8 +209,8 @@ MOE_EXPORT moe_status_t moe_route(const moe_shape_t* shape, const void* x, const
     MOE_TRY(check_device());
     cudaGetLastError();
     const Layout L = layout(D);
-    return do_route(D, x, centroids, topk_idx, topk_gate, at<float>(ws, L.rpart), at<uint32_t>(ws, L.err),
-                    (cudaStream_t)stream);
+    return do_route(D, x, centroids, router_bias, topk_idx, topk_gate, at<float>(ws, L.rpart),
+                    at<uint32_t>(ws, L.err), (cudaStream_t)stream);
 }
 
 MOE_EXPORT moe_status_t moe_permute(const moe_shape_t* shape, const int32_t* topk_idx, const float* topk_gate,
@@ -291,7 +294,7 @@ namespace {
 // The whole layer; when `ev` is non-NULL, ev[i] is recorded on the stream before stage i
 // and ev[MOE_NUM_STAGES] after the last one.
 moe_status_t layer_forward_impl(const moe_shape_t* shape, const void* x, const void* centroids,
-                                const moe_ffn_weights_t* routed, const moe_ffn_weights_t* shared, void* out,
+                                const float* router_bias, const moe_ffn_weights_t* routed, const moe_ffn_weights_t* shared, void* out,
                                 int32_t* topk_idx_out, float* topk_gate_out, int32_t* counts_out, void* ws,
                                 size_t ws_bytes, cudaStream_t st, cudaEvent_t const* ev) {
     Dims D;
@@ -322,7 +325,7 @@ moe_status_t layer_forward_impl(const moe_shape_t* shape, const void* x, const v
     auto mark = [&](int i) -> bool { return !ev || cudaEventRecord(ev[i], st) == cudaSuccess; };
 
     if (!mark(0)) return MOE_ERR_CUDA;
-    MOE_TRY(do_route(D, x, centroids, idx, gate, at<float>(ws, L.rpart), err, st));
+    MOE_TRY(do_route(D, x, centroids, router_bias, idx, gate, at<float>(ws, L.rpart), err, st));
     if (!mark(1)) return MOE_ERR_CUDA;
     MOE_CUDA(launch_permute(D, idx, gate, counts, offsets, stok, sgate, slot_of, at<int32_t>(ws, L.hist), err, st));
     if (!mark(2)) return MOE_ERR_CUDA;
@@ -357,23 +360,24 @@ moe_status_t layer_forward_impl(const moe_shape_t* shape, const void* x, const v
 extern "C" {
 
 MOE_EXPORT moe_status_t moe_layer_forward(const moe_shape_t* shape, const void* x, const void* centroids,
-                                          const moe_ffn_weights_t* routed, const moe_ffn_weights_t* shared, void* out,
+                                          const float* router_bias, const moe_ffn_weights_t* routed, const moe_ffn_weights_t* shared, void* out,
                                           int32_t* topk_idx_out, float* topk_gate_out, int32_t* counts_out, void* ws,
                                           size_t ws_bytes, moe_stream_t stream) {
-    return layer_forward_impl(shape, x, centroids, routed, shared, out, topk_idx_out, topk_gate_out, counts_out, ws,
-                              ws_bytes, (cudaStream_t)stream, nullptr);
+    return layer_forward_impl(shape, x, centroids, router_bias, routed, shared, out, topk_idx_out, topk_gate_out,
+                              counts_out, ws, ws_bytes, (cudaStream_t)stream, nullptr);
 }
 
 MOE_EXPORT moe_status_t moe_layer_forward_timed(const moe_shape_t* shape, const void* x, const void* centroids,
-                                                const moe_ffn_weights_t* routed, const moe_ffn_weights_t* shared,
+                                                const float* router_bias, const moe_ffn_weights_t* routed, const moe_ffn_weights_t* shared,
                                                 void* out, int32_t* topk_idx_out, float* topk_gate_out,
                                                 int32_t* counts_out, void* ws, size_t ws_bytes, moe_stream_t stream,
                                                 void* const* stage_events, int32_t n_events) {
     if (!stage_events || n_events != MOE_NUM_STAGES + 1) return MOE_ERR_INVALID_ARG;
     for (int i = 0; i < n_events; ++i)
         if (!stage_events[i]) return MOE_ERR_INVALID_ARG;
-    return layer_forward_impl(shape, x, centroids, routed, shared, out, topk_idx_out, topk_gate_out, counts_out, ws,
-                              ws_bytes, (cudaStream_t)stream, reinterpret_cast<cudaEvent_t const*>(stage_events));
+    return layer_forward_impl(shape, x, centroids, router_bias, routed, shared, out, topk_idx_out, topk_gate_out,
+                              counts_out, ws, ws_bytes, (cudaStream_t)stream,
+                              reinterpret_cast<cudaEvent_t const*>(stage_events));
 }
 
 }  // extern "C"

@@ -1,6 +1,8 @@
 // CUDA-core router of the DeepSeekMoE layer ("《DeepSeekMoE》深度解读报告" §3.1, Eq. 3-5 in
 // prose): z = x . e_i for every expert centroid, softmax over all N_m experts, keep the
-// N_r largest probabilities as gates (no renormalisation; ties to the lower index).
+// N_r largest probabilities as gates (no renormalisation; ties to the lower index).  Also the
+// two router variants: softmax over the top-k logits of a biased router (the FineGrainedMoE
+// listing of the DeepSeek-V2 explainer, §3.1) and a sigmoid gate with a selection-only bias.
 //
 // Used for fp32 layers and for expert counts the tensor-core router does not take.  Phase
 // 1 computes a [32 tokens x N_m] block of fp32 logits from shared-memory tiles of x and the
@@ -18,45 +20,74 @@ constexpr int RT_EXP = 64;      // experts per score tile
 constexpr int RT_K = 64;        // hidden elements per score tile
 constexpr int RT_THREADS = 256;
 
-// Softmax over the E logits in zr (shared memory, clobbered) and the top-k picks by one warp:
-// max and sum of exponentials by shuffles, then k rounds of warp argmax on (logit, -index),
-// so equal logits go to the lower index and picks come out by descending score.
-__device__ void warp_softmax_topk(float* zr, int E, int k, int lane, int32_t* idx_row, float* gate_row) {
-    float m = -INFINITY;
-    for (int e = lane; e < E; e += 32) m = fmaxf(m, zr[e]);
+// Picks and gates of one token by one warp from its E logits zr (shared memory, unchanged).
+// The selection key is z + bias (gate modes 0 and 1) or sigmoid(z) + bias (mode 2); lane l owns
+// experts l + 32 i and marks its picks in a bit mask.  k rounds of warp argmax on (key, -index)
+// give the picks in descending key, equal keys to the lower index.  Gates: mode 0 the softmax of
+// z + bias over all E experts read at the picks; mode 1 the softmax over the k picked keys;
+// mode 2 sigmoid(z) at the picks divided by their sum.
+__device__ void warp_route(const float* zr, int E, int k, int mode, const float* __restrict__ bias, int lane,
+                           int32_t* idx_row, float* gate_row) {
+    auto key_of = [&](int e) {
+        const float z = zr[e];
+        const float bb = bias ? bias[e] : 0.f;
+        return mode == 2 ? 1.0f / (1.0f + expf(-z)) + bb : z + bb;
+    };
+    float m = -INFINITY, inv = 0.f;
+    if (mode == 0) {
+        for (int e = lane; e < E; e += 32) m = fmaxf(m, key_of(e));
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    float s = 0.f;
-    for (int e = lane; e < E; e += 32) s += expf(zr[e] - m);
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        float s = 0.f;
+        for (int e = lane; e < E; e += 32) s += expf(key_of(e) - m);
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-    const float inv = 1.0f / s;
+        for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+        inv = 1.0f / s;
+    }
+    uint32_t taken = 0;
+    float first = 0.f, norm = 0.f;
     for (int j = 0; j < k; ++j) {
         float bv = -INFINITY;
         int bi = 0x7fffffff;
-        for (int e = lane; e < E; e += 32) {
-            float v = zr[e];
-            if (v > bv) { bv = v; bi = e; }     // ascending e: equal values keep the lower index
+        for (int e = lane, i = 0; e < E; e += 32, ++i) {
+            if (taken & (1u << i)) continue;
+            const float v = key_of(e);
+            if (v > bv) { bv = v; bi = e; }     // ascending e: equal keys keep the lower index
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) {
-            float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-            int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+            const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+            const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
             if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
         }
+        if (bi < E && (bi & 31) == lane) taken |= 1u << (bi >> 5);
         if (lane == 0) {
             idx_row[j] = bi;
-            gate_row[j] = expf(bv - m) * inv;
+            float g;
+            if (mode == 0) {
+                g = expf(bv - m) * inv;
+            } else if (mode == 1) {
+                if (j == 0) first = bv;
+                g = expf(bv - first);
+                norm += g;
+            } else {
+                g = 1.0f / (1.0f + expf(-zr[bi]));
+                norm += g;
+            }
+            gate_row[j] = g;
         }
-        if (bi < E && (bi % 32) == lane) zr[bi] = -INFINITY;   // owner lane removes the pick
         __syncwarp();
+    }
+    if (lane == 0 && mode != 0) {
+        const float r = 1.0f / norm;
+        for (int j = 0; j < k; ++j) gate_row[j] *= r;
     }
 }
 
 template <typename T>
 __global__ void __launch_bounds__(RT_THREADS)
-router_simt_kernel(const T* __restrict__ x, const T* __restrict__ cen, int32_t* __restrict__ idx_out,
-                   float* __restrict__ gate_out, int Tn, int d, int E, int k) {
+router_simt_kernel(const T* __restrict__ x, const T* __restrict__ cen, const float* __restrict__ bias, int mode,
+                   int32_t* __restrict__ idx_out, float* __restrict__ gate_out, int Tn, int d, int E, int k) {
     extern __shared__ float sm[];
     float* xs = sm;                                  // [RT_TOK][RT_K + 1]
     float* cs = xs + RT_TOK * (RT_K + 1);            // [RT_EXP][RT_K + 1]
@@ -103,7 +134,7 @@ router_simt_kernel(const T* __restrict__ x, const T* __restrict__ cen, int32_t* 
     for (int r = warp; r < RT_TOK; r += RT_THREADS / 32) {
         const int t = t0 + r;
         if (t >= Tn) break;
-        warp_softmax_topk(z + r * E, E, k, lane, idx_out + (size_t)t * k, gate_out + (size_t)t * k);
+        warp_route(z + r * E, E, k, mode, bias, lane, idx_out + (size_t)t * k, gate_out + (size_t)t * k);
     }
 }
 
@@ -113,8 +144,8 @@ router_simt_kernel(const T* __restrict__ x, const T* __restrict__ cen, int32_t* 
 // each sum a float4 of consecutive experts over the splits (coalesced across the block), then
 // warp 0 ranks the token.
 __global__ void __launch_bounds__(256)
-router_finish_kernel(const float* __restrict__ partial, int nsplit, int Tn, int E, int k, int32_t* __restrict__ idx_out,
-                     float* __restrict__ gate_out) {
+router_finish_kernel(const float* __restrict__ partial, int nsplit, int Tn, int E, int k, const float* __restrict__ bias,
+                     int mode, int32_t* __restrict__ idx_out, float* __restrict__ gate_out) {
     extern __shared__ float zs[];
     const int t = blockIdx.x;
     const int E4 = E / 4;
@@ -138,34 +169,35 @@ router_finish_kernel(const float* __restrict__ partial, int nsplit, int Tn, int 
         reinterpret_cast<float4*>(zs)[e4] = acc;
     }
     __syncthreads();
-    if (threadIdx.x < 32) warp_softmax_topk(zs, E, k, threadIdx.x, idx_out + (size_t)t * k, gate_out + (size_t)t * k);
+    if (threadIdx.x < 32) warp_route(zs, E, k, mode, bias, threadIdx.x, idx_out + (size_t)t * k, gate_out + (size_t)t * k);
 }
 
 }  // namespace
 
-cudaError_t launch_router_simt(const Dims& D, const void* x, const void* centroids, int32_t* idx, float* gate,
-                               cudaStream_t stream) {
+cudaError_t launch_router_simt(const Dims& D, const void* x, const void* centroids, const float* bias, int32_t* idx,
+                               float* gate, cudaStream_t stream) {
     const int blocks = ceil_div(D.T, RT_TOK);
     const size_t smem = sizeof(float) * ((size_t)RT_TOK * (RT_K + 1) + (size_t)RT_EXP * (RT_K + 1) + (size_t)RT_TOK * D.E);
     if (D.bf16) {
         auto kern = router_simt_kernel<__nv_bfloat16>;
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        kern<<<blocks, RT_THREADS, smem, stream>>>((const __nv_bfloat16*)x, (const __nv_bfloat16*)centroids, idx, gate,
-                                                   D.T, D.d, D.E, D.k);
+        kern<<<blocks, RT_THREADS, smem, stream>>>((const __nv_bfloat16*)x, (const __nv_bfloat16*)centroids, bias,
+                                                   D.gate_mode, idx, gate, D.T, D.d, D.E, D.k);
     } else {
         auto kern = router_simt_kernel<float>;
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        kern<<<blocks, RT_THREADS, smem, stream>>>((const float*)x, (const float*)centroids, idx, gate, D.T, D.d, D.E,
-                                                   D.k);
+        kern<<<blocks, RT_THREADS, smem, stream>>>((const float*)x, (const float*)centroids, bias, D.gate_mode, idx, gate,
+                                                   D.T, D.d, D.E, D.k);
     }
     return cudaGetLastError();
 }
 
-cudaError_t launch_router_finish(const Dims& D, const float* partial, int nsplit, int32_t* idx, float* gate,
-                                 cudaStream_t stream) {
+cudaError_t launch_router_finish(const Dims& D, const float* partial, int nsplit, const float* bias, int32_t* idx,
+                                 float* gate, cudaStream_t stream) {
     const int E4 = D.E / 4;
     const int threads = E4 < 32 ? 32 : (E4 > 256 ? 256 : (E4 + 31) / 32 * 32);
-    router_finish_kernel<<<D.T, threads, sizeof(float) * D.E, stream>>>(partial, nsplit, D.T, D.E, D.k, idx, gate);
+    router_finish_kernel<<<D.T, threads, sizeof(float) * D.E, stream>>>(partial, nsplit, D.T, D.E, D.k, bias,
+                                                                         D.gate_mode, idx, gate);
     return cudaGetLastError();
 }
 

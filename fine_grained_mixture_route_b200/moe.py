@@ -16,6 +16,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe_b200
 
 MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_CUDA, MOE_ERR_INTERNAL = range(6)
 MOE_F32, MOE_BF16 = 0, 1
+GATE_SOFTMAX_TOPK, GATE_TOPK_SOFTMAX, GATE_SIGMOID_BIAS = 0, 1, 2
 
 EXPORTED = ("moe_workspace_bytes", "moe_layer_launches", "moe_status_string", "moe_version", "moe_check_device_error", "moe_ws_init",
             "moe_route", "moe_permute", "moe_expert_ffn", "moe_combine", "moe_layer_forward",
@@ -26,7 +27,8 @@ STAGE_NAMES = ("router", "permute", "plan", "gather", "gemm1_swiglu", "gemm2", "
 
 class MoeShape(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in
-                ("T", "d", "n_experts", "inter", "top_k", "n_shared", "inter_shared", "has_bias", "dtype")]
+                ("T", "d", "n_experts", "inter", "top_k", "n_shared", "inter_shared", "has_bias", "dtype",
+                 "gate_mode")]
 
 
 class MoeWeights(ctypes.Structure):
@@ -63,12 +65,12 @@ def _lib():
         lib.moe_version.restype = ctypes.c_char_p
         lib.moe_check_device_error.argtypes = [vp, sz, vp, ctypes.POINTER(ctypes.c_uint32)]
         lib.moe_ws_init.argtypes = [vp, sz, vp]
-        lib.moe_route.argtypes = [sh, vp, vp, i32p, f32p, vp, sz, vp]
+        lib.moe_route.argtypes = [sh, vp, vp, f32p, i32p, f32p, vp, sz, vp]
         lib.moe_permute.argtypes = [sh, i32p, f32p, i32p, i32p, i32p, f32p, i32p, vp, sz, vp]
         lib.moe_expert_ffn.argtypes = [sh, vp, i32p, i32p, f32p, wp, vp, vp, sz, vp]
         lib.moe_combine.argtypes = [sh, vp, wp, vp, i32p, vp, vp, sz, vp]
-        lib.moe_layer_forward.argtypes = [sh, vp, vp, wp, wp, vp, i32p, f32p, i32p, vp, sz, vp]
-        lib.moe_layer_forward_timed.argtypes = [sh, vp, vp, wp, wp, vp, i32p, f32p, i32p, vp, sz, vp,
+        lib.moe_layer_forward.argtypes = [sh, vp, vp, f32p, wp, wp, vp, i32p, f32p, i32p, vp, sz, vp]
+        lib.moe_layer_forward_timed.argtypes = [sh, vp, vp, f32p, wp, wp, vp, i32p, f32p, i32p, vp, sz, vp,
                                                 ctypes.POINTER(ctypes.c_void_p), ctypes.c_int32]
         for n in ("moe_check_device_error", "moe_ws_init", "moe_route", "moe_permute", "moe_expert_ffn",
                   "moe_combine", "moe_layer_forward", "moe_layer_forward_timed"):
@@ -97,17 +99,26 @@ def _check(status: int, where: str):
 
 
 def make_shape(T: int, d: int, n_experts: int, inter: int, top_k: int, n_shared: int = 0, inter_shared: int = 0,
-               has_bias: bool = True, dtype: torch.dtype = torch.bfloat16) -> MoeShape:
+               has_bias: bool = True, dtype: torch.dtype = torch.bfloat16, gate_mode: int = GATE_SOFTMAX_TOPK) -> MoeShape:
     return MoeShape(T, d, n_experts, inter, top_k, n_shared, inter_shared if n_shared else 0, int(bool(has_bias)),
-                    MOE_BF16 if dtype == torch.bfloat16 else MOE_F32)
+                    MOE_BF16 if dtype == torch.bfloat16 else MOE_F32, gate_mode)
 
 
-def shape_of(x: torch.Tensor, centroids_or_E, routed: Dict, top_k: int, shared: Optional[Dict] = None) -> MoeShape:
+def shape_of(x: torch.Tensor, centroids_or_E, routed: Dict, top_k: int, shared: Optional[Dict] = None,
+             gate_mode: int = GATE_SOFTMAX_TOPK) -> MoeShape:
     E = centroids_or_E if isinstance(centroids_or_E, int) else centroids_or_E.shape[0]
     I = routed["w1"].shape[1]
     Ks = 0 if shared is None else shared["w1"].shape[0]
     Is = 0 if shared is None else shared["w1"].shape[1]
-    return make_shape(x.shape[0], x.shape[1], E, I, top_k, Ks, Is, routed.get("b1") is not None, x.dtype)
+    return make_shape(x.shape[0], x.shape[1], E, I, top_k, Ks, Is, routed.get("b1") is not None, x.dtype, gate_mode)
+
+
+def _bias_ptr(router_bias: Optional[torch.Tensor]):
+    if router_bias is None:
+        return None
+    if router_bias.dtype != torch.float32 or not router_bias.is_contiguous():
+        raise ValueError("router_bias must be a contiguous float32 tensor [n_experts]")
+    return ctypes.c_void_p(router_bias.data_ptr())
 
 
 def _weights(w: Optional[Dict]):
@@ -147,12 +158,12 @@ def check_device_error(ws: torch.Tensor, stream=None) -> int:
     return 0
 
 
-def route(shape: MoeShape, x, centroids, ws, idx=None, gate=None, stream=None):
+def route(shape: MoeShape, x, centroids, ws, idx=None, gate=None, stream=None, router_bias=None):
     T, k = shape.T, shape.top_k
     idx = torch.empty((T, k), dtype=torch.int32, device=x.device) if idx is None else idx
     gate = torch.empty((T, k), dtype=torch.float32, device=x.device) if gate is None else gate
-    _check(_lib().moe_route(ctypes.byref(shape), _ptr(x), _ptr(centroids), _ptr(idx), _ptr(gate), _ptr(ws),
-                            ws.numel(), _stream(stream)), "moe_route")
+    _check(_lib().moe_route(ctypes.byref(shape), _ptr(x), _ptr(centroids), _bias_ptr(router_bias), _ptr(idx),
+                            _ptr(gate), _ptr(ws), ws.numel(), _stream(stream)), "moe_route")
     return idx, gate
 
 
@@ -189,12 +200,12 @@ def combine(shape: MoeShape, x, shared: Optional[Dict], y_sorted, slot_of, ws, o
 
 
 def layer_forward(shape: MoeShape, x, centroids, routed: Dict, shared: Optional[Dict], ws, out=None,
-                  idx=None, gate=None, counts=None, stream=None):
+                  idx=None, gate=None, counts=None, stream=None, router_bias=None):
     """One call of the whole layer; idx / gate / counts are optional output tensors."""
     out = torch.empty((shape.T, shape.d), dtype=x.dtype, device=x.device) if out is None else out
     rw = _weights(routed)
     sw = _weights(shared)
-    _check(_lib().moe_layer_forward(ctypes.byref(shape), _ptr(x), _ptr(centroids), ctypes.byref(rw),
+    _check(_lib().moe_layer_forward(ctypes.byref(shape), _ptr(x), _ptr(centroids), _bias_ptr(router_bias), ctypes.byref(rw),
                                     None if sw is None else ctypes.byref(sw), _ptr(out), _ptr(idx), _ptr(gate),
                                     _ptr(counts), _ptr(ws), ws.numel(), _stream(stream)), "moe_layer_forward")
     return out
@@ -210,13 +221,14 @@ def stage_events(stream=None):
 
 
 def layer_forward_timed(shape: MoeShape, x, centroids, routed: Dict, shared: Optional[Dict], ws, events,
-                        out=None, idx=None, gate=None, counts=None, stream=None):
+                        out=None, idx=None, gate=None, counts=None, stream=None, router_bias=None):
     """layer_forward that also records `events` (from stage_events) at the stage boundaries."""
     out = torch.empty((shape.T, shape.d), dtype=x.dtype, device=x.device) if out is None else out
     rw = _weights(routed)
     sw = _weights(shared)
     arr = (ctypes.c_void_p * len(events))(*[e.cuda_event for e in events])
-    _check(_lib().moe_layer_forward_timed(ctypes.byref(shape), _ptr(x), _ptr(centroids), ctypes.byref(rw),
+    _check(_lib().moe_layer_forward_timed(ctypes.byref(shape), _ptr(x), _ptr(centroids), _bias_ptr(router_bias),
+                                          ctypes.byref(rw),
                                           None if sw is None else ctypes.byref(sw), _ptr(out), _ptr(idx), _ptr(gate),
                                           _ptr(counts), _ptr(ws), ws.numel(), _stream(stream), arr, len(events)),
            "moe_layer_forward_timed")

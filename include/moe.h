@@ -63,6 +63,18 @@ typedef enum {
 
 typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype_t;
 
+/* Router gate (z = x . e_i + bias_i, bias optional):
+ *   MOE_GATE_SOFTMAX_TOPK  softmax of z over all experts, keep it at the top_k largest z,
+ *                          no renormalisation ("《DeepSeekMoE》深度解读报告" §3.1; the default).
+ *   MOE_GATE_TOPK_SOFTMAX  top_k largest z, softmax over those k logits (gates sum to 1; the
+ *                          FineGrainedMoE listing of the DeepSeek-V2 explainer, §3.1, whose
+ *                          router is a Linear layer with a bias).
+ *   MOE_GATE_SIGMOID_BIAS  s = sigmoid(x . e_i); picks = top_k largest s_i + bias_i (the bias
+ *                          steers only the choice); gates = s at the picks over their sum (a
+ *                          reading of the sigmoid gate with aux-loss-free balancing the report
+ *                          mentions for DeepSeek-V3, §6.2; no formula on the pages). */
+typedef enum { MOE_GATE_SOFTMAX_TOPK = 0, MOE_GATE_TOPK_SOFTMAX = 1, MOE_GATE_SIGMOID_BIAS = 2 } moe_gate_mode_t;
+
 typedef struct {
     int32_t T;            /* tokens */
     int32_t d;            /* hidden size */
@@ -73,6 +85,7 @@ typedef struct {
     int32_t inter_shared; /* intermediate size of a shared expert (ignored when n_shared == 0) */
     int32_t has_bias;     /* 1: every Linear has a bias (the page's Expert); 0: no biases */
     int32_t dtype;        /* moe_dtype_t */
+    int32_t gate_mode;    /* moe_gate_mode_t (0 = the report's softmax gate) */
 } moe_shape_t;
 
 /* One stack of experts (routed: E = n_experts; shared: E = n_shared), nn.Linear layout. */
@@ -110,14 +123,16 @@ moe_status_t moe_check_device_error(void* ws, size_t ws_bytes, moe_stream_t stre
 moe_status_t moe_ws_init(void* ws, size_t ws_bytes, moe_stream_t stream);
 
 /*
- * Router: scores, softmax over all experts, top_k picks and gates ("《DeepSeekMoE》深度解读报告"
- * §3.1, Eq. 3-5 in prose).
- *   x:          [T, d]           dtype
- *   centroids:  [n_experts, d]   dtype (the expert centroids e_i)
- *   topk_idx:   [T, top_k] int32 out: expert indices, descending score, ties to lower index
- *   topk_gate:  [T, top_k] fp32  out: softmax probability of each pick (not renormalised)
+ * Router: scores, top_k picks and gates ("《DeepSeekMoE》深度解读报告" §3.1, Eq. 3-5 in prose,
+ * with the variants of shape->gate_mode).
+ *   x:           [T, d]           dtype
+ *   centroids:   [n_experts, d]   dtype (the expert centroids e_i)
+ *   router_bias: [n_experts] fp32 or NULL (no bias)
+ *   topk_idx:    [T, top_k] int32 out: expert indices, descending selection key, ties to the
+ *                lower index
+ *   topk_gate:   [T, top_k] fp32  out: the gate of each pick (see moe_gate_mode_t)
  */
-moe_status_t moe_route(const moe_shape_t* shape, const void* x, const void* centroids,
+moe_status_t moe_route(const moe_shape_t* shape, const void* x, const void* centroids, const float* router_bias,
                        int32_t* topk_idx, float* topk_gate,
                        void* ws, size_t ws_bytes, moe_stream_t stream);
 
@@ -169,13 +184,13 @@ moe_status_t moe_combine(const moe_shape_t* shape, const void* x, const moe_ffn_
 /*
  * The whole layer: moe_route -> moe_permute -> moe_expert_ffn -> moe_combine, all on
  * `stream`, every intermediate in `ws`.
- *   x: [T, d]; centroids: [n_experts, d]; routed / shared weights as above (shared NULL iff
- *   n_shared == 0); out: [T, d].
+ *   x: [T, d]; centroids: [n_experts, d]; router_bias: [n_experts] fp32 or NULL; routed / shared
+ *   weights as above (shared NULL iff n_shared == 0); out: [T, d].
  *   topk_idx_out [T, top_k], topk_gate_out [T, top_k] and counts_out [n_experts] are
  *   optional (NULL = not returned).
  */
 moe_status_t moe_layer_forward(const moe_shape_t* shape, const void* x, const void* centroids,
-                               const moe_ffn_weights_t* routed, const moe_ffn_weights_t* shared,
+                               const float* router_bias, const moe_ffn_weights_t* routed, const moe_ffn_weights_t* shared,
                                void* out, int32_t* topk_idx_out, float* topk_gate_out,
                                int32_t* counts_out, void* ws, size_t ws_bytes, moe_stream_t stream);
 
@@ -193,7 +208,7 @@ moe_status_t moe_layer_forward(const moe_shape_t* shape, const void* x, const vo
  */
 #define MOE_NUM_STAGES 7
 moe_status_t moe_layer_forward_timed(const moe_shape_t* shape, const void* x, const void* centroids,
-                                     const moe_ffn_weights_t* routed, const moe_ffn_weights_t* shared,
+                                     const float* router_bias, const moe_ffn_weights_t* routed, const moe_ffn_weights_t* shared,
                                      void* out, int32_t* topk_idx_out, float* topk_gate_out,
                                      int32_t* counts_out, void* ws, size_t ws_bytes, moe_stream_t stream,
                                      void* const* stage_events, int32_t n_events);

@@ -39,10 +39,12 @@ def normwise(gpu: np.ndarray, ref: np.ndarray) -> float:
     return float(np.abs(gpu - ref).max()) / den
 
 
-def check_routing(idx_gpu: np.ndarray, gate_gpu: np.ndarray, x64: np.ndarray, c64: np.ndarray, k: int):
-    """Returns (near_tie_token_mask, n_set_ties, n_order_ties) after asserting parity."""
-    r = O.route(x64, c64, k)
-    z = r["z"]
+def check_routing(idx_gpu: np.ndarray, gate_gpu: np.ndarray, x64: np.ndarray, c64: np.ndarray, k: int,
+                  gate_mode: int = 0, bias=None):
+    """Returns (near_tie_token_mask, n_set_ties, n_order_ties) after asserting parity.  Near
+    ties are measured on the selection key of the gate mode (the logit, or sigmoid + bias)."""
+    r = O.route(x64, c64, k, gate_mode, bias)
+    z = r["key"]
     idx_ref = r["idx"]
     set_tie = r["gap"] < NEAR_TIE
     order_tie = r["gap_order"] < NEAR_TIE
@@ -57,7 +59,7 @@ def check_routing(idx_gpu: np.ndarray, gate_gpu: np.ndarray, x64: np.ndarray, c6
         boundary = zs[k - 1]
         assert (z[t, sel] >= boundary - NEAR_TIE).all(), f"token {t}: pick far below the k-th score"
         assert (np.diff(z[t, sel]) <= NEAR_TIE).all(), f"token {t}: picks not in descending order"
-    g_ref = O.gates_from_indices(x64, c64, idx_gpu)
+    g_ref = O.gates_from_indices(x64, c64, idx_gpu, gate_mode, bias)
     rel = np.abs(gate_gpu - g_ref) / np.abs(g_ref)
     assert rel.max() <= GATE_RTOL, f"gate error {rel.max():.3e}"
     return ~same, int(set_tie.sum()), int(order_tie.sum())

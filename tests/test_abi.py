@@ -47,7 +47,7 @@ def test_version_and_status_strings(lib):
 
 def _shape(**kw):
     base = dict(T=256, d=7168, n_experts=256, inter=2048, top_k=8, n_shared=1, inter_shared=2048, has_bias=1,
-                dtype=moe.MOE_BF16)
+                dtype=moe.MOE_BF16, gate_mode=0)
     base.update(kw)
     return moe.MoeShape(*[base[f] for f, _ in moe.MoeShape._fields_])
 
@@ -65,7 +65,7 @@ def test_workspace_bytes(lib):
     assert moe.workspace_bytes(_shape(dtype=moe.MOE_F32)) < 2 * n
     for bad in (dict(top_k=0), dict(top_k=300), dict(n_experts=0), dict(d=0), dict(T=-1), dict(dtype=7),
                 dict(n_experts=2048, top_k=8), dict(d=7170), dict(inter=2047), dict(top_k=33, n_experts=64),
-                dict(has_bias=2), dict(n_shared=1, inter_shared=0)):
+                dict(has_bias=2), dict(n_shared=1, inter_shared=0), dict(gate_mode=3), dict(gate_mode=-1)):
         assert moe.workspace_bytes(_shape(**bad)) == 0, bad
     assert moe.workspace_bytes(_shape(d=7170, dtype=moe.MOE_F32)) > 0
 
@@ -87,8 +87,8 @@ def test_argument_errors_return_before_any_launch(lib):
     w = moe.MoeWeights(fake.value, fake.value, fake.value, fake.value, fake.value, fake.value)
     S = ctypes.byref
     # null pointers
-    assert lib.moe_route(S(sh), None, fake, fake, fake, fake, n, None) == moe.MOE_ERR_INVALID_ARG
-    assert lib.moe_layer_forward(S(sh), fake, fake, None, S(w), fake, None, None, None, fake, n, None) == \
+    assert lib.moe_route(S(sh), None, fake, None, fake, fake, fake, n, None) == moe.MOE_ERR_INVALID_ARG
+    assert lib.moe_layer_forward(S(sh), fake, fake, None, None, S(w), fake, None, None, None, fake, n, None) == \
         moe.MOE_ERR_INVALID_ARG
     # bias pointers must match has_bias
     wnb = moe.MoeWeights(fake.value, None, fake.value, None, fake.value, None)
@@ -100,19 +100,20 @@ def test_argument_errors_return_before_any_launch(lib):
     assert lib.moe_combine(S(sh0), fake, S(w), fake, fake, fake, fake, n, None) == moe.MOE_ERR_INVALID_ARG
     assert lib.moe_combine(S(sh), fake, None, fake, fake, fake, fake, n, None) == moe.MOE_ERR_INVALID_ARG
     # workspace too small, missing or misaligned
-    assert lib.moe_route(S(sh), fake, fake, fake, fake, fake, n - 1, None) == moe.MOE_ERR_WORKSPACE
-    assert lib.moe_route(S(sh), fake, fake, fake, fake, None, n, None) == moe.MOE_ERR_WORKSPACE
-    assert lib.moe_route(S(sh), fake, fake, fake, fake, ctypes.c_void_p((1 << 40) + 8), n, None) == \
+    assert lib.moe_route(S(sh), fake, fake, None, fake, fake, fake, n - 1, None) == moe.MOE_ERR_WORKSPACE
+    assert lib.moe_route(S(sh), fake, fake, None, fake, fake, None, n, None) == moe.MOE_ERR_WORKSPACE
+    assert lib.moe_route(S(sh), fake, fake, None, fake, fake, ctypes.c_void_p((1 << 40) + 8), n, None) == \
         moe.MOE_ERR_WORKSPACE
     # unsupported sizes
-    assert lib.moe_route(S(_shape(d=7172)), fake, fake, fake, fake, fake, n, None) == moe.MOE_ERR_UNSUPPORTED
-    assert lib.moe_route(S(_shape(top_k=40, n_experts=64)), fake, fake, fake, fake, fake, n, None) == \
+    assert lib.moe_route(S(_shape(d=7172)), fake, fake, None, fake, fake, fake, n, None) == moe.MOE_ERR_UNSUPPORTED
+    assert lib.moe_route(S(_shape(top_k=40, n_experts=64)), fake, fake, None, fake, fake, fake, n, None) == \
         moe.MOE_ERR_UNSUPPORTED
-    assert lib.moe_route(None, fake, fake, fake, fake, fake, n, None) == moe.MOE_ERR_INVALID_ARG
+    assert lib.moe_route(None, fake, fake, None, fake, fake, fake, n, None) == moe.MOE_ERR_INVALID_ARG
+    assert lib.moe_route(S(_shape(gate_mode=5)), fake, fake, None, fake, fake, fake, n, None) == moe.MOE_ERR_INVALID_ARG
     # T == 0 is a valid no-op (returns before any CUDA call)
     sh_e = _shape(T=0)
     ne = moe.workspace_bytes(sh_e)
-    assert lib.moe_route(S(sh_e), fake, fake, fake, fake, fake, ne, None) == moe.MOE_OK
-    assert lib.moe_layer_forward(S(sh_e), fake, fake, S(w), S(w), fake, None, None, None, fake, ne, None) == moe.MOE_OK
+    assert lib.moe_route(S(sh_e), fake, fake, None, fake, fake, fake, ne, None) == moe.MOE_OK
+    assert lib.moe_layer_forward(S(sh_e), fake, fake, None, S(w), S(w), fake, None, None, None, fake, ne, None) == moe.MOE_OK
     assert lib.moe_ws_init(None, 0, None) == moe.MOE_ERR_WORKSPACE
     assert lib.moe_check_device_error(None, 0, None, None) == moe.MOE_ERR_WORKSPACE

@@ -183,3 +183,48 @@ def test_host_pipeline_matches_device_calls():
     moe.check_device_error(ws)
     for w, o in zip(want, oh):
         assert torch.equal(w, o)
+
+
+ROUTER_CASES = [
+    # (name, base config, overrides): tensor-core router with one CTA per token tile, split-K
+    # tensor-core router, CUDA-core router (bf16 with N_m = 20, and fp32)
+    ("tc_tiles", "small", dict(T=4500, d=256, n_experts=64, top_k=6, inter=64, inter_shared=64)),
+    ("tc_splitk", "small", dict(T=512)),
+    ("simt_bf16", "small", dict(T=300, n_experts=20, top_k=3, d=256, inter=64, inter_shared=64)),
+    ("simt_f32", "tiny", dict(T=100)),
+]
+
+
+@pytest.mark.parametrize("gate_mode", [1, 2])
+@pytest.mark.parametrize("with_bias", [False, True])
+@pytest.mark.parametrize("case", ROUTER_CASES, ids=[c[0] for c in ROUTER_CASES])
+def test_router_variants(case, with_bias, gate_mode):
+    """Gate modes 1 (softmax over the top-k logits of a biased router) and 2 (sigmoid gate with
+    a selection bias) through the fused layer: picks exact outside near-ties of the selection
+    key, gates within 1e-4, outputs within the layer tolerance."""
+    _, base, kw = case
+    cfg = W.scaled(W.CONFIGS[base], **kw)
+    L = W.make_layer(cfg, "cuda", seed=7)
+    bias = None
+    if with_bias:
+        g = torch.Generator(device="cpu").manual_seed(3)
+        bias = (0.5 * torch.randn(cfg.n_experts, generator=g)).to(torch.float32).cuda()
+    x, C, R, Sh = L["x"], L["centroids"], L["routed"], L["shared"]
+    shape = moe.shape_of(x, C, R, cfg.top_k, Sh, gate_mode=gate_mode)
+    ws = moe.new_workspace(shape)
+    idx = torch.empty((cfg.T, cfg.top_k), dtype=torch.int32, device="cuda")
+    gate = torch.empty((cfg.T, cfg.top_k), dtype=torch.float32, device="cuda")
+    out = moe.layer_forward(shape, x, C, R, Sh, ws, idx=idx, gate=gate, router_bias=bias)
+    idx2, gate2 = moe.route(shape, x, C, ws, router_bias=bias)
+    moe.check_device_error(ws)
+    assert torch.equal(idx, idx2) and torch.equal(gate, gate2)
+    x64, c64 = f64(x), f64(C)
+    b64 = None if bias is None else bias.double().cpu().numpy()
+    idx_np, gate_np = idx.cpu().numpy().astype(np.int64), gate.cpu().numpy()
+    check_routing(idx_np, gate_np, x64, c64, cfg.top_k, gate_mode, b64)
+    assert np.allclose(gate_np.sum(1), 1.0, rtol=0, atol=1e-5)
+    rows = np.arange(min(cfg.T, 160))
+    ref = O.layer(x64[rows], c64, expert_source(R), cfg.n_experts, cfg.top_k,
+                  expert_source(Sh) if Sh is not None else None, cfg.n_shared, idx_override=idx_np[rows],
+                  gate_mode=gate_mode, router_bias=b64)
+    assert normwise(f64(out)[rows], ref["out"]) <= TOL[cfg.dtype]
