@@ -238,19 +238,20 @@ def layer_forward_timed(shape: MoeShape, x, centroids, routed: Dict, shared: Opt
 class MoELayer:
     """Convenience holder: the layer's device tensors, its shape and one workspace."""
 
-    def __init__(self, centroids: torch.Tensor, routed: Dict, shared: Optional[Dict], top_k: int, max_tokens: int):
+    def __init__(self, centroids: torch.Tensor, routed: Dict, shared: Optional[Dict], top_k: int, max_tokens: int,
+                 gate_mode: int = GATE_SOFTMAX_TOPK, router_bias: Optional[torch.Tensor] = None):
         self.centroids, self.routed, self.shared, self.top_k = centroids, routed, shared, top_k
-        self.max_tokens = max_tokens
+        self.max_tokens, self.gate_mode, self.router_bias = max_tokens, gate_mode, router_bias
         dummy = torch.empty((max_tokens, centroids.shape[1]), dtype=centroids.dtype, device="meta")
-        self.shape_max = shape_of(dummy, centroids, routed, top_k, shared)
+        self.shape_max = shape_of(dummy, centroids, routed, top_k, shared, gate_mode)
         self.ws = new_workspace(self.shape_max, centroids.device)
 
     def __call__(self, x: torch.Tensor, out=None, idx=None, gate=None, counts=None, stream=None):
         if x.shape[0] > self.max_tokens:
             raise ValueError("more tokens than the workspace was sized for")
-        shape = shape_of(x, self.centroids, self.routed, self.top_k, self.shared)
+        shape = shape_of(x, self.centroids, self.routed, self.top_k, self.shared, self.gate_mode)
         return layer_forward(shape, x, self.centroids, self.routed, self.shared, self.ws, out, idx, gate, counts,
-                             stream)
+                             stream, router_bias=self.router_bias)
 
 
 class HostPipeline:
@@ -262,8 +263,10 @@ class HostPipeline:
     memory use is fixed.  Every batch still crosses PCIe both ways.
     """
 
-    def __init__(self, shape: MoeShape, centroids, routed: Dict, shared: Optional[Dict], ws, device=None):
+    def __init__(self, shape: MoeShape, centroids, routed: Dict, shared: Optional[Dict], ws, device=None,
+                 router_bias=None):
         self.shape, self.centroids, self.routed, self.shared, self.ws = shape, centroids, routed, shared, ws
+        self.router_bias = router_bias
         dev = centroids.device if device is None else device
         T, d = shape.T, shape.d
         self.xd = [torch.empty((T, d), dtype=centroids.dtype, device=dev) for _ in range(2)]
@@ -292,7 +295,7 @@ class HostPipeline:
                 self.s_comp.wait_event(self.in_done[b])
                 self.s_comp.wait_event(self.out_done[b])         # copy-out of batch i-2 has read od[b]
                 layer_forward(self.shape, self.xd[b], self.centroids, self.routed, self.shared, self.ws,
-                              out=self.od[b], stream=self.s_comp)
+                              out=self.od[b], stream=self.s_comp, router_bias=self.router_bias)
                 self.comp_done[b].record(self.s_comp)
             with torch.cuda.stream(self.s_out):
                 self.s_out.wait_event(self.comp_done[b])
