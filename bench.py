@@ -222,11 +222,13 @@ class HostExperts:
         return {k: (None if v is None else v.float().numpy().astype(np.float64)) for k, v in h.items()}
 
 
-def oracle_sample(O, L, cfg, host_routed, host_shared, tokens):
+def oracle_sample(O, L, cfg, host_routed, host_shared, tokens, gate_mode=0, router_bias=None):
     x = L["x"][tokens].float().cpu().numpy().astype(np.float64)
     c = L["centroids"].float().cpu().numpy().astype(np.float64)
+    b = None if router_bias is None else router_bias.double().cpu().numpy()
     t0 = time.perf_counter()
-    O.layer(x, c, host_routed, cfg.n_experts, cfg.top_k, host_shared, cfg.n_shared)
+    O.layer(x, c, host_routed, cfg.n_experts, cfg.top_k, host_shared, cfg.n_shared, gate_mode=gate_mode,
+            router_bias=b)
     return time.perf_counter() - t0
 
 
@@ -241,7 +243,7 @@ def blas_threads():
     return os.cpu_count() or 1
 
 
-def cpu_baseline(cfg, L, idx_gpu, n_tokens=16):
+def cpu_baseline(cfg, L, idx_gpu, n_tokens=16, gate_mode=0, router_bias=None):
     """The oracle, as it stands, on the first n_tokens tokens of this step's batch."""
     import oracle.moe_oracle as O
     tokens = np.arange(min(n_tokens, cfg.T))
@@ -250,7 +252,7 @@ def cpu_baseline(cfg, L, idx_gpu, n_tokens=16):
     hr.prefetch(np.unique(idx_gpu[tokens]))
     if hs is not None:
         hs.prefetch(range(cfg.n_shared))
-    dt = oracle_sample(O, L, cfg, hr, hs, tokens)
+    dt = oracle_sample(O, L, cfg, hr, hs, tokens, gate_mode, router_bias)
     return {"value": len(tokens) / dt, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
             "sample": f"fp64 NumPy oracle on the first {len(tokens)} tokens of the {cfg.name} batch "
                       f"(all experts they route to; weights staged in host memory as bf16, converted by the oracle)",
@@ -305,7 +307,11 @@ def run_ours(args, cfg, rank, world, local_rank):
     if rank > 0:
         L["x"] = W.make_x(cfg, dev, seed=1000 + rank)
     x, C, R, Sh = L["x"], L["centroids"], L["routed"], L["shared"]
-    shape = moe.shape_of(x, C, R, cfg.top_k, Sh)
+    shape = moe.shape_of(x, C, R, cfg.top_k, Sh, gate_mode=args.gate_mode)
+    rbias = None
+    if args.gate_mode != 0:   # a seeded per-expert router bias, N(0, 0.006) like every other parameter
+        g = torch.Generator(device="cpu").manual_seed(W.seed_for(0, "centroids", 10**6))
+        rbias = (W.INIT_STD * torch.randn(cfg.n_experts, generator=g)).to(dev)
     ws = moe.new_workspace(shape, dev)
     out = torch.empty_like(x)
     idx = torch.empty((cfg.T, cfg.top_k), dtype=torch.int32, device=dev)
@@ -313,7 +319,7 @@ def run_ours(args, cfg, rank, world, local_rank):
     counts = torch.empty(cfg.n_experts, dtype=torch.int32, device=dev)
 
     for _ in range(args.warmup):
-        moe.layer_forward(shape, x, C, R, Sh, ws, out=out, idx=idx, gate=gate, counts=counts)
+        moe.layer_forward(shape, x, C, R, Sh, ws, out=out, idx=idx, gate=gate, counts=counts, router_bias=rbias)
     moe.check_device_error(ws)
     touched = int((counts > 0).sum().item())
     work = stage_work(cfg, touched)
@@ -326,7 +332,8 @@ def run_ours(args, cfg, rank, world, local_rank):
     sampler = ClockSampler(visible_gpu_id(local_rank))
     start.record(stream)
     for i in range(args.steps):
-        moe.layer_forward_timed(shape, x, C, R, Sh, ws, evs[i], out=out, idx=idx, gate=gate, counts=counts)
+        moe.layer_forward_timed(shape, x, C, R, Sh, ws, evs[i], out=out, idx=idx, gate=gate, counts=counts,
+                                router_bias=rbias)
     stop.record(stream)
     torch.cuda.synchronize()
     clocks = sampler.stop()
@@ -345,7 +352,7 @@ def run_ours(args, cfg, rank, world, local_rank):
     if not args.no_e2e:
         xh = x.detach().to("cpu").pin_memory()
         ohs = [torch.empty(x.shape, dtype=x.dtype).pin_memory() for _ in range(2)]
-        pipe = moe.HostPipeline(shape, C, R, Sh, ws, dev)
+        pipe = moe.HostPipeline(shape, C, R, Sh, ws, dev, router_bias=rbias)
         pipe.run([xh] * 2, ohs)                                         # warm-up
         torch.cuda.synchronize()
         barrier()
@@ -394,7 +401,7 @@ def run_ours(args, cfg, rank, world, local_rank):
         "vs_baseline": None, "dtype": "bf16" if cfg.dtype == torch.bfloat16 else "f32", "data": "synthetic",
         "config": {"workload": cfg.name, "T": cfg.T, "d": cfg.d, "n_experts": cfg.n_experts, "inter": cfg.inter,
                    "top_k": cfg.top_k, "n_shared": cfg.n_shared, "inter_shared": cfg.inter_shared,
-                   "bias": cfg.has_bias, "routing": cfg.centroid_init,
+                   "bias": cfg.has_bias, "routing": cfg.centroid_init, "gate_mode": args.gate_mode,
                    "parallelism": f"replicas{world}" if world > 1 else "single",
                    "l2": "inputs larger than L2 (weights and activations), no flush",
                    "tokens_per_gpu": cfg.T},
@@ -409,7 +416,7 @@ def run_ours(args, cfg, rank, world, local_rank):
     }
     del evs
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(cfg, L, idx.cpu().numpy())
+        line["cpu_baseline"] = cpu_baseline(cfg, L, idx.cpu().numpy(), gate_mode=args.gate_mode, router_bias=rbias)
     if rank == 0:
         print(json.dumps(line), flush=True)
 
@@ -421,6 +428,9 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="prefill", choices=sorted(W.CONFIGS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--gate-mode", type=int, default=0, choices=[0, 1, 2],
+                    help="router gate: 0 softmax over all experts (default), 1 softmax over the top-k logits of a "
+                         "biased router, 2 sigmoid with a selection bias")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args(argv)
