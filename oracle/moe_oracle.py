@@ -26,6 +26,15 @@ What it computes, and where it comes from:
 * Per-expert token lists (DeepSeek-V2 explainer, eliteato.com/news/32734, §3.1 and §3.3:
   top-k indices first, then a gather of tokens per expert): a stable grouping of the T*N_r
   (token, pick) slots by expert, ascending token order inside an expert.
+* FP8 routed experts (an extension; the pages name FP8 for DeepSeek-V3 and for fine-grained
+  MoE but give no recipe, so the recipe is this project's reading): the routed experts' weights
+  are e4m3 codes with one fp32 scale per output channel; each expert input row (a token's
+  hidden state) is quantised to e4m3 with one scale per row, scale = row max |.| / 448; the
+  SwiGLU hidden row is rounded to bf16 and quantised the same way before w2.  Every
+  quantisation decision is taken in fp32 (division and e4m3 round-to-nearest-even, saturating
+  at 448), so it is exact and reproducible; the products and sums run in fp64 on the exact
+  dequantised values.  The e4m3 format is taken from its definition (1 sign, 4 exponent bits
+  with bias 7, 3 mantissa bits, subnormals, S.1111.111 = NaN, no infinities).
 * Accounting helpers: ptflops-style MAC and parameter counts of one Expert (the ptflops
   printout on the first page), the expert-hit entropy diagnostic (DeepSeek-V2 explainer
   §6), and the combination count of fine-grained routing (DeepSeekMoE report §2.2).
@@ -188,6 +197,70 @@ def permute(idx: np.ndarray, gate: np.ndarray, n_experts: int) -> Dict[str, np.n
 
 
 # --------------------------------------------------------------------------------------
+# FP8 (e4m3) format and per-row quantisation
+# --------------------------------------------------------------------------------------
+E4M3_MAX = 448.0
+
+
+def e4m3_decode(codes: np.ndarray) -> np.ndarray:
+    """uint8 e4m3 codes -> float64 values, from the format's bit fields."""
+    c = np.asarray(codes, np.uint8).astype(np.int64)
+    sign = np.where(c >> 7, -1.0, 1.0)
+    e = (c >> 3) & 15
+    m = (c & 7).astype(np.float64)
+    mag = np.where(e == 0, m / 8.0 * 2.0 ** -6, (1.0 + m / 8.0) * np.exp2((e - 7).astype(np.float64)))
+    mag = np.where((e == 15) & (c & 7 == 7), np.nan, mag)
+    return sign * mag
+
+
+def e4m3_round(v: np.ndarray) -> np.ndarray:
+    """Round to the nearest e4m3 value, ties to the even mantissa, saturating at +-448.
+
+    In the binade [2^e, 2^(e+1)) the e4m3 values are 2^(e-3) apart; below 2^-6 (subnormals)
+    they are 2^-9 apart.  Dividing by that spacing is exact, and rint rounds half to even."""
+    v = np.asarray(v, np.float64)
+    a = np.abs(v)
+    _, ex = np.frexp(a)                       # a = f * 2^ex with f in [0.5, 1)
+    e = np.maximum(ex - 1, -6)
+    step = np.ldexp(1.0, e - 3)
+    q = np.minimum(np.rint(a / step) * step, E4M3_MAX)
+    return np.copysign(q, v)
+
+
+def bf16_round(a: np.ndarray) -> np.ndarray:
+    """fp64 -> fp32 -> bf16 (round to nearest even on the fp32 bit pattern) -> fp64."""
+    u = np.asarray(a, np.float64).astype(np.float32).view(np.uint32).astype(np.uint64)
+    u = (u + 0x7FFF + ((u >> 16) & 1)) & 0xFFFF0000
+    return u.astype(np.uint32).view(np.float32).astype(np.float64)
+
+
+def quantize_rows_e4m3(a: np.ndarray):
+    """Per-row e4m3 quantisation of fp32-representable values: scale = max|row| / 448 in fp32
+    (1 for an all-zero row), codes = e4m3_round(row / scale) with the division in fp32.
+    Returns (values on the e4m3 grid as fp64, fp32 scales); the row stands for values * scale."""
+    a32 = np.asarray(a, np.float64).astype(np.float32)
+    amax = np.abs(a32).max(axis=-1) if a32.shape[-1] else np.zeros(a32.shape[:-1], np.float32)
+    scale = np.where(amax > 0, amax / np.float32(E4M3_MAX), np.float32(1.0)).astype(np.float32)
+    v = (a32 / scale[..., None]).astype(np.float64)
+    return e4m3_round(v), scale
+
+
+def dequantized_rows(a: np.ndarray) -> np.ndarray:
+    """The values a per-row e4m3 quantisation of a stands for (codes * scale, exact in fp64)."""
+    q, s = quantize_rows_e4m3(a)
+    return q * s.astype(np.float64)[..., None]
+
+
+def e4m3_weights(w: Weights) -> Weights:
+    """One expert in the FP8 format (codes w1/w3/w2 as uint8, per-output-channel scales
+    s1/s3/s2) -> fp64 weights codes * scale; biases unchanged."""
+    out = {k: v for k, v in w.items() if k not in ("s1", "s3", "s2")}
+    for name, sname in (("w1", "s1"), ("w3", "s3"), ("w2", "s2")):
+        out[name] = e4m3_decode(w[name]) * np.asarray(w[sname], np.float64)[:, None]
+    return out
+
+
+# --------------------------------------------------------------------------------------
 # the layer
 # --------------------------------------------------------------------------------------
 ExpertSource = Union[Weights, Callable[[int], Weights]]
@@ -202,7 +275,8 @@ def _expert(src: ExpertSource, e: int) -> Weights:
 def layer(x: np.ndarray, centroids: np.ndarray, routed: ExpertSource, n_experts: int, top_k: int,
           shared: Optional[ExpertSource] = None, n_shared: int = 0,
           idx_override: Optional[np.ndarray] = None, keep_hidden: bool = False,
-          gate_mode: int = GATE_SOFTMAX_TOPK, router_bias: Optional[np.ndarray] = None) -> Dict[str, np.ndarray]:
+          gate_mode: int = GATE_SOFTMAX_TOPK, router_bias: Optional[np.ndarray] = None,
+          routed_e4m3: bool = False) -> Dict[str, np.ndarray]:
     """The DeepSeekMoE layer forward in fp64.
 
     routed / shared: either dicts of stacked arrays (w1,b1,w3,b3,w2,b2 indexed by expert) or
@@ -210,6 +284,9 @@ def layer(x: np.ndarray, centroids: np.ndarray, routed: ExpertSource, n_experts:
     idx_override: route with these picks instead of the oracle's own (gates are then the
     gates those picks receive); used where a near-tie makes another pick set valid.
     gate_mode / router_bias: see route().
+    routed_e4m3: the routed experts are in the FP8 format (e4m3_weights); their inputs and
+    hidden rows are quantised per row (quantize_rows_e4m3, the hidden row after rounding to
+    bf16).  The router and the shared experts are unchanged.
 
     Returns out [T,d], routed_sum, shared_sum, idx, gate, gap, gap_order, counts, and
     Y [T*k, d] = gate * Expert_e(x_t) per slot (slot = t*k + j); with keep_hidden also
@@ -226,12 +303,15 @@ def layer(x: np.ndarray, centroids: np.ndarray, routed: ExpertSource, n_experts:
     k = top_k
     Y = np.zeros((T * k, d))
     H = None
+    xq = dequantized_rows(x) if routed_e4m3 else x
     for e in np.unique(idx):
         w = _expert(routed, int(e))
+        if routed_e4m3:
+            w = e4m3_weights(w)
         tt, jj = np.nonzero(idx == e)
-        xe = x[tt]
+        xe = xq[tt]
         he = swiglu_hidden(xe, w["w1"], w["b1"], w["w3"], w["b3"])
-        ye = linear(he, w["w2"], w["b2"])
+        ye = linear(dequantized_rows(bf16_round(he)) if routed_e4m3 else he, w["w2"], w["b2"])
         if keep_hidden:
             if H is None:
                 H = np.zeros((T * k, he.shape[1]))

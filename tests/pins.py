@@ -352,6 +352,132 @@ def check_gate_modes(O):
     assert np.allclose(res["out"], want, rtol=1e-11, atol=1e-11)
 
 
+def _e4m3_grid():
+    """All finite e4m3 values from the format's definition (1 sign, 4 exponent bits with bias 7,
+    3 mantissa bits, subnormals at exponent 0, S.1111.111 = NaN) with the mantissa parity of each."""
+    vals = {}
+    for e in range(16):
+        for m in range(8):
+            if e == 15 and m == 7:
+                continue
+            v = (m / 8.0) * 2.0 ** -6 if e == 0 else (1 + m / 8.0) * 2.0 ** (e - 7)
+            vals[v] = m % 2
+            vals[-v] = m % 2
+    g = sorted(vals)
+    return np.array(g), np.array([vals[v] for v in g])
+
+
+def _torch_e4m3(v):
+    return torch.from_numpy(np.asarray(v, np.float32)).to(torch.float8_e4m3fn).double().numpy()
+
+
+def _torch_quant_rows(a):
+    """Per-row e4m3 quantisation written with torch's float8 cast (a library rounding)."""
+    a32 = torch.from_numpy(np.asarray(a, np.float64)).float()
+    amax = a32.abs().amax(dim=-1)
+    sc = torch.where(amax > 0, amax / 448.0, torch.ones_like(amax))
+    q = (a32 / sc.unsqueeze(-1)).to(torch.float8_e4m3fn).double()
+    return (q * sc.double().unsqueeze(-1)).numpy()
+
+
+def check_e4m3_format(O):
+    """The e4m3 decoder, rounding, bf16 rounding and per-row quantiser against the format's
+    definition, torch's float8_e4m3fn / bfloat16 casts and brute-force nearest-value search."""
+    codes = np.arange(256, dtype=np.uint8)
+    dec = O.e4m3_decode(codes)
+    ref = torch.from_numpy(codes.copy()).view(torch.float8_e4m3fn).double().numpy()
+    assert np.array_equal(np.isnan(dec), np.isnan(ref)) and np.isnan(dec).sum() == 2
+    fin = ~np.isnan(ref)
+    assert np.array_equal(dec[fin], ref[fin])
+    assert dec[0x7E] == 448.0 and dec[0x01] == 2.0 ** -9 and dec[0x08] == 2.0 ** -6
+    assert dec[0x38] == 1.0 and dec[0xB8] == -1.0 and dec[0x80] == 0.0
+    grid, parity = _e4m3_grid()
+    assert O.E4M3_MAX == grid.max() == 448.0
+    # rounding: random fp32 values over every binade, exact midpoints, subnormals, saturation
+    rng = _rng(21)
+    v = (rng.standard_normal(4000) * np.exp2(rng.uniform(-12, 9, 4000))).astype(np.float32)
+    v = v[np.abs(v) < 464].astype(np.float64)
+    mids = ((grid[1:] + grid[:-1]) / 2)[np.abs((grid[1:] + grid[:-1]) / 2) < 448]
+    vals = np.concatenate([v, mids, [0.0, -0.0, 2.0 ** -10, 3 * 2.0 ** -10, 1.0625, 1.1875]])
+    got = O.e4m3_round(vals)
+    assert np.array_equal(got, _torch_e4m3(vals))
+    assert O.e4m3_round(np.array([1.0625, 1.1875, 2.0 ** -10, 3 * 2.0 ** -10])).tolist() == [1.0, 1.25, 0.0, 2.0 ** -8]
+    for x, q in zip(vals[:300], got[:300]):                   # brute force: nearest, ties to even
+        dist = np.abs(grid - x)
+        near = np.nonzero(dist == dist.min())[0]
+        want = grid[near[0]] if len(near) == 1 else grid[near[parity[near] == 0][0]]
+        assert q == want or (q == 0 and want == 0)
+    assert O.e4m3_round(np.array([449.0, 463.9, 465.0, 1e6, -1e6])).tolist() == [448.0, 448.0, 448.0, 448.0, -448.0]
+    # bf16 rounding against torch's cast, ties included
+    w = (rng.standard_normal(3000) * np.exp2(rng.uniform(-20, 20, 3000))).astype(np.float32)
+    ties = (np.float32(1.0) + np.float32(2.0 ** -8) * np.arange(1, 40, 2, dtype=np.float32)).astype(np.float32)
+    w = np.concatenate([w, ties, -ties])
+    assert np.array_equal(O.bf16_round(w), torch.from_numpy(w).bfloat16().double().numpy())
+    # per-row quantiser
+    a = rng.standard_normal((7, 33)) * np.exp2(rng.uniform(-8, 8, (7, 1)))
+    a[3] = 0.0
+    a = a.astype(np.float32).astype(np.float64)
+    q, sc = O.quantize_rows_e4m3(a)
+    assert sc.dtype == np.float32 and sc[3] == 1.0 and not q[3].any()
+    live = [0, 1, 2, 4, 5, 6]
+    assert np.array_equal(np.abs(q[live]).max(axis=1), np.full(6, 448.0))
+    assert np.array_equal(sc[live], (np.abs(a[live]).max(axis=1).astype(np.float32) / np.float32(448)))
+    assert np.array_equal(O.dequantized_rows(a), _torch_quant_rows(a))
+    rel = np.abs(O.dequantized_rows(a) - a)[live] / np.abs(a[live]).max(axis=1, keepdims=True)
+    assert rel.max() <= 16.0 / 448.0          # half of the widest step (32, in [256, 448]) per scale unit
+
+
+def check_fp8_layer_closed_form(O):
+    """The FP8 routed path on experts whose weight matrices hold one e4m3 code per row (a
+    selection of one input per output, so each Linear reduces to a scaled copy): the layer
+    must equal the closed form built from torch's e4m3 / bf16 casts and scipy's expit, with
+    routing, per-row activation scales, per-output-channel weight scales and an unquantised
+    shared expert."""
+    rng = _rng(22)
+    T, d, I, N, k = 6, 16, 8, 3, 2
+    x = rng.standard_normal((T, d)) * np.exp2(rng.uniform(-4, 4, (T, 1)))
+    x[2] = 0.0
+    x = x.astype(np.float32).astype(np.float64)
+    c = rng.normal(0, 0.5, (N, d))
+    experts, dense = [], []
+    for _ in range(N):
+        e = {}
+        for name, (rows, cols) in (("w1", (I, d)), ("w3", (I, d)), ("w2", (d, I))):
+            pick = rng.choice(cols, rows, replace=rows > cols)
+            code = rng.choice([cc for cc in range(256) if cc not in (0x7F, 0xFF)], rows).astype(np.uint8)
+            q = np.zeros((rows, cols), np.uint8)
+            q[np.arange(rows), pick] = code
+            e[name] = q
+            e["s" + name[1]] = np.exp2(rng.uniform(-9, -3, rows)).astype(np.float32)
+            e["p" + name[1]] = pick
+        for b, n in (("b1", I), ("b3", I), ("b2", d)):
+            e[b] = rng.normal(0, 0.1, n)
+        experts.append(e)
+    shared = _rand_expert(rng, d, 5, std=0.2)
+    stack = _stack([{k_: v for k_, v in e.items() if not k_.startswith("p")} for e in experts])
+    res = O.layer(x, c, stack, N, k, shared=_stack([shared]), n_shared=1, routed_e4m3=True)
+    r = O.route(x, c, k)
+    xq = _torch_quant_rows(x)
+
+    def val(e, name, rows):
+        code = e[name][np.arange(rows), e["p" + name[1]]]
+        return torch.from_numpy(code.copy()).view(torch.float8_e4m3fn).double().numpy() * e["s" + name[1]]
+
+    want = torch_expert(shared, x)
+    for t in range(T):
+        for j in range(k):
+            e = experts[r["idx"][t, j]]
+            a = val(e, "w1", I) * xq[t, e["p1"]] + e["b1"]
+            g = val(e, "w3", I) * xq[t, e["p3"]] + e["b3"]
+            h = a * scipy.special.expit(a) * g
+            hb = torch.from_numpy(h).float().bfloat16().double().numpy()
+            hq = _torch_quant_rows(hb[None])[0]
+            y = val(e, "w2", d) * hq[e["p2"]] + e["b2"]
+            want[t] += r["gate"][t, j] * y
+    assert np.allclose(res["out"], want, rtol=1e-12, atol=1e-12)
+
+
 ALL_CHECKS = [check_ptflops_printout, check_combinations, check_textbook_single_expert,
               check_gate_invariants, check_bruteforce_routing, check_split_identity,
-              check_shared_bypasses_router, check_hit_entropy, check_permute, check_gate_modes]
+              check_shared_bypasses_router, check_hit_entropy, check_permute, check_gate_modes,
+              check_e4m3_format, check_fp8_layer_closed_form]

@@ -10,7 +10,8 @@ import oracle.moe_oracle as O
 from tests import pins
 
 _orig = {name: getattr(O, name) for name in ("silu", "linear", "route", "swiglu_hidden", "permute",
-                                             "expert_macs", "split_expert", "hit_entropy")}
+                                             "expert_macs", "split_expert", "hit_entropy", "e4m3_round",
+                                             "quantize_rows_e4m3", "e4m3_weights", "e4m3_decode")}
 
 
 def _sigmoid_for_silu(a):                      # silu without the factor a
@@ -89,6 +90,57 @@ def _entropy_log2(idx, n):
     return e / np.log(2.0), a, c
 
 
+def _e4m3_truncate(v):                         # rounds toward zero instead of to nearest
+    v = np.asarray(v, np.float64)
+    a = np.abs(v)
+    _, ex = np.frexp(a)
+    step = np.ldexp(1.0, np.maximum(ex - 1, -6) - 3)
+    return np.copysign(np.minimum(np.floor(a / step) * step, 448.0), v)
+
+
+def _e4m3_ties_away(v):                        # ties away from zero
+    v = np.asarray(v, np.float64)
+    a = np.abs(v)
+    _, ex = np.frexp(a)
+    step = np.ldexp(1.0, np.maximum(ex - 1, -6) - 3)
+    return np.copysign(np.minimum(np.floor(a / step + 0.5) * step, 448.0), v)
+
+
+def _quant_per_tensor(a):                      # one scale for the whole matrix
+    a32 = np.asarray(a, np.float64).astype(np.float32)
+    amax = np.float32(np.abs(a32).max()) if a32.size else np.float32(0)
+    sc = np.full(a32.shape[:-1], amax / np.float32(448) if amax > 0 else np.float32(1), np.float32)
+    return O.e4m3_round((a32 / sc[..., None]).astype(np.float64)), sc
+
+
+def _quant_identity(a):                        # activations not quantised at all
+    a = np.asarray(a, np.float64)
+    return a, np.ones(a.shape[:-1], np.float32)
+
+
+def _weights_scale_by_column(w):               # channel scales applied along the input axis
+    out = {k: v for k, v in w.items() if k not in ("s1", "s3", "s2")}
+    for name, sname in (("w1", "s1"), ("w3", "s3"), ("w2", "s2")):
+        dec = O.e4m3_decode(w[name])
+        sc = np.asarray(w[sname], np.float64)
+        sc = np.resize(sc, dec.shape[1])
+        out[name] = dec * sc[None, :]
+    return out
+
+
+def _decode_no_subnormals(codes):              # exponent field 0 read as a normal number
+    c = np.asarray(codes, np.uint8).astype(np.int64)
+    e = (c >> 3) & 15
+    v = _orig["e4m3_decode"](codes)
+    m = (c & 7).astype(np.float64)
+    return np.where(e == 0, np.where(c >> 7, -1.0, 1.0) * (1 + m / 8.0) * 2.0 ** -7, v)
+
+
+def _bf16_truncate(a):                         # rounds toward zero on the fp32 pattern
+    u = np.asarray(a, np.float64).astype(np.float32).view(np.uint32) & np.uint32(0xFFFF0000)
+    return u.view(np.float32).astype(np.float64)
+
+
 MUTANTS = {
     "silu_is_sigmoid": ("silu", _sigmoid_for_silu),
     "linear_drops_bias": ("linear", _linear_no_bias),
@@ -101,6 +153,13 @@ MUTANTS = {
     "macs_without_bias": ("expert_macs", _macs_no_bias),
     "split_keeps_full_b2": ("split_expert", _split_no_b2_scale),
     "entropy_in_bits": ("hit_entropy", _entropy_log2),
+    "e4m3_truncates": ("e4m3_round", _e4m3_truncate),
+    "e4m3_ties_away": ("e4m3_round", _e4m3_ties_away),
+    "fp8_scale_per_tensor": ("quantize_rows_e4m3", _quant_per_tensor),
+    "fp8_activations_unquantised": ("quantize_rows_e4m3", _quant_identity),
+    "fp8_weight_scale_by_column": ("e4m3_weights", _weights_scale_by_column),
+    "e4m3_no_subnormals": ("e4m3_decode", _decode_no_subnormals),
+    "bf16_truncates": ("bf16_round", _bf16_truncate),
 }
 
 
