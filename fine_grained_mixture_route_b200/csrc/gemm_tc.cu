@@ -91,6 +91,9 @@ struct Params {
     float* partial;            // ROUTERP: [nsplit][T][E] fp32 partial logits
     int kb_per_split;          // ROUTERP: K blocks per split
     int group_m;               // tile raster: bands of group_m M-tiles swept across all N-tiles
+    int q8;                    // routed tiles read e4m3 A and B (K blocks of 128 bytes)
+    const float* a_scale;      // q8: per-row scale of the routed A rows (x_perm or h rows)
+    const float *ws1, *ws3, *ws2;  // q8: per-output-channel weight scales [E, I], [E, I], [E, d]
     int fold_shared;           // GEMM2R: shared-expert GEMM2 tiles follow the routed ones (-> sout)
     uint32_t* err;
 };
@@ -176,6 +179,19 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int n) {
     return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
 }
 
+// Instruction descriptor, kind::f8f6f4: fp32 accumulator, e4m3 A and B (format 0), K-major, M=128.
+__host__ __device__ constexpr uint32_t idesc_e4m3(int n) {
+    return (1u << 4) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+}
+// One e4m3 MMA: K = 32 (32 bytes of each operand row, like the 16 bf16 of mma_bf16).
+__device__ __forceinline__ void mma_e4m3(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a), "l"(b), "r"(idesc), "r"(acc)
+        : "memory");
+}
 __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
@@ -340,7 +356,7 @@ __device__ __forceinline__ Tile decode(const Params& p, int t) {
         band_mn(local, mt, ceil_div(shared ? p.Is : p.I, 128), p.group_m, m, n);
         x.m0 = m * TM;
         x.n0 = n * 128;
-        x.num_kb = ceil_div(p.d, BK);
+        x.num_kb = ceil_div(p.d, (p.q8 && !shared) ? 2 * BK : BK);
     } else if (MODE == GEMM2R && t >= p.tile_start[p.E]) {
         // shared-expert tile (fold_shared): all K_s experts accumulated along K
         const int mt = ceil_div(p.T, TM);
@@ -361,7 +377,7 @@ __device__ __forceinline__ Tile decode(const Params& p, int t) {
         band_mn(local, mt, ceil_div(p.d, 256), p.group_m, m, n);
         x.m0 = m * TM;
         x.n0 = n * 256;
-        x.num_kb = ceil_div(p.I, BK);
+        x.num_kb = ceil_div(p.I, p.q8 ? 2 * BK : BK);
     } else {
         const int mt = ceil_div(p.T, TM);
         x.g = 0; x.rows = p.T; x.row0 = 0;
@@ -461,7 +477,10 @@ __device__ __forceinline__ void epilogue_router(const Params& p, const Tile& x, 
     }
 }
 
-// GEMM1: the two epilogue warps of a TMEM lane quadrant split the 128 hidden columns.
+// GEMM1: the two epilogue warps of a TMEM lane quadrant split the 128 hidden columns.  On an
+// e4m3 routed tile (Q8) the accumulators are first multiplied by the row's activation scale
+// and the column's weight scale.
+template <bool Q8 = false>
 __device__ __forceinline__ void epilogue_gemm1(const Params& p, const Tile& x, uint32_t tacc, int row, int half) {
     const bool shared = x.g >= p.E;
     const int e = shared ? x.g - p.E : x.g;
@@ -470,8 +489,12 @@ __device__ __forceinline__ void epilogue_gemm1(const Params& p, const Tile& x, u
     const __nv_bfloat16* b3 = shared ? p.sb3 : p.b3;
     if (b1) b1 += (size_t)e * I;
     if (b3) b3 += (size_t)e * I;
+    const bool scaled = Q8 && !shared;          // e4m3 routed tile
+    const float* sc1 = scaled ? p.ws1 + (size_t)e * I : nullptr;
+    const float* sc3 = scaled ? p.ws3 + (size_t)e * I : nullptr;
     const int r = x.m0 + row;
     const bool live = r < x.rows;
+    const float rs = (scaled && live) ? p.a_scale[x.row0 + r] : 1.f;
     __nv_bfloat16* hrow = shared ? p.h_s + ((size_t)e * p.T + r) * I : p.h_r + (size_t)(x.row0 + r) * I;
 #pragma unroll 1
     for (int c = half * 2; c < half * 2 + 2; ++c) {
@@ -492,8 +515,12 @@ __device__ __forceinline__ void epilogue_gemm1(const Params& p, const Tile& x, u
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
                     const int j = q * 8 + i * 2 + h;
-                    float a = __uint_as_float(u[j]) + (b1 ? __bfloat162float(b1[col + i * 2 + h]) : 0.f);
-                    float g = __uint_as_float(v[j]) + (b3 ? __bfloat162float(b3[col + i * 2 + h]) : 0.f);
+                    const int cc = col + i * 2 + h;
+                    float a = __uint_as_float(u[j]);
+                    float g = __uint_as_float(v[j]);
+                    if (scaled) { a *= rs * sc1[cc]; g *= rs * sc3[cc]; }
+                    a += b1 ? __bfloat162float(b1[cc]) : 0.f;
+                    g += b3 ? __bfloat162float(b3[cc]) : 0.f;
                     hv[h] = silu_f32(a) * g;
                 }
                 pk[i] = pack_bf16(hv[0], hv[1]);
@@ -503,13 +530,18 @@ __device__ __forceinline__ void epilogue_gemm1(const Params& p, const Tile& x, u
     }
 }
 
-// GEMM2R: each epilogue warp of a quadrant takes 128 of the 256 output columns.
+// GEMM2R: each epilogue warp of a quadrant takes 128 of the 256 output columns.  On e4m3 tiles
+// (Q8) the accumulator is multiplied by the h row's scale and the column's weight scale before
+// b2 and the gate.
+template <bool Q8 = false>
 __device__ __forceinline__ void epilogue_gemm2r(const Params& p, const Tile& x, uint32_t tacc, int row, int half) {
     const int r = x.m0 + row;
     const bool live = r < x.rows;
     const long long pos = x.row0 + r;
     const float gate = live ? (p.sorted_gate ? p.sorted_gate[pos] : 1.f) : 0.f;
     const __nv_bfloat16* b2 = p.b2 ? p.b2 + (size_t)x.g * p.d : nullptr;
+    const float* sc2 = Q8 ? p.ws2 + (size_t)x.g * p.d : nullptr;
+    const float rs = (Q8 && live) ? p.a_scale[pos] : 1.f;
     __nv_bfloat16* yrow = p.y + (size_t)pos * p.d;
 #pragma unroll 1
     for (int c = half * 4; c < half * 4 + 4; ++c) {
@@ -526,8 +558,11 @@ __device__ __forceinline__ void epilogue_gemm2r(const Params& p, const Tile& x, 
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 const int j = q * 8 + i * 2;
-                float a = __uint_as_float(u[j]) + (b2 ? __bfloat162float(b2[col + i * 2]) : 0.f);
-                float b = __uint_as_float(u[j + 1]) + (b2 ? __bfloat162float(b2[col + i * 2 + 1]) : 0.f);
+                float a = __uint_as_float(u[j]);
+                float b = __uint_as_float(u[j + 1]);
+                if (Q8) { a *= rs * sc2[col + i * 2]; b *= rs * sc2[col + i * 2 + 1]; }
+                a += b2 ? __bfloat162float(b2[col + i * 2]) : 0.f;
+                b += b2 ? __bfloat162float(b2[col + i * 2 + 1]) : 0.f;
                 pk[i] = pack_bf16(gate * a, gate * b);
             }
             *reinterpret_cast<uint4*>(yrow + col) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
@@ -593,8 +628,13 @@ __device__ __forceinline__ void epilogue_router_partial(const Params& p, const T
 // leader's "accumulator empty" barrier.  A cluster barrier after set-up makes the leader's
 // barriers valid before any peer copy lands, and one before teardown keeps every shared
 // memory and TMEM range alive until the leader's last MMA has finished.
-template <int MODE, int KMAX, bool PAIR_>
+//
+// Q8 (single CTAs, GEMM1 / GEMM2R): routed tiles read e4m3 operands, K blocks of 128 (the same
+// 128-byte swizzle rows as 64 bf16), and run kind::f8f6f4 MMAs; shared-expert tiles of the
+// same launch stay bf16.
+template <int MODE, int KMAX, bool PAIR_, bool Q8 = false>
 __global__ void __launch_bounds__(THREADS, 1) moe_tc_kernel(const __grid_constant__ Params p) {
+    static_assert(!Q8 || (!PAIR_ && (MODE == GEMM1 || MODE == GEMM2R)), "e4m3 tiles: single-CTA expert GEMMs");
     using C = Cfg<MODE, PAIR_>;
     constexpr bool PAIR = C::PAIR;
     constexpr int STAGES = C::STAGES;
@@ -702,12 +742,14 @@ __global__ void __launch_bounds__(THREADS, 1) moe_tc_kernel(const __grid_constan
                         if (MODE == GEMM1) {
                             const bool shared = x.g >= p.E;
                             const int e = shared ? x.g - p.E : x.g;
-                            tma_load_2d(a_dst, &p.tmA[shared ? 1 : 0], fb, kb * BK, x.row0 + x.m0);
-                            tma_load_3d(b_dst, &p.tmB[shared ? 2 : 0], fb, kb * BK, x.n0, e);
-                            tma_load_3d(b_dst + B_BYTES / 2, &p.tmB[shared ? 3 : 1], fb, kb * BK, x.n0, e);
+                            const int kc = kb * ((Q8 && !shared) ? 2 * BK : BK);   // K element offset
+                            tma_load_2d(a_dst, &p.tmA[shared ? 1 : 0], fb, kc, x.row0 + x.m0);
+                            tma_load_3d(b_dst, &p.tmB[shared ? 2 : 0], fb, kc, x.n0, e);
+                            tma_load_3d(b_dst + B_BYTES / 2, &p.tmB[shared ? 3 : 1], fb, kc, x.n0, e);
                         } else if (MODE == GEMM2R && x.g >= 0) {
-                            tma_load_2d(a_dst, &p.tmA[0], fb, kb * BK, x.row0 + x.m0);
-                            tma_load_3d(b_dst, &p.tmB[0], fb, kb * BK, x.n0, x.g);
+                            const int kc = kb * (Q8 ? 2 * BK : BK);
+                            tma_load_2d(a_dst, &p.tmA[0], fb, kc, x.row0 + x.m0);
+                            tma_load_3d(b_dst, &p.tmB[0], fb, kc, x.n0, x.g);
                         } else if (MODE == GEMM2R) {
                             const int kbs = ceil_div(p.Is, BK);
                             const int s = kb / kbs, kk = kb % kbs;
@@ -745,6 +787,8 @@ __global__ void __launch_bounds__(THREADS, 1) moe_tc_kernel(const __grid_constan
             bool ok = true;
             for (int t = cta_slot; ok && t < ntiles; t += cta_slots) {
                 const Tile x = decode<MODE, PAIR>(p, t);
+                const bool q8tile = Q8 && (MODE == GEMM1 ? x.g < p.E : x.g >= 0);
+                const uint32_t idesc_t = q8tile ? idesc_e4m3(p.n_mma) : idesc;
                 if (!mbar_wait(tempty_bar(acc), acc_phase ^ 1u, abort_flag, p.err)) break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + (uint32_t)(acc * ACC_COLS);
@@ -757,7 +801,8 @@ __global__ void __launch_bounds__(THREADS, 1) moe_tc_kernel(const __grid_constan
                         const uint64_t ad = sw128_desc(a_addr + k * 32), bd = sw128_desc(b_addr + k * 32);
                         const uint32_t accum = (kb > 0 || k > 0) ? 1u : 0u;
                         if (PAIR) mma_bf16_pair(d_tmem, ad, bd, idesc, accum);
-                        else mma_bf16(d_tmem, ad, bd, idesc, accum);
+                        else if (q8tile) mma_e4m3(d_tmem, ad, bd, idesc_t, accum);
+                        else mma_bf16(d_tmem, ad, bd, idesc_t, accum);
                     }
                     if (PAIR) mma_commit_pair_both(empty_bar(stage));
                     else mma_commit(empty_bar(stage));
@@ -791,9 +836,9 @@ __global__ void __launch_bounds__(THREADS, 1) moe_tc_kernel(const __grid_constan
             } else if (MODE == ROUTERP) {
                 epilogue_router_partial(p, x, tacc, row, half);
             } else if (MODE == GEMM1) {
-                epilogue_gemm1(p, x, tacc, row, half);
+                epilogue_gemm1<Q8>(p, x, tacc, row, half);
             } else if (MODE == GEMM2R) {
-                if (x.g >= 0) epilogue_gemm2r(p, x, tacc, row, half);
+                if (x.g >= 0) epilogue_gemm2r<Q8>(p, x, tacc, row, half);
                 else epilogue_gemm2s(p, x, tacc, row, half);
             } else {
                 epilogue_gemm2s(p, x, tacc, row, half);
@@ -854,11 +899,27 @@ bool make_map(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t mid, uin
     return r == CUDA_SUCCESS;
 }
 
+// e4m3 (byte) tensor [outer][mid][inner] with a box of box_inner x box_mid (x 1); inner must
+// be a multiple of 16 (16-byte strides)
+bool make_map_u8(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t mid, uint64_t outer, uint32_t box_inner,
+                 uint32_t box_mid, bool three_d) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn || inner % 16) return false;
+    cuuint64_t dims[3] = {inner, mid, outer};
+    cuuint64_t strides[2] = {inner, inner * mid};
+    cuuint32_t box[3] = {box_inner, box_mid, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, three_d ? 3 : 2, const_cast<void*>(ptr), dims, strides, box,
+                    estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 // Launches MODE.  Pair modes run as clusters of 2 CTAs; `tiles` bounds the useful CTAs (pairs
 // for pair modes), and the grid never exceeds what can be resident at once (persistent loop).
-template <int MODE, int KMAX, bool PAIR = false>
+template <int MODE, int KMAX, bool PAIR = false, bool Q8 = false>
 cudaError_t launch(const Params& p, int tiles, cudaStream_t stream) {
-    auto kern = moe_tc_kernel<MODE, KMAX, PAIR>;
+    auto kern = moe_tc_kernel<MODE, KMAX, PAIR, Q8>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
@@ -1039,6 +1100,69 @@ cudaError_t launch_tc_gemm2_shared(const Dims& D, const FfnWeights& Sh, const vo
     const int n = ceil_div(D.d, 256);
     return tc::pairs_for(D) ? launch<GEMM2S, 8, true>(p, ceil_div(D.T, 256) * n, stream)
                          : launch<GEMM2S, 8, false>(p, ceil_div(D.T, 128) * n, stream);
+}
+
+// e4m3 routed experts: GEMM1 over x8_perm (e4m3 rows, one scale per row in xs) and the e4m3
+// W1 / W3 codes with their channel scales; shared groups [E, g_end) stay bf16 on x.
+cudaError_t launch_tc_gemm1_q8(const Dims& D, const void* x, const void* x8_perm, const float* xs,
+                               const int32_t* offsets, const int32_t* tile_start1, const FfnWeights& R,
+                               const FfnWeights& Sh, void* h_r, void* h_s, int g_end, uint32_t* err,
+                               cudaStream_t stream) {
+    using namespace tc;
+    if (D.T == 0) return cudaSuccess;
+    if (!R.s1 || !R.s3 || !xs) return cudaErrorInvalidValue;
+    Params p = base_params(D, err);
+    p.q8 = 1;
+    p.a_scale = xs;
+    p.ws1 = R.s1; p.ws3 = R.s3;
+    p.tile_start = tile_start1;
+    p.offsets = offsets;
+    p.g_begin = 0;
+    p.g_end = g_end;
+    p.b1 = (const __nv_bfloat16*)R.b1; p.b3 = (const __nv_bfloat16*)R.b3;
+    p.sb1 = (const __nv_bfloat16*)Sh.b1; p.sb3 = (const __nv_bfloat16*)Sh.b3;
+    p.h_r = (__nv_bfloat16*)h_r; p.h_s = (__nv_bfloat16*)h_s;
+    bool ok = make_map_u8(&p.tmA[0], x8_perm, D.d, (uint64_t)D.slots(), 1, 2 * BK, BM, false);
+    ok &= make_map_u8(&p.tmB[0], R.w1, D.d, D.I, D.E, 2 * BK, 128, true);
+    ok &= make_map_u8(&p.tmB[1], R.w3, D.d, D.I, D.E, 2 * BK, 128, true);
+    if (g_end > D.E) {
+        ok &= make_map(&p.tmA[1], x, D.d, D.T, 1, BK, BM, false);
+        ok &= make_map(&p.tmB[2], Sh.w1, D.d, D.Is, D.Ks, BK, 128, true);
+        ok &= make_map(&p.tmB[3], Sh.w3, D.d, D.Is, D.Ks, BK, 128, true);
+    }
+    if (!ok) return cudaErrorInvalidValue;
+    return launch<GEMM1, 8, false, true>(p, num_sms(), stream);
+}
+
+// e4m3 routed GEMM2 over h8 (e4m3 rows, scale per row in hs) and the e4m3 W2 codes; with Sh the
+// shared experts' bf16 GEMM2 tiles follow in the same launch (-> sout), as in the bf16 path.
+cudaError_t launch_tc_gemm2_routed_q8(const Dims& D, const int32_t* offsets, const int32_t* tile_start2,
+                                      const float* sorted_gate, const FfnWeights& R, const void* h8,
+                                      const float* hs, void* y_sorted, const FfnWeights* Sh, const void* h_s,
+                                      float* sout, uint32_t* err, cudaStream_t stream) {
+    using namespace tc;
+    if (D.T == 0) return cudaSuccess;
+    if (!R.s2 || !hs) return cudaErrorInvalidValue;
+    Params p = base_params(D, err);
+    p.q8 = 1;
+    p.a_scale = hs;
+    p.ws2 = R.s2;
+    p.tile_start = tile_start2;
+    p.offsets = offsets;
+    p.sorted_gate = sorted_gate;
+    p.b2 = (const __nv_bfloat16*)R.b2;
+    p.y = (__nv_bfloat16*)y_sorted;
+    bool ok = make_map_u8(&p.tmA[0], h8, D.I, (uint64_t)D.slots(), 1, 2 * BK, BM, false);
+    ok &= make_map_u8(&p.tmB[0], R.w2, D.I, D.d, D.E, 2 * BK, 256, true);
+    if (Sh && D.Ks > 0 && sout) {
+        p.fold_shared = 1;
+        p.sb2 = (const __nv_bfloat16*)Sh->b2;
+        p.sout = sout;
+        ok &= make_map(&p.tmA[1], h_s, D.Is, D.T, D.Ks, BK, BM, true);
+        ok &= make_map(&p.tmB[1], Sh->w2, D.Is, D.d, D.Ks, BK, 256, true);
+    }
+    if (!ok) return cudaErrorInvalidValue;
+    return launch<GEMM2R, 8, false, true>(p, num_sms(), stream);
 }
 
 }  // namespace moe

@@ -15,6 +15,7 @@ struct Dims {
     bool bias;
     bool bf16;
     int gate_mode = 0;     // moe_gate_mode_t
+    bool q8 = false;       // routed experts in e4m3 (moe_expert_fmt_t MOE_FMT_E4M3)
     long long slots() const { return (long long)T * k; }
 };
 
@@ -47,6 +48,13 @@ cudaError_t launch_plan(const Dims& D, const int32_t* offsets, int32_t* tile_sta
 cudaError_t launch_gather(const Dims& D, const void* x, const int32_t* sorted_token, void* x_perm,
                           uint32_t* err, cudaStream_t stream);
 
+// Per-row e4m3 quantisation of bf16 rows: for each output row p, src row r = row_of[p] (or p
+// when row_of is NULL, r checked against src_rows), scale[p] = max|src[r]| / 448 (1 for a zero
+// row), dst[p, :] = e4m3 round-to-nearest-even (saturating) of src[r, :] / scale[p], the
+// division in IEEE fp32.  width % 8 == 0.
+cudaError_t launch_quant_rows(const void* src, const int32_t* row_of, long long n_rows, int src_rows, int width,
+                              uint8_t* dst, float* scale, uint32_t* err, cudaStream_t stream);
+
 // out[t, :] = base[t, :] + sum_j y_sorted[slot_of[t*k + j], :] in fp32, rounded once; base is
 // the shared experts' fp32 output [T, d], or NULL when there are none.
 cudaError_t launch_combine(const Dims& D, const void* y_sorted, const int32_t* slot_of, const float* base,
@@ -55,6 +63,7 @@ cudaError_t launch_combine(const Dims& D, const void* y_sorted, const int32_t* s
 // ---- CUDA-core grouped FFN (fp32 layers) ----------------------------------------------
 struct FfnWeights {
     const void *w1, *b1, *w3, *b3, *w2, *b2;
+    const float *s1 = nullptr, *s3 = nullptr, *s2 = nullptr;   // e4m3 codes: per-output-channel scales
 };
 
 // h rows of groups [g_begin, g_end): routed group e -> h_r[offsets[e] + r], shared group
@@ -103,5 +112,18 @@ cudaError_t launch_tc_gemm2_shared(const Dims& D, const FfnWeights& shared, cons
                                    uint32_t* err, cudaStream_t stream);
 
 int num_sms();
+
+// e4m3 routed experts (D.q8).  GEMM1: routed groups read x8_perm rows (scale per row in xs)
+// against the W1 / W3 codes (R.s1, R.s3); shared groups [E, g_end) run bf16 on x in the same
+// launch.  GEMM2R: h8 rows (scale per row in hs) against the W2 codes (R.s2); with Sh the
+// shared experts' bf16 GEMM2 tiles follow (-> sout).
+cudaError_t launch_tc_gemm1_q8(const Dims& D, const void* x, const void* x8_perm, const float* xs,
+                               const int32_t* offsets, const int32_t* tile_start1, const FfnWeights& R,
+                               const FfnWeights& Sh, void* h_r, void* h_s, int g_end, uint32_t* err,
+                               cudaStream_t stream);
+cudaError_t launch_tc_gemm2_routed_q8(const Dims& D, const int32_t* offsets, const int32_t* tile_start2,
+                                      const float* sorted_gate, const FfnWeights& R, const void* h8,
+                                      const float* hs, void* y_sorted, const FfnWeights* Sh, const void* h_s,
+                                      float* sout, uint32_t* err, cudaStream_t stream);
 
 }  // namespace moe

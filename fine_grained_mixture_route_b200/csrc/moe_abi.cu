@@ -14,7 +14,9 @@ namespace {
 size_t al(size_t x) { return (x + 255) & ~(size_t)255; }
 
 struct Layout {
-    size_t err, hist, rpart, sout, ts1, ts2, idx, gate, counts, offsets, stok, sgate, slot_of, xperm, hr, hs, y, total;
+    size_t err, hist, rpart, sout, ts1, ts2, idx, gate, counts, offsets, stok, sgate, slot_of, xperm, hr, hs, y;
+    size_t xs, h8, hsc;    // e4m3 routed experts: row scales of x8 (in xperm), h8 rows and their scales
+    size_t total;
 };
 
 Layout layout(const Dims& D) {
@@ -40,6 +42,9 @@ Layout layout(const Dims& D) {
     L.hr = o; o += al(S * D.I * esz);
     L.hs = o; o += al((size_t)D.Ks * D.T * (D.Ks ? D.Is : 0) * esz);
     L.y = o; o += al(S * D.d * esz);
+    L.xs = o; o += D.q8 ? al(S * 4) : 0;
+    L.h8 = o; o += D.q8 ? al(S * D.I) : 0;
+    L.hsc = o; o += D.q8 ? al(S * 4) : 0;
     L.total = o;
     return L;
 }
@@ -58,10 +63,14 @@ moe_status_t to_dims(const moe_shape_t* s, Dims* D) {
     if (s->dtype == MOE_BF16) {
         if (s->d % 8 || s->inter % 8 || (s->n_shared > 0 && s->inter_shared % 8)) return MOE_ERR_UNSUPPORTED;
     }
+    if (s->routed_fmt != MOE_FMT_NATIVE && s->routed_fmt != MOE_FMT_E4M3) return MOE_ERR_INVALID_ARG;
+    if (s->routed_fmt == MOE_FMT_E4M3 && (s->dtype != MOE_BF16 || s->d % 16 || s->inter % 16))
+        return MOE_ERR_UNSUPPORTED;
     D->T = s->T; D->d = s->d; D->E = s->n_experts; D->I = s->inter; D->k = s->top_k;
     D->Ks = s->n_shared; D->Is = s->n_shared > 0 ? s->inter_shared : 0;
     D->bias = s->has_bias != 0; D->bf16 = s->dtype == MOE_BF16;
     D->gate_mode = s->gate_mode;
+    D->q8 = s->routed_fmt == MOE_FMT_E4M3;
     return MOE_OK;
 }
 
@@ -70,11 +79,16 @@ moe_status_t check_ws(const Dims& D, void* ws, size_t ws_bytes) {
     return MOE_OK;
 }
 
-moe_status_t check_weights(const Dims& D, const moe_ffn_weights_t* w) {
+// e4m3: the stack must carry its three scale arrays (routed experts of an MOE_FMT_E4M3
+// layer); otherwise all three must be NULL.
+moe_status_t check_weights(const Dims& D, const moe_ffn_weights_t* w, bool e4m3 = false) {
     if (!w || !w->w1 || !w->w3 || !w->w2) return MOE_ERR_INVALID_ARG;
     const bool b = w->b1 && w->b3 && w->b2;
     const bool none = !w->b1 && !w->b3 && !w->b2;
     if (D.bias ? !b : !none) return MOE_ERR_INVALID_ARG;
+    const bool sc = w->s1 && w->s3 && w->s2;
+    const bool nosc = !w->s1 && !w->s3 && !w->s2;
+    if (e4m3 ? !sc : !nosc) return MOE_ERR_INVALID_ARG;
     return MOE_OK;
 }
 
@@ -101,7 +115,10 @@ T* at(void* ws, size_t off) { return reinterpret_cast<T*>(static_cast<char*>(ws)
 
 FfnWeights to_ffn(const moe_ffn_weights_t* w) {
     FfnWeights f = {nullptr, nullptr, nullptr, nullptr, nullptr, nullptr};
-    if (w) { f.w1 = w->w1; f.b1 = w->b1; f.w3 = w->w3; f.b3 = w->b3; f.w2 = w->w2; f.b2 = w->b2; }
+    if (w) {
+        f.w1 = w->w1; f.b1 = w->b1; f.w3 = w->w3; f.b3 = w->b3; f.w2 = w->w2; f.b2 = w->b2;
+        f.s1 = w->s1; f.s3 = w->s3; f.s2 = w->s2;
+    }
     return f;
 }
 
@@ -121,7 +138,17 @@ moe_status_t do_expert_ffn(const Dims& D, const Layout& L, void* ws, const void*
     int32_t* ts1 = at<int32_t>(ws, L.ts1);
     int32_t* ts2 = at<int32_t>(ws, L.ts2);
     if (!plan_done) MOE_CUDA(launch_plan(D, offsets, ts1, ts2, err, st));
-    if (D.bf16) {
+    if (D.q8) {
+        uint8_t* x8 = at<uint8_t>(ws, L.xperm);
+        float* xs = at<float>(ws, L.xs);
+        MOE_CUDA(launch_quant_rows(x, stok, D.slots(), D.T, D.d, x8, xs, err, st));
+        FfnWeights none = {nullptr, nullptr, nullptr, nullptr, nullptr, nullptr};
+        MOE_CUDA(launch_tc_gemm1_q8(D, x, x8, xs, offsets, ts1, R, none, at<void>(ws, L.hr), nullptr, D.E, err, st));
+        uint8_t* h8 = at<uint8_t>(ws, L.h8);
+        float* hsc = at<float>(ws, L.hsc);
+        MOE_CUDA(launch_quant_rows(at<void>(ws, L.hr), nullptr, D.slots(), (int)D.slots(), D.I, h8, hsc, err, st));
+        MOE_CUDA(launch_tc_gemm2_routed_q8(D, offsets, ts2, sgate, R, h8, hsc, y, nullptr, nullptr, nullptr, err, st));
+    } else if (D.bf16) {
         void* xp = at<void>(ws, L.xperm);
         MOE_CUDA(launch_gather(D, x, stok, xp, err, st));
         FfnWeights none = {nullptr, nullptr, nullptr, nullptr, nullptr, nullptr};
@@ -170,8 +197,9 @@ MOE_EXPORT int32_t moe_layer_launches(const moe_shape_t* shape) {
     else n += 1;
     n += 3;                                                         // histogram, scan, scatter
     n += 1;                                                         // tile tables
-    if (D.bf16) n += 1;                                             // row gather
+    if (D.bf16) n += 1;                                             // row gather (+ e4m3 quantisation)
     n += 3;                                   // GEMM1, GEMM2 (routed + shared tiles), combine
+    if (D.q8) n += 1;                                               // hidden-row quantisation
     return n;
 }
 
@@ -236,7 +264,7 @@ MOE_EXPORT moe_status_t moe_expert_ffn(const moe_shape_t* shape, const void* x, 
     Dims D;
     MOE_TRY(to_dims(shape, &D));
     if (!x || !offsets || !sorted_token || !y_sorted) return MOE_ERR_INVALID_ARG;
-    MOE_TRY(check_weights(D, routed));
+    MOE_TRY(check_weights(D, routed, D.q8));
     MOE_TRY(check_ws(D, ws, ws_bytes));
     if (D.T == 0) return MOE_OK;
     MOE_TRY(check_device());
@@ -286,6 +314,22 @@ MOE_EXPORT moe_status_t moe_combine(const moe_shape_t* shape, const void* x, con
     return MOE_OK;
 }
 
+MOE_EXPORT moe_status_t moe_quantize_rows_e4m3(const void* src, const int32_t* row_of, int64_t n_rows,
+                                               int32_t src_rows, int32_t width, uint8_t* dst, float* scale, void* ws,
+                                               size_t ws_bytes, moe_stream_t stream) {
+    if (n_rows < 0 || src_rows < 0 || width < 1 || n_rows >= (1LL << 31)) return MOE_ERR_INVALID_ARG;
+    if (!row_of && n_rows > src_rows) return MOE_ERR_INVALID_ARG;
+    if (width % 8) return MOE_ERR_UNSUPPORTED;
+    if (!ws || ws_bytes < 256 || ((uintptr_t)ws & 15u)) return MOE_ERR_WORKSPACE;
+    if (n_rows == 0) return MOE_OK;
+    if (!src || !dst || !scale) return MOE_ERR_INVALID_ARG;
+    MOE_TRY(check_device());
+    cudaGetLastError();
+    MOE_CUDA(launch_quant_rows(src, row_of, n_rows, src_rows, width, dst, scale, static_cast<uint32_t*>(ws),
+                               (cudaStream_t)stream));
+    return MOE_OK;
+}
+
 }  // extern "C"
 
 namespace moe {
@@ -300,7 +344,7 @@ moe_status_t layer_forward_impl(const moe_shape_t* shape, const void* x, const v
     Dims D;
     MOE_TRY(to_dims(shape, &D));
     if (!x || !centroids || !out) return MOE_ERR_INVALID_ARG;
-    MOE_TRY(check_weights(D, routed));
+    MOE_TRY(check_weights(D, routed, D.q8));
     if (D.Ks > 0) MOE_TRY(check_weights(D, shared));
     else if (shared) return MOE_ERR_INVALID_ARG;
     MOE_TRY(check_ws(D, ws, ws_bytes));
@@ -331,7 +375,22 @@ moe_status_t layer_forward_impl(const moe_shape_t* shape, const void* x, const v
     if (!mark(2)) return MOE_ERR_CUDA;
     MOE_CUDA(launch_plan(D, offsets, ts1, ts2, err, st));
     if (!mark(3)) return MOE_ERR_CUDA;
-    if (D.bf16) {
+    if (D.q8) {
+        uint8_t* x8 = at<uint8_t>(ws, L.xperm);
+        float* xs = at<float>(ws, L.xs);
+        MOE_CUDA(launch_quant_rows(x, stok, D.slots(), D.T, D.d, x8, xs, err, st));
+        if (!mark(4)) return MOE_ERR_CUDA;
+        MOE_CUDA(launch_tc_gemm1_q8(D, x, x8, xs, offsets, ts1, R, Sh, hr, hs, D.E + D.Ks, err, st));
+        if (!mark(5)) return MOE_ERR_CUDA;
+        uint8_t* h8 = at<uint8_t>(ws, L.h8);
+        float* hsc = at<float>(ws, L.hsc);
+        MOE_CUDA(launch_quant_rows(hr, nullptr, D.slots(), (int)D.slots(), D.I, h8, hsc, err, st));
+        float* sout = D.Ks > 0 ? at<float>(ws, L.sout) : nullptr;
+        MOE_CUDA(launch_tc_gemm2_routed_q8(D, offsets, ts2, sgate, R, h8, hsc, y, D.Ks > 0 ? &Sh : nullptr, hs, sout,
+                                           err, st));
+        if (!mark(6)) return MOE_ERR_CUDA;
+        MOE_CUDA(launch_combine(D, y, slot_of, sout, out, err, st));
+    } else if (D.bf16) {
         void* xp = at<void>(ws, L.xperm);
         MOE_CUDA(launch_gather(D, x, stok, xp, err, st));
         if (!mark(4)) return MOE_ERR_CUDA;

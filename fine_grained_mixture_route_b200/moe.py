@@ -17,10 +17,11 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe_b200
 MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_CUDA, MOE_ERR_INTERNAL = range(6)
 MOE_F32, MOE_BF16 = 0, 1
 GATE_SOFTMAX_TOPK, GATE_TOPK_SOFTMAX, GATE_SIGMOID_BIAS = 0, 1, 2
+FMT_NATIVE, FMT_E4M3 = 0, 1        # storage of the routed experts' weights (moe_expert_fmt_t)
 
 EXPORTED = ("moe_workspace_bytes", "moe_layer_launches", "moe_status_string", "moe_version", "moe_check_device_error", "moe_ws_init",
             "moe_route", "moe_permute", "moe_expert_ffn", "moe_combine", "moe_layer_forward",
-            "moe_layer_forward_timed", "moe_permute_no_alloc")
+            "moe_layer_forward_timed", "moe_permute_no_alloc", "moe_quantize_rows_e4m3")
 NUM_STAGES = 7
 STAGE_NAMES = ("router", "permute", "plan", "gather", "gemm1_swiglu", "gemm2", "combine")
 
@@ -28,11 +29,11 @@ STAGE_NAMES = ("router", "permute", "plan", "gather", "gemm1_swiglu", "gemm2", "
 class MoeShape(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in
                 ("T", "d", "n_experts", "inter", "top_k", "n_shared", "inter_shared", "has_bias", "dtype",
-                 "gate_mode")]
+                 "gate_mode", "routed_fmt")]
 
 
 class MoeWeights(ctypes.Structure):
-    _fields_ = [(n, ctypes.c_void_p) for n in ("w1", "b1", "w3", "b3", "w2", "b2")]
+    _fields_ = [(n, ctypes.c_void_p) for n in ("w1", "b1", "w3", "b3", "w2", "b2", "s1", "s3", "s2")]
 
 
 class MoeError(RuntimeError):
@@ -72,8 +73,10 @@ def _lib():
         lib.moe_layer_forward.argtypes = [sh, vp, vp, f32p, wp, wp, vp, i32p, f32p, i32p, vp, sz, vp]
         lib.moe_layer_forward_timed.argtypes = [sh, vp, vp, f32p, wp, wp, vp, i32p, f32p, i32p, vp, sz, vp,
                                                 ctypes.POINTER(ctypes.c_void_p), ctypes.c_int32]
+        lib.moe_quantize_rows_e4m3.argtypes = [vp, i32p, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, vp, f32p,
+                                               vp, sz, vp]
         for n in ("moe_check_device_error", "moe_ws_init", "moe_route", "moe_permute", "moe_expert_ffn",
-                  "moe_combine", "moe_layer_forward", "moe_layer_forward_timed"):
+                  "moe_combine", "moe_layer_forward", "moe_layer_forward_timed", "moe_quantize_rows_e4m3"):
             getattr(lib, n).restype = ctypes.c_int
         _LIB = lib
     return _LIB
@@ -99,9 +102,10 @@ def _check(status: int, where: str):
 
 
 def make_shape(T: int, d: int, n_experts: int, inter: int, top_k: int, n_shared: int = 0, inter_shared: int = 0,
-               has_bias: bool = True, dtype: torch.dtype = torch.bfloat16, gate_mode: int = GATE_SOFTMAX_TOPK) -> MoeShape:
+               has_bias: bool = True, dtype: torch.dtype = torch.bfloat16, gate_mode: int = GATE_SOFTMAX_TOPK,
+               routed_fmt: int = FMT_NATIVE) -> MoeShape:
     return MoeShape(T, d, n_experts, inter, top_k, n_shared, inter_shared if n_shared else 0, int(bool(has_bias)),
-                    MOE_BF16 if dtype == torch.bfloat16 else MOE_F32, gate_mode)
+                    MOE_BF16 if dtype == torch.bfloat16 else MOE_F32, gate_mode, routed_fmt)
 
 
 def shape_of(x: torch.Tensor, centroids_or_E, routed: Dict, top_k: int, shared: Optional[Dict] = None,
@@ -110,7 +114,9 @@ def shape_of(x: torch.Tensor, centroids_or_E, routed: Dict, top_k: int, shared: 
     I = routed["w1"].shape[1]
     Ks = 0 if shared is None else shared["w1"].shape[0]
     Is = 0 if shared is None else shared["w1"].shape[1]
-    return make_shape(x.shape[0], x.shape[1], E, I, top_k, Ks, Is, routed.get("b1") is not None, x.dtype, gate_mode)
+    fmt = FMT_E4M3 if routed["w1"].dtype == torch.uint8 else FMT_NATIVE    # e4m3 codes (quant.quantize_stack)
+    return make_shape(x.shape[0], x.shape[1], E, I, top_k, Ks, Is, routed.get("b1") is not None, x.dtype, gate_mode,
+                      fmt)
 
 
 def _bias_ptr(router_bias: Optional[torch.Tensor]):
@@ -124,11 +130,16 @@ def _bias_ptr(router_bias: Optional[torch.Tensor]):
 def _weights(w: Optional[Dict]):
     if w is None:
         return None
-    for k in ("w1", "w3", "w2", "b1", "b3", "b2"):
+    for k in ("w1", "w3", "w2", "b1", "b3", "b2", "s1", "s3", "s2"):
         t = w.get(k)
         if t is not None and not t.is_contiguous():
             raise ValueError(f"weight {k} must be contiguous")
-    return MoeWeights(*(None if w.get(k) is None else w[k].data_ptr() for k in ("w1", "b1", "w3", "b3", "w2", "b2")))
+    if w["w1"].dtype == torch.uint8:
+        for k in ("s1", "s3", "s2"):
+            if w.get(k) is None or w[k].dtype != torch.float32:
+                raise ValueError(f"e4m3 weights need float32 scales {k}")
+    names = ("w1", "b1", "w3", "b3", "w2", "b2", "s1", "s3", "s2")
+    return MoeWeights(*(None if w.get(k) is None else w[k].data_ptr() for k in names))
 
 
 def workspace_bytes(shape: MoeShape) -> int:
@@ -209,6 +220,20 @@ def layer_forward(shape: MoeShape, x, centroids, routed: Dict, shared: Optional[
                                     None if sw is None else ctypes.byref(sw), _ptr(out), _ptr(idx), _ptr(gate),
                                     _ptr(counts), _ptr(ws), ws.numel(), _stream(stream)), "moe_layer_forward")
     return out
+
+
+def quantize_rows_e4m3(src: torch.Tensor, ws: torch.Tensor, row_of: Optional[torch.Tensor] = None, stream=None):
+    """Per-row e4m3 quantisation of bf16 rows (moe_quantize_rows_e4m3): returns (codes uint8
+    [n_rows, width], scales fp32 [n_rows]); rows are src[row_of[p]] when row_of is given."""
+    if src.dtype != torch.bfloat16 or src.dim() != 2 or not src.is_contiguous():
+        raise ValueError("src must be a contiguous bf16 matrix")
+    n = src.shape[0] if row_of is None else row_of.shape[0]
+    codes = torch.empty((n, src.shape[1]), dtype=torch.uint8, device=src.device)
+    scales = torch.empty(n, dtype=torch.float32, device=src.device)
+    _check(_lib().moe_quantize_rows_e4m3(_ptr(src), _ptr(row_of), n, src.shape[0], src.shape[1], _ptr(codes),
+                                         _ptr(scales), _ptr(ws), ws.numel(), _stream(stream)),
+           "moe_quantize_rows_e4m3")
+    return codes, scales
 
 
 def stage_events(stream=None):

@@ -38,6 +38,16 @@
  *    n_experts); 0 <= n_shared <= 16; d, inter, inter_shared >= 1.  For MOE_BF16, d, inter
  *    and inter_shared must be multiples of 8 (16-byte rows for the tensor-memory-access
  *    unit).  T == 0 is a valid no-op.
+ *  - FP8 routed experts (shape->routed_fmt == MOE_FMT_E4M3; dtype must be MOE_BF16, d and inter
+ *    multiples of 16): the routed w1, w3, w2 are e4m3 codes (1 byte each, same layouts) with
+ *    fp32 scales per output channel in s1 [E, inter], s3 [E, inter], s2 [E, d]; the weight is
+ *    code * scale.  Each routed expert's input row and each SwiGLU hidden row (rounded to bf16)
+ *    is quantised to e4m3 with scale = row max |.| / 448 (division in IEEE fp32, round to
+ *    nearest even, saturating), and the expert GEMMs run on the e4m3 tensor-core path with the
+ *    scales applied to the fp32 accumulators.  Biases, the router, the shared experts (bf16)
+ *    and every output keep shape->dtype.  The pages name FP8 for fine-grained MoE and for
+ *    DeepSeek-V3 ("DeepSeek MoE模型优化与未来演进及字节超稀疏内存技术" and the report's §6.2)
+ *    without a recipe; this recipe is the library's own.
  */
 #ifndef MOE_B200_H
 #define MOE_B200_H
@@ -75,6 +85,10 @@ typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype_t;
  *                          mentions for DeepSeek-V3, §6.2; no formula on the pages). */
 typedef enum { MOE_GATE_SOFTMAX_TOPK = 0, MOE_GATE_TOPK_SOFTMAX = 1, MOE_GATE_SIGMOID_BIAS = 2 } moe_gate_mode_t;
 
+/* Storage of the routed experts' weight matrices: MOE_FMT_NATIVE = shape->dtype,
+ * MOE_FMT_E4M3 = e4m3 codes with per-output-channel fp32 scales (see above). */
+typedef enum { MOE_FMT_NATIVE = 0, MOE_FMT_E4M3 = 1 } moe_expert_fmt_t;
+
 typedef struct {
     int32_t T;            /* tokens */
     int32_t d;            /* hidden size */
@@ -86,6 +100,7 @@ typedef struct {
     int32_t has_bias;     /* 1: every Linear has a bias (the page's Expert); 0: no biases */
     int32_t dtype;        /* moe_dtype_t */
     int32_t gate_mode;    /* moe_gate_mode_t (0 = the report's softmax gate) */
+    int32_t routed_fmt;   /* moe_expert_fmt_t (0 = weights in dtype) */
 } moe_shape_t;
 
 /* One stack of experts (routed: E = n_experts; shared: E = n_shared), nn.Linear layout. */
@@ -96,6 +111,9 @@ typedef struct {
     const void* b3; /* [E, I] or NULL */
     const void* w2; /* [E, d, I] */
     const void* b2; /* [E, d] or NULL */
+    const float* s1; /* MOE_FMT_E4M3 routed experts: [E, I] scales of w1's rows; NULL otherwise */
+    const float* s3; /* MOE_FMT_E4M3: [E, I] scales of w3's rows; NULL otherwise */
+    const float* s2; /* MOE_FMT_E4M3: [E, d] scales of w2's rows; NULL otherwise */
 } moe_ffn_weights_t;
 
 /* Bytes of workspace every entry point needs for this shape (0 if the shape is invalid). */
@@ -202,7 +220,9 @@ moe_status_t moe_layer_forward(const moe_shape_t* shape, const void* x, const vo
  *   0 router (scores, softmax, top-k)      1 grouping (histogram, scan, scatter)
  *   2 tile tables of the grouped GEMMs     3 row gather of the routed tokens (bf16 only)
  *   4 GEMM1 + SwiGLU (routed and shared)   5 GEMM2: routed with gates, then (bf16) the
- *                                            shared experts' tiles in the same launch
+ *                                            shared experts' tiles in the same launch;
+ *     (with MOE_FMT_E4M3, stage 3 also quantises the gathered rows and stage 5 starts with
+ *      the quantisation of the hidden rows)
  *   6 combine (fp32 layers: shared GEMM2 and combine in one kernel)
  * n_events must be MOE_NUM_STAGES + 1; MOE_ERR_INVALID_ARG otherwise.
  */
@@ -212,6 +232,22 @@ moe_status_t moe_layer_forward_timed(const moe_shape_t* shape, const void* x, co
                                      void* out, int32_t* topk_idx_out, float* topk_gate_out,
                                      int32_t* counts_out, void* ws, size_t ws_bytes, moe_stream_t stream,
                                      void* const* stage_events, int32_t n_events);
+
+/*
+ * Per-row e4m3 quantisation of bf16 rows, the step that prepares the FP8 routed experts'
+ * inputs (MOE_FMT_E4M3 above), also usable on its own (e.g. for weights: one row = one output
+ * channel).  For p in [0, n_rows): r = row_of ? row_of[p] : p;
+ *   scale[p]  = max_j |src[r, j]| / 448 (IEEE fp32 division; 1 for an all-zero row)
+ *   dst[p, j] = e4m3 code of src[r, j] / scale[p] (IEEE fp32 division, round to nearest even,
+ *               saturating at +-448)
+ *   src: [src_rows, width] bf16; row_of: [n_rows] int32 or NULL (then n_rows <= src_rows);
+ *   dst: [n_rows, width] uint8 out; scale: [n_rows] fp32 out; width a multiple of 8.
+ * ws (>= 256 bytes, as for the other calls) only holds the error word: a row_of entry outside
+ * [0, src_rows) sets bit 4 and that row comes out as zeros with scale 1.
+ */
+moe_status_t moe_quantize_rows_e4m3(const void* src, const int32_t* row_of, int64_t n_rows, int32_t src_rows,
+                                    int32_t width, uint8_t* dst, float* scale, void* ws, size_t ws_bytes,
+                                    moe_stream_t stream);
 
 /*
  * moe_permute_no_alloc — the paper has no counterpart to this entry point; it exists for

@@ -47,7 +47,7 @@ def test_version_and_status_strings(lib):
 
 def _shape(**kw):
     base = dict(T=256, d=7168, n_experts=256, inter=2048, top_k=8, n_shared=1, inter_shared=2048, has_bias=1,
-                dtype=moe.MOE_BF16, gate_mode=0)
+                dtype=moe.MOE_BF16, gate_mode=0, routed_fmt=moe.FMT_NATIVE)
     base.update(kw)
     return moe.MoeShape(*[base[f] for f, _ in moe.MoeShape._fields_])
 
@@ -68,6 +68,13 @@ def test_workspace_bytes(lib):
                 dict(has_bias=2), dict(n_shared=1, inter_shared=0), dict(gate_mode=3), dict(gate_mode=-1)):
         assert moe.workspace_bytes(_shape(**bad)) == 0, bad
     assert moe.workspace_bytes(_shape(d=7170, dtype=moe.MOE_F32)) > 0
+    # e4m3 routed experts: h8 rows and the two per-row scale arrays on top (x8 reuses x_perm)
+    n8 = moe.workspace_bytes(_shape(routed_fmt=moe.FMT_E4M3))
+    assert S * I + 2 * 4 * S <= n8 - n <= S * I + 2 * 4 * S + 3 * 256
+    for bad in (dict(routed_fmt=2), dict(routed_fmt=-1)):
+        assert moe.workspace_bytes(_shape(**bad)) == 0, bad
+    for unsupported in (dict(dtype=moe.MOE_F32), dict(d=7176), dict(inter=2056)):
+        assert moe.workspace_bytes(_shape(routed_fmt=moe.FMT_E4M3, **unsupported)) == 0, unsupported
 
 
 def test_launch_count(lib):
@@ -76,6 +83,7 @@ def test_launch_count(lib):
     assert moe.layer_launches(_shape(T=16384, n_shared=0)) == 9
     assert moe.layer_launches(_shape(T=128, d=256, n_experts=16, inter=64, inter_shared=64, top_k=4,
                                      dtype=moe.MOE_F32)) == 8
+    assert moe.layer_launches(_shape(routed_fmt=moe.FMT_E4M3)) == 11      # + hidden-row quantisation
     assert moe.layer_launches(_shape(T=0)) == 0
     assert moe.layer_launches(_shape(top_k=0)) == -1
 
@@ -117,3 +125,25 @@ def test_argument_errors_return_before_any_launch(lib):
     assert lib.moe_layer_forward(S(sh_e), fake, fake, None, S(w), S(w), fake, None, None, None, fake, ne, None) == moe.MOE_OK
     assert lib.moe_ws_init(None, 0, None) == moe.MOE_ERR_WORKSPACE
     assert lib.moe_check_device_error(None, 0, None, None) == moe.MOE_ERR_WORKSPACE
+    # scales: required by e4m3 routed experts, refused elsewhere (native routed, shared)
+    sh8 = _shape(routed_fmt=moe.FMT_E4M3)
+    n8 = moe.workspace_bytes(sh8)
+    w8 = moe.MoeWeights(*([fake.value] * 9))
+    assert lib.moe_expert_ffn(S(sh8), fake, fake, fake, fake, S(w), fake, fake, n8, None) == moe.MOE_ERR_INVALID_ARG
+    assert lib.moe_expert_ffn(S(sh), fake, fake, fake, fake, S(w8), fake, fake, n, None) == moe.MOE_ERR_INVALID_ARG
+    assert lib.moe_layer_forward(S(sh8), fake, fake, None, S(w8), S(w8), fake, None, None, None, fake, n8, None) == \
+        moe.MOE_ERR_INVALID_ARG
+    assert lib.moe_layer_forward(S(sh8), fake, fake, None, S(w8), S(w), fake, None, None, None, fake, n8 - 1, None) == \
+        moe.MOE_ERR_WORKSPACE
+
+
+def test_quantize_rows_argument_errors(lib):
+    fake = ctypes.c_void_p(1 << 40)
+    q = lib.moe_quantize_rows_e4m3
+    assert q(fake, None, 10, 10, 12, fake, fake, fake, 4096, None) == moe.MOE_ERR_UNSUPPORTED   # width % 8
+    assert q(fake, None, 11, 10, 16, fake, fake, fake, 4096, None) == moe.MOE_ERR_INVALID_ARG   # n_rows > src_rows
+    assert q(fake, None, -1, 10, 16, fake, fake, fake, 4096, None) == moe.MOE_ERR_INVALID_ARG
+    assert q(fake, None, 10, 10, 0, fake, fake, fake, 4096, None) == moe.MOE_ERR_INVALID_ARG
+    assert q(fake, None, 10, 10, 16, fake, fake, None, 0, None) == moe.MOE_ERR_WORKSPACE
+    assert q(None, None, 10, 10, 16, fake, fake, fake, 4096, None) == moe.MOE_ERR_INVALID_ARG
+    assert q(fake, fake, 0, 10, 16, fake, fake, fake, 4096, None) == moe.MOE_OK                # no rows: no-op

@@ -58,3 +58,19 @@ def test_zero_rows_and_stack_round_trip():
         err = (back[k] - st[k].float()).abs().max() / st[k].float().abs().max()
         assert err.item() < 2.0 ** -4
     assert back["b1"] is st["b1"]
+
+
+def test_weight_codes_match_the_oracle_quantiser():
+    """The offline weight converter and the oracle's per-row quantiser (written separately from
+    the e4m3 definition) give the same codes and scales, bf16 weights included."""
+    import numpy as np
+
+    import oracle.moe_oracle as O
+    g = torch.Generator().manual_seed(3)
+    w = (torch.randn(40, 96, generator=g) * torch.exp2(torch.empty(40, 1).uniform_(-14, 6, generator=g)))
+    w[4] = 0.0
+    for src in (w, w.bfloat16()):
+        q, s = quant.quantize_rows(src)
+        q_ref, s_ref = O.quantize_rows_e4m3(src.double().numpy())
+        assert np.array_equal(s.numpy(), s_ref)
+        assert np.array_equal(O.e4m3_decode(q.numpy()), q_ref)
