@@ -2,7 +2,7 @@
 """Benchmark of the B200 DeepSeekMoE layer forward.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload prefill|decode|mid|small|tiny]
-                    [--impl ours|reference]
+                    [--impl ours|reference] [--gate-mode 0|1|2] [--routed-fmt bf16|e4m3]
 
 One step = one moe_layer_forward over one batch of synthetic tokens (router, grouping, row
 gather, GEMM1+SwiGLU, GEMM2+gate, shared GEMM2+combine), inputs resident in HBM.  The
@@ -14,6 +14,9 @@ between steps.
 Multi-GPU runs are replicas: every rank holds the same weights and processes its own batch
 (the layer is independent per token; there is no exchange), so the per-GPU work is fixed
 (weak scaling) and value = tokens of all ranks / the slowest rank's time.
+
+--routed-fmt e4m3 stores the routed experts' weights as e4m3 codes with per-channel scales
+(converted once before timing) and runs their GEMMs on the FP8 tensor-core path.
 
 --impl reference times the fp64 CPU oracle (the only reference that exists for this layer)
 on bounded samples of the same workload, on rank 0 only.
@@ -82,17 +85,36 @@ def aggregate_throughput(tokens_per_rank: int, n_ranks: int, max_ms_per_step: fl
     return tokens_per_rank * n_ranks / (max_ms_per_step / 1e3)
 
 
-def stage_work(cfg: W.LayerConfig, touched: int):
+def stage_work(cfg: W.LayerConfig, touched: int, e4m3: bool = False):
     """Algorithmic FLOPs and HBM bytes of each stage of one layer call.
 
     Bytes count each operand once at its storage size: weights of the experts that received
     at least one token (`touched`), activations read and written by the stage, routing
-    metadata.  FLOPs count 2 per multiply-add of the contractions only.
+    metadata.  FLOPs count 2 per multiply-add of the contractions only.  With e4m3 routed
+    experts their weights, the gathered rows and the quantised hidden rows are 1 byte each,
+    plus one fp32 scale per weight row and per activation row; the gemm2 stage includes the
+    hidden-row quantisation (bf16 h read, e4m3 h written).
     """
     T, d, E, I, k, Ks, Is = cfg.T, cfg.d, cfg.n_experts, cfg.inter, cfg.top_k, cfg.n_shared, cfg.inter_shared
     b = cfg.elem_bytes()
     S = T * k
     bias = 1 if cfg.has_bias else 0
+    if e4m3:
+        return {
+            "router": (2.0 * T * d * E, (T * d + E * d) * b + S * 8),
+            "permute": (0.0, S * 8 + S * 16),
+            "plan": (0.0, (E + 1) * 4),
+            "gather": (0.0, S * d * b + S * d + S * 8),
+            "gemm1_swiglu": (2.0 * S * d * 2 * I + 2.0 * Ks * T * d * 2 * Is,
+                             touched * (2 * I * d + 2 * I * 4 + 2 * I * bias * b) + S * d + S * 4
+                             + Ks * (2 * Is * d + 2 * Is * bias) * b + (T * d * b if Ks else 0)
+                             + (S * I + Ks * T * Is) * b),
+            "gemm2": (2.0 * S * I * d + 2.0 * Ks * T * Is * d,
+                      S * I * b + S * I + S * 4                                  # h quantisation
+                      + touched * (d * I + d * 4 + d * bias * b) + S * I + S * 4 + S * d * b + S * 4
+                      + Ks * (d * Is + d * bias) * b + Ks * T * Is * b + (T * d * 4 if Ks else 0)),
+            "combine": (0.0, S * d * b + (T * d * 4 if Ks else 0) + T * d * b + S * 4),
+        }
     w = {
         "router": (2.0 * T * d * E, (T * d + E * d) * b + S * 8),
         "permute": (0.0, S * 8 + S * 16),
@@ -113,12 +135,14 @@ def stage_work(cfg: W.LayerConfig, touched: int):
     return w
 
 
-def layer_bytes(cfg: W.LayerConfig, touched: int) -> float:
+def layer_bytes(cfg: W.LayerConfig, touched: int, e4m3: bool = False) -> float:
     """Algorithmic bytes of the whole layer: weights of touched experts, shared experts,
     centroids, x in and out once (intermediates excluded: the method need not keep them)."""
     b = cfg.elem_bytes()
     bias = 1 if cfg.has_bias else 0
-    return (touched * (3 * cfg.d * cfg.inter + (2 * cfg.inter + cfg.d) * bias) * b
+    routed = (3 * cfg.d * cfg.inter + (2 * cfg.inter + cfg.d) * 4 + (2 * cfg.inter + cfg.d) * bias * b) if e4m3 \
+        else (3 * cfg.d * cfg.inter + (2 * cfg.inter + cfg.d) * bias) * b
+    return (touched * routed
             + cfg.n_shared * (3 * cfg.d * cfg.inter_shared + (2 * cfg.inter_shared + cfg.d) * bias) * b
             + cfg.n_experts * cfg.d * b + 2 * cfg.T * cfg.d * b)
 
@@ -128,6 +152,7 @@ def src_hash(path: str) -> str:
 
 
 def ncu_traffic(workload: str, stage: str):
+    # workload keys: the config name, with "+e4m3" for FP8 routed experts
     """Per-launch DRAM bytes of a kernel from the committed ncu summary, if the kernel's
     source has not changed since the counters were taken; else None."""
     p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
@@ -222,13 +247,13 @@ class HostExperts:
         return {k: (None if v is None else v.float().numpy().astype(np.float64)) for k, v in h.items()}
 
 
-def oracle_sample(O, L, cfg, host_routed, host_shared, tokens, gate_mode=0, router_bias=None):
+def oracle_sample(O, L, cfg, host_routed, host_shared, tokens, gate_mode=0, router_bias=None, e4m3=False):
     x = L["x"][tokens].float().cpu().numpy().astype(np.float64)
     c = L["centroids"].float().cpu().numpy().astype(np.float64)
     b = None if router_bias is None else router_bias.double().cpu().numpy()
     t0 = time.perf_counter()
     O.layer(x, c, host_routed, cfg.n_experts, cfg.top_k, host_shared, cfg.n_shared, gate_mode=gate_mode,
-            router_bias=b)
+            router_bias=b, routed_e4m3=e4m3)
     return time.perf_counter() - t0
 
 
@@ -243,7 +268,7 @@ def blas_threads():
     return os.cpu_count() or 1
 
 
-def cpu_baseline(cfg, L, idx_gpu, n_tokens=16, gate_mode=0, router_bias=None):
+def cpu_baseline(cfg, L, idx_gpu, n_tokens=16, gate_mode=0, router_bias=None, e4m3=False):
     """The oracle, as it stands, on the first n_tokens tokens of this step's batch."""
     import oracle.moe_oracle as O
     tokens = np.arange(min(n_tokens, cfg.T))
@@ -252,10 +277,11 @@ def cpu_baseline(cfg, L, idx_gpu, n_tokens=16, gate_mode=0, router_bias=None):
     hr.prefetch(np.unique(idx_gpu[tokens]))
     if hs is not None:
         hs.prefetch(range(cfg.n_shared))
-    dt = oracle_sample(O, L, cfg, hr, hs, tokens, gate_mode, router_bias)
+    dt = oracle_sample(O, L, cfg, hr, hs, tokens, gate_mode, router_bias, e4m3)
+    fmt = "e4m3 routed codes + scales and bf16 shared" if e4m3 else "bf16"
     return {"value": len(tokens) / dt, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
             "sample": f"fp64 NumPy oracle on the first {len(tokens)} tokens of the {cfg.name} batch "
-                      f"(all experts they route to; weights staged in host memory as bf16, converted by the oracle)",
+                      f"(all experts they route to; weights staged in host memory as {fmt}, converted by the oracle)",
             "seconds": dt}
 
 
@@ -266,11 +292,15 @@ def run_reference(args, cfg, rank, world):
     import oracle.moe_oracle as O
     dev = "cuda" if torch.cuda.is_available() else "cpu"
     L = W.make_layer(cfg, dev, seed=0)
+    e4m3 = args.routed_fmt == "e4m3"
+    if e4m3:
+        from fine_grained_mixture_route_b200 import quant
+        L["routed"] = quant.quantize_stack(L["routed"])
     hr = HostExperts(L["routed"])
     hs = HostExperts(L["shared"]) if L["shared"] is not None else None
     budget_s = 150.0
     n = min(8, cfg.T)
-    t_first = oracle_sample(O, L, cfg, hr, hs, np.arange(n))           # sizing run (also warms the cache)
+    t_first = oracle_sample(O, L, cfg, hr, hs, np.arange(n), e4m3=e4m3)   # sizing run (also warms the cache)
     per_tok = t_first / n
     n = int(max(1, min(64, cfg.T, budget_s / max(1, args.steps + args.warmup) / max(per_tok, 1e-6))))
     pos = 0
@@ -278,7 +308,7 @@ def run_reference(args, cfg, rank, world):
     for i in range(args.warmup + args.steps):
         toks = (np.arange(n) + pos) % cfg.T
         pos += n
-        dt = oracle_sample(O, L, cfg, hr, hs, toks)
+        dt = oracle_sample(O, L, cfg, hr, hs, toks, e4m3=e4m3)
         if i >= args.warmup:
             times.append(dt)
     total = sum(times)
@@ -288,7 +318,8 @@ def run_reference(args, cfg, rank, world):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": cfg.name, "tokens_per_step": n, "T": cfg.T, "d": cfg.d,
                        "n_experts": cfg.n_experts, "inter": cfg.inter, "top_k": cfg.top_k,
-                       "n_shared": cfg.n_shared, "parallelism": "replicas" if world > 1 else "single"},
+                       "n_shared": cfg.n_shared, "routed_fmt": args.routed_fmt,
+                       "parallelism": "replicas" if world > 1 else "single"},
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
                              "sample": f"{n} consecutive tokens of the {cfg.name} batch per step"},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -306,6 +337,11 @@ def run_ours(args, cfg, rank, world, local_rank):
     L = W.make_layer(cfg, dev, seed=0)
     if rank > 0:
         L["x"] = W.make_x(cfg, dev, seed=1000 + rank)
+    e4m3 = args.routed_fmt == "e4m3"
+    if e4m3:   # one-off weight conversion before anything is timed
+        from fine_grained_mixture_route_b200 import quant
+        L["routed"] = quant.quantize_stack(L["routed"])
+        torch.cuda.empty_cache()
     x, C, R, Sh = L["x"], L["centroids"], L["routed"], L["shared"]
     shape = moe.shape_of(x, C, R, cfg.top_k, Sh, gate_mode=args.gate_mode)
     rbias = None
@@ -322,7 +358,7 @@ def run_ours(args, cfg, rank, world, local_rank):
         moe.layer_forward(shape, x, C, R, Sh, ws, out=out, idx=idx, gate=gate, counts=counts, router_bias=rbias)
     moe.check_device_error(ws)
     touched = int((counts > 0).sum().item())
-    work = stage_work(cfg, touched)
+    work = stage_work(cfg, touched, e4m3)
 
     # ---- device-timed region: K steps, per-stage events on the launching stream
     evs = [moe.stage_events(stream) for _ in range(args.steps)]
@@ -371,37 +407,48 @@ def run_ours(args, cfg, rank, world, local_rank):
     # dominant stage and its roofline
     dom = max(stage_ms, key=stage_ms.get)
     flops, nbytes = work[dom]
-    ridge = peaks["bf16_tflops_sustained"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    tc_peak = peaks["bf16_tflops_sustained"]
+    if e4m3 and dom in ("gemm1_swiglu", "gemm2"):
+        # routed FLOPs at the e4m3 rate (2x bf16: 4.5 vs 2.25 PFLOP/s nominal dense), shared at bf16
+        Ks, Is, T, d, I = cfg.n_shared, cfg.inter_shared, cfg.T, cfg.d, cfg.inter
+        f_sh = 2.0 * Ks * T * d * 2 * Is if dom == "gemm1_swiglu" else 2.0 * Ks * T * Is * d
+        tc_peak = flops / ((flops - f_sh) / (2 * tc_peak) + f_sh / tc_peak)
+    ridge = tc_peak * 1e12 / (peaks["hbm_gbs"] * 1e9)
     if cfg.dtype == torch.float32:
         bound = "hbm" if nbytes > 0 and flops / nbytes < 10 else "alu"
     else:
         bound = "tensor" if nbytes == 0 or flops / nbytes > ridge else "hbm"
     t = stage_ms[dom] / 1e3
     if bound == "tensor":
-        achieved, peak, unit = flops / t / 1e12, peaks["bf16_tflops_sustained"], "TFLOP/s"
+        achieved, peak, unit = flops / t / 1e12, tc_peak, "TFLOP/s"
     elif bound == "hbm":
         achieved, peak, unit = nbytes / t / 1e9, peaks["hbm_gbs"], "GB/s"
     else:
         # fp32 CUDA-core FMA peak: 148 SMs x 128 lanes x 2 FLOP x max SM clock
         achieved, peak, unit = flops / t / 1e12, 148 * 128 * 2 * 1.965e9 / 1e12, "TFLOP/s"
+    tensor_src = ("bf16 sustained; routed FLOPs at 2x (e4m3/bf16 nominal dense ratio), shared at 1x"
+                  if e4m3 and peak != peaks["bf16_tflops_sustained"] else "bf16 sustained")
     roofline = {"bound": bound, "kernel": dom, "achieved": achieved, "peak": peak, "unit": unit,
-                "frac": achieved / peak, "peak_source": f"{peak_src} ({'bf16 sustained' if bound == 'tensor' else 'HBM copy' if bound == 'hbm' else 'fp32 FMA nominal'})",
-                "traffic": ncu_traffic(cfg.name, dom),
+                "frac": achieved / peak,
+                "peak_source": f"{peak_src} ({tensor_src if bound == 'tensor' else 'HBM copy' if bound == 'hbm' else 'fp32 FMA nominal'})",
+                "traffic": ncu_traffic(cfg.name + ("+e4m3" if e4m3 else ""), dom),
                 "algorithmic_per_launch": flops if bound != "hbm" else nbytes}
     if bound == "tensor":
-        roofline["frac_of_burst"] = achieved / peaks["bf16_tflops"]
+        roofline["frac_of_burst"] = achieved / (peaks["bf16_tflops"] * tc_peak / peaks["bf16_tflops_sustained"])
 
     step_s = ms / 1e3
     total_flops = cfg.flops()
-    lbytes = layer_bytes(cfg, touched)
+    lbytes = layer_bytes(cfg, touched, e4m3)
     value = aggregate_throughput(cfg.T, world, ms)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16" if cfg.dtype == torch.bfloat16 else "f32", "data": "synthetic",
+        "vs_baseline": None, "dtype": ("e4m3/bf16" if e4m3 else "bf16") if cfg.dtype == torch.bfloat16 else "f32",
+        "data": "synthetic",
         "config": {"workload": cfg.name, "T": cfg.T, "d": cfg.d, "n_experts": cfg.n_experts, "inter": cfg.inter,
                    "top_k": cfg.top_k, "n_shared": cfg.n_shared, "inter_shared": cfg.inter_shared,
                    "bias": cfg.has_bias, "routing": cfg.centroid_init, "gate_mode": args.gate_mode,
+                   "routed_fmt": args.routed_fmt,
                    "parallelism": f"replicas{world}" if world > 1 else "single",
                    "l2": "inputs larger than L2 (weights and activations), no flush",
                    "tokens_per_gpu": cfg.T},
@@ -416,7 +463,8 @@ def run_ours(args, cfg, rank, world, local_rank):
     }
     del evs
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(cfg, L, idx.cpu().numpy(), gate_mode=args.gate_mode, router_bias=rbias)
+        line["cpu_baseline"] = cpu_baseline(cfg, L, idx.cpu().numpy(), gate_mode=args.gate_mode, router_bias=rbias,
+                                            e4m3=e4m3)
     if rank == 0:
         print(json.dumps(line), flush=True)
 
@@ -431,6 +479,9 @@ def main(argv=None):
     ap.add_argument("--gate-mode", type=int, default=0, choices=[0, 1, 2],
                     help="router gate: 0 softmax over all experts (default), 1 softmax over the top-k logits of a "
                          "biased router, 2 sigmoid with a selection bias")
+    ap.add_argument("--routed-fmt", default="bf16", choices=["bf16", "e4m3"],
+                    help="storage of the routed experts' weights: bf16, or e4m3 codes with per-channel scales "
+                         "(FP8 tensor-core path; activations quantised per row)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args(argv)
@@ -440,6 +491,8 @@ def main(argv=None):
     if world != args.gpus and world > 1:
         ap.error(f"--gpus {args.gpus} but WORLD_SIZE={world}")
     cfg = W.CONFIGS[args.workload]
+    if args.routed_fmt == "e4m3" and cfg.dtype != torch.bfloat16:
+        ap.error("--routed-fmt e4m3 needs a bf16 workload")
     if args.impl == "reference":
         run_reference(args, cfg, rank, world)
         return

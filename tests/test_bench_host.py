@@ -54,6 +54,15 @@ def test_stage_work_sums_to_layer_flops():
     # weight bytes of the whole layer when every expert is touched: 256 routed + 1 shared
     per_expert = (3 * 7168 * 2048 + 2 * 2048 + 7168) * 2
     assert abs(bench.layer_bytes(dec, 256) - (257 * per_expert + 256 * 7168 * 2 + 2 * 256 * 7168 * 2)) < 1
+    # e4m3 routed experts: same FLOPs; routed weights at 1 byte plus one fp32 scale per row
+    for name, cfg in W.CONFIGS.items():
+        if cfg.dtype == torch.bfloat16:
+            w8 = bench.stage_work(cfg, cfg.n_experts, e4m3=True)
+            assert abs(sum(f for f, _ in w8.values()) - cfg.flops()) < 1e-6 * cfg.flops(), name
+            assert w8["gemm1_swiglu"][1] < bench.stage_work(cfg, cfg.n_experts)["gemm1_swiglu"][1]
+    routed8 = 3 * 7168 * 2048 + (2 * 2048 + 7168) * 4 + (2 * 2048 + 7168) * 2
+    assert abs(bench.layer_bytes(dec, 256, e4m3=True)
+               - (256 * routed8 + per_expert + 256 * 7168 * 2 + 2 * 256 * 7168 * 2)) < 1
 
 
 def test_reference_arm_line():
@@ -70,3 +79,5 @@ def test_reference_arm_line():
 def test_warmup_must_be_three():
     with pytest.raises(SystemExit):
         bench.main(["--warmup", "2"])
+    with pytest.raises(SystemExit):                     # e4m3 routed experts need a bf16 layer
+        bench.main(["--workload", "tiny", "--routed-fmt", "e4m3"])
