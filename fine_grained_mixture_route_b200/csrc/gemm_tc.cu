@@ -282,6 +282,18 @@ __device__ __forceinline__ void mbar_arrive_rank0(uint32_t bar) {
     asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(remote) : "memory");
 }
 // Instruction descriptor for the pair MMA: M = 256 (128 rows per CTA).
+// kind::f8f6f4 e4m3 MMA across a CTA pair (M = 256)
+__device__ __forceinline__ void mma_e4m3_pair(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a), "l"(b), "r"(idesc), "r"(acc)
+        : "memory");
+}
+__host__ __device__ constexpr uint32_t idesc_e4m3_pair(int n) {
+    return (1u << 4) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(256 >> 4) << 24);
+}
 __host__ __device__ constexpr uint32_t idesc_bf16_pair(int n) {
     return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(256 >> 4) << 24);
 }
@@ -629,12 +641,12 @@ __device__ __forceinline__ void epilogue_router_partial(const Params& p, const T
 // barriers valid before any peer copy lands, and one before teardown keeps every shared
 // memory and TMEM range alive until the leader's last MMA has finished.
 //
-// Q8 (single CTAs, GEMM1 / GEMM2R): routed tiles read e4m3 operands, K blocks of 128 (the same
-// 128-byte swizzle rows as 64 bf16), and run kind::f8f6f4 MMAs; shared-expert tiles of the
-// same launch stay bf16.
+// Q8 (GEMM1 / GEMM2R, single CTAs or pairs): routed tiles read e4m3 operands, K blocks of 128
+// (the same 128-byte swizzle rows as 64 bf16), and run kind::f8f6f4 MMAs; shared-expert tiles
+// of the same launch stay bf16.
 template <int MODE, int KMAX, bool PAIR_, bool Q8 = false>
 __global__ void __launch_bounds__(THREADS, 1) moe_tc_kernel(const __grid_constant__ Params p) {
-    static_assert(!Q8 || (!PAIR_ && (MODE == GEMM1 || MODE == GEMM2R)), "e4m3 tiles: single-CTA expert GEMMs");
+    static_assert(!Q8 || MODE == GEMM1 || MODE == GEMM2R, "e4m3 tiles: routed expert GEMMs only");
     using C = Cfg<MODE, PAIR_>;
     constexpr bool PAIR = C::PAIR;
     constexpr int STAGES = C::STAGES;
@@ -721,11 +733,13 @@ __global__ void __launch_bounds__(THREADS, 1) moe_tc_kernel(const __grid_constan
                             // follower: the same rows of W3 (columns 128-255)
                             const bool shared = x.g >= p.E;
                             const int e = shared ? x.g - p.E : x.g;
-                            tma_load_2d_pair(a_dst, &p.tmA[shared ? 1 : 0], fb, kb * BK, x.row0 + x.m0 + arow);
-                            tma_load_3d_pair(b_dst, &p.tmB[(shared ? 2 : 0) + (int)rank], fb, kb * BK, x.n0, e);
+                            const int kc = kb * ((Q8 && !shared) ? 2 * BK : BK);   // K element offset
+                            tma_load_2d_pair(a_dst, &p.tmA[shared ? 1 : 0], fb, kc, x.row0 + x.m0 + arow);
+                            tma_load_3d_pair(b_dst, &p.tmB[(shared ? 2 : 0) + (int)rank], fb, kc, x.n0, e);
                         } else if (MODE == GEMM2R && x.g >= 0) {
-                            tma_load_2d_pair(a_dst, &p.tmA[0], fb, kb * BK, x.row0 + x.m0 + arow);
-                            tma_load_3d_pair(b_dst, &p.tmB[0], fb, kb * BK, x.n0 + arow, x.g);
+                            const int kc = kb * (Q8 ? 2 * BK : BK);
+                            tma_load_2d_pair(a_dst, &p.tmA[0], fb, kc, x.row0 + x.m0 + arow);
+                            tma_load_3d_pair(b_dst, &p.tmB[0], fb, kc, x.n0 + arow, x.g);
                         } else if (MODE == GEMM2R) {
                             const int kbs = ceil_div(p.Is, BK);
                             const int s = kb / kbs, kk = kb % kbs;
@@ -788,7 +802,7 @@ __global__ void __launch_bounds__(THREADS, 1) moe_tc_kernel(const __grid_constan
             for (int t = cta_slot; ok && t < ntiles; t += cta_slots) {
                 const Tile x = decode<MODE, PAIR>(p, t);
                 const bool q8tile = Q8 && (MODE == GEMM1 ? x.g < p.E : x.g >= 0);
-                const uint32_t idesc_t = q8tile ? idesc_e4m3(p.n_mma) : idesc;
+                const uint32_t idesc_t = q8tile ? (PAIR ? idesc_e4m3_pair(p.n_mma) : idesc_e4m3(p.n_mma)) : idesc;
                 if (!mbar_wait(tempty_bar(acc), acc_phase ^ 1u, abort_flag, p.err)) break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + (uint32_t)(acc * ACC_COLS);
@@ -800,7 +814,8 @@ __global__ void __launch_bounds__(THREADS, 1) moe_tc_kernel(const __grid_constan
                     for (int k = 0; k < BK / 16; ++k) {
                         const uint64_t ad = sw128_desc(a_addr + k * 32), bd = sw128_desc(b_addr + k * 32);
                         const uint32_t accum = (kb > 0 || k > 0) ? 1u : 0u;
-                        if (PAIR) mma_bf16_pair(d_tmem, ad, bd, idesc, accum);
+                        if (PAIR && q8tile) mma_e4m3_pair(d_tmem, ad, bd, idesc_t, accum);
+                        else if (PAIR) mma_bf16_pair(d_tmem, ad, bd, idesc_t, accum);
                         else if (q8tile) mma_e4m3(d_tmem, ad, bd, idesc_t, accum);
                         else mma_bf16(d_tmem, ad, bd, idesc_t, accum);
                     }
@@ -977,9 +992,12 @@ int num_sms() {
 }
 
 // Whether the expert GEMMs run on CTA pairs.  Measured on one B200 with both variants
-// interleaved (prefill 14.3 vs 15.0 ms per layer, decode 3.9 vs 5.8 ms, mid 0.73 vs 0.77 ms),
-// single CTAs are faster for every layer shape here, so pairs are off unless a build sets
-// MOE_PAIR_POLICY=1.
+// interleaved, single CTAs are faster or equal for every layer shape here: bf16 prefill 14.3 vs
+// 15.0 ms per layer, decode 3.9 vs 5.8 ms, mid 0.73 vs 0.77 ms; e4m3 routed experts, prefill
+// 10.2 vs 10.3 ms (GEMM1 5.07 vs 5.15 ms, clock-normalised), although a pair reads 8 KB of
+// operands per SM for each 256 x 256 x 32 e4m3 step where a single CTA reads 12 KB per
+// 128 x 256 x 32.  Pairs (bf16 and e4m3 tiles, both parity-tested) stay available through a
+// build with MOE_PAIR_POLICY=1.
 bool gemm_pairs(const Dims& D) {
     (void)D;
 #if defined(MOE_PAIR_POLICY) && MOE_PAIR_POLICY > 0
@@ -1131,7 +1149,8 @@ cudaError_t launch_tc_gemm1_q8(const Dims& D, const void* x, const void* x8_perm
         ok &= make_map(&p.tmB[3], Sh.w3, D.d, D.Is, D.Ks, BK, 128, true);
     }
     if (!ok) return cudaErrorInvalidValue;
-    return launch<GEMM1, 8, false, true>(p, num_sms(), stream);
+    return tc::pairs_for(D) ? launch<GEMM1, 8, true, true>(p, num_sms(), stream)
+                            : launch<GEMM1, 8, false, true>(p, num_sms(), stream);
 }
 
 // e4m3 routed GEMM2 over h8 (e4m3 rows, scale per row in hs) and the e4m3 W2 codes; with Sh the
@@ -1152,17 +1171,19 @@ cudaError_t launch_tc_gemm2_routed_q8(const Dims& D, const int32_t* offsets, con
     p.sorted_gate = sorted_gate;
     p.b2 = (const __nv_bfloat16*)R.b2;
     p.y = (__nv_bfloat16*)y_sorted;
+    const bool pairs = tc::pairs_for(D);
     bool ok = make_map_u8(&p.tmA[0], h8, D.I, (uint64_t)D.slots(), 1, 2 * BK, BM, false);
-    ok &= make_map_u8(&p.tmB[0], R.w2, D.I, D.d, D.E, 2 * BK, 256, true);
+    ok &= make_map_u8(&p.tmB[0], R.w2, D.I, D.d, D.E, 2 * BK, pairs ? 128 : 256, true);
     if (Sh && D.Ks > 0 && sout) {
         p.fold_shared = 1;
         p.sb2 = (const __nv_bfloat16*)Sh->b2;
         p.sout = sout;
         ok &= make_map(&p.tmA[1], h_s, D.Is, D.T, D.Ks, BK, BM, true);
-        ok &= make_map(&p.tmB[1], Sh->w2, D.Is, D.d, D.Ks, BK, 256, true);
+        ok &= make_map(&p.tmB[1], Sh->w2, D.Is, D.d, D.Ks, BK, pairs ? 128 : 256, true);
     }
     if (!ok) return cudaErrorInvalidValue;
-    return launch<GEMM2R, 8, false, true>(p, num_sms(), stream);
+    return pairs ? launch<GEMM2R, 8, true, true>(p, num_sms(), stream)
+                 : launch<GEMM2R, 8, false, true>(p, num_sms(), stream);
 }
 
 }  // namespace moe

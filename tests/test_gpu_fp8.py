@@ -128,6 +128,12 @@ FP8_EDGE = [
     ("odd_dims", "small", dict(T=131, d=144, inter=48, inter_shared=24, n_experts=48, top_k=5)),
     ("all_experts", "small", dict(T=200, n_experts=16, top_k=16, inter=64, inter_shared=64)),
     ("zipf_empty_experts", "prefill", dict(T=1000, d=512, inter=128, inter_shared=128, n_experts=64)),
+    # >= 256 rows per expert on average, several M-tiles per expert (a MOE_PAIR_POLICY=1 build runs
+    # these on CTA pairs; they passed there too)
+    ("many_rows_odd_dims", "small", dict(T=1000, d=144, inter=48, inter_shared=40, n_experts=16, top_k=5)),
+    ("many_rows_no_shared", "small", dict(T=2048, n_shared=0, n_experts=32, top_k=4)),
+    ("many_rows_zipf_two_shared", "prefill", dict(T=3000, d=512, inter=256, n_shared=2, inter_shared=136,
+                                                  n_experts=32, top_k=6)),
 ]
 
 
