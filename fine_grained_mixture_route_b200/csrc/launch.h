@@ -54,6 +54,12 @@ cudaError_t launch_gather(const Dims& D, const void* x, const int32_t* sorted_to
 // division in IEEE fp32.  width % 8 == 0.
 cudaError_t launch_quant_rows(const void* src, const int32_t* row_of, long long n_rows, int src_rows, int width,
                               uint8_t* dst, float* scale, uint32_t* err, cudaStream_t stream);
+// dst[p, :] = src[row_of[p], :] for byte rows of row_bytes (a multiple of 16), and dscale[p] =
+// sscale[row_of[p]] when dscale is given; an index outside [0, src_rows) sets bit 4 and gives a
+// zero row with scale 1.
+cudaError_t launch_gather_code_rows(const uint8_t* src, const float* sscale, const int32_t* row_of, long long n_rows,
+                                    int src_rows, int row_bytes, uint8_t* dst, float* dscale, uint32_t* err,
+                                    cudaStream_t stream);
 
 // out[t, :] = base[t, :] + sum_j y_sorted[slot_of[t*k + j], :] in fp32, rounded once; base is
 // the shared experts' fp32 output [T, d], or NULL when there are none.

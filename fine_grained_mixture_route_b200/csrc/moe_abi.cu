@@ -16,6 +16,7 @@ size_t al(size_t x) { return (x + 255) & ~(size_t)255; }
 struct Layout {
     size_t err, hist, rpart, sout, ts1, ts2, idx, gate, counts, offsets, stok, sgate, slot_of, xperm, hr, hs, y;
     size_t xs, h8, hsc;    // e4m3 routed experts: row scales of x8 (in xperm), h8 rows and their scales
+    size_t x8t, xst;       // e4m3: x quantised once per token, and its scales
     size_t total;
 };
 
@@ -45,6 +46,8 @@ Layout layout(const Dims& D) {
     L.xs = o; o += D.q8 ? al(S * 4) : 0;
     L.h8 = o; o += D.q8 ? al(S * D.I) : 0;
     L.hsc = o; o += D.q8 ? al(S * 4) : 0;
+    L.x8t = o; o += D.q8 ? al((size_t)D.T * D.d) : 0;
+    L.xst = o; o += D.q8 ? al((size_t)D.T * 4) : 0;
     L.total = o;
     return L;
 }
@@ -122,6 +125,18 @@ FfnWeights to_ffn(const moe_ffn_weights_t* w) {
     return f;
 }
 
+// e4m3 routed experts: x quantised once per token, then its code rows (and scales) gathered
+// into expert order for the GEMM1 A operand.
+moe_status_t quant_gather_x(const Dims& D, const Layout& L, void* ws, const void* x, const int32_t* stok,
+                            uint32_t* err, cudaStream_t st) {
+    uint8_t* x8t = at<uint8_t>(ws, L.x8t);
+    float* xst = at<float>(ws, L.xst);
+    MOE_CUDA(launch_quant_rows(x, nullptr, D.T, D.T, D.d, x8t, xst, err, st));
+    MOE_CUDA(launch_gather_code_rows(x8t, xst, stok, D.slots(), D.T, D.d, at<uint8_t>(ws, L.xperm), at<float>(ws, L.xs),
+                                     err, st));
+    return MOE_OK;
+}
+
 moe_status_t do_route(const Dims& D, const void* x, const void* c, const float* bias, int32_t* idx, float* gate,
                       float* partial, uint32_t* err, cudaStream_t st) {
     if (D.T == 0) return MOE_OK;
@@ -141,7 +156,7 @@ moe_status_t do_expert_ffn(const Dims& D, const Layout& L, void* ws, const void*
     if (D.q8) {
         uint8_t* x8 = at<uint8_t>(ws, L.xperm);
         float* xs = at<float>(ws, L.xs);
-        MOE_CUDA(launch_quant_rows(x, stok, D.slots(), D.T, D.d, x8, xs, err, st));
+        MOE_TRY(quant_gather_x(D, L, ws, x, stok, err, st));
         FfnWeights none = {nullptr, nullptr, nullptr, nullptr, nullptr, nullptr};
         MOE_CUDA(launch_tc_gemm1_q8(D, x, x8, xs, offsets, ts1, R, none, at<void>(ws, L.hr), nullptr, D.E, err, st));
         uint8_t* h8 = at<uint8_t>(ws, L.h8);
@@ -199,7 +214,7 @@ MOE_EXPORT int32_t moe_layer_launches(const moe_shape_t* shape) {
     n += 1;                                                         // tile tables
     if (D.bf16) n += 1;                                             // row gather (+ e4m3 quantisation)
     n += 3;                                   // GEMM1, GEMM2 (routed + shared tiles), combine
-    if (D.q8) n += 1;                                               // hidden-row quantisation
+    if (D.q8) n += 2;                           // per-token x quantisation, hidden-row quantisation
     return n;
 }
 
@@ -378,7 +393,7 @@ moe_status_t layer_forward_impl(const moe_shape_t* shape, const void* x, const v
     if (D.q8) {
         uint8_t* x8 = at<uint8_t>(ws, L.xperm);
         float* xs = at<float>(ws, L.xs);
-        MOE_CUDA(launch_quant_rows(x, stok, D.slots(), D.T, D.d, x8, xs, err, st));
+        MOE_TRY(quant_gather_x(D, L, ws, x, stok, err, st));
         if (!mark(4)) return MOE_ERR_CUDA;
         MOE_CUDA(launch_tc_gemm1_q8(D, x, x8, xs, offsets, ts1, R, Sh, hr, hs, D.E + D.Ks, err, st));
         if (!mark(5)) return MOE_ERR_CUDA;

@@ -14,9 +14,6 @@
 namespace moe {
 namespace {
 
-constexpr int QT = 256;    // threads per row
-constexpr int QREG = 4;    // 16-byte chunks per thread kept in registers between the passes
-
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
@@ -39,46 +36,117 @@ __device__ __forceinline__ uint2 chunk_quant(const uint4& v, float sc) {
     return make_uint2(pk[0] | (pk[1] << 16), pk[2] | (pk[3] << 16));
 }
 
-__global__ void __launch_bounds__(QT) quant_rows_kernel(const uint4* __restrict__ src,
-                                                        const int32_t* __restrict__ row_of, long long n_rows,
-                                                        int src_rows, int nv, uint2* __restrict__ dst,
-                                                        float* __restrict__ scale, uint32_t* err) {
-    __shared__ float red[QT / 32];
-    const int tid = threadIdx.x;
-    for (long long p = blockIdx.x; p < n_rows; p += gridDim.x) {
+// One warp per row, the whole row in registers (CPL 16-byte chunks per lane): loads of a row
+// are all issued before the reduction, and no block barrier sits between rows.
+template <int CPL>
+__global__ void __launch_bounds__(256) quant_rows_warp_kernel(const uint4* __restrict__ src,
+                                                              const int32_t* __restrict__ row_of, long long n_rows,
+                                                              int src_rows, int nv, uint2* __restrict__ dst,
+                                                              float* __restrict__ scale, uint32_t* err) {
+    const int lane = threadIdx.x & 31;
+    const long long warps = (long long)gridDim.x * (blockDim.x >> 5);
+    for (long long p = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); p < n_rows; p += warps) {
         int r = row_of ? row_of[p] : (int)p;
         const bool ok = r >= 0 && r < src_rows;
         if (!ok) {
-            if (tid == 0) flag_error(err, ERR_INDEX_RANGE);
+            if (lane == 0) flag_error(err, ERR_INDEX_RANGE);
             r = 0;
         }
         const uint4* s = src + (size_t)r * nv;
-        uint4 keep[QREG];
+        uint4 keep[CPL];
         float m = 0.f;
 #pragma unroll
-        for (int c = 0; c < QREG; ++c) {
-            const int i = tid + c * QT;
+        for (int c = 0; c < CPL; ++c) {
+            const int i = lane + c * 32;
             keep[c] = (ok && i < nv) ? __ldg(s + i) : make_uint4(0, 0, 0, 0);
-            m = chunk_amax(keep[c], m);
         }
-        for (int i = tid + QREG * QT; ok && i < nv; i += QT) m = chunk_amax(__ldg(s + i), m);
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) m = chunk_amax(keep[c], m);
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-        __syncthreads();                       // red[] of the previous row has been read
-        if ((tid & 31) == 0) red[tid >> 5] = m;
-        __syncthreads();
-        float amax = red[0];
-#pragma unroll
-        for (int w = 1; w < QT / 32; ++w) amax = fmaxf(amax, red[w]);
-        const float sc = amax > 0.f ? __fdiv_rn(amax, 448.f) : 1.f;
-        if (tid == 0) scale[p] = sc;
+        const float sc = m > 0.f ? __fdiv_rn(m, 448.f) : 1.f;
+        if (lane == 0) scale[p] = sc;
         uint2* d = dst + (size_t)p * nv;
 #pragma unroll
-        for (int c = 0; c < QREG; ++c) {
-            const int i = tid + c * QT;
+        for (int c = 0; c < CPL; ++c) {
+            const int i = lane + c * 32;
             if (i < nv) d[i] = chunk_quant(keep[c], sc);
         }
-        for (int i = tid + QREG * QT; i < nv; i += QT) d[i] = ok ? chunk_quant(__ldg(s + i), sc) : make_uint2(0, 0);
+    }
+}
+
+// One warp per row for rows wider than the register-resident kernels take: the row is read
+// twice, in batches of 8 chunks per lane (the second pass finds it in L1 / L2).
+__global__ void __launch_bounds__(256) quant_rows_warp2_kernel(const uint4* __restrict__ src,
+                                                               const int32_t* __restrict__ row_of, long long n_rows,
+                                                               int src_rows, int nv, uint2* __restrict__ dst,
+                                                               float* __restrict__ scale, uint32_t* err) {
+    constexpr int B = 8;
+    const int lane = threadIdx.x & 31;
+    const long long warps = (long long)gridDim.x * (blockDim.x >> 5);
+    for (long long p = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); p < n_rows; p += warps) {
+        int r = row_of ? row_of[p] : (int)p;
+        const bool ok = r >= 0 && r < src_rows;
+        if (!ok) {
+            if (lane == 0) flag_error(err, ERR_INDEX_RANGE);
+            r = 0;
+        }
+        const uint4* s = src + (size_t)r * nv;
+        float m = 0.f;
+        for (int base = 0; ok && base < nv; base += 32 * B) {
+            uint4 v[B];
+#pragma unroll
+            for (int c = 0; c < B; ++c) {
+                const int i = base + lane + c * 32;
+                v[c] = i < nv ? __ldg(s + i) : make_uint4(0, 0, 0, 0);
+            }
+#pragma unroll
+            for (int c = 0; c < B; ++c) m = chunk_amax(v[c], m);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        const float sc = m > 0.f ? __fdiv_rn(m, 448.f) : 1.f;
+        if (lane == 0) scale[p] = sc;
+        uint2* d = dst + (size_t)p * nv;
+        for (int base = 0; base < nv; base += 32 * B) {
+            uint4 v[B];
+#pragma unroll
+            for (int c = 0; c < B; ++c) {
+                const int i = base + lane + c * 32;
+                v[c] = (ok && i < nv) ? __ldg(s + i) : make_uint4(0, 0, 0, 0);
+            }
+#pragma unroll
+            for (int c = 0; c < B; ++c) {
+                const int i = base + lane + c * 32;
+                if (i < nv) d[i] = chunk_quant(v[c], sc);
+            }
+        }
+    }
+}
+
+template <int CPL>
+cudaError_t launch_warp(const void* src, const int32_t* row_of, long long n_rows, int src_rows, int nv, uint8_t* dst,
+                        float* scale, uint32_t* err, cudaStream_t stream) {
+    const long long cap = (long long)num_sms() * 8;                 // 8 blocks of 8 warps per SM at most
+    const long long need = (n_rows + 7) / 8;
+    quant_rows_warp_kernel<CPL><<<(int)(need < cap ? need : cap), 256, 0, stream>>>(
+        (const uint4*)src, row_of, n_rows, src_rows, nv, (uint2*)dst, scale, err);
+    return cudaGetLastError();
+}
+
+// dst[p] = src[row_of[p]] for rows of `row_bytes` bytes (a multiple of 16), and, when given,
+// dscale[p] = sscale[row_of[p]]; one block per row per grid-stride step.
+__global__ void gather_code_rows_kernel(const uint4* __restrict__ src, const float* __restrict__ sscale,
+                                        const int32_t* __restrict__ row_of, long long n_rows, int src_rows, int nv,
+                                        uint4* __restrict__ dst, float* __restrict__ dscale, uint32_t* err) {
+    for (long long p = blockIdx.x; p < n_rows; p += gridDim.x) {
+        const int r = row_of[p];
+        const bool ok = r >= 0 && r < src_rows;
+        if (!ok && threadIdx.x == 0) flag_error(err, ERR_INDEX_RANGE);
+        const uint4* s = src + (size_t)(ok ? r : 0) * nv;
+        uint4* d = dst + (size_t)p * nv;
+        for (int i = threadIdx.x; i < nv; i += blockDim.x) d[i] = ok ? __ldg(s + i) : make_uint4(0, 0, 0, 0);
+        if (dscale && threadIdx.x == 0) dscale[p] = ok ? sscale[r] : 1.f;
     }
 }
 
@@ -88,10 +156,27 @@ cudaError_t launch_quant_rows(const void* src, const int32_t* row_of, long long 
                               uint8_t* dst, float* scale, uint32_t* err, cudaStream_t stream) {
     if (n_rows <= 0) return cudaSuccess;
     if (width <= 0 || width % 8) return cudaErrorInvalidValue;
+    const int nv = width / 8;
+    if (nv <= 32) return launch_warp<1>(src, row_of, n_rows, src_rows, nv, dst, scale, err, stream);
+    if (nv <= 64) return launch_warp<2>(src, row_of, n_rows, src_rows, nv, dst, scale, err, stream);
+    if (nv <= 128) return launch_warp<4>(src, row_of, n_rows, src_rows, nv, dst, scale, err, stream);
+    if (nv <= 256) return launch_warp<8>(src, row_of, n_rows, src_rows, nv, dst, scale, err, stream);
     const long long cap = (long long)num_sms() * 8;
+    const long long need = (n_rows + 7) / 8;
+    quant_rows_warp2_kernel<<<(int)(need < cap ? need : cap), 256, 0, stream>>>(
+        (const uint4*)src, row_of, n_rows, src_rows, nv, (uint2*)dst, scale, err);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_gather_code_rows(const uint8_t* src, const float* sscale, const int32_t* row_of, long long n_rows,
+                                    int src_rows, int row_bytes, uint8_t* dst, float* dscale, uint32_t* err,
+                                    cudaStream_t stream) {
+    if (n_rows <= 0) return cudaSuccess;
+    if (row_bytes <= 0 || row_bytes % 16) return cudaErrorInvalidValue;
+    const long long cap = (long long)num_sms() * 16;
     const int blocks = (int)(n_rows < cap ? n_rows : cap);
-    quant_rows_kernel<<<blocks, QT, 0, stream>>>((const uint4*)src, row_of, n_rows, src_rows, width / 8,
-                                                 (uint2*)dst, scale, err);
+    gather_code_rows_kernel<<<blocks, 128, 0, stream>>>((const uint4*)src, sscale, row_of, n_rows, src_rows,
+                                                        row_bytes / 16, (uint4*)dst, dscale, err);
     return cudaGetLastError();
 }
 

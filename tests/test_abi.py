@@ -68,9 +68,11 @@ def test_workspace_bytes(lib):
                 dict(has_bias=2), dict(n_shared=1, inter_shared=0), dict(gate_mode=3), dict(gate_mode=-1)):
         assert moe.workspace_bytes(_shape(**bad)) == 0, bad
     assert moe.workspace_bytes(_shape(d=7170, dtype=moe.MOE_F32)) > 0
-    # e4m3 routed experts: h8 rows and the two per-row scale arrays on top (x8 reuses x_perm)
+    # e4m3 routed experts: h8 rows, per-token x codes and the per-row scale arrays on top (the
+    # gathered x codes reuse x_perm)
     n8 = moe.workspace_bytes(_shape(routed_fmt=moe.FMT_E4M3))
-    assert S * I + 2 * 4 * S <= n8 - n <= S * I + 2 * 4 * S + 3 * 256
+    extra = S * I + 2 * 4 * S + 256 * d + 4 * 256
+    assert extra <= n8 - n <= extra + 5 * 256
     for bad in (dict(routed_fmt=2), dict(routed_fmt=-1)):
         assert moe.workspace_bytes(_shape(**bad)) == 0, bad
     for unsupported in (dict(dtype=moe.MOE_F32), dict(d=7176), dict(inter=2056)):
@@ -83,7 +85,7 @@ def test_launch_count(lib):
     assert moe.layer_launches(_shape(T=16384, n_shared=0)) == 9
     assert moe.layer_launches(_shape(T=128, d=256, n_experts=16, inter=64, inter_shared=64, top_k=4,
                                      dtype=moe.MOE_F32)) == 8
-    assert moe.layer_launches(_shape(routed_fmt=moe.FMT_E4M3)) == 11      # + hidden-row quantisation
+    assert moe.layer_launches(_shape(routed_fmt=moe.FMT_E4M3)) == 12      # + x per token, hidden rows
     assert moe.layer_launches(_shape(T=0)) == 0
     assert moe.layer_launches(_shape(top_k=0)) == -1
 

@@ -25,7 +25,7 @@ def _ws():
     return torch.zeros(4096, dtype=torch.uint8, device="cuda")
 
 
-@pytest.mark.parametrize("width", [8, 136, 2048, 7168, 9216])
+@pytest.mark.parametrize("width", [8, 136, 512, 1024, 2048, 2056, 4104, 7168, 9216])
 def test_quantize_rows_bit_exact(width):
     g = torch.Generator(device="cpu").manual_seed(width)
     n = 300
