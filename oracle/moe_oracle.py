@@ -35,6 +35,10 @@ What it computes, and where it comes from:
   at 448), so it is exact and reproducible; the products and sums run in fp64 on the exact
   dequantised values.  The e4m3 format is taken from its definition (1 sign, 4 exponent bits
   with bias 7, 3 mantissa bits, subnormals, S.1111.111 = NaN, no infinities).
+* Backward pass (an extension; the pages discuss it only through SonicMoE's backward kernels):
+  the chain rule of the forward above (layer_backward), and the balance statistics that the
+  DeepSeekMoE report's expert- and device-level balance losses are built from (balance_stats;
+  the formulas are stripped from the page, so these are a reading, PARITY UNPINNED).
 * Accounting helpers: ptflops-style MAC and parameter counts of one Expert (the ptflops
   printout on the first page), the expert-hit entropy diagnostic (DeepSeek-V2 explainer
   §6), and the combination count of fine-grained routing (DeepSeekMoE report §2.2).
@@ -334,6 +338,163 @@ def layer(x: np.ndarray, centroids: np.ndarray, routed: ExpertSource, n_experts:
         res["H"] = H if H is not None else np.zeros((T * k, 0))
         res["Hs"] = np.stack(Hs) if Hs else None
     return res
+
+
+# --------------------------------------------------------------------------------------
+# backward pass (chain rule of the forward above) and balance statistics
+# --------------------------------------------------------------------------------------
+def silu_grad(a: np.ndarray) -> np.ndarray:
+    """d/da [a * sigmoid(a)] = sigmoid(a) * (1 + a * (1 - sigmoid(a)))."""
+    sg = _sigmoid(a)
+    return sg * (1.0 + a * (1.0 - sg))
+
+
+def expert_backward(x: np.ndarray, w: Weights, dy: np.ndarray):
+    """Backward of one Expert, y = w2(silu(w1 x + b1) * (w3 x + b3)) + b2, for rows x [n, d] and
+    output gradients dy [n, d].  Returns (dx [n, d], grads {w1,b1,w3,b3,w2,b2}, y, h)."""
+    a = linear(x, w["w1"], w["b1"])
+    g = linear(x, w["w3"], w["b3"])
+    h = silu(a) * g
+    y = linear(h, w["w2"], w["b2"])
+    dh = dy @ w["w2"]
+    da = dh * g * silu_grad(a)
+    dg = dh * silu(a)
+    dx = da @ w["w1"] + dg @ w["w3"]
+    bias = w["b1"] is not None
+    grads = {"w1": da.T @ x, "b1": da.sum(0) if bias else None, "w3": dg.T @ x, "b3": dg.sum(0) if bias else None,
+             "w2": dy.T @ h, "b2": dy.sum(0) if bias else None}
+    return dx, grads, y, h
+
+
+def gate_backward(x: np.ndarray, centroids: np.ndarray, idx: np.ndarray, dgate: np.ndarray,
+                  gate_mode: int = GATE_SOFTMAX_TOPK, bias: Optional[np.ndarray] = None) -> np.ndarray:
+    """Gradient of the loss with respect to the router logits z = x . e_i (+ bias), given the
+    gradients dgate [T, N_r] of the gates of the picks idx (picks are a discrete choice and carry
+    no gradient).
+      mode 0: gate_j = s_{idx_j}, s = softmax(z):   dz_i = sum_j dgate_j s_{idx_j} (delta_{i,idx_j} - s_i)
+      mode 1: gate = softmax of the picked logits: dz_{idx_j} = gate_j (dgate_j - sum_l gate_l dgate_l)
+      mode 2: gate_j = sigma_j / sum_l sigma_l, sigma = sigmoid(z) (the routing bias only selects):
+              dz_{idx_j} = sigma_j (1 - sigma_j) (dgate_j - sum_l gate_l dgate_l) / sum_l sigma_l"""
+    x = np.asarray(x, np.float64)
+    c = np.asarray(centroids, np.float64)
+    idx = np.asarray(idx, np.int64)
+    T, N = x.shape[0], c.shape[0]
+    b = np.zeros(N) if bias is None else np.asarray(bias, np.float64)
+    z = x @ c.T
+    dz = np.zeros((T, N))
+    rows = np.arange(T)[:, None]
+    if gate_mode == GATE_SOFTMAX_TOPK:
+        z = z + b
+        e = np.exp(z - z.max(axis=1, keepdims=True))
+        s = e / e.sum(axis=1, keepdims=True)
+        sp = np.take_along_axis(s, idx, axis=1)
+        w = dgate * sp                                       # dgate_j s_{idx_j}
+        np.add.at(dz, (np.broadcast_to(rows, idx.shape), idx), w)
+        dz -= s * w.sum(axis=1, keepdims=True)
+    elif gate_mode == GATE_TOPK_SOFTMAX:
+        zp = np.take_along_axis(z + b, idx, axis=1)
+        ep = np.exp(zp - zp.max(axis=1, keepdims=True))
+        gate = ep / ep.sum(axis=1, keepdims=True)
+        d = gate * (dgate - (gate * dgate).sum(axis=1, keepdims=True))
+        np.add.at(dz, (np.broadcast_to(rows, idx.shape), idx), d)
+    elif gate_mode == GATE_SIGMOID_BIAS:
+        sg = np.take_along_axis(_sigmoid(z), idx, axis=1)
+        tot = sg.sum(axis=1, keepdims=True)
+        gate = sg / tot
+        d = sg * (1.0 - sg) * (dgate - (gate * dgate).sum(axis=1, keepdims=True)) / tot
+        np.add.at(dz, (np.broadcast_to(rows, idx.shape), idx), d)
+    else:
+        raise ValueError("unknown gate_mode")
+    return dz
+
+
+def layer_backward(x: np.ndarray, centroids: np.ndarray, routed: ExpertSource, n_experts: int, top_k: int,
+                   dout: np.ndarray, shared: Optional[ExpertSource] = None, n_shared: int = 0,
+                   idx_override: Optional[np.ndarray] = None, gate_mode: int = GATE_SOFTMAX_TOPK,
+                   router_bias: Optional[np.ndarray] = None, tokens: Optional[np.ndarray] = None,
+                   experts: Optional[Sequence[int]] = None) -> Dict[str, object]:
+    """Gradients of the layer output contracted with dout [T, d] (the backward of layer()).
+
+    Returns dx [T, d] (rows outside `tokens` are left zero when a token subset is given), the
+    routed experts' gradients {e: {w1,b1,w3,b3,w2,b2}} for the experts in `experts` (default: all
+    experts that received a token; each over ALL of its tokens), the shared experts' gradients
+    [{...}] (over all tokens), dcentroids [N_m, d], drouter_bias [N_m] (None when the bias only
+    selects, gate mode 2, or there is none), dgate [T, N_r] and dz [T, N_m].
+
+    Chain rule of the forward: dy_{t,j} = gate_{t,j} dout_t; dgate_{t,j} = <dout_t, y_{t,j}> (y the
+    expert output before the gate, bias included); each expert's backward (expert_backward);
+    shared experts with gate 1; router: dz from dgate (gate_backward), dx += dz C, dC = dz^T x,
+    dbias = sum_t dz_t.  Like layer(), routing uses idx_override when given.
+    """
+    x = np.asarray(x, np.float64)
+    dout = np.asarray(dout, np.float64)
+    c = np.asarray(centroids, np.float64)
+    T, d = x.shape
+    r = route(x, c, top_k, gate_mode, router_bias)
+    if idx_override is not None:
+        idx = np.asarray(idx_override, np.int64)
+        gate = gates_from_indices(x, c, idx, gate_mode, router_bias)
+    else:
+        idx, gate = r["idx"], r["gate"]
+    want_tok = np.ones(T, bool) if tokens is None else np.isin(np.arange(T), np.asarray(tokens))
+    want_exp = set(int(e) for e in (np.unique(idx) if experts is None else experts))
+    dx = np.zeros((T, d))
+    dgate = np.zeros(idx.shape)
+    grads = {}
+    for e in np.unique(idx):
+        e = int(e)
+        tt, jj = np.nonzero(idx == e)
+        if e not in want_exp:
+            keep = want_tok[tt]
+            tt, jj = tt[keep], jj[keep]
+        if len(tt) == 0:
+            continue
+        w = _expert(routed, e)
+        dy = gate[tt, jj][:, None] * dout[tt]
+        dxe, ge, y, _ = expert_backward(x[tt], w, dy)
+        dgate[tt, jj] = (dout[tt] * y).sum(axis=1)
+        np.add.at(dx, tt, dxe)
+        if e in want_exp:
+            grads[e] = ge
+    shared_grads = []
+    for j in range(n_shared):
+        dxs, gs, _, _ = expert_backward(x, _expert(shared, j), dout)
+        dx += dxs
+        shared_grads.append(gs)
+    sel = np.nonzero(want_tok)[0]
+    dz = np.zeros((T, c.shape[0]))
+    dz[sel] = gate_backward(x[sel], c, idx[sel], dgate[sel], gate_mode, router_bias)
+    dx += dz @ c
+    dc = dz.T @ x
+    dbias = dz.sum(axis=0) if (router_bias is not None and gate_mode != GATE_SIGMOID_BIAS) else None
+    dx[~want_tok] = 0.0
+    return {"dx": dx, "routed": grads, "shared": shared_grads, "dcentroids": dc, "drouter_bias": dbias,
+            "dgate": dgate, "dz": dz, "idx": idx, "gate": gate}
+
+
+def balance_stats(s: np.ndarray, idx: np.ndarray, n_experts: int, top_k: int, n_groups: int = 1):
+    """Expert- and device-level balance statistics of one batch (DeepSeekMoE report §2.5 and §3:
+    per expert, the batch mean of its gate scores and its hit rate; losses that penalise their
+    imbalance, weights alpha1 / alpha2).  The pages give the quantities in prose only; the
+    formulas below are this project's reading (PARITY UNPINNED against the pages):
+      f_i = N_m / (N_r T) * #{(t, j): idx_{t,j} = i}     (1 for every expert under uniform routing)
+      P_i = (1 / T) * sum_t s_{i,t}                      (s: the router's scores over all experts)
+      expert-level term  sum_i f_i P_i
+      device-level (experts split into n_groups equal contiguous groups E_g):
+      f'_g = mean_{i in E_g} f_i,  P'_g = sum_{i in E_g} P_i,  term  sum_g f'_g P'_g
+    Returns f [N_m], P [N_m], the two terms and the hit counts."""
+    s = np.asarray(s, np.float64)
+    T = s.shape[0]
+    counts = np.bincount(np.asarray(idx).reshape(-1), minlength=n_experts).astype(np.float64)
+    f = counts * n_experts / (top_k * T) if T else np.zeros(n_experts)
+    P = s.mean(axis=0) if T else np.zeros(n_experts)
+    if n_experts % n_groups:
+        raise ValueError("n_groups must divide n_experts")
+    per = n_experts // n_groups
+    fg = f.reshape(n_groups, per).mean(axis=1)
+    Pg = P.reshape(n_groups, per).sum(axis=1)
+    return {"f": f, "P": P, "expert_term": float((f * P).sum()), "device_term": float((fg * Pg).sum()),
+            "counts": counts}
 
 
 # --------------------------------------------------------------------------------------

@@ -477,7 +477,135 @@ def check_fp8_layer_closed_form(O):
     assert np.allclose(res["out"], want, rtol=1e-12, atol=1e-12)
 
 
+def _torch_layer_loss(x, c, bias, experts, shared, idx, dout, gate_mode):
+    """The layer in float64 torch with the picks fixed to idx: L = <out, dout>.  Returns L and the
+    leaf tensors (x, c, bias, routed expert modules, shared expert modules)."""
+    xt = torch.from_numpy(x).requires_grad_(True)
+    ct = torch.from_numpy(c).requires_grad_(True)
+    bt = torch.from_numpy(bias).requires_grad_(True)
+    it = torch.from_numpy(np.asarray(idx, np.int64))
+    mods = [TorchExpert(w) for w in experts]
+    smods = [TorchExpert(w) for w in shared]
+    z = xt @ ct.T
+    if gate_mode == 2:
+        sg = torch.sigmoid(z).gather(1, it)
+        gate = sg / sg.sum(1, keepdim=True)
+    elif gate_mode == 1:
+        gate = torch.softmax((z + bt).gather(1, it), dim=1)
+    else:
+        gate = torch.softmax(z + bt, dim=1).gather(1, it)
+    out = sum(m(xt) for m in smods) if smods else torch.zeros_like(xt)
+    for t in range(x.shape[0]):
+        for j in range(it.shape[1]):
+            out = out.index_add(0, torch.tensor([t]), gate[t, j] * mods[int(it[t, j])](xt[t:t + 1]))
+    L = (out * torch.from_numpy(dout)).sum()
+    return L, xt, ct, bt, mods, smods
+
+
+def check_backward_autograd(O):
+    """layer_backward (the chain rule written out) against torch.autograd on the same layer in
+    float64, for every gate mode, with biases, a router bias and two shared experts."""
+    rng = _rng(31)
+    T, d, N, k, I, Is = 7, 12, 6, 3, 5, 4
+    x = rng.normal(0, 1, (T, d))
+    c = rng.normal(0, 0.5, (N, d))
+    bias = rng.normal(0, 0.3, N)
+    experts = [_rand_expert(rng, d, I) for _ in range(N)]
+    shared = [_rand_expert(rng, d, Is) for _ in range(2)]
+    dout = rng.normal(0, 1, (T, d))
+    for mode in (0, 1, 2):
+        res = O.layer_backward(x, c, _stack(experts), N, k, dout, _stack(shared), 2, gate_mode=mode, router_bias=bias)
+        L, xt, ct, bt, mods, smods = _torch_layer_loss(x, c, bias, experts, shared, res["idx"], dout, mode)
+        L.backward()
+        assert np.allclose(res["dx"], xt.grad.numpy(), rtol=1e-10, atol=1e-12), mode
+        assert np.allclose(res["dcentroids"], ct.grad.numpy(), rtol=1e-10, atol=1e-12), mode
+        if mode == 2:                       # the routing bias only selects: no gradient
+            assert res["drouter_bias"] is None
+            assert bt.grad is None or not bt.grad.abs().max().item() > 0
+        else:
+            assert np.allclose(res["drouter_bias"], bt.grad.numpy(), rtol=1e-10, atol=1e-12), mode
+        for e, g in res["routed"].items():
+            m = mods[e]
+            for name, lin in (("w1", m.w1), ("w3", m.w3), ("w2", m.w2)):
+                assert np.allclose(g[name], lin.weight.grad.numpy(), rtol=1e-10, atol=1e-12), (mode, e, name)
+                assert np.allclose(g["b" + name[1]], lin.bias.grad.numpy(), rtol=1e-10, atol=1e-12), (mode, e, name)
+        assert set(res["routed"]) == set(np.unique(res["idx"]).tolist())
+        for j, g in enumerate(res["shared"]):
+            assert np.allclose(g["w2"], smods[j].w2.weight.grad.numpy(), rtol=1e-10, atol=1e-12)
+            assert np.allclose(g["b1"], smods[j].w1.bias.grad.numpy(), rtol=1e-10, atol=1e-12)
+    # token and expert subsets: the same numbers where they are asked for
+    full = O.layer_backward(x, c, _stack(experts), N, k, dout, _stack(shared), 2)
+    part = O.layer_backward(x, c, _stack(experts), N, k, dout, _stack(shared), 2, tokens=[1, 4],
+                            experts=[int(full["idx"][0, 0])])
+    assert np.allclose(part["dx"][[1, 4]], full["dx"][[1, 4]], rtol=1e-13, atol=1e-14)
+    assert not part["dx"][[0, 2, 3, 5, 6]].any()
+    e0 = int(full["idx"][0, 0])
+    assert set(part["routed"]) == {e0}
+    assert np.allclose(part["routed"][e0]["w1"], full["routed"][e0]["w1"], rtol=1e-13, atol=1e-14)
+
+
+def check_backward_finite_differences(O):
+    """layer_backward against central differences of <layer(...)["out"], dout> (the pinned forward
+    oracle), on well-separated picks so no perturbation changes them."""
+    rng = _rng(32)
+    T, d, N, k, I = 4, 6, 5, 2, 3
+    x = rng.normal(0, 1, (T, d))
+    c = rng.normal(0, 1.0, (N, d))
+    experts = [_rand_expert(rng, d, I) for _ in range(N)]
+    shared = [_rand_expert(rng, d, I)]
+    dout = rng.normal(0, 1, (T, d))
+    assert O.route(x, c, k)["gap"].min() > 1e-3
+    res = O.layer_backward(x, c, _stack(experts), N, k, dout, _stack(shared), 1)
+    h = 1e-6
+
+    def loss(xx=x, cc=c, st=None):
+        return float((O.layer(xx, cc, st or _stack(experts), N, k, _stack(shared), 1)["out"] * dout).sum())
+    for (t, i) in ((0, 0), (2, 5), (3, 3)):
+        xp, xm = x.copy(), x.copy()
+        xp[t, i] += h
+        xm[t, i] -= h
+        assert abs((loss(xx=xp) - loss(xx=xm)) / (2 * h) - res["dx"][t, i]) < 1e-6
+    for (e, i) in ((1, 2), (4, 0)):
+        cp, cm = c.copy(), c.copy()
+        cp[e, i] += h
+        cm[e, i] -= h
+        assert abs((loss(cc=cp) - loss(cc=cm)) / (2 * h) - res["dcentroids"][e, i]) < 1e-6
+    e = int(res["idx"][0, 0])
+    for name, pos in (("w1", (1, 2)), ("w3", (0, 4)), ("w2", (5, 1)), ("b2", (3,))):
+        sp, sm = _stack(experts), _stack(experts)
+        sp[name] = sp[name].copy(); sm[name] = sm[name].copy()
+        sp[name][(e,) + pos] += h
+        sm[name][(e,) + pos] -= h
+        assert abs((loss(st=sp) - loss(st=sm)) / (2 * h) - res["routed"][e][name][pos]) < 1e-6, name
+
+
+def check_balance_stats(O):
+    """Balance statistics: closed forms for uniform and collapsed routing, sums fixed by the
+    definitions, hit counts as hit_entropy counts them."""
+    T, N, k = 64, 8, 2
+    idx = np.stack([np.arange(T) % N, (np.arange(T) + 1) % N], axis=1)
+    s = np.full((T, N), 1.0 / N)
+    b = O.balance_stats(s, idx, N, k, n_groups=4)
+    assert np.allclose(b["f"], 1.0) and np.allclose(b["P"], 1.0 / N)
+    assert abs(b["expert_term"] - 1.0) < 1e-14 and abs(b["device_term"] - 1.0) < 1e-14
+    idx_c = np.tile([0, 1], (T, 1))
+    s_c = np.zeros((T, N)); s_c[:, :2] = 0.5
+    bc = O.balance_stats(s_c, idx_c, N, k, n_groups=2)
+    assert abs(bc["expert_term"] - N / k) < 1e-12
+    # group 0 (experts 0-3) holds both hit experts: f' = (N/k + N/k) / 4, P' = 1; group 1 adds 0
+    assert abs(bc["device_term"] - 2 * (N / k) / (N // 2)) < 1e-12
+    rng = _rng(33)
+    z = rng.normal(0, 1, (T, N))
+    sr = np.exp(z) / np.exp(z).sum(1, keepdims=True)
+    idx_r = np.argsort(-z, axis=1, kind="stable")[:, :k]
+    br = O.balance_stats(sr, idx_r, N, k)
+    assert abs(br["f"].sum() - N) < 1e-12 and abs(br["P"].sum() - 1.0) < 1e-12
+    assert np.array_equal(br["counts"], O.hit_entropy(idx_r, N)[2])
+    assert abs(br["device_term"] - br["f"].mean() * 1.0) < 1e-12            # one group: f' = mean f, P' = 1
+
+
 ALL_CHECKS = [check_ptflops_printout, check_combinations, check_textbook_single_expert,
               check_gate_invariants, check_bruteforce_routing, check_split_identity,
               check_shared_bypasses_router, check_hit_entropy, check_permute, check_gate_modes,
-              check_e4m3_format, check_fp8_layer_closed_form]
+              check_e4m3_format, check_fp8_layer_closed_form, check_backward_autograd,
+              check_backward_finite_differences, check_balance_stats]

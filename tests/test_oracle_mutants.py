@@ -11,7 +11,8 @@ from tests import pins
 
 _orig = {name: getattr(O, name) for name in ("silu", "linear", "route", "swiglu_hidden", "permute",
                                              "expert_macs", "split_expert", "hit_entropy", "e4m3_round",
-                                             "quantize_rows_e4m3", "e4m3_weights", "e4m3_decode")}
+                                             "quantize_rows_e4m3", "e4m3_weights", "e4m3_decode",
+                                             "silu_grad", "gate_backward", "expert_backward", "balance_stats")}
 
 
 def _sigmoid_for_silu(a):                      # silu without the factor a
@@ -141,6 +142,43 @@ def _bf16_truncate(a):                         # rounds toward zero on the fp32 
     return u.view(np.float32).astype(np.float64)
 
 
+def _silu_grad_sigmoid(a):                     # derivative of silu taken as sigmoid(a)
+    return 1.0 / (1.0 + np.exp(-np.asarray(a, np.float64)))
+
+
+def _gate_backward_no_softmax_term(x, c, idx, dgate, gate_mode=0, bias=None):   # drops -s_i sum_j ...
+    if gate_mode != 0:
+        return _orig["gate_backward"](x, c, idx, dgate, gate_mode, bias)
+    z = np.asarray(x, np.float64) @ np.asarray(c, np.float64).T
+    if bias is not None:
+        z = z + bias
+    e = np.exp(z - z.max(1, keepdims=True)); sm = e / e.sum(1, keepdims=True)
+    dz = np.zeros_like(z)
+    rows = np.arange(z.shape[0])[:, None]
+    np.add.at(dz, (np.broadcast_to(rows, idx.shape), idx), dgate * np.take_along_axis(sm, idx, 1))
+    return dz
+
+
+def _expert_backward_no_gate_factor(x, w, dy):  # da without the factor g
+    a = O.linear(x, w["w1"], w["b1"]); g = O.linear(x, w["w3"], w["b3"])
+    h = O.silu(a) * g
+    y = O.linear(h, w["w2"], w["b2"])
+    dh = dy @ w["w2"]
+    da = dh * O.silu_grad(a)
+    dg = dh * O.silu(a)
+    bias = w["b1"] is not None
+    grads = {"w1": da.T @ x, "b1": da.sum(0) if bias else None, "w3": dg.T @ x, "b3": dg.sum(0) if bias else None,
+             "w2": dy.T @ h, "b2": dy.sum(0) if bias else None}
+    return da @ w["w1"] + dg @ w["w3"], grads, y, h
+
+
+def _balance_unnormalised(s, idx, n, k, n_groups=1):   # f as raw hit counts
+    b = dict(_orig["balance_stats"](s, idx, n, k, n_groups))
+    b["f"] = b["counts"].copy()
+    b["expert_term"] = float((b["f"] * b["P"]).sum())
+    return b
+
+
 MUTANTS = {
     "silu_is_sigmoid": ("silu", _sigmoid_for_silu),
     "linear_drops_bias": ("linear", _linear_no_bias),
@@ -160,6 +198,10 @@ MUTANTS = {
     "fp8_weight_scale_by_column": ("e4m3_weights", _weights_scale_by_column),
     "e4m3_no_subnormals": ("e4m3_decode", _decode_no_subnormals),
     "bf16_truncates": ("bf16_round", _bf16_truncate),
+    "silu_grad_is_sigmoid": ("silu_grad", _silu_grad_sigmoid),
+    "gate_backward_drops_softmax_term": ("gate_backward", _gate_backward_no_softmax_term),
+    "expert_backward_drops_g": ("expert_backward", _expert_backward_no_gate_factor),
+    "balance_f_unnormalised": ("balance_stats", _balance_unnormalised),
 }
 
 
