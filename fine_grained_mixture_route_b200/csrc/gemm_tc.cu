@@ -54,7 +54,12 @@ constexpr unsigned long long WAIT_NS = 4000000000ull;
 #endif
 constexpr uint32_t PEER_BIT_MASK = 0xFEFFFFFFu;   // shared::cluster address of CTA rank 0 of a pair
 
-enum Mode : int { ROUTER = 0, GEMM1 = 1, GEMM2R = 2, GEMM2S = 3, ROUTERP = 4 };
+enum Mode : int { ROUTER = 0, GEMM1 = 1, GEMM2R = 2, GEMM2S = 3, ROUTERP = 4, DH = 5, DX = 6, DXS = 7, DW = 8 };
+// Backward modes (B operand MN-major: contraction along rows, 64-column boxes):
+//   DH  dh = dout . W2 per routed / shared group, SwiGLU backward and the gate gradient in the epilogue
+//   DX  dx per routed slot = [da | dg] . [W1 ; W3]
+//   DXS shared experts' dx + the router's dz . C, accumulated along K, fp32 per token
+//   DW  weight gradients: A and B both MN-major, K = the rows (tokens) of a group
 
 // The expert GEMMs can run on CTA pairs (cta_group::2): a 256-row tile, each CTA holding 128
 // rows of A, half of the 256 B rows and its 128 x 256 slice of the accumulator, so each SM
@@ -95,6 +100,25 @@ struct Params {
     const float* a_scale;      // q8: per-row scale of the routed A rows (x_perm or h rows)
     const float *ws1, *ws3, *ws2;  // q8: per-output-channel weight scales [E, I], [E, I], [E, d]
     int fold_shared;           // GEMM2R: shared-expert GEMM2 tiles follow the routed ones (-> sout)
+    // ---- forward for training: GEMM1 also stores the pre-activations a = x W1^T + b1, g = x W3^T + b3
+    __nv_bfloat16 *a_out, *g_out;      // routed [S][I] (grouped order)
+    __nv_bfloat16 *as_out, *gs_out;    // shared [Ks][T][Is]
+    // ---- backward
+    const int32_t* offs_pad;           // [E+1] starts of the 64-row-padded groups (dout / x / dag / hg rows)
+    const __nv_bfloat16 *a_sv, *g_sv;  // saved pre-activations, routed [S][I]
+    const __nv_bfloat16 *as_sv, *gs_sv;  // shared [Ks][T][Is]
+    __nv_bfloat16 *dag, *hg;           // DH out, routed: [S_pad][2I] (da | dg), [S_pad][I] (gate * h)
+    __nv_bfloat16 *dag_s, *hg_s;       // DH out, shared: [Ks][T][2Is], [Ks][T][Is]
+    float* dgate_part;                 // DH out: [S][n_parts] partial sums of dh_raw * h
+    int n_parts;
+    __nv_bfloat16* dx_slot;            // DX out: [S][d] (grouped order)
+    int dw_kind;                       // DW: 0 out [g][M][N]; 1 rows < M/2 -> out0, rest -> out1; 2 fp32 [M][N]
+    int dw_groups, dw_M, dw_N;         // DW: groups and output rows / columns per group
+    int dw_a3d, dw_b3d;                // DW: operand map is 3-D (third coordinate = group)
+    const int32_t* dw_rows;            // DW: group row starts [groups+1] (padded), or null: rows = dw_K
+    int dw_K;
+    __nv_bfloat16 *dw_out0, *dw_out1;
+    float* dw_out_f32;
     uint32_t* err;
 };
 
@@ -174,6 +198,19 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t addr) {
     d |= (uint64_t)2 << 61;
     return d;
 }
+// Shared-memory descriptor of an MN-major operand, 128-byte swizzle: 64-element rows along MN,
+// 8-row K groups 1024 bytes apart (stride byte offset), 64-wide MN blocks 8 KB apart (leading
+// byte offset: one TMA box of 64 K rows each).
+__device__ __forceinline__ uint64_t mn_sw128_desc(uint32_t addr) {
+    uint64_t d = 0;
+    d |= (uint64_t)((addr & 0x3FFFFu) >> 4);
+    d |= (uint64_t)(8192 >> 4) << 16;
+    d |= (uint64_t)(1024 >> 4) << 32;
+    d |= (uint64_t)1 << 46;
+    d |= (uint64_t)2 << 61;
+    return d;
+}
+constexpr uint32_t IDESC_A_MN = 1u << 15, IDESC_B_MN = 1u << 16;   // operand major-ness bits
 // Instruction descriptor, kind::f16: fp32 accumulator, bf16 A and B, both K-major, M=128.
 __host__ __device__ constexpr uint32_t idesc_bf16(int n) {
     return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
@@ -317,6 +354,9 @@ __device__ __forceinline__ int total_tiles(const Params& p) {
     if (MODE == GEMM1) return p.tile_start[p.g_end] - p.tile_start[p.g_begin];
     if (MODE == GEMM2R)
         return p.tile_start[p.E] + (p.fold_shared ? ceil_div(p.T, TM) * ceil_div(p.d, 256) : 0);
+    if (MODE == DH) return p.tile_start[p.E + p.Ks];
+    if (MODE == DX) return p.tile_start[p.E];
+    if (MODE == DW) return p.dw_groups * ceil_div(p.dw_M, TM) * ceil_div(p.dw_N, 256);
     return ceil_div(p.T, TM) * ceil_div(p.d, 256);
 }
 
@@ -369,6 +409,47 @@ __device__ __forceinline__ Tile decode(const Params& p, int t) {
         x.m0 = m * TM;
         x.n0 = n * 128;
         x.num_kb = ceil_div(p.d, (p.q8 && !shared) ? 2 * BK : BK);
+    } else if (MODE == DH) {
+        const int g = find_group(p.tile_start, 0, p.E + p.Ks, t);
+        const int local = t - p.tile_start[g];
+        const bool shared = g >= p.E;
+        x.g = g;
+        x.rows = shared ? p.T : p.offsets[g + 1] - p.offsets[g];
+        x.row0 = shared ? 0 : p.offs_pad[g];
+        int m, n;
+        band_mn(local, ceil_div(x.rows, TM), ceil_div(shared ? p.Is : p.I, 256), p.group_m, m, n);
+        x.m0 = m * TM;
+        x.n0 = n * 256;
+        x.num_kb = ceil_div(p.d, BK);
+    } else if (MODE == DX) {
+        const int e = find_group(p.tile_start, 0, p.E, t);
+        const int local = t - p.tile_start[e];
+        x.g = e;
+        x.rows = p.offsets[e + 1] - p.offsets[e];
+        x.row0 = p.offs_pad[e];
+        int m, n;
+        band_mn(local, ceil_div(x.rows, TM), ceil_div(p.d, 256), p.group_m, m, n);
+        x.m0 = m * TM;
+        x.n0 = n * 256;
+        x.num_kb = 2 * ceil_div(p.I, BK);
+    } else if (MODE == DXS) {
+        x.g = 0; x.rows = p.T; x.row0 = 0;
+        int m, n;
+        band_mn(t, ceil_div(p.T, TM), ceil_div(p.d, 256), p.group_m, m, n);
+        x.m0 = m * TM;
+        x.n0 = n * 256;
+        x.num_kb = p.Ks * 2 * ceil_div(p.Is, BK) + ceil_div(p.E, BK);
+    } else if (MODE == DW) {
+        const int mt = ceil_div(p.dw_M, TM), nt = ceil_div(p.dw_N, 256);
+        const int g = t / (mt * nt);
+        int m, n;
+        band_mn(t - g * mt * nt, mt, nt, p.group_m, m, n);
+        x.g = g;
+        x.m0 = m * TM;
+        x.n0 = n * 256;
+        x.row0 = p.dw_rows ? p.dw_rows[g] : 0;
+        x.rows = p.dw_rows ? p.dw_rows[g + 1] - p.dw_rows[g] : p.dw_K;
+        x.num_kb = ceil_div(x.rows, BK);
     } else if (MODE == GEMM2R && t >= p.tile_start[p.E]) {
         // shared-expert tile (fold_shared): all K_s experts accumulated along K
         const int mt = ceil_div(p.T, TM);
@@ -508,6 +589,13 @@ __device__ __forceinline__ void epilogue_gemm1(const Params& p, const Tile& x, u
     const bool live = r < x.rows;
     const float rs = (scaled && live) ? p.a_scale[x.row0 + r] : 1.f;
     __nv_bfloat16* hrow = shared ? p.h_s + ((size_t)e * p.T + r) * I : p.h_r + (size_t)(x.row0 + r) * I;
+    __nv_bfloat16* arow = nullptr;
+    __nv_bfloat16* grow = nullptr;
+    if (p.a_out) {
+        const size_t o = shared ? ((size_t)e * p.T + r) * I : (size_t)(x.row0 + r) * I;
+        arow = (shared ? p.as_out : p.a_out) + o;
+        grow = (shared ? p.gs_out : p.g_out) + o;
+    }
 #pragma unroll 1
     for (int c = half * 2; c < half * 2 + 2; ++c) {
         uint32_t u[32], v[32];
@@ -520,10 +608,10 @@ __device__ __forceinline__ void epilogue_gemm1(const Params& p, const Tile& x, u
         for (int q = 0; q < 4; ++q) {
             const int col = col0 + q * 8;
             if (col >= I) break;
-            uint32_t pk[4];
+            uint32_t pk[4], pa[4], pg[4];
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                float hv[2];
+                float hv[2], av[2], gv[2];
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
                     const int j = q * 8 + i * 2 + h;
@@ -534,10 +622,18 @@ __device__ __forceinline__ void epilogue_gemm1(const Params& p, const Tile& x, u
                     a += b1 ? __bfloat162float(b1[cc]) : 0.f;
                     g += b3 ? __bfloat162float(b3[cc]) : 0.f;
                     hv[h] = silu_f32(a) * g;
+                    av[h] = a;
+                    gv[h] = g;
                 }
                 pk[i] = pack_bf16(hv[0], hv[1]);
+                pa[i] = pack_bf16(av[0], av[1]);
+                pg[i] = pack_bf16(gv[0], gv[1]);
             }
             *reinterpret_cast<uint4*>(hrow + col) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            if (arow) {
+                *reinterpret_cast<uint4*>(arow + col) = make_uint4(pa[0], pa[1], pa[2], pa[3]);
+                *reinterpret_cast<uint4*>(grow + col) = make_uint4(pg[0], pg[1], pg[2], pg[3]);
+            }
         }
     }
 }
@@ -627,6 +723,143 @@ __device__ __forceinline__ void epilogue_router_partial(const Params& p, const T
                 *reinterpret_cast<float4*>(dst + c0 + q * 4) =
                     make_float4(__uint_as_float(r[q * 4]), __uint_as_float(r[q * 4 + 1]), __uint_as_float(r[q * 4 + 2]),
                                 __uint_as_float(r[q * 4 + 3]));
+        }
+    }
+}
+
+// DH: for a routed group the rows are grouped slots (A = dout rows of the slot's token, in the
+// 64-row-padded layout), for a shared group the tokens.  Per element of the hidden row:
+// dh_raw = (dout . W2)[c]; a, g = the saved pre-activations; sg = sigmoid(a); h = a sg g;
+// dh = gate dh_raw; da = dh g sg (1 + a (1 - sg)); dg = dh a sg; and the row's partial sum of
+// dh_raw h (the gate gradient, without its b2 term) over this thread's 128 columns.  Writes da | dg
+// and gate * h (the B operand of the w2 gradient); the padding rows of a routed group (up to the
+// next multiple of 64) get zeros, so the weight-gradient GEMMs can run whole 64-row K blocks.
+__device__ __forceinline__ void epilogue_dh(const Params& p, const Tile& x, uint32_t tacc, int row, int half) {
+    const bool shared = x.g >= p.E;
+    const int e = shared ? x.g - p.E : x.g;
+    const int I = shared ? p.Is : p.I;
+    const int r = x.m0 + row;
+    const bool live = r < x.rows;
+    const bool pad = !shared && !live && r < ceil_div(x.rows, 64) * 64;
+    const long long pu = shared ? r : (long long)p.offsets[e] + r;       // grouped slot (routed) / token
+    const long long pp = shared ? r : (long long)x.row0 + r;             // padded row (routed) / token
+    const size_t so = shared ? ((size_t)e * p.T + r) * I : (size_t)pu * I;
+    const __nv_bfloat16* arow = (shared ? p.as_sv : p.a_sv) + so;
+    const __nv_bfloat16* grow = (shared ? p.gs_sv : p.g_sv) + so;
+    __nv_bfloat16* dagrow = shared ? p.dag_s + ((size_t)e * p.T + r) * 2 * I : p.dag + (size_t)pp * 2 * I;
+    __nv_bfloat16* hgrow = shared ? p.hg_s + ((size_t)e * p.T + r) * I : p.hg + (size_t)pp * I;
+    const float gate = (!shared && live) ? p.sorted_gate[pu] : 1.f;
+    float dot = 0.f;
+#pragma unroll 1
+    for (int c = half * 4; c < half * 4 + 4; ++c) {
+        uint32_t u[32];
+        tmem_ld32(tacc + c * 32, u);
+        tmem_wait_ld();
+        const int col0 = x.n0 + c * 32;
+        if ((!live && !pad) || col0 >= I) continue;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int col = col0 + q * 8;
+            if (col >= I) break;
+            uint32_t pda[4] = {0, 0, 0, 0}, pdg[4] = {0, 0, 0, 0}, phg[4] = {0, 0, 0, 0};
+            if (live) {
+                const uint4 av = *reinterpret_cast<const uint4*>(arow + col);
+                const uint4 gv = *reinterpret_cast<const uint4*>(grow + col);
+                const uint32_t aw[4] = {av.x, av.y, av.z, av.w}, gw[4] = {gv.x, gv.y, gv.z, gv.w};
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    float da2[2], dg2[2], hg2[2];
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const float a = __uint_as_float(h ? (aw[i] & 0xFFFF0000u) : (aw[i] << 16));
+                        const float g = __uint_as_float(h ? (gw[i] & 0xFFFF0000u) : (gw[i] << 16));
+                        const float dhr = __uint_as_float(u[q * 8 + i * 2 + h]);
+                        const float sg = 1.0f / (1.0f + expf(-a));
+                        const float si = a * sg;
+                        const float hv = si * g;
+                        dot += dhr * hv;
+                        const float dh = gate * dhr;
+                        da2[h] = dh * g * sg * (1.0f + a * (1.0f - sg));
+                        dg2[h] = dh * si;
+                        hg2[h] = gate * hv;
+                    }
+                    pda[i] = pack_bf16(da2[0], da2[1]);
+                    pdg[i] = pack_bf16(dg2[0], dg2[1]);
+                    phg[i] = pack_bf16(hg2[0], hg2[1]);
+                }
+            }
+            *reinterpret_cast<uint4*>(dagrow + col) = make_uint4(pda[0], pda[1], pda[2], pda[3]);
+            *reinterpret_cast<uint4*>(dagrow + I + col) = make_uint4(pdg[0], pdg[1], pdg[2], pdg[3]);
+            *reinterpret_cast<uint4*>(hgrow + col) = make_uint4(phg[0], phg[1], phg[2], phg[3]);
+        }
+    }
+    if (!shared && live) p.dgate_part[(size_t)pu * p.n_parts + (x.n0 / 256) * 2 + half] = dot;
+}
+
+// DX: dx of a routed slot (grouped order), bf16.
+__device__ __forceinline__ void epilogue_dx(const Params& p, const Tile& x, uint32_t tacc, int row, int half) {
+    const int r = x.m0 + row;
+    const bool live = r < x.rows;
+    __nv_bfloat16* orow = p.dx_slot + ((size_t)p.offsets[x.g] + r) * p.d;
+#pragma unroll 1
+    for (int c = half * 4; c < half * 4 + 4; ++c) {
+        uint32_t u[32];
+        tmem_ld32(tacc + c * 32, u);
+        tmem_wait_ld();
+        const int col0 = x.n0 + c * 32;
+        if (!live || col0 >= p.d) continue;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int col = col0 + q * 8;
+            if (col >= p.d) break;
+            uint32_t pk[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                pk[i] = pack_bf16(__uint_as_float(u[q * 8 + i * 2]), __uint_as_float(u[q * 8 + i * 2 + 1]));
+            *reinterpret_cast<uint4*>(orow + col) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        }
+    }
+}
+
+// DW: one 128 x 256 tile of a group's weight gradient (zeros when the group has no rows).
+__device__ __forceinline__ void epilogue_dw(const Params& p, const Tile& x, uint32_t tacc, int row, int half) {
+    const int m = x.m0 + row;
+    const bool live = m < p.dw_M;
+    const bool zero = x.num_kb == 0;
+    const int Mh = p.dw_M / 2;
+    __nv_bfloat16* orow = nullptr;
+    float* frow = nullptr;
+    if (p.dw_kind == 0) orow = p.dw_out0 + ((size_t)x.g * p.dw_M + m) * p.dw_N;
+    else if (p.dw_kind == 1) orow = m < Mh ? p.dw_out0 + ((size_t)x.g * Mh + m) * p.dw_N
+                                           : p.dw_out1 + ((size_t)x.g * Mh + m - Mh) * p.dw_N;
+    else frow = p.dw_out_f32 + ((size_t)x.g * p.dw_M + m) * p.dw_N;
+#pragma unroll 1
+    for (int c = half * 4; c < half * 4 + 4; ++c) {
+        uint32_t u[32];
+        tmem_ld32(tacc + c * 32, u);
+        tmem_wait_ld();
+        const int col0 = x.n0 + c * 32;
+        if (!live || col0 >= p.dw_N) continue;
+        if (zero) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) u[i] = 0u;
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int col = col0 + q * 8;
+            if (col >= p.dw_N) break;
+            if (frow) {
+                *reinterpret_cast<float4*>(frow + col) = make_float4(__uint_as_float(u[q * 8]), __uint_as_float(u[q * 8 + 1]),
+                                                                     __uint_as_float(u[q * 8 + 2]), __uint_as_float(u[q * 8 + 3]));
+                *reinterpret_cast<float4*>(frow + col + 4) = make_float4(__uint_as_float(u[q * 8 + 4]), __uint_as_float(u[q * 8 + 5]),
+                                                                         __uint_as_float(u[q * 8 + 6]), __uint_as_float(u[q * 8 + 7]));
+            } else {
+                uint32_t pk[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    pk[i] = pack_bf16(__uint_as_float(u[q * 8 + i * 2]), __uint_as_float(u[q * 8 + i * 2 + 1]));
+                *reinterpret_cast<uint4*>(orow + col) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            }
         }
     }
 }
@@ -751,6 +984,52 @@ __global__ void __launch_bounds__(THREADS, 1) moe_tc_kernel(const __grid_constan
                             tma_load_3d_pair(a_dst, &p.tmA[0], fb, kk * BK, x.m0 + arow, s);
                             tma_load_3d_pair(b_dst, &p.tmB[0], fb, kk * BK, x.n0 + arow, s);
                         }
+                    } else if (MODE == DH || MODE == DX || MODE == DXS || MODE == DW) {
+                        // MN-major B: four 64-column boxes of BK rows, 8 KB apart; DW's A likewise (two)
+                        mbar_expect_tx(fb, A_BYTES + B_BYTES);
+                        if (MODE == DH) {
+                            const bool shared = x.g >= p.E;
+                            const int e = shared ? x.g - p.E : x.g;
+                            tma_load_2d(a_dst, &p.tmA[shared ? 1 : 0], fb, kb * BK, x.row0 + x.m0);
+#pragma unroll
+                            for (int j = 0; j < 4; ++j)
+                                tma_load_3d(b_dst + j * 8192, &p.tmB[shared ? 1 : 0], fb, x.n0 + 64 * j, kb * BK, e);
+                        } else if (MODE == DX) {
+                            const int kbh = ceil_div(p.I, BK);
+                            const int hb = kb >= kbh ? 1 : 0;                  // 0: da . W1, 1: dg . W3
+                            tma_load_2d(a_dst, &p.tmA[0], fb, kb * BK, x.row0 + x.m0);
+#pragma unroll
+                            for (int j = 0; j < 4; ++j)
+                                tma_load_3d(b_dst + j * 8192, &p.tmB[hb], fb, x.n0 + 64 * j, (kb - hb * kbh) * BK, x.g);
+                        } else if (MODE == DXS) {
+                            const int kbs = 2 * ceil_div(p.Is, BK);
+                            if (kb < p.Ks * kbs) {
+                                const int sx = kb / kbs, kk = kb % kbs;
+                                const int hb = kk >= kbs / 2 ? 1 : 0;
+                                tma_load_3d(a_dst, &p.tmA[0], fb, kk * BK, x.m0, sx);
+#pragma unroll
+                                for (int j = 0; j < 4; ++j)
+                                    tma_load_3d(b_dst + j * 8192, &p.tmB[hb], fb, x.n0 + 64 * j, (kk - hb * (kbs / 2)) * BK, sx);
+                            } else {
+                                const int kr = kb - p.Ks * kbs;            // router: dz . C
+                                tma_load_2d(a_dst, &p.tmA[1], fb, kr * BK, x.m0);
+#pragma unroll
+                                for (int j = 0; j < 4; ++j)
+                                    tma_load_2d(b_dst + j * 8192, &p.tmB[2], fb, x.n0 + 64 * j, kr * BK);
+                            }
+                        } else {
+                            const int kr = x.row0 + kb * BK;
+#pragma unroll
+                            for (int j = 0; j < 2; ++j) {
+                                if (p.dw_a3d) tma_load_3d(a_dst + j * 8192, &p.tmA[0], fb, x.m0 + 64 * j, kb * BK, x.g);
+                                else tma_load_2d(a_dst + j * 8192, &p.tmA[0], fb, x.m0 + 64 * j, kr);
+                            }
+#pragma unroll
+                            for (int j = 0; j < 4; ++j) {
+                                if (p.dw_b3d) tma_load_3d(b_dst + j * 8192, &p.tmB[0], fb, x.n0 + 64 * j, kb * BK, x.g);
+                                else tma_load_2d(b_dst + j * 8192, &p.tmB[0], fb, x.n0 + 64 * j, kr);
+                            }
+                        }
                     } else {
                         mbar_expect_tx(fb, A_BYTES + B_BYTES);
                         if (MODE == GEMM1) {
@@ -802,7 +1081,10 @@ __global__ void __launch_bounds__(THREADS, 1) moe_tc_kernel(const __grid_constan
             for (int t = cta_slot; ok && t < ntiles; t += cta_slots) {
                 const Tile x = decode<MODE, PAIR>(p, t);
                 const bool q8tile = Q8 && (MODE == GEMM1 ? x.g < p.E : x.g >= 0);
-                const uint32_t idesc_t = q8tile ? (PAIR ? idesc_e4m3_pair(p.n_mma) : idesc_e4m3(p.n_mma)) : idesc;
+                constexpr bool B_MN = MODE == DH || MODE == DX || MODE == DXS || MODE == DW;
+                constexpr bool A_MN = MODE == DW;
+                const uint32_t idesc_t = q8tile ? (PAIR ? idesc_e4m3_pair(p.n_mma) : idesc_e4m3(p.n_mma))
+                                                : idesc | (B_MN ? IDESC_B_MN : 0u) | (A_MN ? IDESC_A_MN : 0u);
                 if (!mbar_wait(tempty_bar(acc), acc_phase ^ 1u, abort_flag, p.err)) break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + (uint32_t)(acc * ACC_COLS);
@@ -812,7 +1094,8 @@ __global__ void __launch_bounds__(THREADS, 1) moe_tc_kernel(const __grid_constan
                     const uint32_t a_addr = sA + stage * A_BYTES, b_addr = sB + stage * B_BYTES;
 #pragma unroll
                     for (int k = 0; k < BK / 16; ++k) {
-                        const uint64_t ad = sw128_desc(a_addr + k * 32), bd = sw128_desc(b_addr + k * 32);
+                        const uint64_t ad = A_MN ? mn_sw128_desc(a_addr + k * 2048) : sw128_desc(a_addr + k * 32);
+                        const uint64_t bd = B_MN ? mn_sw128_desc(b_addr + k * 2048) : sw128_desc(b_addr + k * 32);
                         const uint32_t accum = (kb > 0 || k > 0) ? 1u : 0u;
                         if (PAIR && q8tile) mma_e4m3_pair(d_tmem, ad, bd, idesc_t, accum);
                         else if (PAIR) mma_bf16_pair(d_tmem, ad, bd, idesc_t, accum);
@@ -855,6 +1138,12 @@ __global__ void __launch_bounds__(THREADS, 1) moe_tc_kernel(const __grid_constan
             } else if (MODE == GEMM2R) {
                 if (x.g >= 0) epilogue_gemm2r<Q8>(p, x, tacc, row, half);
                 else epilogue_gemm2s(p, x, tacc, row, half);
+            } else if (MODE == DH) {
+                epilogue_dh(p, x, tacc, row, half);
+            } else if (MODE == DX) {
+                epilogue_dx(p, x, tacc, row, half);
+            } else if (MODE == DW) {
+                epilogue_dw(p, x, tacc, row, half);
             } else {
                 epilogue_gemm2s(p, x, tacc, row, half);
             }
@@ -1051,10 +1340,14 @@ cudaError_t launch_tc_router(const Dims& D, const void* x, const void* centroids
 
 cudaError_t launch_tc_gemm1(const Dims& D, const void* x, const void* x_perm, const int32_t* offsets,
                             const int32_t* tile_start1, const FfnWeights& R, const FfnWeights& Sh, void* h_r, void* h_s,
-                            int g_begin, int g_end, uint32_t* err, cudaStream_t stream) {
+                            int g_begin, int g_end, uint32_t* err, cudaStream_t stream, const SavedAG* save) {
     using namespace tc;
     if (D.T == 0 || g_end <= g_begin) return cudaSuccess;
     Params p = base_params(D, err);
+    if (save) {
+        p.a_out = (__nv_bfloat16*)save->a; p.g_out = (__nv_bfloat16*)save->g;
+        p.as_out = (__nv_bfloat16*)save->as; p.gs_out = (__nv_bfloat16*)save->gs;
+    }
     p.tile_start = tile_start1;
     p.offsets = offsets;
     p.g_begin = g_begin;
@@ -1184,6 +1477,101 @@ cudaError_t launch_tc_gemm2_routed_q8(const Dims& D, const int32_t* offsets, con
     if (!ok) return cudaErrorInvalidValue;
     return pairs ? launch<GEMM2R, 8, true, true>(p, num_sms(), stream)
                  : launch<GEMM2R, 8, false, true>(p, num_sms(), stream);
+}
+
+// ------------------------------------------------------------------------------ backward
+// fp32 router logits z = x . C^T [T][N_m] (the split-K router's partial-logit mode with one split)
+cudaError_t launch_router_logits(const Dims& D, const void* x, const void* centroids, float* z, uint32_t* err,
+                                 cudaStream_t stream) {
+    using namespace tc;
+    if (D.T == 0) return cudaSuccess;
+    if (!tc_router_supported(D)) return cudaErrorInvalidValue;
+    Params p = base_params(D, err);
+    p.n_mma = D.E;
+    p.partial = z;
+    p.kb_per_split = ceil_div(D.d, BK);
+    if (!make_map(&p.tmA[0], x, D.d, D.T, 1, BK, BM, false)) return cudaErrorInvalidValue;
+    if (!make_map(&p.tmB[0], centroids, D.d, D.E, 1, BK, D.E, false)) return cudaErrorInvalidValue;
+    return launch<ROUTERP, 8>(p, ceil_div(D.T, BM), stream);
+}
+
+cudaError_t launch_tc_dh(const Dims& D, const BwdBufs& B, const FfnWeights& R, const FfnWeights& Sh, const void* dout,
+                         uint32_t* err, cudaStream_t stream) {
+    using namespace tc;
+    if (D.T == 0) return cudaSuccess;
+    Params p = base_params(D, err);
+    p.tile_start = B.ts_dh;
+    p.offsets = B.offsets;
+    p.offs_pad = B.offs_pad;
+    p.sorted_gate = B.sorted_gate;
+    p.a_sv = (const __nv_bfloat16*)B.a_sv; p.g_sv = (const __nv_bfloat16*)B.g_sv;
+    p.as_sv = (const __nv_bfloat16*)B.as_sv; p.gs_sv = (const __nv_bfloat16*)B.gs_sv;
+    p.dag = (__nv_bfloat16*)B.dag; p.hg = (__nv_bfloat16*)B.hg;
+    p.dag_s = (__nv_bfloat16*)B.dag_s; p.hg_s = (__nv_bfloat16*)B.hg_s;
+    p.dgate_part = B.dgate_part;
+    p.n_parts = 2 * ceil_div(D.I, 256);
+    bool ok = make_map(&p.tmA[0], B.dout_pad, D.d, (uint64_t)B.S_pad, 1, BK, BM, false);
+    ok &= make_map(&p.tmB[0], R.w2, D.I, D.d, D.E, 64, BK, true);
+    if (D.Ks > 0) {
+        ok &= make_map(&p.tmA[1], dout, D.d, D.T, 1, BK, BM, false);
+        ok &= make_map(&p.tmB[1], Sh.w2, D.Is, D.d, D.Ks, 64, BK, true);
+    }
+    if (!ok) return cudaErrorInvalidValue;
+    return launch<DH, 8>(p, num_sms(), stream);
+}
+
+cudaError_t launch_tc_dx(const Dims& D, const BwdBufs& B, const FfnWeights& R, uint32_t* err, cudaStream_t stream) {
+    using namespace tc;
+    if (D.T == 0) return cudaSuccess;
+    Params p = base_params(D, err);
+    p.tile_start = B.ts_dx;
+    p.offsets = B.offsets;
+    p.offs_pad = B.offs_pad;
+    p.dx_slot = (__nv_bfloat16*)B.dx_slot;
+    bool ok = make_map(&p.tmA[0], B.dag, 2 * (uint64_t)D.I, (uint64_t)B.S_pad, 1, BK, BM, false);
+    ok &= make_map(&p.tmB[0], R.w1, D.d, D.I, D.E, 64, BK, true);
+    ok &= make_map(&p.tmB[1], R.w3, D.d, D.I, D.E, 64, BK, true);
+    if (!ok) return cudaErrorInvalidValue;
+    return launch<DX, 8>(p, num_sms(), stream);
+}
+
+cudaError_t launch_tc_dxs(const Dims& D, const BwdBufs& B, const FfnWeights& Sh, const void* centroids, uint32_t* err,
+                          cudaStream_t stream) {
+    using namespace tc;
+    if (D.T == 0) return cudaSuccess;
+    Params p = base_params(D, err);
+    p.sout = B.base;
+    p.sb2 = nullptr;
+    bool ok = make_map(&p.tmA[1], B.dz_bf16, D.E, D.T, 1, BK, BM, false);
+    ok &= make_map(&p.tmB[2], centroids, D.d, D.E, 1, 64, BK, false);
+    if (D.Ks > 0) {
+        ok &= make_map(&p.tmA[0], B.dag_s, 2 * (uint64_t)D.Is, D.T, D.Ks, BK, BM, true);
+        ok &= make_map(&p.tmB[0], Sh.w1, D.d, D.Is, D.Ks, 64, BK, true);
+        ok &= make_map(&p.tmB[1], Sh.w3, D.d, D.Is, D.Ks, 64, BK, true);
+    } else {                                   // keep every map the kernel prefetches valid
+        ok &= make_map(&p.tmA[0], B.dz_bf16, D.E, D.T, 1, BK, BM, false);
+        ok &= make_map(&p.tmB[0], centroids, D.d, D.E, 1, 64, BK, false);
+    }
+    if (!ok) return cudaErrorInvalidValue;
+    return launch<DXS, 8>(p, ceil_div(D.T, BM) * ceil_div(D.d, 256), stream);
+}
+
+cudaError_t launch_tc_dw(const Dims& D, const DwSpec& w, uint32_t* err, cudaStream_t stream) {
+    using namespace tc;
+    if (w.groups <= 0 || w.M <= 0 || w.N <= 0) return cudaSuccess;
+    Params p = base_params(D, err);
+    p.dw_kind = w.kind;
+    p.dw_groups = w.groups; p.dw_M = w.M; p.dw_N = w.N;
+    p.dw_a3d = w.a3d; p.dw_b3d = w.b3d;
+    p.dw_rows = w.rows;
+    p.dw_K = w.K;
+    p.dw_out0 = (__nv_bfloat16*)w.out0; p.dw_out1 = (__nv_bfloat16*)w.out1;
+    p.dw_out_f32 = w.out_f32;
+    bool ok = make_map(&p.tmA[0], w.a, (uint64_t)w.M, (uint64_t)w.a_rows, w.a3d ? w.groups : 1, 64, BK, w.a3d);
+    ok &= make_map(&p.tmB[0], w.b, (uint64_t)w.N, (uint64_t)w.b_rows, w.b3d ? w.groups : 1, 64, BK, w.b3d);
+    if (!ok) return cudaErrorInvalidValue;
+    const long long tiles = (long long)w.groups * ceil_div(w.M, BM) * ceil_div(w.N, 256);
+    return launch<DW, 8>(p, (int)(tiles < num_sms() ? tiles : num_sms()), stream);
 }
 
 }  // namespace moe

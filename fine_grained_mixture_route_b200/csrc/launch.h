@@ -103,9 +103,15 @@ cudaError_t launch_tc_router(const Dims& D, const void* x, const void* centroids
 cudaError_t launch_router_finish(const Dims& D, const float* partial, int nsplit, const float* bias, int32_t* idx,
                                  float* gate, cudaStream_t stream);
 // GEMM1 + SwiGLU over groups [g_begin, g_end): A rows from x_perm (routed) or x (shared).
+// Pre-activations a = x W1^T + b1 and g = x W3^T + b3 stored by GEMM1 for the backward pass
+// (bf16): routed [T*N_r][I] in grouped order, shared [K_s][T][I_s].
+struct SavedAG {
+    void *a, *g, *as, *gs;
+};
 cudaError_t launch_tc_gemm1(const Dims& D, const void* x, const void* x_perm, const int32_t* offsets,
                             const int32_t* tile_start1, const FfnWeights& routed, const FfnWeights& shared,
-                            void* h_r, void* h_s, int g_begin, int g_end, uint32_t* err, cudaStream_t stream);
+                            void* h_r, void* h_s, int g_begin, int g_end, uint32_t* err, cudaStream_t stream,
+                            const SavedAG* save = nullptr);
 // routed GEMM2 with the gate (and b2) applied in the epilogue -> y_sorted; when shared and
 // sout are given, the shared experts' GEMM2 tiles (-> fp32 sout, their b2 added) follow the
 // routed tiles in the same launch.
@@ -131,5 +137,58 @@ cudaError_t launch_tc_gemm2_routed_q8(const Dims& D, const int32_t* offsets, con
                                       const float* sorted_gate, const FfnWeights& R, const void* h8,
                                       const float* hs, void* y_sorted, const FfnWeights* Sh, const void* h_s,
                                       float* sout, uint32_t* err, cudaStream_t stream);
+
+// ---- backward ----------------------------------------------------------------------
+// Buffers of one backward call.  Routed rows of the weight-gradient operands (dout_pad, x_pad,
+// dag, hg) are grouped by expert in 64-row-padded groups starting at offs_pad[e] (pad rows zero).
+struct BwdBufs {
+    const int32_t *offsets, *offs_pad, *ts_dh, *ts_dx;
+    const float* sorted_gate;
+    long long S_pad;
+    const void *a_sv, *g_sv, *as_sv, *gs_sv;     // saved pre-activations (forward for training)
+    void *dout_pad, *x_pad;                      // [S_pad][d]
+    void *dag, *hg;                              // [S_pad][2I], [S_pad][I]
+    void *dag_s, *hg_s;                          // [K_s][T][2I_s], [K_s][T][I_s]
+    float* dgate_part;                           // [S][2 * ceil(I / 256)]
+    void* dx_slot;                               // [S][d]
+    void* dz_bf16;                               // [T][N_m]
+    float* base;                                 // [T][d] fp32: shared experts' dx + router dx
+};
+// One weight-gradient GEMM: per group, out[M][N] = A^T B over the group's rows (K), with A
+// [rows][M] and B [rows][N] row-major (MN-major operands).  rows: group row starts [groups+1]
+// into 2-D operands, or null with K rows per group (3-D operands index the group, 2-D ones are
+// shared by all groups).  kind 0: out0 [groups][M][N]; 1: rows < M/2 -> out0, the rest -> out1
+// (each [groups][M/2][N]); 2: out_f32 [groups][M][N].
+struct DwSpec {
+    int kind, groups, M, N;
+    const void* a; long long a_rows; int a3d;
+    const void* b; long long b_rows; int b3d;
+    const int32_t* rows; int K;
+    void *out0, *out1;
+    float* out_f32;
+};
+cudaError_t launch_router_logits(const Dims& D, const void* x, const void* centroids, float* z, uint32_t* err,
+                                 cudaStream_t stream);
+cudaError_t launch_tc_dh(const Dims& D, const BwdBufs& B, const FfnWeights& R, const FfnWeights& Sh, const void* dout,
+                         uint32_t* err, cudaStream_t stream);
+cudaError_t launch_tc_dx(const Dims& D, const BwdBufs& B, const FfnWeights& R, uint32_t* err, cudaStream_t stream);
+cudaError_t launch_tc_dxs(const Dims& D, const BwdBufs& B, const FfnWeights& Sh, const void* centroids, uint32_t* err,
+                          cudaStream_t stream);
+cudaError_t launch_tc_dw(const Dims& D, const DwSpec& w, uint32_t* err, cudaStream_t stream);
+// offs_pad[E+1] (64-row-padded group starts), ts_dh[E+Ks+1], ts_dx[E+1] from the grouping offsets
+cudaError_t launch_plan_bwd(const Dims& D, const int32_t* offsets, int32_t* offs_pad, int32_t* ts_dh, int32_t* ts_dx,
+                            cudaStream_t stream);
+// padded grouped rows of dout and x, the padded gate column, and b2dot[p] = <dout_t, b2_e> (b2 may be null)
+cudaError_t launch_bwd_gather(const Dims& D, const void* dout, const void* x, const void* b2, const int32_t* offsets,
+                              const int32_t* offs_pad, const int32_t* stok, const float* sgate, void* dout_pad,
+                              void* x_pad, float* gate_pad, float* b2dot, uint32_t* err, cudaStream_t stream);
+// gate gradients -> logit gradients dz [T][N_m] (fp32 and bf16); dgate_out [T][k] optional
+cudaError_t launch_router_bwd(const Dims& D, const float* z, const float* bias, const int32_t* idx,
+                              const int32_t* slot_of, const float* dgate_part, int n_parts, const float* b2dot,
+                              float* dz, void* dz_bf16, float* dgate_out, cudaStream_t stream);
+// grouped, weighted column sums (bias gradients); see backward.cu
+cudaError_t launch_colsum(bool src_f32, bool out_f32, const void* src, long long group_stride, int ld,
+                          const int32_t* starts, int n_rows, const float* w, int groups, int W, int split, void* out0,
+                          void* out1, cudaStream_t stream);
 
 }  // namespace moe

@@ -52,6 +52,66 @@ Layout layout(const Dims& D) {
     return L;
 }
 
+// Training context: what moe_layer_forward_train keeps for moe_layer_backward.
+struct CtxLayout {
+    size_t idx, gate, counts, offsets, stok, sgate, slot_of, a, g, as, gs, total;
+};
+CtxLayout ctx_layout(const Dims& D) {
+    CtxLayout C;
+    const size_t S = (size_t)D.slots();
+    size_t o = 0;
+    C.idx = o; o += al(S * 4);
+    C.gate = o; o += al(S * 4);
+    C.counts = o; o += al((size_t)D.E * 4);
+    C.offsets = o; o += al((size_t)(D.E + 1) * 4);
+    C.stok = o; o += al(S * 4);
+    C.sgate = o; o += al(S * 4);
+    C.slot_of = o; o += al(S * 4);
+    C.a = o; o += al(S * D.I * 2);
+    C.g = o; o += al(S * D.I * 2);
+    C.as = o; o += al((size_t)D.Ks * D.T * (D.Ks ? D.Is : 0) * 2);
+    C.gs = o; o += al((size_t)D.Ks * D.T * (D.Ks ? D.Is : 0) * 2);
+    C.total = o;
+    return C;
+}
+
+// Backward workspace.
+struct BwdLayout {
+    size_t err, offs_pad, ts_dh, ts_dx, dout_pad, x_pad, gate_pad, b2dot, z, dgate_part, dag, hg, dag_s, hg_s, dz,
+        dz_bf16, dx_slot, base, total;
+    long long S_pad_max;
+    int n_parts;
+};
+BwdLayout bwd_layout(const Dims& D) {
+    BwdLayout B;
+    const size_t S = (size_t)D.slots();
+    B.S_pad_max = (long long)S + 64LL * D.E;
+    const size_t Sp = (size_t)B.S_pad_max;
+    const size_t Is = D.Ks ? D.Is : 0;
+    B.n_parts = 2 * ((D.I + 255) / 256);
+    size_t o = 0;
+    B.err = o; o += 256;
+    B.offs_pad = o; o += al((size_t)(D.E + 1) * 4);
+    B.ts_dh = o; o += al((size_t)(D.E + D.Ks + 1) * 4);
+    B.ts_dx = o; o += al((size_t)(D.E + 1) * 4);
+    B.dout_pad = o; o += al(Sp * D.d * 2);
+    B.x_pad = o; o += al(Sp * D.d * 2);
+    B.gate_pad = o; o += al(Sp * 4);
+    B.b2dot = o; o += al(S * 4);
+    B.z = o; o += al((size_t)D.T * D.E * 4);
+    B.dgate_part = o; o += al(S * B.n_parts * 4);
+    B.dag = o; o += al(Sp * 2 * D.I * 2);
+    B.hg = o; o += al(Sp * D.I * 2);
+    B.dag_s = o; o += al((size_t)D.Ks * D.T * 2 * Is * 2);
+    B.hg_s = o; o += al((size_t)D.Ks * D.T * Is * 2);
+    B.dz = o; o += al((size_t)D.T * D.E * 4);
+    B.dz_bf16 = o; o += al((size_t)D.T * D.E * 2);
+    B.dx_slot = o; o += al(S * D.d * 2);
+    B.base = o; o += al((size_t)D.T * D.d * 4);
+    B.total = o;
+    return B;
+}
+
 moe_status_t to_dims(const moe_shape_t* s, Dims* D) {
     if (!s) return MOE_ERR_INVALID_ARG;
     if (s->dtype != MOE_F32 && s->dtype != MOE_BF16) return MOE_ERR_INVALID_ARG;
@@ -92,6 +152,14 @@ moe_status_t check_weights(const Dims& D, const moe_ffn_weights_t* w, bool e4m3 
     const bool sc = w->s1 && w->s3 && w->s2;
     const bool nosc = !w->s1 && !w->s3 && !w->s2;
     if (e4m3 ? !sc : !nosc) return MOE_ERR_INVALID_ARG;
+    return MOE_OK;
+}
+
+// Layers the training path (forward_train + backward) handles: bf16, native routed weights, a
+// tensor-core router (it recomputes the logits), and d, inter, inter_shared multiples of 64.
+moe_status_t check_train(const Dims& D) {
+    if (!D.bf16 || D.q8 || !tc_router_supported(D)) return MOE_ERR_UNSUPPORTED;
+    if (D.d % 64 || D.I % 64 || (D.Ks > 0 && D.Is % 64)) return MOE_ERR_UNSUPPORTED;
     return MOE_OK;
 }
 
@@ -355,7 +423,8 @@ namespace {
 moe_status_t layer_forward_impl(const moe_shape_t* shape, const void* x, const void* centroids,
                                 const float* router_bias, const moe_ffn_weights_t* routed, const moe_ffn_weights_t* shared, void* out,
                                 int32_t* topk_idx_out, float* topk_gate_out, int32_t* counts_out, void* ws,
-                                size_t ws_bytes, cudaStream_t st, cudaEvent_t const* ev) {
+                                size_t ws_bytes, cudaStream_t st, cudaEvent_t const* ev, void* ctx = nullptr,
+                                size_t ctx_bytes = 0) {
     Dims D;
     MOE_TRY(to_dims(shape, &D));
     if (!x || !centroids || !out) return MOE_ERR_INVALID_ARG;
@@ -363,6 +432,10 @@ moe_status_t layer_forward_impl(const moe_shape_t* shape, const void* x, const v
     if (D.Ks > 0) MOE_TRY(check_weights(D, shared));
     else if (shared) return MOE_ERR_INVALID_ARG;
     MOE_TRY(check_ws(D, ws, ws_bytes));
+    if (ctx) {
+        MOE_TRY(check_train(D));
+        if (ctx_bytes < ctx_layout(D).total || ((uintptr_t)ctx & 15u)) return MOE_ERR_WORKSPACE;
+    }
     if (D.T == 0) return MOE_OK;
     MOE_TRY(check_device());
     cudaGetLastError();
@@ -375,6 +448,14 @@ moe_status_t layer_forward_impl(const moe_shape_t* shape, const void* x, const v
     int32_t* stok = at<int32_t>(ws, L.stok);
     float* sgate = at<float>(ws, L.sgate);
     int32_t* slot_of = at<int32_t>(ws, L.slot_of);
+    SavedAG save = {nullptr, nullptr, nullptr, nullptr};
+    if (ctx) {          // forward for training: routing, grouping and pre-activations go to ctx
+        const CtxLayout C = ctx_layout(D);
+        idx = at<int32_t>(ctx, C.idx); gate = at<float>(ctx, C.gate); counts = at<int32_t>(ctx, C.counts);
+        offsets = at<int32_t>(ctx, C.offsets); stok = at<int32_t>(ctx, C.stok); sgate = at<float>(ctx, C.sgate);
+        slot_of = at<int32_t>(ctx, C.slot_of);
+        save = {at<void>(ctx, C.a), at<void>(ctx, C.g), at<void>(ctx, C.as), at<void>(ctx, C.gs)};
+    }
     void* y = at<void>(ws, L.y);
     void* hr = at<void>(ws, L.hr);
     void* hs = at<void>(ws, L.hs);
@@ -409,7 +490,7 @@ moe_status_t layer_forward_impl(const moe_shape_t* shape, const void* x, const v
         void* xp = at<void>(ws, L.xperm);
         MOE_CUDA(launch_gather(D, x, stok, xp, err, st));
         if (!mark(4)) return MOE_ERR_CUDA;
-        MOE_CUDA(launch_tc_gemm1(D, x, xp, offsets, ts1, R, Sh, hr, hs, 0, D.E + D.Ks, err, st));
+        MOE_CUDA(launch_tc_gemm1(D, x, xp, offsets, ts1, R, Sh, hr, hs, 0, D.E + D.Ks, err, st, ctx ? &save : nullptr));
         if (!mark(5)) return MOE_ERR_CUDA;
         float* sout = D.Ks > 0 ? at<float>(ws, L.sout) : nullptr;
         MOE_CUDA(launch_tc_gemm2_routed(D, offsets, ts2, sgate, R, hr, y, D.Ks > 0 ? &Sh : nullptr, hs, sout, err, st));
@@ -425,6 +506,106 @@ moe_status_t layer_forward_impl(const moe_shape_t* shape, const void* x, const v
         else MOE_CUDA(launch_combine(D, y, slot_of, nullptr, out, err, st));
     }
     if (!mark(7)) return MOE_ERR_CUDA;
+    return MOE_OK;
+}
+
+// Backward of the layer (moe_layer_backward).
+moe_status_t layer_backward_impl(const moe_shape_t* shape, const void* x, const void* centroids,
+                                 const float* router_bias, const moe_ffn_weights_t* routed,
+                                 const moe_ffn_weights_t* shared, const void* dout, const void* ctx, size_t ctx_bytes,
+                                 void* dx, float* dcentroids, float* drouter_bias, const moe_ffn_grads_t* groutes,
+                                 const moe_ffn_grads_t* gshared, void* ws, size_t ws_bytes, cudaStream_t st) {
+    Dims D;
+    MOE_TRY(to_dims(shape, &D));
+    MOE_TRY(check_train(D));
+    if (!x || !centroids || !dout || !ctx || !dx || !dcentroids) return MOE_ERR_INVALID_ARG;
+    MOE_TRY(check_weights(D, routed));
+    if (D.Ks > 0) MOE_TRY(check_weights(D, shared));
+    else if (shared || gshared) return MOE_ERR_INVALID_ARG;
+    auto check_grads = [&](const moe_ffn_grads_t* g) -> bool {
+        if (!g || !g->w1 || !g->w3 || !g->w2) return false;
+        const bool b = g->b1 && g->b3 && g->b2, none = !g->b1 && !g->b3 && !g->b2;
+        return D.bias ? b : none;
+    };
+    if (!check_grads(groutes) || (D.Ks > 0 && !check_grads(gshared))) return MOE_ERR_INVALID_ARG;
+    if (drouter_bias && (!router_bias || D.gate_mode == MOE_GATE_SIGMOID_BIAS)) return MOE_ERR_INVALID_ARG;
+    const CtxLayout C = ctx_layout(D);
+    if (ctx_bytes < C.total || ((uintptr_t)ctx & 15u)) return MOE_ERR_WORKSPACE;
+    const BwdLayout L = bwd_layout(D);
+    if (!ws || ws_bytes < L.total || ((uintptr_t)ws & 15u)) return MOE_ERR_WORKSPACE;
+    if (D.T == 0) return MOE_OK;
+    MOE_TRY(check_device());
+    cudaGetLastError();
+    uint32_t* err = at<uint32_t>(ws, L.err);
+    auto cp = [&](size_t off) { return const_cast<char*>(static_cast<const char*>(ctx)) + off; };
+    const int32_t* idx = reinterpret_cast<const int32_t*>(cp(C.idx));
+    const int32_t* offsets = reinterpret_cast<const int32_t*>(cp(C.offsets));
+    const int32_t* stok = reinterpret_cast<const int32_t*>(cp(C.stok));
+    const float* sgate = reinterpret_cast<const float*>(cp(C.sgate));
+    const int32_t* slot_of = reinterpret_cast<const int32_t*>(cp(C.slot_of));
+    const FfnWeights R = to_ffn(routed), Sh = to_ffn(shared);
+    BwdBufs B;
+    B.offsets = offsets;
+    B.offs_pad = at<int32_t>(ws, L.offs_pad);
+    B.ts_dh = at<int32_t>(ws, L.ts_dh);
+    B.ts_dx = at<int32_t>(ws, L.ts_dx);
+    B.sorted_gate = sgate;
+    B.S_pad = L.S_pad_max;
+    B.a_sv = cp(C.a); B.g_sv = cp(C.g); B.as_sv = cp(C.as); B.gs_sv = cp(C.gs);
+    B.dout_pad = at<void>(ws, L.dout_pad); B.x_pad = at<void>(ws, L.x_pad);
+    B.dag = at<void>(ws, L.dag); B.hg = at<void>(ws, L.hg);
+    B.dag_s = at<void>(ws, L.dag_s); B.hg_s = at<void>(ws, L.hg_s);
+    B.dgate_part = at<float>(ws, L.dgate_part);
+    B.dx_slot = at<void>(ws, L.dx_slot);
+    B.dz_bf16 = at<void>(ws, L.dz_bf16);
+    B.base = at<float>(ws, L.base);
+    float* gate_pad = at<float>(ws, L.gate_pad);
+    float* b2dot = D.bias ? at<float>(ws, L.b2dot) : nullptr;
+    float* z = at<float>(ws, L.z);
+    float* dz = at<float>(ws, L.dz);
+
+    MOE_CUDA(launch_plan_bwd(D, offsets, const_cast<int32_t*>(B.offs_pad), const_cast<int32_t*>(B.ts_dh),
+                             const_cast<int32_t*>(B.ts_dx), st));
+    MOE_CUDA(launch_bwd_gather(D, dout, x, R.b2, offsets, B.offs_pad, stok, sgate, B.dout_pad, B.x_pad, gate_pad, b2dot,
+                               err, st));
+    MOE_CUDA(launch_router_logits(D, x, centroids, z, err, st));
+    MOE_CUDA(launch_tc_dh(D, B, R, Sh, dout, err, st));
+    MOE_CUDA(launch_router_bwd(D, z, router_bias, idx, slot_of, B.dgate_part, L.n_parts, b2dot, dz, B.dz_bf16, nullptr,
+                               st));
+    MOE_CUDA(launch_tc_dx(D, B, R, err, st));
+    MOE_CUDA(launch_tc_dxs(D, B, Sh, centroids, err, st));
+    MOE_CUDA(launch_combine(D, B.dx_slot, slot_of, B.base, dx, err, st));
+    // weight gradients
+    const long long T = D.T;
+    DwSpec w2 = {0, D.E, D.d, D.I, B.dout_pad, L.S_pad_max, 0, B.hg, L.S_pad_max, 0, B.offs_pad, 0,
+                 groutes->w2, nullptr, nullptr};
+    MOE_CUDA(launch_tc_dw(D, w2, err, st));
+    DwSpec w13 = {1, D.E, 2 * D.I, D.d, B.dag, L.S_pad_max, 0, B.x_pad, L.S_pad_max, 0, B.offs_pad, 0,
+                  groutes->w1, groutes->w3, nullptr};
+    MOE_CUDA(launch_tc_dw(D, w13, err, st));
+    if (D.Ks > 0) {
+        DwSpec s2 = {0, D.Ks, D.d, D.Is, dout, T, 0, B.hg_s, T, 1, nullptr, D.T, gshared->w2, nullptr, nullptr};
+        MOE_CUDA(launch_tc_dw(D, s2, err, st));
+        DwSpec s13 = {1, D.Ks, 2 * D.Is, D.d, B.dag_s, T, 1, x, T, 0, nullptr, D.T, gshared->w1, gshared->w3, nullptr};
+        MOE_CUDA(launch_tc_dw(D, s13, err, st));
+    }
+    DwSpec dc = {2, 1, D.E, D.d, B.dz_bf16, T, 0, x, T, 0, nullptr, D.T, nullptr, nullptr, dcentroids};
+    MOE_CUDA(launch_tc_dw(D, dc, err, st));
+    // bias gradients (deterministic column sums)
+    if (D.bias) {
+        MOE_CUDA(launch_colsum(false, false, B.dout_pad, 0, D.d, B.offs_pad, 0, gate_pad, D.E, D.d, D.d, groutes->b2,
+                               nullptr, st));
+        MOE_CUDA(launch_colsum(false, false, B.dag, 0, 2 * D.I, B.offs_pad, 0, nullptr, D.E, 2 * D.I, D.I, groutes->b1,
+                               groutes->b3, st));
+        if (D.Ks > 0) {
+            MOE_CUDA(launch_colsum(false, false, dout, 0, D.d, nullptr, D.T, nullptr, D.Ks, D.d, D.d, gshared->b2,
+                                   nullptr, st));
+            MOE_CUDA(launch_colsum(false, false, B.dag_s, (long long)D.T * 2 * D.Is, 2 * D.Is, nullptr, D.T, nullptr,
+                                   D.Ks, 2 * D.Is, D.Is, gshared->b1, gshared->b3, st));
+        }
+    }
+    if (drouter_bias)
+        MOE_CUDA(launch_colsum(true, true, dz, 0, D.E, nullptr, D.T, nullptr, 1, D.E, D.E, drouter_bias, nullptr, st));
     return MOE_OK;
 }
 
@@ -452,6 +633,37 @@ MOE_EXPORT moe_status_t moe_layer_forward_timed(const moe_shape_t* shape, const 
     return layer_forward_impl(shape, x, centroids, router_bias, routed, shared, out, topk_idx_out, topk_gate_out,
                               counts_out, ws, ws_bytes, (cudaStream_t)stream,
                               reinterpret_cast<cudaEvent_t const*>(stage_events));
+}
+
+MOE_EXPORT size_t moe_train_ctx_bytes(const moe_shape_t* shape) {
+    Dims D;
+    if (to_dims(shape, &D) != MOE_OK || check_train(D) != MOE_OK) return 0;
+    return ctx_layout(D).total;
+}
+
+MOE_EXPORT size_t moe_backward_workspace_bytes(const moe_shape_t* shape) {
+    Dims D;
+    if (to_dims(shape, &D) != MOE_OK || check_train(D) != MOE_OK) return 0;
+    return bwd_layout(D).total;
+}
+
+MOE_EXPORT moe_status_t moe_layer_forward_train(const moe_shape_t* shape, const void* x, const void* centroids,
+                                                const float* router_bias, const moe_ffn_weights_t* routed,
+                                                const moe_ffn_weights_t* shared, void* out, void* ctx, size_t ctx_bytes,
+                                                void* ws, size_t ws_bytes, moe_stream_t stream) {
+    if (!ctx) return MOE_ERR_INVALID_ARG;
+    return layer_forward_impl(shape, x, centroids, router_bias, routed, shared, out, nullptr, nullptr, nullptr, ws,
+                              ws_bytes, (cudaStream_t)stream, nullptr, ctx, ctx_bytes);
+}
+
+MOE_EXPORT moe_status_t moe_layer_backward(const moe_shape_t* shape, const void* x, const void* centroids,
+                                           const float* router_bias, const moe_ffn_weights_t* routed,
+                                           const moe_ffn_weights_t* shared, const void* dout, const void* ctx,
+                                           size_t ctx_bytes, void* dx, float* dcentroids, float* drouter_bias,
+                                           const moe_ffn_grads_t* routed_grads, const moe_ffn_grads_t* shared_grads,
+                                           void* ws, size_t ws_bytes, moe_stream_t stream) {
+    return layer_backward_impl(shape, x, centroids, router_bias, routed, shared, dout, ctx, ctx_bytes, dx, dcentroids,
+                               drouter_bias, routed_grads, shared_grads, ws, ws_bytes, (cudaStream_t)stream);
 }
 
 }  // extern "C"

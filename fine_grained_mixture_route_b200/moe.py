@@ -21,7 +21,8 @@ FMT_NATIVE, FMT_E4M3 = 0, 1        # storage of the routed experts' weights (moe
 
 EXPORTED = ("moe_workspace_bytes", "moe_layer_launches", "moe_status_string", "moe_version", "moe_check_device_error", "moe_ws_init",
             "moe_route", "moe_permute", "moe_expert_ffn", "moe_combine", "moe_layer_forward",
-            "moe_layer_forward_timed", "moe_permute_no_alloc", "moe_quantize_rows_e4m3")
+            "moe_layer_forward_timed", "moe_permute_no_alloc", "moe_quantize_rows_e4m3", "moe_train_ctx_bytes",
+            "moe_backward_workspace_bytes", "moe_layer_forward_train", "moe_layer_backward")
 NUM_STAGES = 7
 STAGE_NAMES = ("router", "permute", "plan", "gather", "gemm1_swiglu", "gemm2", "combine")
 
@@ -34,6 +35,10 @@ class MoeShape(ctypes.Structure):
 
 class MoeWeights(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in ("w1", "b1", "w3", "b3", "w2", "b2", "s1", "s3", "s2")]
+
+
+class MoeGrads(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in ("w1", "b1", "w3", "b3", "w2", "b2")]
 
 
 class MoeError(RuntimeError):
@@ -75,8 +80,16 @@ def _lib():
                                                 ctypes.POINTER(ctypes.c_void_p), ctypes.c_int32]
         lib.moe_quantize_rows_e4m3.argtypes = [vp, i32p, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, vp, f32p,
                                                vp, sz, vp]
+        gp = ctypes.POINTER(MoeGrads)
+        lib.moe_train_ctx_bytes.argtypes = [sh]
+        lib.moe_train_ctx_bytes.restype = sz
+        lib.moe_backward_workspace_bytes.argtypes = [sh]
+        lib.moe_backward_workspace_bytes.restype = sz
+        lib.moe_layer_forward_train.argtypes = [sh, vp, vp, f32p, wp, wp, vp, vp, sz, vp, sz, vp]
+        lib.moe_layer_backward.argtypes = [sh, vp, vp, f32p, wp, wp, vp, vp, sz, vp, f32p, f32p, gp, gp, vp, sz, vp]
         for n in ("moe_check_device_error", "moe_ws_init", "moe_route", "moe_permute", "moe_expert_ffn",
-                  "moe_combine", "moe_layer_forward", "moe_layer_forward_timed", "moe_quantize_rows_e4m3"):
+                  "moe_combine", "moe_layer_forward", "moe_layer_forward_timed", "moe_quantize_rows_e4m3",
+                  "moe_layer_forward_train", "moe_layer_backward"):
             getattr(lib, n).restype = ctypes.c_int
         _LIB = lib
     return _LIB
@@ -234,6 +247,61 @@ def quantize_rows_e4m3(src: torch.Tensor, ws: torch.Tensor, row_of: Optional[tor
                                          _ptr(scales), _ptr(ws), ws.numel(), _stream(stream)),
            "moe_quantize_rows_e4m3")
     return codes, scales
+
+
+def train_ctx_bytes(shape: MoeShape) -> int:
+    return int(_lib().moe_train_ctx_bytes(ctypes.byref(shape)))
+
+
+def backward_workspace_bytes(shape: MoeShape) -> int:
+    return int(_lib().moe_backward_workspace_bytes(ctypes.byref(shape)))
+
+
+def new_train_buffers(shape: MoeShape, device="cuda"):
+    """(ctx, backward workspace) for moe_layer_forward_train / moe_layer_backward."""
+    nc, nb = train_ctx_bytes(shape), backward_workspace_bytes(shape)
+    if nc == 0 or nb == 0:
+        raise ValueError("layer shape not supported for training")
+    ctx = torch.empty(nc, dtype=torch.uint8, device=device)
+    wsb = torch.empty(nb, dtype=torch.uint8, device=device)
+    _check(_lib().moe_ws_init(_ptr(wsb), nb, _stream()), "moe_ws_init")
+    return ctx, wsb
+
+
+def layer_forward_train(shape: MoeShape, x, centroids, routed: Dict, shared: Optional[Dict], ws, ctx, out=None,
+                        stream=None, router_bias=None):
+    """moe_layer_forward plus the training context in ctx."""
+    out = torch.empty((shape.T, shape.d), dtype=x.dtype, device=x.device) if out is None else out
+    rw, sw = _weights(routed), _weights(shared)
+    _check(_lib().moe_layer_forward_train(ctypes.byref(shape), _ptr(x), _ptr(centroids), _bias_ptr(router_bias),
+                                          ctypes.byref(rw), None if sw is None else ctypes.byref(sw), _ptr(out),
+                                          _ptr(ctx), ctx.numel(), _ptr(ws), ws.numel(), _stream(stream)),
+           "moe_layer_forward_train")
+    return out
+
+
+def _grad_stack(w: Dict):
+    g = {k: (None if w.get(k) is None else torch.empty_like(w[k])) for k in ("w1", "b1", "w3", "b3", "w2", "b2")}
+    return g, MoeGrads(*(None if g[k] is None else g[k].data_ptr() for k in ("w1", "b1", "w3", "b3", "w2", "b2")))
+
+
+def layer_backward(shape: MoeShape, x, centroids, routed: Dict, shared: Optional[Dict], dout, ctx, ws_bwd,
+                   stream=None, router_bias=None, router_bias_grad: bool = False):
+    """moe_layer_backward: returns {dx, dcentroids, drouter_bias (or None), routed: {...}, shared:
+    {...} or None} with the gradient tensors allocated here."""
+    dx = torch.empty_like(x)
+    dc = torch.empty(centroids.shape, dtype=torch.float32, device=x.device)
+    db = torch.empty(centroids.shape[0], dtype=torch.float32, device=x.device) if router_bias_grad else None
+    gr, gr_c = _grad_stack(routed)
+    gs, gs_c = _grad_stack(shared) if shared is not None else (None, None)
+    rw, sw = _weights(routed), _weights(shared)
+    _check(_lib().moe_layer_backward(ctypes.byref(shape), _ptr(x), _ptr(centroids), _bias_ptr(router_bias),
+                                     ctypes.byref(rw), None if sw is None else ctypes.byref(sw), _ptr(dout), _ptr(ctx),
+                                     ctx.numel(), _ptr(dx), _ptr(dc), _ptr(db), ctypes.byref(gr_c),
+                                     None if gs_c is None else ctypes.byref(gs_c), _ptr(ws_bwd), ws_bwd.numel(),
+                                     _stream(stream)),
+           "moe_layer_backward")
+    return {"dx": dx, "dcentroids": dc, "drouter_bias": db, "routed": gr, "shared": gs}
 
 
 def stage_events(stream=None):

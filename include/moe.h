@@ -250,6 +250,64 @@ moe_status_t moe_quantize_rows_e4m3(const void* src, const int32_t* row_of, int6
                                     moe_stream_t stream);
 
 /*
+ * Training: the forward that keeps what the backward needs, and the backward.
+ *
+ * The pages discuss the backward only through SonicMoE's kernels (the dH kernel, activation
+ * memory that does not grow with expert granularity: "DeepSeek做大→Mega MoE，Tri Dao团队加快→SonicMoE");
+ * the gradients here are the chain rule of the forward above.  Supported layers: MOE_BF16 with
+ * native routed weights, a tensor-core router (n_experts a multiple of 16, 16..256) and d, inter,
+ * inter_shared multiples of 64; other shapes give MOE_ERR_UNSUPPORTED.
+ *
+ * The training context (`ctx`, moe_train_ctx_bytes(shape) bytes, caller-owned, 16-byte aligned)
+ * holds the picks, gates, grouping and the pre-activations a = x W1^T + b1, g = x W3^T + b3 of
+ * every routed slot and shared expert (bf16; T*N_r*inter*4 + K_s*T*inter_shared*4 bytes) and
+ * nothing that grows with d*N_r: the expert outputs are not kept.  moe_layer_forward_train writes
+ * it (and out, exactly as moe_layer_forward); moe_layer_backward reads it.  Between the two the
+ * caller must not change x, the weights or ctx.
+ */
+typedef struct {
+    void* w1; /* [E, I, d], layer dtype */
+    void* b1; /* [E, I] or NULL (NULL iff has_bias == 0) */
+    void* w3; /* [E, I, d] */
+    void* b3; /* [E, I] or NULL */
+    void* w2; /* [E, d, I] */
+    void* b2; /* [E, d] or NULL */
+} moe_ffn_grads_t;
+
+/* Bytes of the training context / of the backward workspace for this shape (0 if the shape
+ * is invalid or not supported for training). */
+size_t moe_train_ctx_bytes(const moe_shape_t* shape);
+size_t moe_backward_workspace_bytes(const moe_shape_t* shape);
+
+/* moe_layer_forward, and in addition the training context in ctx.  ws as for moe_layer_forward. */
+moe_status_t moe_layer_forward_train(const moe_shape_t* shape, const void* x, const void* centroids,
+                                     const float* router_bias, const moe_ffn_weights_t* routed,
+                                     const moe_ffn_weights_t* shared, void* out, void* ctx, size_t ctx_bytes,
+                                     void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * Gradients of L = <out, dout> for the layer run by moe_layer_forward_train with the same
+ * arguments and ctx (the picks are held fixed; they carry no gradient):
+ *   dout [T, d] (layer dtype)  in
+ *   dx [T, d] (layer dtype)    out: through the routed experts, the shared experts and the router
+ *   dcentroids [N_m, d] fp32   out
+ *   drouter_bias [N_m] fp32    out, or NULL; must be NULL without a router bias and in gate mode
+ *                              MOE_GATE_SIGMOID_BIAS (there the bias only selects)
+ *   routed_grads, shared_grads out: weight and bias gradients in the layer dtype (all experts;
+ *                              an expert without tokens gets zeros); shared_grads NULL iff
+ *                              n_shared == 0
+ * Sums are fp32 on the tensor cores and in fixed order (deterministic); dx adds the routed terms
+ * in pick order to the shared and router terms.  ws: moe_backward_workspace_bytes(shape) bytes
+ * (its first 256 bytes are the error word, as for the other calls).
+ */
+moe_status_t moe_layer_backward(const moe_shape_t* shape, const void* x, const void* centroids,
+                                const float* router_bias, const moe_ffn_weights_t* routed,
+                                const moe_ffn_weights_t* shared, const void* dout, const void* ctx, size_t ctx_bytes,
+                                void* dx, float* dcentroids, float* drouter_bias,
+                                const moe_ffn_grads_t* routed_grads, const moe_ffn_grads_t* shared_grads,
+                                void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
  * moe_permute_no_alloc — the paper has no counterpart to this entry point; it exists for
  * callers of this library that cannot allocate device memory.  moe_permute needs scratch
  * space, which it takes from the caller's workspace.  A caller that cannot call cudaMalloc

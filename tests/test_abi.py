@@ -149,3 +149,40 @@ def test_quantize_rows_argument_errors(lib):
     assert q(fake, None, 10, 10, 16, fake, fake, None, 0, None) == moe.MOE_ERR_WORKSPACE
     assert q(None, None, 10, 10, 16, fake, fake, fake, 4096, None) == moe.MOE_ERR_INVALID_ARG
     assert q(fake, fake, 0, 10, 16, fake, fake, fake, 4096, None) == moe.MOE_OK                # no rows: no-op
+
+
+def test_training_entry_points_validate(lib):
+    fake = ctypes.c_void_p(1 << 40)
+    S = ctypes.byref
+    sh = _shape()
+    assert moe.train_ctx_bytes(sh) > 0 and moe.backward_workspace_bytes(sh) > 0
+    # ctx holds picks, grouping and the bf16 pre-activations a, g (routed and shared)
+    Sl, I, T = 256 * 8, 2048, 256
+    assert moe.train_ctx_bytes(sh) >= 2 * 2 * (Sl * I + T * 2048)
+    for unsupported in (dict(dtype=moe.MOE_F32), dict(routed_fmt=moe.FMT_E4M3), dict(n_experts=512, top_k=8),
+                        dict(n_experts=20, top_k=3), dict(d=7168 + 8), dict(inter=2048 + 16),
+                        dict(inter_shared=2048 + 32)):
+        assert moe.train_ctx_bytes(_shape(**unsupported)) == 0, unsupported
+        assert moe.backward_workspace_bytes(_shape(**unsupported)) == 0, unsupported
+    n, nb, nc = moe.workspace_bytes(sh), moe.backward_workspace_bytes(sh), moe.train_ctx_bytes(sh)
+    w = moe.MoeWeights(*([fake.value] * 6))
+    g = moe.MoeGrads(*([fake.value] * 6))
+    f = lib.moe_layer_forward_train
+    assert f(S(sh), fake, fake, None, S(w), S(w), fake, None, nc, fake, n, None) == moe.MOE_ERR_INVALID_ARG
+    assert f(S(sh), fake, fake, None, S(w), S(w), fake, fake, nc - 1, fake, n, None) == moe.MOE_ERR_WORKSPACE
+    assert f(S(_shape(dtype=moe.MOE_F32)), fake, fake, None, S(w), S(w), fake, fake, nc, fake, n, None) == \
+        moe.MOE_ERR_UNSUPPORTED
+    b = lib.moe_layer_backward
+    args = lambda **kw: [S(kw.get("sh", sh)), fake, fake, kw.get("rb", None), S(w), S(w), fake, fake,
+                         kw.get("nc", nc), fake, fake, kw.get("drb", None), S(kw.get("g", g)), S(g), fake,
+                         kw.get("nb", nb), None]
+    assert b(*args(nc=nc - 1)) == moe.MOE_ERR_WORKSPACE
+    assert b(*args(nb=nb - 1)) == moe.MOE_ERR_WORKSPACE
+    assert b(*args(drb=fake)) == moe.MOE_ERR_INVALID_ARG            # router-bias gradient without a bias
+    assert b(*args(g=moe.MoeGrads(fake.value, None, fake.value, fake.value, fake.value, fake.value))) == \
+        moe.MOE_ERR_INVALID_ARG                                      # bias gradient pointers must match has_bias
+    sh2 = _shape(gate_mode=2)
+    assert b(*args(sh=sh2, rb=fake, drb=fake, nc=moe.train_ctx_bytes(sh2), nb=moe.backward_workspace_bytes(sh2))) \
+        == moe.MOE_ERR_INVALID_ARG                                   # gate mode 2: the bias only selects
+    sh0 = _shape(T=0)
+    assert b(*args(sh=sh0, nc=moe.train_ctx_bytes(sh0), nb=moe.backward_workspace_bytes(sh0))) == moe.MOE_OK
