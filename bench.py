@@ -135,6 +135,32 @@ def stage_work(cfg: W.LayerConfig, touched: int, e4m3: bool = False):
     return w
 
 
+def bwd_stage_work(cfg: W.LayerConfig, touched: int):
+    """Algorithmic FLOPs and HBM bytes of each backward stage (moe_layer_backward_timed), counted
+    like stage_work: operands once at their storage size; every expert's weight gradient is
+    written (zeros for experts without tokens)."""
+    T, d, E, I, k, Ks, Is = cfg.T, cfg.d, cfg.n_experts, cfg.inter, cfg.top_k, cfg.n_shared, cfg.inter_shared
+    b = cfg.elem_bytes()
+    S = T * k
+    parts = 2 * math.ceil(I / 256)
+    bias = 1 if cfg.has_bias else 0
+    return {
+        "bwd_prep": (2.0 * T * d * E, 4 * S * d * b + T * d * b + E * d * b + T * E * 4 + S * 8),
+        "bwd_dh": (2.0 * S * d * I + 2.0 * Ks * T * d * Is,
+                   touched * d * I * b + Ks * d * Is * b + S * d * b + (T * d * b if Ks else 0)
+                   + 5 * S * I * b + 5 * Ks * T * Is * b + S * parts * 4),
+        "bwd_router": (0.0, T * E * 4 + S * parts * 4 + S * 4 + T * E * 6),
+        "bwd_dx": (4.0 * S * I * d + 4.0 * Ks * T * Is * d + 2.0 * T * E * d,
+                   2 * S * I * b + 2 * touched * I * d * b + 2 * Ks * Is * d * b + 2 * Ks * T * Is * b + T * E * b
+                   + E * d * b + 2 * S * d * b + 2 * T * d * 4 + T * d * b),
+        "bwd_dw2": (2.0 * S * d * I, S * d * b + S * I * b + E * d * I * b),
+        "bwd_dw13": (4.0 * S * I * d, 2 * S * I * b + S * d * b + 2 * E * I * d * b),
+        "bwd_shared_dc_bias": (6.0 * Ks * T * d * Is + 2.0 * T * E * d,
+                               3 * Ks * d * Is * b + Ks * (T * d * b + 3 * T * Is * b) + T * E * b + T * d * b
+                               + E * d * 4 + bias * (S * d * b + 2 * S * I * b + E * (2 * I + d) * b)),
+    }
+
+
 def layer_bytes(cfg: W.LayerConfig, touched: int, e4m3: bool = False) -> float:
     """Algorithmic bytes of the whole layer: weights of touched experts, shared experts,
     centroids, x in and out once (intermediates excluded: the method need not keep them)."""
@@ -469,6 +495,95 @@ def run_ours(args, cfg, rank, world, local_rank):
         print(json.dumps(line), flush=True)
 
 
+def run_train(args, cfg, rank, world, local_rank):
+    """--pass train: one step = moe_layer_forward_train + moe_layer_backward on the same batch
+    (dout synthetic, resident), per-stage events on both."""
+    from fine_grained_mixture_route_b200 import moe
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+    L = W.make_layer(cfg, dev, seed=0)
+    if rank > 0:
+        L["x"] = W.make_x(cfg, dev, seed=1000 + rank)
+    x, C, R, Sh = L["x"], L["centroids"], L["routed"], L["shared"]
+    shape = moe.shape_of(x, C, R, cfg.top_k, Sh, gate_mode=args.gate_mode)
+    ws = moe.new_workspace(shape, dev)
+    ctx, wsb = moe.new_train_buffers(shape, dev)
+    g = torch.Generator(device="cpu").manual_seed(W.seed_for(0, "x", 10**6))
+    dout = torch.randn(cfg.T, cfg.d, generator=g).to(cfg.dtype).to(dev)
+    out = torch.empty_like(x)
+    grads = moe.new_grads(x, C, R, Sh)
+    for _ in range(args.warmup):
+        moe.layer_forward_train(shape, x, C, R, Sh, ws, ctx, out=out)
+        moe.layer_backward(shape, x, C, R, Sh, dout, ctx, wsb, grads=grads)
+    moe.check_device_error(ws)
+    moe.check_device_error(wsb)
+    counts = torch.empty(cfg.n_experts, dtype=torch.int32, device=dev)
+    moe.layer_forward(shape, x, C, R, Sh, ws, counts=counts)
+    touched = int((counts > 0).sum().item())
+    fw = stage_work(cfg, touched)
+    bw = bwd_stage_work(cfg, touched)
+
+    fev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    bev = [moe.stage_events(stream, moe.BWD_STAGES) for _ in range(args.steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(visible_gpu_id(local_rank))
+    start.record(stream)
+    for i in range(args.steps):
+        fev[i][0].record(stream)
+        moe.layer_forward_train(shape, x, C, R, Sh, ws, ctx, out=out)
+        fev[i][1].record(stream)
+        moe.layer_backward(shape, x, C, R, Sh, dout, ctx, wsb, grads=grads, events=bev[i])
+    stop.record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    barrier()
+    moe.check_device_error(ws)
+    moe.check_device_error(wsb)
+    ms = reduce_max(start.elapsed_time(stop) / args.steps, dev)
+    stage_ms = {"forward_train": statistics.mean(a.elapsed_time(b) for a, b in fev)}
+    for j, name in enumerate(moe.BWD_STAGE_NAMES):
+        stage_ms[name] = statistics.mean(e[j].elapsed_time(e[j + 1]) for e in bev)
+    peaks, peak_src = load_peaks()
+    dom = max((k for k in stage_ms if k != "forward_train"), key=stage_ms.get)
+    flops, nbytes = bw[dom]
+    ridge = peaks["bf16_tflops_sustained"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    bound = "tensor" if nbytes == 0 or flops / nbytes > ridge else "hbm"
+    t = stage_ms[dom] / 1e3
+    if bound == "tensor":
+        achieved, peak, unit = flops / t / 1e12, peaks["bf16_tflops_sustained"], "TFLOP/s"
+    else:
+        achieved, peak, unit = nbytes / t / 1e9, peaks["hbm_gbs"], "GB/s"
+    fwd_flops = sum(f for f, _ in fw.values())
+    bwd_flops = sum(f for f, _ in bw.values())
+    line = {
+        "metric": METRIC, "value": aggregate_throughput(cfg.T, world, ms), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": cfg.name, "pass": "forward_train+backward", "T": cfg.T, "d": cfg.d,
+                   "n_experts": cfg.n_experts, "inter": cfg.inter, "top_k": cfg.top_k, "n_shared": cfg.n_shared,
+                   "bias": cfg.has_bias, "gate_mode": args.gate_mode,
+                   "parallelism": f"replicas{world}" if world > 1 else "single",
+                   "l2": "inputs larger than L2 (weights, gradients, activations), no flush"},
+        "tflops": (fwd_flops + bwd_flops) / (ms / 1e3) / 1e12 * world,
+        "backward_tflops": bwd_flops / (sum(v for k, v in stage_ms.items() if k != "forward_train") / 1e3) / 1e12,
+        "experts_touched": touched,
+        "stage_ms": stage_ms,
+        "roofline": {"bound": bound, "kernel": dom, "achieved": achieved, "peak": peak, "unit": unit,
+                     "frac": achieved / peak,
+                     "peak_source": f"{peak_src} ({'bf16 sustained' if bound == 'tensor' else 'HBM copy'})",
+                     "traffic": None, "algorithmic_per_launch": flops if bound == "tensor" else nbytes},
+        "gpu_launches": (moe.layer_launches(shape) + moe.backward_launches(shape)) * args.steps,
+        "clocks": clocks,
+        "e2e": None,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -482,6 +597,8 @@ def main(argv=None):
     ap.add_argument("--routed-fmt", default="bf16", choices=["bf16", "e4m3"],
                     help="storage of the routed experts' weights: bf16, or e4m3 codes with per-channel scales "
                          "(FP8 tensor-core path; activations quantised per row)")
+    ap.add_argument("--pass", dest="pass_", default="forward", choices=["forward", "train"],
+                    help="forward: the layer forward (default); train: forward for training + backward")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args(argv)
@@ -498,7 +615,12 @@ def main(argv=None):
         return
     init_dist(world, "nccl")
     try:
-        run_ours(args, cfg, rank, world, local_rank)
+        if args.pass_ == "train":
+            if args.routed_fmt != "bf16" or cfg.dtype != torch.bfloat16:
+                raise SystemExit("--pass train needs a bf16 workload with bf16 routed experts")
+            run_train(args, cfg, rank, world, local_rank)
+        else:
+            run_ours(args, cfg, rank, world, local_rank)
     finally:
         if torch.distributed.is_available() and torch.distributed.is_initialized():
             torch.distributed.destroy_process_group()

@@ -514,7 +514,8 @@ moe_status_t layer_backward_impl(const moe_shape_t* shape, const void* x, const 
                                  const float* router_bias, const moe_ffn_weights_t* routed,
                                  const moe_ffn_weights_t* shared, const void* dout, const void* ctx, size_t ctx_bytes,
                                  void* dx, float* dcentroids, float* drouter_bias, const moe_ffn_grads_t* groutes,
-                                 const moe_ffn_grads_t* gshared, void* ws, size_t ws_bytes, cudaStream_t st) {
+                                 const moe_ffn_grads_t* gshared, void* ws, size_t ws_bytes, cudaStream_t st,
+                                 cudaEvent_t const* ev = nullptr) {
     Dims D;
     MOE_TRY(to_dims(shape, &D));
     MOE_TRY(check_train(D));
@@ -564,25 +565,33 @@ moe_status_t layer_backward_impl(const moe_shape_t* shape, const void* x, const 
     float* z = at<float>(ws, L.z);
     float* dz = at<float>(ws, L.dz);
 
+    auto mark = [&](int i) -> bool { return !ev || cudaEventRecord(ev[i], st) == cudaSuccess; };
+    if (!mark(0)) return MOE_ERR_CUDA;
     MOE_CUDA(launch_plan_bwd(D, offsets, const_cast<int32_t*>(B.offs_pad), const_cast<int32_t*>(B.ts_dh),
                              const_cast<int32_t*>(B.ts_dx), st));
     MOE_CUDA(launch_bwd_gather(D, dout, x, R.b2, offsets, B.offs_pad, stok, sgate, B.dout_pad, B.x_pad, gate_pad, b2dot,
                                err, st));
     MOE_CUDA(launch_router_logits(D, x, centroids, z, err, st));
+    if (!mark(1)) return MOE_ERR_CUDA;
     MOE_CUDA(launch_tc_dh(D, B, R, Sh, dout, err, st));
+    if (!mark(2)) return MOE_ERR_CUDA;
     MOE_CUDA(launch_router_bwd(D, z, router_bias, idx, slot_of, B.dgate_part, L.n_parts, b2dot, dz, B.dz_bf16, nullptr,
                                st));
+    if (!mark(3)) return MOE_ERR_CUDA;
     MOE_CUDA(launch_tc_dx(D, B, R, err, st));
     MOE_CUDA(launch_tc_dxs(D, B, Sh, centroids, err, st));
     MOE_CUDA(launch_combine(D, B.dx_slot, slot_of, B.base, dx, err, st));
+    if (!mark(4)) return MOE_ERR_CUDA;
     // weight gradients
     const long long T = D.T;
     DwSpec w2 = {0, D.E, D.d, D.I, B.dout_pad, L.S_pad_max, 0, B.hg, L.S_pad_max, 0, B.offs_pad, 0,
                  groutes->w2, nullptr, nullptr};
     MOE_CUDA(launch_tc_dw(D, w2, err, st));
+    if (!mark(5)) return MOE_ERR_CUDA;
     DwSpec w13 = {1, D.E, 2 * D.I, D.d, B.dag, L.S_pad_max, 0, B.x_pad, L.S_pad_max, 0, B.offs_pad, 0,
                   groutes->w1, groutes->w3, nullptr};
     MOE_CUDA(launch_tc_dw(D, w13, err, st));
+    if (!mark(6)) return MOE_ERR_CUDA;
     if (D.Ks > 0) {
         DwSpec s2 = {0, D.Ks, D.d, D.Is, dout, T, 0, B.hg_s, T, 1, nullptr, D.T, gshared->w2, nullptr, nullptr};
         MOE_CUDA(launch_tc_dw(D, s2, err, st));
@@ -606,6 +615,7 @@ moe_status_t layer_backward_impl(const moe_shape_t* shape, const void* x, const 
     }
     if (drouter_bias)
         MOE_CUDA(launch_colsum(true, true, dz, 0, D.E, nullptr, D.T, nullptr, 1, D.E, D.E, drouter_bias, nullptr, st));
+    if (!mark(7)) return MOE_ERR_CUDA;
     return MOE_OK;
 }
 
@@ -664,6 +674,31 @@ MOE_EXPORT moe_status_t moe_layer_backward(const moe_shape_t* shape, const void*
                                            void* ws, size_t ws_bytes, moe_stream_t stream) {
     return layer_backward_impl(shape, x, centroids, router_bias, routed, shared, dout, ctx, ctx_bytes, dx, dcentroids,
                                drouter_bias, routed_grads, shared_grads, ws, ws_bytes, (cudaStream_t)stream);
+}
+
+MOE_EXPORT moe_status_t moe_layer_backward_timed(const moe_shape_t* shape, const void* x, const void* centroids,
+                                                 const float* router_bias, const moe_ffn_weights_t* routed,
+                                                 const moe_ffn_weights_t* shared, const void* dout, const void* ctx,
+                                                 size_t ctx_bytes, void* dx, float* dcentroids, float* drouter_bias,
+                                                 const moe_ffn_grads_t* routed_grads,
+                                                 const moe_ffn_grads_t* shared_grads, void* ws, size_t ws_bytes,
+                                                 moe_stream_t stream, void* const* stage_events, int32_t n_events) {
+    if (!stage_events || n_events != MOE_BWD_STAGES + 1) return MOE_ERR_INVALID_ARG;
+    for (int i = 0; i < n_events; ++i)
+        if (!stage_events[i]) return MOE_ERR_INVALID_ARG;
+    return layer_backward_impl(shape, x, centroids, router_bias, routed, shared, dout, ctx, ctx_bytes, dx, dcentroids,
+                               drouter_bias, routed_grads, shared_grads, ws, ws_bytes, (cudaStream_t)stream,
+                               reinterpret_cast<cudaEvent_t const*>(stage_events));
+}
+
+MOE_EXPORT int32_t moe_backward_launches(const moe_shape_t* shape) {
+    Dims D;
+    if (to_dims(shape, &D) != MOE_OK || check_train(D) != MOE_OK) return -1;
+    if (D.T == 0) return 0;
+    int n = 3 + 1 + 1 + 3 + 2 + 1;            // plan, gather, logits; DH; router bwd; DX, DXS, combine; dW2, dW13; dC
+    if (D.Ks > 0) n += 2;                      // shared dW2, dW13
+    if (D.bias) n += 2 + (D.Ks > 0 ? 2 : 0);   // routed db2, db1|db3 (+ shared)
+    return n;                                  // (+1 when a router-bias gradient is asked for)
 }
 
 }  // extern "C"

@@ -22,9 +22,12 @@ FMT_NATIVE, FMT_E4M3 = 0, 1        # storage of the routed experts' weights (moe
 EXPORTED = ("moe_workspace_bytes", "moe_layer_launches", "moe_status_string", "moe_version", "moe_check_device_error", "moe_ws_init",
             "moe_route", "moe_permute", "moe_expert_ffn", "moe_combine", "moe_layer_forward",
             "moe_layer_forward_timed", "moe_permute_no_alloc", "moe_quantize_rows_e4m3", "moe_train_ctx_bytes",
-            "moe_backward_workspace_bytes", "moe_layer_forward_train", "moe_layer_backward")
+            "moe_backward_workspace_bytes", "moe_layer_forward_train", "moe_layer_backward",
+            "moe_layer_backward_timed", "moe_backward_launches")
 NUM_STAGES = 7
 STAGE_NAMES = ("router", "permute", "plan", "gather", "gemm1_swiglu", "gemm2", "combine")
+BWD_STAGES = 7
+BWD_STAGE_NAMES = ("bwd_prep", "bwd_dh", "bwd_router", "bwd_dx", "bwd_dw2", "bwd_dw13", "bwd_shared_dc_bias")
 
 
 class MoeShape(ctypes.Structure):
@@ -87,9 +90,13 @@ def _lib():
         lib.moe_backward_workspace_bytes.restype = sz
         lib.moe_layer_forward_train.argtypes = [sh, vp, vp, f32p, wp, wp, vp, vp, sz, vp, sz, vp]
         lib.moe_layer_backward.argtypes = [sh, vp, vp, f32p, wp, wp, vp, vp, sz, vp, f32p, f32p, gp, gp, vp, sz, vp]
+        lib.moe_layer_backward_timed.argtypes = [sh, vp, vp, f32p, wp, wp, vp, vp, sz, vp, f32p, f32p, gp, gp, vp, sz,
+                                                 vp, ctypes.POINTER(ctypes.c_void_p), ctypes.c_int32]
+        lib.moe_backward_launches.argtypes = [sh]
+        lib.moe_backward_launches.restype = ctypes.c_int32
         for n in ("moe_check_device_error", "moe_ws_init", "moe_route", "moe_permute", "moe_expert_ffn",
                   "moe_combine", "moe_layer_forward", "moe_layer_forward_timed", "moe_quantize_rows_e4m3",
-                  "moe_layer_forward_train", "moe_layer_backward"):
+                  "moe_layer_forward_train", "moe_layer_backward", "moe_layer_backward_timed"):
             getattr(lib, n).restype = ctypes.c_int
         _LIB = lib
     return _LIB
@@ -285,28 +292,50 @@ def _grad_stack(w: Dict):
     return g, MoeGrads(*(None if g[k] is None else g[k].data_ptr() for k in ("w1", "b1", "w3", "b3", "w2", "b2")))
 
 
+def backward_launches(shape: MoeShape) -> int:
+    return int(_lib().moe_backward_launches(ctypes.byref(shape)))
+
+
+def new_grads(x, centroids, routed: Dict, shared: Optional[Dict], router_bias_grad: bool = False):
+    """Output tensors of layer_backward (reusable across calls)."""
+    return {"dx": torch.empty_like(x),
+            "dcentroids": torch.empty(centroids.shape, dtype=torch.float32, device=x.device),
+            "drouter_bias": torch.empty(centroids.shape[0], dtype=torch.float32, device=x.device) if router_bias_grad
+            else None,
+            "routed": _grad_stack(routed)[0], "shared": _grad_stack(shared)[0] if shared is not None else None}
+
+
+def _grad_struct(g: Optional[Dict]):
+    if g is None:
+        return None
+    return MoeGrads(*(None if g.get(k) is None else g[k].data_ptr() for k in ("w1", "b1", "w3", "b3", "w2", "b2")))
+
+
 def layer_backward(shape: MoeShape, x, centroids, routed: Dict, shared: Optional[Dict], dout, ctx, ws_bwd,
-                   stream=None, router_bias=None, router_bias_grad: bool = False):
-    """moe_layer_backward: returns {dx, dcentroids, drouter_bias (or None), routed: {...}, shared:
-    {...} or None} with the gradient tensors allocated here."""
-    dx = torch.empty_like(x)
-    dc = torch.empty(centroids.shape, dtype=torch.float32, device=x.device)
-    db = torch.empty(centroids.shape[0], dtype=torch.float32, device=x.device) if router_bias_grad else None
-    gr, gr_c = _grad_stack(routed)
-    gs, gs_c = _grad_stack(shared) if shared is not None else (None, None)
+                   stream=None, router_bias=None, router_bias_grad: bool = False, grads: Optional[Dict] = None,
+                   events=None):
+    """moe_layer_backward (moe_layer_backward_timed when `events` holds BWD_STAGES + 1 events):
+    returns {dx, dcentroids, drouter_bias (or None), routed: {...}, shared: {...} or None}, written
+    into `grads` when given (see new_grads), else into tensors allocated here."""
+    g = new_grads(x, centroids, routed, shared, router_bias_grad) if grads is None else grads
+    gr_c, gs_c = _grad_struct(g["routed"]), _grad_struct(g["shared"])
     rw, sw = _weights(routed), _weights(shared)
-    _check(_lib().moe_layer_backward(ctypes.byref(shape), _ptr(x), _ptr(centroids), _bias_ptr(router_bias),
-                                     ctypes.byref(rw), None if sw is None else ctypes.byref(sw), _ptr(dout), _ptr(ctx),
-                                     ctx.numel(), _ptr(dx), _ptr(dc), _ptr(db), ctypes.byref(gr_c),
-                                     None if gs_c is None else ctypes.byref(gs_c), _ptr(ws_bwd), ws_bwd.numel(),
-                                     _stream(stream)),
-           "moe_layer_backward")
-    return {"dx": dx, "dcentroids": dc, "drouter_bias": db, "routed": gr, "shared": gs}
+    args = [ctypes.byref(shape), _ptr(x), _ptr(centroids), _bias_ptr(router_bias), ctypes.byref(rw),
+            None if sw is None else ctypes.byref(sw), _ptr(dout), _ptr(ctx), ctx.numel(), _ptr(g["dx"]),
+            _ptr(g["dcentroids"]), _ptr(g["drouter_bias"]), ctypes.byref(gr_c),
+            None if gs_c is None else ctypes.byref(gs_c), _ptr(ws_bwd), ws_bwd.numel(), _stream(stream)]
+    if events is None:
+        _check(_lib().moe_layer_backward(*args), "moe_layer_backward")
+    else:
+        arr = (ctypes.c_void_p * len(events))(*[e.cuda_event for e in events])
+        _check(_lib().moe_layer_backward_timed(*args, arr, len(events)), "moe_layer_backward_timed")
+    return g
 
 
-def stage_events(stream=None):
-    """NUM_STAGES + 1 recorded torch CUDA events whose handles the timed entry point reuses."""
-    evs = [torch.cuda.Event(enable_timing=True) for _ in range(NUM_STAGES + 1)]
+def stage_events(stream=None, n_stages: int = NUM_STAGES):
+    """n_stages + 1 recorded torch CUDA events whose handles a timed entry point reuses
+    (NUM_STAGES for the forward, BWD_STAGES for the backward)."""
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(n_stages + 1)]
     s = torch.cuda.current_stream() if stream is None else stream
     for e in evs:
         e.record(s)            # creates the underlying CUDA event

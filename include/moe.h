@@ -308,6 +308,27 @@ moe_status_t moe_layer_backward(const moe_shape_t* shape, const void* x, const v
                                 void* ws, size_t ws_bytes, moe_stream_t stream);
 
 /*
+ * moe_layer_backward with stage timing (as moe_layer_forward_timed): stage_events[i] is recorded
+ * before stage i and stage_events[MOE_BWD_STAGES] after the last.  Stages:
+ *   0 tile tables, row gathers, router logits    1 dH GEMM (+ SwiGLU backward, gate-gradient partials)
+ *   2 router backward (dz)                        3 dx: routed GEMM, shared + router GEMM, combine
+ *   4 routed dW2 GEMM                             5 routed dW1 | dW3 GEMM
+ *   6 shared experts' dW, dcentroids GEMM, bias-gradient sums
+ */
+#define MOE_BWD_STAGES 7
+moe_status_t moe_layer_backward_timed(const moe_shape_t* shape, const void* x, const void* centroids,
+                                      const float* router_bias, const moe_ffn_weights_t* routed,
+                                      const moe_ffn_weights_t* shared, const void* dout, const void* ctx,
+                                      size_t ctx_bytes, void* dx, float* dcentroids, float* drouter_bias,
+                                      const moe_ffn_grads_t* routed_grads, const moe_ffn_grads_t* shared_grads,
+                                      void* ws, size_t ws_bytes, moe_stream_t stream, void* const* stage_events,
+                                      int32_t n_events);
+
+/* Kernel launches of one moe_layer_backward call without a router-bias gradient (one more with
+ * it); -1 for an unsupported shape, 0 when T == 0. */
+int32_t moe_backward_launches(const moe_shape_t* shape);
+
+/*
  * moe_permute_no_alloc — the paper has no counterpart to this entry point; it exists for
  * callers of this library that cannot allocate device memory.  moe_permute needs scratch
  * space, which it takes from the caller's workspace.  A caller that cannot call cudaMalloc

@@ -65,6 +65,19 @@ def test_stage_work_sums_to_layer_flops():
                - (256 * routed8 + per_expert + 256 * 7168 * 2 + 2 * 256 * 7168 * 2)) < 1
 
 
+def test_backward_work_is_twice_the_forward():
+    """Backward FLOPs: twice the expert and shared FLOPs of the forward (data and weight gradients)
+    plus three router-sized products (recomputed logits, dz . C, dz^T x) against the forward's one."""
+    for name, cfg in W.CONFIGS.items():
+        if cfg.dtype != torch.bfloat16:
+            continue
+        fw = sum(f for f, _ in bench.stage_work(cfg, cfg.n_experts).values())
+        bw = sum(f for f, _ in bench.bwd_stage_work(cfg, cfg.n_experts).values())
+        router = 2.0 * cfg.T * cfg.d * cfg.n_experts
+        assert abs(bw - (2 * fw + router)) < 1e-9 * bw, name
+        assert all(b > 0 for _, b in bench.bwd_stage_work(cfg, cfg.n_experts).values())
+
+
 def test_reference_arm_line():
     r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--workload", "tiny",
                         "--steps", "3", "--warmup", "3"], capture_output=True, text=True, timeout=600,
