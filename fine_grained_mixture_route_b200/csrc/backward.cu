@@ -85,13 +85,16 @@ __device__ __forceinline__ int group_of(const int32_t* starts, int n, int q) {  
 
 // Rows of the padded grouped layout: q in [0, offs_pad[E]).  A live row (slot p = offsets[e] + r)
 // gets dout and x of its token, its gate, and b2dot[p] = <dout_t, b2_e>; a pad row gets zeros.
+// x_pad rows end with 64 extra columns (1 for a live row, then zeros) and hg rows (I + 64 long,
+// whose first I columns the DH GEMM writes) with the gate, then zeros.
 __global__ void bwd_gather_kernel(const uint4* __restrict__ dout, const uint4* __restrict__ x,
                                   const __nv_bfloat16* __restrict__ b2, const int32_t* __restrict__ offsets,
                                   const int32_t* __restrict__ offs_pad, const int32_t* __restrict__ stok,
-                                  const float* __restrict__ sgate, int E, int T, int d, uint4* dout_pad, uint4* x_pad,
-                                  float* gate_pad, float* b2dot, uint32_t* err) {
+                                  const float* __restrict__ sgate, int E, int T, int d, int I, uint4* dout_pad,
+                                  uint4* x_pad, __nv_bfloat16* hg, float* gate_pad, float* b2dot, uint32_t* err) {
     __shared__ float red[32];
     const int nv = d / 8;
+    const int nvx = nv + 8;                         // x_pad row: d + 64 bf16
     const int total = offs_pad[E];
     for (int q = blockIdx.x; q < total; q += gridDim.x) {
         const int e = group_of(offs_pad, E, q);
@@ -119,9 +122,17 @@ __global__ void bwd_gather_kernel(const uint4* __restrict__ dout, const uint4* _
                 }
             }
             dout_pad[(size_t)q * nv + i] = dv;
-            x_pad[(size_t)q * nv + i] = xv;
+            x_pad[(size_t)q * nvx + i] = xv;
         }
-        if (threadIdx.x == 0) gate_pad[q] = t >= 0 ? sgate[p] : 0.f;
+        const float gq = t >= 0 ? sgate[p] : 0.f;
+        if (threadIdx.x < 8) {
+            const uint32_t one = t >= 0 ? 0x3F80u : 0u;                     // bf16 1.0
+            const uint32_t gb = __bfloat16_as_ushort(__float2bfloat16_rn(gq));
+            x_pad[(size_t)q * nvx + nv + threadIdx.x] = make_uint4(threadIdx.x == 0 ? one : 0u, 0, 0, 0);
+            reinterpret_cast<uint4*>(hg + (size_t)q * (I + 64) + I)[threadIdx.x] =
+                make_uint4(threadIdx.x == 0 ? gb : 0u, 0, 0, 0);
+        }
+        if (threadIdx.x == 0) gate_pad[q] = gq;
         if (b2 && live) {
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
@@ -231,24 +242,50 @@ __global__ void router_bwd_kernel(const float* __restrict__ z, const float* __re
     }
 }
 
-// Column sums over the rows of each group, fp32 in row order (deterministic):
-//   out[g][c] = sum_{r in group g} w[r] * src[r][c]   (w = 1 when null)
-// rows of group g: [starts[g], starts[g+1]) when starts is given, else [0, n_rows) of the
-// group's slice src + g * group_stride.  Columns c < split go to out0[g][c], the rest to
-// out1[g][c - split] (out1 null: split = W).  bf16 or fp32 source; bf16 or fp32 output.
-template <typename TS, typename TO>
-__global__ void colsum_kernel(const TS* __restrict__ src, long long group_stride, int ld, const int32_t* __restrict__ starts,
-                              int n_rows, const float* __restrict__ w, int W, int split, TO* out0, TO* out1) {
+// Column sums over the T rows of each group, deterministic, in two passes:
+//   partial[g][j][c] = sum of rows [256 j, 256 j + 256) of src_g[.][c]  (src_g = src + g * group_stride)
+//   out[g][c] = sum_j partial[g][j][c] in order; columns c < split -> out0[g][c], the rest -> out1[g][c - split]
+constexpr int COLSUM_ROWS = 256;
+template <typename TS>
+__global__ void colsum_partial_kernel(const TS* __restrict__ src, long long group_stride, int ld, int n_rows, int W,
+                                      float* partial) {
+    const int g = blockIdx.z, j = blockIdx.y;
+    const int c = blockIdx.x * blockDim.x + threadIdx.x;
+    if (c >= W) return;
+    const int nch = (n_rows + COLSUM_ROWS - 1) / COLSUM_ROWS;
+    const TS* base = src + (size_t)g * group_stride;
+    const int r0 = j * COLSUM_ROWS, r1 = min(n_rows, r0 + COLSUM_ROWS);
+    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+    int r = r0;
+    for (; r + 3 < r1; r += 4) {
+        a0 += to_f32<TS>(base[(size_t)r * ld + c]);
+        a1 += to_f32<TS>(base[(size_t)(r + 1) * ld + c]);
+        a2 += to_f32<TS>(base[(size_t)(r + 2) * ld + c]);
+        a3 += to_f32<TS>(base[(size_t)(r + 3) * ld + c]);
+    }
+    for (; r < r1; ++r) a0 += to_f32<TS>(base[(size_t)r * ld + c]);
+    partial[((size_t)g * nch + j) * W + c] = (a0 + a1) + (a2 + a3);
+}
+
+template <typename TO>
+__global__ void colsum_final_kernel(const float* __restrict__ partial, int nch, int W, int split, TO* out0, TO* out1) {
     const int g = blockIdx.y;
     const int c = blockIdx.x * blockDim.x + threadIdx.x;
     if (c >= W) return;
-    const int r0 = starts ? starts[g] : 0;
-    const int r1 = starts ? starts[g + 1] : n_rows;
-    const TS* base = src + (size_t)g * group_stride;
     float acc = 0.f;
-    for (int r = r0; r < r1; ++r) acc += (w ? w[r] : 1.f) * to_f32<TS>(base[(size_t)r * ld + c]);
+    for (int j = 0; j < nch; ++j) acc += partial[((size_t)g * nch + j) * W + c];
     if (c < split) out0[(size_t)g * split + c] = from_f32<TO>(acc);
     else out1[(size_t)g * (W - split) + (c - split)] = from_f32<TO>(acc);
+}
+
+// hg_s rows (K_s x T, I_s + 64 long): column I_s = 1, the other extra columns 0
+__global__ void fill_aug_kernel(__nv_bfloat16* rows, long long n_rows, int ld, int col) {
+    const long long n = n_rows * 8;
+    for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
+        const long long r = i / 8;
+        const int j = (int)(i % 8);
+        reinterpret_cast<uint4*>(rows + (size_t)r * ld + col)[j] = make_uint4(j == 0 ? 0x3F80u : 0u, 0, 0, 0);
+    }
 }
 
 }  // namespace
@@ -261,13 +298,13 @@ cudaError_t launch_plan_bwd(const Dims& D, const int32_t* offsets, int32_t* offs
 
 cudaError_t launch_bwd_gather(const Dims& D, const void* dout, const void* x, const void* b2, const int32_t* offsets,
                               const int32_t* offs_pad, const int32_t* stok, const float* sgate, void* dout_pad,
-                              void* x_pad, float* gate_pad, float* b2dot, uint32_t* err, cudaStream_t stream) {
+                              void* x_pad, void* hg, float* gate_pad, float* b2dot, uint32_t* err, cudaStream_t stream) {
     if (D.T == 0) return cudaSuccess;
     const long long rows = D.slots() + 64LL * D.E;
     const long long cap = (long long)num_sms() * 16;
     bwd_gather_kernel<<<(int)(rows < cap ? rows : cap), 128, 0, stream>>>(
-        (const uint4*)dout, (const uint4*)x, (const __nv_bfloat16*)b2, offsets, offs_pad, stok, sgate, D.E, D.T, D.d,
-        (uint4*)dout_pad, (uint4*)x_pad, gate_pad, b2dot, err);
+        (const uint4*)dout, (const uint4*)x, (const __nv_bfloat16*)b2, offsets, offs_pad, stok, sgate, D.E, D.T, D.d, D.I,
+        (uint4*)dout_pad, (uint4*)x_pad, (__nv_bfloat16*)hg, gate_pad, b2dot, err);
     return cudaGetLastError();
 }
 
@@ -284,26 +321,27 @@ cudaError_t launch_router_bwd(const Dims& D, const float* z, const float* bias, 
     return cudaGetLastError();
 }
 
-cudaError_t launch_colsum(bool src_f32, bool out_f32, const void* src, long long group_stride, int ld,
-                          const int32_t* starts, int n_rows, const float* w, int groups, int W, int split, void* out0,
-                          void* out1, cudaStream_t stream) {
-    if (groups <= 0 || W <= 0) return cudaSuccess;
+cudaError_t launch_colsum(bool src_f32, bool out_f32, const void* src, long long group_stride, int ld, int n_rows,
+                          int groups, int W, int split, void* out0, void* out1, float* partial, cudaStream_t stream) {
+    if (groups <= 0 || W <= 0 || n_rows <= 0) return cudaSuccess;
     if (!out1) split = W;
-    const dim3 grid((W + 255) / 256, groups);
-    if (src_f32 && out_f32)
-        colsum_kernel<float, float><<<grid, 256, 0, stream>>>((const float*)src, group_stride, ld, starts, n_rows, w, W,
-                                                              split, (float*)out0, (float*)out1);
-    else if (src_f32)
-        colsum_kernel<float, __nv_bfloat16><<<grid, 256, 0, stream>>>((const float*)src, group_stride, ld, starts, n_rows,
-                                                                      w, W, split, (__nv_bfloat16*)out0,
-                                                                      (__nv_bfloat16*)out1);
-    else if (out_f32)
-        colsum_kernel<__nv_bfloat16, float><<<grid, 256, 0, stream>>>((const __nv_bfloat16*)src, group_stride, ld, starts,
-                                                                      n_rows, w, W, split, (float*)out0, (float*)out1);
-    else
-        colsum_kernel<__nv_bfloat16, __nv_bfloat16><<<grid, 256, 0, stream>>>(
-            (const __nv_bfloat16*)src, group_stride, ld, starts, n_rows, w, W, split, (__nv_bfloat16*)out0,
-            (__nv_bfloat16*)out1);
+    const int nch = (n_rows + COLSUM_ROWS - 1) / COLSUM_ROWS;
+    const dim3 g1((W + 255) / 256, nch, groups), g2((W + 255) / 256, groups);
+    if (src_f32) colsum_partial_kernel<float><<<g1, 256, 0, stream>>>((const float*)src, group_stride, ld, n_rows, W, partial);
+    else colsum_partial_kernel<__nv_bfloat16><<<g1, 256, 0, stream>>>((const __nv_bfloat16*)src, group_stride, ld,
+                                                                      n_rows, W, partial);
+    if (out_f32) colsum_final_kernel<float><<<g2, 256, 0, stream>>>(partial, nch, W, split, (float*)out0, (float*)out1);
+    else colsum_final_kernel<__nv_bfloat16><<<g2, 256, 0, stream>>>(partial, nch, W, split, (__nv_bfloat16*)out0,
+                                                                    (__nv_bfloat16*)out1);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_fill_aug(void* rows, long long n_rows, int ld, int col, cudaStream_t stream) {
+    if (n_rows <= 0) return cudaSuccess;
+    const long long n = n_rows * 8;
+    const long long cap = (long long)num_sms() * 8;
+    const long long blocks = (n + 255) / 256;
+    fill_aug_kernel<<<(int)(blocks < cap ? blocks : cap), 256, 0, stream>>>((__nv_bfloat16*)rows, n_rows, ld, col);
     return cudaGetLastError();
 }
 

@@ -47,7 +47,8 @@ constexpr int EPI_WARPS = 8;
 constexpr int TMEM_COLS = 512;
 constexpr int ACC_COLS = 256;
 constexpr int RING_BYTES = 192 * 1024;   // shared-memory ring (stages x (A + B))
-constexpr int SMEM_BYTES = 1024 /*align slack*/ + RING_BYTES + 256 /*barriers*/;
+constexpr int STAGE_OUT_BYTES = 2048;     // per epilogue warp: a 32 x 32 bf16 chunk being transposed
+constexpr int SMEM_BYTES = 1024 /*align slack*/ + RING_BYTES + 256 /*barriers*/ + EPI_WARPS * STAGE_OUT_BYTES;
 constexpr unsigned long long WAIT_NS = 4000000000ull;
 #ifndef MOE_GROUP_M
 #define MOE_GROUP_M 8                    // M-tiles per raster band of the expert GEMMs
@@ -119,6 +120,9 @@ struct Params {
     int dw_K;
     __nv_bfloat16 *dw_out0, *dw_out1;
     float* dw_out_f32;
+    int dw_Nt;                         // DW: columns the tiles cover (dw_N, or dw_N + 1 with a bias column)
+    int dw_bias_col;                   // DW: B column dw_N holds the row weights of a bias gradient (or -1):
+    __nv_bfloat16 *dw_bias0, *dw_bias1;  //    out column dw_N -> bias0 [g][M] (kind 1: rows >= M/2 -> bias1)
     uint32_t* err;
 };
 
@@ -356,7 +360,7 @@ __device__ __forceinline__ int total_tiles(const Params& p) {
         return p.tile_start[p.E] + (p.fold_shared ? ceil_div(p.T, TM) * ceil_div(p.d, 256) : 0);
     if (MODE == DH) return p.tile_start[p.E + p.Ks];
     if (MODE == DX) return p.tile_start[p.E];
-    if (MODE == DW) return p.dw_groups * ceil_div(p.dw_M, TM) * ceil_div(p.dw_N, 256);
+    if (MODE == DW) return p.dw_groups * ceil_div(p.dw_M, TM) * ceil_div(p.dw_Nt, 256);
     return ceil_div(p.T, TM) * ceil_div(p.d, 256);
 }
 
@@ -440,7 +444,7 @@ __device__ __forceinline__ Tile decode(const Params& p, int t) {
         x.n0 = n * 256;
         x.num_kb = p.Ks * 2 * ceil_div(p.Is, BK) + ceil_div(p.E, BK);
     } else if (MODE == DW) {
-        const int mt = ceil_div(p.dw_M, TM), nt = ceil_div(p.dw_N, 256);
+        const int mt = ceil_div(p.dw_M, TM), nt = ceil_div(p.dw_Nt, 256);
         const int g = t / (mt * nt);
         int m, n;
         band_mn(t - g * mt * nt, mt, nt, p.group_m, m, n);
@@ -727,6 +731,36 @@ __device__ __forceinline__ void epilogue_router_partial(const Params& p, const T
     }
 }
 
+// Stores a warp's 32 x 32 bf16 chunk (lane = row, pk = its 32 columns packed in pairs) through a
+// per-warp shared-memory transpose, so that each store instruction writes 64 contiguous bytes of
+// eight rows instead of 16 bytes of 32 rows.  In shared memory row r keeps its four 16-byte pieces
+// rotated by r/2, which makes both the writes and the reads free of bank conflicts.  row_ptr is
+// this lane's destination row (already offset to column 0 of the chunk), or null to skip the row;
+// ncols (multiple of 8) limits the columns written.
+__device__ __forceinline__ void warp_store_chunk_bf16(uint32_t stage, const uint32_t (&pk)[16], __nv_bfloat16* row_ptr,
+                                                      int ncols, int lane) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const uint32_t a = stage + lane * 64 + (((j + (lane >> 1)) & 3) << 4);
+        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(pk[4 * j]), "r"(pk[4 * j + 1]),
+                     "r"(pk[4 * j + 2]), "r"(pk[4 * j + 3])
+                     : "memory");
+    }
+    __syncwarp();
+    const int j = lane & 3;
+#pragma unroll
+    for (int sgrp = 0; sgrp < 4; ++sgrp) {
+        const int r = sgrp * 8 + (lane >> 2);
+        __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(
+            __shfl_sync(0xffffffffu, reinterpret_cast<unsigned long long>(row_ptr), r));
+        uint4 v;
+        const uint32_t a = stage + r * 64 + (((j + (r >> 1)) & 3) << 4);
+        asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
+        if (dst && j * 8 < ncols) *reinterpret_cast<uint4*>(dst + j * 8) = v;
+    }
+    __syncwarp();
+}
+
 // DH: for a routed group the rows are grouped slots (A = dout rows of the slot's token, in the
 // 64-row-padded layout), for a shared group the tokens.  Per element of the hidden row:
 // dh_raw = (dout . W2)[c]; a, g = the saved pre-activations; sg = sigmoid(a); h = a sg g;
@@ -747,7 +781,8 @@ __device__ __forceinline__ void epilogue_dh(const Params& p, const Tile& x, uint
     const __nv_bfloat16* arow = (shared ? p.as_sv : p.a_sv) + so;
     const __nv_bfloat16* grow = (shared ? p.gs_sv : p.g_sv) + so;
     __nv_bfloat16* dagrow = shared ? p.dag_s + ((size_t)e * p.T + r) * 2 * I : p.dag + (size_t)pp * 2 * I;
-    __nv_bfloat16* hgrow = shared ? p.hg_s + ((size_t)e * p.T + r) * I : p.hg + (size_t)pp * I;
+    // gate * h rows carry 64 extra columns (the bias-gradient column of the w2 gradient GEMM)
+    __nv_bfloat16* hgrow = shared ? p.hg_s + ((size_t)e * p.T + r) * (I + 64) : p.hg + (size_t)pp * (I + 64);
     const float gate = (!shared && live) ? p.sorted_gate[pu] : 1.f;
     float dot = 0.f;
 #pragma unroll 1
@@ -821,45 +856,60 @@ __device__ __forceinline__ void epilogue_dx(const Params& p, const Tile& x, uint
     }
 }
 
-// DW: one 128 x 256 tile of a group's weight gradient (zeros when the group has no rows).
-__device__ __forceinline__ void epilogue_dw(const Params& p, const Tile& x, uint32_t tacc, int row, int half) {
+// DW: one 128 x 256 tile of a group's weight gradient (zeros when the group has no rows).  bf16
+// outputs go through the per-warp transpose (warp_store_chunk_bf16); column dw_N, when it is the
+// bias column, goes to the bias gradient.
+__device__ __forceinline__ void epilogue_dw(const Params& p, const Tile& x, uint32_t tacc, int row, int half,
+                                            uint32_t stage, int lane) {
     const int m = x.m0 + row;
     const bool live = m < p.dw_M;
     const bool zero = x.num_kb == 0;
     const int Mh = p.dw_M / 2;
     __nv_bfloat16* orow = nullptr;
     float* frow = nullptr;
-    if (p.dw_kind == 0) orow = p.dw_out0 + ((size_t)x.g * p.dw_M + m) * p.dw_N;
-    else if (p.dw_kind == 1) orow = m < Mh ? p.dw_out0 + ((size_t)x.g * Mh + m) * p.dw_N
-                                           : p.dw_out1 + ((size_t)x.g * Mh + m - Mh) * p.dw_N;
-    else frow = p.dw_out_f32 + ((size_t)x.g * p.dw_M + m) * p.dw_N;
+    if (live) {
+        if (p.dw_kind == 0) orow = p.dw_out0 + ((size_t)x.g * p.dw_M + m) * p.dw_N;
+        else if (p.dw_kind == 1) orow = m < Mh ? p.dw_out0 + ((size_t)x.g * Mh + m) * p.dw_N
+                                               : p.dw_out1 + ((size_t)x.g * Mh + m - Mh) * p.dw_N;
+        else frow = p.dw_out_f32 + ((size_t)x.g * p.dw_M + m) * p.dw_N;
+    }
 #pragma unroll 1
     for (int c = half * 4; c < half * 4 + 4; ++c) {
         uint32_t u[32];
         tmem_ld32(tacc + c * 32, u);
         tmem_wait_ld();
         const int col0 = x.n0 + c * 32;
-        if (!live || col0 >= p.dw_N) continue;
+        if (col0 >= p.dw_Nt) continue;                     // warp-uniform
         if (zero) {
 #pragma unroll
             for (int i = 0; i < 32; ++i) u[i] = 0u;
         }
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const int col = col0 + q * 8;
-            if (col >= p.dw_N) break;
-            if (frow) {
-                *reinterpret_cast<float4*>(frow + col) = make_float4(__uint_as_float(u[q * 8]), __uint_as_float(u[q * 8 + 1]),
-                                                                     __uint_as_float(u[q * 8 + 2]), __uint_as_float(u[q * 8 + 3]));
-                *reinterpret_cast<float4*>(frow + col + 4) = make_float4(__uint_as_float(u[q * 8 + 4]), __uint_as_float(u[q * 8 + 5]),
-                                                                         __uint_as_float(u[q * 8 + 6]), __uint_as_float(u[q * 8 + 7]));
+        if (live && p.dw_bias_col >= 0 && col0 + 32 > p.dw_N && col0 <= p.dw_N) {
+            // dw_N is a multiple of 64 (d, inter, inter_shared are) and chunks start at multiples of
+            // 32, so the bias column is the chunk's first column
+            const __nv_bfloat16 bv = __float2bfloat16_rn(__uint_as_float(u[0]));
+            if (p.dw_kind == 1) {
+                if (m < Mh) p.dw_bias0[(size_t)x.g * Mh + m] = bv;
+                else p.dw_bias1[(size_t)x.g * Mh + m - Mh] = bv;
             } else {
-                uint32_t pk[4];
-#pragma unroll
-                for (int i = 0; i < 4; ++i)
-                    pk[i] = pack_bf16(__uint_as_float(u[q * 8 + i * 2]), __uint_as_float(u[q * 8 + i * 2 + 1]));
-                *reinterpret_cast<uint4*>(orow + col) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                p.dw_bias0[(size_t)x.g * p.dw_M + m] = bv;
             }
+        }
+        const int ncols = min(32, p.dw_N - col0);
+        if (ncols <= 0) continue;                          // warp-uniform
+        if (p.dw_kind == 2) {
+            if (!live) continue;
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+                if (q * 4 < ncols)
+                    *reinterpret_cast<float4*>(frow + col0 + q * 4) =
+                        make_float4(__uint_as_float(u[q * 4]), __uint_as_float(u[q * 4 + 1]),
+                                    __uint_as_float(u[q * 4 + 2]), __uint_as_float(u[q * 4 + 3]));
+        } else {
+            uint32_t pk[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) pk[i] = pack_bf16(__uint_as_float(u[2 * i]), __uint_as_float(u[2 * i + 1]));
+            warp_store_chunk_bf16(stage, pk, orow ? orow + col0 : nullptr, ncols, lane);
         }
     }
 }
@@ -1143,7 +1193,7 @@ __global__ void __launch_bounds__(THREADS, 1) moe_tc_kernel(const __grid_constan
             } else if (MODE == DX) {
                 epilogue_dx(p, x, tacc, row, half);
             } else if (MODE == DW) {
-                epilogue_dw(p, x, tacc, row, half);
+                epilogue_dw(p, x, tacc, row, half, bar0 + 256 + (warp - 2) * STAGE_OUT_BYTES, lane);
             } else {
                 epilogue_gemm2s(p, x, tacc, row, half);
             }
@@ -1567,10 +1617,15 @@ cudaError_t launch_tc_dw(const Dims& D, const DwSpec& w, uint32_t* err, cudaStre
     p.dw_K = w.K;
     p.dw_out0 = (__nv_bfloat16*)w.out0; p.dw_out1 = (__nv_bfloat16*)w.out1;
     p.dw_out_f32 = w.out_f32;
+    p.dw_bias_col = w.bias0 ? w.N : -1;
+    p.dw_Nt = w.bias0 ? w.N + 1 : w.N;
+    p.dw_bias0 = (__nv_bfloat16*)w.bias0; p.dw_bias1 = (__nv_bfloat16*)w.bias1;
+    const int b_ld = w.b_ld > 0 ? w.b_ld : w.N;
+    if (w.bias0 && b_ld < w.N + 1) return cudaErrorInvalidValue;
     bool ok = make_map(&p.tmA[0], w.a, (uint64_t)w.M, (uint64_t)w.a_rows, w.a3d ? w.groups : 1, 64, BK, w.a3d);
-    ok &= make_map(&p.tmB[0], w.b, (uint64_t)w.N, (uint64_t)w.b_rows, w.b3d ? w.groups : 1, 64, BK, w.b3d);
+    ok &= make_map(&p.tmB[0], w.b, (uint64_t)b_ld, (uint64_t)w.b_rows, w.b3d ? w.groups : 1, 64, BK, w.b3d);
     if (!ok) return cudaErrorInvalidValue;
-    const long long tiles = (long long)w.groups * ceil_div(w.M, BM) * ceil_div(w.N, 256);
+    const long long tiles = (long long)w.groups * ceil_div(w.M, BM) * ceil_div(p.dw_Nt, 256);
     return launch<DW, 8>(p, (int)(tiles < num_sms() ? tiles : num_sms()), stream);
 }
 

@@ -141,6 +141,9 @@ cudaError_t launch_tc_gemm2_routed_q8(const Dims& D, const int32_t* offsets, con
 // ---- backward ----------------------------------------------------------------------
 // Buffers of one backward call.  Routed rows of the weight-gradient operands (dout_pad, x_pad,
 // dag, hg) are grouped by expert in 64-row-padded groups starting at offs_pad[e] (pad rows zero).
+// x_pad rows are d + 64 long and hg / hg_s rows I + 64 / I_s + 64: the first extra column holds 1
+// (x_pad, live rows; hg_s) or the slot's gate (hg), so the weight-gradient GEMMs also produce
+// the bias gradients (sum over rows of dag, resp. of gate * dout).
 struct BwdBufs {
     const int32_t *offsets, *offs_pad, *ts_dh, *ts_dx;
     const float* sorted_gate;
@@ -159,6 +162,9 @@ struct BwdBufs {
 // into 2-D operands, or null with K rows per group (3-D operands index the group, 2-D ones are
 // shared by all groups).  kind 0: out0 [groups][M][N]; 1: rows < M/2 -> out0, the rest -> out1
 // (each [groups][M/2][N]); 2: out_f32 [groups][M][N].
+// With bias0 set, B has a column N (its rows' weights: the gate, or 1) whose output column is a
+// bias gradient: out column N -> bias0[g][M] (kind 1: rows < M/2 -> bias0[g][M/2], the rest ->
+// bias1); b_ld is B's row length (>= N + 1 then; 0 means N).
 struct DwSpec {
     int kind, groups, M, N;
     const void* a; long long a_rows; int a3d;
@@ -166,6 +172,8 @@ struct DwSpec {
     const int32_t* rows; int K;
     void *out0, *out1;
     float* out_f32;
+    int b_ld;
+    void *bias0, *bias1;
 };
 cudaError_t launch_router_logits(const Dims& D, const void* x, const void* centroids, float* z, uint32_t* err,
                                  cudaStream_t stream);
@@ -181,14 +189,16 @@ cudaError_t launch_plan_bwd(const Dims& D, const int32_t* offsets, int32_t* offs
 // padded grouped rows of dout and x, the padded gate column, and b2dot[p] = <dout_t, b2_e> (b2 may be null)
 cudaError_t launch_bwd_gather(const Dims& D, const void* dout, const void* x, const void* b2, const int32_t* offsets,
                               const int32_t* offs_pad, const int32_t* stok, const float* sgate, void* dout_pad,
-                              void* x_pad, float* gate_pad, float* b2dot, uint32_t* err, cudaStream_t stream);
+                              void* x_pad, void* hg, float* gate_pad, float* b2dot, uint32_t* err, cudaStream_t stream);
 // gate gradients -> logit gradients dz [T][N_m] (fp32 and bf16); dgate_out [T][k] optional
 cudaError_t launch_router_bwd(const Dims& D, const float* z, const float* bias, const int32_t* idx,
                               const int32_t* slot_of, const float* dgate_part, int n_parts, const float* b2dot,
                               float* dz, void* dz_bf16, float* dgate_out, cudaStream_t stream);
-// grouped, weighted column sums (bias gradients); see backward.cu
-cudaError_t launch_colsum(bool src_f32, bool out_f32, const void* src, long long group_stride, int ld,
-                          const int32_t* starts, int n_rows, const float* w, int groups, int W, int split, void* out0,
-                          void* out1, cudaStream_t stream);
+// column sums over n_rows rows of each group (two passes through partial [groups][ceil(n_rows/256)][W]
+// fp32, deterministic); see backward.cu
+cudaError_t launch_colsum(bool src_f32, bool out_f32, const void* src, long long group_stride, int ld, int n_rows,
+                          int groups, int W, int split, void* out0, void* out1, float* partial, cudaStream_t stream);
+// rows[r][col] = 1 and rows[r][col + 1 .. col + 63] = 0 (bf16), r < n_rows
+cudaError_t launch_fill_aug(void* rows, long long n_rows, int ld, int col, cudaStream_t stream);
 
 }  // namespace moe

@@ -78,7 +78,7 @@ CtxLayout ctx_layout(const Dims& D) {
 // Backward workspace.
 struct BwdLayout {
     size_t err, offs_pad, ts_dh, ts_dx, dout_pad, x_pad, gate_pad, b2dot, z, dgate_part, dag, hg, dag_s, hg_s, dz,
-        dz_bf16, dx_slot, base, total;
+        dz_bf16, dx_slot, base, cpart, total;
     long long S_pad_max;
     int n_parts;
 };
@@ -95,19 +95,20 @@ BwdLayout bwd_layout(const Dims& D) {
     B.ts_dh = o; o += al((size_t)(D.E + D.Ks + 1) * 4);
     B.ts_dx = o; o += al((size_t)(D.E + 1) * 4);
     B.dout_pad = o; o += al(Sp * D.d * 2);
-    B.x_pad = o; o += al(Sp * D.d * 2);
+    B.x_pad = o; o += al(Sp * (D.d + 64) * 2);           // + the bias-gradient column block
     B.gate_pad = o; o += al(Sp * 4);
     B.b2dot = o; o += al(S * 4);
     B.z = o; o += al((size_t)D.T * D.E * 4);
     B.dgate_part = o; o += al(S * B.n_parts * 4);
     B.dag = o; o += al(Sp * 2 * D.I * 2);
-    B.hg = o; o += al(Sp * D.I * 2);
+    B.hg = o; o += al(Sp * (D.I + 64) * 2);
     B.dag_s = o; o += al((size_t)D.Ks * D.T * 2 * Is * 2);
-    B.hg_s = o; o += al((size_t)D.Ks * D.T * Is * 2);
+    B.hg_s = o; o += al((size_t)D.Ks * D.T * (D.Ks ? Is + 64 : 0) * 2);
     B.dz = o; o += al((size_t)D.T * D.E * 4);
     B.dz_bf16 = o; o += al((size_t)D.T * D.E * 2);
     B.dx_slot = o; o += al(S * D.d * 2);
     B.base = o; o += al((size_t)D.T * D.d * 4);
+    B.cpart = o; o += al((size_t)(D.Ks * 2 * Is + D.E) * ((D.T + 255) / 256) * 4);   // column-sum partials
     B.total = o;
     return B;
 }
@@ -569,8 +570,9 @@ moe_status_t layer_backward_impl(const moe_shape_t* shape, const void* x, const 
     if (!mark(0)) return MOE_ERR_CUDA;
     MOE_CUDA(launch_plan_bwd(D, offsets, const_cast<int32_t*>(B.offs_pad), const_cast<int32_t*>(B.ts_dh),
                              const_cast<int32_t*>(B.ts_dx), st));
-    MOE_CUDA(launch_bwd_gather(D, dout, x, R.b2, offsets, B.offs_pad, stok, sgate, B.dout_pad, B.x_pad, gate_pad, b2dot,
-                               err, st));
+    MOE_CUDA(launch_bwd_gather(D, dout, x, R.b2, offsets, B.offs_pad, stok, sgate, B.dout_pad, B.x_pad, B.hg, gate_pad,
+                               b2dot, err, st));
+    if (D.Ks > 0) MOE_CUDA(launch_fill_aug(B.hg_s, (long long)D.Ks * D.T, D.Is + 64, D.Is, st));
     MOE_CUDA(launch_router_logits(D, x, centroids, z, err, st));
     if (!mark(1)) return MOE_ERR_CUDA;
     MOE_CUDA(launch_tc_dh(D, B, R, Sh, dout, err, st));
@@ -582,39 +584,35 @@ moe_status_t layer_backward_impl(const moe_shape_t* shape, const void* x, const 
     MOE_CUDA(launch_tc_dxs(D, B, Sh, centroids, err, st));
     MOE_CUDA(launch_combine(D, B.dx_slot, slot_of, B.base, dx, err, st));
     if (!mark(4)) return MOE_ERR_CUDA;
-    // weight gradients
+    // weight gradients; the routed experts' and the shared experts' w2 bias gradients come out of
+    // the same GEMMs through the extra B column (gate, resp. 1)
     const long long T = D.T;
+    void* nb = nullptr;
     DwSpec w2 = {0, D.E, D.d, D.I, B.dout_pad, L.S_pad_max, 0, B.hg, L.S_pad_max, 0, B.offs_pad, 0,
-                 groutes->w2, nullptr, nullptr};
+                 groutes->w2, nullptr, nullptr, D.I + 64, D.bias ? groutes->b2 : nb, nullptr};
     MOE_CUDA(launch_tc_dw(D, w2, err, st));
     if (!mark(5)) return MOE_ERR_CUDA;
     DwSpec w13 = {1, D.E, 2 * D.I, D.d, B.dag, L.S_pad_max, 0, B.x_pad, L.S_pad_max, 0, B.offs_pad, 0,
-                  groutes->w1, groutes->w3, nullptr};
+                  groutes->w1, groutes->w3, nullptr, D.d + 64, D.bias ? groutes->b1 : nb, D.bias ? groutes->b3 : nb};
     MOE_CUDA(launch_tc_dw(D, w13, err, st));
     if (!mark(6)) return MOE_ERR_CUDA;
+    float* cpart = at<float>(ws, L.cpart);
     if (D.Ks > 0) {
-        DwSpec s2 = {0, D.Ks, D.d, D.Is, dout, T, 0, B.hg_s, T, 1, nullptr, D.T, gshared->w2, nullptr, nullptr};
+        DwSpec s2 = {0, D.Ks, D.d, D.Is, dout, T, 0, B.hg_s, T, 1, nullptr, D.T, gshared->w2, nullptr, nullptr,
+                     D.Is + 64, D.bias ? gshared->b2 : nb, nullptr};
         MOE_CUDA(launch_tc_dw(D, s2, err, st));
-        DwSpec s13 = {1, D.Ks, 2 * D.Is, D.d, B.dag_s, T, 1, x, T, 0, nullptr, D.T, gshared->w1, gshared->w3, nullptr};
+        DwSpec s13 = {1, D.Ks, 2 * D.Is, D.d, B.dag_s, T, 1, x, T, 0, nullptr, D.T, gshared->w1, gshared->w3, nullptr,
+                      0, nullptr, nullptr};
         MOE_CUDA(launch_tc_dw(D, s13, err, st));
+        if (D.bias)
+            MOE_CUDA(launch_colsum(false, false, B.dag_s, (long long)D.T * 2 * D.Is, 2 * D.Is, D.T, D.Ks, 2 * D.Is, D.Is,
+                                   gshared->b1, gshared->b3, cpart, st));
     }
-    DwSpec dc = {2, 1, D.E, D.d, B.dz_bf16, T, 0, x, T, 0, nullptr, D.T, nullptr, nullptr, dcentroids};
+    DwSpec dc = {2, 1, D.E, D.d, B.dz_bf16, T, 0, x, T, 0, nullptr, D.T, nullptr, nullptr, dcentroids, 0, nullptr,
+                 nullptr};
     MOE_CUDA(launch_tc_dw(D, dc, err, st));
-    // bias gradients (deterministic column sums)
-    if (D.bias) {
-        MOE_CUDA(launch_colsum(false, false, B.dout_pad, 0, D.d, B.offs_pad, 0, gate_pad, D.E, D.d, D.d, groutes->b2,
-                               nullptr, st));
-        MOE_CUDA(launch_colsum(false, false, B.dag, 0, 2 * D.I, B.offs_pad, 0, nullptr, D.E, 2 * D.I, D.I, groutes->b1,
-                               groutes->b3, st));
-        if (D.Ks > 0) {
-            MOE_CUDA(launch_colsum(false, false, dout, 0, D.d, nullptr, D.T, nullptr, D.Ks, D.d, D.d, gshared->b2,
-                                   nullptr, st));
-            MOE_CUDA(launch_colsum(false, false, B.dag_s, (long long)D.T * 2 * D.Is, 2 * D.Is, nullptr, D.T, nullptr,
-                                   D.Ks, 2 * D.Is, D.Is, gshared->b1, gshared->b3, st));
-        }
-    }
     if (drouter_bias)
-        MOE_CUDA(launch_colsum(true, true, dz, 0, D.E, nullptr, D.T, nullptr, 1, D.E, D.E, drouter_bias, nullptr, st));
+        MOE_CUDA(launch_colsum(true, true, dz, 0, D.E, D.T, 1, D.E, D.E, drouter_bias, nullptr, cpart, st));
     if (!mark(7)) return MOE_ERR_CUDA;
     return MOE_OK;
 }
@@ -696,9 +694,9 @@ MOE_EXPORT int32_t moe_backward_launches(const moe_shape_t* shape) {
     if (to_dims(shape, &D) != MOE_OK || check_train(D) != MOE_OK) return -1;
     if (D.T == 0) return 0;
     int n = 3 + 1 + 1 + 3 + 2 + 1;            // plan, gather, logits; DH; router bwd; DX, DXS, combine; dW2, dW13; dC
-    if (D.Ks > 0) n += 2;                      // shared dW2, dW13
-    if (D.bias) n += 2 + (D.Ks > 0 ? 2 : 0);   // routed db2, db1|db3 (+ shared)
-    return n;                                  // (+1 when a router-bias gradient is asked for)
+    if (D.Ks > 0) n += 3;                      // hg_s bias column, shared dW2, dW13
+    if (D.bias && D.Ks > 0) n += 2;            // shared db1 | db3 column sums (two passes)
+    return n;                                  // (+2 when a router-bias gradient is asked for)
 }
 
 }  // extern "C"

@@ -324,7 +324,7 @@ moe_status_t moe_layer_backward_timed(const moe_shape_t* shape, const void* x, c
                                       void* ws, size_t ws_bytes, moe_stream_t stream, void* const* stage_events,
                                       int32_t n_events);
 
-/* Kernel launches of one moe_layer_backward call without a router-bias gradient (one more with
+/* Kernel launches of one moe_layer_backward call without a router-bias gradient (two more with
  * it); -1 for an unsupported shape, 0 when T == 0. */
 int32_t moe_backward_launches(const moe_shape_t* shape);
 
