@@ -574,11 +574,43 @@ __device__ __forceinline__ void epilogue_router(const Params& p, const Tile& x, 
     }
 }
 
+// Stores a warp's 32 x 32 bf16 chunk (lane = row, pk = its 32 columns packed in pairs) through a
+// per-warp shared-memory transpose, so that each store instruction writes 64 contiguous bytes of
+// eight rows instead of 16 bytes of 32 rows.  In shared memory row r keeps its four 16-byte pieces
+// rotated by r/2, which makes both the writes and the reads free of bank conflicts.  row_ptr is
+// this lane's destination row (already offset to column 0 of the chunk), or null to skip the row;
+// ncols (multiple of 8) limits the columns written.
+__device__ __forceinline__ void warp_store_chunk_bf16(uint32_t stage, const uint32_t (&pk)[16], __nv_bfloat16* row_ptr,
+                                                      int ncols, int lane) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const uint32_t a = stage + lane * 64 + (((j + (lane >> 1)) & 3) << 4);
+        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(pk[4 * j]), "r"(pk[4 * j + 1]),
+                     "r"(pk[4 * j + 2]), "r"(pk[4 * j + 3])
+                     : "memory");
+    }
+    __syncwarp();
+    const int j = lane & 3;
+#pragma unroll
+    for (int sgrp = 0; sgrp < 4; ++sgrp) {
+        const int r = sgrp * 8 + (lane >> 2);
+        __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(
+            __shfl_sync(0xffffffffu, reinterpret_cast<unsigned long long>(row_ptr), r));
+        uint4 v;
+        const uint32_t a = stage + r * 64 + (((j + (r >> 1)) & 3) << 4);
+        asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
+        if (dst && j * 8 < ncols) *reinterpret_cast<uint4*>(dst + j * 8) = v;
+    }
+    __syncwarp();
+}
+
 // GEMM1: the two epilogue warps of a TMEM lane quadrant split the 128 hidden columns.  On an
 // e4m3 routed tile (Q8) the accumulators are first multiplied by the row's activation scale
-// and the column's weight scale.
+// and the column's weight scale.  Rows are stored through the per-warp transpose (all lanes
+// take part; rows past the group's end pass a null row).
 template <bool Q8 = false>
-__device__ __forceinline__ void epilogue_gemm1(const Params& p, const Tile& x, uint32_t tacc, int row, int half) {
+__device__ __forceinline__ void epilogue_gemm1(const Params& p, const Tile& x, uint32_t tacc, int row, int half,
+                                               uint32_t stage, int lane) {
     const bool shared = x.g >= p.E;
     const int e = shared ? x.g - p.E : x.g;
     const int I = shared ? p.Is : p.I;
@@ -592,14 +624,10 @@ __device__ __forceinline__ void epilogue_gemm1(const Params& p, const Tile& x, u
     const int r = x.m0 + row;
     const bool live = r < x.rows;
     const float rs = (scaled && live) ? p.a_scale[x.row0 + r] : 1.f;
-    __nv_bfloat16* hrow = shared ? p.h_s + ((size_t)e * p.T + r) * I : p.h_r + (size_t)(x.row0 + r) * I;
-    __nv_bfloat16* arow = nullptr;
-    __nv_bfloat16* grow = nullptr;
-    if (p.a_out) {
-        const size_t o = shared ? ((size_t)e * p.T + r) * I : (size_t)(x.row0 + r) * I;
-        arow = (shared ? p.as_out : p.a_out) + o;
-        grow = (shared ? p.gs_out : p.g_out) + o;
-    }
+    const size_t ro = shared ? ((size_t)e * p.T + r) * I : (size_t)(x.row0 + r) * I;
+    __nv_bfloat16* hrow = live ? (shared ? p.h_s : p.h_r) + ro : nullptr;
+    __nv_bfloat16* arow = (live && p.a_out) ? (shared ? p.as_out : p.a_out) + ro : nullptr;
+    __nv_bfloat16* grow = (live && p.a_out) ? (shared ? p.gs_out : p.g_out) + ro : nullptr;
 #pragma unroll 1
     for (int c = half * 2; c < half * 2 + 2; ++c) {
         uint32_t u[32], v[32];
@@ -607,46 +635,43 @@ __device__ __forceinline__ void epilogue_gemm1(const Params& p, const Tile& x, u
         tmem_ld32(tacc + 128 + c * 32, v);
         tmem_wait_ld();
         const int col0 = x.n0 + c * 32;
-        if (!live || col0 >= I) continue;
+        if (col0 >= I) continue;                                // warp-uniform
+        const int ncols = min(32, I - col0);
+        uint32_t pk[16], pa[16], pg[16];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const int col = col0 + q * 8;
-            if (col >= I) break;
-            uint32_t pk[4], pa[4], pg[4];
+        for (int i = 0; i < 16; ++i) {
+            float hv[2], av[2], gv[2];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                float hv[2], av[2], gv[2];
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const int j = q * 8 + i * 2 + h;
-                    const int cc = col + i * 2 + h;
-                    float a = __uint_as_float(u[j]);
-                    float g = __uint_as_float(v[j]);
-                    if (scaled) { a *= rs * sc1[cc]; g *= rs * sc3[cc]; }
-                    a += b1 ? __bfloat162float(b1[cc]) : 0.f;
-                    g += b3 ? __bfloat162float(b3[cc]) : 0.f;
-                    hv[h] = silu_f32(a) * g;
-                    av[h] = a;
-                    gv[h] = g;
-                }
-                pk[i] = pack_bf16(hv[0], hv[1]);
-                pa[i] = pack_bf16(av[0], av[1]);
-                pg[i] = pack_bf16(gv[0], gv[1]);
+            for (int h = 0; h < 2; ++h) {
+                const int j = 2 * i + h;
+                const int cc = min(col0 + j, I - 1);
+                float a = __uint_as_float(u[j]);
+                float g = __uint_as_float(v[j]);
+                if (scaled) { a *= rs * sc1[cc]; g *= rs * sc3[cc]; }
+                a += b1 ? __bfloat162float(b1[cc]) : 0.f;
+                g += b3 ? __bfloat162float(b3[cc]) : 0.f;
+                hv[h] = silu_f32(a) * g;
+                av[h] = a;
+                gv[h] = g;
             }
-            *reinterpret_cast<uint4*>(hrow + col) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-            if (arow) {
-                *reinterpret_cast<uint4*>(arow + col) = make_uint4(pa[0], pa[1], pa[2], pa[3]);
-                *reinterpret_cast<uint4*>(grow + col) = make_uint4(pg[0], pg[1], pg[2], pg[3]);
-            }
+            pk[i] = pack_bf16(hv[0], hv[1]);
+            pa[i] = pack_bf16(av[0], av[1]);
+            pg[i] = pack_bf16(gv[0], gv[1]);
+        }
+        warp_store_chunk_bf16(stage, pk, hrow ? hrow + col0 : nullptr, ncols, lane);
+        if (p.a_out) {                                          // warp-uniform
+            warp_store_chunk_bf16(stage, pa, arow ? arow + col0 : nullptr, ncols, lane);
+            warp_store_chunk_bf16(stage, pg, grow ? grow + col0 : nullptr, ncols, lane);
         }
     }
 }
 
 // GEMM2R: each epilogue warp of a quadrant takes 128 of the 256 output columns.  On e4m3 tiles
 // (Q8) the accumulator is multiplied by the h row's scale and the column's weight scale before
-// b2 and the gate.
+// b2 and the gate.  Rows are stored through the per-warp transpose.
 template <bool Q8 = false>
-__device__ __forceinline__ void epilogue_gemm2r(const Params& p, const Tile& x, uint32_t tacc, int row, int half) {
+__device__ __forceinline__ void epilogue_gemm2r(const Params& p, const Tile& x, uint32_t tacc, int row, int half,
+                                                uint32_t stage, int lane) {
     const int r = x.m0 + row;
     const bool live = r < x.rows;
     const long long pos = x.row0 + r;
@@ -654,31 +679,27 @@ __device__ __forceinline__ void epilogue_gemm2r(const Params& p, const Tile& x, 
     const __nv_bfloat16* b2 = p.b2 ? p.b2 + (size_t)x.g * p.d : nullptr;
     const float* sc2 = Q8 ? p.ws2 + (size_t)x.g * p.d : nullptr;
     const float rs = (Q8 && live) ? p.a_scale[pos] : 1.f;
-    __nv_bfloat16* yrow = p.y + (size_t)pos * p.d;
+    __nv_bfloat16* yrow = live ? p.y + (size_t)pos * p.d : nullptr;
 #pragma unroll 1
     for (int c = half * 4; c < half * 4 + 4; ++c) {
         uint32_t u[32];
         tmem_ld32(tacc + c * 32, u);
         tmem_wait_ld();
         const int col0 = x.n0 + c * 32;
-        if (!live || col0 >= p.d) continue;
+        if (col0 >= p.d) continue;                              // warp-uniform
+        const int ncols = min(32, p.d - col0);
+        uint32_t pk[16];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const int col = col0 + q * 8;
-            if (col >= p.d) break;
-            uint32_t pk[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int j = q * 8 + i * 2;
-                float a = __uint_as_float(u[j]);
-                float b = __uint_as_float(u[j + 1]);
-                if (Q8) { a *= rs * sc2[col + i * 2]; b *= rs * sc2[col + i * 2 + 1]; }
-                a += b2 ? __bfloat162float(b2[col + i * 2]) : 0.f;
-                b += b2 ? __bfloat162float(b2[col + i * 2 + 1]) : 0.f;
-                pk[i] = pack_bf16(gate * a, gate * b);
-            }
-            *reinterpret_cast<uint4*>(yrow + col) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        for (int i = 0; i < 16; ++i) {
+            const int ca = min(col0 + 2 * i, p.d - 1), cb = min(col0 + 2 * i + 1, p.d - 1);
+            float a = __uint_as_float(u[2 * i]);
+            float b = __uint_as_float(u[2 * i + 1]);
+            if (Q8) { a *= rs * sc2[ca]; b *= rs * sc2[cb]; }
+            a += b2 ? __bfloat162float(b2[ca]) : 0.f;
+            b += b2 ? __bfloat162float(b2[cb]) : 0.f;
+            pk[i] = pack_bf16(gate * a, gate * b);
         }
+        warp_store_chunk_bf16(stage, pk, yrow ? yrow + col0 : nullptr, ncols, lane);
     }
 }
 
@@ -731,36 +752,6 @@ __device__ __forceinline__ void epilogue_router_partial(const Params& p, const T
     }
 }
 
-// Stores a warp's 32 x 32 bf16 chunk (lane = row, pk = its 32 columns packed in pairs) through a
-// per-warp shared-memory transpose, so that each store instruction writes 64 contiguous bytes of
-// eight rows instead of 16 bytes of 32 rows.  In shared memory row r keeps its four 16-byte pieces
-// rotated by r/2, which makes both the writes and the reads free of bank conflicts.  row_ptr is
-// this lane's destination row (already offset to column 0 of the chunk), or null to skip the row;
-// ncols (multiple of 8) limits the columns written.
-__device__ __forceinline__ void warp_store_chunk_bf16(uint32_t stage, const uint32_t (&pk)[16], __nv_bfloat16* row_ptr,
-                                                      int ncols, int lane) {
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        const uint32_t a = stage + lane * 64 + (((j + (lane >> 1)) & 3) << 4);
-        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(pk[4 * j]), "r"(pk[4 * j + 1]),
-                     "r"(pk[4 * j + 2]), "r"(pk[4 * j + 3])
-                     : "memory");
-    }
-    __syncwarp();
-    const int j = lane & 3;
-#pragma unroll
-    for (int sgrp = 0; sgrp < 4; ++sgrp) {
-        const int r = sgrp * 8 + (lane >> 2);
-        __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(
-            __shfl_sync(0xffffffffu, reinterpret_cast<unsigned long long>(row_ptr), r));
-        uint4 v;
-        const uint32_t a = stage + r * 64 + (((j + (r >> 1)) & 3) << 4);
-        asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
-        if (dst && j * 8 < ncols) *reinterpret_cast<uint4*>(dst + j * 8) = v;
-    }
-    __syncwarp();
-}
-
 // DH: for a routed group the rows are grouped slots (A = dout rows of the slot's token, in the
 // 64-row-padded layout), for a shared group the tokens.  Per element of the hidden row:
 // dh_raw = (dout . W2)[c]; a, g = the saved pre-activations; sg = sigmoid(a); h = a sg g;
@@ -768,7 +759,8 @@ __device__ __forceinline__ void warp_store_chunk_bf16(uint32_t stage, const uint
 // dh_raw h (the gate gradient, without its b2 term) over this thread's 128 columns.  Writes da | dg
 // and gate * h (the B operand of the w2 gradient); the padding rows of a routed group (up to the
 // next multiple of 64) get zeros, so the weight-gradient GEMMs can run whole 64-row K blocks.
-__device__ __forceinline__ void epilogue_dh(const Params& p, const Tile& x, uint32_t tacc, int row, int half) {
+__device__ __forceinline__ void epilogue_dh(const Params& p, const Tile& x, uint32_t tacc, int row, int half,
+                                            uint32_t stage, int lane) {
     const bool shared = x.g >= p.E;
     const int e = shared ? x.g - p.E : x.g;
     const int I = shared ? p.Is : p.I;
@@ -780,9 +772,13 @@ __device__ __forceinline__ void epilogue_dh(const Params& p, const Tile& x, uint
     const size_t so = shared ? ((size_t)e * p.T + r) * I : (size_t)pu * I;
     const __nv_bfloat16* arow = (shared ? p.as_sv : p.a_sv) + so;
     const __nv_bfloat16* grow = (shared ? p.gs_sv : p.g_sv) + so;
-    __nv_bfloat16* dagrow = shared ? p.dag_s + ((size_t)e * p.T + r) * 2 * I : p.dag + (size_t)pp * 2 * I;
-    // gate * h rows carry 64 extra columns (the bias-gradient column of the w2 gradient GEMM)
-    __nv_bfloat16* hgrow = shared ? p.hg_s + ((size_t)e * p.T + r) * (I + 64) : p.hg + (size_t)pp * (I + 64);
+    __nv_bfloat16* dagrow = nullptr;
+    __nv_bfloat16* hgrow = nullptr;
+    if (live || pad) {
+        dagrow = shared ? p.dag_s + ((size_t)e * p.T + r) * 2 * I : p.dag + (size_t)pp * 2 * I;
+        // gate * h rows carry 64 extra columns (the bias-gradient column of the w2 gradient GEMM)
+        hgrow = shared ? p.hg_s + ((size_t)e * p.T + r) * (I + 64) : p.hg + (size_t)pp * (I + 64);
+    }
     const float gate = (!shared && live) ? p.sorted_gate[pu] : 1.f;
     float dot = 0.f;
 #pragma unroll 1
@@ -791,68 +787,63 @@ __device__ __forceinline__ void epilogue_dh(const Params& p, const Tile& x, uint
         tmem_ld32(tacc + c * 32, u);
         tmem_wait_ld();
         const int col0 = x.n0 + c * 32;
-        if ((!live && !pad) || col0 >= I) continue;
+        if (col0 >= I) continue;                                // warp-uniform
+        uint32_t pda[16], pdg[16], phg[16];
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-            const int col = col0 + q * 8;
-            if (col >= I) break;
-            uint32_t pda[4] = {0, 0, 0, 0}, pdg[4] = {0, 0, 0, 0}, phg[4] = {0, 0, 0, 0};
+            uint4 av = make_uint4(0, 0, 0, 0), gv = make_uint4(0, 0, 0, 0);
             if (live) {
-                const uint4 av = *reinterpret_cast<const uint4*>(arow + col);
-                const uint4 gv = *reinterpret_cast<const uint4*>(grow + col);
-                const uint32_t aw[4] = {av.x, av.y, av.z, av.w}, gw[4] = {gv.x, gv.y, gv.z, gv.w};
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    float da2[2], dg2[2], hg2[2];
-#pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        const float a = __uint_as_float(h ? (aw[i] & 0xFFFF0000u) : (aw[i] << 16));
-                        const float g = __uint_as_float(h ? (gw[i] & 0xFFFF0000u) : (gw[i] << 16));
-                        const float dhr = __uint_as_float(u[q * 8 + i * 2 + h]);
-                        const float sg = 1.0f / (1.0f + expf(-a));
-                        const float si = a * sg;
-                        const float hv = si * g;
-                        dot += dhr * hv;
-                        const float dh = gate * dhr;
-                        da2[h] = dh * g * sg * (1.0f + a * (1.0f - sg));
-                        dg2[h] = dh * si;
-                        hg2[h] = gate * hv;
-                    }
-                    pda[i] = pack_bf16(da2[0], da2[1]);
-                    pdg[i] = pack_bf16(dg2[0], dg2[1]);
-                    phg[i] = pack_bf16(hg2[0], hg2[1]);
-                }
+                av = *reinterpret_cast<const uint4*>(arow + col0 + q * 8);
+                gv = *reinterpret_cast<const uint4*>(grow + col0 + q * 8);
             }
-            *reinterpret_cast<uint4*>(dagrow + col) = make_uint4(pda[0], pda[1], pda[2], pda[3]);
-            *reinterpret_cast<uint4*>(dagrow + I + col) = make_uint4(pdg[0], pdg[1], pdg[2], pdg[3]);
-            *reinterpret_cast<uint4*>(hgrow + col) = make_uint4(phg[0], phg[1], phg[2], phg[3]);
+            const uint32_t aw[4] = {av.x, av.y, av.z, av.w}, gw[4] = {gv.x, gv.y, gv.z, gv.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                float da2[2], dg2[2], hg2[2];
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const float a = __uint_as_float(h ? (aw[i] & 0xFFFF0000u) : (aw[i] << 16));
+                    const float g = __uint_as_float(h ? (gw[i] & 0xFFFF0000u) : (gw[i] << 16));
+                    const float dhr = live ? __uint_as_float(u[q * 8 + i * 2 + h]) : 0.f;
+                    const float sg = 1.0f / (1.0f + expf(-a));
+                    const float si = a * sg;
+                    const float hv = si * g;
+                    dot += dhr * hv;
+                    const float dh = gate * dhr;
+                    da2[h] = dh * g * sg * (1.0f + a * (1.0f - sg));
+                    dg2[h] = dh * si;
+                    hg2[h] = gate * hv;
+                }
+                pda[q * 4 + i] = pack_bf16(da2[0], da2[1]);
+                pdg[q * 4 + i] = pack_bf16(dg2[0], dg2[1]);
+                phg[q * 4 + i] = pack_bf16(hg2[0], hg2[1]);
+            }
         }
+        // I is a multiple of 64: whole chunks
+        warp_store_chunk_bf16(stage, pda, dagrow ? dagrow + col0 : nullptr, 32, lane);
+        warp_store_chunk_bf16(stage, pdg, dagrow ? dagrow + I + col0 : nullptr, 32, lane);
+        warp_store_chunk_bf16(stage, phg, hgrow ? hgrow + col0 : nullptr, 32, lane);
     }
     if (!shared && live) p.dgate_part[(size_t)pu * p.n_parts + (x.n0 / 256) * 2 + half] = dot;
 }
 
-// DX: dx of a routed slot (grouped order), bf16.
-__device__ __forceinline__ void epilogue_dx(const Params& p, const Tile& x, uint32_t tacc, int row, int half) {
+// DX: dx of a routed slot (grouped order), bf16, stored through the per-warp transpose.
+__device__ __forceinline__ void epilogue_dx(const Params& p, const Tile& x, uint32_t tacc, int row, int half,
+                                            uint32_t stage, int lane) {
     const int r = x.m0 + row;
     const bool live = r < x.rows;
-    __nv_bfloat16* orow = p.dx_slot + ((size_t)p.offsets[x.g] + r) * p.d;
+    __nv_bfloat16* orow = live ? p.dx_slot + ((size_t)p.offsets[x.g] + r) * p.d : nullptr;
 #pragma unroll 1
     for (int c = half * 4; c < half * 4 + 4; ++c) {
         uint32_t u[32];
         tmem_ld32(tacc + c * 32, u);
         tmem_wait_ld();
         const int col0 = x.n0 + c * 32;
-        if (!live || col0 >= p.d) continue;
+        if (col0 >= p.d) continue;                              // warp-uniform
+        uint32_t pk[16];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const int col = col0 + q * 8;
-            if (col >= p.d) break;
-            uint32_t pk[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-                pk[i] = pack_bf16(__uint_as_float(u[q * 8 + i * 2]), __uint_as_float(u[q * 8 + i * 2 + 1]));
-            *reinterpret_cast<uint4*>(orow + col) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-        }
+        for (int i = 0; i < 16; ++i) pk[i] = pack_bf16(__uint_as_float(u[2 * i]), __uint_as_float(u[2 * i + 1]));
+        warp_store_chunk_bf16(stage, pk, orow ? orow + col0 : nullptr, min(32, p.d - col0), lane);
     }
 }
 
@@ -1170,6 +1161,7 @@ __global__ void __launch_bounds__(THREADS, 1) moe_tc_kernel(const __grid_constan
     } else {
         // ------------------------------------------------------------------ epilogue
         const int quad = warp & 3;                  // TMEM lanes 32*quad .. 32*quad+31
+        const uint32_t stage_out = bar0 + 256 + (warp - 2) * STAGE_OUT_BYTES;   // this warp's transpose buffer
         const int half = (warp - 2) / 4;            // which half of the columns (0 or 1)
         const int row = (int)rank * BM + quad * 32 + lane;   // row inside the (pair) tile
         int acc = 0;
@@ -1184,16 +1176,16 @@ __global__ void __launch_bounds__(THREADS, 1) moe_tc_kernel(const __grid_constan
             } else if (MODE == ROUTERP) {
                 epilogue_router_partial(p, x, tacc, row, half);
             } else if (MODE == GEMM1) {
-                epilogue_gemm1<Q8>(p, x, tacc, row, half);
+                epilogue_gemm1<Q8>(p, x, tacc, row, half, stage_out, lane);
             } else if (MODE == GEMM2R) {
-                if (x.g >= 0) epilogue_gemm2r<Q8>(p, x, tacc, row, half);
+                if (x.g >= 0) epilogue_gemm2r<Q8>(p, x, tacc, row, half, stage_out, lane);
                 else epilogue_gemm2s(p, x, tacc, row, half);
             } else if (MODE == DH) {
-                epilogue_dh(p, x, tacc, row, half);
+                epilogue_dh(p, x, tacc, row, half, stage_out, lane);
             } else if (MODE == DX) {
-                epilogue_dx(p, x, tacc, row, half);
+                epilogue_dx(p, x, tacc, row, half, stage_out, lane);
             } else if (MODE == DW) {
-                epilogue_dw(p, x, tacc, row, half, bar0 + 256 + (warp - 2) * STAGE_OUT_BYTES, lane);
+                epilogue_dw(p, x, tacc, row, half, stage_out, lane);
             } else {
                 epilogue_gemm2s(p, x, tacc, row, half);
             }
