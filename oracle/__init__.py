@@ -8,5 +8,5 @@ from .moe_oracle import (  # noqa: F401
     linear_macs, linear_params, expert_macs, expert_params, hit_entropy, n_routings,
     split_expert, GATE_SOFTMAX_TOPK, GATE_TOPK_SOFTMAX, GATE_SIGMOID_BIAS,
     E4M3_MAX, e4m3_decode, e4m3_round, bf16_round, quantize_rows_e4m3, dequantized_rows, e4m3_weights,
-    silu_grad, expert_backward, gate_backward, layer_backward, balance_stats,
+    silu_grad, expert_backward, gate_backward, layer_backward, balance_stats, balance_scores,
 )

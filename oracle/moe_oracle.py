@@ -472,6 +472,24 @@ def layer_backward(x: np.ndarray, centroids: np.ndarray, routed: ExpertSource, n
             "dgate": dgate, "dz": dz, "idx": idx, "gate": gate}
 
 
+def balance_scores(x: np.ndarray, centroids: np.ndarray, gate_mode: int = GATE_SOFTMAX_TOPK,
+                   bias: Optional[np.ndarray] = None) -> np.ndarray:
+    """The per-token score distribution over all N_m experts that the balance statistics average
+    (a reading; the pages name "the mean of each expert's gate scores" only): gate modes 0 and 1,
+    softmax of the (biased) logits over all experts; mode 2, the sigmoid scores divided by their
+    sum over all experts (the routing bias only selects, so it is left out).  Rows sum to 1."""
+    x = np.asarray(x, np.float64)
+    c = np.asarray(centroids, np.float64)
+    z = x @ c.T
+    if gate_mode == GATE_SIGMOID_BIAS:
+        sg = _sigmoid(z)
+        return sg / sg.sum(axis=1, keepdims=True)
+    if bias is not None:
+        z = z + np.asarray(bias, np.float64)
+    e = np.exp(z - z.max(axis=1, keepdims=True))
+    return e / e.sum(axis=1, keepdims=True)
+
+
 def balance_stats(s: np.ndarray, idx: np.ndarray, n_experts: int, top_k: int, n_groups: int = 1):
     """Expert- and device-level balance statistics of one batch (DeepSeekMoE report §2.5 and §3:
     per expert, the batch mean of its gate scores and its hit rate; losses that penalise their

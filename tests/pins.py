@@ -602,6 +602,16 @@ def check_balance_stats(O):
     assert abs(br["f"].sum() - N) < 1e-12 and abs(br["P"].sum() - 1.0) < 1e-12
     assert np.array_equal(br["counts"], O.hit_entropy(idx_r, N)[2])
     assert abs(br["device_term"] - br["f"].mean() * 1.0) < 1e-12            # one group: f' = mean f, P' = 1
+    # the score distributions: rows sum to 1; mode 0 equals the router's softmax, mode 2 the
+    # normalised expit
+    xx = rng.normal(0, 1, (9, 5)); cc = rng.normal(0, 1, (N, 5)); bb = rng.normal(0, 1, N)
+    for mode in (0, 1, 2):
+        sc = O.balance_scores(xx, cc, mode, bb)
+        assert np.allclose(sc.sum(axis=1), 1.0, rtol=0, atol=1e-14) and (sc > 0).all()
+    assert np.allclose(O.balance_scores(xx, cc, 0, bb), scipy.special.softmax(xx @ cc.T + bb, axis=1), rtol=1e-13)
+    assert np.allclose(O.balance_scores(xx, cc, 0, bb), O.route(xx, cc, 2, 0, bb)["s"], rtol=1e-13)
+    e2 = scipy.special.expit(xx @ cc.T)
+    assert np.allclose(O.balance_scores(xx, cc, 2, bb), e2 / e2.sum(1, keepdims=True), rtol=1e-13)
 
 
 ALL_CHECKS = [check_ptflops_printout, check_combinations, check_textbook_single_expert,
