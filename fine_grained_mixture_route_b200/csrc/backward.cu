@@ -288,7 +288,74 @@ __global__ void fill_aug_kernel(__nv_bfloat16* rows, long long n_rows, int ld, i
     }
 }
 
+// One warp per token: the row of router logits z (fp32, in place) becomes the score
+// distribution the balance statistics average: softmax of z + bias (gate modes 0, 1) or
+// sigmoid(z) normalised over the experts (mode 2).
+__global__ void balance_scores_kernel(float* z, const float* __restrict__ bias, int T, int E, int mode) {
+    const int lane = threadIdx.x & 31;
+    const int warps = gridDim.x * (blockDim.x >> 5);
+    for (int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < T; t += warps) {
+        float* zr = z + (size_t)t * E;
+        if (mode == 2) {
+            float sum = 0.f;
+            for (int i = lane; i < E; i += 32) sum += 1.0f / (1.0f + expf(-zr[i]));
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+            __syncwarp();
+            for (int i = lane; i < E; i += 32) zr[i] = (1.0f / (1.0f + expf(-zr[i]))) / sum;
+        } else {
+            float m = -INFINITY;
+            for (int i = lane; i < E; i += 32) m = fmaxf(m, zr[i] + (bias ? bias[i] : 0.f));
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+            float sum = 0.f;
+            for (int i = lane; i < E; i += 32) sum += expf(zr[i] + (bias ? bias[i] : 0.f) - m);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+            __syncwarp();
+            for (int i = lane; i < E; i += 32) zr[i] = expf(zr[i] + (bias ? bias[i] : 0.f) - m) / sum;
+        }
+    }
+}
+
+// f_i = N_m / (N_r T) * counts_i, P_i = Psum_i / T, terms[0] = sum_i f_i P_i, terms[1] = sum over
+// n_groups equal contiguous groups of mean(f) * sum(P).  One block, fixed summation order.
+__global__ void balance_final_kernel(const float* __restrict__ psum, const int32_t* __restrict__ counts, int T, int E,
+                                     int k, int n_groups, float* f, float* P, float* terms) {
+    __shared__ float fs[1024], ps[1024];
+    for (int i = threadIdx.x; i < E; i += blockDim.x) {
+        const float fi = (float)counts[i] * (float)E / ((float)k * (float)T);
+        const float pi = psum[i] / (float)T;
+        f[i] = fi; P[i] = pi; fs[i] = fi; ps[i] = pi;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        float te = 0.f, td = 0.f;
+        for (int i = 0; i < E; ++i) te += fs[i] * ps[i];
+        const int per = E / n_groups;
+        for (int g = 0; g < n_groups; ++g) {
+            float fg = 0.f, pg = 0.f;
+            for (int i = g * per; i < (g + 1) * per; ++i) { fg += fs[i]; pg += ps[i]; }
+            td += (fg / (float)per) * pg;
+        }
+        terms[0] = te;
+        terms[1] = td;
+    }
+}
+
 }  // namespace
+
+cudaError_t launch_balance(const Dims& D, float* z, const float* bias, const int32_t* counts, int n_groups,
+                           float* partial, float* psum, float* f, float* P, float* terms, cudaStream_t stream) {
+    if (D.T == 0) return cudaSuccess;
+    const long long need = (D.T + 7) / 8, cap = (long long)num_sms() * 8;
+    balance_scores_kernel<<<(int)(need < cap ? need : cap), 256, 0, stream>>>(
+        z, D.gate_mode == MOE_GATE_SIGMOID_BIAS ? nullptr : bias, D.T, D.E, D.gate_mode);
+    cudaError_t e = launch_colsum(true, true, z, 0, D.E, D.T, 1, D.E, D.E, psum, nullptr, partial, stream);
+    if (e != cudaSuccess) return e;
+    balance_final_kernel<<<1, 256, 0, stream>>>(psum, counts, D.T, D.E, D.k, n_groups, f, P, terms);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_plan_bwd(const Dims& D, const int32_t* offsets, int32_t* offs_pad, int32_t* ts_dh, int32_t* ts_dx,
                             cudaStream_t stream) {

@@ -198,6 +198,10 @@ cudaError_t launch_router_bwd(const Dims& D, const float* z, const float* bias, 
 // fp32, deterministic); see backward.cu
 cudaError_t launch_colsum(bool src_f32, bool out_f32, const void* src, long long group_stride, int ld, int n_rows,
                           int groups, int W, int split, void* out0, void* out1, float* partial, cudaStream_t stream);
+// balance statistics from the router logits z [T][N_m] (turned into scores in place) and the hit
+// counts: f, P [N_m], terms [2] (expert-level, device-level over n_groups)
+cudaError_t launch_balance(const Dims& D, float* z, const float* bias, const int32_t* counts, int n_groups,
+                           float* partial, float* psum, float* f, float* P, float* terms, cudaStream_t stream);
 // rows[r][col] = 1 and rows[r][col + 1 .. col + 63] = 0 (bf16), r < n_rows
 cudaError_t launch_fill_aug(void* rows, long long n_rows, int ld, int col, cudaStream_t stream);
 

@@ -699,4 +699,33 @@ MOE_EXPORT int32_t moe_backward_launches(const moe_shape_t* shape) {
     return n;                                  // (+2 when a router-bias gradient is asked for)
 }
 
+MOE_EXPORT size_t moe_balance_workspace_bytes(const moe_shape_t* shape) {
+    Dims D;
+    if (to_dims(shape, &D) != MOE_OK || !D.bf16 || !tc_router_supported(D)) return 0;
+    return 256 + al((size_t)D.T * D.E * 4) + al((size_t)D.E * ((D.T + 255) / 256) * 4) + al((size_t)D.E * 4);
+}
+
+MOE_EXPORT moe_status_t moe_balance_stats(const moe_shape_t* shape, const void* x, const void* centroids,
+                                          const float* router_bias, const int32_t* counts, int32_t n_groups, float* f,
+                                          float* P, float* terms, void* ws, size_t ws_bytes, moe_stream_t stream) {
+    Dims D;
+    MOE_TRY(to_dims(shape, &D));
+    if (!D.bf16 || !tc_router_supported(D)) return MOE_ERR_UNSUPPORTED;
+    if (!x || !centroids || !counts || !f || !P || !terms) return MOE_ERR_INVALID_ARG;
+    if (n_groups < 1 || D.E % n_groups || D.E > 1024) return MOE_ERR_INVALID_ARG;
+    const size_t need = moe_balance_workspace_bytes(shape);
+    if (!ws || ws_bytes < need || ((uintptr_t)ws & 15u)) return MOE_ERR_WORKSPACE;
+    if (D.T == 0) return MOE_OK;
+    MOE_TRY(check_device());
+    cudaGetLastError();
+    cudaStream_t st = (cudaStream_t)stream;
+    size_t o = 256;
+    float* z = at<float>(ws, o); o += al((size_t)D.T * D.E * 4);
+    float* partial = at<float>(ws, o); o += al((size_t)D.E * ((D.T + 255) / 256) * 4);
+    float* psum = at<float>(ws, o);
+    MOE_CUDA(launch_router_logits(D, x, centroids, z, at<uint32_t>(ws, 0), st));
+    MOE_CUDA(launch_balance(D, z, router_bias, counts, n_groups, partial, psum, f, P, terms, st));
+    return MOE_OK;
+}
+
 }  // extern "C"

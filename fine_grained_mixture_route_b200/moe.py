@@ -23,7 +23,8 @@ EXPORTED = ("moe_workspace_bytes", "moe_layer_launches", "moe_status_string", "m
             "moe_route", "moe_permute", "moe_expert_ffn", "moe_combine", "moe_layer_forward",
             "moe_layer_forward_timed", "moe_permute_no_alloc", "moe_quantize_rows_e4m3", "moe_train_ctx_bytes",
             "moe_backward_workspace_bytes", "moe_layer_forward_train", "moe_layer_backward",
-            "moe_layer_backward_timed", "moe_backward_launches")
+            "moe_layer_backward_timed", "moe_backward_launches", "moe_balance_workspace_bytes",
+            "moe_balance_stats")
 NUM_STAGES = 7
 STAGE_NAMES = ("router", "permute", "plan", "gather", "gemm1_swiglu", "gemm2", "combine")
 BWD_STAGES = 7
@@ -92,11 +93,14 @@ def _lib():
         lib.moe_layer_backward.argtypes = [sh, vp, vp, f32p, wp, wp, vp, vp, sz, vp, f32p, f32p, gp, gp, vp, sz, vp]
         lib.moe_layer_backward_timed.argtypes = [sh, vp, vp, f32p, wp, wp, vp, vp, sz, vp, f32p, f32p, gp, gp, vp, sz,
                                                  vp, ctypes.POINTER(ctypes.c_void_p), ctypes.c_int32]
+        lib.moe_balance_workspace_bytes.argtypes = [sh]
+        lib.moe_balance_workspace_bytes.restype = sz
+        lib.moe_balance_stats.argtypes = [sh, vp, vp, f32p, i32p, ctypes.c_int32, f32p, f32p, f32p, vp, sz, vp]
         lib.moe_backward_launches.argtypes = [sh]
         lib.moe_backward_launches.restype = ctypes.c_int32
         for n in ("moe_check_device_error", "moe_ws_init", "moe_route", "moe_permute", "moe_expert_ffn",
                   "moe_combine", "moe_layer_forward", "moe_layer_forward_timed", "moe_quantize_rows_e4m3",
-                  "moe_layer_forward_train", "moe_layer_backward", "moe_layer_backward_timed"):
+                  "moe_layer_forward_train", "moe_layer_backward", "moe_layer_backward_timed", "moe_balance_stats"):
             getattr(lib, n).restype = ctypes.c_int
         _LIB = lib
     return _LIB
@@ -330,6 +334,23 @@ def layer_backward(shape: MoeShape, x, centroids, routed: Dict, shared: Optional
         arr = (ctypes.c_void_p * len(events))(*[e.cuda_event for e in events])
         _check(_lib().moe_layer_backward_timed(*args, arr, len(events)), "moe_layer_backward_timed")
     return g
+
+
+def balance_stats(shape: MoeShape, x, centroids, counts, n_groups: int = 1, router_bias=None, ws=None, stream=None):
+    """moe_balance_stats: returns {f, P (fp32 [n_experts]), expert_term, device_term (0-d fp32)}."""
+    n = int(_lib().moe_balance_workspace_bytes(ctypes.byref(shape)))
+    if n == 0:
+        raise ValueError("layer shape not supported for balance statistics")
+    if ws is None or ws.numel() < n:
+        ws = torch.zeros(n, dtype=torch.uint8, device=x.device)
+    E = centroids.shape[0]
+    f = torch.empty(E, dtype=torch.float32, device=x.device)
+    P = torch.empty(E, dtype=torch.float32, device=x.device)
+    terms = torch.empty(2, dtype=torch.float32, device=x.device)
+    _check(_lib().moe_balance_stats(ctypes.byref(shape), _ptr(x), _ptr(centroids), _bias_ptr(router_bias),
+                                    _ptr(counts), n_groups, _ptr(f), _ptr(P), _ptr(terms), _ptr(ws), ws.numel(),
+                                    _stream(stream)), "moe_balance_stats")
+    return {"f": f, "P": P, "expert_term": terms[0], "device_term": terms[1]}
 
 
 def stage_events(stream=None, n_stages: int = NUM_STAGES):

@@ -329,6 +329,26 @@ moe_status_t moe_layer_backward_timed(const moe_shape_t* shape, const void* x, c
 int32_t moe_backward_launches(const moe_shape_t* shape);
 
 /*
+ * Balance statistics of one batch, the quantities the expert- and device-level balance losses of
+ * the DeepSeekMoE report are built from (§2.5 and §3: per expert, the batch mean of its gate
+ * scores and its hit rate; the formulas are stripped from the page, so these are a reading):
+ *   f[i] = N_m / (N_r T) * counts[i]          (1 for every expert under uniform routing)
+ *   P[i] = mean over tokens of the score distribution s_t: softmax of the (biased) router logits
+ *          over all experts (gate modes 0, 1), or the sigmoid scores normalised over the experts
+ *          (mode 2)
+ *   terms[0] = sum_i f[i] P[i]                (expert level; a loss multiplies it by alpha1)
+ *   terms[1] = sum_g mean_{i in g} f[i] * sum_{i in g} P[i] over n_groups equal contiguous groups
+ *              of experts (device level; alpha2)
+ * counts [n_experts] int32 as moe_layer_forward's counts_out; f, P [n_experts], terms [2] fp32
+ * out.  Needs a bf16 layer with a tensor-core router (it recomputes the logits); fixed
+ * summation order (deterministic).  ws: moe_balance_workspace_bytes(shape) bytes.
+ */
+size_t moe_balance_workspace_bytes(const moe_shape_t* shape);
+moe_status_t moe_balance_stats(const moe_shape_t* shape, const void* x, const void* centroids,
+                               const float* router_bias, const int32_t* counts, int32_t n_groups, float* f, float* P,
+                               float* terms, void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
  * moe_permute_no_alloc — the paper has no counterpart to this entry point; it exists for
  * callers of this library that cannot allocate device memory.  moe_permute needs scratch
  * space, which it takes from the caller's workspace.  A caller that cannot call cudaMalloc

@@ -186,3 +186,20 @@ def test_training_entry_points_validate(lib):
         == moe.MOE_ERR_INVALID_ARG                                   # gate mode 2: the bias only selects
     sh0 = _shape(T=0)
     assert b(*args(sh=sh0, nc=moe.train_ctx_bytes(sh0), nb=moe.backward_workspace_bytes(sh0))) == moe.MOE_OK
+
+
+def test_balance_stats_validate(lib):
+    fake = ctypes.c_void_p(1 << 40)
+    S = ctypes.byref
+    sh = _shape()
+    n = lib.moe_balance_workspace_bytes(S(sh))
+    assert n >= 256 * 256 * 4                                   # the T x N_m score matrix at least
+    assert lib.moe_balance_workspace_bytes(S(_shape(dtype=moe.MOE_F32))) == 0
+    assert lib.moe_balance_workspace_bytes(S(_shape(n_experts=512))) == 0
+    q = lib.moe_balance_stats
+    assert q(S(sh), fake, fake, None, fake, 3, fake, fake, fake, fake, n, None) == moe.MOE_ERR_INVALID_ARG   # 3 !| 256
+    assert q(S(sh), fake, fake, None, fake, 0, fake, fake, fake, fake, n, None) == moe.MOE_ERR_INVALID_ARG
+    assert q(S(sh), fake, fake, None, None, 4, fake, fake, fake, fake, n, None) == moe.MOE_ERR_INVALID_ARG
+    assert q(S(sh), fake, fake, None, fake, 4, fake, fake, fake, fake, n - 1, None) == moe.MOE_ERR_WORKSPACE
+    assert q(S(_shape(dtype=moe.MOE_F32)), fake, fake, None, fake, 4, fake, fake, fake, fake, n, None) == \
+        moe.MOE_ERR_UNSUPPORTED
