@@ -847,14 +847,77 @@ __device__ __forceinline__ void epilogue_dx(const Params& p, const Tile& x, uint
     }
 }
 
+// Second half of warp_store_chunk_bf16 with the eight-row destinations precomputed: dst[sg] is the
+// row (sg * 8 + lane / 4) of the warp's 32 rows, already offset to this chunk's column 0.
+__device__ __forceinline__ void warp_store_chunk_pre(uint32_t stage, const uint32_t (&pk)[16],
+                                                     __nv_bfloat16* const (&dst)[4], int ncols, int lane) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const uint32_t a = stage + lane * 64 + (((j + (lane >> 1)) & 3) << 4);
+        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(pk[4 * j]), "r"(pk[4 * j + 1]),
+                     "r"(pk[4 * j + 2]), "r"(pk[4 * j + 3])
+                     : "memory");
+    }
+    __syncwarp();
+    const int j = lane & 3;
+#pragma unroll
+    for (int sgrp = 0; sgrp < 4; ++sgrp) {
+        const int r = sgrp * 8 + (lane >> 2);
+        uint4 v;
+        const uint32_t a = stage + r * 64 + (((j + (r >> 1)) & 3) << 4);
+        asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
+        if (dst[sgrp] && j * 8 < ncols) *reinterpret_cast<uint4*>(dst[sgrp] + j * 8) = v;
+    }
+    __syncwarp();
+}
+
 // DW: one 128 x 256 tile of a group's weight gradient (zeros when the group has no rows).  bf16
-// outputs go through the per-warp transpose (warp_store_chunk_bf16); column dw_N, when it is the
-// bias column, goes to the bias gradient.
+// outputs go through the per-warp transpose; the four chunks of a warp are loaded from tensor
+// memory one ahead of the one being stored.  Column dw_N, when it is the bias column, goes to
+// the bias gradient.
+__device__ __forceinline__ void dw_chunk(const Params& p, const Tile& x, const uint32_t (&u)[32], int c, int m,
+                                         bool live, int Mh, __nv_bfloat16* orow, float* frow,
+                                         __nv_bfloat16* const (&drow)[4], uint32_t stage, int lane) {
+    const int col0 = x.n0 + c * 32;
+    if (col0 >= p.dw_Nt) return;                               // warp-uniform
+    const bool zero = x.num_kb == 0;
+    if (live && p.dw_bias_col >= 0 && col0 + 32 > p.dw_N && col0 <= p.dw_N) {
+        // dw_N is a multiple of 64 (d, inter, inter_shared are) and chunks start at multiples of
+        // 32, so the bias column is the chunk's first column
+        const __nv_bfloat16 bv = __float2bfloat16_rn(zero ? 0.f : __uint_as_float(u[0]));
+        if (p.dw_kind == 1) {
+            if (m < Mh) p.dw_bias0[(size_t)x.g * Mh + m] = bv;
+            else p.dw_bias1[(size_t)x.g * Mh + m - Mh] = bv;
+        } else {
+            p.dw_bias0[(size_t)x.g * p.dw_M + m] = bv;
+        }
+    }
+    const int ncols = min(32, p.dw_N - col0);
+    if (ncols <= 0) return;                                     // warp-uniform
+    if (p.dw_kind == 2) {
+        if (!live) return;
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+            if (q * 4 < ncols)
+                *reinterpret_cast<float4*>(frow + col0 + q * 4) =
+                    zero ? make_float4(0.f, 0.f, 0.f, 0.f)
+                         : make_float4(__uint_as_float(u[q * 4]), __uint_as_float(u[q * 4 + 1]),
+                                       __uint_as_float(u[q * 4 + 2]), __uint_as_float(u[q * 4 + 3]));
+        return;
+    }
+    uint32_t pk[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+        pk[i] = zero ? 0u : pack_bf16(__uint_as_float(u[2 * i]), __uint_as_float(u[2 * i + 1]));
+    __nv_bfloat16* const dst[4] = {drow[0] ? drow[0] + col0 : nullptr, drow[1] ? drow[1] + col0 : nullptr,
+                                   drow[2] ? drow[2] + col0 : nullptr, drow[3] ? drow[3] + col0 : nullptr};
+    warp_store_chunk_pre(stage, pk, dst, ncols, lane);
+}
+
 __device__ __forceinline__ void epilogue_dw(const Params& p, const Tile& x, uint32_t tacc, int row, int half,
                                             uint32_t stage, int lane) {
     const int m = x.m0 + row;
     const bool live = m < p.dw_M;
-    const bool zero = x.num_kb == 0;
     const int Mh = p.dw_M / 2;
     __nv_bfloat16* orow = nullptr;
     float* frow = nullptr;
@@ -864,45 +927,26 @@ __device__ __forceinline__ void epilogue_dw(const Params& p, const Tile& x, uint
                                                : p.dw_out1 + ((size_t)x.g * Mh + m - Mh) * p.dw_N;
         else frow = p.dw_out_f32 + ((size_t)x.g * p.dw_M + m) * p.dw_N;
     }
-#pragma unroll 1
-    for (int c = half * 4; c < half * 4 + 4; ++c) {
-        uint32_t u[32];
-        tmem_ld32(tacc + c * 32, u);
-        tmem_wait_ld();
-        const int col0 = x.n0 + c * 32;
-        if (col0 >= p.dw_Nt) continue;                     // warp-uniform
-        if (zero) {
+    // destinations of the transposed stores: rows sg * 8 + lane / 4 of this warp's 32 rows
+    __nv_bfloat16* drow[4];
 #pragma unroll
-            for (int i = 0; i < 32; ++i) u[i] = 0u;
-        }
-        if (live && p.dw_bias_col >= 0 && col0 + 32 > p.dw_N && col0 <= p.dw_N) {
-            // dw_N is a multiple of 64 (d, inter, inter_shared are) and chunks start at multiples of
-            // 32, so the bias column is the chunk's first column
-            const __nv_bfloat16 bv = __float2bfloat16_rn(__uint_as_float(u[0]));
-            if (p.dw_kind == 1) {
-                if (m < Mh) p.dw_bias0[(size_t)x.g * Mh + m] = bv;
-                else p.dw_bias1[(size_t)x.g * Mh + m - Mh] = bv;
-            } else {
-                p.dw_bias0[(size_t)x.g * p.dw_M + m] = bv;
-            }
-        }
-        const int ncols = min(32, p.dw_N - col0);
-        if (ncols <= 0) continue;                          // warp-uniform
-        if (p.dw_kind == 2) {
-            if (!live) continue;
-#pragma unroll
-            for (int q = 0; q < 8; ++q)
-                if (q * 4 < ncols)
-                    *reinterpret_cast<float4*>(frow + col0 + q * 4) =
-                        make_float4(__uint_as_float(u[q * 4]), __uint_as_float(u[q * 4 + 1]),
-                                    __uint_as_float(u[q * 4 + 2]), __uint_as_float(u[q * 4 + 3]));
-        } else {
-            uint32_t pk[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i) pk[i] = pack_bf16(__uint_as_float(u[2 * i]), __uint_as_float(u[2 * i + 1]));
-            warp_store_chunk_bf16(stage, pk, orow ? orow + col0 : nullptr, ncols, lane);
-        }
-    }
+    for (int sg = 0; sg < 4; ++sg)
+        drow[sg] = reinterpret_cast<__nv_bfloat16*>(
+            __shfl_sync(0xffffffffu, reinterpret_cast<unsigned long long>(orow), sg * 8 + (lane >> 2)));
+    uint32_t ua[32], ub[32];
+    const int c0 = half * 4;
+    tmem_ld32(tacc + c0 * 32, ua);
+    tmem_wait_ld();
+    tmem_ld32(tacc + (c0 + 1) * 32, ub);
+    dw_chunk(p, x, ua, c0, m, live, Mh, orow, frow, drow, stage, lane);
+    tmem_wait_ld();
+    tmem_ld32(tacc + (c0 + 2) * 32, ua);
+    dw_chunk(p, x, ub, c0 + 1, m, live, Mh, orow, frow, drow, stage, lane);
+    tmem_wait_ld();
+    tmem_ld32(tacc + (c0 + 3) * 32, ub);
+    dw_chunk(p, x, ua, c0 + 2, m, live, Mh, orow, frow, drow, stage, lane);
+    tmem_wait_ld();
+    dw_chunk(p, x, ub, c0 + 3, m, live, Mh, orow, frow, drow, stage, lane);
 }
 
 // ------------------------------------------------------------------------------ the kernel
@@ -1609,6 +1653,10 @@ cudaError_t launch_tc_dw(const Dims& D, const DwSpec& w, uint32_t* err, cudaStre
     p.dw_K = w.K;
     p.dw_out0 = (__nv_bfloat16*)w.out0; p.dw_out1 = (__nv_bfloat16*)w.out1;
     p.dw_out_f32 = w.out_f32;
+    // Raster: the smaller operand of a group stays in L2 while the larger streams once.  kind 0
+    // (A = dout rows, d wide; B = gate * h, I wide): all N tiles of an M tile in a row; kinds 1, 2
+    // (A = da | dg or dz, narrower than B = x): all M tiles of an N tile in a row.
+    p.group_m = w.kind == 0 ? 1 : ceil_div(w.M, BM);
     p.dw_bias_col = w.bias0 ? w.N : -1;
     p.dw_Nt = w.bias0 ? w.N + 1 : w.N;
     p.dw_bias0 = (__nv_bfloat16*)w.bias0; p.dw_bias1 = (__nv_bfloat16*)w.bias1;
