@@ -54,6 +54,9 @@ cudaError_t launch_gather(const Dims& D, const void* x, const int32_t* sorted_to
 // division in IEEE fp32.  width % 8 == 0.
 cudaError_t launch_quant_rows(const void* src, const int32_t* row_of, long long n_rows, int src_rows, int width,
                               uint8_t* dst, float* scale, uint32_t* err, cudaStream_t stream);
+// dst[p, :] = src[row_of[p], :] for rows of row_bytes (a multiple of 4) bytes; bad index -> bit 4, zeros
+cudaError_t launch_gather_rows_generic(const void* src, const int32_t* row_of, long long n_rows, long long src_rows,
+                                       int row_bytes, void* dst, uint32_t* err, cudaStream_t stream);
 // dst[p, :] = src[row_of[p], :] for byte rows of row_bytes (a multiple of 16), and dscale[p] =
 // sscale[row_of[p]] when dscale is given; an index outside [0, src_rows) sets bit 4 and gives a
 // zero row with scale 1.

@@ -728,4 +728,18 @@ MOE_EXPORT moe_status_t moe_balance_stats(const moe_shape_t* shape, const void* 
     return MOE_OK;
 }
 
+MOE_EXPORT moe_status_t moe_gather_rows(const void* src, const int32_t* row_of, int64_t n_rows, int64_t src_rows,
+                                        int32_t row_bytes, void* dst, void* ws, size_t ws_bytes, moe_stream_t stream) {
+    if (n_rows < 0 || src_rows < 0 || row_bytes < 1) return MOE_ERR_INVALID_ARG;
+    if (row_bytes % 4) return MOE_ERR_UNSUPPORTED;
+    if (!ws || ws_bytes < 256 || ((uintptr_t)ws & 15u)) return MOE_ERR_WORKSPACE;
+    if (n_rows == 0) return MOE_OK;
+    if (!src || !row_of || !dst) return MOE_ERR_INVALID_ARG;
+    MOE_TRY(check_device());
+    cudaGetLastError();
+    MOE_CUDA(launch_gather_rows_generic(src, row_of, n_rows, src_rows, row_bytes, dst, static_cast<uint32_t*>(ws),
+                                        (cudaStream_t)stream));
+    return MOE_OK;
+}
+
 }  // extern "C"

@@ -150,7 +150,48 @@ __global__ void gather_code_rows_kernel(const uint4* __restrict__ src, const flo
     }
 }
 
+// dst[p] = src[row_of[p]] for rows of nw 4-byte words (16-byte vectors when nw % 4 == 0); an
+// index outside [0, src_rows) sets bit 4 and gives a zero row.
+template <bool V16>
+__global__ void gather_rows_generic_kernel(const uint32_t* __restrict__ src, const int32_t* __restrict__ row_of,
+                                           long long n_rows, long long src_rows, int nw, uint32_t* __restrict__ dst,
+                                           uint32_t* err) {
+    const int nv = V16 ? nw / 4 : nw;
+    for (long long p = blockIdx.x; p < n_rows; p += gridDim.x) {
+        const long long r = row_of[p];
+        const bool ok = r >= 0 && r < src_rows;
+        if (!ok && threadIdx.x == 0) flag_error(err, ERR_INDEX_RANGE);
+        if (V16) {
+            const uint4* s = reinterpret_cast<const uint4*>(src) + (size_t)(ok ? r : 0) * nv;
+            uint4* d = reinterpret_cast<uint4*>(dst) + (size_t)p * nv;
+            for (int i = threadIdx.x; i < nv; i += blockDim.x) d[i] = ok ? __ldg(s + i) : make_uint4(0, 0, 0, 0);
+        } else {
+            const uint32_t* s = src + (size_t)(ok ? r : 0) * nv;
+            uint32_t* d = dst + (size_t)p * nv;
+            for (int i = threadIdx.x; i < nv; i += blockDim.x) d[i] = ok ? __ldg(s + i) : 0u;
+        }
+    }
+}
+
 }  // namespace
+
+cudaError_t launch_gather_rows_generic(const void* src, const int32_t* row_of, long long n_rows, long long src_rows,
+                                       int row_bytes, void* dst, uint32_t* err, cudaStream_t stream) {
+    if (n_rows <= 0) return cudaSuccess;
+    if (row_bytes <= 0 || row_bytes % 4) return cudaErrorInvalidValue;
+    const int nw = row_bytes / 4;
+    const bool v16 = nw % 4 == 0 && ((uintptr_t)src & 15u) == 0 && ((uintptr_t)dst & 15u) == 0;
+    const int threads = nw >= 512 ? 128 : 32;
+    const long long cap = (long long)num_sms() * 16;
+    const int blocks = (int)(n_rows < cap ? n_rows : cap);
+    if (v16)
+        gather_rows_generic_kernel<true><<<blocks, threads, 0, stream>>>((const uint32_t*)src, row_of, n_rows, src_rows,
+                                                                         nw, (uint32_t*)dst, err);
+    else
+        gather_rows_generic_kernel<false><<<blocks, threads, 0, stream>>>((const uint32_t*)src, row_of, n_rows,
+                                                                          src_rows, nw, (uint32_t*)dst, err);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_quant_rows(const void* src, const int32_t* row_of, long long n_rows, int src_rows, int width,
                               uint8_t* dst, float* scale, uint32_t* err, cudaStream_t stream) {

@@ -24,7 +24,7 @@ EXPORTED = ("moe_workspace_bytes", "moe_layer_launches", "moe_status_string", "m
             "moe_layer_forward_timed", "moe_permute_no_alloc", "moe_quantize_rows_e4m3", "moe_train_ctx_bytes",
             "moe_backward_workspace_bytes", "moe_layer_forward_train", "moe_layer_backward",
             "moe_layer_backward_timed", "moe_backward_launches", "moe_balance_workspace_bytes",
-            "moe_balance_stats")
+            "moe_balance_stats", "moe_gather_rows")
 NUM_STAGES = 7
 STAGE_NAMES = ("router", "permute", "plan", "gather", "gemm1_swiglu", "gemm2", "combine")
 BWD_STAGES = 7
@@ -96,11 +96,13 @@ def _lib():
         lib.moe_balance_workspace_bytes.argtypes = [sh]
         lib.moe_balance_workspace_bytes.restype = sz
         lib.moe_balance_stats.argtypes = [sh, vp, vp, f32p, i32p, ctypes.c_int32, f32p, f32p, f32p, vp, sz, vp]
+        lib.moe_gather_rows.argtypes = [vp, i32p, ctypes.c_int64, ctypes.c_int64, ctypes.c_int32, vp, vp, sz, vp]
         lib.moe_backward_launches.argtypes = [sh]
         lib.moe_backward_launches.restype = ctypes.c_int32
         for n in ("moe_check_device_error", "moe_ws_init", "moe_route", "moe_permute", "moe_expert_ffn",
                   "moe_combine", "moe_layer_forward", "moe_layer_forward_timed", "moe_quantize_rows_e4m3",
-                  "moe_layer_forward_train", "moe_layer_backward", "moe_layer_backward_timed", "moe_balance_stats"):
+                  "moe_layer_forward_train", "moe_layer_backward", "moe_layer_backward_timed", "moe_balance_stats",
+                  "moe_gather_rows"):
             getattr(lib, n).restype = ctypes.c_int
         _LIB = lib
     return _LIB
@@ -351,6 +353,19 @@ def balance_stats(shape: MoeShape, x, centroids, counts, n_groups: int = 1, rout
                                     _ptr(counts), n_groups, _ptr(f), _ptr(P), _ptr(terms), _ptr(ws), ws.numel(),
                                     _stream(stream)), "moe_balance_stats")
     return {"f": f, "P": P, "expert_term": terms[0], "device_term": terms[1]}
+
+
+def gather_rows(src: torch.Tensor, row_of: torch.Tensor, ws: torch.Tensor, out=None, stream=None):
+    """moe_gather_rows: out[p] = src[row_of[p]] (rows = the first dimension; any dtype whose row
+    size is a multiple of 4 bytes)."""
+    if not src.is_contiguous() or row_of.dtype != torch.int32:
+        raise ValueError("src must be contiguous and row_of int32")
+    n = row_of.numel()
+    out = torch.empty((n,) + tuple(src.shape[1:]), dtype=src.dtype, device=src.device) if out is None else out
+    row_bytes = src[0].numel() * src.element_size() if src.shape[0] else src.element_size()
+    _check(_lib().moe_gather_rows(_ptr(src), _ptr(row_of), n, src.shape[0], row_bytes, _ptr(out), _ptr(ws), ws.numel(),
+                                  _stream(stream)), "moe_gather_rows")
+    return out
 
 
 def stage_events(stream=None, n_stages: int = NUM_STAGES):

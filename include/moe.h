@@ -349,6 +349,17 @@ moe_status_t moe_balance_stats(const moe_shape_t* shape, const void* x, const vo
                                float* terms, void* ws, size_t ws_bytes, moe_stream_t stream);
 
 /*
+ * Row gather: dst[p, :] = src[row_of[p], :] for p < n_rows, rows of row_bytes bytes (a multiple
+ * of 4; 16-byte vectors when row_bytes % 16 == 0 and both buffers are 16-byte aligned).  The
+ * expert-parallel layer (the "all_to_all to the experts' devices, then back" scheme of the
+ * DeepSeek-V2 explainer, eliteato.com/news/32734, §3.3) moves token rows, gates and expert outputs
+ * with it between its exchanges.  A row_of entry outside [0, src_rows) sets error bit 4 in ws
+ * (>= 256 bytes) and gives a zero row.
+ */
+moe_status_t moe_gather_rows(const void* src, const int32_t* row_of, int64_t n_rows, int64_t src_rows,
+                             int32_t row_bytes, void* dst, void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
  * moe_permute_no_alloc — the paper has no counterpart to this entry point; it exists for
  * callers of this library that cannot allocate device memory.  moe_permute needs scratch
  * space, which it takes from the caller's workspace.  A caller that cannot call cudaMalloc
