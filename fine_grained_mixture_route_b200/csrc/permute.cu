@@ -234,7 +234,14 @@ __global__ void __launch_bounds__(128) combine_kernel(const T* __restrict__ y, c
         __syncthreads();
         for (int v = threadIdx.x; v < nv; v += blockDim.x) {
             float acc[V];
-            if (base) {
+            if (base && V % 4 == 0) {            // 16-byte loads (d % V == 0, base 16-byte aligned)
+                const float4* b4 = reinterpret_cast<const float4*>(base + (size_t)t * d + (size_t)v * V);
+#pragma unroll
+                for (int i = 0; i < V / 4; ++i) {
+                    const float4 f = b4[i];
+                    acc[4 * i] = f.x; acc[4 * i + 1] = f.y; acc[4 * i + 2] = f.z; acc[4 * i + 3] = f.w;
+                }
+            } else if (base) {
 #pragma unroll
                 for (int i = 0; i < V; ++i) acc[i] = base[(size_t)t * d + (size_t)v * V + i];
             } else {
