@@ -49,6 +49,8 @@ constexpr int ACC_COLS = 256;
 constexpr int RING_BYTES = 192 * 1024;   // shared-memory ring (stages x (A + B))
 constexpr int STAGE_OUT_BYTES = 2048;     // per epilogue warp: a 32 x 32 bf16 chunk being transposed
 constexpr int SMEM_BYTES = 1024 /*align slack*/ + RING_BYTES + 256 /*barriers*/ + EPI_WARPS * STAGE_OUT_BYTES;
+constexpr int ZERO_BYTES = 16384;         // DW: zeros that TMA stores copy to the gradients of groups without rows
+constexpr int SMEM_BYTES_DW = SMEM_BYTES + ZERO_BYTES;
 constexpr unsigned long long WAIT_NS = 4000000000ull;
 #ifndef MOE_GROUP_M
 #define MOE_GROUP_M 8                    // M-tiles per raster band of the expert GEMMs
@@ -78,6 +80,7 @@ struct Cfg {
 struct Params {
     CUtensorMap tmA[2];
     CUtensorMap tmB[4];
+    CUtensorMap tmZ[2];        // DW (dw_zero): the gradient outputs, 2-D, box dw_zbw x 32 rows, no swizzle
     const int32_t* tile_start;
     const int32_t* offsets;
     int g_begin, g_end;
@@ -123,6 +126,11 @@ struct Params {
     int dw_Nt;                         // DW: columns the tiles cover (dw_N, or dw_N + 1 with a bias column)
     int dw_bias_col;                   // DW: B column dw_N holds the row weights of a bias gradient (or -1):
     __nv_bfloat16 *dw_bias0, *dw_bias1;  //    out column dw_N -> bias0 [g][M] (kind 1: rows >= M/2 -> bias1)
+    int dw_zero;                       // DW: a group without rows is written by the producer's TMA stores of
+    int dw_zbw;                        //    zeros (box dw_zbw columns x 32 rows); its tiles skip MMA and epilogue
+    int mn_wide;                       // MN-major operands read through 4-D views {64 columns, rows, column
+                                       // blocks, groups}: one request per operand and stage instead of one per
+                                       // 64-column block (DW: tmA[1] / tmB[1]; DH, DX, DXS: their B maps)
     uint32_t* err;
 };
 
@@ -186,9 +194,33 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
         "l"((unsigned long long)map), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
         : "memory");
 }
+__device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* map, uint32_t bar, int c0, int c1, int c2,
+                                            int c3) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(
+            dst),
+        "l"((unsigned long long)map), "r"(bar), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+        : "memory");
+}
 __device__ __forceinline__ void prefetch_map(const CUtensorMap* map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"((unsigned long long)map) : "memory");
 }
+// shared -> global tensor store (bulk-group completion); the box starts inside the tensor and
+// is clipped at its far edges
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t src, int c0, int c1) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                     (unsigned long long)map),
+                 "r"(src), "r"(c0), "r"(c1)
+                 : "memory");
+}
+// shared -> global bulk copy of `bytes` (multiple of 16; both addresses 16-byte aligned)
+__device__ __forceinline__ void bulk_store(void* dst, uint32_t src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"((unsigned long long)dst), "r"(src),
+                 "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 // Shared-memory matrix descriptor: K-major operand, 128-byte swizzle, 8-row core-matrix
 // groups 1024 bytes apart (stride byte offset); leading byte offset unused for this layout;
@@ -949,6 +981,29 @@ __device__ __forceinline__ void epilogue_dw(const Params& p, const Tile& x, uint
     dw_chunk(p, x, ub, c0 + 3, m, live, Mh, orow, frow, drow, stage, lane);
 }
 
+// DW, a tile of a group without rows (dw_zero): the producer thread writes its gradient block
+// as zeros with TMA stores from the zeroed shared-memory block (32 rows per store), and the bias
+// gradient rows of the tile that holds the bias column with bulk copies; M, M/2 and N are
+// multiples of 32 rows / 64 columns, so no store crosses from one output matrix into the next.
+__device__ __forceinline__ void dw_zero_tile(const Params& p, const Tile& x, uint32_t zbuf) {
+    const int Mh = p.dw_M / 2;
+    const bool bias_tile = p.dw_bias_col >= 0 && x.n0 <= p.dw_N && p.dw_N < x.n0 + 256;
+    for (int rb = 0; rb < 4; ++rb) {
+        const int m = x.m0 + 32 * rb;
+        if (m >= p.dw_M) break;
+        const bool hi = p.dw_kind == 1 && m >= Mh;
+        const CUtensorMap* map = &p.tmZ[hi ? 1 : 0];
+        const int y = p.dw_kind == 1 ? x.g * Mh + (hi ? m - Mh : m) : x.g * p.dw_M + m;
+        for (int c = x.n0; c < x.n0 + 256 && c < p.dw_N; c += p.dw_zbw) tma_store_2d(map, zbuf, c, y);
+        if (bias_tile) {
+            __nv_bfloat16* b = p.dw_kind == 1 ? (hi ? p.dw_bias1 : p.dw_bias0) + (size_t)x.g * Mh + (hi ? m - Mh : m)
+                                              : p.dw_bias0 + (size_t)x.g * p.dw_M + m;
+            bulk_store(b, zbuf, 32 * 2);
+        }
+    }
+    bulk_commit();
+}
+
 // ------------------------------------------------------------------------------ the kernel
 // Pair protocol (expert GEMMs): both CTAs of a cluster pair run the same roles.  Each CTA's
 // producer waits on its own "empty" barriers and loads its halves of A and B into its own
@@ -1001,6 +1056,12 @@ __global__ void __launch_bounds__(THREADS, 1) moe_tc_kernel(const __grid_constan
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     }
+    const uint32_t zbuf = bar0 + 256 + EPI_WARPS * STAGE_OUT_BYTES;   // DW: ZERO_BYTES of zeros
+    if (MODE == DW && p.dw_zero) {
+        for (int i = threadIdx.x; i < ZERO_BYTES / 16; i += THREADS)
+            asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(zbuf + 16u * i), "r"(0u) : "memory");
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // visible to the TMA stores
+    }
     if (warp == 1) {
         if (PAIR) {
             asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_holder)),
@@ -1035,6 +1096,12 @@ __global__ void __launch_bounds__(THREADS, 1) moe_tc_kernel(const __grid_constan
             const int arow = (int)rank * BM;                 // this CTA's rows inside a pair tile
             for (int t = cta_slot; ok && t < ntiles; t += cta_slots) {
                 const Tile x = decode<MODE, PAIR>(p, t);
+                if (MODE == DW && p.dw_zero && x.num_kb == 0) {
+                    dw_zero_tile(p, x, zbuf);
+                    continue;
+                }
+                // DW: a tile holding only the bias column loads one 64-column box of B (N = 64 MMAs)
+                const int nbox = (MODE == DW && x.n0 >= p.dw_N) ? 1 : 4;
                 for (int kk_ = 0; kk_ < x.num_kb; ++kk_) {
                     const int kb = x.kb0 + kk_;
                     if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, p.err)) { ok = false; break; }
@@ -1071,37 +1138,54 @@ __global__ void __launch_bounds__(THREADS, 1) moe_tc_kernel(const __grid_constan
                         }
                     } else if (MODE == DH || MODE == DX || MODE == DXS || MODE == DW) {
                         // MN-major B: four 64-column boxes of BK rows, 8 KB apart; DW's A likewise (two)
-                        mbar_expect_tx(fb, A_BYTES + B_BYTES);
+                        mbar_expect_tx(fb, A_BYTES + ((MODE == DW && !p.mn_wide) ? nbox * 8192 : B_BYTES));
                         if (MODE == DH) {
                             const bool shared = x.g >= p.E;
                             const int e = shared ? x.g - p.E : x.g;
                             tma_load_2d(a_dst, &p.tmA[shared ? 1 : 0], fb, kb * BK, x.row0 + x.m0);
+                            if (p.mn_wide) tma_load_4d(b_dst, &p.tmB[shared ? 1 : 0], fb, 0, kb * BK, x.n0 / 64, e);
+                            else
 #pragma unroll
-                            for (int j = 0; j < 4; ++j)
-                                tma_load_3d(b_dst + j * 8192, &p.tmB[shared ? 1 : 0], fb, x.n0 + 64 * j, kb * BK, e);
+                                for (int j = 0; j < 4; ++j)
+                                    tma_load_3d(b_dst + j * 8192, &p.tmB[shared ? 1 : 0], fb, x.n0 + 64 * j, kb * BK, e);
                         } else if (MODE == DX) {
                             const int kbh = ceil_div(p.I, BK);
                             const int hb = kb >= kbh ? 1 : 0;                  // 0: da . W1, 1: dg . W3
                             tma_load_2d(a_dst, &p.tmA[0], fb, kb * BK, x.row0 + x.m0);
+                            if (p.mn_wide) tma_load_4d(b_dst, &p.tmB[hb], fb, 0, (kb - hb * kbh) * BK, x.n0 / 64, x.g);
+                            else
 #pragma unroll
-                            for (int j = 0; j < 4; ++j)
-                                tma_load_3d(b_dst + j * 8192, &p.tmB[hb], fb, x.n0 + 64 * j, (kb - hb * kbh) * BK, x.g);
+                                for (int j = 0; j < 4; ++j)
+                                    tma_load_3d(b_dst + j * 8192, &p.tmB[hb], fb, x.n0 + 64 * j, (kb - hb * kbh) * BK,
+                                                x.g);
                         } else if (MODE == DXS) {
                             const int kbs = 2 * ceil_div(p.Is, BK);
                             if (kb < p.Ks * kbs) {
                                 const int sx = kb / kbs, kk = kb % kbs;
                                 const int hb = kk >= kbs / 2 ? 1 : 0;
                                 tma_load_3d(a_dst, &p.tmA[0], fb, kk * BK, x.m0, sx);
+                                if (p.mn_wide)
+                                    tma_load_4d(b_dst, &p.tmB[hb], fb, 0, (kk - hb * (kbs / 2)) * BK, x.n0 / 64, sx);
+                                else
 #pragma unroll
-                                for (int j = 0; j < 4; ++j)
-                                    tma_load_3d(b_dst + j * 8192, &p.tmB[hb], fb, x.n0 + 64 * j, (kk - hb * (kbs / 2)) * BK, sx);
+                                    for (int j = 0; j < 4; ++j)
+                                        tma_load_3d(b_dst + j * 8192, &p.tmB[hb], fb, x.n0 + 64 * j,
+                                                    (kk - hb * (kbs / 2)) * BK, sx);
                             } else {
                                 const int kr = kb - p.Ks * kbs;            // router: dz . C
                                 tma_load_2d(a_dst, &p.tmA[1], fb, kr * BK, x.m0);
+                                if (p.mn_wide) tma_load_4d(b_dst, &p.tmB[2], fb, 0, kr * BK, x.n0 / 64, 0);
+                                else
 #pragma unroll
-                                for (int j = 0; j < 4; ++j)
-                                    tma_load_2d(b_dst + j * 8192, &p.tmB[2], fb, x.n0 + 64 * j, kr * BK);
+                                    for (int j = 0; j < 4; ++j)
+                                        tma_load_2d(b_dst + j * 8192, &p.tmB[2], fb, x.n0 + 64 * j, kr * BK);
                             }
+                        } else if (p.mn_wide) {
+                            // the 2 (A) and 4 (B) 64-column blocks of the stage in one request each,
+                            // block j landing 8 KB after block j - 1 as with separate boxes
+                            const int kr = x.row0 + kb * BK;
+                            tma_load_4d(a_dst, &p.tmA[1], fb, 0, p.dw_a3d ? kb * BK : kr, x.m0 / 64, p.dw_a3d ? x.g : 0);
+                            tma_load_4d(b_dst, &p.tmB[1], fb, 0, p.dw_b3d ? kb * BK : kr, x.n0 / 64, p.dw_b3d ? x.g : 0);
                         } else {
                             const int kr = x.row0 + kb * BK;
 #pragma unroll
@@ -1109,8 +1193,7 @@ __global__ void __launch_bounds__(THREADS, 1) moe_tc_kernel(const __grid_constan
                                 if (p.dw_a3d) tma_load_3d(a_dst + j * 8192, &p.tmA[0], fb, x.m0 + 64 * j, kb * BK, x.g);
                                 else tma_load_2d(a_dst + j * 8192, &p.tmA[0], fb, x.m0 + 64 * j, kr);
                             }
-#pragma unroll
-                            for (int j = 0; j < 4; ++j) {
+                            for (int j = 0; j < nbox; ++j) {
                                 if (p.dw_b3d) tma_load_3d(b_dst + j * 8192, &p.tmB[0], fb, x.n0 + 64 * j, kb * BK, x.g);
                                 else tma_load_2d(b_dst + j * 8192, &p.tmB[0], fb, x.n0 + 64 * j, kr);
                             }
@@ -1153,6 +1236,7 @@ __global__ void __launch_bounds__(THREADS, 1) moe_tc_kernel(const __grid_constan
                 if (leader) mbar_wait(full_bar(s), (uint32_t)last_parity[s], abort_flag, p.err, false);
                 else mbar_wait(empty_bar(s), (uint32_t)last_parity[s], abort_flag, p.err, false);
             }
+            if (MODE == DW && p.dw_zero) bulk_wait_all();   // zero stores done before the block is freed
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------------ MMA issuer
@@ -1165,10 +1249,13 @@ __global__ void __launch_bounds__(THREADS, 1) moe_tc_kernel(const __grid_constan
             bool ok = true;
             for (int t = cta_slot; ok && t < ntiles; t += cta_slots) {
                 const Tile x = decode<MODE, PAIR>(p, t);
+                if (MODE == DW && p.dw_zero && x.num_kb == 0) continue;      // written by the producer
                 const bool q8tile = Q8 && (MODE == GEMM1 ? x.g < p.E : x.g >= 0);
                 constexpr bool B_MN = MODE == DH || MODE == DX || MODE == DXS || MODE == DW;
                 constexpr bool A_MN = MODE == DW;
+                const bool narrow = MODE == DW && x.n0 >= p.dw_N;             // bias column only
                 const uint32_t idesc_t = q8tile ? (PAIR ? idesc_e4m3_pair(p.n_mma) : idesc_e4m3(p.n_mma))
+                                       : narrow ? idesc_bf16(64) | IDESC_B_MN | IDESC_A_MN
                                                 : idesc | (B_MN ? IDESC_B_MN : 0u) | (A_MN ? IDESC_A_MN : 0u);
                 if (!mbar_wait(tempty_bar(acc), acc_phase ^ 1u, abort_flag, p.err)) break;
                 tc_fence_after();
@@ -1212,6 +1299,7 @@ __global__ void __launch_bounds__(THREADS, 1) moe_tc_kernel(const __grid_constan
         uint32_t acc_phase = 0;
         for (int t = cta_slot; t < ntiles; t += cta_slots) {
             const Tile x = decode<MODE, PAIR>(p, t);
+            if (MODE == DW && p.dw_zero && x.num_kb == 0) continue;          // written by the producer
             if (!mbar_wait(tfull_bar(acc), acc_phase, abort_flag, p.err)) break;
             tc_fence_after();
             const uint32_t tacc = tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(acc * ACC_COLS);
@@ -1289,6 +1377,39 @@ bool make_map(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t mid, uin
     return r == CUDA_SUCCESS;
 }
 
+// bf16 matrix [outer][rows][ld] read MN-major: the 4-D view {64 columns, rows, ld / 64 column
+// blocks, outer} (strides ld * 2, 128, rows * ld * 2 bytes) with a box of 64 x box_rows x nblk x 1,
+// so that one request brings nblk consecutive 64-column blocks, each a 128B-swizzled
+// [box_rows][64] block, 8 KB apart in shared memory.  ld must be a multiple of 64.
+bool make_map_mn(CUtensorMap* m, const void* ptr, uint64_t ld, uint64_t rows, uint64_t outer, uint32_t box_rows,
+                 uint32_t nblk) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn || ld % 64) return false;
+    cuuint64_t dims[4] = {64, rows, ld / 64, outer};
+    cuuint64_t strides[3] = {ld * 2, 128, rows * ld * 2};
+    cuuint32_t box[4] = {64, box_rows, nblk, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// bf16 matrix [rows][inner] as the target of TMA stores: box box_inner x box_rows, no swizzle
+bool make_store_map(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t rows, uint32_t box_inner,
+                    uint32_t box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {inner, rows};
+    cuuint64_t strides[1] = {inner * 2};
+    cuuint32_t box[2] = {box_inner, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 // e4m3 (byte) tensor [outer][mid][inner] with a box of box_inner x box_mid (x 1); inner must
 // be a multiple of 16 (16-byte strides)
 bool make_map_u8(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t mid, uint64_t outer, uint32_t box_inner,
@@ -1310,12 +1431,13 @@ bool make_map_u8(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t mid, 
 template <int MODE, int KMAX, bool PAIR = false, bool Q8 = false>
 cudaError_t launch(const Params& p, int tiles, cudaStream_t stream) {
     auto kern = moe_tc_kernel<MODE, KMAX, PAIR, Q8>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    constexpr int smem = MODE == DW ? SMEM_BYTES_DW : SMEM_BYTES;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[1];
     cfg.blockDim = dim3(THREADS);
-    cfg.dynamicSmemBytes = SMEM_BYTES;
+    cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
     if (Cfg<MODE, PAIR>::PAIR) {
         attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -1603,6 +1725,12 @@ cudaError_t launch_tc_dh(const Dims& D, const BwdBufs& B, const FfnWeights& R, c
         ok &= make_map(&p.tmB[1], Sh.w2, D.Is, D.d, D.Ks, 64, BK, true);
     }
     if (!ok) return cudaErrorInvalidValue;
+    CUtensorMap w[2];
+    if (make_map_mn(&w[0], R.w2, D.I, D.d, D.E, BK, 4) && (D.Ks == 0 || make_map_mn(&w[1], Sh.w2, D.Is, D.d, D.Ks, BK, 4))) {
+        p.tmB[0] = w[0];
+        if (D.Ks > 0) p.tmB[1] = w[1];
+        p.mn_wide = 1;
+    }
     return launch<DH, 8>(p, num_sms(), stream);
 }
 
@@ -1618,6 +1746,12 @@ cudaError_t launch_tc_dx(const Dims& D, const BwdBufs& B, const FfnWeights& R, u
     ok &= make_map(&p.tmB[0], R.w1, D.d, D.I, D.E, 64, BK, true);
     ok &= make_map(&p.tmB[1], R.w3, D.d, D.I, D.E, 64, BK, true);
     if (!ok) return cudaErrorInvalidValue;
+    CUtensorMap w[2];
+    if (make_map_mn(&w[0], R.w1, D.d, D.I, D.E, BK, 4) && make_map_mn(&w[1], R.w3, D.d, D.I, D.E, BK, 4)) {
+        p.tmB[0] = w[0];
+        p.tmB[1] = w[1];
+        p.mn_wide = 1;
+    }
     return launch<DX, 8>(p, num_sms(), stream);
 }
 
@@ -1639,6 +1773,15 @@ cudaError_t launch_tc_dxs(const Dims& D, const BwdBufs& B, const FfnWeights& Sh,
         ok &= make_map(&p.tmB[0], centroids, D.d, D.E, 1, 64, BK, false);
     }
     if (!ok) return cudaErrorInvalidValue;
+    CUtensorMap w[3];
+    if (make_map_mn(&w[2], centroids, D.d, D.E, 1, BK, 4) &&
+        (D.Ks > 0 ? make_map_mn(&w[0], Sh.w1, D.d, D.Is, D.Ks, BK, 4) && make_map_mn(&w[1], Sh.w3, D.d, D.Is, D.Ks, BK, 4)
+                  : make_map_mn(&w[0], centroids, D.d, D.E, 1, BK, 4))) {
+        p.tmB[0] = w[0];
+        if (D.Ks > 0) p.tmB[1] = w[1];
+        p.tmB[2] = w[2];
+        p.mn_wide = 1;
+    }
     return launch<DXS, 8>(p, ceil_div(D.T, BM) * ceil_div(D.d, 256), stream);
 }
 
@@ -1664,6 +1807,24 @@ cudaError_t launch_tc_dw(const Dims& D, const DwSpec& w, uint32_t* err, cudaStre
     if (w.bias0 && b_ld < w.N + 1) return cudaErrorInvalidValue;
     bool ok = make_map(&p.tmA[0], w.a, (uint64_t)w.M, (uint64_t)w.a_rows, w.a3d ? w.groups : 1, 64, BK, w.a3d);
     ok &= make_map(&p.tmB[0], w.b, (uint64_t)b_ld, (uint64_t)w.b_rows, w.b3d ? w.groups : 1, 64, BK, w.b3d);
+    // one request per operand and stage where both widths are whole 64-column blocks (the view
+    // must not reach past a row's end), else one request per 64-column block
+    if (w.M % 64 == 0 && b_ld % 64 == 0)
+        p.mn_wide = make_map_mn(&p.tmA[1], w.a, (uint64_t)w.M, (uint64_t)w.a_rows, w.a3d ? w.groups : 1, BK, 2) &&
+                    make_map_mn(&p.tmB[1], w.b, (uint64_t)b_ld, (uint64_t)w.b_rows, w.b3d ? w.groups : 1, BK, 4);
+    if (w.rows && w.kind != 2) {
+        // groups may be empty: their bf16 gradients (and bias gradients) are zero-filled by the
+        // producer's TMA stores, 32 rows x up to 256 columns each
+        const int Mo = w.kind == 1 ? w.M / 2 : w.M;
+        auto a16 = [](const void* q) { return ((uintptr_t)q & 15u) == 0; };
+        if (w.N % 64 || Mo % 32 || !a16(w.out0) || (w.kind == 1 && !a16(w.out1)) || (w.bias0 && !a16(w.bias0)) ||
+            (w.bias1 && !a16(w.bias1)))
+            return cudaErrorInvalidValue;
+        p.dw_zero = 1;
+        p.dw_zbw = w.N < 256 ? w.N : 256;
+        ok &= make_store_map(&p.tmZ[0], w.out0, (uint64_t)w.N, (uint64_t)w.groups * Mo, p.dw_zbw, 32);
+        if (w.kind == 1) ok &= make_store_map(&p.tmZ[1], w.out1, (uint64_t)w.N, (uint64_t)w.groups * Mo, p.dw_zbw, 32);
+    }
     if (!ok) return cudaErrorInvalidValue;
     const long long tiles = (long long)w.groups * ceil_div(w.M, BM) * ceil_div(p.dw_Nt, 256);
     return launch<DW, 8>(p, (int)(tiles < num_sms() ? tiles : num_sms()), stream);

@@ -524,11 +524,14 @@ moe_status_t layer_backward_impl(const moe_shape_t* shape, const void* x, const 
     MOE_TRY(check_weights(D, routed));
     if (D.Ks > 0) MOE_TRY(check_weights(D, shared));
     else if (shared || gshared) return MOE_ERR_INVALID_ARG;
+    auto a16 = [](const void* q) { return ((uintptr_t)q & 15u) == 0; };   // 16-byte vector / TMA stores
     auto check_grads = [&](const moe_ffn_grads_t* g) -> bool {
         if (!g || !g->w1 || !g->w3 || !g->w2) return false;
+        if (!a16(g->w1) || !a16(g->w3) || !a16(g->w2) || !a16(g->b1) || !a16(g->b3) || !a16(g->b2)) return false;
         const bool b = g->b1 && g->b3 && g->b2, none = !g->b1 && !g->b3 && !g->b2;
         return D.bias ? b : none;
     };
+    if (!a16(dx) || !a16(dcentroids)) return MOE_ERR_INVALID_ARG;
     if (!check_grads(groutes) || (D.Ks > 0 && !check_grads(gshared))) return MOE_ERR_INVALID_ARG;
     if (drouter_bias && (!router_bias || D.gate_mode == MOE_GATE_SIGMOID_BIAS)) return MOE_ERR_INVALID_ARG;
     const CtxLayout C = ctx_layout(D);

@@ -296,6 +296,9 @@ moe_status_t moe_layer_forward_train(const moe_shape_t* shape, const void* x, co
  *   routed_grads, shared_grads out: weight and bias gradients in the layer dtype (all experts;
  *                              an expert without tokens gets zeros); shared_grads NULL iff
  *                              n_shared == 0
+ * dx, dcentroids and every gradient buffer must be 16-byte aligned (MOE_ERR_INVALID_ARG
+ * otherwise): they are written with 16-byte vector stores and, for the zeros of experts without
+ * tokens, with tensor-memory-access stores.
  * Sums are fp32 on the tensor cores and in fixed order (deterministic); dx adds the routed terms
  * in pick order to the shared and router terms.  ws: moe_backward_workspace_bytes(shape) bytes
  * (its first 256 bytes are the error word, as for the other calls).
