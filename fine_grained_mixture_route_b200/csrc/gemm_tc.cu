@@ -128,6 +128,8 @@ struct Params {
     __nv_bfloat16 *dw_bias0, *dw_bias1;  //    out column dw_N -> bias0 [g][M] (kind 1: rows >= M/2 -> bias1)
     int dw_zero;                       // DW: a group without rows is written by the producer's TMA stores of
     int dw_zbw;                        //    zeros (box dw_zbw columns x 32 rows); its tiles skip MMA and epilogue
+    int w13_one;                       // GEMM1: bit 0 routed, bit 1 shared: tmB[0] / tmB[2] is a 4-D view
+                                       // {d, I, W1 | W3, expert} and one request brings both weight blocks
     int mn_wide;                       // MN-major operands read through 4-D views {64 columns, rows, column
                                        // blocks, groups}: one request per operand and stage instead of one per
                                        // 64-column block (DW: tmA[1] / tmB[1]; DH, DX, DXS: their B maps)
@@ -1205,8 +1207,12 @@ __global__ void __launch_bounds__(THREADS, 1) moe_tc_kernel(const __grid_constan
                             const int e = shared ? x.g - p.E : x.g;
                             const int kc = kb * ((Q8 && !shared) ? 2 * BK : BK);   // K element offset
                             tma_load_2d(a_dst, &p.tmA[shared ? 1 : 0], fb, kc, x.row0 + x.m0);
-                            tma_load_3d(b_dst, &p.tmB[shared ? 2 : 0], fb, kc, x.n0, e);
-                            tma_load_3d(b_dst + B_BYTES / 2, &p.tmB[shared ? 3 : 1], fb, kc, x.n0, e);
+                            if (p.w13_one & (shared ? 2 : 1)) {         // W3's block lands B_BYTES / 2 after W1's
+                                tma_load_4d(b_dst, &p.tmB[shared ? 2 : 0], fb, kc, x.n0, 0, e);
+                            } else {
+                                tma_load_3d(b_dst, &p.tmB[shared ? 2 : 0], fb, kc, x.n0, e);
+                                tma_load_3d(b_dst + B_BYTES / 2, &p.tmB[shared ? 3 : 1], fb, kc, x.n0, e);
+                            }
                         } else if (MODE == GEMM2R && x.g >= 0) {
                             const int kc = kb * (Q8 ? 2 * BK : BK);
                             tma_load_2d(a_dst, &p.tmA[0], fb, kc, x.row0 + x.m0);
@@ -1395,6 +1401,27 @@ bool make_map_mn(CUtensorMap* m, const void* ptr, uint64_t ld, uint64_t rows, ui
     return r == CUDA_SUCCESS;
 }
 
+// W1 and W3 stacks [E][I][d] (esz-byte elements) at a fixed positive distance, e.g. the two
+// halves of one [2][E][I][d] buffer: the 4-D view {d, I, 2, E} whose third coordinate selects W1
+// or W3, with a box of box_k x 128 rows x 2, brings a tile's 128 rows of both in one request (W3's
+// rows 128 * box_k * esz bytes after W1's, as two separate boxes would land).  False when the
+// distance does not fit the view (the caller then loads the two blocks separately).
+bool make_map_w13(CUtensorMap* m, const void* w1, const void* w3, uint64_t d, uint64_t I, uint64_t E, uint32_t box_k,
+                  bool u8) {
+    EncodeTiledFn fn = encode_fn();
+    const long long gap = (long long)((const char*)w3 - (const char*)w1);
+    if (!fn || gap <= 0 || gap % 16 || gap >= (1ll << 40)) return false;
+    const uint64_t esz = u8 ? 1 : 2;
+    cuuint64_t dims[4] = {d, I, 2, E};
+    cuuint64_t strides[3] = {d * esz, (cuuint64_t)gap, I * d * esz};
+    cuuint32_t box[4] = {box_k, 128, 2, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = fn(m, u8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(w1),
+                    dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 // bf16 matrix [rows][inner] as the target of TMA stores: box box_inner x box_rows, no swizzle
 bool make_store_map(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t rows, uint32_t box_inner,
                     uint32_t box_rows) {
@@ -1575,6 +1602,11 @@ cudaError_t launch_tc_gemm1(const Dims& D, const void* x, const void* x_perm, co
         ok &= make_map(&p.tmB[3], Sh.w3, D.d, D.Is, D.Ks, BK, 128, true);
     }
     if (!ok) return cudaErrorInvalidValue;
+    if (!tc::pairs_for(D)) {                   // one request for both weight blocks where the layout allows
+        CUtensorMap w;
+        if (g_begin < D.E && make_map_w13(&w, R.w1, R.w3, D.d, D.I, D.E, BK, false)) { p.tmB[0] = w; p.w13_one |= 1; }
+        if (g_end > D.E && make_map_w13(&w, Sh.w1, Sh.w3, D.d, D.Is, D.Ks, BK, false)) { p.tmB[2] = w; p.w13_one |= 2; }
+    }
     // tile count lives on the device
     return tc::pairs_for(D) ? launch<GEMM1, 8, true>(p, num_sms(), stream) : launch<GEMM1, 8, false>(p, num_sms(), stream);
 }
@@ -1650,6 +1682,11 @@ cudaError_t launch_tc_gemm1_q8(const Dims& D, const void* x, const void* x8_perm
         ok &= make_map(&p.tmB[3], Sh.w3, D.d, D.Is, D.Ks, BK, 128, true);
     }
     if (!ok) return cudaErrorInvalidValue;
+    if (!tc::pairs_for(D)) {
+        CUtensorMap w;
+        if (make_map_w13(&w, R.w1, R.w3, D.d, D.I, D.E, 2 * BK, true)) { p.tmB[0] = w; p.w13_one |= 1; }
+        if (g_end > D.E && make_map_w13(&w, Sh.w1, Sh.w3, D.d, D.Is, D.Ks, BK, false)) { p.tmB[2] = w; p.w13_one |= 2; }
+    }
     return tc::pairs_for(D) ? launch<GEMM1, 8, true, true>(p, num_sms(), stream)
                             : launch<GEMM1, 8, false, true>(p, num_sms(), stream);
 }

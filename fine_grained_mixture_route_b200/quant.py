@@ -33,11 +33,19 @@ def dequantize_rows(q: torch.Tensor, scale: torch.Tensor) -> torch.Tensor:
 
 def quantize_stack(stack: Dict[str, Optional[torch.Tensor]]) -> Dict[str, Optional[torch.Tensor]]:
     """Routed expert stack (w1, w3 [E, I, d]; w2 [E, d, I]; biases unchanged) -> codes in
-    w1/w3/w2 (uint8) and per-row scales in s1, s3 [E, I] and s2 [E, d]."""
+    w1/w3/w2 (uint8; w1 and w3 the two halves of one [2, E, I, d] buffer) and per-row scales in
+    s1, s3 [E, I] and s2 [E, d]."""
     out = dict(stack)
+    codes13 = None
     for w, sname in (("w1", "s1"), ("w3", "s3"), ("w2", "s2")):
         q, sc = quantize_rows(stack[w])
-        out[w] = q.contiguous()
+        if w in ("w1", "w3"):                 # W1 and W3 codes as the two halves of one buffer
+            if codes13 is None:
+                codes13 = torch.empty((2,) + tuple(q.shape), dtype=q.dtype, device=q.device)
+            codes13[0 if w == "w1" else 1].copy_(q)
+            out[w] = codes13[0 if w == "w1" else 1]
+        else:
+            out[w] = q.contiguous()
         out[sname] = sc
     return out
 

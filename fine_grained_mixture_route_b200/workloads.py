@@ -139,11 +139,15 @@ def make_expert_stack(cfg: LayerConfig, shared: bool, device="cpu", seed: int = 
     n = len(ids)
     out: Dict[str, Optional[torch.Tensor]] = {}
     shapes = {"w1": (I, d), "w3": (I, d), "w2": (d, I), "b1": (I,), "b3": (I,), "b2": (d,)}
+    # W1 and W3 are the two halves of one buffer, so the up-projection can fetch a tile of both
+    # with one request
+    w13 = torch.empty((2, n, I, d), dtype=cfg.dtype, device=device)
     for name, shp in shapes.items():
         if name.startswith("b") and not cfg.has_bias:
             out[name] = None
             continue
-        t = torch.empty((n,) + shp, dtype=cfg.dtype, device=device)
+        t = w13[0] if name == "w1" else w13[1] if name == "w3" else torch.empty((n,) + shp, dtype=cfg.dtype,
+                                                                                  device=device)
         for j, e in enumerate(ids):
             t[j] = _normal(shp, INIT_STD, device, seed, p + name, e).to(cfg.dtype)
         out[name] = t
