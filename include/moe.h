@@ -103,7 +103,10 @@ typedef struct {
     int32_t routed_fmt;   /* moe_expert_fmt_t (0 = weights in dtype) */
 } moe_shape_t;
 
-/* One stack of experts (routed: E = n_experts; shared: E = n_shared), nn.Linear layout. */
+/* One stack of experts (routed: E = n_experts; shared: E = n_shared), nn.Linear layout.
+ * Layout hint: when w3 lies a positive multiple of 16 bytes after w1 (for instance the two halves
+ * of one [2, E, I, d] buffer), the up-projection fetches a tile's W1 and W3 rows with one request;
+ * any other placement is accepted and costs one extra request per pipeline stage. */
 typedef struct {
     const void* w1; /* [E, I, d] */
     const void* b1; /* [E, I] or NULL */
