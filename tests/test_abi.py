@@ -174,13 +174,22 @@ def test_training_entry_points_validate(lib):
         moe.MOE_ERR_UNSUPPORTED
     b = lib.moe_layer_backward
     args = lambda **kw: [S(kw.get("sh", sh)), fake, fake, kw.get("rb", None), S(w), S(w), fake, fake,
-                         kw.get("nc", nc), fake, fake, kw.get("drb", None), S(kw.get("g", g)), S(g), fake,
-                         kw.get("nb", nb), None]
+                         kw.get("nc", nc), kw.get("dx", fake), fake, kw.get("drb", None), S(kw.get("g", g)),
+                         S(kw.get("gs", g)), fake, kw.get("nb", nb), None]
     assert b(*args(nc=nc - 1)) == moe.MOE_ERR_WORKSPACE
     assert b(*args(nb=nb - 1)) == moe.MOE_ERR_WORKSPACE
     assert b(*args(drb=fake)) == moe.MOE_ERR_INVALID_ARG            # router-bias gradient without a bias
     assert b(*args(g=moe.MoeGrads(fake.value, None, fake.value, fake.value, fake.value, fake.value))) == \
         moe.MOE_ERR_INVALID_ARG                                      # bias gradient pointers must match has_bias
+    # gradients, dx and dcentroids take 16-byte vector and tensor-memory-access stores
+    odd = ctypes.c_void_p((1 << 40) + 8)
+    assert b(*args()) not in (moe.MOE_OK, moe.MOE_ERR_INVALID_ARG)   # aligned: past validation (no device here)
+    assert b(*args(dx=odd)) == moe.MOE_ERR_INVALID_ARG
+    for i in range(6):
+        ptrs = [fake.value] * 6
+        ptrs[i] = odd.value
+        assert b(*args(g=moe.MoeGrads(*ptrs))) == moe.MOE_ERR_INVALID_ARG, i
+        assert b(*args(gs=moe.MoeGrads(*ptrs))) == moe.MOE_ERR_INVALID_ARG, i
     sh2 = _shape(gate_mode=2)
     assert b(*args(sh=sh2, rb=fake, drb=fake, nc=moe.train_ctx_bytes(sh2), nb=moe.backward_workspace_bytes(sh2))) \
         == moe.MOE_ERR_INVALID_ARG                                   # gate mode 2: the bias only selects
