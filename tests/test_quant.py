@@ -74,3 +74,14 @@ def test_weight_codes_match_the_oracle_quantiser():
         q_ref, s_ref = O.quantize_rows_e4m3(src.double().numpy())
         assert np.array_equal(s.numpy(), s_ref)
         assert np.array_equal(O.e4m3_decode(q.numpy()), q_ref)
+
+
+def test_quantized_w1_w3_share_one_buffer():
+    cfg = W.scaled(W.CONFIGS["small"], T=8, d=64, n_experts=4, inter=32, inter_shared=32)
+    q = quant.quantize_stack(W.make_expert_stack(cfg, False))
+    w1, w3 = q["w1"], q["w3"]
+    assert w1.dtype == torch.uint8 and w1.is_contiguous() and w3.is_contiguous()
+    assert w3.data_ptr() - w1.data_ptr() == w1.numel()
+    # the codes are the per-matrix quantisation of each, unchanged by the shared placement
+    ref1, _ = quant.quantize_rows(W.make_expert_stack(cfg, False)["w1"])
+    assert torch.equal(w1, ref1)

@@ -55,3 +55,20 @@ def test_zipf_centroid_norms():
     srt = torch.sort(n, descending=True).values
     want = torch.tensor([R * (r + 1) ** -1.1 for r in range(64)])
     assert torch.allclose(srt, want, rtol=1e-5)
+
+
+def test_w1_w3_share_one_buffer():
+    # W1 and W3 are the two halves of one [2, E, I, d] buffer: w3 starts a fixed, 16-byte-multiple
+    # distance after w1, the placement that lets the up-projection fetch both with one request
+    for name in ("small", "mid"):
+        cfg = W.scaled(W.CONFIGS[name], T=8, d=64, n_experts=4, inter=32, inter_shared=32)
+        L = W.make_layer(cfg)
+        for stack in (L["routed"], L["shared"]):
+            w1, w3 = stack["w1"], stack["w3"]
+            assert w1.is_contiguous() and w3.is_contiguous()
+            gap = w3.data_ptr() - w1.data_ptr()
+            assert gap == w1.numel() * w1.element_size() and gap % 16 == 0
+            assert w1.untyped_storage().data_ptr() == w3.untyped_storage().data_ptr()
+        # slices of experts keep the distance (expert-parallel ranks pass such slices)
+        r = L["routed"]
+        assert r["w3"][1:3].data_ptr() - r["w1"][1:3].data_ptr() == r["w1"].numel() * r["w1"].element_size()
