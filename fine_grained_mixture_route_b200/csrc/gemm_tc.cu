@@ -1,9 +1,12 @@
-// Tensor-core kernels of the bf16 DeepSeekMoE layer: one persistent, warp-specialised
-// tcgen05 pipeline with four epilogues.
+// Tensor-core kernels of the DeepSeekMoE layer: one persistent, warp-specialised tcgen05
+// pipeline whose modes differ in their tile tables, operand loads and epilogues.
 //
+// Forward:
 //   ROUTER  scores z = x C^T of 128 tokens x N_m experts; the epilogue thread that owns a
 //           token row does the softmax over all N_m experts and the top-N_r selection
 //           ("《DeepSeekMoE》深度解读报告" §3.1, Eq. 3-5 in prose).
+//   ROUTERP split-K variant of ROUTER for few token tiles: fp32 partial logits per K range,
+//           summed and ranked by a small CUDA-core kernel afterwards.
 //   GEMM1   [x_e] [w1_e | w3_e]^T for 128 rows x (128 + 128) columns with bias and SwiGLU in
 //           the epilogue: h = silu(x w1^T + b1) * (x w3^T + b3) (the `Expert` module of
 //           "DeepSeek MoE模型优化与未来演进及字节超稀疏内存技术").  Routed groups read the
@@ -14,22 +17,28 @@
 //           the epilogue adds the shared biases and writes the fp32 shared output, to which
 //           the combine kernel adds each token's gated routed rows in pick order (§2.3 and
 //           §3.1 of the DeepSeekMoE report: shared experts first, then the gated routed sum).
+//   Q8      GEMM1 / GEMM2R with e4m3 routed tiles (kind::f8f6f4, per-row scales applied to
+//           the fp32 accumulator in the epilogue); shared tiles of the same launch stay bf16.
+// Backward (MN-major B operands, read through 4-D TMA views, one request per stage):
+//   DH      dout W2 with the SwiGLU backward and the gate-gradient partial sums in the epilogue;
+//   DX      [da | dg] [W1 ; W3] per routed slot;  DXS  shared experts + dz C per token (fp32);
+//   DW      weight gradients, both operands MN-major, K = a group's rows; groups without rows
+//           are zero-filled by the producer's TMA stores and skip the MMA and epilogue.
 //
 // Pipeline (320 threads, one CTA per SM, persistent over a static round-robin tile order):
-//   warp 0      TMA producer: 128B-swizzled K-major tiles of A (16 KB) and B (up to 32 KB)
-//               into a 4-stage shared-memory ring, completion counted on mbarriers;
+//   warp 0      TMA producer: 128B-swizzled tiles of A (16 KB) and B (up to 32 KB) into a
+//               4-stage shared-memory ring, completion counted on mbarriers;
 //   warp 1      allocates 512 TMEM columns; one thread issues tcgen05.mma (M=128, N<=256,
-//               K=16, bf16 x bf16 -> fp32) and commits each stage back to the producer and
-//               each finished accumulator to the epilogue;
+//               bf16 K=16 or e4m3 K=32, fp32 accumulate) and commits each stage back to the
+//               producer and each finished accumulator to the epilogue;
 //   warps 2-9   epilogue: tcgen05.ld of their 32 TMEM lanes (one accumulator row per
 //               thread; the two warps of a lane quadrant split the columns), fp32 math,
-//               bf16 stores.  Two accumulators (2 x 256 columns) let the epilogue of one
-//               tile overlap the main loop of the next.
-//   ROUTERP     split-K variant of ROUTER for few token tiles: fp32 partial logits per
-//               K range, summed and ranked by a small CUDA-core kernel afterwards.
+//               stores through a per-warp shared-memory transpose.  Two accumulators
+//               (2 x 256 columns) let the epilogue of one tile overlap the main loop of the next.
 // Every mbarrier wait is bounded (a few seconds of %globaltimer); on expiry the kernel sets
 // an error bit, stops issuing, waits (bounded) for its own copies and MMAs in flight, frees
-// TMEM and returns.  No cluster launch and no multicast anywhere.
+// TMEM and returns.  A CTA-pair variant of the expert GEMMs (cta_group::2, clusters of two,
+// off by default) is in the source; no TMA load anywhere uses cluster multicast.
 #include <cuda.h>
 
 #include "common.cuh"
