@@ -124,3 +124,53 @@ def test_expert_parallel_two_gloo_ranks(gate_mode):
     for rank, err, eloc in res:
         assert eloc == 4, f"rank {rank}: {err}"
         assert err < 1e-12, f"rank {rank}: max error {err}"
+
+
+def _rank4(rank, world, port, q, tokens):
+    import torch.distributed as dist
+    import oracle.moe_oracle as O
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        rng = np.random.default_rng(9)
+        E, d, I, k, Is = 8, 10, 4, 3, 6
+        C = torch.from_numpy(rng.normal(0, 0.6, (E, d)))
+        routed = _stack(rng, E, d, I)
+        shared = _stack(rng, 2, d, Is)
+        bias = torch.from_numpy(rng.normal(0, 0.3, E))
+        xr = np.random.default_rng(200 + rank).normal(0, 1, (tokens[rank], d))
+        lo, hi = ep.expert_range(rank, world, E)
+        layer = ep.ExpertParallelMoE(C, {kk: v[lo:hi] for kk, v in routed.items()}, shared, k, gate_mode=2,
+                                     router_bias=bias, backend=OracleBackend(O))
+        out = layer(torch.from_numpy(xr)).numpy()
+        if tokens[rank] == 0:
+            err = 0.0 if out.shape == (0, d) else float("inf")
+        else:
+            ref = O.layer(xr, C.numpy(), {kk: v.numpy() for kk, v in routed.items()}, E, k,
+                          {kk: v.numpy() for kk, v in shared.items()}, 2, gate_mode=2, router_bias=bias.numpy())["out"]
+            err = float(np.abs(out - ref).max())
+        q.put((rank, err, layer.E_loc))
+    except Exception as exc:
+        q.put((rank, repr(exc), -1))
+        raise
+    finally:
+        dist.destroy_process_group()
+
+
+def test_expert_parallel_four_gloo_ranks_one_without_tokens():
+    # 2 experts per rank, sigmoid gates with a selection bias, 2 shared experts, and a rank that
+    # sends and receives nothing of its own (its experts still serve the other ranks)
+    tokens = [7, 0, 13, 4]
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = 29900 + os.getpid() % 90
+    procs = [ctx.Process(target=_rank4, args=(r, 4, port, q, tokens)) for r in range(4)]
+    for p in procs:
+        p.start()
+    res = sorted((q.get(timeout=240) for _ in procs), key=lambda r: r[0])
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for rank, err, eloc in res:
+        assert eloc == 2, f"rank {rank}: {err}"
+        assert err < 1e-12, f"rank {rank}: max error {err}"
