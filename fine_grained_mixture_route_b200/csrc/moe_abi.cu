@@ -315,7 +315,7 @@ MOE_EXPORT moe_status_t moe_route(const moe_shape_t* shape, const void* x, const
                                   size_t ws_bytes, moe_stream_t stream) {
     Dims D;
     MOE_TRY(to_dims(shape, &D));
-    if (!x || !centroids || !topk_idx || !topk_gate) return MOE_ERR_INVALID_ARG;
+    if (!centroids || (D.T > 0 && (!x || !topk_idx || !topk_gate))) return MOE_ERR_INVALID_ARG;
     MOE_TRY(check_ws(D, ws, ws_bytes));
     if (D.T == 0) return MOE_OK;
     MOE_TRY(check_device());
@@ -347,7 +347,7 @@ MOE_EXPORT moe_status_t moe_expert_ffn(const moe_shape_t* shape, const void* x, 
                                        moe_stream_t stream) {
     Dims D;
     MOE_TRY(to_dims(shape, &D));
-    if (!x || !offsets || !sorted_token || !y_sorted) return MOE_ERR_INVALID_ARG;
+    if (!offsets || (D.T > 0 && (!x || !sorted_token || !y_sorted))) return MOE_ERR_INVALID_ARG;
     MOE_TRY(check_weights(D, routed, D.q8));
     MOE_TRY(check_ws(D, ws, ws_bytes));
     if (D.T == 0) return MOE_OK;
@@ -363,9 +363,9 @@ MOE_EXPORT moe_status_t moe_combine(const moe_shape_t* shape, const void* x, con
                                     size_t ws_bytes, moe_stream_t stream) {
     Dims D;
     MOE_TRY(to_dims(shape, &D));
-    if (!y_sorted || !slot_of || !out) return MOE_ERR_INVALID_ARG;
+    if (D.T > 0 && (!y_sorted || !slot_of || !out)) return MOE_ERR_INVALID_ARG;
     if (D.Ks > 0) {
-        if (!x) return MOE_ERR_INVALID_ARG;
+        if (D.T > 0 && !x) return MOE_ERR_INVALID_ARG;
         MOE_TRY(check_weights(D, shared));
     } else if (shared) {
         return MOE_ERR_INVALID_ARG;
@@ -428,7 +428,7 @@ moe_status_t layer_forward_impl(const moe_shape_t* shape, const void* x, const v
                                 size_t ctx_bytes = 0) {
     Dims D;
     MOE_TRY(to_dims(shape, &D));
-    if (!x || !centroids || !out) return MOE_ERR_INVALID_ARG;
+    if (!centroids || (D.T > 0 && (!x || !out))) return MOE_ERR_INVALID_ARG;
     MOE_TRY(check_weights(D, routed, D.q8));
     if (D.Ks > 0) MOE_TRY(check_weights(D, shared));
     else if (shared) return MOE_ERR_INVALID_ARG;
@@ -520,7 +520,7 @@ moe_status_t layer_backward_impl(const moe_shape_t* shape, const void* x, const 
     Dims D;
     MOE_TRY(to_dims(shape, &D));
     MOE_TRY(check_train(D));
-    if (!x || !centroids || !dout || !ctx || !dx || !dcentroids) return MOE_ERR_INVALID_ARG;
+    if (!centroids || !ctx || !dcentroids || (D.T > 0 && (!x || !dout || !dx))) return MOE_ERR_INVALID_ARG;
     MOE_TRY(check_weights(D, routed));
     if (D.Ks > 0) MOE_TRY(check_weights(D, shared));
     else if (shared || gshared) return MOE_ERR_INVALID_ARG;

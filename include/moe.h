@@ -37,7 +37,9 @@
  *  - Sizes: 0 <= T, T * top_k < 2^31; 1 <= n_experts <= 1024; 1 <= top_k <= min(32,
  *    n_experts); 0 <= n_shared <= 16; d, inter, inter_shared >= 1.  For MOE_BF16, d, inter
  *    and inter_shared must be multiples of 8 (16-byte rows for the tensor-memory-access
- *    unit).  T == 0 is a valid no-op.
+ *    unit).  T == 0 is a valid no-op: nothing is launched (moe_permute still writes zero counts
+ *    and offsets), and pointers to per-token arrays (x, out, picks, gates, slot lists, routed
+ *    rows, dout, dx) may then be NULL, as empty framework tensors' data pointers are.
  *  - FP8 routed experts (shape->routed_fmt == MOE_FMT_E4M3; dtype must be MOE_BF16, d and inter
  *    multiples of 16): the routed w1, w3, w2 are e4m3 codes (1 byte each, same layouts) with
  *    fp32 scales per output channel in s1 [E, inter], s3 [E, inter], s2 [E, d]; the weight is

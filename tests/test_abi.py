@@ -125,6 +125,15 @@ def test_argument_errors_return_before_any_launch(lib):
     ne = moe.workspace_bytes(sh_e)
     assert lib.moe_route(S(sh_e), fake, fake, None, fake, fake, fake, ne, None) == moe.MOE_OK
     assert lib.moe_layer_forward(S(sh_e), fake, fake, None, S(w), S(w), fake, None, None, None, fake, ne, None) == moe.MOE_OK
+    # ... also with the null data pointers of empty tensors for every per-token array
+    assert lib.moe_route(S(sh_e), None, fake, None, None, None, fake, ne, None) == moe.MOE_OK
+    assert lib.moe_expert_ffn(S(sh_e), None, fake, None, None, S(w), None, fake, ne, None) == moe.MOE_OK
+    assert lib.moe_combine(S(sh_e), None, S(w), None, None, None, fake, ne, None) == moe.MOE_OK
+    assert lib.moe_layer_forward(S(sh_e), None, fake, None, S(w), S(w), None, None, None, None, fake, ne, None) == \
+        moe.MOE_OK
+    # ... but the per-expert and weight arguments are still required
+    assert lib.moe_route(S(sh_e), None, None, None, None, None, fake, ne, None) == moe.MOE_ERR_INVALID_ARG
+    assert lib.moe_expert_ffn(S(sh_e), None, None, None, None, S(w), None, fake, ne, None) == moe.MOE_ERR_INVALID_ARG
     assert lib.moe_ws_init(None, 0, None) == moe.MOE_ERR_WORKSPACE
     assert lib.moe_check_device_error(None, 0, None, None) == moe.MOE_ERR_WORKSPACE
     # scales: required by e4m3 routed experts, refused elsewhere (native routed, shared)
@@ -195,6 +204,9 @@ def test_training_entry_points_validate(lib):
         == moe.MOE_ERR_INVALID_ARG                                   # gate mode 2: the bias only selects
     sh0 = _shape(T=0)
     assert b(*args(sh=sh0, nc=moe.train_ctx_bytes(sh0), nb=moe.backward_workspace_bytes(sh0))) == moe.MOE_OK
+    a0 = args(sh=sh0, nc=moe.train_ctx_bytes(sh0), nb=moe.backward_workspace_bytes(sh0))
+    a0[1], a0[6], a0[9] = None, None, None                          # x, dout, dx of an empty batch
+    assert b(*a0) == moe.MOE_OK
 
 
 def test_balance_stats_validate(lib):
