@@ -145,6 +145,58 @@ def shape_of(x: torch.Tensor, centroids_or_E, routed: Dict, top_k: int, shared: 
                       fmt)
 
 
+# ----------------------------------------------------------------------------- argument checks
+# The C ABI sees only pointers: a tensor of the wrong element type or size would make a kernel read
+# or write past its allocation.  Every entry point below checks, before any call, that each tensor
+# has the element type the shape implies, is contiguous, holds at least the elements the kernels
+# touch, and lives on the layer's CUDA device.
+def _layer_dtype(shape: MoeShape) -> torch.dtype:
+    return torch.bfloat16 if shape.dtype == MOE_BF16 else torch.float32
+
+
+def _need(t, name: str, numel: int, dtype: torch.dtype, device: Optional[torch.device]):
+    if t is None:
+        return
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} has dtype {t.dtype}; this layer shape needs {dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if t.numel() < numel:
+        raise ValueError(f"{name} holds {t.numel()} elements; the layer shape needs {numel}")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}; the layer runs on {device}")
+
+
+def _device(x: torch.Tensor) -> torch.device:
+    if not isinstance(x, torch.Tensor):
+        raise TypeError("expected a torch.Tensor")
+    return x.device
+
+
+def _on_cuda(dev: torch.device):
+    """Last check of every entry point: there is no CPU path."""
+    if dev.type != "cuda":
+        raise ValueError(f"the layer runs on a CUDA device (sm_100a); got tensors on {dev}")
+
+
+def _need_stack(w: Optional[Dict], name: str, shape: MoeShape, shared: bool, device, grads: bool = False):
+    """An expert stack (or its gradients, grads=True) in the layout of include/moe.h."""
+    if w is None:
+        return
+    E = shape.n_shared if shared else shape.n_experts
+    I = shape.inter_shared if shared else shape.inter
+    d, dt = shape.d, _layer_dtype(shape)
+    codes = not shared and not grads and shape.routed_fmt == FMT_E4M3
+    wdt = torch.uint8 if codes else dt
+    for k, n, kdt in (("w1", E * I * d, wdt), ("w3", E * I * d, wdt), ("w2", E * d * I, wdt),
+                      ("b1", E * I, dt), ("b3", E * I, dt), ("b2", E * d, dt),
+                      ("s1", E * I, torch.float32), ("s3", E * I, torch.float32), ("s2", E * d, torch.float32)):
+        if k in w:
+            _need(w[k], f"{name}.{k}", n, kdt, device)
+
+
 def _bias_ptr(router_bias: Optional[torch.Tensor]):
     if router_bias is None:
         return None
@@ -197,6 +249,13 @@ def check_device_error(ws: torch.Tensor, stream=None) -> int:
 
 def route(shape: MoeShape, x, centroids, ws, idx=None, gate=None, stream=None, router_bias=None):
     T, k = shape.T, shape.top_k
+    dev, dt = _device(x), _layer_dtype(shape)
+    _need(x, "x", T * shape.d, dt, dev)
+    _need(centroids, "centroids", shape.n_experts * shape.d, dt, dev)
+    _need(idx, "idx", T * k, torch.int32, dev)
+    _need(gate, "gate", T * k, torch.float32, dev)
+    _need(router_bias, "router_bias", shape.n_experts, torch.float32, dev)
+    _on_cuda(dev)
     idx = torch.empty((T, k), dtype=torch.int32, device=x.device) if idx is None else idx
     gate = torch.empty((T, k), dtype=torch.float32, device=x.device) if gate is None else gate
     _check(_lib().moe_route(ctypes.byref(shape), _ptr(x), _ptr(centroids), _bias_ptr(router_bias), _ptr(idx),
@@ -206,7 +265,10 @@ def route(shape: MoeShape, x, centroids, ws, idx=None, gate=None, stream=None, r
 
 def permute(shape: MoeShape, idx, gate, ws, stream=None):
     S, E = shape.T * shape.top_k, shape.n_experts
-    dev = idx.device
+    dev = _device(idx)
+    _need(idx, "idx", S, torch.int32, dev)
+    _need(gate, "gate", S, torch.float32, dev)
+    _on_cuda(dev)
     counts = torch.empty(E, dtype=torch.int32, device=dev)
     offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
     sorted_token = torch.empty(S, dtype=torch.int32, device=dev)
@@ -221,6 +283,14 @@ def permute(shape: MoeShape, idx, gate, ws, stream=None):
 
 def expert_ffn(shape: MoeShape, x, offsets, sorted_token, sorted_gate, routed: Dict, ws, y=None, stream=None):
     S = shape.T * shape.top_k
+    dev, dt = _device(x), _layer_dtype(shape)
+    _need(x, "x", shape.T * shape.d, dt, dev)
+    _need(offsets, "offsets", shape.n_experts + 1, torch.int32, dev)
+    _need(sorted_token, "sorted_token", S, torch.int32, dev)
+    _need(sorted_gate, "sorted_gate", S, torch.float32, dev)
+    _need(y, "y", S * shape.d, dt, dev)
+    _need_stack(routed, "routed", shape, False, dev)
+    _on_cuda(dev)
     y = torch.empty((S, shape.d), dtype=x.dtype, device=x.device) if y is None else y
     w = _weights(routed)
     _check(_lib().moe_expert_ffn(ctypes.byref(shape), _ptr(x), _ptr(offsets), _ptr(sorted_token), _ptr(sorted_gate),
@@ -229,6 +299,14 @@ def expert_ffn(shape: MoeShape, x, offsets, sorted_token, sorted_gate, routed: D
 
 
 def combine(shape: MoeShape, x, shared: Optional[Dict], y_sorted, slot_of, ws, out=None, stream=None):
+    dev, dt = _device(y_sorted), _layer_dtype(shape)
+    S = shape.T * shape.top_k
+    _need(x if shape.n_shared > 0 else None, "x", shape.T * shape.d, dt, dev)
+    _need(y_sorted, "y_sorted", S * shape.d, dt, dev)
+    _need(slot_of, "slot_of", S, torch.int32, dev)
+    _need(out, "out", shape.T * shape.d, dt, dev)
+    _need_stack(shared, "shared", shape, True, dev)
+    _on_cuda(dev)
     out = torch.empty((shape.T, shape.d), dtype=y_sorted.dtype, device=y_sorted.device) if out is None else out
     w = _weights(shared)
     _check(_lib().moe_combine(ctypes.byref(shape), _ptr(x), None if w is None else ctypes.byref(w), _ptr(y_sorted),
@@ -236,9 +314,26 @@ def combine(shape: MoeShape, x, shared: Optional[Dict], y_sorted, slot_of, ws, o
     return out
 
 
+def _need_layer(shape: MoeShape, x, centroids, routed, shared, out=None, idx=None, gate=None, counts=None,
+                router_bias=None):
+    dev, dt = _device(x), _layer_dtype(shape)
+    T, d, E, k = shape.T, shape.d, shape.n_experts, shape.top_k
+    _need(x, "x", T * d, dt, dev)
+    _need(centroids, "centroids", E * d, dt, dev)
+    _need(out, "out", T * d, dt, dev)
+    _need(idx, "idx", T * k, torch.int32, dev)
+    _need(gate, "gate", T * k, torch.float32, dev)
+    _need(counts, "counts", E, torch.int32, dev)
+    _need(router_bias, "router_bias", E, torch.float32, dev)
+    _need_stack(routed, "routed", shape, False, dev)
+    _need_stack(shared, "shared", shape, True, dev)
+    return dev
+
+
 def layer_forward(shape: MoeShape, x, centroids, routed: Dict, shared: Optional[Dict], ws, out=None,
                   idx=None, gate=None, counts=None, stream=None, router_bias=None):
     """One call of the whole layer; idx / gate / counts are optional output tensors."""
+    _on_cuda(_need_layer(shape, x, centroids, routed, shared, out, idx, gate, counts, router_bias))
     out = torch.empty((shape.T, shape.d), dtype=x.dtype, device=x.device) if out is None else out
     rw = _weights(routed)
     sw = _weights(shared)
@@ -284,6 +379,7 @@ def new_train_buffers(shape: MoeShape, device="cuda"):
 def layer_forward_train(shape: MoeShape, x, centroids, routed: Dict, shared: Optional[Dict], ws, ctx, out=None,
                         stream=None, router_bias=None):
     """moe_layer_forward plus the training context in ctx."""
+    _on_cuda(_need_layer(shape, x, centroids, routed, shared, out, router_bias=router_bias))
     out = torch.empty((shape.T, shape.d), dtype=x.dtype, device=x.device) if out is None else out
     rw, sw = _weights(routed), _weights(shared)
     _check(_lib().moe_layer_forward_train(ctypes.byref(shape), _ptr(x), _ptr(centroids), _bias_ptr(router_bias),
@@ -323,7 +419,15 @@ def layer_backward(shape: MoeShape, x, centroids, routed: Dict, shared: Optional
     """moe_layer_backward (moe_layer_backward_timed when `events` holds BWD_STAGES + 1 events):
     returns {dx, dcentroids, drouter_bias (or None), routed: {...}, shared: {...} or None}, written
     into `grads` when given (see new_grads), else into tensors allocated here."""
+    dev = _need_layer(shape, x, centroids, routed, shared, router_bias=router_bias)
+    _need(dout, "dout", shape.T * shape.d, _layer_dtype(shape), dev)
     g = new_grads(x, centroids, routed, shared, router_bias_grad) if grads is None else grads
+    _need(g["dx"], "dx", shape.T * shape.d, _layer_dtype(shape), dev)
+    _need(g["dcentroids"], "dcentroids", shape.n_experts * shape.d, torch.float32, dev)
+    _need(g.get("drouter_bias"), "drouter_bias", shape.n_experts, torch.float32, dev)
+    _need_stack(g["routed"], "grads.routed", shape, False, dev, grads=True)
+    _need_stack(g["shared"], "grads.shared", shape, True, dev, grads=True)
+    _on_cuda(dev)
     gr_c, gs_c = _grad_struct(g["routed"]), _grad_struct(g["shared"])
     rw, sw = _weights(routed), _weights(shared)
     args = [ctypes.byref(shape), _ptr(x), _ptr(centroids), _bias_ptr(router_bias), ctypes.byref(rw),
@@ -340,6 +444,12 @@ def layer_backward(shape: MoeShape, x, centroids, routed: Dict, shared: Optional
 
 def balance_stats(shape: MoeShape, x, centroids, counts, n_groups: int = 1, router_bias=None, ws=None, stream=None):
     """moe_balance_stats: returns {f, P (fp32 [n_experts]), expert_term, device_term (0-d fp32)}."""
+    dev = _device(x)
+    _need(x, "x", shape.T * shape.d, _layer_dtype(shape), dev)
+    _need(centroids, "centroids", shape.n_experts * shape.d, _layer_dtype(shape), dev)
+    _need(counts, "counts", shape.n_experts, torch.int32, dev)
+    _need(router_bias, "router_bias", shape.n_experts, torch.float32, dev)
+    _on_cuda(dev)
     n = int(_lib().moe_balance_workspace_bytes(ctypes.byref(shape)))
     if n == 0:
         raise ValueError("layer shape not supported for balance statistics")
@@ -381,6 +491,7 @@ def stage_events(stream=None, n_stages: int = NUM_STAGES):
 def layer_forward_timed(shape: MoeShape, x, centroids, routed: Dict, shared: Optional[Dict], ws, events,
                         out=None, idx=None, gate=None, counts=None, stream=None, router_bias=None):
     """layer_forward that also records `events` (from stage_events) at the stage boundaries."""
+    _on_cuda(_need_layer(shape, x, centroids, routed, shared, out, idx, gate, counts, router_bias))
     out = torch.empty((shape.T, shape.d), dtype=x.dtype, device=x.device) if out is None else out
     rw = _weights(routed)
     sw = _weights(shared)
