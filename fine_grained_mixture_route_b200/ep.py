@@ -71,8 +71,8 @@ class CudaBackend:
         from fine_grained_mixture_route_b200 import moe
         self.moe = moe
 
-    def shape(self, T, d, E, I, k, Ks, Is, bias, dtype, gate_mode):
-        return self.moe.make_shape(T, d, E, I, k, Ks, Is, bias, dtype, gate_mode)
+    def shape(self, T, d, E, I, k, Ks, Is, bias, dtype, gate_mode, routed_fmt=0):
+        return self.moe.make_shape(T, d, E, I, k, Ks, Is, bias, dtype, gate_mode, routed_fmt)
 
     def workspace(self, shape, device):
         return self.moe.new_workspace(shape, device)
@@ -147,7 +147,10 @@ class ExpertParallelMoE:
         row_of_t = torch.from_numpy(row_of).to(x.device)
         inv_t = torch.from_numpy(inv).to(x.device)
         offs_t = torch.from_numpy(offs).to(x.device)
-        shape_loc = be.shape(R, d, Eloc, I, 1, 0, 0, bias, x.dtype, 0)
+        # FP8 routed experts (e4m3 codes with their scales, quant.quantize_stack) run on the local
+        # expert call only; routing, exchange and combine do not touch the routed weights
+        fp8 = {"routed_fmt": 1} if self.routed["w1"].dtype == torch.uint8 else {}
+        shape_loc = be.shape(R, d, Eloc, I, 1, 0, 0, bias, x.dtype, 0, **fp8)
         if R > 0:
             ws_loc = be.workspace(shape_loc, x.device)
             x_loc = be.gather(x_recv, row_of_t, ws_loc)
