@@ -161,6 +161,11 @@ def bwd_stage_work(cfg: W.LayerConfig, touched: int):
     }
 
 
+def fmt_label(args, cfg: W.LayerConfig) -> str:
+    """Storage of the routed experts' weights: e4m3 codes, else the layer dtype."""
+    return "e4m3" if args.routed_fmt == "e4m3" else ("bf16" if cfg.dtype == torch.bfloat16 else "fp32")
+
+
 def layer_bytes(cfg: W.LayerConfig, touched: int, e4m3: bool = False) -> float:
     """Algorithmic bytes of the whole layer: weights of touched experts, shared experts,
     centroids, x in and out once (intermediates excluded: the method need not keep them)."""
@@ -344,7 +349,7 @@ def run_reference(args, cfg, rank, world):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": cfg.name, "tokens_per_step": n, "T": cfg.T, "d": cfg.d,
                        "n_experts": cfg.n_experts, "inter": cfg.inter, "top_k": cfg.top_k,
-                       "n_shared": cfg.n_shared, "routed_fmt": args.routed_fmt,
+                       "n_shared": cfg.n_shared, "routed_fmt": fmt_label(args, cfg),
                        "parallelism": "replicas" if world > 1 else "single"},
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
                              "sample": f"{n} consecutive tokens of the {cfg.name} batch per step"},
@@ -474,7 +479,7 @@ def run_ours(args, cfg, rank, world, local_rank):
         "config": {"workload": cfg.name, "T": cfg.T, "d": cfg.d, "n_experts": cfg.n_experts, "inter": cfg.inter,
                    "top_k": cfg.top_k, "n_shared": cfg.n_shared, "inter_shared": cfg.inter_shared,
                    "bias": cfg.has_bias, "routing": cfg.centroid_init, "gate_mode": args.gate_mode,
-                   "routed_fmt": args.routed_fmt,
+                   "routed_fmt": fmt_label(args, cfg),
                    "parallelism": f"replicas{world}" if world > 1 else "single",
                    "l2": "inputs larger than L2 (weights and activations), no flush",
                    "tokens_per_gpu": cfg.T},
