@@ -94,3 +94,17 @@ def test_warmup_must_be_three():
         bench.main(["--warmup", "2"])
     with pytest.raises(SystemExit):                     # e4m3 routed experts need a bf16 layer
         bench.main(["--workload", "tiny", "--routed-fmt", "e4m3"])
+
+
+def test_cpu_baseline_sample_grows_to_the_target():
+    import oracle.moe_oracle as O
+    cfg = W.CONFIGS["tiny"]
+    L = W.make_layer(cfg, "cpu", 0)
+    idx = O.route(L["x"].double().numpy(), L["centroids"].double().numpy(), cfg.top_k)["idx"]
+    # a first sample under min_s grows (here up to max_tokens); one at or above it is reported as is
+    grown = bench.cpu_baseline(cfg, L, idx, n_tokens=4, target_s=1e9, min_s=1e9, max_tokens=40)
+    assert "first 40 tokens" in grown["sample"] and grown["value"] > 0 and grown["kind"] == "oracle"
+    kept = bench.cpu_baseline(cfg, L, idx, n_tokens=4, min_s=0.0)
+    assert "first 4 tokens" in kept["sample"]
+    capped = bench.cpu_baseline(cfg, L, idx, n_tokens=4, target_s=1e9, min_s=1e9, max_tokens=10**6)
+    assert f"first {cfg.T} tokens" in capped["sample"]                 # never more than the batch
