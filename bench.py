@@ -161,6 +161,19 @@ def bwd_stage_work(cfg: W.LayerConfig, touched: int):
     }
 
 
+def routing_stats(counts) -> dict:
+    """Expert load of one batch from the per-expert slot counts: experts with tokens, max and mean
+    slots per expert, their ratio, and the hit entropy -sum p log p of p = counts / slots (at most
+    log N_m, reached by uniform counts)."""
+    c = np.asarray(counts, dtype=np.float64)
+    S = c.sum()
+    p = c[c > 0] / S if S > 0 else np.zeros(0)
+    mean = S / len(c)
+    return {"experts_touched": int((c > 0).sum()), "max_slots": int(c.max()), "mean_slots": mean,
+            "max_over_mean": float(c.max() / mean) if mean > 0 else 0.0,
+            "hit_entropy": float(-(p * np.log(p)).sum()), "hit_entropy_max": float(np.log(len(c)))}
+
+
 def fmt_label(args, cfg: W.LayerConfig) -> str:
     """Storage of the routed experts' weights: e4m3 codes, else the layer dtype."""
     return "e4m3" if args.routed_fmt == "e4m3" else ("bf16" if cfg.dtype == torch.bfloat16 else "fp32")
@@ -494,6 +507,7 @@ def run_ours(args, cfg, rank, world, local_rank):
         "tflops": total_flops / step_s / 1e12 * world,
         "hbm_gbs_algorithmic": lbytes / step_s / 1e9,
         "experts_touched": touched,
+        "routing": routing_stats(counts.cpu().numpy()),
         "stage_ms": stage_ms,
         "roofline": roofline,
         "gpu_launches": launches_per_step * args.steps,
@@ -584,6 +598,7 @@ def run_train(args, cfg, rank, world, local_rank):
         "tflops": (fwd_flops + bwd_flops) / (ms / 1e3) / 1e12 * world,
         "backward_tflops": bwd_flops / (sum(v for k, v in stage_ms.items() if k != "forward_train") / 1e3) / 1e12,
         "experts_touched": touched,
+        "routing": routing_stats(counts.cpu().numpy()),
         "stage_ms": stage_ms,
         "roofline": {"bound": bound, "kernel": dom, "achieved": achieved, "peak": peak, "unit": unit,
                      "frac": achieved / peak,

@@ -108,3 +108,14 @@ def test_cpu_baseline_sample_grows_to_the_target():
     assert "first 4 tokens" in kept["sample"]
     capped = bench.cpu_baseline(cfg, L, idx, n_tokens=4, target_s=1e9, min_s=1e9, max_tokens=10**6)
     assert f"first {cfg.T} tokens" in capped["sample"]                 # never more than the batch
+
+
+def test_routing_stats():
+    import math
+    u = bench.routing_stats([5] * 8)
+    assert u["experts_touched"] == 8 and u["max_over_mean"] == 1.0
+    assert abs(u["hit_entropy"] - math.log(8)) < 1e-12 and u["hit_entropy"] == pytest.approx(u["hit_entropy_max"])
+    one = bench.routing_stats([0, 0, 12, 0])
+    assert one["experts_touched"] == 1 and one["hit_entropy"] == 0.0 and one["max_over_mean"] == 4.0
+    two = bench.routing_stats([3, 1, 0, 0])
+    assert two["hit_entropy"] == pytest.approx(-(0.75 * math.log(0.75) + 0.25 * math.log(0.25)))
