@@ -4,6 +4,7 @@
 #include <cstring>
 
 #include "common.cuh"
+#include "abi_checks.h"
 #include "launch.h"
 
 #define MOE_EXPORT __attribute__((visibility("default")))
@@ -113,6 +114,9 @@ BwdLayout bwd_layout(const Dims& D) {
     return B;
 }
 
+}  // namespace
+
+// Shape and device checks shared with the allocation-free grouping entry point (abi_checks.h).
 moe_status_t to_dims(const moe_shape_t* s, Dims* D) {
     if (!s) return MOE_ERR_INVALID_ARG;
     if (s->dtype != MOE_F32 && s->dtype != MOE_BF16) return MOE_ERR_INVALID_ARG;
@@ -171,6 +175,8 @@ moe_status_t check_device() {
     if (major != 10) return MOE_ERR_UNSUPPORTED;   // built for sm_100a only
     return MOE_OK;
 }
+
+namespace {
 
 #define MOE_TRY(expr)                              \
     do {                                           \

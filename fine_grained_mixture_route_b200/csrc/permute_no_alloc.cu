@@ -11,11 +11,15 @@
 //
 // The array is MOE_PERMUTE_NO_ALLOC_SCRATCH_BYTES (1 MiB) of every GPU that loads the
 // library, held until the process exits.  Host code must not pass the array's name to a
-// kernel (on the host it is only a stand-in symbol); its device address is looked up once
-// per device with cudaGetSymbolAddress, with that device current, on the first call made
-// on that device.
+// kernel (on the host it is only a stand-in symbol); its device address is looked up with
+// cudaGetSymbolAddress, with the device current, on the first call made in each CUDA context
+// (each device's primary context, and again after cudaDeviceReset or in a context the caller
+// created), and kept under that context's process-unique id.
+#include <cuda.h>
+
 #include <mutex>
 
+#include "abi_checks.h"
 #include "common.cuh"
 #include "launch.h"
 
@@ -25,7 +29,6 @@ namespace moe {
 namespace {
 
 constexpr size_t kScratchBytes = MOE_PERMUTE_NO_ALLOC_SCRATCH_BYTES;
-constexpr int kMaxDevices = 64;
 
 // The scratch: one int32 per (histogram block, expert).  Nothing in it has to start at zero:
 // the histogram kernel of every call overwrites each entry that the scan and scatter kernels
@@ -34,20 +37,67 @@ constexpr int kMaxDevices = 64;
 static __device__ __align__(256) int32_t g_permute_scratch[kScratchBytes / sizeof(int32_t)];
 
 std::mutex g_mutex;
-int32_t* g_scratch_ptr[kMaxDevices] = {};
 
-// Device address of the scratch on the current device (looked up once per device).
-moe_status_t scratch_for_current_device(int32_t** out) {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
-    if (dev < 0 || dev >= kMaxDevices) return MOE_ERR_UNSUPPORTED;
-    std::lock_guard<std::mutex> lock(g_mutex);
-    if (!g_scratch_ptr[dev]) {
-        void* p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_permute_scratch) != cudaSuccess || !p) return MOE_ERR_CUDA;
-        g_scratch_ptr[dev] = static_cast<int32_t*>(p);
+// Context ids (cuCtxGetId: unique for the life of the process, never reused) with the scratch
+// address that was looked up in that context.  A context that is destroyed and replaced (for
+// instance by cudaDeviceReset) gets a new id, so a stale address is never handed out.
+constexpr int kMaxContexts = 64;
+struct CachedAddress {
+    unsigned long long ctx_id;
+    int32_t* ptr;
+};
+CachedAddress g_cache[kMaxContexts] = {};
+int g_cached = 0;
+
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+
+// Id of the calling thread's current context; false when it has none yet or the driver
+// cannot tell.
+bool current_context_id(unsigned long long* id) {
+    static CtxGetCurrentFn get_current = nullptr;
+    static CtxGetIdFn get_id = nullptr;
+    static bool resolved = false;
+    if (!resolved) {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_current = (CtxGetCurrentFn)f;
+        f = nullptr;
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = (CtxGetIdFn)f;
+        resolved = true;
     }
-    *out = g_scratch_ptr[dev];
+    if (!get_current || !get_id) return false;
+    CUcontext ctx = nullptr;
+    if (get_current(&ctx) != CUDA_SUCCESS || !ctx) return false;
+    return get_id(ctx, id) == CUDA_SUCCESS;
+}
+
+// Device address of the scratch in the current context (looked up on the first call there).
+moe_status_t scratch_for_current_context(int32_t** out) {
+    std::lock_guard<std::mutex> lock(g_mutex);
+    unsigned long long id = 0;
+    const bool have_id = current_context_id(&id);
+    if (have_id)
+        for (int i = 0; i < g_cached; ++i)
+            if (g_cache[i].ctx_id == id) {
+                *out = g_cache[i].ptr;
+                return MOE_OK;
+            }
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_permute_scratch) != cudaSuccess || !p) return MOE_ERR_CUDA;
+    // the lookup makes the device's primary context current if no context was
+    unsigned long long id2 = 0;
+    if (current_context_id(&id2)) {
+        if (g_cached == kMaxContexts) g_cached = 0;       // many contexts: start the table over
+        g_cache[g_cached].ctx_id = id2;
+        g_cache[g_cached].ptr = static_cast<int32_t*>(p);
+        ++g_cached;
+    }
+    *out = static_cast<int32_t*>(p);
     return MOE_OK;
 }
 
@@ -60,19 +110,18 @@ extern "C" MOE_EXPORT moe_status_t moe_permute_no_alloc(const moe_shape_t* s, co
                                                         const float* topk_gate, int32_t* counts, int32_t* offsets,
                                                         int32_t* sorted_token, float* sorted_gate, int32_t* slot_of,
                                                         moe_stream_t stream) {
-    if (!s || (s->dtype != MOE_F32 && s->dtype != MOE_BF16)) return MOE_ERR_INVALID_ARG;
-    if (s->T < 0 || s->n_experts < 1 || s->top_k < 1 || s->top_k > s->n_experts) return MOE_ERR_INVALID_ARG;
-    if (s->n_experts > 1024 || s->top_k > 32 || (long long)s->T * s->top_k >= (1LL << 31)) return MOE_ERR_UNSUPPORTED;
-    if (!counts || !offsets || (s->T > 0 && (!topk_idx || !topk_gate || !sorted_token || !sorted_gate || !slot_of)))
-        return MOE_ERR_INVALID_ARG;
     Dims D = {};
-    D.T = s->T; D.d = s->d; D.E = s->n_experts; D.I = s->inter; D.k = s->top_k;
-    D.Ks = 0; D.Is = 0; D.bias = false; D.bf16 = s->dtype == MOE_BF16;
+    moe_status_t st = to_dims(s, &D);                     // the shape rules of moe_permute
+    if (st != MOE_OK) return st;
+    if (!counts || !offsets || (D.T > 0 && (!topk_idx || !topk_gate || !sorted_token || !sorted_gate || !slot_of)))
+        return MOE_ERR_INVALID_ARG;
     const long long nblk = permute_blocks(D);
     const long long need = (nblk > 0 ? nblk : 1) * (long long)D.E * (long long)sizeof(int32_t);
     if (need > (long long)kScratchBytes) return MOE_ERR_UNSUPPORTED;   // beyond the fixed scratch
+    st = check_device();
+    if (st != MOE_OK) return st;
     int32_t* scratch = nullptr;
-    moe_status_t st = scratch_for_current_device(&scratch);
+    st = scratch_for_current_context(&scratch);
     if (st != MOE_OK) return st;
     cudaGetLastError();
     if (launch_permute(D, topk_idx, topk_gate, counts, offsets, sorted_token, sorted_gate, slot_of, scratch, nullptr,

@@ -383,13 +383,16 @@ moe_status_t moe_gather_rows(const void* src, const int32_t* row_of, int64_t n_r
  *   GPU that loads the library until the process exits.  A call needs
  *   ceil(T*top_k / 1024) * n_experts * 4 bytes of it (e.g. up to 1,048,576 slots with 256
  *   experts); larger shapes are rejected with MOE_ERR_UNSUPPORTED before any launch.
- *   Set-up: the first call on each device looks up the scratch's device address
- *   (cudaGetSymbolAddress, with that device current); make that first call before any
- *   stream capture.
+ *   Set-up: the first call in each CUDA context (a device's primary context, a context the
+ *   caller made, or the new primary context after cudaDeviceReset) looks up the scratch's
+ *   device address (cudaGetSymbolAddress, with that device current) and keeps it under the
+ *   context's process-unique id; make that first call before any stream capture.
  *   Sharing: every call on a device uses the same scratch, which keeps the last call's
  *   contents (nothing in it needs to start at zero).  Calls that overlap on the GPU race:
  *   order them on one stream.
- *   Errors: argument errors as moe_permute.  This variant has no error word: an expert
+ *   Errors: argument errors as moe_permute (the same shape rules, and MOE_ERR_UNSUPPORTED
+ *   on a GPU other than sm_100), checked before any launch.  This variant has no error
+ *   word, so unlike every other entry point it does not report bad indices: an expert
  *   index outside [0, n_experts) drops that slot, its slot_of entry is -1 and
  *   offsets[n_experts] comes out smaller than T*top_k.
  */
