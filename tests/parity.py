@@ -1,7 +1,8 @@
 """Comparison of the CUDA path with the fp64 oracle (used by the GPU tests and smoke()).
 
 Tolerances (from the layer's stated accuracy targets): outputs within a normwise relative
-error  max|gpu - ref| / max|ref|  of 2e-2 for bf16 layers and 1e-4 for fp32 layers; gates
+error  max|gpu - ref| / max|ref|  of 2e-2 for bf16 layers and 1e-4 for fp32 layers (the
+element-wise relative error with a 1e-3 * max|ref| floor is reported beside it); gates
 (fp32 in both) within 1e-4 relative.  Expert picks must equal the oracle's exactly except at
 near-ties, where the fp64 logit gap between the k-th and (k+1)-th expert (or between two
 consecutive picks, for the order) is below 1e-5; there any pick set whose every member
@@ -30,6 +31,31 @@ def expert_source(stack: Dict[str, Optional[torch.Tensor]]):
     def get(e: int):
         return {k: (None if v is None else f64(v[e])) for k, v in stack.items()}
     return get
+
+
+ELEM_FLOOR = 1e-3
+REPORT: list = []          # per-check error records, written out by tests/conftest.py when asked
+
+
+def elementwise(gpu: np.ndarray, ref: np.ndarray) -> float:
+    """Element-wise relative error with a floor: max_i |gpu_i - ref_i| / max(|ref_i|, 1e-3 max|ref|)
+    (reported beside the normwise error; the floor keeps elements near zero from dominating)."""
+    if not ref.size:
+        return 0.0
+    floor = ELEM_FLOOR * float(np.abs(ref).max())
+    den = np.maximum(np.abs(ref), floor)
+    if floor == 0.0:
+        den = np.where(den == 0.0, 1.0, den)
+    return float((np.abs(gpu - ref) / den).max())
+
+
+def record(case: str, tensor: str, gpu: np.ndarray, ref: np.ndarray, tol: float) -> float:
+    """Normwise error of one tensor (returned and asserted by the caller) and its element-wise
+    error, both kept in REPORT."""
+    e = normwise(gpu, ref)
+    REPORT.append({"case": case, "tensor": tensor, "normwise": e, "elementwise": elementwise(gpu, ref),
+                   "tol_normwise": tol})
+    return e
 
 
 def normwise(gpu: np.ndarray, ref: np.ndarray) -> float:

@@ -16,7 +16,7 @@ import torch
 import oracle.moe_oracle as O
 from fine_grained_mixture_route_b200 import moe
 from fine_grained_mixture_route_b200 import workloads as W
-from tests.parity import (TOL, check_permute, check_routing, expert_source, f64, normwise)
+from tests.parity import (TOL, check_permute, check_routing, expert_source, f64, normwise, record)
 
 pytestmark = pytest.mark.gpu
 
@@ -55,7 +55,7 @@ def _steps(shape, L, ws, idx_ref=None):
     return idx, gate, perm, y, out
 
 
-def _full_check(cfg, L, tokens=None):
+def _full_check(cfg, L, tokens=None, case=None):
     shape, ws, out, idx, gate, counts = _run(cfg, L)
     x64, c64 = f64(L["x"]), f64(L["centroids"])
     idx_np, gate_np = idx.cpu().numpy().astype(np.int64), gate.cpu().numpy()
@@ -75,15 +75,16 @@ def _full_check(cfg, L, tokens=None):
     ref = O.layer(x64[sel], c64, expert_source(L["routed"]), cfg.n_experts, cfg.top_k,
                   expert_source(Sh) if Sh is not None else None, cfg.n_shared, idx_override=idx_np[sel])
     tol = TOL[cfg.dtype]
-    e_out = normwise(f64(out)[sel], ref["out"])
+    case = case or cfg.name
+    e_out = record(case, "out", f64(out)[sel], ref["out"], tol)
     assert e_out <= tol, f"out error {e_out:.3e} > {tol}"
     # routed rows (gate * expert output) on their own: the shared term cannot hide them
     k = cfg.top_k
     slots = (sel[:, None] * k + np.arange(k)[None, :]).reshape(-1)
     y_np = f64(y)[p["slot_of"][slots]]
-    e_y = normwise(y_np, ref["Y"])
+    e_y = record(case, "Y", y_np, ref["Y"], tol)
     assert e_y <= tol, f"routed Y error {e_y:.3e} > {tol}"
-    e_routed = normwise(y_np.reshape(len(sel), k, -1).sum(1), ref["routed_sum"])
+    e_routed = record(case, "routed_sum", y_np.reshape(len(sel), k, -1).sum(1), ref["routed_sum"], tol)
     assert e_routed <= tol, f"routed sum error {e_routed:.3e}"
 
     # determinism
@@ -130,7 +131,7 @@ EDGE = [
 def test_edge_cases(case):
     _, base, kw = case
     cfg = W.scaled(W.CONFIGS[base], **kw)
-    stats = _full_check(cfg, W.make_layer(cfg, "cuda", seed=3))
+    stats = _full_check(cfg, W.make_layer(cfg, "cuda", seed=3), case=case[0])
     print(case[0], stats)
 
 
@@ -228,3 +229,74 @@ def test_router_variants(case, with_bias, gate_mode):
                   expert_source(Sh) if Sh is not None else None, cfg.n_shared, idx_override=idx_np[rows],
                   gate_mode=gate_mode, router_bias=b64)
     assert normwise(f64(out)[rows], ref["out"]) <= TOL[cfg.dtype]
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32], ids=["bf16", "f32"])
+@pytest.mark.parametrize("m", [4, 16])
+def test_split_identity_through_the_layer(m, dtype):
+    """Fine-grained segmentation (《DeepSeekMoE》深度解读报告 §2.2): one FFN split along its
+    intermediate dimension into m experts (oracle.split_expert: rows of w1 / w3 / b1 / b3, columns
+    of w2, b2 / m each), m identical centroids and N_r = N_m = m, no shared expert.  Every token
+    then picks all m experts with gate 1/m, so m * out equals the unsplit FFN: checked through the
+    library against the FFN in fp64, within the layer tolerance."""
+    T, d, I = 300, 256, 1024
+    one = W.scaled(W.CONFIGS["small"], T=T, d=d, n_experts=1, inter=I, top_k=1, n_shared=0, inter_shared=0,
+                   dtype=dtype)
+    st = W.make_expert_stack(one, False, "cpu", seed=4)
+    full = {k: (None if v is None else v[0].double().numpy()) for k, v in st.items()}
+    pieces = O.split_expert(full, m)
+    stack = {k: torch.from_numpy(np.stack([pc[k] for pc in pieces])).to(dtype).contiguous().cuda()
+             for k in ("w1", "b1", "w3", "b3", "w2", "b2")}
+    # the pieces are exact in the layer dtype: slices, and b2 / m with m a power of two
+    for k in ("w1", "w3", "b1", "b3", "b2"):
+        assert np.array_equal(f64(stack[k]), np.stack([pc[k] for pc in pieces])), k
+    w13 = torch.empty((2,) + tuple(stack["w1"].shape), dtype=dtype, device="cuda")
+    w13[0].copy_(stack["w1"]); w13[1].copy_(stack["w3"])
+    stack["w1"], stack["w3"] = w13[0], w13[1]
+    x = W.make_x(one, "cuda", seed=4)
+    C = W.make_centroids(W.scaled(one, n_experts=1), "cuda", seed=4).repeat(m, 1).contiguous()
+    shape = moe.shape_of(x, C, stack, m, None)
+    ws = moe.new_workspace(shape)
+    idx = torch.empty((T, m), dtype=torch.int32, device="cuda")
+    gate = torch.empty((T, m), dtype=torch.float32, device="cuda")
+    out = moe.layer_forward(shape, x, C, stack, None, ws, idx=idx, gate=gate)
+    moe.check_device_error(ws)
+    # every token picks all m experts (equal scores: lowest index first) with gate 1/m
+    assert torch.equal(idx.sort(dim=1).values.cpu(), torch.arange(m, dtype=torch.int32).repeat(T, 1))
+    assert torch.allclose(gate.cpu(), torch.full((T, m), 1.0 / m), rtol=1e-6, atol=0)
+    ref = O.expert_ffn(f64(x), full["w1"], full["b1"], full["w3"], full["b3"], full["w2"], full["b2"])
+    tol = TOL[dtype]
+    e = record(f"split_m{m}_{'bf16' if dtype == torch.bfloat16 else 'f32'}", "m*out", m * f64(out), ref, tol)
+    assert e <= tol, f"m * out vs the unsplit FFN: {e:.3e} > {tol}"
+
+
+@pytest.mark.parametrize("base,kw", [("small", dict(T=500, d=512, n_experts=32, top_k=4, inter=128, n_shared=2,
+                                                    inter_shared=192)),
+                                     ("tiny", dict(T=200, n_shared=2, inter_shared=48))], ids=["bf16", "f32"])
+def test_shared_experts_ignore_the_router(base, kw):
+    """Shared-expert isolation (《DeepSeekMoE》深度解读报告 §2.3): the shared experts see every
+    token whatever the router does.  Through the library: the combine with the routed rows set
+    to zero gives the shared part alone; it is bit-for-bit the same under two unrelated centroid
+    sets (which route the tokens differently), equals the oracle's shared sum within the layer
+    tolerance, and adding the routed rows back gives the layer output of that routing."""
+    cfg = W.scaled(W.CONFIGS[base], **kw)
+    L = W.make_layer(cfg, "cuda", seed=6)
+    x, R, Sh = L["x"], L["routed"], L["shared"]
+    C2 = W.make_centroids(cfg, "cuda", seed=7)
+    shared_only, picks = [], []
+    for C in (L["centroids"], C2):
+        shape = moe.shape_of(x, C, R, cfg.top_k, Sh)
+        ws = moe.new_workspace(shape)
+        idx, gate, perm, y, out = _steps(shape, dict(L, centroids=C), ws)
+        s_only = moe.combine(shape, x, Sh, torch.zeros_like(y), perm["slot_of"], ws)
+        moe.check_device_error(ws)
+        assert torch.equal(out, moe.layer_forward(shape, x, C, R, Sh, ws))
+        shared_only.append(s_only)
+        picks.append(idx)
+    assert not torch.equal(picks[0], picks[1]), "the two centroid sets should route differently"
+    assert torch.equal(shared_only[0], shared_only[1])
+    ref = O.layer(f64(x), f64(C2), expert_source(R), cfg.n_experts, cfg.top_k, expert_source(Sh), cfg.n_shared,
+                  idx_override=picks[1].cpu().numpy().astype(np.int64))
+    tol = TOL[cfg.dtype]
+    e = record(f"shared_bypass_{base}", "shared_only", f64(shared_only[0]), ref["shared_sum"], tol)
+    assert e <= tol, f"shared part vs oracle: {e:.3e}"
