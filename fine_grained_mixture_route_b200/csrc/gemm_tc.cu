@@ -174,22 +174,31 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
-// Bounded wait; false when the pipeline was aborted or the wait ran out of time.
-__device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag, uint32_t* err,
-                                       bool honour_abort = true) {
+// Bounded wait on the phase `parity` of an mbarrier: true once it completes; false when the
+// pipeline was aborted (abort_flag set by another role) or the wait gave up after limit_ns of
+// %globaltimer or WAIT_MAX_POLLS polls, whichever comes first; giving up sets abort_flag and
+// error bit 2.
+constexpr uint32_t WAIT_MAX_POLLS = 1u << 30;
+__device__ __forceinline__ bool mbar_wait_limit(uint32_t bar, uint32_t parity, volatile int* abort_flag, uint32_t* err,
+                                                bool honour_abort, unsigned long long limit_ns) {
     if (mbar_try_wait(bar, parity)) return true;
     const unsigned long long t0 = globaltimer();
     for (uint32_t i = 1;; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
         if ((i & 63u) == 0u) {
             if (honour_abort && *abort_flag) return false;
-            if (globaltimer() - t0 > WAIT_NS) {
+            if (globaltimer() - t0 > limit_ns || i >= WAIT_MAX_POLLS) {
                 *abort_flag = 1;
                 flag_error(err, ERR_PIPE_TIMEOUT);
                 return false;
             }
         }
     }
+}
+// The pipeline's wait: a few seconds at most.
+__device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag, uint32_t* err,
+                                       bool honour_abort = true) {
+    return mbar_wait_limit(bar, parity, abort_flag, err, honour_abort, WAIT_NS);
 }
 
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar, int c0, int c1) {
@@ -1360,6 +1369,43 @@ __global__ void __launch_bounds__(THREADS, 1) moe_tc_kernel(const __grid_constan
     }
 }
 
+// Self-test of the bounded wait (the path a pipeline takes when a barrier is never completed):
+// one warp allocates tensor memory as the pipeline does, thread 0 initialises an mbarrier that
+// nothing arrives at and waits on it through mbar_wait_limit; the wait can only end by giving up
+// (error bit 2).  Then the warp frees the tensor memory and the kernel returns; out (if given):
+// out[0] = 1 if the wait gave up (0 if it somehow completed), out[1] = the ns it waited.
+__global__ void __launch_bounds__(32, 1) wait_selftest_kernel(unsigned long long limit_ns, uint32_t* err,
+                                                              unsigned long long* out) {
+    __shared__ __align__(8) uint64_t bar;
+    __shared__ uint32_t tmem_holder;
+    __shared__ int abort_flag;
+    const uint32_t b = smem_u32(&bar);
+    if (threadIdx.x == 0) {
+        mbar_init(b, 1);
+        abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&tmem_holder)),
+                 "r"(32)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    tc_fence_before();
+    __syncwarp();
+    tc_fence_after();
+    if (threadIdx.x == 0) {
+        const unsigned long long t0 = globaltimer();
+        const bool done = mbar_wait_limit(b, 0, &abort_flag, err, true, limit_ns);
+        if (out) {
+            out[0] = done ? 0ull : 1ull;
+            out[1] = globaltimer() - t0;
+        }
+    }
+    tc_fence_before();
+    __syncwarp();
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_holder), "r"(32) : "memory");
+}
+
 // ------------------------------------------------------------------------------ host side
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -1512,6 +1558,12 @@ Params base_params(const Dims& D, uint32_t* err) {
 }
 
 }  // namespace tc
+
+cudaError_t launch_wait_selftest(unsigned long long limit_ns, uint32_t* err, unsigned long long* out,
+                                 cudaStream_t stream) {
+    tc::wait_selftest_kernel<<<1, 32, 0, stream>>>(limit_ns, err, out);
+    return cudaGetLastError();
+}
 
 int num_sms() {
     static int n = 0;

@@ -57,6 +57,16 @@ cudaError_t launch_quant_rows(const void* src, const int32_t* row_of, long long 
 // dst[p, :] = src[row_of[p], :] for rows of row_bytes (a multiple of 4) bytes; bad index -> bit 4, zeros
 cudaError_t launch_gather_rows_generic(const void* src, const int32_t* row_of, long long n_rows, long long src_rows,
                                        int row_bytes, void* dst, uint32_t* err, cudaStream_t stream);
+// Self-test of the GEMM pipeline's bounded wait: one warp allocates 32 tensor-memory columns,
+// waits on an mbarrier that nothing completes until limit_ns pass (error bit 2), frees them;
+// out (optional, 2 x u64): 1 if the wait gave up, and the ns waited
+cudaError_t launch_wait_selftest(unsigned long long limit_ns, uint32_t* err, unsigned long long* out,
+                                 cudaStream_t stream);
+// ids[r] = (segment holding row r) % modulo for segments of counts[q] consecutive rows
+// (n_seg <= SEGMENT_MAX); rows past the last segment get -1 and bit 4, as do negative counts
+constexpr int SEGMENT_MAX = 4096;
+cudaError_t launch_segment_ids(const int32_t* counts, int n_seg, int modulo, long long n_rows, int32_t* ids,
+                               uint32_t* err, cudaStream_t stream);
 // dst[p, :] = src[row_of[p], :] for byte rows of row_bytes (a multiple of 16), and dscale[p] =
 // sscale[row_of[p]] when dscale is given; an index outside [0, src_rows) sets bit 4 and gives a
 // zero row with scale 1.

@@ -751,4 +751,30 @@ MOE_EXPORT moe_status_t moe_gather_rows(const void* src, const int32_t* row_of, 
     return MOE_OK;
 }
 
+MOE_EXPORT moe_status_t moe_selftest_wait_timeout(uint64_t limit_ns, uint64_t* out, void* ws, size_t ws_bytes,
+                                                  moe_stream_t stream) {
+    if (limit_ns < 1000ull || limit_ns > 10000000000ull) return MOE_ERR_INVALID_ARG;
+    if (!ws || ws_bytes < 256 || ((uintptr_t)ws & 15u)) return MOE_ERR_WORKSPACE;
+    if (out && ((uintptr_t)out & 7u)) return MOE_ERR_INVALID_ARG;
+    MOE_TRY(check_device());
+    cudaGetLastError();
+    MOE_CUDA(launch_wait_selftest(limit_ns, static_cast<uint32_t*>(ws), reinterpret_cast<unsigned long long*>(out),
+                                  (cudaStream_t)stream));
+    return MOE_OK;
+}
+
+MOE_EXPORT moe_status_t moe_segment_ids(const int32_t* counts, int32_t n_segments, int32_t modulo, int64_t n_rows,
+                                        int32_t* ids, void* ws, size_t ws_bytes, moe_stream_t stream) {
+    if (n_segments < 1 || modulo < 1 || n_rows < 0) return MOE_ERR_INVALID_ARG;
+    if (n_segments > SEGMENT_MAX) return MOE_ERR_UNSUPPORTED;
+    if (!ws || ws_bytes < 256 || ((uintptr_t)ws & 15u)) return MOE_ERR_WORKSPACE;
+    if (n_rows == 0) return MOE_OK;
+    if (!counts || !ids) return MOE_ERR_INVALID_ARG;
+    MOE_TRY(check_device());
+    cudaGetLastError();
+    MOE_CUDA(launch_segment_ids(counts, n_segments, modulo, n_rows, ids, static_cast<uint32_t*>(ws),
+                                (cudaStream_t)stream));
+    return MOE_OK;
+}
+
 }  // extern "C"

@@ -173,6 +173,57 @@ __global__ void gather_rows_generic_kernel(const uint32_t* __restrict__ src, con
     }
 }
 
+// ids[r] = q % modulo for the segment q that holds row r, the segments being consecutive runs
+// of counts[q] rows.  Every block scans the (at most SEGMENT_MAX) counts into shared memory,
+// then finds the segment of each of its rows by binary search over the segment starts.  A
+// negative count is taken as 0 and a row past the last segment gets -1; both set bit 4.
+constexpr int SEG_THREADS = 256;
+__global__ void __launch_bounds__(SEG_THREADS) segment_ids_kernel(const int32_t* __restrict__ counts, int n_seg,
+                                                                  int modulo, long long n_rows,
+                                                                  int32_t* __restrict__ ids, uint32_t* err) {
+    __shared__ long long start[SEGMENT_MAX + 1];
+    __shared__ long long chunk[SEG_THREADS];
+    const int per = (n_seg + SEG_THREADS - 1) / SEG_THREADS;
+    const int b = threadIdx.x * per, e = min(n_seg, b + per);
+    long long run = 0;
+    for (int q = b; q < e; ++q) {
+        const int c = counts[q];
+        if (c < 0 && blockIdx.x == 0) flag_error(err, ERR_INDEX_RANGE);
+        start[q] = run;                          // local start inside this thread's chunk
+        run += c > 0 ? c : 0;
+    }
+    chunk[threadIdx.x] = run;
+    __syncthreads();
+    if (threadIdx.x == 0) {                      // exclusive scan of the 256 chunk sums
+        long long acc = 0;
+        for (int i = 0; i < SEG_THREADS; ++i) {
+            const long long v = chunk[i];
+            chunk[i] = acc;
+            acc += v;
+        }
+        start[n_seg] = acc;
+    }
+    __syncthreads();
+    for (int q = b; q < e; ++q) start[q] += chunk[threadIdx.x];
+    __syncthreads();
+    const long long total = start[n_seg];
+    for (long long r = (long long)blockIdx.x * SEG_THREADS + threadIdx.x; r < n_rows;
+         r += (long long)gridDim.x * SEG_THREADS) {
+        if (r >= total) {
+            ids[r] = -1;
+            flag_error(err, ERR_INDEX_RANGE);
+            continue;
+        }
+        int lo = 0, hi = n_seg;                  // largest q with start[q] <= r: start[lo] <= r < start[hi]
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (start[mid] <= r) lo = mid;
+            else hi = mid;
+        }
+        ids[r] = lo % modulo;
+    }
+}
+
 }  // namespace
 
 cudaError_t launch_gather_rows_generic(const void* src, const int32_t* row_of, long long n_rows, long long src_rows,
@@ -218,6 +269,17 @@ cudaError_t launch_gather_code_rows(const uint8_t* src, const float* sscale, con
     const int blocks = (int)(n_rows < cap ? n_rows : cap);
     gather_code_rows_kernel<<<blocks, 128, 0, stream>>>((const uint4*)src, sscale, row_of, n_rows, src_rows,
                                                         row_bytes / 16, (uint4*)dst, dscale, err);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_segment_ids(const int32_t* counts, int n_seg, int modulo, long long n_rows, int32_t* ids,
+                               uint32_t* err, cudaStream_t stream) {
+    if (n_rows <= 0) return cudaSuccess;
+    if (n_seg < 1 || n_seg > SEGMENT_MAX || modulo < 1) return cudaErrorInvalidValue;
+    const long long need = (n_rows + SEG_THREADS - 1) / SEG_THREADS;
+    const long long cap = (long long)num_sms() * 4;
+    segment_ids_kernel<<<(int)(need < cap ? need : cap), SEG_THREADS, 0, stream>>>(counts, n_seg, modulo, n_rows, ids,
+                                                                                  err);
     return cudaGetLastError();
 }
 

@@ -10,15 +10,20 @@ Per forward (NCCL collectives through torch.distributed; every data step runs in
 kernels):
   1. route + group the local slots by expert (moe_route, moe_permute)
   2. exchange the per-expert slot counts (all_to_all of N x E/N int32) and read them on the host
-     (the row all_to_alls need their split sizes there)
-  3. gather the slot rows and gates in expert order (moe_gather_rows) and send them (all_to_all)
-  4. regroup the received rows by local expert (moe_gather_rows), run the local experts with the
-     gates (moe_expert_ffn, one slot per row), put the rows back in received order and return
-     them (all_to_all)
+     (the only host read: the row all_to_alls need their split sizes there)
+  3. gather the slot rows in expert order (moe_gather_rows) and send them with their gates
+     (all_to_all)
+  4. regroup the received rows by local expert on the device (moe_segment_ids gives each row its
+     local expert from the received counts, moe_permute with one pick per row groups them stably,
+     sources in order), run the local experts on them with the gates (moe_expert_ffn reads the
+     rows through the grouping), put the results back in received order (moe_gather_rows) and
+     return them (all_to_all)
   5. combine with the shared experts (moe_combine), exactly as the single-GPU layer does.
 
-The host-side plan (split sizes, regrouping permutation) is plain integer arithmetic in the
-functions below; the step functions come from a backend object (the CUDA one by default).
+Workspaces are kept between calls and grow only when a call needs more.  The host-side plan
+functions below (split sizes, and the regrouping permutation written out on the host) state
+what the device steps compute; the tests check them against brute force, and the CPU test
+backend uses them.
 """
 from __future__ import annotations
 
@@ -65,28 +70,42 @@ def regroup_plan(recv_counts: np.ndarray) -> Tuple[np.ndarray, np.ndarray, np.nd
 
 # ----------------------------------------------------------------------------- CUDA backend
 class CudaBackend:
-    """The library's kernels (the product path)."""
+    """The library's kernels (the product path).  Workspaces are cached per use and grow only
+    when a call needs more, so steady-state forwards allocate none."""
 
     def __init__(self):
         from fine_grained_mixture_route_b200 import moe
         self.moe = moe
+        self._ws: Dict[str, torch.Tensor] = {}
 
     def shape(self, T, d, E, I, k, Ks, Is, bias, dtype, gate_mode, routed_fmt=0):
         return self.moe.make_shape(T, d, E, I, k, Ks, Is, bias, dtype, gate_mode, routed_fmt)
 
-    def workspace(self, shape, device):
-        return self.moe.new_workspace(shape, device)
+    def workspace(self, shape, device, use: str = "layer"):
+        need = max(self.moe.workspace_bytes(shape), 256)
+        ws = self._ws.get(use)
+        if ws is None or ws.numel() < need or ws.device != torch.device(device):
+            ws = self.moe.new_workspace(shape, device)
+            self._ws[use] = ws
+        return ws
 
     def route_permute(self, shape, x, centroids, ws, router_bias):
         idx, gate = self.moe.route(shape, x, centroids, ws, router_bias=router_bias)
-        return self.moe.permute(shape, idx, gate, ws)
+        return dict(self.moe.permute(shape, idx, gate, ws), idx=idx, gate=gate)
 
     def gather(self, src, row_of, ws):
         return self.moe.gather_rows(src, row_of, ws)
 
-    def expert_ffn(self, shape, x, offsets, gates, routed, ws):
-        rows = torch.arange(x.shape[0], dtype=torch.int32, device=x.device)
-        return self.moe.expert_ffn(shape, x, offsets, rows, gates, routed, ws)
+    def regroup(self, shape_loc, recv_counts, gates, ws):
+        """Received rows (source-major, inside a source expert by expert) -> expert-major grouping:
+        offsets [E_loc + 1], sorted_token (received row of each grouped position), sorted_gate,
+        slot_of (grouped position of each received row)."""
+        R = shape_loc.T
+        ids = self.moe.segment_ids(recv_counts, shape_loc.n_experts, R, ws)
+        return self.moe.permute(shape_loc, ids.reshape(R, 1), gates.reshape(R, 1), ws)
+
+    def expert_ffn(self, shape, x, offsets, sorted_token, gates, routed, ws):
+        return self.moe.expert_ffn(shape, x, offsets, sorted_token, gates, routed, ws)
 
     def combine(self, shape, x, shared, y, slot_of, ws):
         return self.moe.combine(shape, x, shared, y, slot_of, ws)
@@ -118,7 +137,10 @@ class ExpertParallelMoE:
         else:
             dist.all_to_all_single(out, inp, out_splits, in_splits, group=self.group)
 
-    def forward(self, x: torch.Tensor) -> torch.Tensor:
+    def forward(self, x: torch.Tensor, keep: Optional[Dict] = None) -> torch.Tensor:
+        """keep: if a dict, receives this rank's picks and gates ("idx", "gate"), its grouping
+        ("slot_of") and the gated routed rows returned to it ("y", [T * top_k, d] in its grouped
+        order, so row slot_of[t * top_k + j] belongs to token t's j-th pick)."""
         be, N, E, Eloc = self.be, self.n_ranks, self.E, self.E_loc
         T, d = x.shape
         I = self.routed["w1"].shape[1]
@@ -142,25 +164,23 @@ class ExpertParallelMoE:
         g_recv = torch.empty((R, 1), dtype=g_send.dtype, device=x.device)
         self._a2a(x_recv, x_send, r_split, s_split)
         self._a2a(g_recv, g_send, r_split, s_split)
-        # local experts on their rows (grouped by expert), then back in received order
-        row_of, offs, inv = regroup_plan(rc)
-        row_of_t = torch.from_numpy(row_of).to(x.device)
-        inv_t = torch.from_numpy(inv).to(x.device)
-        offs_t = torch.from_numpy(offs).to(x.device)
         # FP8 routed experts (e4m3 codes with their scales, quant.quantize_stack) run on the local
         # expert call only; routing, exchange and combine do not touch the routed weights
         fp8 = {"routed_fmt": 1} if self.routed["w1"].dtype == torch.uint8 else {}
         shape_loc = be.shape(R, d, Eloc, I, 1, 0, 0, bias, x.dtype, 0, **fp8)
         if R > 0:
-            ws_loc = be.workspace(shape_loc, x.device)
-            x_loc = be.gather(x_recv, row_of_t, ws_loc)
-            g_loc = be.gather(g_recv, row_of_t, ws_loc).reshape(-1)
-            y_loc = be.expert_ffn(shape_loc, x_loc, offs_t, g_loc, self.routed, ws_loc)
-            y_back = be.gather(y_loc, inv_t, ws_loc)
+            # local experts on their rows, grouped by expert on the device, then back in received order
+            ws_loc = be.workspace(shape_loc, x.device, "local")
+            grp = be.regroup(shape_loc, recv_counts, g_recv, ws_loc)
+            y_loc = be.expert_ffn(shape_loc, x_recv, grp["offsets"], grp["sorted_token"], grp["sorted_gate"],
+                                  self.routed, ws_loc)
+            y_back = be.gather(y_loc, grp["slot_of"], ws_loc)
         else:
             y_back = torch.empty((0, d), dtype=x.dtype, device=x.device)
         y_src = torch.empty((T * self.top_k, d), dtype=x.dtype, device=x.device)
         self._a2a(y_src, y_back, s_split, r_split)
+        if keep is not None:
+            keep.update(idx=perm.get("idx"), gate=perm.get("gate"), slot_of=perm["slot_of"], y=y_src)
         return be.combine(shape, x, self.shared, y_src, perm["slot_of"], ws)
 
     __call__ = forward

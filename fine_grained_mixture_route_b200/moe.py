@@ -24,7 +24,7 @@ EXPORTED = ("moe_workspace_bytes", "moe_layer_launches", "moe_status_string", "m
             "moe_layer_forward_timed", "moe_permute_no_alloc", "moe_quantize_rows_e4m3", "moe_train_ctx_bytes",
             "moe_backward_workspace_bytes", "moe_layer_forward_train", "moe_layer_backward",
             "moe_layer_backward_timed", "moe_backward_launches", "moe_balance_workspace_bytes",
-            "moe_balance_stats", "moe_gather_rows")
+            "moe_balance_stats", "moe_gather_rows", "moe_segment_ids", "moe_selftest_wait_timeout")
 NUM_STAGES = 7
 STAGE_NAMES = ("router", "permute", "plan", "gather", "gemm1_swiglu", "gemm2", "combine")
 BWD_STAGES = 7
@@ -97,12 +97,14 @@ def _lib():
         lib.moe_balance_workspace_bytes.restype = sz
         lib.moe_balance_stats.argtypes = [sh, vp, vp, f32p, i32p, ctypes.c_int32, f32p, f32p, f32p, vp, sz, vp]
         lib.moe_gather_rows.argtypes = [vp, i32p, ctypes.c_int64, ctypes.c_int64, ctypes.c_int32, vp, vp, sz, vp]
+        lib.moe_segment_ids.argtypes = [i32p, ctypes.c_int32, ctypes.c_int32, ctypes.c_int64, i32p, vp, sz, vp]
+        lib.moe_selftest_wait_timeout.argtypes = [ctypes.c_uint64, vp, vp, sz, vp]
         lib.moe_backward_launches.argtypes = [sh]
         lib.moe_backward_launches.restype = ctypes.c_int32
         for n in ("moe_check_device_error", "moe_ws_init", "moe_route", "moe_permute", "moe_expert_ffn",
                   "moe_combine", "moe_layer_forward", "moe_layer_forward_timed", "moe_quantize_rows_e4m3",
                   "moe_layer_forward_train", "moe_layer_backward", "moe_layer_backward_timed", "moe_balance_stats",
-                  "moe_gather_rows"):
+                  "moe_gather_rows", "moe_segment_ids", "moe_selftest_wait_timeout"):
             getattr(lib, n).restype = ctypes.c_int
         _LIB = lib
     return _LIB
@@ -475,6 +477,27 @@ def gather_rows(src: torch.Tensor, row_of: torch.Tensor, ws: torch.Tensor, out=N
     row_bytes = src[0].numel() * src.element_size() if src.shape[0] else src.element_size()
     _check(_lib().moe_gather_rows(_ptr(src), _ptr(row_of), n, src.shape[0], row_bytes, _ptr(out), _ptr(ws), ws.numel(),
                                   _stream(stream)), "moe_gather_rows")
+    return out
+
+
+def segment_ids(counts: torch.Tensor, modulo: int, n_rows: int, ws: torch.Tensor, out=None, stream=None):
+    """ids[r] = (segment holding row r) % modulo for segments of counts[q] consecutive rows
+    (moe_segment_ids); int32 [n_rows]."""
+    if counts.dtype != torch.int32 or counts.dim() != 1 or not counts.is_contiguous():
+        raise ValueError("counts must be a contiguous int32 vector")
+    out = torch.empty(n_rows, dtype=torch.int32, device=counts.device) if out is None else out
+    _need(out, "ids", n_rows, torch.int32, counts.device)
+    _check(_lib().moe_segment_ids(_ptr(counts), counts.numel(), modulo, n_rows, _ptr(out), _ptr(ws), ws.numel(),
+                                  _stream(stream)), "moe_segment_ids")
+    return out
+
+
+def selftest_wait_timeout(limit_ns: int, ws: torch.Tensor, out: Optional[torch.Tensor] = None, stream=None):
+    """moe_selftest_wait_timeout: runs the bounded-wait give-up path once (error bit 2 in ws);
+    out (int64 [2], optional) receives 1 if the wait gave up and the nanoseconds it waited."""
+    _need(out, "out", 2, torch.int64, ws.device)
+    _check(_lib().moe_selftest_wait_timeout(limit_ns, _ptr(out), _ptr(ws), ws.numel(), _stream(stream)),
+           "moe_selftest_wait_timeout")
     return out
 
 

@@ -368,6 +368,34 @@ moe_status_t moe_gather_rows(const void* src, const int32_t* row_of, int64_t n_r
                              int32_t row_bytes, void* dst, void* ws, size_t ws_bytes, moe_stream_t stream);
 
 /*
+ * Self-test of the bounded waits (no counterpart on the pages: a check of this library's hang
+ * safety).  Every wait of the tensor-core pipelines is bounded; when one gives up, the kernel
+ * sets error bit 2 in ws, stops issuing work, frees its tensor memory and returns, so the
+ * context stays usable and moe_check_device_error() reports MOE_ERR_INTERNAL.  This call runs
+ * that path on purpose: one warp allocates tensor memory, waits through the same bounded wait
+ * on an mbarrier that nothing completes, gives up after limit_ns nanoseconds (1 us .. 10 s),
+ * frees the memory and returns.  out (device, 8-byte aligned, may be NULL) receives 2 uint64:
+ * 1 if the wait gave up (0 if it completed), and the nanoseconds it waited.  Asynchronous on
+ * stream; ws >= 256 bytes (its error word).
+ */
+moe_status_t moe_selftest_wait_timeout(uint64_t limit_ns, uint64_t* out, void* ws, size_t ws_bytes,
+                                       moe_stream_t stream);
+
+/*
+ * Segment ids: ids[r] = q mod modulo, where segment q holds row r and the segments are
+ * consecutive runs of counts[q] rows (q < n_segments <= 4096), for r < n_rows.  The expert-
+ * parallel layer (the all_to_all scheme of the DeepSeek-V2 explainer, eliteato.com/news/32734,
+ * §3.3) receives its rows source by source and, inside a source, expert by expert; with
+ * counts = the [sources x local experts] received counts and modulo = the local expert count,
+ * ids is each received row's local expert, which moe_permute (T = n_rows, top_k = 1) then
+ * turns into the expert-major regrouping on the device.  A negative count is taken as 0 and a
+ * row past the last segment gets -1; both set error bit 4 in ws (>= 256 bytes).
+ * MOE_ERR_UNSUPPORTED for more than 4096 segments.
+ */
+moe_status_t moe_segment_ids(const int32_t* counts, int32_t n_segments, int32_t modulo, int64_t n_rows,
+                             int32_t* ids, void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
  * moe_permute_no_alloc — the paper has no counterpart to this entry point; it exists for
  * callers of this library that cannot allocate device memory.  moe_permute needs scratch
  * space, which it takes from the caller's workspace.  A caller that cannot call cudaMalloc

@@ -224,3 +224,23 @@ def test_balance_stats_validate(lib):
     assert q(S(sh), fake, fake, None, fake, 4, fake, fake, fake, fake, n - 1, None) == moe.MOE_ERR_WORKSPACE
     assert q(S(_shape(dtype=moe.MOE_F32)), fake, fake, None, fake, 4, fake, fake, fake, fake, n, None) == \
         moe.MOE_ERR_UNSUPPORTED
+
+
+def test_segment_ids_and_wait_selftest_argument_errors(lib):
+    """The expert-parallel segment-id call and the bounded-wait self-test reject bad arguments
+    before any launch."""
+    fake = ctypes.c_void_p(1 << 40)
+    ws = ctypes.c_void_p(1 << 41)
+    assert lib.moe_segment_ids(fake, 0, 4, 10, fake, ws, 256, None) == moe.MOE_ERR_INVALID_ARG      # no segments
+    assert lib.moe_segment_ids(fake, 8, 0, 10, fake, ws, 256, None) == moe.MOE_ERR_INVALID_ARG      # modulo 0
+    assert lib.moe_segment_ids(fake, 8, 4, -1, fake, ws, 256, None) == moe.MOE_ERR_INVALID_ARG      # negative rows
+    assert lib.moe_segment_ids(fake, 4097, 4, 10, fake, ws, 256, None) == moe.MOE_ERR_UNSUPPORTED   # > 4096 segments
+    assert lib.moe_segment_ids(fake, 8, 4, 10, fake, None, 256, None) == moe.MOE_ERR_WORKSPACE
+    assert lib.moe_segment_ids(fake, 8, 4, 10, fake, ws, 255, None) == moe.MOE_ERR_WORKSPACE
+    assert lib.moe_segment_ids(fake, 8, 4, 0, None, ws, 256, None) == moe.MOE_OK                  # nothing to do
+    assert lib.moe_segment_ids(None, 8, 4, 10, fake, ws, 256, None) == moe.MOE_ERR_INVALID_ARG
+    assert lib.moe_selftest_wait_timeout(999, None, ws, 256, None) == moe.MOE_ERR_INVALID_ARG        # < 1 us
+    assert lib.moe_selftest_wait_timeout(10**10 + 1, None, ws, 256, None) == moe.MOE_ERR_INVALID_ARG  # > 10 s
+    assert lib.moe_selftest_wait_timeout(10**6, None, None, 256, None) == moe.MOE_ERR_WORKSPACE
+    assert lib.moe_selftest_wait_timeout(10**6, ctypes.c_void_p((1 << 40) + 4), ws, 256, None) == \
+        moe.MOE_ERR_INVALID_ARG                                                                       # misaligned out

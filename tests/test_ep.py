@@ -39,7 +39,7 @@ class OracleBackend:
     def shape(self, T, d, E, I, k, Ks, Is, bias, dtype, gate_mode):
         return types.SimpleNamespace(T=T, d=d, E=E, I=I, k=k, Ks=Ks, Is=Is, gate_mode=gate_mode)
 
-    def workspace(self, shape, device):
+    def workspace(self, shape, device, use="layer"):
         return None
 
     def route_permute(self, shape, x, centroids, ws, router_bias):
@@ -53,13 +53,20 @@ class OracleBackend:
     def gather(self, src, row_of, ws):
         return src[row_of.long()].clone()
 
-    def expert_ffn(self, shape, x, offsets, gates, routed, ws):
-        y = torch.zeros_like(x)
+    def regroup(self, shape_loc, recv_counts, gates, ws):
+        row_of, offs, inv = ep.regroup_plan(recv_counts.numpy().reshape(-1, shape_loc.E))
+        t = lambda a: torch.from_numpy(np.ascontiguousarray(a))  # noqa: E731
+        return {"offsets": t(offs), "sorted_token": t(row_of), "sorted_gate": gates.reshape(-1)[row_of.astype(np.int64)],
+                "slot_of": t(inv)}
+
+    def expert_ffn(self, shape, x, offsets, sorted_token, gates, routed, ws):
+        y = torch.zeros((len(sorted_token), x.shape[1]), dtype=x.dtype)
         for e in range(shape.E):
             lo, hi = int(offsets[e]), int(offsets[e + 1])
             if hi > lo:
                 w = {k: (None if v is None else v[e].numpy()) for k, v in routed.items()}
-                ye = self.O.expert_ffn(x[lo:hi].numpy(), w["w1"], w["b1"], w["w3"], w["b3"], w["w2"], w["b2"])
+                xe = x[sorted_token[lo:hi].long()].numpy()
+                ye = self.O.expert_ffn(xe, w["w1"], w["b1"], w["w3"], w["b3"], w["w2"], w["b2"])
                 y[lo:hi] = torch.from_numpy(ye) * gates[lo:hi].reshape(-1, 1).to(x.dtype)
         return y
 
