@@ -7,6 +7,10 @@ dequantized weights q * scale, which are exactly representable, so the fp64 orac
 them directly.  Keeping the shared experts in bf16 follows the quantisation advice of the
 DeepSeek-V2 explainer (eliteato.com/news/32734, §5.5): the always-on experts are the most
 sensitive to quantisation error.
+
+The conversion runs once, offline, in the library's per-row quantiser (moe_quantize_rows_e4m3,
+the same kernel the FP8 layer uses for its activation rows): bf16 weights on the GPU in, codes
+and scales out.  There is no other implementation of the format's arithmetic here.
 """
 from __future__ import annotations
 
@@ -14,38 +18,45 @@ from typing import Dict, Optional, Tuple
 
 import torch
 
+from fine_grained_mixture_route_b200 import moe
+
 E4M3_MAX = 448.0
 
 
-def quantize_rows(w: torch.Tensor) -> Tuple[torch.Tensor, torch.Tensor]:
-    """w [..., out, in] (any float dtype) -> (codes [..., out, in] uint8, scales [..., out] fp32)."""
-    wf = w.float()
-    amax = wf.abs().amax(dim=-1)
-    scale = torch.where(amax > 0, amax / E4M3_MAX, torch.ones_like(amax))
-    q = (wf / scale.unsqueeze(-1)).to(torch.float8_e4m3fn)
-    return q.view(torch.uint8), scale.contiguous()
+def quantize_rows(w: torch.Tensor, ws: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """w [..., out, in] bf16 on a CUDA device -> (codes [..., out, in] uint8, scales [..., out] fp32),
+    by moe_quantize_rows_e4m3 (in must be a multiple of 8)."""
+    if w.dtype != torch.bfloat16 or w.device.type != "cuda":
+        raise ValueError("quantize_rows converts bf16 weights on a CUDA device (the library's e4m3 quantiser)")
+    flat = w.reshape(-1, w.shape[-1]).contiguous()
+    ws = torch.zeros(256, dtype=torch.uint8, device=w.device) if ws is None else ws
+    codes, scales = moe.quantize_rows_e4m3(flat, ws)
+    moe.check_device_error(ws)
+    return codes.reshape(w.shape), scales.reshape(w.shape[:-1])
 
 
 def dequantize_rows(q: torch.Tensor, scale: torch.Tensor) -> torch.Tensor:
-    """codes uint8 + scales -> fp32 weights q * scale."""
+    """codes uint8 + scales -> fp32 weights q * scale (for inspection; the layer never expands them)."""
     return q.view(torch.float8_e4m3fn).float() * scale.unsqueeze(-1)
 
 
 def quantize_stack(stack: Dict[str, Optional[torch.Tensor]]) -> Dict[str, Optional[torch.Tensor]]:
-    """Routed expert stack (w1, w3 [E, I, d]; w2 [E, d, I]; biases unchanged) -> codes in
-    w1/w3/w2 (uint8; w1 and w3 the two halves of one [2, E, I, d] buffer) and per-row scales in
-    s1, s3 [E, I] and s2 [E, d]."""
+    """Routed expert stack (bf16 on the GPU: w1, w3 [E, I, d]; w2 [E, d, I]; biases unchanged) ->
+    codes in w1/w3/w2 (uint8; w1 and w3 the two halves of one [2, E, I, d] buffer) and per-row
+    scales in s1, s3 [E, I] and s2 [E, d]."""
     out = dict(stack)
+    ws = torch.zeros(256, dtype=torch.uint8, device=stack["w1"].device)
     codes13 = None
     for w, sname in (("w1", "s1"), ("w3", "s3"), ("w2", "s2")):
-        q, sc = quantize_rows(stack[w])
+        q, sc = quantize_rows(stack[w], ws)
         if w in ("w1", "w3"):                 # W1 and W3 codes as the two halves of one buffer
             if codes13 is None:
                 codes13 = torch.empty((2,) + tuple(q.shape), dtype=q.dtype, device=q.device)
             codes13[0 if w == "w1" else 1].copy_(q)
             out[w] = codes13[0 if w == "w1" else 1]
+            del q
         else:
-            out[w] = q.contiguous()
+            out[w] = q
         out[sname] = sc
     return out
 

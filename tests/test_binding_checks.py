@@ -4,7 +4,7 @@ refuses such calls before any library or CUDA call, and refuses tensors off the 
 import pytest
 import torch
 
-from fine_grained_mixture_route_b200 import moe, quant
+from fine_grained_mixture_route_b200 import moe
 from fine_grained_mixture_route_b200 import workloads as W
 
 
@@ -44,7 +44,12 @@ def test_weights_of_another_element_type():
 
 def test_fp8_codes_need_the_fp8_shape_and_fp32_scales():
     _, L, shape, ws = _layer()
-    q = quant.quantize_stack(L["routed"])
+    # a stack in the e4m3 layout (codes and fp32 scales); the binding checks types and sizes only
+    q = dict(L["routed"], w1=torch.zeros(L["routed"]["w1"].shape, dtype=torch.uint8),
+             w3=torch.zeros(L["routed"]["w3"].shape, dtype=torch.uint8),
+             w2=torch.zeros(L["routed"]["w2"].shape, dtype=torch.uint8),
+             s1=torch.ones(L["routed"]["w1"].shape[:2]), s3=torch.ones(L["routed"]["w3"].shape[:2]),
+             s2=torch.ones(L["routed"]["w2"].shape[:2]))
     with pytest.raises(ValueError, match=r"routed\.w1 has dtype torch.uint8"):
         _fwd(shape, L, ws, routed=q)                         # native-format shape, e4m3 codes
     s8 = moe.shape_of(L["x"], L["centroids"], q, 2, L["shared"])
