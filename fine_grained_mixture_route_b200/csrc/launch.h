@@ -48,6 +48,11 @@ cudaError_t launch_plan(const Dims& D, const int32_t* offsets, int32_t* tile_sta
 cudaError_t launch_gather(const Dims& D, const void* x, const int32_t* sorted_token, void* x_perm,
                           uint32_t* err, cudaStream_t stream);
 
+// The same rows written in token order: x_perm[slot_of[t*k + j], :] = x[t, :] (each row of x
+// read once); dropped slots (slot_of -1) are skipped.
+cudaError_t launch_scatter_rows(const Dims& D, const void* x, const int32_t* slot_of, void* x_perm, uint32_t* err,
+                                cudaStream_t stream);
+
 // Per-row e4m3 quantisation of bf16 rows: for each output row p, src row r = row_of[p] (or p
 // when row_of is NULL, r checked against src_rows), scale[p] = max|src[r]| / 448 (1 for a zero
 // row), dst[p, :] = e4m3 round-to-nearest-even (saturating) of src[r, :] / scale[p], the
@@ -62,6 +67,11 @@ cudaError_t launch_gather_rows_generic(const void* src, const int32_t* row_of, l
 // out (optional, 2 x u64): 1 if the wait gave up, and the ns waited
 cudaError_t launch_wait_selftest(unsigned long long limit_ns, uint32_t* err, unsigned long long* out,
                                  cudaStream_t stream);
+// dst[slot_of[t*k + j], :] = src[t, :] and dscale[...] = sscale[t] for the picks of each of T
+// rows (each source row read once); dropped slots (-1) skipped, positions >= S flagged (bit 4)
+cudaError_t launch_scatter_code_rows(const uint8_t* src, const float* sscale, const int32_t* slot_of, int T, int k,
+                                     long long S, int row_bytes, uint8_t* dst, float* dscale, uint32_t* err,
+                                     cudaStream_t stream);
 // ids[r] = (segment holding row r) % modulo for segments of counts[q] consecutive rows
 // (n_seg <= SEGMENT_MAX); rows past the last segment get -1 and bit 4, as do negative counts
 constexpr int SEGMENT_MAX = 4096;

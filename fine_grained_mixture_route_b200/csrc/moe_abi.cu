@@ -202,13 +202,19 @@ FfnWeights to_ffn(const moe_ffn_weights_t* w) {
 
 // e4m3 routed experts: x quantised once per token, then its code rows (and scales) gathered
 // into expert order for the GEMM1 A operand.
+// With the slot map at hand (the fused forward) the code rows are written in token order
+// instead: each token's codes are read once and stored at its k slot positions.
 moe_status_t quant_gather_x(const Dims& D, const Layout& L, void* ws, const void* x, const int32_t* stok,
-                            uint32_t* err, cudaStream_t st) {
+                            uint32_t* err, cudaStream_t st, const int32_t* slot_of = nullptr) {
     uint8_t* x8t = at<uint8_t>(ws, L.x8t);
     float* xst = at<float>(ws, L.xst);
     MOE_CUDA(launch_quant_rows(x, nullptr, D.T, D.T, D.d, x8t, xst, err, st));
-    MOE_CUDA(launch_gather_code_rows(x8t, xst, stok, D.slots(), D.T, D.d, at<uint8_t>(ws, L.xperm), at<float>(ws, L.xs),
-                                     err, st));
+    if (slot_of)
+        MOE_CUDA(launch_scatter_code_rows(x8t, xst, slot_of, D.T, D.k, D.slots(), D.d, at<uint8_t>(ws, L.xperm),
+                                          at<float>(ws, L.xs), err, st));
+    else
+        MOE_CUDA(launch_gather_code_rows(x8t, xst, stok, D.slots(), D.T, D.d, at<uint8_t>(ws, L.xperm),
+                                         at<float>(ws, L.xs), err, st));
     return MOE_OK;
 }
 
@@ -481,7 +487,7 @@ moe_status_t layer_forward_impl(const moe_shape_t* shape, const void* x, const v
     if (D.q8) {
         uint8_t* x8 = at<uint8_t>(ws, L.xperm);
         float* xs = at<float>(ws, L.xs);
-        MOE_TRY(quant_gather_x(D, L, ws, x, stok, err, st));
+        MOE_TRY(quant_gather_x(D, L, ws, x, stok, err, st, slot_of));
         if (!mark(4)) return MOE_ERR_CUDA;
         MOE_CUDA(launch_tc_gemm1_q8(D, x, x8, xs, offsets, ts1, R, Sh, hr, hs, D.E + D.Ks, err, st));
         if (!mark(5)) return MOE_ERR_CUDA;
@@ -495,7 +501,7 @@ moe_status_t layer_forward_impl(const moe_shape_t* shape, const void* x, const v
         MOE_CUDA(launch_combine(D, y, slot_of, sout, out, err, st));
     } else if (D.bf16) {
         void* xp = at<void>(ws, L.xperm);
-        MOE_CUDA(launch_gather(D, x, stok, xp, err, st));
+        MOE_CUDA(launch_scatter_rows(D, x, slot_of, xp, err, st));     // token order: each row of x read once
         if (!mark(4)) return MOE_ERR_CUDA;
         MOE_CUDA(launch_tc_gemm1(D, x, xp, offsets, ts1, R, Sh, hr, hs, 0, D.E + D.Ks, err, st, ctx ? &save : nullptr));
         if (!mark(5)) return MOE_ERR_CUDA;

@@ -213,6 +213,35 @@ __global__ void gather_rows_kernel(const uint4* __restrict__ x, const int32_t* _
     }
 }
 
+// x_perm[slot_of[t*k + j]] = x[t] for every pick j of token t: the same rows as
+// gather_rows_kernel, written in token order, so each row of x is read from HBM once and
+// stored k times (a gather re-reads each token's row k times from scattered places, mostly
+// from HBM, since the sorted order visits a token once per expert it picked).  One block per
+// token: the k destinations go to shared memory, then each thread moves 16-byte vectors.  A
+// position outside [0, S) sets bit 4 and is skipped; a dropped slot (-1) is skipped.
+__global__ void __launch_bounds__(128) scatter_rows_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ slot_of,
+                                                           uint4* __restrict__ xp, int T, int k, long long S,
+                                                           int vec_per_row, uint32_t* err) {
+    __shared__ int dst[32];
+    for (int t = blockIdx.x; t < T; t += gridDim.x) {
+        __syncthreads();
+        if ((int)threadIdx.x < k) {
+            int p = slot_of[(size_t)t * k + threadIdx.x];
+            if (p >= S) { flag_error(err, ERR_INDEX_RANGE); p = -1; }
+            dst[threadIdx.x] = p;
+        }
+        __syncthreads();
+        const uint4* src = x + (size_t)t * vec_per_row;
+        for (int v = threadIdx.x; v < vec_per_row; v += blockDim.x) {
+            const uint4 val = __ldg(src + v);
+            for (int j = 0; j < k; ++j) {
+                const int p = dst[j];
+                if (p >= 0) xp[(size_t)p * vec_per_row + v] = val;
+            }
+        }
+    }
+}
+
 // out[t] = base[t] + sum_j y[slot_of[t*k + j]]: the shared experts' fp32 output (optional)
 // first, then the routed rows in ascending pick order, summed in fp32 and rounded once.  One
 // block per token: its slot rows are read as whole contiguous rows, V elements (16 bytes)
@@ -314,6 +343,17 @@ cudaError_t launch_gather(const Dims& D, const void* x, const int32_t* sorted_to
     const int vec = D.d * esz / 16;
     const long long blocks = S < 148LL * 32 ? S : 148LL * 32;
     gather_rows_kernel<<<(int)blocks, 128, 0, stream>>>((const uint4*)x, sorted_token, (uint4*)x_perm, S, D.T, vec, err);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_scatter_rows(const Dims& D, const void* x, const int32_t* slot_of, void* x_perm, uint32_t* err,
+                                cudaStream_t stream) {
+    if (D.T == 0) return cudaSuccess;
+    const int esz = D.bf16 ? 2 : 4;
+    const int vec = D.d * esz / 16;
+    const int blocks = D.T < 148 * 16 ? D.T : 148 * 16;
+    scatter_rows_kernel<<<blocks, 128, 0, stream>>>((const uint4*)x, slot_of, (uint4*)x_perm, D.T, D.k, D.slots(), vec,
+                                                    err);
     return cudaGetLastError();
 }
 

@@ -150,6 +150,31 @@ __global__ void gather_code_rows_kernel(const uint4* __restrict__ src, const flo
     }
 }
 
+// Token-order form of the same move: dst[slot_of[t*k + j]] = src[t] (and its scale) for every
+// pick j of row t, so each source row is read once and stored k times.  A position outside
+// [0, S) sets bit 4 and is skipped; a dropped slot (-1) is skipped.
+__global__ void scatter_code_rows_kernel(const uint4* __restrict__ src, const float* __restrict__ sscale,
+                                         const int32_t* __restrict__ slot_of, int T, int k, long long S, int nv,
+                                         uint4* __restrict__ dst, float* __restrict__ dscale, uint32_t* err) {
+    __shared__ int pos[32];
+    for (int t = blockIdx.x; t < T; t += gridDim.x) {
+        __syncthreads();
+        if ((int)threadIdx.x < k) {
+            int q = slot_of[(size_t)t * k + threadIdx.x];
+            if (q >= S) { flag_error(err, ERR_INDEX_RANGE); q = -1; }
+            pos[threadIdx.x] = q;
+            if (q >= 0) dscale[q] = sscale[t];
+        }
+        __syncthreads();
+        const uint4* s = src + (size_t)t * nv;
+        for (int i = threadIdx.x; i < nv; i += blockDim.x) {
+            const uint4 v = __ldg(s + i);
+            for (int j = 0; j < k; ++j)
+                if (pos[j] >= 0) dst[(size_t)pos[j] * nv + i] = v;
+        }
+    }
+}
+
 // dst[p] = src[row_of[p]] for rows of nw 4-byte words (16-byte vectors when nw % 4 == 0); an
 // index outside [0, src_rows) sets bit 4 and gives a zero row.
 template <bool V16>
@@ -269,6 +294,17 @@ cudaError_t launch_gather_code_rows(const uint8_t* src, const float* sscale, con
     const int blocks = (int)(n_rows < cap ? n_rows : cap);
     gather_code_rows_kernel<<<blocks, 128, 0, stream>>>((const uint4*)src, sscale, row_of, n_rows, src_rows,
                                                         row_bytes / 16, (uint4*)dst, dscale, err);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_scatter_code_rows(const uint8_t* src, const float* sscale, const int32_t* slot_of, int T, int k,
+                                     long long S, int row_bytes, uint8_t* dst, float* dscale, uint32_t* err,
+                                     cudaStream_t stream) {
+    if (T <= 0) return cudaSuccess;
+    if (row_bytes <= 0 || row_bytes % 16 || k > 32) return cudaErrorInvalidValue;
+    const int blocks = T < num_sms() * 16 ? T : num_sms() * 16;
+    scatter_code_rows_kernel<<<blocks, 128, 0, stream>>>((const uint4*)src, sscale, slot_of, T, k, S, row_bytes / 16,
+                                                         (uint4*)dst, dscale, err);
     return cudaGetLastError();
 }
 
