@@ -105,7 +105,8 @@ def stage_work(cfg: W.LayerConfig, touched: int, e4m3: bool = False):
             "router": (2.0 * T * d * E, (T * d + E * d) * b + S * 8),
             "permute": (0.0, S * 8 + S * 16),
             "plan": (0.0, (E + 1) * 4),
-            "gather": (0.0, S * d * b + S * d + S * 8),
+            # x read once (quantised per token), the code rows and scales stored at their slots
+            "gather": (0.0, T * d * b + S * d + S * 4 + S * 4),
             "gemm1_swiglu": (2.0 * S * d * 2 * I + 2.0 * Ks * T * d * 2 * Is,
                              touched * (2 * I * d + 2 * I * 4 + 2 * I * bias * b) + S * d + S * 4
                              + Ks * (2 * Is * d + 2 * Is * bias) * b + (T * d * b if Ks else 0)
@@ -120,7 +121,7 @@ def stage_work(cfg: W.LayerConfig, touched: int, e4m3: bool = False):
         "router": (2.0 * T * d * E, (T * d + E * d) * b + S * 8),
         "permute": (0.0, S * 8 + S * 16),
         "plan": (0.0, (E + 1) * 4),
-        "gather": (0.0, 2 * S * d * b + S * 4),
+        "gather": (0.0, T * d * b + S * d * b + S * 4),        # x read once, written at the k slots of each token
         "gemm1_swiglu": (2.0 * S * d * 2 * I + 2.0 * Ks * T * d * 2 * Is,
                          touched * (2 * I * d + 2 * I * bias) * b + Ks * (2 * Is * d + 2 * Is * bias) * b
                          + S * d * b + (T * d * b if Ks else 0) + (S * I + Ks * T * Is) * b),

@@ -261,7 +261,7 @@ __global__ void __launch_bounds__(128) combine_kernel(const T* __restrict__ y, c
             sl[threadIdx.x] = p;
         }
         __syncthreads();
-        for (int v = threadIdx.x; v < nv; v += blockDim.x) {
+        for (int v = blockIdx.y * blockDim.x + threadIdx.x; v < nv; v += blockDim.x * gridDim.y) {
             float acc[V];
             if (base && V % 4 == 0) {            // 16-byte loads (d % V == 0, base 16-byte aligned)
                 const float4* b4 = reinterpret_cast<const float4*>(base + (size_t)t * d + (size_t)v * V);
@@ -357,25 +357,43 @@ cudaError_t launch_scatter_rows(const Dims& D, const void* x, const int32_t* slo
     return cudaGetLastError();
 }
 
+// The grid is the number of blocks that fit on the GPU at once (one wave; each block loops over
+// tokens), so no partial last wave leaves most SMs idle while a few finish their tokens.  With few
+// tokens (decode) the grid's y dimension also splits each row's columns, so that every thread's
+// loads are in flight at once instead of one column step after another.
+template <typename K>
+int resident_blocks(K kern, int threads) {
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, 0) != cudaSuccess || per_sm < 1)
+        per_sm = 1;
+    return per_sm * num_sms();
+}
+
 template <typename T, int V>
 void combine_dispatch(const Dims& D, const void* y, const int32_t* slot_of, const float* base, void* out, uint32_t* err,
-                      int blocks, cudaStream_t stream) {
-    if (D.k <= 8)
-        combine_kernel<T, V, 8><<<blocks, 128, 0, stream>>>((const T*)y, slot_of, base, (T*)out, D.T, D.d, D.k,
-                                                            D.slots(), err);
-    else
-        combine_kernel<T, V, 0><<<blocks, 128, 0, stream>>>((const T*)y, slot_of, base, (T*)out, D.T, D.d, D.k,
-                                                            D.slots(), err);
+                      cudaStream_t stream) {
+    const int nv = D.d / V;
+    const int chunks = (nv + 127) / 128;
+    if (D.k <= 8) {
+        static const int cap = resident_blocks(combine_kernel<T, V, 8>, 128);
+        const dim3 grid(D.T < cap ? D.T : cap, (long long)D.T * chunks <= 2LL * cap ? chunks : 1);
+        combine_kernel<T, V, 8><<<grid, 128, 0, stream>>>((const T*)y, slot_of, base, (T*)out, D.T, D.d, D.k,
+                                                          D.slots(), err);
+    } else {
+        static const int cap = resident_blocks(combine_kernel<T, V, 0>, 128);
+        const dim3 grid(D.T < cap ? D.T : cap, (long long)D.T * chunks <= 2LL * cap ? chunks : 1);
+        combine_kernel<T, V, 0><<<grid, 128, 0, stream>>>((const T*)y, slot_of, base, (T*)out, D.T, D.d, D.k,
+                                                          D.slots(), err);
+    }
 }
 
 cudaError_t launch_combine(const Dims& D, const void* y_sorted, const int32_t* slot_of, const float* base, void* out,
                            uint32_t* err, cudaStream_t stream) {
     if (D.T == 0) return cudaSuccess;
-    const int blocks = D.T < 148 * 16 ? D.T : 148 * 16;
-    if (D.bf16 && D.d % 8 == 0) combine_dispatch<__nv_bfloat16, 8>(D, y_sorted, slot_of, base, out, err, blocks, stream);
-    else if (D.bf16) combine_dispatch<__nv_bfloat16, 1>(D, y_sorted, slot_of, base, out, err, blocks, stream);
-    else if (D.d % 4 == 0) combine_dispatch<float, 4>(D, y_sorted, slot_of, base, out, err, blocks, stream);
-    else combine_dispatch<float, 1>(D, y_sorted, slot_of, base, out, err, blocks, stream);
+    if (D.bf16 && D.d % 8 == 0) combine_dispatch<__nv_bfloat16, 8>(D, y_sorted, slot_of, base, out, err, stream);
+    else if (D.bf16) combine_dispatch<__nv_bfloat16, 1>(D, y_sorted, slot_of, base, out, err, stream);
+    else if (D.d % 4 == 0) combine_dispatch<float, 4>(D, y_sorted, slot_of, base, out, err, stream);
+    else combine_dispatch<float, 1>(D, y_sorted, slot_of, base, out, err, stream);
     return cudaGetLastError();
 }
 

@@ -66,6 +66,9 @@ CONFIGS: Dict[str, LayerConfig] = {
     "decode": LayerConfig("decode", 256, 7168, 256, 2048, 8, 1, 2048, True, torch.bfloat16, "normal_std"),
     # prefill-shaped layer, same experts, T=16384, Zipf(1.1)-skewed centroid norms
     "prefill": LayerConfig("prefill", 16384, 7168, 256, 2048, 8, 1, 2048, True, torch.bfloat16, "zipf_norm"),
+    # profiling slice of the prefill layer, a few GB on the device: the same expert shape and
+    # Zipf routing over 32 experts, T chosen so that the mean tokens per expert (512) match
+    "prefill_slice": LayerConfig("prefill_slice", 2048, 7168, 32, 2048, 8, 1, 2048, True, torch.bfloat16, "zipf_norm"),
 }
 
 # tensor ids used to derive per-tensor seeds
