@@ -28,6 +28,12 @@ cudaError_t launch_router_simt(const Dims& D, const void* x, const void* centroi
 // ---- per-expert token lists -----------------------------------------------------------
 constexpr int PERMUTE_CHUNK = 1024;  // slots per histogram / scatter block
 inline int permute_blocks(const Dims& D) { return (int)((D.slots() + PERMUTE_CHUNK - 1) / PERMUTE_CHUNK); }
+// Small groupings run the three passes in one block (one launch instead of three).
+constexpr long long PERMUTE_SMALL_SLOTS = 16384;
+constexpr int PERMUTE_SMALL_EXPERTS = 256;
+inline bool permute_small(const Dims& D) {
+    return D.slots() > 0 && D.slots() <= PERMUTE_SMALL_SLOTS && D.E <= PERMUTE_SMALL_EXPERTS;
+}
 
 cudaError_t launch_permute(const Dims& D, const int32_t* idx, const float* gate, int32_t* counts,
                            int32_t* offsets, int32_t* sorted_token, float* sorted_gate, int32_t* slot_of,

@@ -291,7 +291,7 @@ MOE_EXPORT int32_t moe_layer_launches(const moe_shape_t* shape) {
     int n = 0;
     if (tc_router_supported(D)) n += router_splits(D) > 1 ? 2 : 1;   // scores (+ split-K finish)
     else n += 1;
-    n += 3;                                                         // histogram, scan, scatter
+    n += permute_small(D) ? 1 : 3;                                  // histogram, scan, scatter (one block if small)
     n += 1;                                                         // tile tables
     if (D.bf16) n += 1;                                             // row gather (+ e4m3 quantisation)
     n += 3;                                   // GEMM1, GEMM2 (routed + shared tiles), combine

@@ -159,6 +159,75 @@ __global__ void __launch_bounds__(32) permute_scatter_kernel(const int32_t* __re
     }
 }
 
+// The three passes in one block for small groupings (PERMUTE_SMALL_SLOTS slots at most, at most
+// PERMUTE_SMALL_EXPERTS experts): its 32 warps play the part of the histogram / scatter blocks, warp w
+// taking the w-th consecutive slice of the slots, so the order inside an expert is again ascending
+// slot order and the result equals the multi-block passes' bit for bit.  Shared memory: a histogram
+// row per warp [32][E], then the expert totals [E] and 32 scan partials.
+__global__ void __launch_bounds__(1024) permute_small_kernel(const int32_t* __restrict__ idx,
+                                                             const float* __restrict__ gate, long long S, int k, int E,
+                                                             int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
+                                                             int32_t* __restrict__ sorted_token,
+                                                             float* __restrict__ sorted_gate,
+                                                             int32_t* __restrict__ slot_of, uint32_t* err) {
+    extern __shared__ int sh[];
+    int* hist = sh;                   // [32][E]: counts, then each warp's running position per expert
+    int* cnt = sh + 32 * E;           // [E]
+    int* wsum = cnt + E;              // [32]
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const long long chunk = (S + 31) / 32;
+    const long long s0 = warp * chunk, s1 = min(S, s0 + chunk);
+    for (int i = threadIdx.x; i < 32 * E; i += blockDim.x) hist[i] = 0;
+    __syncthreads();
+    for (long long s = s0 + lane; s < s1; s += 32) {
+        const int e = idx[s];
+        if (e >= 0 && e < E) atomicAdd(&hist[warp * E + e], 1);
+        else flag_error(err, ERR_EXPERT_RANGE);
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {         // warp-order bases inside each expert
+        int run = 0;
+        for (int w = 0; w < 32; ++w) {
+            const int c = hist[w * E + e];
+            hist[w * E + e] = run;
+            run += c;
+        }
+        cnt[e] = run;
+        counts[e] = run;
+    }
+    __syncthreads();
+    const int total = block_exclusive_scan(cnt, E, wsum);
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        offsets[e] = cnt[e];
+        for (int w = 0; w < 32; ++w) hist[w * E + e] += cnt[e];
+    }
+    if (threadIdx.x == 0) offsets[E] = total;
+    __syncthreads();
+    int* running = hist + warp * E;
+    const unsigned lt = (1u << lane) - 1u;
+    for (long long b = s0; b < s1; b += 32) {
+        const long long s = b + lane;
+        const bool live = s < s1;
+        int e = live ? idx[s] : -1;
+        const float g = live ? gate[s] : 0.f;
+        const bool ok = live && e >= 0 && e < E;
+        if (!ok) e = -1 - lane;                       // unique key: never matches a real expert
+        const unsigned peers = __match_any_sync(0xffffffffu, e);
+        int pos = 0;
+        if (ok) pos = running[e] + __popc(peers & lt);
+        __syncwarp();
+        if (ok && (peers & lt) == 0) running[e] += __popc(peers);   // group leader advances
+        __syncwarp();
+        if (ok) {
+            sorted_token[pos] = (int32_t)(s / k);
+            sorted_gate[pos] = g;
+            slot_of[s] = pos;
+        } else if (live) {
+            slot_of[s] = -1;
+        }
+    }
+}
+
 // tile tables of the grouped GEMMs (see launch.h)
 __global__ void plan_kernel(const int32_t* __restrict__ offsets, long long S, int T, int d, int E, int I, int Ks,
                             int Is, int tile_rows, int32_t* __restrict__ tile_start1, int32_t* __restrict__ tile_start2, uint32_t* err) {
@@ -312,6 +381,12 @@ cudaError_t launch_permute(const Dims& D, const int32_t* idx, const float* gate,
                            int32_t* sorted_token, float* sorted_gate, int32_t* slot_of, int32_t* block_hist,
                            uint32_t* err, cudaStream_t stream) {
     const long long S = D.slots();
+    if (permute_small(D)) {
+        const size_t smem = sizeof(int) * (33 * (size_t)D.E + 32);
+        permute_small_kernel<<<1, 1024, smem, stream>>>(idx, gate, S, D.k, D.E, counts, offsets, sorted_token,
+                                                        sorted_gate, slot_of, err);
+        return cudaGetLastError();
+    }
     const int nblk = permute_blocks(D);
     const size_t smemE = sizeof(int) * D.E;
     if (nblk > 0) {

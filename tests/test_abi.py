@@ -80,12 +80,15 @@ def test_workspace_bytes(lib):
 
 
 def test_launch_count(lib):
-    assert moe.layer_launches(_shape()) == 10          # split-K router at T=256: scores + finish
+    # T=256: split-K router (scores + finish); 2048 slots grouped by one block (one launch, not three)
+    assert moe.layer_launches(_shape()) == 8
     assert moe.layer_launches(_shape(T=16384)) == 9
     assert moe.layer_launches(_shape(T=16384, n_shared=0)) == 9
+    assert moe.layer_launches(_shape(T=2048)) == 8     # 16384 slots: still one grouping block (split-K router)
+    assert moe.layer_launches(_shape(T=2049)) == 10    # past 16384 slots: the three grouping passes
     assert moe.layer_launches(_shape(T=128, d=256, n_experts=16, inter=64, inter_shared=64, top_k=4,
-                                     dtype=moe.MOE_F32)) == 8
-    assert moe.layer_launches(_shape(routed_fmt=moe.FMT_E4M3)) == 12      # + x per token, hidden rows
+                                     dtype=moe.MOE_F32)) == 6
+    assert moe.layer_launches(_shape(routed_fmt=moe.FMT_E4M3)) == 10      # + x per token, hidden rows
     assert moe.layer_launches(_shape(T=0)) == 0
     assert moe.layer_launches(_shape(top_k=0)) == -1
 

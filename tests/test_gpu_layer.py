@@ -300,3 +300,44 @@ def test_shared_experts_ignore_the_router(base, kw):
     tol = TOL[cfg.dtype]
     e = record(f"shared_bypass_{base}", "shared_only", f64(shared_only[0]), ref["shared_sum"], tol)
     assert e <= tol, f"shared part vs oracle: {e:.3e}"
+
+
+@pytest.mark.parametrize("T,k,E", [(2048, 8, 256), (2049, 8, 256), (4096, 4, 257), (1, 1, 1), (300, 7, 64)],
+                         ids=["S16384_E256_one_block", "S16392_three_passes", "E257_three_passes", "S1", "S2100"])
+def test_grouping_paths_bit_exact(T, k, E):
+    """Groupings of at most 16384 slots over at most 256 experts run the histogram, scan and
+    scatter in one block; larger ones in three launches. Both must give the oracle's stable
+    grouping bit for bit, on either side of the boundary, including a few out-of-range experts
+    (dropped and flagged)."""
+    g = torch.Generator(device="cpu").manual_seed(T + E)
+    idx = torch.randint(0, E, (T, k), generator=g, dtype=torch.int32)
+    if T > 10:
+        idx[3, 0] = -1
+        idx[T - 1, k - 1] = E
+    gate = torch.rand((T, k), generator=g)
+    shape = moe.make_shape(T, 256, E, 64, k, 0, 0, False, torch.bfloat16)
+    ws = moe.new_workspace(shape)
+    perm = moe.permute(shape, idx.cuda(), gate.cuda(), ws)
+    if T > 10:
+        with pytest.raises(moe.MoeError):
+            moe.check_device_error(ws)
+    else:
+        moe.check_device_error(ws)
+    idx_np = idx.numpy().astype(np.int64)
+    ok = (idx_np >= 0) & (idx_np < E)
+    p = O.permute(np.where(ok, idx_np, 0), gate.numpy(), E)
+    got = {key: v.cpu().numpy() for key, v in perm.items()}
+    n = int(ok.sum())
+    counts = np.bincount(idx_np[ok], minlength=E)
+    assert np.array_equal(got["counts"], counts)
+    assert got["offsets"][E] == n and np.array_equal(got["offsets"], np.concatenate([[0], np.cumsum(counts)]))
+    # the valid slots in ascending slot order inside each expert, as the oracle orders them
+    slots = np.arange(T * k)[ok.reshape(-1)]
+    order = slots[np.argsort(idx_np.reshape(-1)[slots], kind="stable")]
+    assert np.array_equal(got["sorted_token"][:n], (order // k).astype(np.int32))
+    assert np.array_equal(got["sorted_gate"][:n], gate.numpy().reshape(-1)[order])
+    slot_of = got["slot_of"]
+    assert (slot_of[~ok.reshape(-1)] == -1).all()
+    assert np.array_equal(slot_of[order], np.arange(n, dtype=np.int32))
+    if ok.all():
+        assert np.array_equal(got["sorted_token"], p["sorted_token"]) and np.array_equal(got["slot_of"], p["slot_of"])
