@@ -73,6 +73,12 @@ cudaError_t launch_gather_rows_generic(const void* src, const int32_t* row_of, l
 // out (optional, 2 x u64): 1 if the wait gave up, and the ns waited
 cudaError_t launch_wait_selftest(unsigned long long limit_ns, uint32_t* err, unsigned long long* out,
                                  cudaStream_t stream);
+// The same move for any rows of row_bytes bytes (a multiple of 16, at most 32 KB, 16-byte aligned
+// buffers) by bulk copies through shared memory; with dscale, dscale[slot_of[t*k + j]] = sscale[t].
+// cudaErrorNotSupported when the rows or buffers do not qualify (nothing launched).
+cudaError_t launch_scatter_rows_bulk(const void* src, const float* sscale, const int32_t* slot_of, int T, int k,
+                                     long long S, uint32_t row_bytes, void* dst, float* dscale, uint32_t* err,
+                                     cudaStream_t stream);
 // dst[slot_of[t*k + j], :] = src[t, :] and dscale[...] = sscale[t] for the picks of each of T
 // rows (each source row read once); dropped slots (-1) skipped, positions >= S flagged (bit 4)
 cudaError_t launch_scatter_code_rows(const uint8_t* src, const float* sscale, const int32_t* slot_of, int T, int k,

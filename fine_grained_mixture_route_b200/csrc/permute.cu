@@ -54,6 +54,11 @@ __device__ int block_exclusive_scan(int* v, int n, int* warp_sums) {
     return total;
 }
 
+__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
+    const __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<const uint32_t*>(&v);
+}
+
 // pass 1: per-block histogram of expert picks
 __global__ void permute_hist_kernel(const int32_t* __restrict__ idx, long long S, int E,
                                     int32_t* __restrict__ block_hist, uint32_t* err) {
@@ -311,6 +316,96 @@ __global__ void __launch_bounds__(128) scatter_rows_kernel(const uint4* __restri
     }
 }
 
+// The same token-order row move by the copy engine: one warp per block, lane 0 bringing each
+// token's whole row into shared memory with one bulk copy (completion counted on an mbarrier)
+// and storing it to the token's k slot positions with k bulk copies, two rows in flight per
+// block (double buffer); lanes < k fetch the positions.  No data passes through registers.
+// Waits on the load barriers are bounded (error bit 2, the remaining copies drained).
+constexpr unsigned long long SCATTER_WAIT_NS = 1000000000ull;
+__device__ __forceinline__ unsigned long long scatter_clock() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+__device__ __forceinline__ bool scatter_wait(uint32_t bar, uint32_t parity) {
+    const unsigned long long t0 = scatter_clock();
+    for (uint32_t i = 0;; ++i) {
+        uint32_t done;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(done)
+            : "r"(bar), "r"(parity)
+            : "memory");
+        if (done) return true;
+        if ((i & 63u) == 63u && (scatter_clock() - t0 > SCATTER_WAIT_NS || i >= (1u << 28))) return false;
+    }
+}
+__global__ void __launch_bounds__(32) scatter_rows_bulk_kernel(const char* __restrict__ x,
+                                                               const int32_t* __restrict__ slot_of,
+                                                               char* __restrict__ xp, int T, int k, long long S,
+                                                               uint32_t row_bytes, const float* __restrict__ sscale,
+                                                               float* __restrict__ dscale, uint32_t* err) {
+    extern __shared__ __align__(128) uint8_t rows[];           // two row buffers
+    __shared__ __align__(8) uint64_t bars[2];
+    const int lane = threadIdx.x;
+    const uint32_t bar0 = (uint32_t)__cvta_generic_to_shared(&bars[0]);
+    const uint32_t buf0 = (uint32_t)__cvta_generic_to_shared(rows);
+    if (lane == 0) {
+        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar0) : "memory");
+        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar0 + 8) : "memory");
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncwarp();
+    const int n = (int)blockIdx.x < T ? (T - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+    auto load = [&](int i) {                                    // lane 0: token i of this block into buffer i & 1
+        const int t = (int)blockIdx.x + i * (int)gridDim.x;
+        const uint32_t b = bar0 + 8u * (i & 1), dst = buf0 + row_bytes * (i & 1);
+        asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(b), "r"(row_bytes) : "memory");
+        asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+                     "l"(x + (size_t)t * row_bytes), "r"(row_bytes), "r"(b)
+                     : "memory");
+    };
+    if (lane == 0 && n > 0) load(0);
+    bool ok = true;
+    int i = 0;
+    for (; i < n; ++i) {
+        const int t = (int)blockIdx.x + i * (int)gridDim.x;
+        int pos = -1;
+        if (lane < k) {
+            pos = slot_of[(size_t)t * k + lane];
+            if (pos >= S) { flag_error(err, ERR_INDEX_RANGE); pos = -1; }
+            if (dscale && pos >= 0) dscale[pos] = sscale[t];   // row scale with the row (e4m3 codes)
+        }
+        if (lane == 0) {
+            if (i + 1 < n) {
+                // buffer (i + 1) & 1 was last read by token i - 1's stores: they must be done reading
+                asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+                load(i + 1);
+            }
+            ok = scatter_wait(bar0 + 8u * (i & 1), (uint32_t)((i >> 1) & 1));
+            if (!ok) flag_error(err, ERR_PIPE_TIMEOUT);
+        }
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) break;
+        for (int j = 0; j < k; ++j) {
+            const int pj = __shfl_sync(0xffffffffu, pos, j);
+            if (lane == 0 && pj >= 0)
+                asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(xp + (size_t)pj * row_bytes),
+                             "r"(buf0 + row_bytes * (i & 1)), "r"(row_bytes)
+                             : "memory");
+        }
+        if (lane == 0) asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+    }
+    if (lane == 0) {
+        if (!ok) {                                   // drain the loads still in flight (token i, and i + 1)
+            scatter_wait(bar0 + 8u * (i & 1), (uint32_t)((i >> 1) & 1));
+            if (i + 1 < n) scatter_wait(bar0 + 8u * ((i + 1) & 1), (uint32_t)(((i + 1) >> 1) & 1));
+        }
+        asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+    }
+    __syncwarp();
+}
+
 // out[t] = base[t] + sum_j y[slot_of[t*k + j]]: the shared experts' fp32 output (optional)
 // first, then the routed rows in ascending pick order, summed in fp32 and rounded once.  One
 // block per token: its slot rows are read as whole contiguous rows, V elements (16 bytes)
@@ -375,6 +470,122 @@ __global__ void __launch_bounds__(128) combine_kernel(const T* __restrict__ y, c
     }
 }
 
+// The combine with its inputs staged by the copy engine: a persistent block walks (token, column
+// chunk) items; thread 0 brings a chunk's k routed-row segments (bf16) and the shared output's
+// segment (fp32) into one of two shared-memory stages with bulk copies counted on the stage's
+// mbarrier, the whole block sums the next item while the following one is in flight, and each
+// thread stores its 8 output columns.  The sum runs in the order of combine_kernel (base, then the
+// picks in ascending j; with at most 8 picks absent ones add +0 as there), so the output is the
+// same bit for bit.  Waits are bounded (error bit 2, the copies in flight drained).
+constexpr int CB_COLS = 1024;                  // columns per chunk (8 per thread, 128 threads)
+__global__ void __launch_bounds__(128) combine_bulk_kernel(const __nv_bfloat16* __restrict__ y,
+                                                           const int32_t* __restrict__ slot_of,
+                                                           const float* __restrict__ base,
+                                                           __nv_bfloat16* __restrict__ out, int Tn, int d, int k,
+                                                           long long S, uint32_t* err) {
+    extern __shared__ __align__(128) uint8_t stage_mem[];
+    __shared__ __align__(8) uint64_t bars[2];
+    __shared__ int pos_s[2][32];
+    __shared__ int abort_s;
+    const int tid = threadIdx.x;
+    const int nch = (d + CB_COLS - 1) / CB_COLS;
+    const uint32_t rows_bytes = (uint32_t)k * CB_COLS * 2;                 // routed segments of a stage
+    const uint32_t stage_bytes = rows_bytes + (base ? CB_COLS * 4u : 0u);
+    const uint32_t bar0 = (uint32_t)__cvta_generic_to_shared(&bars[0]);
+    const uint32_t st0 = (uint32_t)__cvta_generic_to_shared(stage_mem);
+    if (tid == 0) {
+        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar0) : "memory");
+        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar0 + 8) : "memory");
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        abort_s = 0;
+    }
+    __syncthreads();
+    // items of this block: token blockIdx.x + u * gridDim.x, chunk c, in (token, chunk) order
+    const int ntok = (int)blockIdx.x < Tn ? (Tn - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+    const int n = ntok * nch;
+    auto issue = [&](int i) {                                  // thread 0: item i into stage i & 1
+        const int t = (int)blockIdx.x + (i / nch) * (int)gridDim.x;
+        const int c0 = (i % nch) * CB_COLS;
+        const int cb = min(CB_COLS, d - c0);
+        const int sidx = i & 1;
+        const uint32_t b = bar0 + 8u * sidx, dst = st0 + stage_bytes * sidx;
+        uint32_t bytes = 0;
+        for (int j = 0; j < k; ++j) {
+            int p = slot_of[(size_t)t * k + j];
+            if (p >= S) { flag_error(err, ERR_INDEX_RANGE); p = -1; }
+            else if (p < 0) { if (c0 == 0) flag_error(err, ERR_INDEX_RANGE); p = -1; }
+            pos_s[sidx][j] = p;
+            if (p >= 0) bytes += (uint32_t)cb * 2;
+        }
+        if (base) bytes += (uint32_t)cb * 4;
+        asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(b), "r"(bytes) : "memory");
+        for (int j = 0; j < k; ++j) {
+            const int p = pos_s[sidx][j];
+            if (p >= 0)
+                asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                                 dst + (uint32_t)j * CB_COLS * 2),
+                             "l"(y + (size_t)p * d + c0), "r"((uint32_t)cb * 2), "r"(b)
+                             : "memory");
+        }
+        if (base)
+            asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                             dst + rows_bytes),
+                         "l"(base + (size_t)t * d + c0), "r"((uint32_t)cb * 4), "r"(b)
+                         : "memory");
+    };
+    if (tid == 0 && n > 0) issue(0);
+    int i = 0;
+    for (; i < n; ++i) {
+        if (tid == 0 && i + 1 < n) issue(i + 1);               // its stage was released by the barrier below
+        const int sidx = i & 1;
+        if (!scatter_wait(bar0 + 8u * sidx, (uint32_t)((i >> 1) & 1))) {
+            atomicExch(&abort_s, 1);
+            flag_error(err, ERR_PIPE_TIMEOUT);
+        }
+        __syncthreads();
+        if (abort_s) break;
+        const int t = (int)blockIdx.x + (i / nch) * (int)gridDim.x;
+        const int c0 = (i % nch) * CB_COLS;
+        const int cb = min(CB_COLS, d - c0);
+        const int col = tid * 8;
+        if (col < cb) {
+            const uint8_t* sb = stage_mem + (size_t)stage_bytes * sidx;
+            float acc[8];
+            if (base) {
+                const float4* b4 = reinterpret_cast<const float4*>(sb + rows_bytes) + tid * 2;
+                const float4 f0 = b4[0], f1 = b4[1];
+                acc[0] = f0.x; acc[1] = f0.y; acc[2] = f0.z; acc[3] = f0.w;
+                acc[4] = f1.x; acc[5] = f1.y; acc[6] = f1.z; acc[7] = f1.w;
+            } else {
+#pragma unroll
+                for (int q = 0; q < 8; ++q) acc[q] = 0.f;
+            }
+            const int jmax = k <= 8 ? 8 : k;
+            for (int j = 0; j < jmax; ++j) {
+                const bool live = j < k && pos_s[sidx][j] >= 0;
+                if (!live && k > 8) continue;                  // as combine_kernel: zeros added only with <= 8 picks
+                uint4 v = make_uint4(0, 0, 0, 0);
+                if (live) v = *reinterpret_cast<const uint4*>(sb + (size_t)j * CB_COLS * 2 + (size_t)col * 2);
+                const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    acc[2 * q] += __uint_as_float(w[q] << 16);
+                    acc[2 * q + 1] += __uint_as_float(w[q] & 0xFFFF0000u);
+                }
+            }
+            uint4 o;
+            o.x = pack_bf16x2(acc[0], acc[1]); o.y = pack_bf16x2(acc[2], acc[3]);
+            o.z = pack_bf16x2(acc[4], acc[5]); o.w = pack_bf16x2(acc[6], acc[7]);
+            *reinterpret_cast<uint4*>(out + (size_t)t * d + c0 + col) = o;
+        }
+        __syncthreads();                                      // stage sidx free for item i + 2
+    }
+    if (tid == 0 && abort_s) {                                // drain what is still in flight
+        scatter_wait(bar0 + 8u * (i & 1), (uint32_t)((i >> 1) & 1));
+        if (i + 1 < n) scatter_wait(bar0 + 8u * ((i + 1) & 1), (uint32_t)(((i + 1) >> 1) & 1));
+    }
+}
+
 }  // namespace
 
 cudaError_t launch_permute(const Dims& D, const int32_t* idx, const float* gate, int32_t* counts, int32_t* offsets,
@@ -421,10 +632,39 @@ cudaError_t launch_gather(const Dims& D, const void* x, const int32_t* sorted_to
     return cudaGetLastError();
 }
 
+cudaError_t launch_scatter_rows_bulk(const void* src, const float* sscale, const int32_t* slot_of, int T, int k,
+                                     long long S, uint32_t row_bytes, void* dst, float* dscale, uint32_t* err,
+                                     cudaStream_t stream) {
+    if (T <= 0) return cudaSuccess;
+    if (row_bytes % 16 || row_bytes > 32768 || k > 32 || ((uintptr_t)src & 15u) || ((uintptr_t)dst & 15u) ||
+        (dscale && !sscale))
+        return cudaErrorNotSupported;
+    static int per_sm = 0;
+    static uint32_t per_sm_bytes = 0;
+    const int smem = 2 * (int)row_bytes;
+    if (smem > 48 * 1024 &&
+        cudaFuncSetAttribute(scatter_rows_bulk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+        return cudaErrorInvalidValue;
+    if (per_sm_bytes != row_bytes) {
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, scatter_rows_bulk_kernel, 32, smem) != cudaSuccess ||
+            per_sm < 1)
+            per_sm = 1;
+        per_sm_bytes = row_bytes;
+    }
+    const int cap = per_sm * num_sms();
+    scatter_rows_bulk_kernel<<<T < cap ? T : cap, 32, smem, stream>>>((const char*)src, slot_of, (char*)dst, T, k, S,
+                                                                      row_bytes, sscale, dscale, err);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_scatter_rows(const Dims& D, const void* x, const int32_t* slot_of, void* x_perm, uint32_t* err,
                                 cudaStream_t stream) {
     if (D.T == 0) return cudaSuccess;
     const int esz = D.bf16 ? 2 : 4;
+    const uint32_t row_bytes = (uint32_t)D.d * esz;
+    const cudaError_t e = launch_scatter_rows_bulk(x, nullptr, slot_of, D.T, D.k, D.slots(), row_bytes, x_perm, nullptr,
+                                                   err, stream);
+    if (e != cudaErrorNotSupported) return e;                  // else: rows not 16-byte aligned, register copy
     const int vec = D.d * esz / 16;
     const int blocks = D.T < 148 * 16 ? D.T : 148 * 16;
     scatter_rows_kernel<<<blocks, 128, 0, stream>>>((const uint4*)x, slot_of, (uint4*)x_perm, D.T, D.k, D.slots(), vec,
@@ -465,6 +705,25 @@ void combine_dispatch(const Dims& D, const void* y, const int32_t* slot_of, cons
 cudaError_t launch_combine(const Dims& D, const void* y_sorted, const int32_t* slot_of, const float* base, void* out,
                            uint32_t* err, cudaStream_t stream) {
     if (D.T == 0) return cudaSuccess;
+    if (D.bf16 && D.d % 8 == 0 && D.k <= 32 && ((uintptr_t)y_sorted & 15u) == 0 && ((uintptr_t)out & 15u) == 0 &&
+        ((uintptr_t)base & 15u) == 0) {
+        static const int cap8 = resident_blocks(combine_kernel<__nv_bfloat16, 8, 8>, 128);
+        const long long chunks = (D.d / 8 + 127) / 128;
+        if (D.d >= 2048 && (long long)D.T * chunks > 2LL * cap8) {   // many tokens, long rows: bulk-staged inputs
+            const int smem = 2 * (D.k * CB_COLS * 2 + (base ? CB_COLS * 4 : 0));
+            if (cudaFuncSetAttribute(combine_bulk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+                cudaSuccess)
+                return cudaErrorInvalidValue;
+            int per_sm = 0;
+            if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, combine_bulk_kernel, 128, smem) != cudaSuccess ||
+                per_sm < 1)
+                per_sm = 1;
+            const int cap = per_sm * num_sms();
+            combine_bulk_kernel<<<D.T < cap ? D.T : cap, 128, smem, stream>>>(
+                (const __nv_bfloat16*)y_sorted, slot_of, base, (__nv_bfloat16*)out, D.T, D.d, D.k, D.slots(), err);
+            return cudaGetLastError();
+        }
+    }
     if (D.bf16 && D.d % 8 == 0) combine_dispatch<__nv_bfloat16, 8>(D, y_sorted, slot_of, base, out, err, stream);
     else if (D.bf16) combine_dispatch<__nv_bfloat16, 1>(D, y_sorted, slot_of, base, out, err, stream);
     else if (D.d % 4 == 0) combine_dispatch<float, 4>(D, y_sorted, slot_of, base, out, err, stream);

@@ -302,6 +302,9 @@ cudaError_t launch_scatter_code_rows(const uint8_t* src, const float* sscale, co
                                      cudaStream_t stream) {
     if (T <= 0) return cudaSuccess;
     if (row_bytes <= 0 || row_bytes % 16 || k > 32) return cudaErrorInvalidValue;
+    const cudaError_t e = launch_scatter_rows_bulk(src, sscale, slot_of, T, k, S, (uint32_t)row_bytes, dst, dscale, err,
+                                                   stream);
+    if (e != cudaErrorNotSupported) return e;                  // else: the register copy below
     const int blocks = T < num_sms() * 16 ? T : num_sms() * 16;
     scatter_code_rows_kernel<<<blocks, 128, 0, stream>>>((const uint4*)src, sscale, slot_of, T, k, S, row_bytes / 16,
                                                          (uint4*)dst, dscale, err);
