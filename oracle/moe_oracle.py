@@ -35,6 +35,11 @@ What it computes, and where it comes from:
   at 448), so it is exact and reproducible; the products and sums run in fp64 on the exact
   dequantised values.  The e4m3 format is taken from its definition (1 sign, 4 exponent bits
   with bias 7, 3 mantissa bits, subnormals, S.1111.111 = NaN, no infinities).
+  A second weight format keeps one power-of-two scale per run of 32 consecutive elements
+  along each weight row's input axis instead of one scale per row (block scales; the pages
+  give no block size or scale type either, so this is the same kind of reading): the scale is
+  the smallest power of two that keeps every element of the run within +-448, stored as an
+  unsigned exponent byte (mx_block_exponents); activations are quantised per row as above.
 * Backward pass (an extension; the pages discuss it only through SonicMoE's backward kernels):
   the chain rule of the forward above (layer_backward), and the balance statistics that the
   DeepSeekMoE report's expert- and device-level balance losses are built from (balance_stats;
@@ -255,6 +260,54 @@ def dequantized_rows(a: np.ndarray) -> np.ndarray:
     return q * s.astype(np.float64)[..., None]
 
 
+MX_BLOCK = 32
+MX_EXP_MIN, MX_EXP_MAX = -127, 127
+
+
+def mx_block_exponents(a: np.ndarray) -> np.ndarray:
+    """Block exponents of the block-scaled FP8 weight format: the last axis (the contraction
+    axis of a weight row) is cut into runs of MX_BLOCK consecutive elements (the last run may be
+    shorter), and each run gets the smallest integer e with max|run| <= 448 * 2^e, so that no
+    element of the run saturates; an all-zero run gets e = 0; e is kept within [-127, 127], the
+    range of the unsigned byte e + 127 that stores the scale 2^e.  Returns int64 [..., runs]."""
+    a = np.abs(np.asarray(a, np.float64))
+    K = a.shape[-1]
+    runs = -(-K // MX_BLOCK)
+    pad = np.zeros(a.shape[:-1] + (runs * MX_BLOCK - K,))
+    amax = np.concatenate([a, pad], axis=-1).reshape(a.shape[:-1] + (runs, MX_BLOCK)).max(axis=-1)
+    _, ex = np.frexp(amax)                      # amax in [2^(ex-1), 2^ex)
+    e = (ex - 1) - 8                            # 448 * 2^e = 1.75 * 2^(ex-1): the candidate
+    e = e + (amax > E4M3_MAX * np.exp2(e.astype(np.float64)))
+    e = np.where(amax == 0, 0, np.clip(e, MX_EXP_MIN, MX_EXP_MAX))
+    return e.astype(np.int64)
+
+
+def quantize_blocks_e4m3(a: np.ndarray):
+    """Block-scaled e4m3 quantisation of a weight row (or stack of rows): element j of run b
+    becomes e4m3_round(a_j / 2^e_b), exact in fp64.  Returns (values on the e4m3 grid as fp64,
+    exponents from mx_block_exponents); the row stands for values * 2^e of its run."""
+    a = np.asarray(a, np.float64)
+    e = mx_block_exponents(a)
+    scale = np.repeat(np.exp2(e.astype(np.float64)), MX_BLOCK, axis=-1)[..., : a.shape[-1]]
+    return e4m3_round(a / scale), e
+
+
+def dequantized_blocks(a: np.ndarray) -> np.ndarray:
+    """The values a block-scaled e4m3 quantisation of a stands for."""
+    q, e = quantize_blocks_e4m3(a)
+    scale = np.repeat(np.exp2(e.astype(np.float64)), MX_BLOCK, axis=-1)[..., : q.shape[-1]]
+    return q * scale
+
+
+def mx_weights(w: Weights) -> Weights:
+    """One expert with w1, w3, w2 replaced by their block-scaled e4m3 values (each row quantised
+    along its input axis, the axis the GEMMs contract); biases unchanged."""
+    out = dict(w)
+    for name in ("w1", "w3", "w2"):
+        out[name] = dequantized_blocks(w[name])
+    return out
+
+
 def e4m3_weights(w: Weights) -> Weights:
     """One expert in the FP8 format (codes w1/w3/w2 as uint8, per-output-channel scales
     s1/s3/s2) -> fp64 weights codes * scale; biases unchanged."""
@@ -280,7 +333,7 @@ def layer(x: np.ndarray, centroids: np.ndarray, routed: ExpertSource, n_experts:
           shared: Optional[ExpertSource] = None, n_shared: int = 0,
           idx_override: Optional[np.ndarray] = None, keep_hidden: bool = False,
           gate_mode: int = GATE_SOFTMAX_TOPK, router_bias: Optional[np.ndarray] = None,
-          routed_e4m3: bool = False) -> Dict[str, np.ndarray]:
+          routed_e4m3: bool = False, routed_mx: bool = False) -> Dict[str, np.ndarray]:
     """The DeepSeekMoE layer forward in fp64.
 
     routed / shared: either dicts of stacked arrays (w1,b1,w3,b3,w2,b2 indexed by expert) or
@@ -291,6 +344,9 @@ def layer(x: np.ndarray, centroids: np.ndarray, routed: ExpertSource, n_experts:
     routed_e4m3: the routed experts are in the FP8 format (e4m3_weights); their inputs and
     hidden rows are quantised per row (quantize_rows_e4m3, the hidden row after rounding to
     bf16).  The router and the shared experts are unchanged.
+    routed_mx: the routed experts' weights are given as plain values and are quantised here to
+    the block-scaled FP8 format (mx_weights); inputs and hidden rows are quantised per row as
+    with routed_e4m3.
 
     Returns out [T,d], routed_sum, shared_sum, idx, gate, gap, gap_order, counts, and
     Y [T*k, d] = gate * Expert_e(x_t) per slot (slot = t*k + j); with keep_hidden also
@@ -307,15 +363,18 @@ def layer(x: np.ndarray, centroids: np.ndarray, routed: ExpertSource, n_experts:
     k = top_k
     Y = np.zeros((T * k, d))
     H = None
-    xq = dequantized_rows(x) if routed_e4m3 else x
+    fp8 = routed_e4m3 or routed_mx
+    xq = dequantized_rows(x) if fp8 else x
     for e in np.unique(idx):
         w = _expert(routed, int(e))
         if routed_e4m3:
             w = e4m3_weights(w)
+        elif routed_mx:
+            w = mx_weights(w)
         tt, jj = np.nonzero(idx == e)
         xe = xq[tt]
         he = swiglu_hidden(xe, w["w1"], w["b1"], w["w3"], w["b3"])
-        ye = linear(dequantized_rows(bf16_round(he)) if routed_e4m3 else he, w["w2"], w["b2"])
+        ye = linear(dequantized_rows(bf16_round(he)) if fp8 else he, w["w2"], w["b2"])
         if keep_hidden:
             if H is None:
                 H = np.zeros((T * k, he.shape[1]))

@@ -427,6 +427,134 @@ def check_e4m3_format(O):
     assert rel.max() <= 16.0 / 448.0          # half of the widest step (32, in [256, 448]) per scale unit
 
 
+def _mx_exponent_brute(amax):
+    """Smallest integer e in [-127, 127] with amax <= 448 * 2^e, found by trying every e in
+    order (0 for amax == 0): the block-scale rule, searched instead of computed."""
+    if amax == 0:
+        return 0
+    for e in range(-127, 128):
+        if amax <= 448.0 * 2.0 ** e:
+            return e
+    raise AssertionError("no exponent fits")
+
+
+def _torch_mx_values(a, block=32):
+    """Block-scaled e4m3 values of rows a (runs of `block` along the last axis) from the
+    brute-force exponents and torch's float8_e4m3fn cast."""
+    a = np.asarray(a, np.float64)
+    out = np.empty_like(a)
+    for idx in np.ndindex(a.shape[:-1]):
+        row = a[idx]
+        for b0 in range(0, row.shape[0], block):
+            run = row[b0:b0 + block]
+            e = _mx_exponent_brute(float(np.abs(run).max()))
+            out[idx][b0:b0 + block] = _torch_e4m3(run / 2.0 ** e) * 2.0 ** e
+    return out
+
+
+def check_mx_block_format(O):
+    """The block-scaled weight format: exponents against worked examples and a brute-force
+    search, values against torch's e4m3 cast, runs of 32 along the last axis with a ragged last
+    run, and the bounds that the smallest non-saturating power of two implies."""
+    assert O.MX_BLOCK == 32
+    # worked examples (one run each; the rest of the run is zero):
+    #   448 fits 448 * 2^0 exactly                       -> e = 0,  code 448
+    #   449 needs 448 * 2^1 = 896                         -> e = 1,  449 / 2 = 224.5 -> 224 (step 16)
+    #   1.0: 448 * 2^-8 = 1.75 >= 1 > 448 * 2^-9 = 0.875  -> e = -8, code 256
+    #   1.75 fits 448 * 2^-8 exactly                      -> e = -8, code 448
+    #   the next double above 1.75                        -> e = -7, code 224
+    #   a zero run                                        -> e = 0
+    #   2^-140 would need e = -148: clamped to -127       -> code 2^-13 rounds to 0
+    #   -3e38 (near fp32's largest)                       -> e = 120, code -3e38 / 2^120 ~ -225.7 -> -224
+    heads = [448.0, 449.0, 1.0, 1.75, np.nextafter(1.75, 2.0), 0.0, 2.0 ** -140, -3e38]
+    a = np.zeros((len(heads), 32))
+    a[:, 0] = heads
+    e = O.mx_block_exponents(a)
+    assert e.shape == (len(heads), 1) and e.dtype == np.int64
+    assert e[:, 0].tolist() == [0, 1, -8, -8, -7, 0, -127, 120]
+    q, e2 = O.quantize_blocks_e4m3(a)
+    assert np.array_equal(e2, e)
+    assert q[:, 0].tolist() == [448.0, 224.0, 256.0, 448.0, 224.0, 0.0, 0.0, -224.0]
+    # random runs over many binades, element spread within a run up to 2^30; ragged K = 70
+    rng = _rng(31)
+    a = rng.standard_normal((40, 70)) * np.exp2(rng.uniform(-60, 60, (40, 1)))
+    a *= np.exp2(rng.uniform(-30, 0, a.shape))
+    a[3] = 0.0
+    a[5, 32:64] = 0.0
+    a = a.astype(np.float32).astype(np.float64)
+    e = O.mx_block_exponents(a)
+    assert e.shape == (40, 3)
+    runs = [(0, 32), (32, 64), (64, 70)]
+    for i in range(40):
+        for b, (lo, hi) in enumerate(runs):
+            assert e[i, b] == _mx_exponent_brute(float(np.abs(a[i, lo:hi]).max()))
+    assert e[3].tolist() == [0, 0, 0] and e[5, 1] == 0
+    dq = O.dequantized_blocks(a)
+    assert np.array_equal(dq, _torch_mx_values(a))
+    q, _ = O.quantize_blocks_e4m3(a)
+    for i in range(40):
+        for b, (lo, hi) in enumerate(runs):
+            m = np.abs(q[i, lo:hi]).max()
+            assert m == 0 or 224.0 <= m <= 448.0        # smallest non-saturating scale
+            err = np.abs(dq[i, lo:hi] - a[i, lo:hi]).max()
+            assert err <= 16.0 * 2.0 ** e[i, b]         # half the widest e4m3 step, per scale unit
+    # the exponent byte range
+    assert ((e + 127 >= 0) & (e + 127 <= 254)).all()
+    # runs do not interact: changing one run leaves the others' codes alone
+    b2 = a.copy()
+    b2[:, 32:64] *= 1000.0
+    q2, _ = O.quantize_blocks_e4m3(b2)
+    assert np.array_equal(q2[:, :32], q[:, :32]) and np.array_equal(q2[:, 64:], q[:, 64:])
+
+
+def check_mx_layer_closed_form(O):
+    """The block-scaled FP8 routed path on experts whose weight rows hold one non-zero value
+    each (so each run of 32 holds at most one value and each Linear is a scaled selection): the
+    layer must equal the closed form built from brute-force block exponents, torch's e4m3 and
+    bf16 casts and scipy's expit, with per-row activation scales and an unquantised shared
+    expert."""
+    rng = _rng(32)
+    T, d, I, N, k = 5, 64, 40, 3, 2
+    x = rng.standard_normal((T, d)) * np.exp2(rng.uniform(-4, 4, (T, 1)))
+    x = x.astype(np.float32).astype(np.float64)
+    c = rng.normal(0, 0.5, (N, d))
+    experts = []
+    for _ in range(N):
+        e = {}
+        for name, (rows, cols) in (("w1", (I, d)), ("w3", (I, d)), ("w2", (d, I))):
+            pick = rng.integers(0, cols, rows)
+            w = np.zeros((rows, cols))
+            w[np.arange(rows), pick] = (rng.standard_normal(rows) * np.exp2(rng.uniform(-12, 2, rows)))
+            e[name] = torch.from_numpy(w).float().bfloat16().double().numpy()
+            e["p" + name[1]] = pick
+        for b, n in (("b1", I), ("b3", I), ("b2", d)):
+            e[b] = rng.normal(0, 0.1, n)
+        experts.append(e)
+    shared = _rand_expert(rng, d, 8, std=0.2)
+    stack = _stack([{k_: v for k_, v in e.items() if not k_.startswith("p")} for e in experts])
+    res = O.layer(x, c, stack, N, k, shared=_stack([shared]), n_shared=1, routed_mx=True)
+    r = O.route(x, c, k)
+    xq = _torch_quant_rows(x)
+
+    def val(e, name, rows):
+        w = e[name][np.arange(rows), e["p" + name[1]]]
+        ex = np.array([_mx_exponent_brute(abs(v)) for v in w], np.float64)
+        return _torch_e4m3(w / 2.0 ** ex) * 2.0 ** ex
+
+    want = torch_expert(shared, x)
+    for t in range(T):
+        for j in range(k):
+            e = experts[r["idx"][t, j]]
+            a = val(e, "w1", I) * xq[t, e["p1"]] + e["b1"]
+            g = val(e, "w3", I) * xq[t, e["p3"]] + e["b3"]
+            h = a * scipy.special.expit(a) * g
+            hb = torch.from_numpy(h).float().bfloat16().double().numpy()
+            hq = _torch_quant_rows(hb[None])[0]
+            y = val(e, "w2", d) * hq[e["p2"]] + e["b2"]
+            want[t] += r["gate"][t, j] * y
+    assert np.allclose(res["out"], want, rtol=1e-12, atol=1e-12)
+
+
 def check_fp8_layer_closed_form(O):
     """The FP8 routed path on experts whose weight matrices hold one e4m3 code per row (a
     selection of one input per output, so each Linear reduces to a scaled copy): the layer
@@ -617,5 +745,6 @@ def check_balance_stats(O):
 ALL_CHECKS = [check_ptflops_printout, check_combinations, check_textbook_single_expert,
               check_gate_invariants, check_bruteforce_routing, check_split_identity,
               check_shared_bypasses_router, check_hit_entropy, check_permute, check_gate_modes,
-              check_e4m3_format, check_fp8_layer_closed_form, check_backward_autograd,
+              check_e4m3_format, check_fp8_layer_closed_form, check_mx_block_format,
+              check_mx_layer_closed_form, check_backward_autograd,
               check_backward_finite_differences, check_balance_stats]

@@ -12,7 +12,8 @@ from tests import pins
 _orig = {name: getattr(O, name) for name in ("silu", "linear", "route", "swiglu_hidden", "permute",
                                              "expert_macs", "split_expert", "hit_entropy", "e4m3_round",
                                              "quantize_rows_e4m3", "e4m3_weights", "e4m3_decode",
-                                             "silu_grad", "gate_backward", "expert_backward", "balance_stats")}
+                                             "silu_grad", "gate_backward", "expert_backward", "balance_stats",
+                                             "mx_block_exponents", "mx_weights")}
 
 
 def _sigmoid_for_silu(a):                      # silu without the factor a
@@ -179,6 +180,31 @@ def _balance_unnormalised(s, idx, n, k, n_groups=1):   # f as raw hit counts
     return b
 
 
+def _mx_exponent_floor(a):                     # saturating rule: floor(log2 max) - 8, the top of a run clips
+    a = np.abs(np.asarray(a, np.float64))
+    K = a.shape[-1]
+    runs = -(-K // 32)
+    pad = np.zeros(a.shape[:-1] + (runs * 32 - K,))
+    amax = np.concatenate([a, pad], axis=-1).reshape(a.shape[:-1] + (runs, 32)).max(axis=-1)
+    _, ex = np.frexp(amax)
+    return np.where(amax == 0, 0, np.clip(ex - 1 - 8, -127, 127)).astype(np.int64)
+
+
+def _mx_exponent_per_row(a):                   # one exponent for the whole row, repeated per run
+    e = _orig["mx_block_exponents"](a)
+    return np.repeat(e.max(axis=-1, keepdims=True), e.shape[-1], axis=-1)
+
+
+def _mx_exponent_off_by_one(a):                # one power of two too large
+    return _orig["mx_block_exponents"](a) + 1
+
+
+def _mx_weights_skip_w2(w):                    # w2 left unquantised
+    out = _orig["mx_weights"](w)
+    out["w2"] = w["w2"]
+    return out
+
+
 MUTANTS = {
     "silu_is_sigmoid": ("silu", _sigmoid_for_silu),
     "linear_drops_bias": ("linear", _linear_no_bias),
@@ -202,6 +228,11 @@ MUTANTS = {
     "gate_backward_drops_softmax_term": ("gate_backward", _gate_backward_no_softmax_term),
     "expert_backward_drops_g": ("expert_backward", _expert_backward_no_gate_factor),
     "balance_f_unnormalised": ("balance_stats", _balance_unnormalised),
+    "mx_exponent_saturating_floor": ("mx_block_exponents", _mx_exponent_floor),
+    "mx_exponent_per_row": ("mx_block_exponents", _mx_exponent_per_row),
+    "mx_exponent_off_by_one": ("mx_block_exponents", _mx_exponent_off_by_one),
+    "mx_runs_of_16": ("MX_BLOCK", 16),
+    "mx_w2_unquantised": ("mx_weights", _mx_weights_skip_w2),
 }
 
 
