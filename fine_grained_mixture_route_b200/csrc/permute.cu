@@ -6,6 +6,8 @@
 // a scan over (expert, block), and a scatter that ranks equal experts inside a warp with
 // __match_any_sync.  Inside an expert the slots keep ascending order, so the result does not
 // depend on scheduling (no order-dependent atomics).
+#include <atomic>
+
 #include "common.cuh"
 #include "launch.h"
 
@@ -632,6 +634,21 @@ cudaError_t launch_gather(const Dims& D, const void* x, const int32_t* sorted_to
     return cudaGetLastError();
 }
 
+// Blocks of `kern` (threads, smem bytes) resident on the whole GPU, cached per shared-memory size
+// (one entry per kernel instantiation: each call site passes its own cache).  The cached value only
+// sizes persistent grids, so a stale or racing read changes the wave count, never the result.
+template <typename K>
+int resident_blocks_cached(K kern, int threads, int smem, std::atomic<unsigned long long>& cache) {
+    const unsigned long long c = cache.load(std::memory_order_relaxed);
+    if (c && (int)(c >> 32) == smem) return (int)(c & 0xFFFFFFFFu);
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, smem) != cudaSuccess || per_sm < 1)
+        per_sm = 1;
+    const int n = per_sm * num_sms();
+    cache.store(((unsigned long long)(unsigned)smem << 32) | (unsigned)n, std::memory_order_relaxed);
+    return n;
+}
+
 cudaError_t launch_scatter_rows_bulk(const void* src, const float* sscale, const int32_t* slot_of, int T, int k,
                                      long long S, uint32_t row_bytes, void* dst, float* dscale, uint32_t* err,
                                      cudaStream_t stream) {
@@ -639,19 +656,12 @@ cudaError_t launch_scatter_rows_bulk(const void* src, const float* sscale, const
     if (row_bytes % 16 || row_bytes > 32768 || k > 32 || ((uintptr_t)src & 15u) || ((uintptr_t)dst & 15u) ||
         (dscale && !sscale))
         return cudaErrorNotSupported;
-    static int per_sm = 0;
-    static uint32_t per_sm_bytes = 0;
+    static std::atomic<unsigned long long> cache{0};
     const int smem = 2 * (int)row_bytes;
     if (smem > 48 * 1024 &&
         cudaFuncSetAttribute(scatter_rows_bulk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return cudaErrorInvalidValue;
-    if (per_sm_bytes != row_bytes) {
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, scatter_rows_bulk_kernel, 32, smem) != cudaSuccess ||
-            per_sm < 1)
-            per_sm = 1;
-        per_sm_bytes = row_bytes;
-    }
-    const int cap = per_sm * num_sms();
+    const int cap = resident_blocks_cached(scatter_rows_bulk_kernel, 32, smem, cache);
     scatter_rows_bulk_kernel<<<T < cap ? T : cap, 32, smem, stream>>>((const char*)src, slot_of, (char*)dst, T, k, S,
                                                                       row_bytes, sscale, dscale, err);
     return cudaGetLastError();
@@ -714,11 +724,8 @@ cudaError_t launch_combine(const Dims& D, const void* y_sorted, const int32_t* s
             if (cudaFuncSetAttribute(combine_bulk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
                 cudaSuccess)
                 return cudaErrorInvalidValue;
-            int per_sm = 0;
-            if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, combine_bulk_kernel, 128, smem) != cudaSuccess ||
-                per_sm < 1)
-                per_sm = 1;
-            const int cap = per_sm * num_sms();
+            static std::atomic<unsigned long long> cache{0};
+            const int cap = resident_blocks_cached(combine_bulk_kernel, 128, smem, cache);
             combine_bulk_kernel<<<D.T < cap ? D.T : cap, 128, smem, stream>>>(
                 (const __nv_bfloat16*)y_sorted, slot_of, base, (__nv_bfloat16*)out, D.T, D.d, D.k, D.slots(), err);
             return cudaGetLastError();
