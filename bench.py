@@ -2,7 +2,7 @@
 """Benchmark of the B200 DeepSeekMoE layer forward.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload prefill|decode|mid|small|tiny]
-                    [--impl ours|reference] [--gate-mode 0|1|2] [--routed-fmt bf16|e4m3]
+                    [--impl ours|reference] [--gate-mode 0|1|2] [--routed-fmt bf16|e4m3|mxfp8]
 
 One step = one moe_layer_forward over one batch of synthetic tokens (router, grouping, row
 gather, GEMM1+SwiGLU, GEMM2+gate, shared GEMM2+combine), inputs resident in HBM.  The
@@ -16,7 +16,8 @@ Multi-GPU runs are replicas: every rank holds the same weights and processes its
 (weak scaling) and value = tokens of all ranks / the slowest rank's time.
 
 --routed-fmt e4m3 stores the routed experts' weights as e4m3 codes with per-channel scales
-(converted once before timing) and runs their GEMMs on the FP8 tensor-core path.
+(converted once before timing) and runs their GEMMs on the FP8 tensor-core path; mxfp8 keeps a
+power-of-two scale per run of 32 inputs instead, applied by the tensor cores inside the MMA.
 
 --impl reference times the fp64 CPU oracle (the only reference that exists for this layer)
 on bounded samples of the same workload, on rank 0 only.
@@ -86,21 +87,30 @@ def aggregate_throughput(tokens_per_rank: int, n_ranks: int, max_ms_per_step: fl
     return tokens_per_rank * n_ranks / (max_ms_per_step / 1e3)
 
 
-def stage_work(cfg: W.LayerConfig, touched: int, e4m3: bool = False):
+def mx_scale_bytes_per_expert(cfg: W.LayerConfig):
+    """Block-scale bytes one routed expert's weights carry in the tiled layout the GEMMs load:
+    (W1 | W3, W2), 1 KB per (128-row group, 128-input chunk) and per (256-row group, chunk)."""
+    cd = lambda a, b: -(-a // b)
+    return cd(cfg.inter, 128) * cd(cfg.d, 128) * 1024, cd(cfg.d, 256) * cd(cfg.inter, 128) * 1024
+
+
+def stage_work(cfg: W.LayerConfig, touched: int, e4m3: bool = False, mx: bool = False):
     """Algorithmic FLOPs and HBM bytes of each stage of one layer call.
 
     Bytes count each operand once at its storage size: weights of the experts that received
     at least one token (`touched`), activations read and written by the stage, routing
     metadata.  FLOPs count 2 per multiply-add of the contractions only.  With e4m3 routed
     experts their weights, the gathered rows and the quantised hidden rows are 1 byte each,
-    plus one fp32 scale per weight row and per activation row; the gemm2 stage includes the
-    hidden-row quantisation (bf16 h read, e4m3 h written).
+    plus one fp32 scale per weight row and per activation row (mx: the weights' block-scale
+    bytes instead of per-row scales); the gemm2 stage includes the hidden-row quantisation (bf16 h
+    read, e4m3 h written).
     """
     T, d, E, I, k, Ks, Is = cfg.T, cfg.d, cfg.n_experts, cfg.inter, cfg.top_k, cfg.n_shared, cfg.inter_shared
     b = cfg.elem_bytes()
     S = T * k
     bias = 1 if cfg.has_bias else 0
     if e4m3:
+        w13_sc, w2_sc = mx_scale_bytes_per_expert(cfg) if mx else (2 * I * 4, d * 4)
         return {
             "router": (2.0 * T * d * E, (T * d + E * d) * b + S * 8),
             "permute": (0.0, S * 8 + S * 16),
@@ -108,12 +118,12 @@ def stage_work(cfg: W.LayerConfig, touched: int, e4m3: bool = False):
             # x read once (quantised per token), the code rows and scales stored at their slots
             "gather": (0.0, T * d * b + S * d + S * 4 + S * 4),
             "gemm1_swiglu": (2.0 * S * d * 2 * I + 2.0 * Ks * T * d * 2 * Is,
-                             touched * (2 * I * d + 2 * I * 4 + 2 * I * bias * b) + S * d + S * 4
+                             touched * (2 * I * d + w13_sc + 2 * I * bias * b) + S * d + S * 4
                              + Ks * (2 * Is * d + 2 * Is * bias) * b + (T * d * b if Ks else 0)
                              + (S * I + Ks * T * Is) * b),
             "gemm2": (2.0 * S * I * d + 2.0 * Ks * T * Is * d,
                       S * I * b + S * I + S * 4                                  # h quantisation
-                      + touched * (d * I + d * 4 + d * bias * b) + S * I + S * 4 + S * d * b + S * 4
+                      + touched * (d * I + w2_sc + d * bias * b) + S * I + S * 4 + S * d * b + S * 4
                       + Ks * (d * Is + d * bias) * b + Ks * T * Is * b + (T * d * 4 if Ks else 0)),
             "combine": (0.0, S * d * b + (T * d * 4 if Ks else 0) + T * d * b + S * 4),
         }
@@ -177,16 +187,19 @@ def routing_stats(counts) -> dict:
 
 
 def fmt_label(args, cfg: W.LayerConfig) -> str:
-    """Storage of the routed experts' weights: e4m3 codes, else the layer dtype."""
-    return "e4m3" if args.routed_fmt == "e4m3" else ("bf16" if cfg.dtype == torch.bfloat16 else "fp32")
+    """Storage of the routed experts' weights: e4m3 codes (per-row or block scales), else the layer dtype."""
+    if args.routed_fmt in ("e4m3", "mxfp8"):
+        return args.routed_fmt
+    return "bf16" if cfg.dtype == torch.bfloat16 else "fp32"
 
 
-def layer_bytes(cfg: W.LayerConfig, touched: int, e4m3: bool = False) -> float:
+def layer_bytes(cfg: W.LayerConfig, touched: int, e4m3: bool = False, mx: bool = False) -> float:
     """Algorithmic bytes of the whole layer: weights of touched experts, shared experts,
     centroids, x in and out once (intermediates excluded: the method need not keep them)."""
     b = cfg.elem_bytes()
     bias = 1 if cfg.has_bias else 0
-    routed = (3 * cfg.d * cfg.inter + (2 * cfg.inter + cfg.d) * 4 + (2 * cfg.inter + cfg.d) * bias * b) if e4m3 \
+    scales = sum(mx_scale_bytes_per_expert(cfg)) if mx else (2 * cfg.inter + cfg.d) * 4
+    routed = (3 * cfg.d * cfg.inter + scales + (2 * cfg.inter + cfg.d) * bias * b) if e4m3 \
         else (3 * cfg.d * cfg.inter + (2 * cfg.inter + cfg.d) * bias) * b
     return (touched * routed
             + cfg.n_shared * (3 * cfg.d * cfg.inter_shared + (2 * cfg.inter_shared + cfg.d) * bias) * b
@@ -293,13 +306,13 @@ class HostExperts:
         return {k: (None if v is None else v.float().numpy().astype(np.float64)) for k, v in h.items()}
 
 
-def oracle_sample(O, L, cfg, host_routed, host_shared, tokens, gate_mode=0, router_bias=None, e4m3=False):
+def oracle_sample(O, L, cfg, host_routed, host_shared, tokens, gate_mode=0, router_bias=None, e4m3=False, mx=False):
     x = L["x"][tokens].float().cpu().numpy().astype(np.float64)
     c = L["centroids"].float().cpu().numpy().astype(np.float64)
     b = None if router_bias is None else router_bias.double().cpu().numpy()
     t0 = time.perf_counter()
     O.layer(x, c, host_routed, cfg.n_experts, cfg.top_k, host_shared, cfg.n_shared, gate_mode=gate_mode,
-            router_bias=b, routed_e4m3=e4m3)
+            router_bias=b, routed_e4m3=e4m3 and not mx, routed_mx=mx)
     return time.perf_counter() - t0
 
 
@@ -315,12 +328,12 @@ def blas_threads():
 
 
 def cpu_baseline(cfg, L, idx_gpu, n_tokens=16, gate_mode=0, router_bias=None, e4m3=False, target_s=15.0,
-                 min_s=10.0, max_tokens=1024):
+                 min_s=10.0, max_tokens=1024, mx=False):
     """The oracle, as it stands, on the first tokens of this step's batch: n_tokens first; when
     that takes under min_s seconds, again on enough tokens for about target_s seconds of CPU work
     (at most max_tokens), and that sample is reported."""
     import oracle.moe_oracle as O
-    hr = HostExperts(L["routed"])
+    hr = HostExperts(L["routed_bf16"] if mx else L["routed"])     # block scales: the oracle converts bf16
     hs = HostExperts(L["shared"]) if L["shared"] is not None else None
     if hs is not None:
         hs.prefetch(range(cfg.n_shared))
@@ -328,11 +341,12 @@ def cpu_baseline(cfg, L, idx_gpu, n_tokens=16, gate_mode=0, router_bias=None, e4
     while True:
         tokens = np.arange(n)
         hr.prefetch(np.unique(idx_gpu[tokens]))              # weights staged in host memory, untimed
-        dt = oracle_sample(O, L, cfg, hr, hs, tokens, gate_mode, router_bias, e4m3)
+        dt = oracle_sample(O, L, cfg, hr, hs, tokens, gate_mode, router_bias, e4m3, mx)
         if dt >= min_s or n >= min(cfg.T, max_tokens):
             break
         n = min(cfg.T, max_tokens, int(n * target_s / max(dt, 1e-3)) + 1)
-    fmt = "e4m3 routed codes + scales and bf16 shared" if e4m3 else "bf16"
+    fmt = ("bf16 (block-scaled FP8 conversion by the oracle)" if mx
+           else "e4m3 routed codes + scales and bf16 shared" if e4m3 else "bf16")
     return {"value": len(tokens) / dt, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
             "sample": f"fp64 NumPy oracle on the first {len(tokens)} tokens of the {cfg.name} batch "
                       f"(all experts they route to; weights staged in host memory as {fmt}, converted by the oracle)",
@@ -346,15 +360,15 @@ def run_reference(args, cfg, rank, world):
     import oracle.moe_oracle as O
     dev = "cuda" if torch.cuda.is_available() else "cpu"
     L = W.make_layer(cfg, dev, seed=0)
-    e4m3 = args.routed_fmt == "e4m3"
+    e4m3, mx = args.routed_fmt == "e4m3", args.routed_fmt == "mxfp8"
     if e4m3:
         from fine_grained_mixture_route_b200 import quant
         L["routed"] = quant.quantize_stack(L["routed"])
-    hr = HostExperts(L["routed"])
+    hr = HostExperts(L["routed"])                   # block scales: bf16 weights, converted by the oracle
     hs = HostExperts(L["shared"]) if L["shared"] is not None else None
     budget_s = 150.0
     n = min(8, cfg.T)
-    t_first = oracle_sample(O, L, cfg, hr, hs, np.arange(n), e4m3=e4m3)   # sizing run (also warms the cache)
+    t_first = oracle_sample(O, L, cfg, hr, hs, np.arange(n), e4m3=e4m3, mx=mx)   # sizing run (also warms the cache)
     per_tok = t_first / n
     n = int(max(1, min(64, cfg.T, budget_s / max(1, args.steps + args.warmup) / max(per_tok, 1e-6))))
     pos = 0
@@ -362,7 +376,7 @@ def run_reference(args, cfg, rank, world):
     for i in range(args.warmup + args.steps):
         toks = (np.arange(n) + pos) % cfg.T
         pos += n
-        dt = oracle_sample(O, L, cfg, hr, hs, toks, e4m3=e4m3)
+        dt = oracle_sample(O, L, cfg, hr, hs, toks, e4m3=e4m3, mx=mx)
         if i >= args.warmup:
             times.append(dt)
     total = sum(times)
@@ -438,10 +452,10 @@ def decode_arm(moe, args, base_cfg, L, rbias, dev, stream, local_rank, world):
     gate = torch.empty((cfg.T, cfg.top_k), dtype=torch.float32, device=dev)
     counts = torch.empty(cfg.n_experts, dtype=torch.int32, device=dev)
     t = time_layer(moe, args, cfg, shape, x, C, R, Sh, ws, out, idx, gate, counts, rbias, dev, stream, local_rank)
-    e4m3 = args.routed_fmt == "e4m3"
+    e4m3, mx = args.routed_fmt in ("e4m3", "mxfp8"), args.routed_fmt == "mxfp8"
     peaks, peak_src = load_peaks()
-    lbytes = layer_bytes(cfg, t["touched"], e4m3)
-    work = stage_work(cfg, t["touched"], e4m3)
+    lbytes = layer_bytes(cfg, t["touched"], e4m3, mx)
+    work = stage_work(cfg, t["touched"], e4m3, mx)
     gbs = lbytes / (t["ms"] / 1e3) / 1e9
     stage_gbs = {k: work[k][1] / (t["stage_ms"][k] / 1e3) / 1e9 for k in ("gemm1_swiglu", "gemm2")}
     return {"workload": cfg.name, "T": cfg.T, "steps": args.steps, "warmup": args.warmup, "ms_per_step": t["ms"],
@@ -464,10 +478,12 @@ def run_ours(args, cfg, rank, world, local_rank):
     L = W.make_layer(cfg, dev, seed=0)
     if rank > 0:
         L["x"] = W.make_x(cfg, dev, seed=1000 + rank)
-    e4m3 = args.routed_fmt == "e4m3"
+    e4m3, mx = args.routed_fmt in ("e4m3", "mxfp8"), args.routed_fmt == "mxfp8"
     if e4m3:   # one-off weight conversion before anything is timed
         from fine_grained_mixture_route_b200 import quant
-        L["routed"] = quant.quantize_stack(L["routed"])
+        if mx:
+            L["routed_bf16"] = L["routed"]             # what the CPU baseline's oracle converts itself
+        L["routed"] = quant.quantize_stack(L["routed"], fmt=args.routed_fmt)
         torch.cuda.empty_cache()
     x, C, R, Sh = L["x"], L["centroids"], L["routed"], L["shared"]
     shape = moe.shape_of(x, C, R, cfg.top_k, Sh, gate_mode=args.gate_mode)
@@ -483,7 +499,7 @@ def run_ours(args, cfg, rank, world, local_rank):
 
     t = time_layer(moe, args, cfg, shape, x, C, R, Sh, ws, out, idx, gate, counts, rbias, dev, stream, local_rank)
     ms, stage_ms, clocks, touched = t["ms"], t["stage_ms"], t["clocks"], t["touched"]
-    work = stage_work(cfg, touched, e4m3)
+    work = stage_work(cfg, touched, e4m3, mx)
     launches_per_step = moe.layer_launches(shape)
 
     # ---- end to end through the public API: batches in pinned host memory, copied in and
@@ -536,7 +552,7 @@ def run_ours(args, cfg, rank, world, local_rank):
     roofline = {"bound": bound, "kernel": dom, "achieved": achieved, "peak": peak, "unit": unit,
                 "frac": achieved / peak,
                 "peak_source": f"{peak_src} ({tensor_src if bound == 'tensor' else 'HBM copy' if bound == 'hbm' else 'fp32 FMA nominal'})",
-                "traffic": ncu_traffic(cfg.name + ("+e4m3" if e4m3 else ""), dom),
+                "traffic": ncu_traffic(cfg.name + (f"+{args.routed_fmt}" if e4m3 else ""), dom),
                 "algorithmic_per_launch": flops if bound != "hbm" else nbytes}
     if bound == "tensor":
         # the other denominator, for reference: burst and sustained scale the blended peak alike
@@ -548,7 +564,7 @@ def run_ours(args, cfg, rank, world, local_rank):
 
     step_s = ms / 1e3
     total_flops = cfg.flops()
-    lbytes = layer_bytes(cfg, touched, e4m3)
+    lbytes = layer_bytes(cfg, touched, e4m3, mx)
     value = aggregate_throughput(cfg.T, world, ms)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -576,7 +592,7 @@ def run_ours(args, cfg, rank, world, local_rank):
         line["decode"] = decode_arm(moe, args, cfg, L, rbias, dev, stream, local_rank, world)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(cfg, L, idx.cpu().numpy(), gate_mode=args.gate_mode, router_bias=rbias,
-                                            e4m3=e4m3)
+                                            e4m3=e4m3, mx=mx)
     if rank == 0:
         print(json.dumps(line), flush=True)
 
@@ -681,9 +697,10 @@ def main(argv=None):
     ap.add_argument("--gate-mode", type=int, default=0, choices=[0, 1, 2],
                     help="router gate: 0 softmax over all experts (default), 1 softmax over the top-k logits of a "
                          "biased router, 2 sigmoid with a selection bias")
-    ap.add_argument("--routed-fmt", default="bf16", choices=["bf16", "e4m3"],
+    ap.add_argument("--routed-fmt", default="bf16", choices=["bf16", "e4m3", "mxfp8"],
                     help="storage of the routed experts' weights: bf16, or e4m3 codes with per-channel scales "
-                         "(FP8 tensor-core path; activations quantised per row)")
+                         "(e4m3) or with block scales per run of 32 inputs (mxfp8) (FP8 tensor-core path; "
+                         "activations quantised per row)")
     ap.add_argument("--pass", dest="pass_", default="forward", choices=["forward", "train"],
                     help="forward: the layer forward (default); train: forward for training + backward")
     ap.add_argument("--no-e2e", action="store_true")
@@ -697,8 +714,8 @@ def main(argv=None):
     if world != args.gpus and world > 1:
         ap.error(f"--gpus {args.gpus} but WORLD_SIZE={world}")
     cfg = W.CONFIGS[args.workload]
-    if args.routed_fmt == "e4m3" and cfg.dtype != torch.bfloat16:
-        ap.error("--routed-fmt e4m3 needs a bf16 workload")
+    if args.routed_fmt != "bf16" and cfg.dtype != torch.bfloat16:
+        ap.error(f"--routed-fmt {args.routed_fmt} needs a bf16 workload")
     if args.impl == "reference":
         run_reference(args, cfg, rank, world)
         return

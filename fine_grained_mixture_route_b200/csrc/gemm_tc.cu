@@ -60,6 +60,19 @@ constexpr int STAGE_OUT_BYTES = 2048;     // per epilogue warp: a 32 x 32 bf16 c
 constexpr int SMEM_BYTES = 1024 /*align slack*/ + RING_BYTES + 256 /*barriers*/ + EPI_WARPS * STAGE_OUT_BYTES;
 constexpr int ZERO_BYTES = 16384;         // DW: zeros that TMA stores copy to the gradients of groups without rows
 constexpr int SMEM_BYTES_DW = SMEM_BYTES + ZERO_BYTES;
+// Block-scaled weights (mxw): each stage also brings the B tile's scale bytes (256 rows x 4
+// runs of 32 = 1 KB, two 512-byte blocks of 128 rows each, row r at byte (r % 32) * 16 +
+// (r / 32 % 4) * 4 + run), copied from there into tensor-memory columns SFB_COL..SFB_COL + 7
+// before the stage's MMAs; the A side's scales are all 1 (byte 127, columns SFA_COL..+3,
+// written once).  To free those columns the second accumulator starts MX_OVL columns early
+// (224 instead of 256), so the two accumulators share columns 224-255: the epilogue drains
+// that shared chunk first and releases it through ovl_bar before the next tile's MMAs start.
+constexpr int MX_OVL = 32;
+constexpr int SF_STAGE_BYTES = 1024;
+constexpr int SFA_BYTES = 512;
+constexpr uint32_t SFA_COL = 2 * ACC_COLS - MX_OVL;            // 480
+constexpr uint32_t SFB_COL = SFA_COL + 8;                        // 488
+constexpr int SMEM_BYTES_Q8 = SMEM_BYTES + 4 * SF_STAGE_BYTES + SFA_BYTES;
 constexpr unsigned long long WAIT_NS = 4000000000ull;
 #ifndef MOE_GROUP_M
 #define MOE_GROUP_M 8                    // M-tiles per raster band of the expert GEMMs
@@ -112,6 +125,9 @@ struct Params {
     int q8;                    // routed tiles read e4m3 A and B (K blocks of 128 bytes)
     const float* a_scale;      // q8: per-row scale of the routed A rows (x_perm or h rows)
     const float *ws1, *ws3, *ws2;  // q8: per-output-channel weight scales [E, I], [E, I], [E, d]
+    int mxw;                   // q8 with block-scaled weights: the MMAs apply the weights' block scales
+    const uint8_t* sf13;       // mxw: W1 | W3 scale bytes, [E][ceil(I/128)][ceil(d/128)][W1, W3][512]
+    const uint8_t* sf2;        // mxw: W2 scale bytes, [E][ceil(d/256)][ceil(I/128)][2][512]
     int fold_shared;           // GEMM2R: shared-expert GEMM2 tiles follow the routed ones (-> sout)
     // ---- forward for training: GEMM1 also stores the pre-activations a = x W1^T + b1, g = x W3^T + b3
     __nv_bfloat16 *a_out, *g_out;      // routed [S][I] (grouped order)
@@ -293,6 +309,50 @@ __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b
         "l"(a), "l"(b), "r"(idesc), "r"(acc)
         : "memory");
 }
+// ---- block-scaled e4m3 weights (moe_expert_fmt_t MOE_FMT_MXFP8)
+// Instruction descriptor, kind::mxf8f6f4 with block scales: fp32 accumulator, e4m3 A and B
+// (format 0), K-major, M = 128, scale factors UE8M0 (bit 23); the byte of each 32-bit scale
+// column that an MMA reads is selected per operand (A: bits 29-30, B: bits 4-5).
+__host__ __device__ constexpr uint32_t idesc_mx(int n, int sf_byte) {
+    return ((uint32_t)sf_byte << 4) | ((uint32_t)(n >> 3) << 17) | (1u << 23) | ((uint32_t)(BM >> 4) << 24) |
+           ((uint32_t)sf_byte << 29);
+}
+// One block-scaled e4m3 MMA (K = 32): D (+)= (A * 2^sfa[row]) (B * 2^sfb[col])^T, where the scale
+// of A row r is the UE8M0 byte sf_byte of tensor-memory lane r, column sfa + r / 32, and the scale
+// of B row n likewise from column sfb + n / 32.  The byte index travels in bits 30-31 of the two
+// scale addresses as well as in the descriptor.
+__device__ __forceinline__ void mma_mx(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t sfa,
+                                       uint32_t sfb, uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
+        "l"(a), "l"(b), "r"(idesc), "r"(acc), "r"(sfa), "r"(sfb)
+        : "memory");
+}
+// Shared-memory descriptor of a 32-row x 16-byte block (four 8-row core matrices, 128 bytes
+// apart), no swizzle: the source of a 32x128b copy into tensor memory.
+__device__ __forceinline__ uint64_t sf_desc(uint32_t addr) {
+    uint64_t d = 0;
+    d |= (uint64_t)((addr & 0x3FFFFu) >> 4);
+    d |= (uint64_t)(128 >> 4) << 32;
+    d |= (uint64_t)1 << 46;
+    return d;
+}
+// Copy 32 rows x 128 bits of shared memory into tensor-memory columns taddr .. taddr + 3 of
+// lanes 0-31, repeated in the other three lane quarters (asynchronous; ordered before the MMAs
+// this thread issues after it).
+__device__ __forceinline__ void tmem_cp_sf(uint32_t taddr, uint64_t sdesc) {
+    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+// Bulk copy of `bytes` (a multiple of 16, both addresses 16-byte aligned) global -> shared,
+// completing on the mbarrier's transaction count.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+                 "l"(src), "r"(bytes), "r"(bar)
+                 : "memory");
+}
+
 __device__ __forceinline__ void mma_commit(uint32_t bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
 }
@@ -660,9 +720,19 @@ __device__ __forceinline__ void warp_store_chunk_bf16(uint32_t stage, const uint
 // e4m3 routed tile (Q8) the accumulators are first multiplied by the row's activation scale
 // and the column's weight scale.  Rows are stored through the per-warp transpose (all lanes
 // take part; rows past the group's end pass a null row).
+// Overlapping accumulators (mxw): the warp that holds the columns both accumulators share
+// reports them drained (their tensor-memory loads complete) so the next tile's MMAs may start.
+__device__ __forceinline__ void release_shared_cols(uint32_t ovl, int lane) {
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(ovl);
+}
+
+// ovl (mxw): 0, or the barrier this warp releases after loading the shared chunk, which it then
+// loads first (ovl_last: the shared chunk is the last of this warp's chunks).
 template <bool Q8 = false>
 __device__ __forceinline__ void epilogue_gemm1(const Params& p, const Tile& x, uint32_t tacc, int row, int half,
-                                               uint32_t stage, int lane) {
+                                               uint32_t stage, int lane, uint32_t ovl = 0, bool ovl_last = false) {
     const bool shared = x.g >= p.E;
     const int e = shared ? x.g - p.E : x.g;
     const int I = shared ? p.Is : p.I;
@@ -671,8 +741,8 @@ __device__ __forceinline__ void epilogue_gemm1(const Params& p, const Tile& x, u
     if (b1) b1 += (size_t)e * I;
     if (b3) b3 += (size_t)e * I;
     const bool scaled = Q8 && !shared;          // e4m3 routed tile
-    const float* sc1 = scaled ? p.ws1 + (size_t)e * I : nullptr;
-    const float* sc3 = scaled ? p.ws3 + (size_t)e * I : nullptr;
+    const float* sc1 = (scaled && !p.mxw) ? p.ws1 + (size_t)e * I : nullptr;   // block-scaled: in the MMA
+    const float* sc3 = (scaled && !p.mxw) ? p.ws3 + (size_t)e * I : nullptr;
     const int r = x.m0 + row;
     const bool live = r < x.rows;
     const float rs = (scaled && live) ? p.a_scale[x.row0 + r] : 1.f;
@@ -681,11 +751,13 @@ __device__ __forceinline__ void epilogue_gemm1(const Params& p, const Tile& x, u
     __nv_bfloat16* arow = (live && p.a_out) ? (shared ? p.as_out : p.a_out) + ro : nullptr;
     __nv_bfloat16* grow = (live && p.a_out) ? (shared ? p.gs_out : p.g_out) + ro : nullptr;
 #pragma unroll 1
-    for (int c = half * 2; c < half * 2 + 2; ++c) {
+    for (int it = 0; it < 2; ++it) {
+        const int c = half * 2 + (ovl_last ? 1 - it : it);
         uint32_t u[32], v[32];
         tmem_ld32(tacc + c * 32, u);
         tmem_ld32(tacc + 128 + c * 32, v);
         tmem_wait_ld();
+        if (ovl && it == 0) release_shared_cols(ovl, lane);
         const int col0 = x.n0 + c * 32;
         if (col0 >= I) continue;                                // warp-uniform
         const int ncols = min(32, I - col0);
@@ -699,7 +771,10 @@ __device__ __forceinline__ void epilogue_gemm1(const Params& p, const Tile& x, u
                 const int cc = min(col0 + j, I - 1);
                 float a = __uint_as_float(u[j]);
                 float g = __uint_as_float(v[j]);
-                if (scaled) { a *= rs * sc1[cc]; g *= rs * sc3[cc]; }
+                if (scaled) {
+                    a *= rs * (sc1 ? sc1[cc] : 1.f);
+                    g *= rs * (sc3 ? sc3[cc] : 1.f);
+                }
                 a += b1 ? __bfloat162float(b1[cc]) : 0.f;
                 g += b3 ? __bfloat162float(b3[cc]) : 0.f;
                 hv[h] = silu_f32(a) * g;
@@ -723,20 +798,22 @@ __device__ __forceinline__ void epilogue_gemm1(const Params& p, const Tile& x, u
 // b2 and the gate.  Rows are stored through the per-warp transpose.
 template <bool Q8 = false>
 __device__ __forceinline__ void epilogue_gemm2r(const Params& p, const Tile& x, uint32_t tacc, int row, int half,
-                                                uint32_t stage, int lane) {
+                                                uint32_t stage, int lane, uint32_t ovl = 0, bool ovl_last = false) {
     const int r = x.m0 + row;
     const bool live = r < x.rows;
     const long long pos = x.row0 + r;
     const float gate = live ? (p.sorted_gate ? p.sorted_gate[pos] : 1.f) : 0.f;
     const __nv_bfloat16* b2 = p.b2 ? p.b2 + (size_t)x.g * p.d : nullptr;
-    const float* sc2 = Q8 ? p.ws2 + (size_t)x.g * p.d : nullptr;
+    const float* sc2 = (Q8 && !p.mxw) ? p.ws2 + (size_t)x.g * p.d : nullptr;   // block-scaled: in the MMA
     const float rs = (Q8 && live) ? p.a_scale[pos] : 1.f;
     __nv_bfloat16* yrow = live ? p.y + (size_t)pos * p.d : nullptr;
 #pragma unroll 1
-    for (int c = half * 4; c < half * 4 + 4; ++c) {
+    for (int it = 0; it < 4; ++it) {
+        const int c = half * 4 + (ovl_last ? (it + 3) % 4 : it);
         uint32_t u[32];
         tmem_ld32(tacc + c * 32, u);
         tmem_wait_ld();
+        if (ovl && it == 0) release_shared_cols(ovl, lane);
         const int col0 = x.n0 + c * 32;
         if (col0 >= p.d) continue;                              // warp-uniform
         const int ncols = min(32, p.d - col0);
@@ -746,7 +823,10 @@ __device__ __forceinline__ void epilogue_gemm2r(const Params& p, const Tile& x, 
             const int ca = min(col0 + 2 * i, p.d - 1), cb = min(col0 + 2 * i + 1, p.d - 1);
             float a = __uint_as_float(u[2 * i]);
             float b = __uint_as_float(u[2 * i + 1]);
-            if (Q8) { a *= rs * sc2[ca]; b *= rs * sc2[cb]; }
+            if (Q8) {
+                a *= rs * (sc2 ? sc2[ca] : 1.f);
+                b *= rs * (sc2 ? sc2[cb] : 1.f);
+            }
             a += b2 ? __bfloat162float(b2[ca]) : 0.f;
             b += b2 ? __bfloat162float(b2[cb]) : 0.f;
             pk[i] = pack_bf16(gate * a, gate * b);
@@ -756,15 +836,18 @@ __device__ __forceinline__ void epilogue_gemm2r(const Params& p, const Tile& x, 
 }
 
 // GEMM2S: the shared experts' output (accumulator + their b2 summed), fp32, for the combine.
-__device__ __forceinline__ void epilogue_gemm2s(const Params& p, const Tile& x, uint32_t tacc, int row, int half) {
+__device__ __forceinline__ void epilogue_gemm2s(const Params& p, const Tile& x, uint32_t tacc, int row, int half,
+                                                uint32_t ovl = 0, int lane = 0, bool ovl_last = false) {
     const int t = x.m0 + row;
     const bool live = t < p.T;
     float* srow = p.sout + (size_t)t * p.d;
 #pragma unroll 1
-    for (int c = half * 4; c < half * 4 + 4; ++c) {
+    for (int it = 0; it < 4; ++it) {
+        const int c = half * 4 + (ovl_last ? (it + 3) % 4 : it);
         uint32_t u[32];
         tmem_ld32(tacc + c * 32, u);
         tmem_wait_ld();
+        if (ovl && it == 0) release_shared_cols(ovl, lane);
         const int col0 = x.n0 + c * 32;
         if (!live || col0 >= p.d) continue;
 #pragma unroll
@@ -1057,8 +1140,17 @@ __global__ void __launch_bounds__(THREADS, 1) moe_tc_kernel(const __grid_constan
     auto tfull_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + a); };
     auto tempty_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + 2 + a); };
     const uint32_t drain_bar = bar0 + 8u * (2 * STAGES + 4);
-    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(gbase + RING_BYTES + 8 * (2 * STAGES + 5));
+    auto ovl_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + 5 + a); };   // mxw: shared columns drained
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(gbase + RING_BYTES + 8 * (2 * STAGES + 7));
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+    static_assert(8 * (2 * STAGES + 7) + 8 <= 256, "barrier area");
+    static_assert(!Q8 || PAIR || STAGES <= 4, "scale-byte ring sized for 4 stages");
+    // mxw: the stages' B scale bytes and the constant A scale block, after the epilogue buffers
+    const uint32_t sf_base = bar0 + 256 + EPI_WARPS * STAGE_OUT_BYTES;
+    auto sfb_stage = [&](int s) { return sf_base + (uint32_t)(s * SF_STAGE_BYTES); };
+    const uint32_t sfa_buf = sf_base + 4 * SF_STAGE_BYTES;
+    const bool mxw = Q8 && !PAIR && p.mxw;
+    const uint32_t acc_cols = mxw ? (uint32_t)(ACC_COLS - MX_OVL) : (uint32_t)ACC_COLS;   // second accumulator's start
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     const uint32_t rank = PAIR ? cluster_rank() : 0u;        // 0 = leader of the pair
@@ -1070,6 +1162,7 @@ __global__ void __launch_bounds__(THREADS, 1) moe_tc_kernel(const __grid_constan
         for (int a = 0; a < 2; ++a) {
             mbar_init(tfull_bar(a), 1);
             mbar_init(tempty_bar(a), PAIR ? 2 * EPI_WARPS : EPI_WARPS);
+            mbar_init(ovl_bar(a), EPI_WARPS / 2);
         }
         mbar_init(drain_bar, 1);
         *abort_flag = 0;
@@ -1219,7 +1312,18 @@ __global__ void __launch_bounds__(THREADS, 1) moe_tc_kernel(const __grid_constan
                             }
                         }
                     } else {
-                        mbar_expect_tx(fb, A_BYTES + B_BYTES);
+                        // block-scaled e4m3 tile: the stage's 1 KB of B scale bytes come along
+                        const bool sf_tile = mxw && (MODE == GEMM1 ? x.g < p.E : (MODE == GEMM2R && x.g >= 0));
+                        mbar_expect_tx(fb, A_BYTES + B_BYTES + (sf_tile ? SF_STAGE_BYTES : 0));
+                        if (sf_tile) {
+                            const uint8_t* src =
+                                MODE == GEMM1
+                                    ? p.sf13 + (((size_t)x.g * ceil_div(p.I, 128) + x.n0 / 128) * ceil_div(p.d, 128) + kb) *
+                                                   SF_STAGE_BYTES
+                                    : p.sf2 + (((size_t)x.g * ceil_div(p.d, 256) + x.n0 / 256) * ceil_div(p.I, 128) + kb) *
+                                                  SF_STAGE_BYTES;
+                            bulk_load(sfb_stage(stage), src, SF_STAGE_BYTES, fb);
+                        }
                         if (MODE == GEMM1) {
                             const bool shared = x.g >= p.E;
                             const int e = shared ? x.g - p.E : x.g;
@@ -1266,6 +1370,14 @@ __global__ void __launch_bounds__(THREADS, 1) moe_tc_kernel(const __grid_constan
         // ------------------------------------------------------------------ MMA issuer
         if (lane == 0 && leader) {
             const uint32_t idesc = PAIR ? idesc_bf16_pair(p.n_mma) : idesc_bf16(p.n_mma);
+            if (mxw) {
+                // A-side scales: byte 127 (2^0) for every row and run, copied into TMEM once
+                for (int i = 0; i < SFA_BYTES / 16; ++i)
+                    asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(sfa_buf + 16u * i), "r"(0x7F7F7F7Fu)
+                                 : "memory");
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                tmem_cp_sf(tmem_base + SFA_COL, sf_desc(sfa_buf));
+            }
             int stage = 0;
             uint32_t phase = 0;
             int acc = 0;
@@ -1282,18 +1394,29 @@ __global__ void __launch_bounds__(THREADS, 1) moe_tc_kernel(const __grid_constan
                                        : narrow ? idesc_bf16(64) | IDESC_B_MN | IDESC_A_MN
                                                 : idesc | (B_MN ? IDESC_B_MN : 0u) | (A_MN ? IDESC_A_MN : 0u);
                 if (!mbar_wait(tempty_bar(acc), acc_phase ^ 1u, abort_flag, p.err)) break;
+                // mxw: the previous tile (other accumulator) has drained the columns both share
+                if (mxw && !mbar_wait(ovl_bar(acc ^ 1), acc ? acc_phase : acc_phase ^ 1u, abort_flag, p.err)) break;
                 tc_fence_after();
-                const uint32_t d_tmem = tmem_base + (uint32_t)(acc * ACC_COLS);
+                const uint32_t d_tmem = tmem_base + (uint32_t)acc * acc_cols;
+                const bool sf_tile = mxw && q8tile;
                 for (int kb = 0; kb < x.num_kb; ++kb) {
                     if (!mbar_wait(full_bar(stage), phase, abort_flag, p.err)) { ok = false; break; }
                     tc_fence_after();
                     const uint32_t a_addr = sA + stage * A_BYTES, b_addr = sB + stage * B_BYTES;
+                    if (sf_tile) {
+                        // this stage's B scales: B rows 0-127 -> columns SFB_COL..+3, rows 128-255 -> +4..+7
+                        tmem_cp_sf(tmem_base + SFB_COL, sf_desc(sfb_stage(stage)));
+                        tmem_cp_sf(tmem_base + SFB_COL + 4, sf_desc(sfb_stage(stage) + 512));
+                    }
 #pragma unroll
                     for (int k = 0; k < BK / 16; ++k) {
                         const uint64_t ad = A_MN ? mn_sw128_desc(a_addr + k * 2048) : sw128_desc(a_addr + k * 32);
                         const uint64_t bd = B_MN ? mn_sw128_desc(b_addr + k * 2048) : sw128_desc(b_addr + k * 32);
                         const uint32_t accum = (kb > 0 || k > 0) ? 1u : 0u;
-                        if (PAIR && q8tile) mma_e4m3_pair(d_tmem, ad, bd, idesc_t, accum);
+                        if (sf_tile)   // run k of the stage's four runs of 32: scale byte k
+                            mma_mx(d_tmem, ad, bd, idesc_mx(p.n_mma, k), tmem_base + SFA_COL + ((uint32_t)k << 30),
+                                   tmem_base + SFB_COL + ((uint32_t)k << 30), accum);
+                        else if (PAIR && q8tile) mma_e4m3_pair(d_tmem, ad, bd, idesc_t, accum);
                         else if (PAIR) mma_bf16_pair(d_tmem, ad, bd, idesc_t, accum);
                         else if (q8tile) mma_e4m3(d_tmem, ad, bd, idesc_t, accum);
                         else mma_bf16(d_tmem, ad, bd, idesc_t, accum);
@@ -1326,16 +1449,20 @@ __global__ void __launch_bounds__(THREADS, 1) moe_tc_kernel(const __grid_constan
             if (MODE == DW && p.dw_zero && x.num_kb == 0) continue;          // written by the producer
             if (!mbar_wait(tfull_bar(acc), acc_phase, abort_flag, p.err)) break;
             tc_fence_after();
-            const uint32_t tacc = tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(acc * ACC_COLS);
+            const uint32_t tacc = tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)acc * acc_cols;
+            // mxw: accumulator 0 shares its last chunk (half 1's), accumulator 1 its first (half 0's)
+            const bool ovl_owner = mxw && half == (acc == 0 ? 1 : 0);
+            const uint32_t ovl = ovl_owner ? ovl_bar(acc) : 0u;
+            const bool ovl_last = ovl_owner && acc == 0;
             if (MODE == ROUTER) {
                 if (half == 0) epilogue_router<KMAX>(p, x, tacc, row);
             } else if (MODE == ROUTERP) {
                 epilogue_router_partial(p, x, tacc, row, half);
             } else if (MODE == GEMM1) {
-                epilogue_gemm1<Q8>(p, x, tacc, row, half, stage_out, lane);
+                epilogue_gemm1<Q8>(p, x, tacc, row, half, stage_out, lane, ovl, ovl_last);
             } else if (MODE == GEMM2R) {
-                if (x.g >= 0) epilogue_gemm2r<Q8>(p, x, tacc, row, half, stage_out, lane);
-                else epilogue_gemm2s(p, x, tacc, row, half);
+                if (x.g >= 0) epilogue_gemm2r<Q8>(p, x, tacc, row, half, stage_out, lane, ovl, ovl_last);
+                else epilogue_gemm2s(p, x, tacc, row, half, ovl, lane, ovl_last);
             } else if (MODE == DH) {
                 epilogue_dh(p, x, tacc, row, half, stage_out, lane);
             } else if (MODE == DX) {
@@ -1513,7 +1640,7 @@ bool make_map_u8(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t mid, 
 template <int MODE, int KMAX, bool PAIR = false, bool Q8 = false>
 cudaError_t launch(const Params& p, int tiles, cudaStream_t stream) {
     auto kern = moe_tc_kernel<MODE, KMAX, PAIR, Q8>;
-    constexpr int smem = MODE == DW ? SMEM_BYTES_DW : SMEM_BYTES;
+    constexpr int smem = MODE == DW ? SMEM_BYTES_DW : (Q8 && !PAIR) ? SMEM_BYTES_Q8 : SMEM_BYTES;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
@@ -1722,11 +1849,14 @@ cudaError_t launch_tc_gemm1_q8(const Dims& D, const void* x, const void* x8_perm
                                cudaStream_t stream) {
     using namespace tc;
     if (D.T == 0) return cudaSuccess;
-    if (!R.s1 || !R.s3 || !xs) return cudaErrorInvalidValue;
+    if ((D.mx ? !R.sf13 : (!R.s1 || !R.s3)) || !xs) return cudaErrorInvalidValue;
     Params p = base_params(D, err);
     p.q8 = 1;
     p.a_scale = xs;
     p.ws1 = R.s1; p.ws3 = R.s3;
+    p.mxw = D.mx ? 1 : 0;
+    p.sf13 = R.sf13;
+    const bool pairs = tc::pairs_for(D) && !D.mx;          // block scales run on single CTAs
     p.tile_start = tile_start1;
     p.offsets = offsets;
     p.g_begin = 0;
@@ -1743,13 +1873,13 @@ cudaError_t launch_tc_gemm1_q8(const Dims& D, const void* x, const void* x8_perm
         ok &= make_map(&p.tmB[3], Sh.w3, D.d, D.Is, D.Ks, BK, 128, true);
     }
     if (!ok) return cudaErrorInvalidValue;
-    if (!tc::pairs_for(D)) {
+    if (!pairs) {
         CUtensorMap w;
         if (make_map_w13(&w, R.w1, R.w3, D.d, D.I, D.E, 2 * BK, true)) { p.tmB[0] = w; p.w13_one |= 1; }
         if (g_end > D.E && make_map_w13(&w, Sh.w1, Sh.w3, D.d, D.Is, D.Ks, BK, false)) { p.tmB[2] = w; p.w13_one |= 2; }
     }
-    return tc::pairs_for(D) ? launch<GEMM1, 8, true, true>(p, num_sms(), stream)
-                            : launch<GEMM1, 8, false, true>(p, num_sms(), stream);
+    return pairs ? launch<GEMM1, 8, true, true>(p, num_sms(), stream)
+                 : launch<GEMM1, 8, false, true>(p, num_sms(), stream);
 }
 
 // e4m3 routed GEMM2 over h8 (e4m3 rows, scale per row in hs) and the e4m3 W2 codes; with Sh the
@@ -1760,17 +1890,19 @@ cudaError_t launch_tc_gemm2_routed_q8(const Dims& D, const int32_t* offsets, con
                                       float* sout, uint32_t* err, cudaStream_t stream) {
     using namespace tc;
     if (D.T == 0) return cudaSuccess;
-    if (!R.s2 || !hs) return cudaErrorInvalidValue;
+    if ((D.mx ? !R.sf2 : !R.s2) || !hs) return cudaErrorInvalidValue;
     Params p = base_params(D, err);
     p.q8 = 1;
     p.a_scale = hs;
     p.ws2 = R.s2;
+    p.mxw = D.mx ? 1 : 0;
+    p.sf2 = R.sf2;
     p.tile_start = tile_start2;
     p.offsets = offsets;
     p.sorted_gate = sorted_gate;
     p.b2 = (const __nv_bfloat16*)R.b2;
     p.y = (__nv_bfloat16*)y_sorted;
-    const bool pairs = tc::pairs_for(D);
+    const bool pairs = tc::pairs_for(D) && !D.mx;          // block scales run on single CTAs
     bool ok = make_map_u8(&p.tmA[0], h8, D.I, (uint64_t)D.slots(), 1, 2 * BK, BM, false);
     ok &= make_map_u8(&p.tmB[0], R.w2, D.I, D.d, D.E, 2 * BK, pairs ? 128 : 256, true);
     if (Sh && D.Ks > 0 && sout) {

@@ -15,7 +15,8 @@ struct Dims {
     bool bias;
     bool bf16;
     int gate_mode = 0;     // moe_gate_mode_t
-    bool q8 = false;       // routed experts in e4m3 (moe_expert_fmt_t MOE_FMT_E4M3)
+    bool q8 = false;       // routed experts in e4m3 (MOE_FMT_E4M3, or MOE_FMT_MXFP8 with mx)
+    bool mx = false;       // q8 with block-scaled weights (MOE_FMT_MXFP8)
     long long slots() const { return (long long)T * k; }
 };
 
@@ -63,6 +64,12 @@ cudaError_t launch_scatter_rows(const Dims& D, const void* x, const int32_t* slo
 // when row_of is NULL, r checked against src_rows), scale[p] = max|src[r]| / 448 (1 for a zero
 // row), dst[p, :] = e4m3 round-to-nearest-even (saturating) of src[r, :] / scale[p], the
 // division in IEEE fp32.  width % 8 == 0.
+// Block-scaled e4m3 weights (MOE_FMT_MXFP8): kind 0 = W1 / W3 ([E][rows = I][K = d]; which = 0 for W1,
+// 1 for W3; both share one scale array), kind 1 = W2 ([E][rows = d][K = I]).  codes [E][rows][K];
+// sf in the tiled order the GEMM stages load (mx_scale_bytes bytes, pre-filled with 127 by the caller).
+size_t mx_scale_bytes(int kind, long long n_experts, int rows, int K);
+cudaError_t launch_quant_weights_mx(int kind, const void* w, int which, int n_experts, int rows, int K, uint8_t* codes,
+                                    uint8_t* sf, cudaStream_t stream);
 cudaError_t launch_quant_rows(const void* src, const int32_t* row_of, long long n_rows, int src_rows, int width,
                               uint8_t* dst, float* scale, uint32_t* err, cudaStream_t stream);
 // dst[p, :] = src[row_of[p], :] for rows of row_bytes (a multiple of 4) bytes; bad index -> bit 4, zeros
@@ -105,6 +112,7 @@ cudaError_t launch_combine(const Dims& D, const void* y_sorted, const int32_t* s
 struct FfnWeights {
     const void *w1, *b1, *w3, *b3, *w2, *b2;
     const float *s1 = nullptr, *s3 = nullptr, *s2 = nullptr;   // e4m3 codes: per-output-channel scales
+    const uint8_t *sf13 = nullptr, *sf2 = nullptr;              // block-scaled codes: tiled scale bytes
 };
 
 // h rows of groups [g_begin, g_end): routed group e -> h_r[offsets[e] + r], shared group

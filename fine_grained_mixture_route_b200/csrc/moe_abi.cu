@@ -131,14 +131,16 @@ moe_status_t to_dims(const moe_shape_t* s, Dims* D) {
     if (s->dtype == MOE_BF16) {
         if (s->d % 8 || s->inter % 8 || (s->n_shared > 0 && s->inter_shared % 8)) return MOE_ERR_UNSUPPORTED;
     }
-    if (s->routed_fmt != MOE_FMT_NATIVE && s->routed_fmt != MOE_FMT_E4M3) return MOE_ERR_INVALID_ARG;
-    if (s->routed_fmt == MOE_FMT_E4M3 && (s->dtype != MOE_BF16 || s->d % 16 || s->inter % 16))
+    if (s->routed_fmt != MOE_FMT_NATIVE && s->routed_fmt != MOE_FMT_E4M3 && s->routed_fmt != MOE_FMT_MXFP8)
+        return MOE_ERR_INVALID_ARG;
+    if (s->routed_fmt != MOE_FMT_NATIVE && (s->dtype != MOE_BF16 || s->d % 16 || s->inter % 16))
         return MOE_ERR_UNSUPPORTED;
     D->T = s->T; D->d = s->d; D->E = s->n_experts; D->I = s->inter; D->k = s->top_k;
     D->Ks = s->n_shared; D->Is = s->n_shared > 0 ? s->inter_shared : 0;
     D->bias = s->has_bias != 0; D->bf16 = s->dtype == MOE_BF16;
     D->gate_mode = s->gate_mode;
-    D->q8 = s->routed_fmt == MOE_FMT_E4M3;
+    D->q8 = s->routed_fmt != MOE_FMT_NATIVE;
+    D->mx = s->routed_fmt == MOE_FMT_MXFP8;
     return MOE_OK;
 }
 
@@ -147,16 +149,20 @@ moe_status_t check_ws(const Dims& D, void* ws, size_t ws_bytes) {
     return MOE_OK;
 }
 
-// e4m3: the stack must carry its three scale arrays (routed experts of an MOE_FMT_E4M3
-// layer); otherwise all three must be NULL.
-moe_status_t check_weights(const Dims& D, const moe_ffn_weights_t* w, bool e4m3 = false) {
+// The scale arrays a stack carries follow its format: the routed experts of an MOE_FMT_E4M3
+// layer carry s1, s3, s2 (and no scale bytes), those of an MOE_FMT_MXFP8 layer sf13 and sf2 (and
+// no per-channel scales); every other stack (native routed experts, shared experts) carries none.
+moe_status_t check_weights(const Dims& D, const moe_ffn_weights_t* w, bool routed = false) {
     if (!w || !w->w1 || !w->w3 || !w->w2) return MOE_ERR_INVALID_ARG;
     const bool b = w->b1 && w->b3 && w->b2;
     const bool none = !w->b1 && !w->b3 && !w->b2;
     if (D.bias ? !b : !none) return MOE_ERR_INVALID_ARG;
-    const bool sc = w->s1 && w->s3 && w->s2;
-    const bool nosc = !w->s1 && !w->s3 && !w->s2;
+    const bool sc = w->s1 && w->s3 && w->s2, nosc = !w->s1 && !w->s3 && !w->s2;
+    const bool sf = w->sf13 && w->sf2, nosf = !w->sf13 && !w->sf2;
+    const bool e4m3 = routed && D.q8 && !D.mx, mx = routed && D.mx;
     if (e4m3 ? !sc : !nosc) return MOE_ERR_INVALID_ARG;
+    if (mx ? !sf : !nosf) return MOE_ERR_INVALID_ARG;
+    if (mx && (((uintptr_t)w->sf13 | (uintptr_t)w->sf2) & 15u)) return MOE_ERR_INVALID_ARG;
     return MOE_OK;
 }
 
@@ -196,6 +202,7 @@ FfnWeights to_ffn(const moe_ffn_weights_t* w) {
     if (w) {
         f.w1 = w->w1; f.b1 = w->b1; f.w3 = w->w3; f.b3 = w->b3; f.w2 = w->w2; f.b2 = w->b2;
         f.s1 = w->s1; f.s3 = w->s3; f.s2 = w->s2;
+        f.sf13 = w->sf13; f.sf2 = w->sf2;
     }
     return f;
 }
@@ -360,7 +367,7 @@ MOE_EXPORT moe_status_t moe_expert_ffn(const moe_shape_t* shape, const void* x, 
     Dims D;
     MOE_TRY(to_dims(shape, &D));
     if (!offsets || (D.T > 0 && (!x || !sorted_token || !y_sorted))) return MOE_ERR_INVALID_ARG;
-    MOE_TRY(check_weights(D, routed, D.q8));
+    MOE_TRY(check_weights(D, routed, true));
     MOE_TRY(check_ws(D, ws, ws_bytes));
     if (D.T == 0) return MOE_OK;
     MOE_TRY(check_device());
@@ -426,6 +433,30 @@ MOE_EXPORT moe_status_t moe_quantize_rows_e4m3(const void* src, const int32_t* r
     return MOE_OK;
 }
 
+MOE_EXPORT size_t moe_mx_scale_bytes(int32_t kind, int32_t n_experts, int32_t rows, int32_t K) {
+    if ((kind != MOE_MX_UP && kind != MOE_MX_DOWN) || n_experts < 1 || rows < 1 || K < 1) return 0;
+    return mx_scale_bytes(kind, n_experts, rows, K);
+}
+
+MOE_EXPORT moe_status_t moe_quantize_weights_mx(int32_t kind, const void* w_a, const void* w_b, int32_t n_experts,
+                                                int32_t rows, int32_t K, uint8_t* codes_a, uint8_t* codes_b,
+                                                uint8_t* sf, moe_stream_t stream) {
+    if (kind != MOE_MX_UP && kind != MOE_MX_DOWN) return MOE_ERR_INVALID_ARG;
+    if (n_experts < 1 || rows < 1 || K < 1 || (long long)n_experts * rows >= (1LL << 31)) return MOE_ERR_INVALID_ARG;
+    if (!w_a || !codes_a || !sf) return MOE_ERR_INVALID_ARG;
+    if (kind == MOE_MX_UP ? (!w_b || !codes_b) : (w_b || codes_b)) return MOE_ERR_INVALID_ARG;
+    if (K % 16) return MOE_ERR_UNSUPPORTED;
+    const uintptr_t al = (uintptr_t)w_a | (uintptr_t)w_b | (uintptr_t)codes_a | (uintptr_t)codes_b | (uintptr_t)sf;
+    if (al & 15u) return MOE_ERR_INVALID_ARG;
+    MOE_TRY(check_device());
+    cudaGetLastError();
+    const cudaStream_t st = (cudaStream_t)stream;
+    MOE_CUDA(cudaMemsetAsync(sf, 127, mx_scale_bytes(kind, n_experts, rows, K), st));
+    MOE_CUDA(launch_quant_weights_mx(kind, w_a, 0, n_experts, rows, K, codes_a, sf, st));
+    if (kind == MOE_MX_UP) MOE_CUDA(launch_quant_weights_mx(kind, w_b, 1, n_experts, rows, K, codes_b, sf, st));
+    return MOE_OK;
+}
+
 }  // extern "C"
 
 namespace moe {
@@ -441,7 +472,7 @@ moe_status_t layer_forward_impl(const moe_shape_t* shape, const void* x, const v
     Dims D;
     MOE_TRY(to_dims(shape, &D));
     if (!centroids || (D.T > 0 && (!x || !out))) return MOE_ERR_INVALID_ARG;
-    MOE_TRY(check_weights(D, routed, D.q8));
+    MOE_TRY(check_weights(D, routed, true));
     if (D.Ks > 0) MOE_TRY(check_weights(D, shared));
     else if (shared) return MOE_ERR_INVALID_ARG;
     MOE_TRY(check_ws(D, ws, ws_bytes));

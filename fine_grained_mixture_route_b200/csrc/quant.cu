@@ -269,6 +269,96 @@ cudaError_t launch_gather_rows_generic(const void* src, const int32_t* row_of, l
     return cudaGetLastError();
 }
 
+namespace {
+
+// ---- block-scaled e4m3 weights (MOE_FMT_MXFP8) ---------------------------------------
+// Each weight row (one output channel, K inputs) is cut into runs of 32 consecutive inputs; a
+// run's scale is 2^e with e the smallest integer such that max|run| <= 448 * 2^e (no element
+// saturates), 0 for an all-zero run, within [-127, 127]; the codes are e4m3(v * 2^-e), the
+// product exact (a power of two), rounded to nearest even.  The scale is stored as the byte
+// e + 127, in the tiled order the GEMMs' pipeline stages load (see mx_scale_offset).
+
+// e from the fp32 bits of the run maximum: amax in [2^e0, 2^(e0+1)) and 448 * 2^(e0-8) =
+// 1.75 * 2^e0, so e = e0 - 8 when the mantissa is at most 0.75 (0x600000), else e0 - 7.
+__device__ __forceinline__ int mx_exponent(float amax) {
+    const uint32_t b = __float_as_uint(amax);
+    if (b == 0u) return 0;
+    const int eb = (int)(b >> 23);
+    if (eb == 0) return -127;                              // below 2^-126: clamped
+    const int e = eb - 127 - 8 + ((b & 0x7FFFFFu) > 0x600000u ? 1 : 0);
+    return e < -127 ? -127 : (e > 127 ? 127 : e);
+}
+
+// 8 bf16 times a power of two -> 8 e4m3 codes (element j in byte j)
+__device__ __forceinline__ uint2 chunk_quant_mul(const uint4& v, float mul) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint32_t pk[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 f = make_float2(bf16_lo(w[i]) * mul, bf16_hi(w[i]) * mul);
+        pk[i] = (uint32_t)__nv_cvt_float2_to_fp8x2(f, __NV_SATFINITE, __NV_E4M3);
+    }
+    return make_uint2(pk[0] | (pk[1] << 16), pk[2] | (pk[3] << 16));
+}
+
+// Byte offset of the scale of run j of row r of expert e in the tiled layout: rows in groups of
+// P (128 for W1 / W3, 256 for W2), runs in chunks of 4 (one pipeline stage of 128 inputs); the
+// 1 KB block of (e, group, chunk) holds two 512-byte halves (W1 / W3: half = which matrix;
+// W2: half = (r / 128) % 2), and in a half row r's byte for run j sits at
+// (r % 32) * 16 + ((r / 32) % 4) * 4 + j % 4.
+__device__ __forceinline__ size_t mx_scale_offset(int e, int r, int j, int ngrp, int nch, int P, int which) {
+    const size_t blk = ((size_t)e * ngrp + r / P) * nch + j / 4;
+    const int half = P == 128 ? which : (r / 128) & 1;
+    return blk * 1024 + half * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4 + (j & 3);
+}
+
+// One warp per row; lane i of a pass holds 16-byte chunk i (8 elements), so lanes 4q..4q+3 hold
+// run q of the pass and two shuffles give its maximum.
+__global__ void __launch_bounds__(256) quant_weights_mx_kernel(const uint4* __restrict__ src, int E, int rows, int K,
+                                                               int P, int which, uint2* __restrict__ codes,
+                                                               uint8_t* __restrict__ sf) {
+    const int lane = threadIdx.x & 31;
+    const int nv = K / 8;
+    const int nch = (K + 127) / 128;
+    const int ngrp = (rows + P - 1) / P;
+    const long long n_rows = (long long)E * rows;
+    const long long warps = (long long)gridDim.x * (blockDim.x >> 5);
+    for (long long q = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); q < n_rows; q += warps) {
+        const int e = (int)(q / rows), r = (int)(q % rows);
+        const uint4* s = src + (size_t)q * nv;
+        uint2* dst = codes + (size_t)q * nv;
+        for (int base = 0; base < nv; base += 32) {
+            const int i = base + lane;
+            const uint4 v = i < nv ? s[i] : make_uint4(0u, 0u, 0u, 0u);
+            float m = chunk_amax(v, 0.f);
+            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
+            const int ex = mx_exponent(m);
+            const float mul = __uint_as_float((uint32_t)(127 - ex) << 23);   // 2^-ex (ex <= 126 for finite runs)
+            if (i < nv) dst[i] = chunk_quant_mul(v, mul);
+            if ((lane & 3) == 0 && i < nv) sf[mx_scale_offset(e, r, i >> 2, ngrp, nch, P, which)] = (uint8_t)(ex + 127);
+        }
+    }
+}
+
+}  // namespace
+
+size_t mx_scale_bytes(int kind, long long n_experts, int rows, int K) {
+    const int P = kind == 0 ? 128 : 256;
+    return (size_t)n_experts * ((rows + P - 1) / P) * ((K + 127) / 128) * 1024;
+}
+
+cudaError_t launch_quant_weights_mx(int kind, const void* w, int which, int n_experts, int rows, int K, uint8_t* codes,
+                                    uint8_t* sf, cudaStream_t stream) {
+    const long long n = (long long)n_experts * rows;
+    if (n == 0) return cudaSuccess;
+    const long long cap = 8LL * 8 * num_sms();
+    const int blocks = (int)((n + 7) / 8 < cap ? (n + 7) / 8 : cap);
+    quant_weights_mx_kernel<<<blocks, 256, 0, stream>>>((const uint4*)w, n_experts, rows, K, kind == 0 ? 128 : 256,
+                                                        which, (uint2*)codes, sf);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_quant_rows(const void* src, const int32_t* row_of, long long n_rows, int src_rows, int width,
                               uint8_t* dst, float* scale, uint32_t* err, cudaStream_t stream) {
     if (n_rows <= 0) return cudaSuccess;

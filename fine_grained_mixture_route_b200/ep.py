@@ -164,9 +164,11 @@ class ExpertParallelMoE:
         g_recv = torch.empty((R, 1), dtype=g_send.dtype, device=x.device)
         self._a2a(x_recv, x_send, r_split, s_split)
         self._a2a(g_recv, g_send, r_split, s_split)
-        # FP8 routed experts (e4m3 codes with their scales, quant.quantize_stack) run on the local
-        # expert call only; routing, exchange and combine do not touch the routed weights
-        fp8 = {"routed_fmt": 1} if self.routed["w1"].dtype == torch.uint8 else {}
+        # FP8 routed experts (e4m3 codes with per-row or block scales, quant.quantize_stack) run on
+        # the local expert call only; routing, exchange and combine do not touch the routed weights
+        fp8 = {}
+        if self.routed["w1"].dtype == torch.uint8:
+            fp8 = {"routed_fmt": 2 if self.routed.get("sf13") is not None else 1}
         shape_loc = be.shape(R, d, Eloc, I, 1, 0, 0, bias, x.dtype, 0, **fp8)
         if R > 0:
             # local experts on their rows, grouped by expert on the device, then back in received order

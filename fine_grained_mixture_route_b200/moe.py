@@ -17,14 +17,16 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe_b200
 MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_CUDA, MOE_ERR_INTERNAL = range(6)
 MOE_F32, MOE_BF16 = 0, 1
 GATE_SOFTMAX_TOPK, GATE_TOPK_SOFTMAX, GATE_SIGMOID_BIAS = 0, 1, 2
-FMT_NATIVE, FMT_E4M3 = 0, 1        # storage of the routed experts' weights (moe_expert_fmt_t)
+FMT_NATIVE, FMT_E4M3, FMT_MXFP8 = 0, 1, 2   # storage of the routed experts' weights (moe_expert_fmt_t)
+MX_UP, MX_DOWN = 0, 1                        # block-scaled weight stacks: w1 | w3, w2 (moe_mx_kind_t)
 
 EXPORTED = ("moe_workspace_bytes", "moe_layer_launches", "moe_status_string", "moe_version", "moe_check_device_error", "moe_ws_init",
             "moe_route", "moe_permute", "moe_expert_ffn", "moe_combine", "moe_layer_forward",
             "moe_layer_forward_timed", "moe_permute_no_alloc", "moe_quantize_rows_e4m3", "moe_train_ctx_bytes",
             "moe_backward_workspace_bytes", "moe_layer_forward_train", "moe_layer_backward",
             "moe_layer_backward_timed", "moe_backward_launches", "moe_balance_workspace_bytes",
-            "moe_balance_stats", "moe_gather_rows", "moe_segment_ids", "moe_selftest_wait_timeout")
+            "moe_balance_stats", "moe_gather_rows", "moe_segment_ids", "moe_selftest_wait_timeout",
+            "moe_mx_scale_bytes", "moe_quantize_weights_mx")
 NUM_STAGES = 7
 STAGE_NAMES = ("router", "permute", "plan", "gather", "gemm1_swiglu", "gemm2", "combine")
 BWD_STAGES = 7
@@ -38,7 +40,7 @@ class MoeShape(ctypes.Structure):
 
 
 class MoeWeights(ctypes.Structure):
-    _fields_ = [(n, ctypes.c_void_p) for n in ("w1", "b1", "w3", "b3", "w2", "b2", "s1", "s3", "s2")]
+    _fields_ = [(n, ctypes.c_void_p) for n in ("w1", "b1", "w3", "b3", "w2", "b2", "s1", "s3", "s2", "sf13", "sf2")]
 
 
 class MoeGrads(ctypes.Structure):
@@ -99,12 +101,16 @@ def _lib():
         lib.moe_gather_rows.argtypes = [vp, i32p, ctypes.c_int64, ctypes.c_int64, ctypes.c_int32, vp, vp, sz, vp]
         lib.moe_segment_ids.argtypes = [i32p, ctypes.c_int32, ctypes.c_int32, ctypes.c_int64, i32p, vp, sz, vp]
         lib.moe_selftest_wait_timeout.argtypes = [ctypes.c_uint64, vp, vp, sz, vp]
+        lib.moe_mx_scale_bytes.argtypes = [ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32]
+        lib.moe_mx_scale_bytes.restype = sz
+        lib.moe_quantize_weights_mx.argtypes = [ctypes.c_int32, vp, vp, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                                                vp, vp, vp, vp]
         lib.moe_backward_launches.argtypes = [sh]
         lib.moe_backward_launches.restype = ctypes.c_int32
         for n in ("moe_check_device_error", "moe_ws_init", "moe_route", "moe_permute", "moe_expert_ffn",
                   "moe_combine", "moe_layer_forward", "moe_layer_forward_timed", "moe_quantize_rows_e4m3",
                   "moe_layer_forward_train", "moe_layer_backward", "moe_layer_backward_timed", "moe_balance_stats",
-                  "moe_gather_rows", "moe_segment_ids", "moe_selftest_wait_timeout"):
+                  "moe_gather_rows", "moe_segment_ids", "moe_selftest_wait_timeout", "moe_quantize_weights_mx"):
             getattr(lib, n).restype = ctypes.c_int
         _LIB = lib
     return _LIB
@@ -142,7 +148,9 @@ def shape_of(x: torch.Tensor, centroids_or_E, routed: Dict, top_k: int, shared: 
     I = routed["w1"].shape[1]
     Ks = 0 if shared is None else shared["w1"].shape[0]
     Is = 0 if shared is None else shared["w1"].shape[1]
-    fmt = FMT_E4M3 if routed["w1"].dtype == torch.uint8 else FMT_NATIVE    # e4m3 codes (quant.quantize_stack)
+    fmt = FMT_NATIVE                                                         # codes from quant.quantize_stack:
+    if routed["w1"].dtype == torch.uint8:                                    # block scales (sf13) or per-row ones
+        fmt = FMT_MXFP8 if routed.get("sf13") is not None else FMT_E4M3
     return make_shape(x.shape[0], x.shape[1], E, I, top_k, Ks, Is, routed.get("b1") is not None, x.dtype, gate_mode,
                       fmt)
 
@@ -190,11 +198,13 @@ def _need_stack(w: Optional[Dict], name: str, shape: MoeShape, shared: bool, dev
     E = shape.n_shared if shared else shape.n_experts
     I = shape.inter_shared if shared else shape.inter
     d, dt = shape.d, _layer_dtype(shape)
-    codes = not shared and not grads and shape.routed_fmt == FMT_E4M3
+    codes = not shared and not grads and shape.routed_fmt in (FMT_E4M3, FMT_MXFP8)
     wdt = torch.uint8 if codes else dt
     for k, n, kdt in (("w1", E * I * d, wdt), ("w3", E * I * d, wdt), ("w2", E * d * I, wdt),
                       ("b1", E * I, dt), ("b3", E * I, dt), ("b2", E * d, dt),
-                      ("s1", E * I, torch.float32), ("s3", E * I, torch.float32), ("s2", E * d, torch.float32)):
+                      ("s1", E * I, torch.float32), ("s3", E * I, torch.float32), ("s2", E * d, torch.float32),
+                      ("sf13", mx_scale_bytes(MX_UP, E, I, d), torch.uint8),
+                      ("sf2", mx_scale_bytes(MX_DOWN, E, d, I), torch.uint8)):
         if k in w:
             _need(w[k], f"{name}.{k}", n, kdt, device)
 
@@ -210,15 +220,20 @@ def _bias_ptr(router_bias: Optional[torch.Tensor]):
 def _weights(w: Optional[Dict]):
     if w is None:
         return None
-    for k in ("w1", "w3", "w2", "b1", "b3", "b2", "s1", "s3", "s2"):
+    for k in ("w1", "w3", "w2", "b1", "b3", "b2", "s1", "s3", "s2", "sf13", "sf2"):
         t = w.get(k)
         if t is not None and not t.is_contiguous():
             raise ValueError(f"weight {k} must be contiguous")
     if w["w1"].dtype == torch.uint8:
-        for k in ("s1", "s3", "s2"):
-            if w.get(k) is None or w[k].dtype != torch.float32:
-                raise ValueError(f"e4m3 weights need float32 scales {k}")
-    names = ("w1", "b1", "w3", "b3", "w2", "b2", "s1", "s3", "s2")
+        if w.get("sf13") is not None:
+            for k in ("sf13", "sf2"):
+                if w.get(k) is None or w[k].dtype != torch.uint8:
+                    raise ValueError(f"block-scaled e4m3 weights need uint8 scale bytes {k}")
+        else:
+            for k in ("s1", "s3", "s2"):
+                if w.get(k) is None or w[k].dtype != torch.float32:
+                    raise ValueError(f"e4m3 weights need float32 scales {k}")
+    names = ("w1", "b1", "w3", "b3", "w2", "b2", "s1", "s3", "s2", "sf13", "sf2")
     return MoeWeights(*(None if w.get(k) is None else w[k].data_ptr() for k in names))
 
 
@@ -357,6 +372,45 @@ def quantize_rows_e4m3(src: torch.Tensor, ws: torch.Tensor, row_of: Optional[tor
                                          _ptr(scales), _ptr(ws), ws.numel(), _stream(stream)),
            "moe_quantize_rows_e4m3")
     return codes, scales
+
+
+def mx_scale_bytes(kind: int, n_experts: int, rows: int, K: int) -> int:
+    """Bytes of the tiled scale array of a block-scaled weight stack (moe_mx_scale_bytes)."""
+    return int(_lib().moe_mx_scale_bytes(kind, n_experts, rows, K))
+
+
+def quantize_weights_mx(kind: int, w_a: torch.Tensor, w_b: Optional[torch.Tensor] = None,
+                        codes_a: Optional[torch.Tensor] = None, codes_b: Optional[torch.Tensor] = None, stream=None):
+    """Block-scaled e4m3 conversion of bf16 weight stacks (moe_quantize_weights_mx).  MX_UP: w_a = w1, w_b = w3
+    [E, I, d]; MX_DOWN: w_a = w2 [E, d, I].  Returns (codes_a, codes_b or None, scale bytes [E, bytes / E]);
+    codes_a / codes_b may be given (uint8, same shape), e.g. the halves of one [2, E, I, d] buffer."""
+    if kind not in (MX_UP, MX_DOWN):
+        raise ValueError("kind must be MX_UP or MX_DOWN")
+    if (w_b is not None) != (kind == MX_UP):
+        raise ValueError("MX_UP takes w1 and w3, MX_DOWN only w2")
+    mats = [w_a] if w_b is None else [w_a, w_b]
+    for t in mats:
+        if t.dtype != torch.bfloat16 or t.dim() != 3 or not t.is_contiguous() or t.device.type != "cuda":
+            raise ValueError("weights must be contiguous bf16 [E, rows, K] stacks on a CUDA device")
+        if t.shape != w_a.shape or t.device != w_a.device:
+            raise ValueError("w1 and w3 must have the same shape and device")
+    E, rows, K = w_a.shape
+    outs = []
+    for t, c in zip(mats, (codes_a, codes_b)):
+        if c is None:
+            c = torch.empty(t.shape, dtype=torch.uint8, device=t.device)
+        _need(c, "codes", t.numel(), torch.uint8, t.device)
+        if c.shape != t.shape:
+            raise ValueError("codes must have the weights' shape")
+        outs.append(c)
+    nbytes = mx_scale_bytes(kind, E, rows, K)
+    if nbytes == 0:
+        raise ValueError("invalid weight stack shape")
+    sf = torch.empty((E, nbytes // E), dtype=torch.uint8, device=w_a.device)
+    _check(_lib().moe_quantize_weights_mx(kind, _ptr(w_a), _ptr(w_b), E, rows, K, _ptr(outs[0]),
+                                          _ptr(outs[1]) if len(outs) > 1 else None, _ptr(sf), _stream(stream)),
+           "moe_quantize_weights_mx")
+    return outs[0], (outs[1] if len(outs) > 1 else None), sf
 
 
 def train_ctx_bytes(shape: MoeShape) -> int:

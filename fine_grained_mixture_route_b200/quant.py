@@ -11,6 +11,10 @@ sensitive to quantisation error.
 The conversion runs once, offline, in the library's per-row quantiser (moe_quantize_rows_e4m3,
 the same kernel the FP8 layer uses for its activation rows): bf16 weights on the GPU in, codes
 and scales out.  There is no other implementation of the format's arithmetic here.
+
+The block-scaled variant (quantize_stack(..., fmt="mxfp8"), moe_quantize_weights_mx) keeps one
+power-of-two scale per run of 32 inputs of each row instead of one per row: the per-group option
+of the same §5.5 advice, in the form the sm_100a tensor cores apply inside the MMA.
 """
 from __future__ import annotations
 
@@ -40,10 +44,16 @@ def dequantize_rows(q: torch.Tensor, scale: torch.Tensor) -> torch.Tensor:
     return q.view(torch.float8_e4m3fn).float() * scale.unsqueeze(-1)
 
 
-def quantize_stack(stack: Dict[str, Optional[torch.Tensor]]) -> Dict[str, Optional[torch.Tensor]]:
+def quantize_stack(stack: Dict[str, Optional[torch.Tensor]], fmt: str = "e4m3") -> Dict[str, Optional[torch.Tensor]]:
     """Routed expert stack (bf16 on the GPU: w1, w3 [E, I, d]; w2 [E, d, I]; biases unchanged) ->
-    codes in w1/w3/w2 (uint8; w1 and w3 the two halves of one [2, E, I, d] buffer) and per-row
-    scales in s1, s3 [E, I] and s2 [E, d]."""
+    codes in w1/w3/w2 (uint8; w1 and w3 the two halves of one [2, E, I, d] buffer) and
+    fmt "e4m3": per-row scales in s1, s3 [E, I] and s2 [E, d];
+    fmt "mxfp8": block-scale bytes in sf13 (w1 and w3) and sf2 (w2), [E, bytes per expert] in the
+    tiled order of include/moe.h."""
+    if fmt == "mxfp8":
+        return _quantize_stack_mx(stack)
+    if fmt != "e4m3":
+        raise ValueError('fmt must be "e4m3" or "mxfp8"')
     out = dict(stack)
     ws = torch.zeros(256, dtype=torch.uint8, device=stack["w1"].device)
     codes13 = None
@@ -58,6 +68,19 @@ def quantize_stack(stack: Dict[str, Optional[torch.Tensor]]) -> Dict[str, Option
         else:
             out[w] = q
         out[sname] = sc
+    return out
+
+
+def _quantize_stack_mx(stack: Dict[str, Optional[torch.Tensor]]) -> Dict[str, Optional[torch.Tensor]]:
+    w1, w3, w2 = stack["w1"], stack["w3"], stack["w2"]
+    for w in (w1, w3, w2):
+        if w.dtype != torch.bfloat16 or w.device.type != "cuda":
+            raise ValueError("quantize_stack converts bf16 weights on a CUDA device")
+    codes13 = torch.empty((2,) + tuple(w1.shape), dtype=torch.uint8, device=w1.device)
+    _, _, sf13 = moe.quantize_weights_mx(moe.MX_UP, w1.contiguous(), w3.contiguous(), codes13[0], codes13[1])
+    c2, _, sf2 = moe.quantize_weights_mx(moe.MX_DOWN, w2.contiguous())
+    out = {k: v for k, v in stack.items() if k not in ("s1", "s3", "s2")}
+    out.update(w1=codes13[0], w3=codes13[1], w2=c2, sf13=sf13, sf2=sf2)
     return out
 
 

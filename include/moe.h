@@ -50,6 +50,17 @@
  *    and every output keep shape->dtype.  The pages name FP8 for fine-grained MoE and for
  *    DeepSeek-V3 ("DeepSeek MoE模型优化与未来演进及字节超稀疏内存技术" and the report's §6.2)
  *    without a recipe; this recipe is the library's own.
+ *  - Block-scaled FP8 routed experts (shape->routed_fmt == MOE_FMT_MXFP8; same shape rules as
+ *    MOE_FMT_E4M3): w1, w3, w2 hold e4m3 codes as above, but each weight row carries one
+ *    power-of-two scale per run of 32 consecutive inputs instead of one per row: the scale of a
+ *    run is 2^e with e the smallest integer such that max|run| <= 448 * 2^e (0 for an all-zero
+ *    run, within [-127, 127]), stored as the byte e + 127 in sf13 (w1 and w3) and sf2 (w2), in
+ *    the tiled order moe_quantize_weights_mx writes.  The tensor cores apply these scales inside
+ *    the MMA (kind::mxf8f6f4 with block scales); activations are quantised per row as for
+ *    MOE_FMT_E4M3.  The DeepSeek-V2 explainer (§5.5) advises per-channel or per-group scales
+ *    for quantised routed experts, with the shared experts left in 16-bit, as here; it fixes
+ *    no group size or scale type.  Groups of 32 with power-of-two scales are what the sm_100a
+ *    tensor cores apply natively.
  */
 #ifndef MOE_B200_H
 #define MOE_B200_H
@@ -88,8 +99,9 @@ typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype_t;
 typedef enum { MOE_GATE_SOFTMAX_TOPK = 0, MOE_GATE_TOPK_SOFTMAX = 1, MOE_GATE_SIGMOID_BIAS = 2 } moe_gate_mode_t;
 
 /* Storage of the routed experts' weight matrices: MOE_FMT_NATIVE = shape->dtype,
- * MOE_FMT_E4M3 = e4m3 codes with per-output-channel fp32 scales (see above). */
-typedef enum { MOE_FMT_NATIVE = 0, MOE_FMT_E4M3 = 1 } moe_expert_fmt_t;
+ * MOE_FMT_E4M3 = e4m3 codes with per-output-channel fp32 scales, MOE_FMT_MXFP8 = e4m3 codes
+ * with a power-of-two scale per run of 32 inputs (see above). */
+typedef enum { MOE_FMT_NATIVE = 0, MOE_FMT_E4M3 = 1, MOE_FMT_MXFP8 = 2 } moe_expert_fmt_t;
 
 typedef struct {
     int32_t T;            /* tokens */
@@ -119,6 +131,9 @@ typedef struct {
     const float* s1; /* MOE_FMT_E4M3 routed experts: [E, I] scales of w1's rows; NULL otherwise */
     const float* s3; /* MOE_FMT_E4M3: [E, I] scales of w3's rows; NULL otherwise */
     const float* s2; /* MOE_FMT_E4M3: [E, d] scales of w2's rows; NULL otherwise */
+    const uint8_t* sf13; /* MOE_FMT_MXFP8 routed experts: scale bytes of w1 and w3 (moe_quantize_weights_mx,
+                            MOE_MX_UP, moe_mx_scale_bytes bytes); NULL otherwise */
+    const uint8_t* sf2;  /* MOE_FMT_MXFP8: scale bytes of w2 (MOE_MX_DOWN); NULL otherwise */
 } moe_ffn_weights_t;
 
 /* Bytes of workspace every entry point needs for this shape (0 if the shape is invalid). */
@@ -253,6 +268,32 @@ moe_status_t moe_layer_forward_timed(const moe_shape_t* shape, const void* x, co
 moe_status_t moe_quantize_rows_e4m3(const void* src, const int32_t* row_of, int64_t n_rows, int32_t src_rows,
                                     int32_t width, uint8_t* dst, float* scale, void* ws, size_t ws_bytes,
                                     moe_stream_t stream);
+
+/*
+ * Block-scaled FP8 weights (MOE_FMT_MXFP8): converts a stack of bf16 weight matrices, once,
+ * into e4m3 codes and the tiled scale bytes the layer reads.
+ *   MOE_MX_UP:   w_a = w1, w_b = w3, each [E, rows = inter, K = d] bf16; codes_a / codes_b
+ *                [E, inter, d] uint8 out (for one request per pipeline stage, the two halves of one
+ *                [2, E, inter, d] buffer); sf out, shared by w1 and w3.
+ *   MOE_MX_DOWN: w_a = w2 [E, rows = d, K = inter] bf16, w_b and codes_b NULL; codes_a [E, d, inter].
+ * For every row and every run j of 32 inputs (the last run of a row may be shorter):
+ *   e = the smallest integer with max|run| <= 448 * 2^e (0 for an all-zero run), within [-127, 127]
+ *   code = e4m3 of value * 2^-e (exact product, round to nearest even)
+ * sf (moe_mx_scale_bytes(kind, E, rows, K) bytes, 16-byte aligned) holds the byte e + 127 of
+ * each run, tiled as the GEMM stages load it: for rows in groups of P (128 for MOE_MX_UP, 256
+ * for MOE_MX_DOWN) and runs in chunks of 4, the 1 KB block ((e * ceil(rows / P) + r / P) *
+ * ceil(K / 128) + j / 4) holds two 512-byte halves (MOE_MX_UP: w1, then w3; MOE_MX_DOWN: rows
+ * r / 128 even, then odd), and row r's byte for run j sits at (r % 32) * 16 + (r / 32 % 4) * 4
+ * + j % 4 of its half; bytes of rows or runs past the matrix are 127.  K must be a multiple of
+ * 16 (MOE_ERR_UNSUPPORTED otherwise) and every pointer 16-byte aligned.  Asynchronous on the
+ * stream; nothing is allocated and nothing can fail on the device.  No passage on the pages
+ * fixes this format (see MOE_FMT_MXFP8 above).
+ */
+typedef enum { MOE_MX_UP = 0, MOE_MX_DOWN = 1 } moe_mx_kind_t;
+size_t moe_mx_scale_bytes(int32_t kind, int32_t n_experts, int32_t rows, int32_t K);
+moe_status_t moe_quantize_weights_mx(int32_t kind, const void* w_a, const void* w_b, int32_t n_experts, int32_t rows,
+                                     int32_t K, uint8_t* codes_a, uint8_t* codes_b, uint8_t* sf,
+                                     moe_stream_t stream);
 
 /*
  * Training: the forward that keeps what the backward needs, and the backward.

@@ -36,10 +36,12 @@ What it computes, and where it comes from:
   dequantised values.  The e4m3 format is taken from its definition (1 sign, 4 exponent bits
   with bias 7, 3 mantissa bits, subnormals, S.1111.111 = NaN, no infinities).
   A second weight format keeps one power-of-two scale per run of 32 consecutive elements
-  along each weight row's input axis instead of one scale per row (block scales; the pages
-  give no block size or scale type either, so this is the same kind of reading): the scale is
-  the smallest power of two that keeps every element of the run within +-448, stored as an
-  unsigned exponent byte (mx_block_exponents); activations are quantised per row as above.
+  along each weight row's input axis instead of one scale per row (the DeepSeek-V2
+  explainer's §5.5 advises per-channel or per-group scales for quantised routed experts and
+  16-bit shared experts, without a group size or scale type, so the run length and the scale
+  rule are a reading): the scale is the smallest power of two that keeps every element of the
+  run within +-448, stored as an unsigned exponent byte (mx_block_exponents); activations are
+  quantised per row as above.
 * Backward pass (an extension; the pages discuss it only through SonicMoE's backward kernels):
   the chain rule of the forward above (layer_backward), and the balance statistics that the
   DeepSeekMoE report's expert- and device-level balance losses are built from (balance_stats;

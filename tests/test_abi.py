@@ -73,7 +73,7 @@ def test_workspace_bytes(lib):
     n8 = moe.workspace_bytes(_shape(routed_fmt=moe.FMT_E4M3))
     extra = S * I + 2 * 4 * S + 256 * d + 4 * 256
     assert extra <= n8 - n <= extra + 5 * 256
-    for bad in (dict(routed_fmt=2), dict(routed_fmt=-1)):
+    for bad in (dict(routed_fmt=3), dict(routed_fmt=-1)):
         assert moe.workspace_bytes(_shape(**bad)) == 0, bad
     for unsupported in (dict(dtype=moe.MOE_F32), dict(d=7176), dict(inter=2056)):
         assert moe.workspace_bytes(_shape(routed_fmt=moe.FMT_E4M3, **unsupported)) == 0, unsupported
@@ -247,3 +247,49 @@ def test_segment_ids_and_wait_selftest_argument_errors(lib):
     assert lib.moe_selftest_wait_timeout(10**6, None, None, 256, None) == moe.MOE_ERR_WORKSPACE
     assert lib.moe_selftest_wait_timeout(10**6, ctypes.c_void_p((1 << 40) + 4), ws, 256, None) == \
         moe.MOE_ERR_INVALID_ARG                                                                       # misaligned out
+
+
+def test_mxfp8_format_validates(lib):
+    """Block-scaled FP8 routed experts: the layer needs the scale bytes (and no per-row scales),
+    every other stack refuses them, they must be 16-byte aligned; the scale-array size and the
+    quantiser's argument checks follow include/moe.h."""
+    fake = ctypes.c_void_p(1 << 40)
+    S = ctypes.byref
+    shm = _shape(routed_fmt=moe.FMT_MXFP8)
+    nm = moe.workspace_bytes(shm)
+    assert nm == moe.workspace_bytes(_shape(routed_fmt=moe.FMT_E4M3)) > 0
+    assert moe.layer_launches(shm) == moe.layer_launches(_shape(routed_fmt=moe.FMT_E4M3)) == 10
+    for unsupported in (dict(dtype=moe.MOE_F32), dict(d=7176), dict(inter=2056)):
+        assert moe.workspace_bytes(_shape(routed_fmt=moe.FMT_MXFP8, **unsupported)) == 0, unsupported
+    f = fake.value
+    w = moe.MoeWeights(f, f, f, f, f, f)
+    w8 = moe.MoeWeights(f, f, f, f, f, f, f, f, f)
+    wm = moe.MoeWeights(f, f, f, f, f, f, None, None, None, f, f)
+    wboth = moe.MoeWeights(*([f] * 11))
+    wmis = moe.MoeWeights(f, f, f, f, f, f, None, None, None, f + 8, f)
+    ffn = lib.moe_expert_ffn
+    for bad in (w, w8, wboth, wmis):
+        assert ffn(S(shm), fake, fake, fake, fake, S(bad), fake, fake, nm, None) == moe.MOE_ERR_INVALID_ARG
+    sh8, n8 = _shape(routed_fmt=moe.FMT_E4M3), moe.workspace_bytes(_shape(routed_fmt=moe.FMT_E4M3))
+    assert ffn(S(sh8), fake, fake, fake, fake, S(wboth), fake, fake, n8, None) == moe.MOE_ERR_INVALID_ARG
+    sh, n = _shape(), moe.workspace_bytes(_shape())
+    assert ffn(S(sh), fake, fake, fake, fake, S(wm), fake, fake, n, None) == moe.MOE_ERR_INVALID_ARG
+    # shared experts stay bf16: scale bytes on the shared stack are refused
+    assert lib.moe_layer_forward(S(shm), fake, fake, None, S(wm), S(wm), fake, None, None, None, fake, nm, None) == \
+        moe.MOE_ERR_INVALID_ARG
+    # scale-array sizes: 1 KB per (expert, row group, 128-input chunk)
+    sb = lib.moe_mx_scale_bytes
+    assert sb(moe.MX_UP, 256, 2048, 7168) == 256 * 16 * 56 * 1024
+    assert sb(moe.MX_DOWN, 256, 7168, 2048) == 256 * 28 * 16 * 1024
+    assert sb(moe.MX_UP, 3, 200, 208) == 3 * 2 * 2 * 1024
+    assert sb(moe.MX_DOWN, 1, 300, 16) == 2 * 1 * 1024
+    assert sb(2, 1, 1, 1) == 0 and sb(moe.MX_UP, 0, 1, 1) == 0 and sb(moe.MX_UP, 1, 1, 0) == 0
+    q = lib.moe_quantize_weights_mx
+    assert q(2, fake, None, 1, 32, 32, fake, None, fake, None) == moe.MOE_ERR_INVALID_ARG          # kind
+    assert q(moe.MX_DOWN, fake, fake, 1, 32, 32, fake, fake, fake, None) == moe.MOE_ERR_INVALID_ARG  # one matrix
+    assert q(moe.MX_UP, fake, None, 1, 32, 32, fake, None, fake, None) == moe.MOE_ERR_INVALID_ARG    # w3 missing
+    assert q(moe.MX_DOWN, fake, None, 1, 32, 24, fake, None, fake, None) == moe.MOE_ERR_UNSUPPORTED  # K % 16
+    assert q(moe.MX_DOWN, fake, None, 0, 32, 32, fake, None, fake, None) == moe.MOE_ERR_INVALID_ARG
+    assert q(moe.MX_DOWN, None, None, 1, 32, 32, fake, None, fake, None) == moe.MOE_ERR_INVALID_ARG
+    assert q(moe.MX_DOWN, fake, None, 1, 32, 32, fake, None, None, None) == moe.MOE_ERR_INVALID_ARG
+    assert q(moe.MX_DOWN, ctypes.c_void_p(f + 8), None, 1, 32, 32, fake, None, fake, None) == moe.MOE_ERR_INVALID_ARG

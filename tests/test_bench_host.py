@@ -63,6 +63,18 @@ def test_stage_work_sums_to_layer_flops():
     routed8 = 3 * 7168 * 2048 + (2 * 2048 + 7168) * 4 + (2 * 2048 + 7168) * 2
     assert abs(bench.layer_bytes(dec, 256, e4m3=True)
                - (256 * routed8 + per_expert + 256 * 7168 * 2 + 2 * 256 * 7168 * 2)) < 1
+    # block-scaled weights: one scale byte per 32 weights at this shape (whole 1 KB tiles), same FLOPs
+    assert bench.mx_scale_bytes_per_expert(dec) == (2 * 2048 * 7168 // 32, 7168 * 2048 // 32)
+    routed_mx = 3 * 7168 * 2048 + 3 * 7168 * 2048 // 32 + (2 * 2048 + 7168) * 2
+    assert abs(bench.layer_bytes(dec, 256, e4m3=True, mx=True)
+               - (256 * routed_mx + per_expert + 256 * 7168 * 2 + 2 * 256 * 7168 * 2)) < 1
+    wm, w8 = bench.stage_work(dec, 256, e4m3=True, mx=True), bench.stage_work(dec, 256, e4m3=True)
+    assert [f for f, _ in wm.values()] == [f for f, _ in w8.values()]
+    assert wm["gemm1_swiglu"][1] - w8["gemm1_swiglu"][1] == 256 * (2 * 2048 * 7168 // 32 - 2 * 2048 * 4)
+    assert wm["gemm2"][1] - w8["gemm2"][1] == 256 * (7168 * 2048 // 32 - 7168 * 4)
+    # ragged shapes pay whole tiles: inter 80 and d 208 -> one 128-row group, two 128-input chunks
+    rag = W.scaled(W.CONFIGS["small"], d=208, inter=80)
+    assert bench.mx_scale_bytes_per_expert(rag) == (1 * 2 * 1024, 1 * 1 * 1024)
 
 
 def test_backward_work_is_twice_the_forward():
@@ -94,6 +106,8 @@ def test_warmup_must_be_three():
         bench.main(["--warmup", "2"])
     with pytest.raises(SystemExit):                     # e4m3 routed experts need a bf16 layer
         bench.main(["--workload", "tiny", "--routed-fmt", "e4m3"])
+    with pytest.raises(SystemExit):
+        bench.main(["--workload", "tiny", "--routed-fmt", "mxfp8"])
 
 
 def test_cpu_baseline_sample_grows_to_the_target():

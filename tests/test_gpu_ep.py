@@ -3,7 +3,8 @@ fp64 oracle: the exchange degenerates to copies, but every other step (routing, 
 row gathers, the device-side regrouping of received rows, the local experts, the combine) runs
 the library's kernels on the path the multi-rank layer takes.  Checked: picks exact outside
 counted near-ties, gates, routed rows Y and the output within the layer tolerance of
-oracle.layer (bf16 and FP8 routed experts); steady-state forwards reuse their workspaces; and the
+oracle.layer (bf16, FP8 with per-row scales and FP8 with block scales); steady-state forwards
+reuse their workspaces; and the
 EP output equals moe_layer_forward's bit for bit.  Also the row gather and segment-id entry
 points against plain indexing (needs a B200)."""
 import os
@@ -34,18 +35,22 @@ def nccl_group():
         dist.destroy_process_group()
 
 
-EP_CASES = [("small", {}, False), ("small", dict(T=77, n_shared=0), False),
-            ("zipf", dict(T=1000, d=512, inter=128, inter_shared=128, n_experts=64), False),
-            ("small", dict(T=300), True), ("zipf", dict(T=1000, d=512, inter=128, inter_shared=128, n_experts=64), True)]
+EP_CASES = [("small", {}, None), ("small", dict(T=77, n_shared=0), None),
+            ("zipf", dict(T=1000, d=512, inter=128, inter_shared=128, n_experts=64), None),
+            ("small", dict(T=300), "e4m3"), ("zipf", dict(T=1000, d=512, inter=128, inter_shared=128, n_experts=64), "e4m3"),
+            ("small", dict(T=300), "mxfp8"),
+            ("zipf", dict(T=1000, d=512, inter=128, inter_shared=128, n_experts=64), "mxfp8")]
 
 
-@pytest.mark.parametrize("name,kw,fp8", EP_CASES, ids=[f"{c[0]}_{i}{'_e4m3' if c[2] else ''}"
+@pytest.mark.parametrize("name,kw,fmt", EP_CASES, ids=[f"{c[0]}_{i}{'_' + c[2] if c[2] else ''}"
                                                       for i, c in enumerate(EP_CASES)])
-def test_ep_world1_against_oracle(nccl_group, name, kw, fp8):
+def test_ep_world1_against_oracle(nccl_group, name, kw, fmt):
     cfg = W.scaled(W.CONFIGS["prefill" if name == "zipf" else name], **kw)
     L = W.make_layer(cfg, "cuda", 2)
+    R_bf16 = L["routed"]
+    fp8 = fmt is not None
     if fp8:
-        L["routed"] = quant.quantize_stack(L["routed"])
+        L["routed"] = quant.quantize_stack(L["routed"], fmt=fmt)
     x, C, R, Sh = L["x"], L["centroids"], L["routed"], L["shared"]
     layer = ep.ExpertParallelMoE(C, R, Sh, cfg.top_k)
     keep = {}
@@ -56,10 +61,12 @@ def test_ep_world1_against_oracle(nccl_group, name, kw, fp8):
     x64, c64 = f64(x), f64(C)
     idx_np, gate_np = keep["idx"].cpu().numpy().astype(np.int64), keep["gate"].cpu().numpy()
     check_routing(idx_np, gate_np, x64, c64, cfg.top_k)
-    ref = O.layer(x64, c64, expert_source(R), cfg.n_experts, cfg.top_k, expert_source(Sh) if Sh is not None else None,
-                  cfg.n_shared, idx_override=idx_np, routed_e4m3=fp8)
+    # block scales: the oracle converts the bf16 weights itself
+    ref = O.layer(x64, c64, expert_source(R_bf16 if fmt == "mxfp8" else R), cfg.n_experts, cfg.top_k,
+                  expert_source(Sh) if Sh is not None else None, cfg.n_shared, idx_override=idx_np,
+                  routed_e4m3=fmt == "e4m3", routed_mx=fmt == "mxfp8")
     tol = TOL[cfg.dtype]
-    case = f"ep_{name}_T{cfg.T}{'_e4m3' if fp8 else ''}"
+    case = f"ep_{name}_T{cfg.T}{'_' + fmt if fp8 else ''}"
     k = cfg.top_k
     slot_of = keep["slot_of"].cpu().numpy()
     y_np = f64(keep["y"])[slot_of[np.arange(cfg.T * k)]]
