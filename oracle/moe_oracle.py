@@ -40,8 +40,9 @@ What it computes, and where it comes from:
   explainer's §5.5 advises per-channel or per-group scales for quantised routed experts and
   16-bit shared experts, without a group size or scale type, so the run length and the scale
   rule are a reading): the scale is the smallest power of two that keeps every element of the
-  run within +-448, stored as an unsigned exponent byte (mx_block_exponents); activations are
-  quantised per row as above.
+  run within +-448, stored as an unsigned exponent byte (mx_block_exponents).  In that format
+  the routed experts' input rows and (bf16-rounded) hidden rows are quantised the same way, in
+  runs of 32 along the row.
 * Backward pass (an extension; the pages discuss it only through SonicMoE's backward kernels):
   the chain rule of the forward above (layer_backward), and the balance statistics that the
   DeepSeekMoE report's expert- and device-level balance losses are built from (balance_stats;
@@ -347,8 +348,8 @@ def layer(x: np.ndarray, centroids: np.ndarray, routed: ExpertSource, n_experts:
     hidden rows are quantised per row (quantize_rows_e4m3, the hidden row after rounding to
     bf16).  The router and the shared experts are unchanged.
     routed_mx: the routed experts' weights are given as plain values and are quantised here to
-    the block-scaled FP8 format (mx_weights); inputs and hidden rows are quantised per row as
-    with routed_e4m3.
+    the block-scaled FP8 format (mx_weights); their input rows and hidden rows (after rounding
+    to bf16) are quantised in runs of 32 the same way (dequantized_blocks).
 
     Returns out [T,d], routed_sum, shared_sum, idx, gate, gap, gap_order, counts, and
     Y [T*k, d] = gate * Expert_e(x_t) per slot (slot = t*k + j); with keep_hidden also
@@ -366,7 +367,8 @@ def layer(x: np.ndarray, centroids: np.ndarray, routed: ExpertSource, n_experts:
     Y = np.zeros((T * k, d))
     H = None
     fp8 = routed_e4m3 or routed_mx
-    xq = dequantized_rows(x) if fp8 else x
+    act_q = dequantized_blocks if routed_mx else dequantized_rows      # activation quantisation
+    xq = act_q(x) if fp8 else x
     for e in np.unique(idx):
         w = _expert(routed, int(e))
         if routed_e4m3:
@@ -376,7 +378,7 @@ def layer(x: np.ndarray, centroids: np.ndarray, routed: ExpertSource, n_experts:
         tt, jj = np.nonzero(idx == e)
         xe = xq[tt]
         he = swiglu_hidden(xe, w["w1"], w["b1"], w["w3"], w["b3"])
-        ye = linear(dequantized_rows(bf16_round(he)) if fp8 else he, w["w2"], w["b2"])
+        ye = linear(act_q(bf16_round(he)) if fp8 else he, w["w2"], w["b2"])
         if keep_hidden:
             if H is None:
                 H = np.zeros((T * k, he.shape[1]))

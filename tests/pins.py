@@ -511,11 +511,12 @@ def check_mx_layer_closed_form(O):
     """The block-scaled FP8 routed path on experts whose weight rows hold one non-zero value
     each (so each run of 32 holds at most one value and each Linear is a scaled selection): the
     layer must equal the closed form built from brute-force block exponents, torch's e4m3 and
-    bf16 casts and scipy's expit, with per-row activation scales and an unquantised shared
-    expert."""
+    bf16 casts and scipy's expit, with the input and hidden rows quantised in runs of 32 too and
+    an unquantised shared expert."""
     rng = _rng(32)
     T, d, I, N, k = 5, 64, 40, 3, 2
     x = rng.standard_normal((T, d)) * np.exp2(rng.uniform(-4, 4, (T, 1)))
+    x *= np.repeat(np.exp2(rng.uniform(-6, 0, (T, d // 32))), 32, axis=1)   # a magnitude per run of 32
     x = x.astype(np.float32).astype(np.float64)
     c = rng.normal(0, 0.5, (N, d))
     experts = []
@@ -534,7 +535,7 @@ def check_mx_layer_closed_form(O):
     stack = _stack([{k_: v for k_, v in e.items() if not k_.startswith("p")} for e in experts])
     res = O.layer(x, c, stack, N, k, shared=_stack([shared]), n_shared=1, routed_mx=True)
     r = O.route(x, c, k)
-    xq = _torch_quant_rows(x)
+    xq = _torch_mx_values(x)
 
     def val(e, name, rows):
         w = e[name][np.arange(rows), e["p" + name[1]]]
@@ -549,7 +550,7 @@ def check_mx_layer_closed_form(O):
             g = val(e, "w3", I) * xq[t, e["p3"]] + e["b3"]
             h = a * scipy.special.expit(a) * g
             hb = torch.from_numpy(h).float().bfloat16().double().numpy()
-            hq = _torch_quant_rows(hb[None])[0]
+            hq = _torch_mx_values(hb[None])[0]
             y = val(e, "w2", d) * hq[e["p2"]] + e["b2"]
             want[t] += r["gate"][t, j] * y
     assert np.allclose(res["out"], want, rtol=1e-12, atol=1e-12)

@@ -13,7 +13,8 @@ _orig = {name: getattr(O, name) for name in ("silu", "linear", "route", "swiglu_
                                              "expert_macs", "split_expert", "hit_entropy", "e4m3_round",
                                              "quantize_rows_e4m3", "e4m3_weights", "e4m3_decode",
                                              "silu_grad", "gate_backward", "expert_backward", "balance_stats",
-                                             "mx_block_exponents", "mx_weights")}
+                                             "mx_block_exponents", "mx_weights", "dequantized_blocks",
+                                             "dequantized_rows")}
 
 
 def _sigmoid_for_silu(a):                      # silu without the factor a
@@ -205,6 +206,10 @@ def _mx_weights_skip_w2(w):                    # w2 left unquantised
     return out
 
 
+def _blocks_as_rows(a):                        # block-scaled values with one scale per row
+    return _orig["dequantized_rows"](a)
+
+
 MUTANTS = {
     "silu_is_sigmoid": ("silu", _sigmoid_for_silu),
     "linear_drops_bias": ("linear", _linear_no_bias),
@@ -233,6 +238,7 @@ MUTANTS = {
     "mx_exponent_off_by_one": ("mx_block_exponents", _mx_exponent_off_by_one),
     "mx_runs_of_16": ("MX_BLOCK", 16),
     "mx_w2_unquantised": ("mx_weights", _mx_weights_skip_w2),
+    "mx_values_scaled_per_row": ("dequantized_blocks", _blocks_as_rows),
 }
 
 
