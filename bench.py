@@ -17,7 +17,8 @@ Multi-GPU runs are replicas: every rank holds the same weights and processes its
 
 --routed-fmt e4m3 stores the routed experts' weights as e4m3 codes with per-channel scales
 (converted once before timing) and runs their GEMMs on the FP8 tensor-core path; mxfp8 keeps a
-power-of-two scale per run of 32 inputs instead, applied by the tensor cores inside the MMA.
+power-of-two scale per run of 32 inputs instead (weights, expert inputs and hidden rows alike),
+applied by the tensor cores inside the MMA.
 
 --impl reference times the fp64 CPU oracle (the only reference that exists for this layer)
 on bounded samples of the same workload, on rank 0 only.
@@ -101,16 +102,37 @@ def stage_work(cfg: W.LayerConfig, touched: int, e4m3: bool = False, mx: bool = 
     at least one token (`touched`), activations read and written by the stage, routing
     metadata.  FLOPs count 2 per multiply-add of the contractions only.  With e4m3 routed
     experts their weights, the gathered rows and the quantised hidden rows are 1 byte each,
-    plus one fp32 scale per weight row and per activation row (mx: the weights' block-scale
-    bytes instead of per-row scales); the gemm2 stage includes the hidden-row quantisation (bf16 h
-    read, e4m3 h written).
+    plus one fp32 scale per weight row and per activation row, and the gemm2 stage includes the
+    hidden-row quantisation (bf16 h read, e4m3 h written).  Block-scaled (mx): one scale byte per
+    run of 32 instead, for weights (in whole 1 KB tiles) and activations, and GEMM1 writes h as
+    codes directly.
     """
     T, d, E, I, k, Ks, Is = cfg.T, cfg.d, cfg.n_experts, cfg.inter, cfg.top_k, cfg.n_shared, cfg.inter_shared
     b = cfg.elem_bytes()
     S = T * k
     bias = 1 if cfg.has_bias else 0
+    if e4m3 and mx:
+        # block-scaled: weights with their tiled run-scale bytes; x and h as codes with one scale
+        # byte per run of 32 (x quantised per token, its codes and scales placed by grouped row;
+        # GEMM1 writes h as codes and scales itself, so GEMM2 has no quantisation step)
+        w13_sc, w2_sc = mx_scale_bytes_per_expert(cfg)
+        rx, rh = -(-d // 32), -(-I // 32)
+        return {
+            "router": (2.0 * T * d * E, (T * d + E * d) * b + S * 8),
+            "permute": (0.0, S * 8 + S * 16),
+            "plan": (0.0, (E + 1) * 4),
+            "gather": (0.0, T * d * b + S * d + S * rx + S * 4),
+            "gemm1_swiglu": (2.0 * S * d * 2 * I + 2.0 * Ks * T * d * 2 * Is,
+                             touched * (2 * I * d + w13_sc + 2 * I * bias * b) + S * d + S * rx
+                             + Ks * (2 * Is * d + 2 * Is * bias) * b + (T * d * b if Ks else 0)
+                             + S * I + S * rh + Ks * T * Is * b),
+            "gemm2": (2.0 * S * I * d + 2.0 * Ks * T * Is * d,
+                      touched * (d * I + w2_sc + d * bias * b) + S * I + S * rh + S * d * b + S * 4
+                      + Ks * (d * Is + d * bias) * b + Ks * T * Is * b + (T * d * 4 if Ks else 0)),
+            "combine": (0.0, S * d * b + (T * d * 4 if Ks else 0) + T * d * b + S * 4),
+        }
     if e4m3:
-        w13_sc, w2_sc = mx_scale_bytes_per_expert(cfg) if mx else (2 * I * 4, d * 4)
+        w13_sc, w2_sc = (2 * I * 4, d * 4)
         return {
             "router": (2.0 * T * d * E, (T * d + E * d) * b + S * 8),
             "permute": (0.0, S * 8 + S * 16),

@@ -38,4 +38,17 @@ __device__ __forceinline__ float silu_f32(float a) { return a / (1.0f + expf(-a)
 
 __host__ __device__ constexpr inline int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
+// Block-scaled FP8 (MOE_FMT_MXFP8): the exponent e of a run of 32 values from the fp32 bits of
+// its maximum magnitude amax >= 0: the smallest integer with amax <= 448 * 2^e, 0 for amax == 0,
+// within [-127, 127].  amax in [2^e0, 2^(e0+1)) and 448 * 2^(e0-8) = 1.75 * 2^e0, so e = e0 - 8
+// when the mantissa field is at most 0.75 (0x600000), else e0 - 7.
+__device__ __forceinline__ int mx_exponent(float amax) {
+    const uint32_t b = __float_as_uint(amax);
+    if (b == 0u) return 0;
+    const int eb = (int)(b >> 23);
+    if (eb == 0) return -127;                              // below 2^-126: clamped
+    const int e = eb - 127 - 8 + ((b & 0x7FFFFFu) > 0x600000u ? 1 : 0);
+    return e < -127 ? -127 : (e > 127 ? 127 : e);
+}
+
 }  // namespace moe

@@ -40,6 +40,7 @@
 // TMEM and returns.  A CTA-pair variant of the expert GEMMs (cta_group::2, clusters of two,
 // off by default) is in the source; no TMA load anywhere uses cluster multicast.
 #include <cuda.h>
+#include <cuda_fp8.h>
 
 #include "common.cuh"
 #include "launch.h"
@@ -60,19 +61,19 @@ constexpr int STAGE_OUT_BYTES = 2048;     // per epilogue warp: a 32 x 32 bf16 c
 constexpr int SMEM_BYTES = 1024 /*align slack*/ + RING_BYTES + 256 /*barriers*/ + EPI_WARPS * STAGE_OUT_BYTES;
 constexpr int ZERO_BYTES = 16384;         // DW: zeros that TMA stores copy to the gradients of groups without rows
 constexpr int SMEM_BYTES_DW = SMEM_BYTES + ZERO_BYTES;
-// Block-scaled weights (mxw): each stage also brings the B tile's scale bytes (256 rows x 4
+// Block-scaled operands (mxw): each stage also brings the B tile's scale bytes (256 rows x 4
 // runs of 32 = 1 KB, two 512-byte blocks of 128 rows each, row r at byte (r % 32) * 16 +
-// (r / 32 % 4) * 4 + run), copied from there into tensor-memory columns SFB_COL..SFB_COL + 7
-// before the stage's MMAs; the A side's scales are all 1 (byte 127, columns SFA_COL..+3,
-// written once).  To free those columns the second accumulator starts MX_OVL columns early
+// (r / 32 % 4) * 4 + run) and the A tile's (128 rows, one such 512-byte block), copied from
+// there into tensor-memory columns SFB_COL..SFB_COL + 7 and SFA_COL..SFA_COL + 3 before the
+// stage's MMAs.  To free those columns the second accumulator starts MX_OVL columns early
 // (224 instead of 256), so the two accumulators share columns 224-255: the epilogue drains
 // that shared chunk first and releases it through ovl_bar before the next tile's MMAs start.
 constexpr int MX_OVL = 32;
-constexpr int SF_STAGE_BYTES = 1024;
-constexpr int SFA_BYTES = 512;
+constexpr int SF_STAGE_BYTES = 1024;                             // B scales of one stage
+constexpr int SFA_BYTES = 512;                                   // A scales of one stage
 constexpr uint32_t SFA_COL = 2 * ACC_COLS - MX_OVL;            // 480
 constexpr uint32_t SFB_COL = SFA_COL + 8;                        // 488
-constexpr int SMEM_BYTES_Q8 = SMEM_BYTES + 4 * SF_STAGE_BYTES + SFA_BYTES;
+constexpr int SMEM_BYTES_Q8 = SMEM_BYTES + 4 * (SF_STAGE_BYTES + SFA_BYTES);
 constexpr unsigned long long WAIT_NS = 4000000000ull;
 #ifndef MOE_GROUP_M
 #define MOE_GROUP_M 8                    // M-tiles per raster band of the expert GEMMs
@@ -125,9 +126,12 @@ struct Params {
     int q8;                    // routed tiles read e4m3 A and B (K blocks of 128 bytes)
     const float* a_scale;      // q8: per-row scale of the routed A rows (x_perm or h rows)
     const float *ws1, *ws3, *ws2;  // q8: per-output-channel weight scales [E, I], [E, I], [E, d]
-    int mxw;                   // q8 with block-scaled weights: the MMAs apply the weights' block scales
+    int mxw;                   // q8, block-scaled: the MMAs apply the operands' run scales
     const uint8_t* sf13;       // mxw: W1 | W3 scale bytes, [E][ceil(I/128)][ceil(d/128)][W1, W3][512]
     const uint8_t* sf2;        // mxw: W2 scale bytes, [E][ceil(d/256)][ceil(I/128)][2][512]
+    const uint8_t* sfa;        // mxw: the routed A rows' scale bytes, [M-tile][K chunk][512]
+    uint8_t* h8_out;           // mxw GEMM1: routed hidden rows as e4m3 codes [S][I] ...
+    uint8_t* sfh_out;          // ... and their scale bytes, [M-tile][ceil(I/128)][512] (GEMM2's sfa)
     int fold_shared;           // GEMM2R: shared-expert GEMM2 tiles follow the routed ones (-> sout)
     // ---- forward for training: GEMM1 also stores the pre-activations a = x W1^T + b1, g = x W3^T + b3
     __nv_bfloat16 *a_out, *g_out;      // routed [S][I] (grouped order)
@@ -720,6 +724,56 @@ __device__ __forceinline__ void warp_store_chunk_bf16(uint32_t stage, const uint
 // e4m3 routed tile (Q8) the accumulators are first multiplied by the row's activation scale
 // and the column's weight scale.  Rows are stored through the per-warp transpose (all lanes
 // take part; rows past the group's end pass a null row).
+// Block-scaled routed tile (mxw): the global index of its 128-row block among all routed experts'
+// blocks (expert e's blocks start at tile_start[e] / N-tiles per block), which indexes the A-side
+// scale bytes [M-tile][K chunk][512].  GEMM1 and GEMM2 number the blocks alike.
+template <int MODE>
+__device__ __forceinline__ int mx_mtile(const Params& p, const Tile& x) {
+    const int ntn = MODE == GEMM1 ? ceil_div(p.I, 128) : ceil_div(p.d, 256);
+    return p.tile_start[x.g] / ntn + x.m0 / BM;
+}
+
+// Block-scaled tiles: offset of the scale byte of tile row r (0-127), run j, in the tiled layout
+// [M-tile][K chunk of 128][512] (row r at (r % 32) * 16 + (r / 32 % 4) * 4 + j % 4 of its chunk).
+__device__ __forceinline__ size_t mx_scale_byte(int mtile, int chunks, int r, int j) {
+    return ((size_t)mtile * chunks + j / 4) * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4 + (j & 3);
+}
+
+// One run of 32 hidden values (bf16-rounded, packed in pk) of this thread's row -> e4m3 codes
+// with the smallest non-saturating power-of-two scale: ncols codes to dst (null for a padding
+// row, which stores only the neutral scale byte 127), the exponent byte to *sf.
+__device__ __forceinline__ void store_run_e4m3(const Params& p, const uint32_t (&pk)[16], uint8_t* dst, int ncols,
+                                               uint8_t* sf) {
+    (void)p;
+    float v[32];
+    float m = 0.f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        v[2 * i] = __uint_as_float(pk[i] << 16);
+        v[2 * i + 1] = __uint_as_float(pk[i] & 0xFFFF0000u);
+        if (2 * i < ncols) m = fmaxf(m, fabsf(v[2 * i]));
+        if (2 * i + 1 < ncols) m = fmaxf(m, fabsf(v[2 * i + 1]));
+    }
+    const int ex = dst ? mx_exponent(m) : 0;
+    *sf = (uint8_t)(ex + 127);
+    if (!dst) return;
+    const float mul = __uint_as_float((uint32_t)(127 - ex) << 23);   // 2^-ex (ex <= 126 for finite h)
+    uint32_t q[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(v[4 * i] * mul, v[4 * i + 1] * mul), __NV_SATFINITE, __NV_E4M3);
+        const uint32_t hi =
+            __nv_cvt_float2_to_fp8x2(make_float2(v[4 * i + 2] * mul, v[4 * i + 3] * mul), __NV_SATFINITE, __NV_E4M3);
+        q[i] = lo | (hi << 16);
+    }
+    if (ncols == 32) {
+        reinterpret_cast<uint4*>(dst)[0] = make_uint4(q[0], q[1], q[2], q[3]);
+        reinterpret_cast<uint4*>(dst)[1] = make_uint4(q[4], q[5], q[6], q[7]);
+    } else {
+        for (int j = 0; j < ncols; ++j) dst[j] = (uint8_t)(q[j >> 2] >> (8 * (j & 3)));
+    }
+}
+
 // Overlapping accumulators (mxw): the warp that holds the columns both accumulators share
 // reports them drained (their tensor-memory loads complete) so the next tile's MMAs may start.
 __device__ __forceinline__ void release_shared_cols(uint32_t ovl, int lane) {
@@ -745,8 +799,12 @@ __device__ __forceinline__ void epilogue_gemm1(const Params& p, const Tile& x, u
     const float* sc3 = (scaled && !p.mxw) ? p.ws3 + (size_t)e * I : nullptr;
     const int r = x.m0 + row;
     const bool live = r < x.rows;
-    const float rs = (scaled && live) ? p.a_scale[x.row0 + r] : 1.f;
+    // block-scaled tiles: the input rows' scales are applied by the MMA, and h leaves as e4m3 codes
+    // with one scale per run of 32 (this thread's 32-column chunk) for GEMM2's A operand
+    const bool mxq = scaled && p.mxw;
+    const float rs = (scaled && !p.mxw && live) ? p.a_scale[x.row0 + r] : 1.f;
     const size_t ro = shared ? ((size_t)e * p.T + r) * I : (size_t)(x.row0 + r) * I;
+    const int mtile = mxq ? mx_mtile<GEMM1>(p, x) : 0;
     __nv_bfloat16* hrow = live ? (shared ? p.h_s : p.h_r) + ro : nullptr;
     __nv_bfloat16* arow = (live && p.a_out) ? (shared ? p.as_out : p.a_out) + ro : nullptr;
     __nv_bfloat16* grow = (live && p.a_out) ? (shared ? p.gs_out : p.g_out) + ro : nullptr;
@@ -759,7 +817,13 @@ __device__ __forceinline__ void epilogue_gemm1(const Params& p, const Tile& x, u
         tmem_wait_ld();
         if (ovl && it == 0) release_shared_cols(ovl, lane);
         const int col0 = x.n0 + c * 32;
-        if (col0 >= I) continue;                                // warp-uniform
+        if (col0 >= I) {                                        // warp-uniform
+            // block-scaled: a run past I inside GEMM2's last K chunk still gets a finite scale
+            // byte (its codes are zero there), so no scale that GEMM2 reads is left unset
+            if (mxq && col0 / 128 < ceil_div(I, 128))
+                p.sfh_out[mx_scale_byte(mtile, ceil_div(I, 128), row, col0 / 32)] = 127;
+            continue;
+        }
         const int ncols = min(32, I - col0);
         uint32_t pk[16], pa[16], pg[16];
 #pragma unroll
@@ -785,6 +849,11 @@ __device__ __forceinline__ void epilogue_gemm1(const Params& p, const Tile& x, u
             pa[i] = pack_bf16(av[0], av[1]);
             pg[i] = pack_bf16(gv[0], gv[1]);
         }
+        if (mxq) {                                              // warp-uniform
+            store_run_e4m3(p, pk, live ? p.h8_out + ro + col0 : nullptr, ncols,
+                           p.sfh_out + mx_scale_byte(mtile, ceil_div(I, 128), row, col0 / 32));
+            continue;
+        }
         warp_store_chunk_bf16(stage, pk, hrow ? hrow + col0 : nullptr, ncols, lane);
         if (p.a_out) {                                          // warp-uniform
             warp_store_chunk_bf16(stage, pa, arow ? arow + col0 : nullptr, ncols, lane);
@@ -805,7 +874,7 @@ __device__ __forceinline__ void epilogue_gemm2r(const Params& p, const Tile& x, 
     const float gate = live ? (p.sorted_gate ? p.sorted_gate[pos] : 1.f) : 0.f;
     const __nv_bfloat16* b2 = p.b2 ? p.b2 + (size_t)x.g * p.d : nullptr;
     const float* sc2 = (Q8 && !p.mxw) ? p.ws2 + (size_t)x.g * p.d : nullptr;   // block-scaled: in the MMA
-    const float rs = (Q8 && live) ? p.a_scale[pos] : 1.f;
+    const float rs = (Q8 && !p.mxw && live) ? p.a_scale[pos] : 1.f;
     __nv_bfloat16* yrow = live ? p.y + (size_t)pos * p.d : nullptr;
 #pragma unroll 1
     for (int it = 0; it < 4; ++it) {
@@ -1145,10 +1214,10 @@ __global__ void __launch_bounds__(THREADS, 1) moe_tc_kernel(const __grid_constan
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
     static_assert(8 * (2 * STAGES + 7) + 8 <= 256, "barrier area");
     static_assert(!Q8 || PAIR || STAGES <= 4, "scale-byte ring sized for 4 stages");
-    // mxw: the stages' B scale bytes and the constant A scale block, after the epilogue buffers
+    // mxw: the stages' B and A scale bytes, after the epilogue buffers
     const uint32_t sf_base = bar0 + 256 + EPI_WARPS * STAGE_OUT_BYTES;
     auto sfb_stage = [&](int s) { return sf_base + (uint32_t)(s * SF_STAGE_BYTES); };
-    const uint32_t sfa_buf = sf_base + 4 * SF_STAGE_BYTES;
+    auto sfa_stage = [&](int s) { return sf_base + (uint32_t)(4 * SF_STAGE_BYTES + s * SFA_BYTES); };
     const bool mxw = Q8 && !PAIR && p.mxw;
     const uint32_t acc_cols = mxw ? (uint32_t)(ACC_COLS - MX_OVL) : (uint32_t)ACC_COLS;   // second accumulator's start
 
@@ -1312,9 +1381,9 @@ __global__ void __launch_bounds__(THREADS, 1) moe_tc_kernel(const __grid_constan
                             }
                         }
                     } else {
-                        // block-scaled e4m3 tile: the stage's 1 KB of B scale bytes come along
+                        // block-scaled e4m3 tile: the stage's B (1 KB) and A (512 B) scale bytes come along
                         const bool sf_tile = mxw && (MODE == GEMM1 ? x.g < p.E : (MODE == GEMM2R && x.g >= 0));
-                        mbar_expect_tx(fb, A_BYTES + B_BYTES + (sf_tile ? SF_STAGE_BYTES : 0));
+                        mbar_expect_tx(fb, A_BYTES + B_BYTES + (sf_tile ? SF_STAGE_BYTES + SFA_BYTES : 0));
                         if (sf_tile) {
                             const uint8_t* src =
                                 MODE == GEMM1
@@ -1323,6 +1392,8 @@ __global__ void __launch_bounds__(THREADS, 1) moe_tc_kernel(const __grid_constan
                                     : p.sf2 + (((size_t)x.g * ceil_div(p.d, 256) + x.n0 / 256) * ceil_div(p.I, 128) + kb) *
                                                   SF_STAGE_BYTES;
                             bulk_load(sfb_stage(stage), src, SF_STAGE_BYTES, fb);
+                            bulk_load(sfa_stage(stage), p.sfa + ((size_t)mx_mtile<MODE>(p, x) * x.num_kb + kb) * SFA_BYTES,
+                                      SFA_BYTES, fb);
                         }
                         if (MODE == GEMM1) {
                             const bool shared = x.g >= p.E;
@@ -1370,14 +1441,6 @@ __global__ void __launch_bounds__(THREADS, 1) moe_tc_kernel(const __grid_constan
         // ------------------------------------------------------------------ MMA issuer
         if (lane == 0 && leader) {
             const uint32_t idesc = PAIR ? idesc_bf16_pair(p.n_mma) : idesc_bf16(p.n_mma);
-            if (mxw) {
-                // A-side scales: byte 127 (2^0) for every row and run, copied into TMEM once
-                for (int i = 0; i < SFA_BYTES / 16; ++i)
-                    asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(sfa_buf + 16u * i), "r"(0x7F7F7F7Fu)
-                                 : "memory");
-                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-                tmem_cp_sf(tmem_base + SFA_COL, sf_desc(sfa_buf));
-            }
             int stage = 0;
             uint32_t phase = 0;
             int acc = 0;
@@ -1404,7 +1467,9 @@ __global__ void __launch_bounds__(THREADS, 1) moe_tc_kernel(const __grid_constan
                     tc_fence_after();
                     const uint32_t a_addr = sA + stage * A_BYTES, b_addr = sB + stage * B_BYTES;
                     if (sf_tile) {
-                        // this stage's B scales: B rows 0-127 -> columns SFB_COL..+3, rows 128-255 -> +4..+7
+                        // this stage's scales: A rows -> columns SFA_COL..+3; B rows 0-127 -> SFB_COL..+3,
+                        // rows 128-255 -> SFB_COL + 4..+7
+                        tmem_cp_sf(tmem_base + SFA_COL, sf_desc(sfa_stage(stage)));
                         tmem_cp_sf(tmem_base + SFB_COL, sf_desc(sfb_stage(stage)));
                         tmem_cp_sf(tmem_base + SFB_COL + 4, sf_desc(sfb_stage(stage) + 512));
                     }
@@ -1713,7 +1778,7 @@ int num_sms() {
 bool gemm_pairs(const Dims& D) {
     (void)D;
 #if defined(MOE_PAIR_POLICY) && MOE_PAIR_POLICY > 0
-    return true;
+    return !D.mx;                          // block-scaled tiles run on single CTAs only
 #else
     return false;
 #endif
@@ -1846,17 +1911,19 @@ cudaError_t launch_tc_gemm2_shared(const Dims& D, const FfnWeights& Sh, const vo
 cudaError_t launch_tc_gemm1_q8(const Dims& D, const void* x, const void* x8_perm, const float* xs,
                                const int32_t* offsets, const int32_t* tile_start1, const FfnWeights& R,
                                const FfnWeights& Sh, void* h_r, void* h_s, int g_end, uint32_t* err,
-                               cudaStream_t stream) {
+                               cudaStream_t stream, const MxAct* mx) {
     using namespace tc;
     if (D.T == 0) return cudaSuccess;
-    if ((D.mx ? !R.sf13 : (!R.s1 || !R.s3)) || !xs) return cudaErrorInvalidValue;
+    if (D.mx ? (!R.sf13 || !mx || !mx->sfa || !mx->h8 || !mx->sfh) : (!R.s1 || !R.s3 || !xs))
+        return cudaErrorInvalidValue;
     Params p = base_params(D, err);
     p.q8 = 1;
     p.a_scale = xs;
     p.ws1 = R.s1; p.ws3 = R.s3;
     p.mxw = D.mx ? 1 : 0;
     p.sf13 = R.sf13;
-    const bool pairs = tc::pairs_for(D) && !D.mx;          // block scales run on single CTAs
+    if (D.mx) { p.sfa = mx->sfa; p.h8_out = mx->h8; p.sfh_out = mx->sfh; }
+    const bool pairs = tc::pairs_for(D);                   // never for block scales (gemm_pairs)
     p.tile_start = tile_start1;
     p.offsets = offsets;
     p.g_begin = 0;
@@ -1887,22 +1954,23 @@ cudaError_t launch_tc_gemm1_q8(const Dims& D, const void* x, const void* x8_perm
 cudaError_t launch_tc_gemm2_routed_q8(const Dims& D, const int32_t* offsets, const int32_t* tile_start2,
                                       const float* sorted_gate, const FfnWeights& R, const void* h8,
                                       const float* hs, void* y_sorted, const FfnWeights* Sh, const void* h_s,
-                                      float* sout, uint32_t* err, cudaStream_t stream) {
+                                      float* sout, uint32_t* err, cudaStream_t stream, const MxAct* mx) {
     using namespace tc;
     if (D.T == 0) return cudaSuccess;
-    if ((D.mx ? !R.sf2 : !R.s2) || !hs) return cudaErrorInvalidValue;
+    if (D.mx ? (!R.sf2 || !mx || !mx->sfa) : (!R.s2 || !hs)) return cudaErrorInvalidValue;
     Params p = base_params(D, err);
     p.q8 = 1;
     p.a_scale = hs;
     p.ws2 = R.s2;
     p.mxw = D.mx ? 1 : 0;
     p.sf2 = R.sf2;
+    if (D.mx) p.sfa = mx->sfa;
     p.tile_start = tile_start2;
     p.offsets = offsets;
     p.sorted_gate = sorted_gate;
     p.b2 = (const __nv_bfloat16*)R.b2;
     p.y = (__nv_bfloat16*)y_sorted;
-    const bool pairs = tc::pairs_for(D) && !D.mx;          // block scales run on single CTAs
+    const bool pairs = tc::pairs_for(D);                   // never for block scales (gemm_pairs)
     bool ok = make_map_u8(&p.tmA[0], h8, D.I, (uint64_t)D.slots(), 1, 2 * BK, BM, false);
     ok &= make_map_u8(&p.tmB[0], R.w2, D.I, D.d, D.E, 2 * BK, pairs ? 128 : 256, true);
     if (Sh && D.Ks > 0 && sout) {

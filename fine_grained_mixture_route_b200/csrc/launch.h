@@ -70,6 +70,14 @@ cudaError_t launch_scatter_rows(const Dims& D, const void* x, const int32_t* slo
 size_t mx_scale_bytes(int kind, long long n_experts, int rows, int K);
 cudaError_t launch_quant_weights_mx(int kind, const void* w, int which, int n_experts, int rows, int K, uint8_t* codes,
                                     uint8_t* sf, cudaStream_t stream);
+// Block-scaled routed activations: x rows [rows][K] -> codes [rows][K] and run scales [rows][ceil(K/32)];
+// then each grouped position's scales into the GEMM's tiled A-side layout [M-tile][ceil(K/128)][512]
+// (mx_act_scale_bytes bytes for `slots` grouped rows; M-tiles numbered by tile_start1 / ceil(I/128)).
+size_t mx_act_scale_bytes(long long slots, int n_experts, int K);
+cudaError_t launch_quant_rows_mx(const void* src, int rows, int K, uint8_t* codes, uint8_t* sf, cudaStream_t stream);
+cudaError_t launch_scatter_sf_tiled(const uint8_t* xsf, int T, int K, const int32_t* stok, const int32_t* offsets,
+                                    const int32_t* tile_start1, int E, long long S, int I, uint8_t* sfa, uint32_t* err,
+                                    cudaStream_t stream);
 cudaError_t launch_quant_rows(const void* src, const int32_t* row_of, long long n_rows, int src_rows, int width,
                               uint8_t* dst, float* scale, uint32_t* err, cudaStream_t stream);
 // dst[p, :] = src[row_of[p], :] for rows of row_bytes (a multiple of 4) bytes; bad index -> bit 4, zeros
@@ -172,14 +180,22 @@ int num_sms();
 // against the W1 / W3 codes (R.s1, R.s3); shared groups [E, g_end) run bf16 on x in the same
 // launch.  GEMM2R: h8 rows (scale per row in hs) against the W2 codes (R.s2); with Sh the
 // shared experts' bf16 GEMM2 tiles follow (-> sout).
+// Block-scaled routed activations (D.mx): the A rows' tiled scale bytes (GEMM1: x codes, GEMM2: h
+// codes), and for GEMM1 where the hidden rows go as e4m3 codes [S][I] with their tiled scale bytes.
+// The per-row scales (xs, hs) are then unused.
+struct MxAct {
+    const uint8_t* sfa = nullptr;
+    uint8_t* h8 = nullptr;
+    uint8_t* sfh = nullptr;
+};
 cudaError_t launch_tc_gemm1_q8(const Dims& D, const void* x, const void* x8_perm, const float* xs,
                                const int32_t* offsets, const int32_t* tile_start1, const FfnWeights& R,
                                const FfnWeights& Sh, void* h_r, void* h_s, int g_end, uint32_t* err,
-                               cudaStream_t stream);
+                               cudaStream_t stream, const MxAct* mx = nullptr);
 cudaError_t launch_tc_gemm2_routed_q8(const Dims& D, const int32_t* offsets, const int32_t* tile_start2,
                                       const float* sorted_gate, const FfnWeights& R, const void* h8,
                                       const float* hs, void* y_sorted, const FfnWeights* Sh, const void* h_s,
-                                      float* sout, uint32_t* err, cudaStream_t stream);
+                                      float* sout, uint32_t* err, cudaStream_t stream, const MxAct* mx = nullptr);
 
 // ---- backward ----------------------------------------------------------------------
 // Buffers of one backward call.  Routed rows of the weight-gradient operands (dout_pad, x_pad,

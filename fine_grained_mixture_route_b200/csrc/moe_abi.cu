@@ -18,6 +18,7 @@ struct Layout {
     size_t err, hist, rpart, sout, ts1, ts2, idx, gate, counts, offsets, stok, sgate, slot_of, xperm, hr, hs, y;
     size_t xs, h8, hsc;    // e4m3 routed experts: row scales of x8 (in xperm), h8 rows and their scales
     size_t x8t, xst;       // e4m3: x quantised once per token, and its scales
+    size_t xsf, sfa1, sfa2;  // block-scaled: x's run scales per token; GEMM1's and GEMM2's tiled A scales
     size_t total;
 };
 
@@ -49,6 +50,9 @@ Layout layout(const Dims& D) {
     L.hsc = o; o += D.q8 ? al(S * 4) : 0;
     L.x8t = o; o += D.q8 ? al((size_t)D.T * D.d) : 0;
     L.xst = o; o += D.q8 ? al((size_t)D.T * 4) : 0;
+    L.xsf = o; o += D.mx ? al((size_t)D.T * ((D.d + 31) / 32)) : 0;
+    L.sfa1 = o; o += D.mx ? al(mx_act_scale_bytes(D.slots(), D.E, D.d)) : 0;
+    L.sfa2 = o; o += D.mx ? al(mx_act_scale_bytes(D.slots(), D.E, D.I)) : 0;
     L.total = o;
     return L;
 }
@@ -211,18 +215,39 @@ FfnWeights to_ffn(const moe_ffn_weights_t* w) {
 // into expert order for the GEMM1 A operand.
 // With the slot map at hand (the fused forward) the code rows are written in token order
 // instead: each token's codes are read once and stored at its k slot positions.
+// Block-scaled (D.mx): x quantised in runs of 32; the run scales go to GEMM1's tiled A-side
+// layout by grouped position (needs the tile table ts1).
 moe_status_t quant_gather_x(const Dims& D, const Layout& L, void* ws, const void* x, const int32_t* stok,
-                            uint32_t* err, cudaStream_t st, const int32_t* slot_of = nullptr) {
+                            const int32_t* offsets, const int32_t* ts1, uint32_t* err, cudaStream_t st,
+                            const int32_t* slot_of = nullptr) {
     uint8_t* x8t = at<uint8_t>(ws, L.x8t);
-    float* xst = at<float>(ws, L.xst);
-    MOE_CUDA(launch_quant_rows(x, nullptr, D.T, D.T, D.d, x8t, xst, err, st));
+    float* xst = D.mx ? nullptr : at<float>(ws, L.xst);
+    float* xs = D.mx ? nullptr : at<float>(ws, L.xs);
+    if (D.mx) MOE_CUDA(launch_quant_rows_mx(x, D.T, D.d, x8t, at<uint8_t>(ws, L.xsf), st));
+    else MOE_CUDA(launch_quant_rows(x, nullptr, D.T, D.T, D.d, x8t, xst, err, st));
     if (slot_of)
-        MOE_CUDA(launch_scatter_code_rows(x8t, xst, slot_of, D.T, D.k, D.slots(), D.d, at<uint8_t>(ws, L.xperm),
-                                          at<float>(ws, L.xs), err, st));
+        MOE_CUDA(launch_scatter_code_rows(x8t, xst, slot_of, D.T, D.k, D.slots(), D.d, at<uint8_t>(ws, L.xperm), xs,
+                                          err, st));
     else
-        MOE_CUDA(launch_gather_code_rows(x8t, xst, stok, D.slots(), D.T, D.d, at<uint8_t>(ws, L.xperm),
-                                         at<float>(ws, L.xs), err, st));
+        MOE_CUDA(launch_gather_code_rows(x8t, xst, stok, D.slots(), D.T, D.d, at<uint8_t>(ws, L.xperm), xs, err, st));
+    if (D.mx)
+        MOE_CUDA(launch_scatter_sf_tiled(at<uint8_t>(ws, L.xsf), D.T, D.d, stok, offsets, ts1, D.E, D.slots(), D.I,
+                                         at<uint8_t>(ws, L.sfa1), err, st));
     return MOE_OK;
+}
+
+// Block-scaled activations: GEMM1 reads sfa1 and writes the hidden codes and sfa2; GEMM2 reads sfa2.
+MxAct mx_gemm1(const Layout& L, void* ws) {
+    MxAct m;
+    m.sfa = at<uint8_t>(ws, L.sfa1);
+    m.h8 = at<uint8_t>(ws, L.h8);
+    m.sfh = at<uint8_t>(ws, L.sfa2);
+    return m;
+}
+MxAct mx_gemm2(const Layout& L, void* ws) {
+    MxAct m;
+    m.sfa = at<uint8_t>(ws, L.sfa2);
+    return m;
 }
 
 moe_status_t do_route(const Dims& D, const void* x, const void* c, const float* bias, int32_t* idx, float* gate,
@@ -243,14 +268,18 @@ moe_status_t do_expert_ffn(const Dims& D, const Layout& L, void* ws, const void*
     if (!plan_done) MOE_CUDA(launch_plan(D, offsets, ts1, ts2, err, st));
     if (D.q8) {
         uint8_t* x8 = at<uint8_t>(ws, L.xperm);
-        float* xs = at<float>(ws, L.xs);
-        MOE_TRY(quant_gather_x(D, L, ws, x, stok, err, st));
+        float* xs = D.mx ? nullptr : at<float>(ws, L.xs);
+        MOE_TRY(quant_gather_x(D, L, ws, x, stok, offsets, ts1, err, st));
         FfnWeights none = {nullptr, nullptr, nullptr, nullptr, nullptr, nullptr};
-        MOE_CUDA(launch_tc_gemm1_q8(D, x, x8, xs, offsets, ts1, R, none, at<void>(ws, L.hr), nullptr, D.E, err, st));
+        const MxAct m1 = mx_gemm1(L, ws), m2 = mx_gemm2(L, ws);
+        MOE_CUDA(launch_tc_gemm1_q8(D, x, x8, xs, offsets, ts1, R, none, at<void>(ws, L.hr), nullptr, D.E, err, st,
+                                    D.mx ? &m1 : nullptr));
         uint8_t* h8 = at<uint8_t>(ws, L.h8);
-        float* hsc = at<float>(ws, L.hsc);
-        MOE_CUDA(launch_quant_rows(at<void>(ws, L.hr), nullptr, D.slots(), (int)D.slots(), D.I, h8, hsc, err, st));
-        MOE_CUDA(launch_tc_gemm2_routed_q8(D, offsets, ts2, sgate, R, h8, hsc, y, nullptr, nullptr, nullptr, err, st));
+        float* hsc = D.mx ? nullptr : at<float>(ws, L.hsc);
+        if (!D.mx)   // block-scaled: GEMM1 already wrote the hidden rows as codes with their run scales
+            MOE_CUDA(launch_quant_rows(at<void>(ws, L.hr), nullptr, D.slots(), (int)D.slots(), D.I, h8, hsc, err, st));
+        MOE_CUDA(launch_tc_gemm2_routed_q8(D, offsets, ts2, sgate, R, h8, hsc, y, nullptr, nullptr, nullptr, err, st,
+                                           D.mx ? &m2 : nullptr));
     } else if (D.bf16) {
         void* xp = at<void>(ws, L.xperm);
         MOE_CUDA(launch_gather(D, x, stok, xp, err, st));
@@ -302,7 +331,7 @@ MOE_EXPORT int32_t moe_layer_launches(const moe_shape_t* shape) {
     n += 1;                                                         // tile tables
     if (D.bf16) n += 1;                                             // row gather (+ e4m3 quantisation)
     n += 3;                                   // GEMM1, GEMM2 (routed + shared tiles), combine
-    if (D.q8) n += 2;                           // per-token x quantisation, hidden-row quantisation
+    if (D.q8) n += 2;   // per-token x quantisation, hidden-row quantisation (block-scaled: scale scatter)
     return n;
 }
 
@@ -517,17 +546,20 @@ moe_status_t layer_forward_impl(const moe_shape_t* shape, const void* x, const v
     if (!mark(3)) return MOE_ERR_CUDA;
     if (D.q8) {
         uint8_t* x8 = at<uint8_t>(ws, L.xperm);
-        float* xs = at<float>(ws, L.xs);
-        MOE_TRY(quant_gather_x(D, L, ws, x, stok, err, st, slot_of));
+        float* xs = D.mx ? nullptr : at<float>(ws, L.xs);
+        MOE_TRY(quant_gather_x(D, L, ws, x, stok, offsets, ts1, err, st, slot_of));
         if (!mark(4)) return MOE_ERR_CUDA;
-        MOE_CUDA(launch_tc_gemm1_q8(D, x, x8, xs, offsets, ts1, R, Sh, hr, hs, D.E + D.Ks, err, st));
+        const MxAct m1 = mx_gemm1(L, ws), m2 = mx_gemm2(L, ws);
+        MOE_CUDA(launch_tc_gemm1_q8(D, x, x8, xs, offsets, ts1, R, Sh, hr, hs, D.E + D.Ks, err, st,
+                                    D.mx ? &m1 : nullptr));
         if (!mark(5)) return MOE_ERR_CUDA;
         uint8_t* h8 = at<uint8_t>(ws, L.h8);
-        float* hsc = at<float>(ws, L.hsc);
-        MOE_CUDA(launch_quant_rows(hr, nullptr, D.slots(), (int)D.slots(), D.I, h8, hsc, err, st));
+        float* hsc = D.mx ? nullptr : at<float>(ws, L.hsc);
+        if (!D.mx)   // block-scaled: GEMM1 already wrote the hidden rows as codes with their run scales
+            MOE_CUDA(launch_quant_rows(hr, nullptr, D.slots(), (int)D.slots(), D.I, h8, hsc, err, st));
         float* sout = D.Ks > 0 ? at<float>(ws, L.sout) : nullptr;
         MOE_CUDA(launch_tc_gemm2_routed_q8(D, offsets, ts2, sgate, R, h8, hsc, y, D.Ks > 0 ? &Sh : nullptr, hs, sout,
-                                           err, st));
+                                           err, st, D.mx ? &m2 : nullptr));
         if (!mark(6)) return MOE_ERR_CUDA;
         MOE_CUDA(launch_combine(D, y, slot_of, sout, out, err, st));
     } else if (D.bf16) {

@@ -163,7 +163,7 @@ __global__ void scatter_code_rows_kernel(const uint4* __restrict__ src, const fl
             int q = slot_of[(size_t)t * k + threadIdx.x];
             if (q >= S) { flag_error(err, ERR_INDEX_RANGE); q = -1; }
             pos[threadIdx.x] = q;
-            if (q >= 0) dscale[q] = sscale[t];
+            if (q >= 0 && dscale) dscale[q] = sscale[t];
         }
         __syncthreads();
         const uint4* s = src + (size_t)t * nv;
@@ -278,17 +278,6 @@ namespace {
 // product exact (a power of two), rounded to nearest even.  The scale is stored as the byte
 // e + 127, in the tiled order the GEMMs' pipeline stages load (see mx_scale_offset).
 
-// e from the fp32 bits of the run maximum: amax in [2^e0, 2^(e0+1)) and 448 * 2^(e0-8) =
-// 1.75 * 2^e0, so e = e0 - 8 when the mantissa is at most 0.75 (0x600000), else e0 - 7.
-__device__ __forceinline__ int mx_exponent(float amax) {
-    const uint32_t b = __float_as_uint(amax);
-    if (b == 0u) return 0;
-    const int eb = (int)(b >> 23);
-    if (eb == 0) return -127;                              // below 2^-126: clamped
-    const int e = eb - 127 - 8 + ((b & 0x7FFFFFu) > 0x600000u ? 1 : 0);
-    return e < -127 ? -127 : (e > 127 ? 127 : e);
-}
-
 // 8 bf16 times a power of two -> 8 e4m3 codes (element j in byte j)
 __device__ __forceinline__ uint2 chunk_quant_mul(const uint4& v, float mul) {
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
@@ -313,14 +302,16 @@ __device__ __forceinline__ size_t mx_scale_offset(int e, int r, int j, int ngrp,
 }
 
 // One warp per row; lane i of a pass holds 16-byte chunk i (8 elements), so lanes 4q..4q+3 hold
-// run q of the pass and two shuffles give its maximum.
+// run q of the pass and two shuffles give its maximum.  P > 0: weight scales in the tiled order;
+// P == 0: activation rows, row q's scale of run j at sf[q * ceil(K / 32) + j].
 __global__ void __launch_bounds__(256) quant_weights_mx_kernel(const uint4* __restrict__ src, int E, int rows, int K,
                                                                int P, int which, uint2* __restrict__ codes,
                                                                uint8_t* __restrict__ sf) {
     const int lane = threadIdx.x & 31;
     const int nv = K / 8;
     const int nch = (K + 127) / 128;
-    const int ngrp = (rows + P - 1) / P;
+    const int nruns = (K + 31) / 32;
+    const int ngrp = P > 0 ? (rows + P - 1) / P : 0;
     const long long n_rows = (long long)E * rows;
     const long long warps = (long long)gridDim.x * (blockDim.x >> 5);
     for (long long q = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); q < n_rows; q += warps) {
@@ -336,12 +327,78 @@ __global__ void __launch_bounds__(256) quant_weights_mx_kernel(const uint4* __re
             const int ex = mx_exponent(m);
             const float mul = __uint_as_float((uint32_t)(127 - ex) << 23);   // 2^-ex (ex <= 126 for finite runs)
             if (i < nv) dst[i] = chunk_quant_mul(v, mul);
-            if ((lane & 3) == 0 && i < nv) sf[mx_scale_offset(e, r, i >> 2, ngrp, nch, P, which)] = (uint8_t)(ex + 127);
+            if ((lane & 3) == 0 && i < nv)
+                sf[P > 0 ? mx_scale_offset(e, r, i >> 2, ngrp, nch, P, which) : (size_t)q * nruns + (i >> 2)] =
+                    (uint8_t)(ex + 127);
         }
     }
 }
 
+// The A-side scales of the block-scaled GEMM1: grouped position p (token stok[p], in expert e's
+// rows [offsets[e], offsets[e + 1])) is row r = (p - offsets[e]) % 128 of the expert's 128-row
+// block m = (p - offsets[e]) / 128, whose global index is tile_start1[e] / n_tiles + m.  Thread
+// (p, c) copies the token's scale bytes of runs 4c..4c+3 (127 past the row) to that block's
+// chunk c: [M-tile][chunk][512], row r at (r % 32) * 16 + (r / 32 % 4) * 4.
+__global__ void scatter_sf_tiled_kernel(const uint8_t* __restrict__ xsf, int nruns, const int32_t* __restrict__ stok,
+                                        int T, const int32_t* __restrict__ offsets, const int32_t* __restrict__ tile_start1,
+                                        int E, long long S, int n_tiles, int nch, uint8_t* __restrict__ sfa, uint32_t* err) {
+    const long long total = S * nch;
+    for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+         i += (long long)gridDim.x * blockDim.x) {
+        const long long p = i / nch;
+        const int c = (int)(i % nch);
+        const int t = stok[p];
+        if (t < 0 || t >= T) {
+            flag_error(err, ERR_INDEX_RANGE);
+            continue;
+        }
+        int lo = 0, hi = E;                               // the last e with offsets[e] <= p
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (offsets[mid] <= p) lo = mid;
+            else hi = mid - 1;
+        }
+        const int local = (int)(p - offsets[lo]);
+        const long long g = tile_start1[lo] / n_tiles + local / 128;
+        const int r = local & 127;
+        uint32_t w = 0;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int run = 4 * c + j;
+            const uint32_t b = run < nruns ? xsf[(size_t)t * nruns + run] : 127u;
+            w |= b << (8 * j);
+        }
+        *reinterpret_cast<uint32_t*>(sfa + ((size_t)g * nch + c) * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4) = w;
+    }
+}
+
 }  // namespace
+
+size_t mx_act_scale_bytes(long long slots, int n_experts, int K) {
+    return (size_t)((slots + 127) / 128 + n_experts) * ((K + 127) / 128) * 512;
+}
+
+cudaError_t launch_quant_rows_mx(const void* src, int rows, int K, uint8_t* codes, uint8_t* sf, cudaStream_t stream) {
+    if (rows <= 0) return cudaSuccess;
+    if (K % 8) return cudaErrorInvalidValue;
+    const long long cap = 8LL * 8 * num_sms();
+    const int blocks = (int)((rows + 7) / 8 < cap ? (rows + 7) / 8 : cap);
+    quant_weights_mx_kernel<<<blocks, 256, 0, stream>>>((const uint4*)src, 1, rows, K, 0, 0, (uint2*)codes, sf);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_scatter_sf_tiled(const uint8_t* xsf, int T, int K, const int32_t* stok, const int32_t* offsets,
+                                    const int32_t* tile_start1, int E, long long S, int I, uint8_t* sfa, uint32_t* err,
+                                    cudaStream_t stream) {
+    if (S <= 0) return cudaSuccess;
+    const int nch = (K + 127) / 128;
+    const long long total = S * nch;
+    const long long cap = 8LL * 8 * num_sms();
+    const int blocks = (int)((total + 255) / 256 < cap ? (total + 255) / 256 : cap);
+    scatter_sf_tiled_kernel<<<blocks, 256, 0, stream>>>(xsf, (K + 31) / 32, stok, T, offsets, tile_start1, E, S,
+                                                        (I + 127) / 128, nch, sfa, err);
+    return cudaGetLastError();
+}
 
 size_t mx_scale_bytes(int kind, long long n_experts, int rows, int K) {
     const int P = kind == 0 ? 128 : 256;

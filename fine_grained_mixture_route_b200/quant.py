@@ -14,7 +14,8 @@ and scales out.  There is no other implementation of the format's arithmetic her
 
 The block-scaled variant (quantize_stack(..., fmt="mxfp8"), moe_quantize_weights_mx) keeps one
 power-of-two scale per run of 32 inputs of each row instead of one per row: the per-group option
-of the same §5.5 advice, in the form the sm_100a tensor cores apply inside the MMA.
+of the same §5.5 advice, in the form the sm_100a tensor cores apply inside the MMA.  The layer
+then quantises the expert inputs and hidden rows in runs of 32 as well.
 """
 from __future__ import annotations
 

@@ -55,9 +55,11 @@
  *    power-of-two scale per run of 32 consecutive inputs instead of one per row: the scale of a
  *    run is 2^e with e the smallest integer such that max|run| <= 448 * 2^e (0 for an all-zero
  *    run, within [-127, 127]), stored as the byte e + 127 in sf13 (w1 and w3) and sf2 (w2), in
- *    the tiled order moe_quantize_weights_mx writes.  The tensor cores apply these scales inside
- *    the MMA (kind::mxf8f6f4 with block scales); activations are quantised per row as for
- *    MOE_FMT_E4M3.  The DeepSeek-V2 explainer (§5.5) advises per-channel or per-group scales
+ *    the tiled order moe_quantize_weights_mx writes.  The routed experts' input rows and their
+ *    SwiGLU hidden rows (rounded to bf16) are quantised the same way, one such scale per run of
+ *    32 along the row.  The tensor cores apply both operands' scales inside the MMA
+ *    (kind::mxf8f6f4 with block scales), and the up-projection writes the hidden rows directly
+ *    as codes with their scales.  The DeepSeek-V2 explainer (§5.5) advises per-channel or per-group scales
  *    for quantised routed experts, with the shared experts left in 16-bit, as here; it fixes
  *    no group size or scale type.  Groups of 32 with power-of-two scales are what the sm_100a
  *    tensor cores apply natively.

@@ -257,7 +257,12 @@ def test_mxfp8_format_validates(lib):
     S = ctypes.byref
     shm = _shape(routed_fmt=moe.FMT_MXFP8)
     nm = moe.workspace_bytes(shm)
-    assert nm == moe.workspace_bytes(_shape(routed_fmt=moe.FMT_E4M3)) > 0
+    # on top of the e4m3 workspace: x's run scales per token, and the tiled A-side scales of both
+    # GEMMs (one 512-byte block per (128-row block, 128-input chunk); at most S/128 + E blocks)
+    T, d, I, E, slots = 256, 7168, 2048, 256, 256 * 8
+    al = lambda n: (n + 255) // 256 * 256
+    extra = al(T * d // 32) + al((slots // 128 + E) * (d // 128) * 512) + al((slots // 128 + E) * (I // 128) * 512)
+    assert nm - moe.workspace_bytes(_shape(routed_fmt=moe.FMT_E4M3)) == extra
     assert moe.layer_launches(shm) == moe.layer_launches(_shape(routed_fmt=moe.FMT_E4M3)) == 10
     for unsupported in (dict(dtype=moe.MOE_F32), dict(d=7176), dict(inter=2056)):
         assert moe.workspace_bytes(_shape(routed_fmt=moe.FMT_MXFP8, **unsupported)) == 0, unsupported

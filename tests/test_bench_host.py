@@ -70,8 +70,15 @@ def test_stage_work_sums_to_layer_flops():
                - (256 * routed_mx + per_expert + 256 * 7168 * 2 + 2 * 256 * 7168 * 2)) < 1
     wm, w8 = bench.stage_work(dec, 256, e4m3=True, mx=True), bench.stage_work(dec, 256, e4m3=True)
     assert [f for f, _ in wm.values()] == [f for f, _ in w8.values()]
-    assert wm["gemm1_swiglu"][1] - w8["gemm1_swiglu"][1] == 256 * (2 * 2048 * 7168 // 32 - 2 * 2048 * 4)
-    assert wm["gemm2"][1] - w8["gemm2"][1] == 256 * (7168 * 2048 // 32 - 7168 * 4)
+    S = 256 * 8
+    # gemm1: weight scales per run instead of per row; x scales per run instead of per row; h as
+    # codes + run scales instead of bf16
+    assert wm["gemm1_swiglu"][1] - w8["gemm1_swiglu"][1] == \
+        256 * (2 * 2048 * 7168 // 32 - 2 * 2048 * 4) + S * (7168 // 32 - 4) + S * (2048 + 2048 // 32 - 2 * 2048)
+    # gemm2: no hidden-row quantisation (bf16 h read, codes and row scales written), run scales of h and W2
+    assert wm["gemm2"][1] - w8["gemm2"][1] == \
+        256 * (7168 * 2048 // 32 - 7168 * 4) - (S * 2048 * 2 + S * 2048 + S * 4) + S * (2048 // 32 - 4)
+    assert wm["gather"][1] - w8["gather"][1] == S * (7168 // 32 - 4)
     # ragged shapes pay whole tiles: inter 80 and d 208 -> one 128-row group, two 128-input chunks
     rag = W.scaled(W.CONFIGS["small"], d=208, inter=80)
     assert bench.mx_scale_bytes_per_expert(rag) == (1 * 2 * 1024, 1 * 1 * 1024)
