@@ -336,20 +336,21 @@ __global__ void __launch_bounds__(256) quant_weights_mx_kernel(const uint4* __re
 
 // The A-side scales of the block-scaled GEMM1: grouped position p (token stok[p], in expert e's
 // rows [offsets[e], offsets[e + 1])) is row r = (p - offsets[e]) % 128 of the expert's 128-row
-// block m = (p - offsets[e]) / 128, whose global index is tile_start1[e] / n_tiles + m.  Thread
-// (p, c) copies the token's scale bytes of runs 4c..4c+3 (127 past the row) to that block's
-// chunk c: [M-tile][chunk][512], row r at (r % 32) * 16 + (r / 32 % 4) * 4.
-__global__ void scatter_sf_tiled_kernel(const uint8_t* __restrict__ xsf, int nruns, const int32_t* __restrict__ stok,
-                                        int T, const int32_t* __restrict__ offsets, const int32_t* __restrict__ tile_start1,
-                                        int E, long long S, int n_tiles, int nch, uint8_t* __restrict__ sfa, uint32_t* err) {
-    const long long total = S * nch;
-    for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < total;
-         i += (long long)gridDim.x * blockDim.x) {
-        const long long p = i / nch;
-        const int c = (int)(i % nch);
+// block m = (p - offsets[e]) / 128, whose global index is tile_start1[e] / n_tiles + m.  One warp
+// per position finds e (binary search over the offsets, every lane on the same addresses), then
+// lane l copies the token's scale bytes of runs 4c..4c+3 (127 past the row) for chunks
+// c = l, l + 32, ... to the block's chunk c: [M-tile][chunk][512], row r at (r % 32) * 16 +
+// (r / 32 % 4) * 4.
+__global__ void __launch_bounds__(256) scatter_sf_tiled_kernel(
+    const uint8_t* __restrict__ xsf, int nruns, const int32_t* __restrict__ stok, int T,
+    const int32_t* __restrict__ offsets, const int32_t* __restrict__ tile_start1, int E, long long S, int n_tiles,
+    int nch, uint8_t* __restrict__ sfa, uint32_t* err) {
+    const int lane = threadIdx.x & 31;
+    const long long warps = (long long)gridDim.x * (blockDim.x >> 5);
+    for (long long p = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); p < S; p += warps) {
         const int t = stok[p];
         if (t < 0 || t >= T) {
-            flag_error(err, ERR_INDEX_RANGE);
+            if (lane == 0) flag_error(err, ERR_INDEX_RANGE);
             continue;
         }
         int lo = 0, hi = E;                               // the last e with offsets[e] <= p
@@ -359,16 +360,18 @@ __global__ void scatter_sf_tiled_kernel(const uint8_t* __restrict__ xsf, int nru
             else hi = mid - 1;
         }
         const int local = (int)(p - offsets[lo]);
-        const long long g = tile_start1[lo] / n_tiles + local / 128;
-        const int r = local & 127;
-        uint32_t w = 0;
+        const size_t base = (size_t)(tile_start1[lo] / n_tiles + local / 128) * nch * 512 + (local & 31) * 16 +
+                            ((local >> 5) & 3) * 4;
+        const uint8_t* row = xsf + (size_t)t * nruns;
+        for (int c = lane; c < nch; c += 32) {
+            uint32_t w = 0;
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int run = 4 * c + j;
-            const uint32_t b = run < nruns ? xsf[(size_t)t * nruns + run] : 127u;
-            w |= b << (8 * j);
+            for (int q = 0; q < 4; ++q) {
+                const int run = 4 * c + q;
+                w |= (uint32_t)(run < nruns ? row[run] : 127u) << (8 * q);
+            }
+            *reinterpret_cast<uint32_t*>(sfa + base + (size_t)c * 512) = w;
         }
-        *reinterpret_cast<uint32_t*>(sfa + ((size_t)g * nch + c) * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4) = w;
     }
 }
 
@@ -392,9 +395,8 @@ cudaError_t launch_scatter_sf_tiled(const uint8_t* xsf, int T, int K, const int3
                                     cudaStream_t stream) {
     if (S <= 0) return cudaSuccess;
     const int nch = (K + 127) / 128;
-    const long long total = S * nch;
     const long long cap = 8LL * 8 * num_sms();
-    const int blocks = (int)((total + 255) / 256 < cap ? (total + 255) / 256 : cap);
+    const int blocks = (int)((S + 7) / 8 < cap ? (S + 7) / 8 : cap);    // one warp per grouped position
     scatter_sf_tiled_kernel<<<blocks, 256, 0, stream>>>(xsf, (K + 31) / 32, stok, T, offsets, tile_start1, E, S,
                                                         (I + 127) / 128, nch, sfa, err);
     return cudaGetLastError();
