@@ -61,6 +61,31 @@ def test_fp8_codes_need_the_fp8_shape_and_fp32_scales():
         _fwd(s8, L, ws, routed=q)
 
 
+def test_block_scaled_codes_need_their_scale_bytes():
+    cfg, L, shape, ws = _layer()
+    E, I, d = cfg.n_experts, cfg.inter, cfg.d
+    R = L["routed"]
+    # a stack in the block-scaled layout (codes and tiled scale bytes); types and sizes only
+    q = {k: v for k, v in R.items()}
+    q.update(w1=torch.zeros(R["w1"].shape, dtype=torch.uint8), w3=torch.zeros(R["w3"].shape, dtype=torch.uint8),
+             w2=torch.zeros(R["w2"].shape, dtype=torch.uint8),
+             sf13=torch.full((E, moe.mx_scale_bytes(moe.MX_UP, E, I, d) // E), 127, dtype=torch.uint8),
+             sf2=torch.full((E, moe.mx_scale_bytes(moe.MX_DOWN, E, d, I) // E), 127, dtype=torch.uint8))
+    smx = moe.shape_of(L["x"], L["centroids"], q, cfg.top_k, L["shared"])
+    assert smx.routed_fmt == moe.FMT_MXFP8
+    with pytest.raises(ValueError, match=r"routed\.sf13 holds"):
+        _fwd(smx, L, ws, routed=dict(q, sf13=q["sf13"][:, :-1].contiguous()))
+    with pytest.raises(ValueError, match=r"routed\.sf2 has dtype torch.int8"):
+        _fwd(smx, L, ws, routed=dict(q, sf2=q["sf2"].to(torch.int8)))
+    with pytest.raises(ValueError, match="CUDA"):
+        _fwd(smx, L, ws, routed=q)
+    # the converter takes bf16 stacks on the GPU only, and w1 with w3 for the up-projection
+    with pytest.raises(ValueError, match="CUDA"):
+        moe.quantize_weights_mx(moe.MX_UP, R["w1"], R["w3"])
+    with pytest.raises(ValueError, match="MX_UP takes w1 and w3"):
+        moe.quantize_weights_mx(moe.MX_UP, R["w1"])
+
+
 def test_outputs_and_indices_too_small_or_wrong_type():
     cfg, L, shape, ws = _layer()
     T, k, E, d = cfg.T, cfg.top_k, cfg.n_experts, cfg.d
